@@ -1,0 +1,207 @@
+"""CPU oracle for MX / NVFP4 quantisation, dequantisation and the block-scaled matmul.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this package.
+The product library never imports, links or calls it, and it never imports the product.
+
+The arithmetic lives in ``mx_oracle.c`` (plain C, integer bit manipulation, one plain
+loop per block).  This module only marshals numpy arrays through ctypes and builds the
+shared object with gcc when it is missing.
+
+Every function's definition and the passage it follows are documented in ``mx_oracle.c``.
+Parity status: every function here is pinned by the ``-m "not gpu"`` oracle tests
+except the exact NVFP4 step order (pinned only through its invariants and the
+per-tensor-scale definition) and the tcgen05 scale tiling (not defined by the pages;
+pinned on hardware by the block-scaled matmul).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mx_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+# Format and code-kind identifiers (the same numbering as mx_oracle.c).
+E4M3, E5M2, E2M1, NVFP4 = 0, 1, 2, 3
+K_E4M3, K_E5M2, K_E2M1, K_UE4M3, K_E8M0, K_BF16 = 0, 1, 2, 3, 4, 5
+FLOOR, CEIL = 0, 1
+ROW, COL = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile mx_oracle.c with gcc (no fast-math, no FP contraction)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call([
+            "gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off",
+            "-fno-fast-math", "-frounding-math", "-o", tmp, _SRC, "-lm",
+        ])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I = ctypes.c_int
+        _lib.mxo_decode.argtypes = [I, ctypes.c_uint]
+        _lib.mxo_decode.restype = ctypes.c_double
+        _lib.mxo_encode.argtypes = [ctypes.c_double, I]
+        _lib.mxo_encode.restype = ctypes.c_uint
+        _lib.mxo_scale_exponent.argtypes = [ctypes.c_double, I, I]
+        _lib.mxo_scale_exponent.restype = I
+        _lib.mxo_quantize_mx.argtypes = [P, I64, I64, I, I, I, P, P]
+        _lib.mxo_quantize_mx.restype = I
+        _lib.mxo_cast.argtypes = [P, I64, I, P]
+        _lib.mxo_cast.restype = I
+        _lib.mxo_quantize_nvfp4.argtypes = [P, I64, I64, P, P, P]
+        _lib.mxo_quantize_nvfp4.restype = I
+        _lib.mxo_dequantize_mx.argtypes = [P, P, I64, I64, I, P]
+        _lib.mxo_dequantize_mx.restype = I
+        _lib.mxo_dequantize_nvfp4.argtypes = [P, P, ctypes.c_float, I64, I64, P]
+        _lib.mxo_dequantize_nvfp4.restype = I
+        _lib.mxo_tcgen05_scale_bytes.argtypes = [I64, I64]
+        _lib.mxo_tcgen05_scale_bytes.restype = I64
+        _lib.mxo_tcgen05_scale_offset.argtypes = [I64, I64, I64, I64]
+        _lib.mxo_tcgen05_scale_offset.restype = I64
+        _lib.mxo_gemm_ref.argtypes = [P, P, I, P, P, I, I64, I64, I64, P, I64, P, P]
+        _lib.mxo_gemm_ref.restype = I
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what}: invalid arguments (rc={rc})")
+
+
+# ---------------------------------------------------------------- scalar codecs
+def decode(kind: int, code: int) -> float:
+    """Exact value of one code (E4M3, E5M2, E2M1, UE4M3, E8M0 or bf16 bits)."""
+    return lib().mxo_decode(kind, code)
+
+
+def encode(value: float, kind: int) -> int:
+    """Saturating round-to-nearest-even code of one value (no block scale)."""
+    return lib().mxo_encode(float(value), kind)
+
+
+def scale_exponent(amax: float, fmt: int, rounding: int) -> int:
+    """Shared exponent s (clamped to [-127, 127]) for a block maximum."""
+    return lib().mxo_scale_exponent(float(amax), fmt, rounding)
+
+
+def elem_bytes(n_elems: int, fmt: int) -> int:
+    return n_elems // 2 if fmt in (E2M1, NVFP4) else n_elems
+
+
+# ---------------------------------------------------------------- block operations
+def quantize_mx(x_bf16_bits: np.ndarray, fmt: int, axis: int = ROW, rounding: int = CEIL):
+    """MX quantisation of a 2-D bf16 matrix given as uint16 bit patterns.
+
+    Returns (elems, scales): row-wise elems rows x bytes(cols), scales rows x cols/32;
+    col-wise the output is transposed: elems cols x bytes(rows), scales cols x rows/32.
+    """
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    rows, cols = x.shape
+    orow, ocol = (rows, cols) if axis == ROW else (cols, rows)
+    elems = np.zeros((orow, elem_bytes(ocol, fmt)), dtype=np.uint8)
+    scales = np.zeros((orow, ocol // 32), dtype=np.uint8)
+    _check(lib().mxo_quantize_mx(_ptr(x), rows, cols, fmt, axis, rounding, _ptr(elems), _ptr(scales)),
+           "quantize_mx")
+    return elems, scales
+
+
+def cast(x_bf16_bits: np.ndarray, fmt: int) -> np.ndarray:
+    """Direct element cast with no block scale (codes, FP4 packed two per byte)."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16).reshape(-1)
+    out = np.zeros(elem_bytes(x.size, fmt), dtype=np.uint8)
+    _check(lib().mxo_cast(_ptr(x), x.size, fmt, _ptr(out)), "cast")
+    return out
+
+
+def quantize_nvfp4(x_bf16_bits: np.ndarray):
+    """NVFP4 quantisation. Returns (elems rows x cols/2, scales rows x cols/16, g)."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    rows, cols = x.shape
+    elems = np.zeros((rows, cols // 2), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 16), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    _check(lib().mxo_quantize_nvfp4(_ptr(x), rows, cols, _ptr(elems), _ptr(scales), _ptr(g)),
+           "quantize_nvfp4")
+    return elems, scales, float(g[0])
+
+
+def dequantize_mx(elems: np.ndarray, scales: np.ndarray, rows: int, cols: int, fmt: int) -> np.ndarray:
+    """bf16 bits (uint16) of dec(q) * 2^(s-127); scale 0xFF gives NaN."""
+    e = np.ascontiguousarray(elems, dtype=np.uint8)
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    out = np.zeros((rows, cols), dtype=np.uint16)
+    _check(lib().mxo_dequantize_mx(_ptr(e), _ptr(s), rows, cols, fmt, _ptr(out)), "dequantize_mx")
+    return out
+
+
+def dequantize_nvfp4(elems: np.ndarray, scales: np.ndarray, g: float, rows: int, cols: int) -> np.ndarray:
+    e = np.ascontiguousarray(elems, dtype=np.uint8)
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    out = np.zeros((rows, cols), dtype=np.uint16)
+    _check(lib().mxo_dequantize_nvfp4(_ptr(e), _ptr(s), ctypes.c_float(g), rows, cols, _ptr(out)),
+           "dequantize_nvfp4")
+    return out
+
+
+# ---------------------------------------------------------------- tcgen05 scale tiling
+def tcgen05_scale_bytes(rows: int, scale_cols: int) -> int:
+    return lib().mxo_tcgen05_scale_bytes(rows, scale_cols)
+
+
+def to_tcgen05_layout(scales_rowmajor: np.ndarray) -> np.ndarray:
+    """Re-index a row-major scale matrix into the tcgen05 tiling (padding bytes zero)."""
+    s = np.ascontiguousarray(scales_rowmajor, dtype=np.uint8)
+    rows, scols = s.shape
+    out = np.zeros(tcgen05_scale_bytes(rows, scols), dtype=np.uint8)
+    L = lib()
+    for r in range(rows):
+        for c in range(scols):
+            out[L.mxo_tcgen05_scale_offset(r, c, rows, scols)] = s[r, c]
+    return out
+
+
+def tcgen05_offsets(rows: int, scale_cols: int) -> np.ndarray:
+    """Offset of every (r, c) entry in the tcgen05 tiling, as a rows x scale_cols array."""
+    L = lib()
+    out = np.empty((rows, scale_cols), dtype=np.int64)
+    for r in range(rows):
+        for c in range(scale_cols):
+            out[r, c] = L.mxo_tcgen05_scale_offset(r, c, rows, scale_cols)
+    return out
+
+
+# ---------------------------------------------------------------- matmul reference
+def gemm_ref(a_elems, a_scales, a_fmt, b_elems, b_scales, b_fmt, M, N, K, pairs):
+    """fp64 C[m, n] and sum_k |a b| for the requested (m, n) pairs (an array n x 2)."""
+    pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+    c = np.zeros(pr.shape[0], dtype=np.float64)
+    mag = np.zeros(pr.shape[0], dtype=np.float64)
+    ae = np.ascontiguousarray(a_elems, dtype=np.uint8)
+    as_ = np.ascontiguousarray(a_scales, dtype=np.uint8)
+    be = np.ascontiguousarray(b_elems, dtype=np.uint8)
+    bs = np.ascontiguousarray(b_scales, dtype=np.uint8)
+    _check(lib().mxo_gemm_ref(_ptr(ae), _ptr(as_), a_fmt, _ptr(be), _ptr(bs), b_fmt, M, N, K,
+                              _ptr(pr), pr.shape[0], _ptr(c), _ptr(mag)), "gemm_ref")
+    return c, mag

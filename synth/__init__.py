@@ -1,0 +1,89 @@
+"""Seeded synthetic inputs for the five MX workloads.
+
+This module holds only random-number generation: no quantisation, scale or codec
+arithmetic.  Both the CUDA path's tests/benchmark and the CPU oracle read the same
+bytes produced here.  Every generator draws fp32 values with ``numpy.random.default_rng``
+and rounds them to bf16 (round-to-nearest-even, by torch's dtype conversion); the result
+is returned as uint16 bf16 bit patterns, row-major.
+
+Workloads (shapes and distributions of the MX pages' use cases):
+  mx8_rowwise   1024 x 1024, N(0,1) * 2^u per row with u ~ U[-8, 8], 1% of entries x100
+  weight_fp4    4096 x 4096, N(0, 0.02), 0.1% of entries replaced by N(0, 1)
+  activations   16384 x 4096, N(0,1) * per-column 2^v with v ~ U[-4, 4]
+  gradients     16384 x 14336, N(0, 1e-3) with 5% exact zeros
+  gemm operands N(0, 1) activations / N(0, 1) or N(0, 0.02) weights
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+
+def to_bf16_bits(x32: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 (RNE, torch conversion) -> uint16 bit patterns."""
+    t = torch.from_numpy(np.ascontiguousarray(x32, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_float(bits: np.ndarray) -> np.ndarray:
+    """uint16 bf16 bit patterns -> fp32 values (exact)."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def normal(rows: int, cols: int, sigma: float = 1.0, seed: int = 0) -> np.ndarray:
+    rng = np.random.default_rng(seed)
+    return to_bf16_bits(rng.standard_normal((rows, cols), dtype=np.float32) * np.float32(sigma))
+
+
+def mx8_rowwise(rows: int = 1024, cols: int = 1024, seed: int = 0) -> np.ndarray:
+    """N(0,1) times a per-row 2^u, u ~ U[-8, 8]; 1% of entries multiplied by 100."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols), dtype=np.float32)
+    u = rng.uniform(-8.0, 8.0, size=(rows, 1)).astype(np.float32)
+    x *= np.exp2(u)
+    outlier = rng.random((rows, cols)) < 0.01
+    x[outlier] *= np.float32(100.0)
+    return to_bf16_bits(x)
+
+
+def weight_fp4(rows: int = 4096, cols: int = 4096, seed: int = 0) -> np.ndarray:
+    """N(0, 0.02) with 0.1% of entries replaced by N(0, 1) draws."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols), dtype=np.float32) * np.float32(0.02)
+    mask = rng.random((rows, cols)) < 0.001
+    x[mask] = rng.standard_normal(int(mask.sum()), dtype=np.float32)
+    return to_bf16_bits(x)
+
+
+def activations(rows: int = 16384, cols: int = 4096, seed: int = 0) -> np.ndarray:
+    """N(0,1) times a per-channel (column) scale 2^v, v ~ U[-4, 4] (log-uniform)."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols), dtype=np.float32)
+    v = rng.uniform(-4.0, 4.0, size=(1, cols)).astype(np.float32)
+    x *= np.exp2(v)
+    return to_bf16_bits(x)
+
+
+def gradients(rows: int = 16384, cols: int = 14336, seed: int = 1) -> np.ndarray:
+    """N(0, 1e-3) with 5% exact zeros."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols), dtype=np.float32) * np.float32(1e-3)
+    x[rng.random((rows, cols)) < 0.05] = 0.0
+    return to_bf16_bits(x)
+
+
+def special_values_block() -> np.ndarray:
+    """Hand-picked edge values (zeros, subnormals, extremes, Inf, NaN) as bf16 bits."""
+    vals = [0x0000, 0x8000, 0x0001, 0x8001, 0x007F, 0x0080, 0x7F7F, 0xFF7F,
+            0x3F80, 0xBF80, 0x4300, 0x43E0, 0x43E8, 0x43F0, 0x4760, 0x4770]
+    return np.array(vals, dtype=np.uint16)
+
+
+# Workload table used by the benchmark and the full-size parity tests.
+CONFIGS = {
+    1: dict(name="mx8_rowwise_1024x1024_e4m3_ceil", shape=(1024, 1024)),
+    2: dict(name="weight_4096x4096_mxfp4_floor_and_nvfp4", shape=(4096, 4096)),
+    3: dict(name="dual_act_16384x4096_e4m3_grad_16384x14336_e5m2", shape=(16384, 4096)),
+    4: dict(name="gemm_e4m3xe4m3_8192x8192x8192", shape=(8192, 8192, 8192)),
+    5: dict(name="gemm_e4m3_act_x_e2m1_weight_m8192_n14336_k4096", shape=(8192, 14336, 4096)),
+}

@@ -1,0 +1,295 @@
+"""Pins of the oracle's block operations: the worked example, effective bits, NaN
+scales, landing of real blocks, dequantisation, NVFP4 invariants, the fp64 matmul
+reference and the scale tiling (no GPU)."""
+import math
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+import synth
+from conftest import f32_to_bf16_bits, read_golden
+from test_oracle_formats import bf16_bits_to_f64, unpack_fp4
+
+
+def e2m1_values(codes):
+    return np.asarray(codes, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+
+
+# ------------------------------------------------------------------ worked example
+def test_worked_example_direct_cast(oracle):
+    g = read_golden("p4_worked_example.txt")
+    x = f32_to_bf16_bits(g["input"])
+    got = e2m1_values(unpack_fp4(oracle.cast(x, oracle.E2M1), 4))
+    page = list(g["direct_cast_page"])
+    idx, rne = g["direct_cast_tie_rne"]
+    for i in range(4):
+        if i == int(idx):
+            assert got[i] == rne and page[i] != rne   # recorded discrepancy (tie)
+        else:
+            assert got[i] == page[i]
+
+
+@pytest.mark.parametrize("rounding", [0, 1])
+def test_worked_example_shared_scale(oracle, rounding):
+    g = read_golden("p4_worked_example.txt")
+    block = np.zeros((1, 32), dtype=np.uint16)          # a 32-block; the rest are zeros
+    block[0, :4] = f32_to_bf16_bits(g["input"])
+    elems, scales = oracle.quantize_mx(block, oracle.E2M1, oracle.ROW, rounding)
+    assert int(scales[0, 0]) - 127 == int(g["shared_scale_exponent"][0])
+    got = e2m1_values(unpack_fp4(elems[0], 32))[:4]
+    page = list(g["scaled_cast_page"])
+    idx, rne = g["scaled_cast_tie_rne"]
+    for i in range(4):
+        if i == int(idx):
+            assert got[i] == rne and page[i] != rne
+        else:
+            assert got[i] == page[i]
+    assert np.all(e2m1_values(unpack_fp4(elems[0], 32))[4:] == 0)
+
+
+# ------------------------------------------------------------------ effective bits
+def test_effective_bits(oracle):
+    g = read_golden("format_constants.txt")
+    x = synth.normal(64, 256, seed=3)
+    n = x.size
+    e, s = oracle.quantize_mx(x, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    assert (e.nbytes + s.nbytes) * 8 / n == g["bits_mxfp4"][0]
+    for fmt in (oracle.E4M3, oracle.E5M2):
+        e, s = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.CEIL)
+        assert (e.nbytes + s.nbytes) * 8 / n == g["bits_mxfp8"][0]
+    e, s, _ = oracle.quantize_nvfp4(x)
+    assert (e.nbytes + s.nbytes) * 8 / n == g["bits_nvfp4"][0]
+
+
+# ------------------------------------------------------------------ block assembly
+@pytest.mark.parametrize("fmt_name,rounding", [("E4M3", 1), ("E4M3", 0), ("E5M2", 1), ("E2M1", 0), ("E2M1", 1)])
+def test_block_codes_are_the_cast_of_scaled_values(oracle, fmt_name, rounding):
+    """Each block's codes equal the (brute-force-pinned) direct cast of x * 2^-s, with s
+    read back from the E8M0 byte, and the scaled maximum lands per its school."""
+    fmt = getattr(oracle, fmt_name)
+    x = synth.mx8_rowwise(16, 128, seed=5)
+    e, s = oracle.quantize_mx(x, fmt, oracle.ROW, rounding)
+    maxv = {"E4M3": 448.0, "E5M2": 57344.0, "E2M1": 6.0}[fmt_name]
+    xf = bf16_bits_to_f64(x)
+    fp4 = fmt_name == "E2M1"
+    for r in range(x.shape[0]):
+        codes = unpack_fp4(e[r], 128) if fp4 else e[r]
+        for b in range(4):
+            sc = int(s[r, b]) - 127
+            blk = xf[r, 32 * b:32 * b + 32]
+            scaled = np.ldexp(blk, -sc)
+            ref = oracle.cast(f32_to_bf16_bits(scaled.astype(np.float32)), fmt) if np.all(
+                (scaled.astype(np.float32).view(np.uint32) & 0xFFFF) == 0) else None
+            assert ref is not None              # power-of-two scaling keeps bf16 exact here
+            ref = unpack_fp4(ref, 32) if fp4 else ref
+            assert np.array_equal(codes[32 * b:32 * b + 32], ref)
+            top = np.abs(scaled).max()
+            if rounding == 1:
+                assert maxv / 2 < top <= maxv
+            else:
+                assert 2.0 ** {"E4M3": 8, "E5M2": 15, "E2M1": 2}[fmt_name] <= top
+
+
+def test_fp4_nibble_order(oracle):
+    x = np.zeros((1, 32), dtype=np.uint16)
+    x[0, 0] = f32_to_bf16_bits([6.0])[0]      # code 0x7 at even index 0
+    x[0, 1] = f32_to_bf16_bits([-1.0])[0]     # code 0xA at odd index 1
+    e, s = oracle.quantize_mx(x, oracle.E2M1, oracle.ROW, oracle.CEIL)
+    assert s[0, 0] == 127 and e[0, 0] == 0xA7
+
+
+def test_colwise_is_rowwise_of_transpose(oracle):
+    x = synth.activations(64, 96, seed=2)
+    for fmt in (oracle.E4M3, oracle.E2M1):
+        ec, sc = oracle.quantize_mx(x, fmt, oracle.COL, oracle.CEIL)
+        er, sr = oracle.quantize_mx(np.ascontiguousarray(x.T), fmt, oracle.ROW, oracle.CEIL)
+        assert np.array_equal(ec, er) and np.array_equal(sc, sr)
+        assert ec.shape[0] == 96 and sc.shape == (96, 2)
+
+
+def test_nan_or_inf_makes_block_nan(oracle):
+    x = synth.normal(2, 64, seed=1)
+    x[0, 5] = 0x7FC0      # NaN in block (0, 0)
+    x[1, 40] = 0xFF80     # -Inf in block (1, 1)
+    for fmt in (oracle.E4M3, oracle.E5M2, oracle.E2M1):
+        e, s = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.CEIL)
+        assert s[0, 0] == 0xFF and s[1, 1] == 0xFF and s[0, 1] != 0xFF and s[1, 0] != 0xFF
+        d = bf16_bits_to_f64(oracle.dequantize_mx(e, s, 2, 64, fmt))
+        assert np.all(np.isnan(d[0, :32])) and np.all(np.isnan(d[1, 32:]))
+        assert np.all(np.isfinite(d[0, 32:])) and np.all(np.isfinite(d[1, :32]))
+
+
+def test_zero_block(oracle):
+    x = np.zeros((1, 64), dtype=np.uint16)
+    x[0, 33] = 0x8000   # -0
+    e, s = oracle.quantize_mx(x, oracle.E4M3, oracle.ROW, oracle.CEIL)
+    assert list(s[0]) == [0, 0] and e[0, 33] == 0x80 and np.all(np.delete(e[0], 33) == 0)
+
+
+# ------------------------------------------------------------------ dequantisation
+@pytest.mark.parametrize("fmt_name,dtype", [("E4M3", torch.float8_e4m3fn), ("E5M2", torch.float8_e5m2)])
+def test_dequant_is_exponent_add(oracle, fmt_name, dtype):
+    """dec(q) * 2^(s-127) through a library fp8 decode and ldexp (exact, then bf16)."""
+    fmt = getattr(oracle, fmt_name)
+    x = synth.mx8_rowwise(8, 256, seed=7)
+    e, s = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.CEIL)
+    got = bf16_bits_to_f64(oracle.dequantize_mx(e, s, 8, 256, fmt))
+    dec = torch.from_numpy(e).view(dtype).double().numpy()
+    ref = np.ldexp(dec, np.repeat(s.astype(np.int64) - 127, 32, axis=1))
+    ref_bf16 = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()  # single RNE from fp64
+    assert np.array_equal(got, ref_bf16)
+
+
+def test_dequant_value_idempotent(oracle):
+    """quantise(dequantise(quantise(x))) reproduces the same dequantised values."""
+    x = synth.mx8_rowwise(32, 256, seed=11)
+    for fmt in (oracle.E4M3, oracle.E5M2, oracle.E2M1):
+        for rnd in (oracle.FLOOR, oracle.CEIL):
+            e, s = oracle.quantize_mx(x, fmt, oracle.ROW, rnd)
+            d1 = oracle.dequantize_mx(e, s, 32, 256, fmt)
+            e2, s2 = oracle.quantize_mx(d1, fmt, oracle.ROW, rnd)
+            d2 = oracle.dequantize_mx(e2, s2, 32, 256, fmt)
+            assert np.array_equal(d1, d2)
+
+
+def test_dequant_nan_scale_and_subnormal_output(oracle):
+    e = np.full((1, 32), 0x01, dtype=np.uint8)          # E4M3 smallest subnormal 2^-9
+    s = np.array([[0]], dtype=np.uint8)                 # 2^-127 -> 2^-136, below bf16 subnormals' quantum
+    d = oracle.dequantize_mx(e, s, 1, 32, oracle.E4M3)
+    assert np.all(d == 0x0000)                          # 2^-136 rounds to 0 in bf16 (quantum 2^-133)
+    e[:] = 0x08                                         # 2^-6 * 2^-127 = 2^-133: the smallest bf16 subnormal
+    assert np.all(oracle.dequantize_mx(e, s, 1, 32, oracle.E4M3) == 0x0001)
+    s[:] = 0xFF
+    assert np.all(np.isnan(bf16_bits_to_f64(oracle.dequantize_mx(e, s, 1, 32, oracle.E4M3))))
+
+
+# ------------------------------------------------------------------ NVFP4
+def test_nvfp4_global_scale_definition(oracle):
+    g_fix = read_golden("format_constants.txt")
+    assert g_fix["nvfp4_global_divisor"][0] == 6 * 448
+    x = synth.weight_fp4(64, 128, seed=4)
+    _, _, g = oracle.quantize_nvfp4(x)
+    amax = np.abs(bits_to_finite(x)).max()
+    assert g == float(np.float32(amax) / np.float32(g_fix["nvfp4_global_divisor"][0]))
+    # a tensor whose maximum is exactly 6 * 448 has g = 1 and that block's scale is 448
+    y = synth.normal(4, 32, sigma=1.0, seed=9)
+    y[2, 17] = f32_to_bf16_bits([2688.0])[0]
+    e, s, g = oracle.quantize_nvfp4(y)
+    assert g == 1.0 and s[2, 1] == 0x7E and oracle.decode(oracle.K_UE4M3, int(s[2, 1])) == 448.0
+    assert unpack_fp4(e[2], 32)[17] == 0x7                  # 2688 / 448 = 6
+
+
+def bits_to_finite(bits):
+    v = bf16_bits_to_f64(bits)
+    return np.where(np.isfinite(v), v, 0.0)
+
+
+def test_nvfp4_block_scale_is_nearest_ue4m3(oracle):
+    """sb is the nearest (ties even) UE4M3 code to amax_b / (6 g), found by brute force,
+    and the elements are the nearest E2M1 of x / d (up to the fp32 product)."""
+    x = synth.weight_fp4(32, 256, seed=6)
+    e, s, g = oracle.quantize_nvfp4(x)
+    ue = np.array([oracle.decode(oracle.K_UE4M3, c) for c in range(0x7F)])
+    xf = bf16_bits_to_f64(x).astype(np.float32)
+    six_g = np.float32(6.0) * np.float32(g)
+    for r in range(32):
+        codes = unpack_fp4(e[r], 256)
+        for b in range(16):
+            blk = xf[r, 16 * b:16 * b + 16]
+            t = np.float32(np.abs(blk).max()) / six_g
+            d = np.abs(ue - float(t))
+            cand = np.nonzero(d == d.min())[0]
+            want = cand[0] if cand.size == 1 else [c for c in cand if c % 2 == 0][0]
+            assert s[r, b] == want
+            dd = np.float32(ue[want]) * np.float32(g)
+            if dd == 0:
+                assert np.all(codes[16 * b:16 * b + 16] == 0)
+                continue
+            scaled = blk * (np.float32(1.0) / dd)
+            ref = np.array([oracle.encode(float(v), oracle.K_E2M1) for v in scaled])
+            assert np.array_equal(codes[16 * b:16 * b + 16], ref)
+            # error bound: half the widest E2M1 spacing (1.0) times d, plus clipping above 6
+            xh = e2m1_values(codes[16 * b:16 * b + 16]) * float(dd)
+            assert np.all(np.abs(xh - blk) <= float(dd) * 1.0 + np.maximum(np.abs(blk) - 6 * float(dd), 0) + 1e-30)
+
+
+def test_nvfp4_scale_relative_error(oracle):
+    """dec(sb) * g * 6 is within the E4M3 half-ulp (2^-4 relative) of the block max."""
+    x = synth.weight_fp4(64, 256, seed=8)
+    _, s, g = oracle.quantize_nvfp4(x)
+    xf = np.abs(bits_to_finite(x)).reshape(64, 16, 16).max(axis=2)
+    dec = np.array([[oracle.decode(oracle.K_UE4M3, int(c)) for c in row] for row in s])
+    normal = xf / (6 * g) >= 2.0 ** -6
+    rel = np.abs(dec * g * 6 - xf) / xf
+    assert np.all(rel[normal] <= 2.0 ** -4 + 1e-6)
+
+
+def test_nvfp4_dequant_order(oracle):
+    x = synth.weight_fp4(16, 64, seed=10)
+    e, s, g = oracle.quantize_nvfp4(x)
+    got = bf16_bits_to_f64(oracle.dequantize_nvfp4(e, s, g, 16, 64))
+    q = e2m1_values(np.stack([unpack_fp4(r, 64) for r in e])).astype(np.float32)
+    sb = torch.from_numpy(s).view(torch.float8_e4m3fn).float().numpy()
+    ref = (q * np.repeat(sb, 16, axis=1)) * np.float32(g)
+    ref = torch.from_numpy(ref.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(got, ref)
+
+
+def test_nvfp4_nonfinite_block(oracle):
+    x = synth.normal(2, 32, seed=12)
+    x[1, 3] = 0x7F80
+    e, s, g = oracle.quantize_nvfp4(x)
+    assert s[1, 0] == 0x7F and s[1, 1] != 0x7F and np.all(unpack_fp4(e[1], 32)[:16] == 0)
+    assert math.isfinite(g)
+    d = bf16_bits_to_f64(oracle.dequantize_nvfp4(e, s, g, 2, 32))
+    assert np.all(np.isnan(d[1, :16])) and np.all(np.isfinite(d[1, 16:]))
+
+
+# ------------------------------------------------------------------ fp64 matmul reference
+def test_gemm_ref_exact_brute_force(oracle):
+    """Tiny case against exact rational arithmetic over library-decoded operands."""
+    M, N, K = 3, 2, 64
+    a = synth.normal(M, K, seed=13)
+    b = synth.weight_fp4(N, K, seed=14)
+    ae, as_ = oracle.quantize_mx(a, oracle.E4M3, oracle.ROW, oracle.CEIL)
+    be, bs = oracle.quantize_mx(b, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    pairs = [(m, n) for m in range(M) for n in range(N)]
+    c, mag = oracle.gemm_ref(ae, as_, oracle.E4M3, be, bs, oracle.E2M1, M, N, K, pairs)
+    av = torch.from_numpy(ae).view(torch.float8_e4m3fn).double().numpy()
+    bv = e2m1_values(np.stack([unpack_fp4(r, K) for r in be]))
+    for p, (m, n) in enumerate(pairs):
+        exact = sum(Fraction(float(av[m, k])) * Fraction(2) ** (int(as_[m, k // 32]) - 127)
+                    * Fraction(float(bv[n, k])) * Fraction(2) ** (int(bs[n, k // 32]) - 127)
+                    for k in range(K))
+        assert abs(Fraction(c[p]) - exact) <= abs(exact) * Fraction(2) ** -50 + Fraction(2) ** -1000
+        assert mag[p] >= abs(c[p])
+
+
+def test_gemm_ref_one_hot(oracle):
+    K = 96
+    a = np.zeros((1, K), dtype=np.uint16)
+    a[0, 70] = f32_to_bf16_bits([3.0])[0]
+    b = synth.normal(4, K, seed=15)
+    ae, as_ = oracle.quantize_mx(a, oracle.E4M3, oracle.ROW, oracle.CEIL)
+    be, bs = oracle.quantize_mx(b, oracle.E4M3, oracle.ROW, oracle.CEIL)
+    c, _ = oracle.gemm_ref(ae, as_, oracle.E4M3, be, bs, oracle.E4M3, 1, 4, K, [(0, n) for n in range(4)])
+    bdec = bf16_bits_to_f64(oracle.dequantize_mx(be, bs, 4, K, oracle.E4M3))
+    assert np.array_equal(c, 3.0 * bdec[:, 70])
+
+
+# ------------------------------------------------------------------ tcgen05 scale tiling
+def test_tcgen05_tiling_is_a_padded_bijection(oracle):
+    for rows, scols in [(128, 4), (256, 8), (130, 5), (1, 1), (300, 33)]:
+        off = oracle.tcgen05_offsets(rows, scols)
+        total = oracle.tcgen05_scale_bytes(rows, scols)
+        assert total == math.ceil(rows / 128) * math.ceil(scols / 4) * 512
+        assert len(np.unique(off)) == off.size and off.min() >= 0 and off.max() < total
+    # a full 128 x 4 atom is a permutation of 0..511; consecutive scale columns of one
+    # row are adjacent bytes, and 32 rows apart are 4 bytes apart
+    off = oracle.tcgen05_offsets(128, 4)
+    assert sorted(off.ravel()) == list(range(512))
+    assert np.all(np.diff(off, axis=1) == 1)
+    assert np.all(off[32:64] - off[0:32] == 4)
