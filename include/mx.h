@@ -1,0 +1,194 @@
+/*
+ * mx.h -- C ABI of the B200 (sm_100a) microscaling library: MX / NVFP4 quantisation,
+ * dequantisation and the MX block-scaled matmul.
+ *
+ * Sources (page title, section):
+ *   [Q]  "MXFP4 と NVFP4 は何が違うのか調べてみた"
+ *        §1 "E2M1 という共通土台": E2M1 values 0, 0.5, 1, 1.5, 2, 3, 4, 6 and mirrors; max 6.
+ *        §2 "MXFP4 はブロック32と E8M0": blocks of 32 share one E8M0 scale (bias 127,
+ *           0xFF = NaN, no Inf); MXFP8 = E4M3 or E5M2 elements; RNE cast; the scale
+ *           rounding is left to the implementation.
+ *        §3 "NVFP4 はブロック16と E4M3、そして二段目": blocks of 16, unsigned E4M3 block
+ *           scale (max 448), FP32 per-tensor scale = tensor amax / (6 * 448).
+ *        §4 "同じ E2M1 でも、別仕様である" / "精度の差はどこから出るか": the OCP floor
+ *           rule (scaled block max in [4, 8), clipped at 6) and the no-clip rule
+ *           (scaled block max in (3, 6]).
+ *        §6 "DeepSeek-V4 の入れ子構造": training needs the weight in both orientations.
+ *        §7 "ハードウェアの対応状況": Blackwell's 5th-generation tensor cores consume
+ *           MXFP8/MXFP4 natively; MX scale application is an exponent add.
+ *   [P4] gpt-oss MXFP4 explainer, section "MXFP4": the direct cast vs the scaled cast.
+ *
+ * Conventions for every entry point:
+ *   - Ownership: the caller allocates and owns every buffer.  Device pointers must be
+ *     device (or managed) memory of the current CUDA device.  The library keeps, per
+ *     device, only a small scratch array for NVFP4 partial maxima (allocated on the
+ *     first NVFP4 call on that device) and a static watchdog flag.
+ *   - Execution: every call only validates its arguments on the host and enqueues
+ *     kernels on `stream` (0 = the legacy default stream); it returns before the GPU
+ *     work finishes.  Nothing is written to any output before the work runs.
+ *   - Errors: arguments are validated before any launch.  A non-MX_OK status means no
+ *     kernel was launched, except MX_ERR_CUDA, which reports a failed launch (the CUDA
+ *     error code is kept per host thread, see mx_last_cuda_error).  Empty inputs
+ *     (rows == 0 or cols == 0) are valid and launch nothing.
+ *   - bf16 is IEEE binary16-brain (1/8/7), stored as 2-byte little-endian words.
+ *   - Element codes: one byte per FP8 code; FP4 codes pack two per byte with the even
+ *     element index in the low nibble.
+ *   - Overflow saturates to the format maximum (448 E4M3, 57344 E5M2, 6 E2M1); a
+ *     block holding a NaN or Inf gets the NaN scale (0xFF E8M0, 0x7F UE4M3) and
+ *     element codes 0.
+ */
+#ifndef MX_H_
+#define MX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle; the same type as cudaStream_t. */
+struct CUstream_st;
+typedef struct CUstream_st *mx_stream_t;
+
+typedef enum {
+    MX_OK = 0,
+    MX_ERR_ARG = 1,      /* null pointer, unknown enum, unsupported combination */
+    MX_ERR_SHAPE = 2,    /* negative size, or a size that is not a multiple of the block/tile */
+    MX_ERR_ALIGN = 3,    /* a pointer that is not aligned as the call requires */
+    MX_ERR_LAYOUT = 4,   /* scale-layout mask empty, unknown, or missing its second buffer */
+    MX_ERR_CUDA = 5,     /* a CUDA launch or driver call failed; see mx_last_cuda_error */
+    MX_ERR_TIMEOUT = 6   /* a bounded device wait gave up (watchdog); see mx_watchdog_status */
+} mx_status;
+
+typedef enum {
+    MX_FMT_E4M3 = 0,     /* MXFP8, E4M3 elements, block 32, E8M0 scale */
+    MX_FMT_E5M2 = 1,     /* MXFP8, E5M2 elements, block 32, E8M0 scale */
+    MX_FMT_E2M1 = 2,     /* MXFP4, E2M1 elements, block 32, E8M0 scale */
+    MX_FMT_NVFP4 = 3     /* NVFP4, E2M1 elements, block 16, UE4M3 scale, fp32 tensor scale */
+} mx_fmt;
+
+typedef enum {
+    MX_AXIS_ROW = 0,     /* blocks run along a row (contiguous elements) */
+    MX_AXIS_COL = 1      /* blocks run down a column; output is the transposed matrix */
+} mx_axis;
+
+typedef enum {
+    MX_SCALE_FLOOR_OCP = 0,    /* s = floor(log2 amax) - emax_elem ([Q] §4, OCP example) */
+    MX_SCALE_CEIL_RECIPE = 1   /* smallest s with amax <= max_elem * 2^s (no clipping, [Q] §4) */
+} mx_scale_rounding;
+
+typedef enum {
+    MX_LAYOUT_ROWMAJOR = 1,    /* scales[r * S + c], S = blocks per output row */
+    MX_LAYOUT_TCGEN05 = 2      /* tcgen05 tiling: 128-row x 4-column atoms of 512 bytes */
+} mx_scale_layout;             /* used as a bit mask where a call accepts both */
+
+/*
+ * Byte size of a scale buffer for an output of `rows` rows and `scale_cols` scales per
+ * row in `layout` (exactly one bit).  ROWMAJOR: rows * scale_cols.  TCGEN05:
+ * ceil(rows/128) * ceil(scale_cols/4) * 512; inside an atom, scale (r, c) sits at byte
+ * (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4), atoms ordered row-block-major; pad bytes
+ * are written as 0 by the quantisers.  Returns -1 for invalid arguments.  Host only.
+ */
+int64_t mx_scale_bytes(int64_t rows, int64_t scale_cols, mx_scale_layout layout);
+
+/*
+ * mx_quantize -- quantise a bf16 matrix to MXFP8 / MXFP4 / NVFP4 ([Q] §2, §3, §4).
+ *   src_bf16    device, rows x cols bf16 row-major, 16-byte aligned.
+ *   fmt         MX_FMT_E4M3 / E5M2 / E2M1 (block 32, E8M0) or MX_FMT_NVFP4 (block 16).
+ *   axis        ROW: blocks along rows; output rows x cols, scales rows x cols/B.
+ *               COL: blocks down columns; output is the transposed matrix cols x rows
+ *               (K-major for a weight-gradient matmul), scales cols x rows/B.
+ *               NVFP4 supports ROW only.
+ *   rounding    shared-exponent rule (ignored for NVFP4).
+ *   out_elems   device, 16-byte aligned; out_rows x out_cols bytes (FP8) or x out_cols/2 (FP4).
+ *   out_scales  device; first scale layout (the lower set bit of `layout`).
+ *   layout      ROWMAJOR, TCGEN05 or both; with both, out_scales gets ROWMAJOR and
+ *               out_scales_alt gets TCGEN05 (else out_scales_alt must be NULL).
+ *   global_scale  NVFP4 only (else NULL): device fp32, written with g = amax / 2688,
+ *               the per-tensor decode scale (1.0 when the tensor is all zero).
+ *   Shape rule: the blocked dimension (cols for ROW, rows for COL) is a multiple of the
+ *   block (32, or 16 for NVFP4), else MX_ERR_SHAPE.
+ */
+mx_status mx_quantize(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt fmt, mx_axis axis,
+                      mx_scale_rounding rounding, void *out_elems, uint8_t *out_scales,
+                      mx_scale_layout layout, uint8_t *out_scales_alt, float *global_scale,
+                      mx_stream_t stream);
+
+/*
+ * mx_quantize_dual -- one pass over a bf16 matrix producing both orientations ([Q] §6:
+ * training needs the row-wise copy for the forward matmul and the column-wise copy for
+ * the weight-gradient matmul).  The input is read once.
+ *   row_elems / row_scales   as mx_quantize(axis = ROW).
+ *   col_elems / col_scales   as mx_quantize(axis = COL): cols x rows, scales cols x rows/32.
+ *   layout      exactly one of ROWMAJOR / TCGEN05, used for both scale outputs.
+ *   fmt         E4M3, E5M2 or E2M1.  rows and cols are multiples of 32.
+ */
+mx_status mx_quantize_dual(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt fmt,
+                           mx_scale_rounding rounding, void *row_elems, uint8_t *row_scales,
+                           void *col_elems, uint8_t *col_scales, mx_scale_layout layout,
+                           mx_stream_t stream);
+
+/*
+ * mx_dequantize -- codes and scales back to bf16 ([Q] §7: MX is an exponent add,
+ * x = dec(q) * 2^(s - 127), exact before the bf16 rounding; NVFP4 is
+ * (dec(q) * dec(sb)) * g in fp32).  A NaN scale makes the whole block NaN ([Q] §2).
+ *   elems, scales  device, as produced by mx_quantize(axis = ROW) for a rows x cols tensor.
+ *   global_scale   NVFP4 only: device fp32 g (else NULL).
+ *   layout         exactly one of ROWMAJOR / TCGEN05 (the layout of `scales`).
+ *   out_bf16       device, rows x cols bf16, 16-byte aligned; round to nearest even.
+ */
+mx_status mx_dequantize(const void *elems, const uint8_t *scales, const float *global_scale,
+                        int64_t rows, int64_t cols, mx_fmt fmt, mx_scale_layout layout,
+                        void *out_bf16, mx_stream_t stream);
+
+/*
+ * mx_cast -- the direct cast of [P4] "MXFP4": each bf16 value cast to the element format
+ * with no block scale (RNE, saturating).  NaN becomes 0x7F|sign (E4M3, E5M2) or the
+ * signed maximum 0x7|sign (E2M1, which has no NaN).
+ *   n           element count (even for E2M1); src and out 16-byte aligned.
+ */
+mx_status mx_cast(const void *src_bf16, int64_t n, mx_fmt fmt, void *out_elems, mx_stream_t stream);
+
+/*
+ * One operand of the block-scaled matmul: a rows x K matrix of codes, K-major (each row
+ * holds K consecutive codes), with E8M0 scales per 32 along K in the TCGEN05 layout
+ * (rows x K/32 scales), exactly as mx_quantize(axis = ROW, layout = TCGEN05) writes it.
+ */
+typedef struct {
+    const void *elems;
+    const uint8_t *scales;
+    mx_fmt fmt;
+} mx_operand;
+
+/*
+ * mx_gemm -- C = A * B^T with block scaling ([Q] §7; mixed MXFP4 x MXFP8 per [Q] §2
+ * and §6): C[m, n] = sum_k dec(A[m,k]) 2^(sA[m,k/32]-127) dec(B[n,k]) 2^(sB[n,k/32]-127),
+ * accumulated in fp32 on the tensor cores, written as bf16 (RNE).
+ *   A           M x K operand, fmt E4M3 (activations).
+ *   B           N x K operand, fmt E4M3 or E2M1 (weights).
+ *   C_bf16      device, M x N row-major bf16, 16-byte aligned.
+ *   Shapes: M and N multiples of 128, K a multiple of 128 (else MX_ERR_SHAPE).
+ *   Alignment: elems 32-byte aligned, scales 16-byte aligned (else MX_ERR_ALIGN).
+ */
+mx_status mx_gemm(mx_operand A, mx_operand B, void *C_bf16, int64_t M, int64_t N, int64_t K,
+                  mx_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char *mx_status_string(mx_status status);
+
+/* The CUDA error code (cudaError_t value) behind the last MX_ERR_CUDA on this host thread. */
+int mx_last_cuda_error(void);
+
+/*
+ * Watchdog: the pipelined kernels bound every wait on a barrier; a wait that gives up
+ * records a nonzero code in a device flag and the kernel returns early.  This call
+ * synchronises the current device, reads the flag (0 = no timeout) into *code and, if
+ * `clear`, resets it.  Returns MX_ERR_TIMEOUT if the flag was set, MX_OK otherwise.
+ */
+mx_status mx_watchdog_status(int *code, int clear);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MX_H_ */

@@ -1,0 +1,170 @@
+// codec.cuh -- device-side element and scale codecs for the MX kernels (sm_100a).
+//
+// Sources (page title, section):
+//   "MXFP4 と NVFP4 は何が違うのか調べてみた"
+//     §1 "E2M1 という共通土台": E2M1 has 15 values, max 6, no Inf/NaN.
+//     §2 "MXFP4 はブロック32と E8M0": E8M0 = 2^(c-127), 0xFF NaN; roundTiesToEven cast.
+//     §3 "NVFP4 はブロック16と E4M3、そして二段目": UE4M3 block scale, max 448.
+//     §4 "精度の差はどこから出るか": floor rule s = floor(log2 amax) - emax_elem
+//        (scaled max in [2^emax, 2^(emax+1))), and the no-clip rule (one step larger
+//        when the floor rule would clip).
+//
+// Every rounding is done by the hardware cvt.rn.satfinite conversions (round to nearest
+// even, saturate to the largest finite value); scale exponents come from the bf16
+// exponent field by integer arithmetic, and scales are applied as exact power-of-two
+// fp32 multiplies.
+#pragma once
+#include <cstdint>
+
+namespace mxk {
+
+enum : int { FMT_E4M3 = 0, FMT_E5M2 = 1, FMT_E2M1 = 2, FMT_NVFP4 = 3 };
+
+// Exponent of the largest binade of the element format (448 = 1.75 * 2^8,
+// 57344 = 1.75 * 2^15, 6 = 1.5 * 2^2) and 128 x the significand of its maximum.
+__host__ __device__ constexpr int emax_elem(int fmt) {
+    return fmt == FMT_E4M3 ? 8 : (fmt == FMT_E5M2 ? 15 : 2);
+}
+__host__ __device__ constexpr int max_sig128(int fmt) { return fmt == FMT_E2M1 ? 192 : 224; }
+
+// E8M0 code from the block maximum given as |x| bf16 bits (0 .. 0x7FFF).  Any
+// magnitude >= 0x7F80 (Inf or NaN) yields the NaN scale 0xFF.  A zero block yields
+// s = -127 (code 0).  The exponent is clamped to [-127, 127].
+template <int FMT, bool CEIL>
+__device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t a) {
+    if (a >= 0x7F80u) return 0xFFu;
+    if (a == 0u) return 0u;
+    int ef = (int)(a >> 7), mant = (int)(a & 0x7Fu);
+    int E, nm;
+    if (ef > 0) {            // normal: amax = (128 + mant)/128 * 2^(ef-127)
+        E = ef - 127;
+        nm = 128 | mant;
+    } else {                 // subnormal: amax = mant * 2^-133
+        int msb = 31 - __clz(mant);
+        E = -133 + msb;
+        nm = mant << (7 - msb);
+    }
+    int s = E - emax_elem(FMT);
+    if (CEIL && nm > max_sig128(FMT)) s += 1;   // floor rule would clip: one binade up
+    s = s < -127 ? -127 : (s > 127 ? 127 : s);
+    return (uint32_t)(s + 127);
+}
+
+// fp32 value 2^-(code-127), the multiplier that brings a block into the element range.
+__device__ __forceinline__ float e8m0_inverse_multiplier(uint32_t code) {
+    return code <= 253u ? __uint_as_float((254u - code) << 23) : __uint_as_float(0x00400000u);
+}
+
+// fp32 value 2^(code-127) for dequantisation (code 0 is the fp32 subnormal 2^-127).
+__device__ __forceinline__ float e8m0_multiplier(uint32_t code) {
+    return code >= 1u ? __uint_as_float(code << 23) : __uint_as_float(0x00400000u);
+}
+
+// bf16 pair packed in a 32-bit word (element 2i in the low half) -> two fp32.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Per-halfword |x| maximum over a 16-byte chunk of eight bf16 values.
+__device__ __forceinline__ uint32_t abs_max_bf16x8(const uint4 &v) {
+    uint32_t m = __vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu);
+    m = __vmaxu2(m, __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+    return m;
+}
+__device__ __forceinline__ uint32_t hmax(uint32_t m) { return max(m & 0xFFFFu, m >> 16); }
+
+// Same, ignoring Inf/NaN lanes (magnitude >= 0x7F80 treated as 0): NVFP4 tensor amax.
+__device__ __forceinline__ uint32_t finite_abs_max_bf16x8(const uint4 &v) {
+    uint32_t a0 = v.x & 0x7FFF7FFFu, a1 = v.y & 0x7FFF7FFFu, a2 = v.z & 0x7FFF7FFFu, a3 = v.w & 0x7FFF7FFFu;
+    a0 &= __vcmpltu2(a0, 0x7F807F80u);
+    a1 &= __vcmpltu2(a1, 0x7F807F80u);
+    a2 &= __vcmpltu2(a2, 0x7F807F80u);
+    a3 &= __vcmpltu2(a3, 0x7F807F80u);
+    return __vmaxu2(__vmaxu2(a0, a1), __vmaxu2(a2, a3));
+}
+
+// ---- hardware conversions (round to nearest even, satfinite) ---------------------------
+// Two fp32 -> two FP8 codes in one 16-bit word, `lo` in the low byte.
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt_fp8x2(float lo, float hi) {
+    uint16_t r;
+    if constexpr (FMT == FMT_E4M3)
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    else
+        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return (uint32_t)r;
+}
+
+// Eight fp32 -> eight E2M1 codes in one 32-bit word (element i in nibble i).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&x)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(x[0]), "f"(x[1]), "f"(x[2]), "f"(x[3]), "f"(x[4]), "f"(x[5]), "f"(x[6]), "f"(x[7]));
+    return r;
+}
+
+// Eight fp32 -> eight FP8 codes (uint2, element i in byte i).
+template <int FMT>
+__device__ __forceinline__ uint2 cvt_fp8x8(const float (&x)[8]) {
+    uint2 r;
+    r.x = cvt_fp8x2<FMT>(x[0], x[1]) | (cvt_fp8x2<FMT>(x[2], x[3]) << 16);
+    r.y = cvt_fp8x2<FMT>(x[4], x[5]) | (cvt_fp8x2<FMT>(x[6], x[7]) << 16);
+    return r;
+}
+
+// Two FP8 codes (16-bit word, element 2i low) -> two fp32, exact (via f16x2).
+template <int FMT>
+__device__ __forceinline__ void fp8x2_to_f32(uint32_t codes16, float &lo, float &hi) {
+    uint32_t h2;
+    uint16_t c = (uint16_t)codes16;
+    if constexpr (FMT == FMT_E4M3)
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    else
+        asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h2) : "h"(c));
+    asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(h2));
+}
+
+// Eight E2M1 codes (nibble i = element i) -> eight fp32, exact.
+__device__ __forceinline__ void e2m1x8_to_f32(uint32_t codes, float (&y)[8]) {
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(codes));
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        asm("{\n\t.reg .f16 l, hh;\n\tmov.b32 {l, hh}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, hh;\n\t}"
+            : "=f"(y[2 * i]), "=f"(y[2 * i + 1]) : "r"(h[i]));
+    }
+}
+
+// Two fp32 -> bf16x2 word (round to nearest even), `lo` in the low half.
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// UE4M3 code (0 .. 0x7E) -> fp32, exact (the NVFP4 block scale; [Q] §3 unsigned E4M3).
+__device__ __forceinline__ float ue4m3_to_f32(uint32_t code) {
+    float lo, hi;
+    fp8x2_to_f32<FMT_E4M3>(code & 0x7Fu, lo, hi);
+    return lo;
+}
+
+// tcgen05 scale tiling: byte offset of scale (r, c) for an output with S scale columns.
+__device__ __forceinline__ int64_t tcgen05_scale_offset(int64_t r, int64_t c, int64_t S) {
+    int64_t col_atoms = (S + 3) >> 2;
+    return (((r >> 7) * col_atoms + (c >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (c & 3);
+}
+
+}  // namespace mxk

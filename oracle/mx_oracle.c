@@ -345,7 +345,8 @@ int mxo_cast(const uint16_t *x, int64_t n, int fmt, uint8_t *out) {
  *      UE4M3 NaN code 0x7F and all element codes 0;
  *      t = amax_b / (6.0f * g);  sb = UE4M3 RNE-saturated code of t.
  *   4. d = dec(sb) * g.  If d == 0 every code is 0; otherwise r = 1.0f / d and
- *      q_i = E2M1 RNE-saturated code of (x_i * r).
+ *      q_i = E2M1 RNE-saturated code of (x_i * r); when 1/d overflows to Inf and x_i
+ *      is a zero, the NaN product is replaced by x_i itself (a signed zero code).
  * g is written to *g_out.  rows x cols row-major; blocks along rows (cols % 16 == 0);
  * elems rows x cols/2 bytes (even index low nibble), scales rows x cols/16.
  */
@@ -384,7 +385,9 @@ int mxo_quantize_nvfp4(const uint16_t *x, int64_t rows, int64_t cols, uint8_t *e
                     unsigned q = 0;
                     if (d != 0.0f) {
                         volatile float rcp = 1.0f / d;
-                        volatile float y = (float)bf16_value(blk[i]) * rcp;
+                        volatile float xi = (float)bf16_value(blk[i]);
+                        volatile float y = xi * rcp;
+                        if (isnan(y)) y = xi;     /* 0 * Inf when 1/d overflows: keep the signed zero */
                         q = mxo_encode((double)y, K_E2M1);
                     }
                     put_code(elems + r * (cols / 2), b * B + i, q, 1);
