@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the MX hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-breakdown]
+
+One step = one pass of the weight-quantisation workload over a 4096 x 4096 bf16 matrix
+(N(0, 0.02) with 0.1% N(0, 1) outliers): MXFP4 (E2M1, block 32, E8M0, floor scale) and
+NVFP4 (E2M1, block 16, UE4M3 + fp32 tensor scale), each emitting both the row-major and
+the tcgen05 scale layouts.  value = algorithmic bytes of the step / step time (GB/s).
+The input (32 MiB) is smaller than L2, so L2 is flushed (a 256 MiB write) between timed
+steps, outside the per-step CUDA-event pairs.  Every other row of the hot path (row-wise
+MXFP8 quantise + dequantise, dual-orientation quantisation, dequantisation, the two
+block-scaled matmuls) is measured in "breakdown", each against its own roofline.
+
+Multi-GPU (torchrun): every rank quantises its own weight matrix (independent units, no
+data-path collective); value = all ranks' bytes / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MX quantize GB/s (frac of HBM peak); block-scaled GEMM TFLOPS (frac of MX peak)"
+HBM_NOMINAL_GBS = 8000.0
+MX_NOMINAL_TFLOPS = 4500.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# algorithmic bytes (read input once + write codes and scales once)
+R2 = C2 = 4096
+BYTES_MXFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 32)            # 42,991,616
+BYTES_NVFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 16) + 4         # 44,040,196
+STEP_BYTES = BYTES_MXFP4 + BYTES_NVFP4
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK, source="fallback")
+
+
+# ----------------------------------------------------------------------------- utilities
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+class L2Flush:
+    def __init__(self, dev):
+        self.buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1)
+
+
+def to_dev(bits, dev):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def event_pair():
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+# ----------------------------------------------------------------------------- our step
+class WeightQuantStep:
+    """MXFP4 (floor) + NVFP4 quantisation of one 4096 x 4096 bf16 weight, both layouts."""
+
+    def __init__(self, mx, x_dev):
+        from microscaling_precision_number_b200 import _lib as L
+        self.mx, self.L = mx, L
+        self.x = x_dev
+        dev = x_dev.device
+        R, C = x_dev.shape
+        self.R, self.C = R, C
+        self.e4 = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
+        self.s4 = torch.empty(R * C // 32, dtype=torch.uint8, device=dev)
+        self.s4t = torch.empty(mx.scale_bytes(R, C // 32, "tcgen05"), dtype=torch.uint8, device=dev)
+        self.en = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
+        self.sn = torch.empty(R * C // 16, dtype=torch.uint8, device=dev)
+        self.snt = torch.empty(mx.scale_bytes(R, C // 16, "tcgen05"), dtype=torch.uint8, device=dev)
+        self.g = torch.empty(1, dtype=torch.float32, device=dev)
+        self.launches_per_step = 3      # MXFP4 quantiser; NVFP4 amax + quantiser (no padding at 4096)
+
+    def mxfp4(self, stream):
+        L = self.L
+        L.check(L.lib.mx_quantize(self.x.data_ptr(), self.R, self.C, L.MX_FMT_E2M1, L.MX_AXIS_ROW,
+                                  L.MX_SCALE_FLOOR_OCP, self.e4.data_ptr(), self.s4.data_ptr(), 3,
+                                  self.s4t.data_ptr(), None, stream), "mx_quantize(mxfp4)")
+
+    def nvfp4(self, stream):
+        L = self.L
+        L.check(L.lib.mx_quantize(self.x.data_ptr(), self.R, self.C, L.MX_FMT_NVFP4, L.MX_AXIS_ROW,
+                                  L.MX_SCALE_CEIL_RECIPE, self.en.data_ptr(), self.sn.data_ptr(), 3,
+                                  self.snt.data_ptr(), self.g.data_ptr(), stream), "mx_quantize(nvfp4)")
+
+    def outputs(self):
+        return [self.e4, self.s4, self.s4t, self.en, self.sn, self.snt, self.g]
+
+
+def run_ours(args, rank, world, dev):
+    import microscaling_precision_number_b200 as mx
+
+    pk = peaks()
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    sptr = stream.cuda_stream
+    x_bits = synth.weight_fp4(seed=rank)
+    x = to_dev(x_bits, dev)
+    step = WeightQuantStep(mx, x)
+    flush = L2Flush(dev)
+
+    for _ in range(args.warmup):
+        step.mxfp4(sptr)
+        step.nvfp4(sptr)
+    torch.cuda.synchronize()
+
+    # timed region: K steps, per-call events, L2 flushed between steps (outside the events)
+    ev = [[event_pair(), event_pair()] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for k in range(args.steps):
+            flush()
+            (a0, a1), (b0, b1) = ev[k]
+            a0.record(stream)
+            step.mxfp4(sptr)
+            a1.record(stream)
+            b0.record(stream)
+            step.nvfp4(sptr)
+            b1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t_mx = [e[0][0].elapsed_time(e[0][1]) for e in ev]
+    t_nv = [e[1][0].elapsed_time(e[1][1]) for e in ev]
+    step_ms = [a + b for a, b in zip(t_mx, t_nv)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = STEP_BYTES * world * args.steps / (total_ms * 1e-3) / 1e9
+
+    # dominant call and its roofline
+    mean_mx, mean_nv = statistics.mean(t_mx), statistics.mean(t_nv)
+    if mean_nv >= mean_mx:
+        dom = {"kernel": "mx_quantize(NVFP4): nvfp4_amax_kernel + nvfp4_quant_kernel", "ms": mean_nv,
+               "bytes": BYTES_NVFP4}
+    else:
+        dom = {"kernel": "mx_quantize(MXFP4): quant_rows_mx_kernel<E2M1,floor,both layouts>", "ms": mean_mx,
+               "bytes": BYTES_MXFP4}
+    achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                "peak_source": pk["source"] + " copy bandwidth (MEASURED_PEAKS hbm_gbs)",
+                "kernel": dom["kernel"], "algorithmic_bytes_per_launch": dom["bytes"],
+                "ms_per_launch": round(dom["ms"], 5),
+                "calls": {"mxfp4_ms": round(mean_mx, 5), "mxfp4_GBps": round(BYTES_MXFP4 / mean_mx / 1e6, 1),
+                          "nvfp4_ms": round(mean_nv, 5), "nvfp4_GBps": round(BYTES_NVFP4 / mean_nv / 1e6, 1)},
+                "frac_of_nominal_8TBps": round(achieved / HBM_NOMINAL_GBS, 4)}
+
+    # end to end through the public API with host buffers (pinned), copies inside the timing
+    x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in step.outputs()]
+    h2d = x_host.numel() * 2
+    d2h = sum(o.numel() * o.element_size() for o in outs_host)
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        step.mxfp4(sptr)
+        step.nvfp4(sptr)
+        for h, d in zip(outs_host, step.outputs()):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = event_pair()
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(STEP_BYTES * world * args.steps / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": round(e2e_ms / args.steps, 4)}
+
+    breakdown = None
+    if not args.no_breakdown and rank == 0:
+        breakdown = run_breakdown(mx, dev, pk, flush)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(x_bits, target_s=args.cpu_seconds)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (numpy default_rng, seed = rank)",
+                "config": {"workload": "weight_4096x4096_mxfp4_floor_and_nvfp4_both_scale_layouts",
+                           "shape": [R2, C2], "formats": ["MXFP4 E2M1/E8M0 floor block 32",
+                                                          "NVFP4 E2M1/UE4M3+fp32 block 16"],
+                           "step_bytes": STEP_BYTES, "l2": "flushed between steps (256 MiB write)",
+                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": step.launches_per_step * args.steps, "clocks": clk.summary()}
+        if breakdown is not None:
+            line["breakdown"] = breakdown
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- breakdown
+def timed(fn, iters, flush, stream):
+    ts = []
+    for _ in range(iters):
+        if flush is not None:
+            flush()
+        a, b = event_pair()
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return statistics.median(ts)
+
+
+def run_breakdown(mx, dev, pk, flush):
+    stream = torch.cuda.current_stream()
+    out = {}
+    hbm = pk["hbm_gbs"]
+    mx_peak = 2.0 * pk["bf16_tflops"]          # FP8 / mxf8f6f4 rate = 2 x the bf16 rate
+
+    # C1: MXFP8 E4M3 row-wise quantise + dequantise, 1024 x 1024 (launch-latency bound)
+    x1 = to_dev(synth.mx8_rowwise(), dev)
+    q1 = mx.quantize(x1, "e4m3", "row", "ceil", layout="rowmajor")
+    for _ in range(5):
+        mx.quantize(x1, "e4m3", "row", "ceil", layout="rowmajor")
+    tq = timed(lambda: mx.quantize(x1, "e4m3", "row", "ceil", layout="rowmajor"), 30, flush, stream)
+    td = timed(lambda: mx.dequantize(q1, "rowmajor"), 30, flush, stream)
+    b1 = 1024 * 1024 * 2 + 1024 * 1024 + 1024 * 32
+    out["c1_mxfp8_rowwise_1024"] = {"quantize_us": round(tq * 1e3, 2), "dequantize_us": round(td * 1e3, 2),
+                                    "quantize_GBps": round(b1 / tq / 1e6, 1),
+                                    "dequantize_GBps": round(b1 / td / 1e6, 1),
+                                    "frac_hbm": round(b1 / tq / 1e6 / hbm, 4),
+                                    "note": "3.2 MB per call: launch-latency bound"}
+    del x1, q1
+
+    # a7: dequantise the config-2 weight (MXFP4 and NVFP4), tcgen05 scales
+    xw = to_dev(synth.weight_fp4(), dev)
+    q4 = mx.quantize(xw, "e2m1", "row", "floor", layout="tcgen05")
+    qn = mx.quantize(xw, "nvfp4", "row", "ceil", layout="tcgen05")
+    t4 = timed(lambda: mx.dequantize(q4, "tcgen05"), 20, flush, stream)
+    tn = timed(lambda: mx.dequantize(qn, "tcgen05"), 20, flush, stream)
+    bd4 = R2 * C2 // 2 + R2 * C2 // 32 + R2 * C2 * 2
+    bdn = R2 * C2 // 2 + R2 * C2 // 16 + 4 + R2 * C2 * 2
+    out["a7_dequantize_4096"] = {"mxfp4_GBps": round(bd4 / t4 / 1e6, 1), "mxfp4_frac_hbm": round(bd4 / t4 / 1e6 / hbm, 4),
+                                 "nvfp4_GBps": round(bdn / tn / 1e6, 1), "nvfp4_frac_hbm": round(bdn / tn / 1e6 / hbm, 4)}
+    del xw, q4, qn
+
+    # C3: dual-orientation MXFP8, activations (E4M3) and gradients (E5M2), tcgen05 scales
+    for name, gen, fmt in (("act_16384x4096_e4m3", synth.activations, "e4m3"),
+                           ("grad_16384x14336_e5m2", synth.gradients, "e5m2")):
+        xb = gen()
+        R, C = xb.shape
+        x3 = to_dev(xb, dev)
+        del xb
+        res = mx.quantize_dual(x3, fmt, "ceil", "tcgen05")
+        t = timed(lambda: mx.quantize_dual(x3, fmt, "ceil", "tcgen05"), 10, None, stream)
+        nbytes = R * C * 2 + 2 * (R * C + R * C // 32)
+        out[f"c3_dual_{name}"] = {"ms": round(t, 4), "GBps": round(nbytes / t / 1e6, 1),
+                                  "frac_hbm": round(nbytes / t / 1e6 / hbm, 4), "algorithmic_bytes": nbytes,
+                                  "l2": "input larger than L2"}
+        del x3, res
+        torch.cuda.empty_cache()
+
+    # C4 / C5: block-scaled matmuls (operands quantised outside the timing)
+    for name, (M, N, K), bfmt, bsig in (("c4_gemm_e4m3_8192", (8192, 8192, 8192), "e4m3", 1.0),
+                                       ("c5_gemm_e4m3_x_e2m1_8192x14336x4096", (8192, 14336, 4096), "e2m1", 0.02)):
+        a = mx.quantize(to_dev(synth.normal(M, K, seed=40), dev), "e4m3", "row", "ceil", layout="tcgen05")
+        b = mx.quantize(to_dev(synth.normal(N, K, sigma=bsig, seed=41), dev), bfmt, "row",
+                        "floor" if bfmt == "e2m1" else "ceil", layout="tcgen05")
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            mx.gemm(a, b, c)
+        t = timed(lambda: mx.gemm(a, b, c), 10, None, stream)
+        tf = 2.0 * M * N * K / (t * 1e-3) / 1e12
+        out[name] = {"ms": round(t, 4), "TFLOPS": round(tf, 1), "frac_mx_peak_measured": round(tf / mx_peak, 4),
+                     "mx_peak_measured_TFLOPS": mx_peak, "frac_mx_nominal_4500": round(tf / MX_NOMINAL_TFLOPS, 4),
+                     "peak_note": "bf16 burst (MEASURED_PEAKS) x 2, the FP8/f8f6f4 to bf16 nominal ratio"}
+        del a, b, c
+        torch.cuda.empty_cache()
+    return out
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(x_bits, target_s=12.0):
+    """The oracle as it stands, single-threaded, on a bounded row sample of the workload."""
+    import oracle
+    oracle.lib()
+    rows = 64
+    t0 = time.perf_counter()
+    done_rows = 0
+    while True:
+        xs = np.ascontiguousarray(x_bits[done_rows % R2: done_rows % R2 + rows])
+        e4, s4 = oracle.quantize_mx(xs, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+        oracle.to_tcgen05_layout(s4)
+        en, sn, g = oracle.quantize_nvfp4(xs)
+        oracle.to_tcgen05_layout(sn)
+        done_rows += rows
+        if time.perf_counter() - t0 > target_s or done_rows >= R2:
+            break
+    dt = time.perf_counter() - t0
+    bytes_done = STEP_BYTES * done_rows / R2
+    return {"value": round(bytes_done / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done_rows} of {R2} rows of the 4096x4096 weight (MXFP4 + NVFP4, both layouts), "
+                      f"{dt:.1f} s single-threaded", "seconds": round(dt, 2)}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: rank 0 only, bounded sample per step."""
+    if rank != 0:
+        return
+    x_bits = synth.weight_fp4(seed=0)
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(x_bits, target_s=per_step)
+    vals, secs = [], []
+    for _ in range(args.steps):
+        r = cpu_baseline(x_bits, target_s=per_step)
+        vals.append(r["value"])
+        secs.append(r["seconds"])
+        sample = r["sample"]
+    v = statistics.mean(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (numpy default_rng, seed 0)",
+            "config": {"workload": "weight_4096x4096_mxfp4_floor_and_nvfp4_both_scale_layouts", "shape": [R2, C2]},
+            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(v, 5)},
+            "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        run_ours(args, rank, world, dev)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

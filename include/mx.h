@@ -185,6 +185,9 @@ int mx_last_cuda_error(void);
  * records a nonzero code in a device flag and the kernel returns early.  This call
  * synchronises the current device, reads the flag (0 = no timeout) into *code and, if
  * `clear`, resets it.  Returns MX_ERR_TIMEOUT if the flag was set, MX_OK otherwise.
+ * While the flag is set, pipelined kernels give up their waits at once (so one stuck
+ * CTA cannot stall a whole grid); outputs of calls made while it is set are undefined.
+ * Clear it to resume normal operation.
  */
 mx_status mx_watchdog_status(int *code, int clear);
 

@@ -1,0 +1,70 @@
+"""ctypes loader for libmx.so, the C ABI declared in include/mx.h.
+
+Only argument marshalling lives here.  There is no fallback: if the shared library is
+missing or cannot be loaded, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmx.so")
+
+# enum values of include/mx.h
+MX_OK, MX_ERR_ARG, MX_ERR_SHAPE, MX_ERR_ALIGN, MX_ERR_LAYOUT, MX_ERR_CUDA, MX_ERR_TIMEOUT = range(7)
+MX_FMT_E4M3, MX_FMT_E5M2, MX_FMT_E2M1, MX_FMT_NVFP4 = 0, 1, 2, 3
+MX_AXIS_ROW, MX_AXIS_COL = 0, 1
+MX_SCALE_FLOOR_OCP, MX_SCALE_CEIL_RECIPE = 0, 1
+MX_LAYOUT_ROWMAJOR, MX_LAYOUT_TCGEN05 = 1, 2
+
+# Every function the header declares (the CPU test checks the library exports them all).
+EXPORTS = ("mx_scale_bytes", "mx_quantize", "mx_quantize_dual", "mx_dequantize", "mx_cast",
+           "mx_gemm", "mx_status_string", "mx_last_cuda_error", "mx_watchdog_status")
+
+
+class MxOperand(ctypes.Structure):
+    _fields_ = [("elems", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("fmt", ctypes.c_int)]
+
+
+class MxError(RuntimeError):
+    def __init__(self, status: int, where: str, lib):
+        self.status = status
+        msg = lib.mx_status_string(status).decode()
+        if status == MX_ERR_CUDA:
+            msg += f" (cudaError {lib.mx_last_cuda_error()})"
+        super().__init__(f"{where}: {msg}")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libmx.so not built ({LIB_PATH}); run python -m microscaling_precision_number_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I, U8P = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+    lib.mx_scale_bytes.argtypes = [I64, I64, I]
+    lib.mx_scale_bytes.restype = I64
+    lib.mx_quantize.argtypes = [P, I64, I64, I, I, I, P, U8P, I, U8P, P, P]
+    lib.mx_quantize.restype = I
+    lib.mx_quantize_dual.argtypes = [P, I64, I64, I, I, P, U8P, P, U8P, I, P]
+    lib.mx_quantize_dual.restype = I
+    lib.mx_dequantize.argtypes = [P, U8P, P, I64, I64, I, I, P, P]
+    lib.mx_dequantize.restype = I
+    lib.mx_cast.argtypes = [P, I64, I, P, P]
+    lib.mx_cast.restype = I
+    lib.mx_gemm.argtypes = [MxOperand, MxOperand, P, I64, I64, I64, P]
+    lib.mx_gemm.restype = I
+    lib.mx_status_string.argtypes = [I]
+    lib.mx_status_string.restype = ctypes.c_char_p
+    lib.mx_last_cuda_error.argtypes = []
+    lib.mx_last_cuda_error.restype = I
+    lib.mx_watchdog_status.argtypes = [ctypes.POINTER(ctypes.c_int), I]
+    lib.mx_watchdog_status.restype = I
+    return lib
+
+
+lib = _load()
+
+
+def check(status: int, where: str) -> None:
+    if status != MX_OK:
+        raise MxError(status, where, lib)

@@ -1,0 +1,146 @@
+"""Torch-facing wrappers over the C ABI: allocate outputs with torch (device memory),
+pass raw pointers and the current CUDA stream, check the status.  No arithmetic of the
+method happens here; every step runs in the CUDA kernels behind libmx.so.
+"""
+from __future__ import annotations
+
+from typing import NamedTuple, Optional
+
+import torch
+
+from . import _lib as L
+
+FMTS = {"e4m3": L.MX_FMT_E4M3, "e5m2": L.MX_FMT_E5M2, "e2m1": L.MX_FMT_E2M1, "nvfp4": L.MX_FMT_NVFP4}
+ROUNDING = {"floor": L.MX_SCALE_FLOOR_OCP, "ceil": L.MX_SCALE_CEIL_RECIPE}
+LAYOUTS = {"rowmajor": L.MX_LAYOUT_ROWMAJOR, "tcgen05": L.MX_LAYOUT_TCGEN05,
+           "both": L.MX_LAYOUT_ROWMAJOR | L.MX_LAYOUT_TCGEN05}
+
+
+def _fmt(f) -> int:
+    return FMTS[f] if isinstance(f, str) else int(f)
+
+
+def block_of(fmt) -> int:
+    return 16 if _fmt(fmt) == L.MX_FMT_NVFP4 else 32
+
+
+def is_fp4(fmt) -> bool:
+    return _fmt(fmt) in (L.MX_FMT_E2M1, L.MX_FMT_NVFP4)
+
+
+def elem_bytes(rows: int, cols: int, fmt) -> int:
+    return rows * cols // 2 if is_fp4(fmt) else rows * cols
+
+
+def scale_bytes(rows: int, scale_cols: int, layout) -> int:
+    lay = LAYOUTS[layout] if isinstance(layout, str) else int(layout)
+    n = L.lib.mx_scale_bytes(rows, scale_cols, lay)
+    if n < 0:
+        raise ValueError("invalid scale layout")
+    return n
+
+
+def _stream(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _check_src(x: torch.Tensor):
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() != 2:
+        raise ValueError("expected a contiguous 2-D bf16 CUDA tensor")
+
+
+class Quantized(NamedTuple):
+    elems: torch.Tensor          # uint8 codes (FP4: two per byte, even index low nibble)
+    scales: torch.Tensor         # uint8 scales in the first layout
+    scales_alt: Optional[torch.Tensor]   # tcgen05 scales when layout == "both"
+    global_scale: Optional[torch.Tensor]  # NVFP4 fp32 g
+    rows: int                    # shape of the quantised (possibly transposed) matrix
+    cols: int
+    fmt: int
+
+
+def quantize(x: torch.Tensor, fmt="e4m3", axis: str = "row", rounding: str = "ceil",
+             layout: str = "rowmajor", stream=None) -> Quantized:
+    _check_src(x)
+    f = _fmt(fmt)
+    rows, cols = x.shape
+    orows, ocols = (rows, cols) if axis == "row" else (cols, rows)
+    B = block_of(f)
+    dev = x.device
+    elems = torch.empty(elem_bytes(orows, ocols, f), dtype=torch.uint8, device=dev)
+    lay = LAYOUTS[layout]
+    first = "rowmajor" if layout in ("rowmajor", "both") else "tcgen05"
+    scales = torch.empty(scale_bytes(orows, ocols // B, first), dtype=torch.uint8, device=dev)
+    alt = torch.empty(scale_bytes(orows, ocols // B, "tcgen05"), dtype=torch.uint8, device=dev) \
+        if layout == "both" else None
+    g = torch.empty(1, dtype=torch.float32, device=dev) if f == L.MX_FMT_NVFP4 else None
+    st = L.lib.mx_quantize(x.data_ptr(), rows, cols, f, L.MX_AXIS_ROW if axis == "row" else L.MX_AXIS_COL,
+                           ROUNDING[rounding], elems.data_ptr(), scales.data_ptr(), lay, _ptr(alt), _ptr(g),
+                           _stream(stream))
+    L.check(st, "mx_quantize")
+    return Quantized(elems, scales, alt, g, orows, ocols, f)
+
+
+def quantize_dual(x: torch.Tensor, fmt="e4m3", rounding: str = "ceil", layout: str = "tcgen05", stream=None):
+    """Row-wise and column-wise (transposed) quantisation from one read of x."""
+    _check_src(x)
+    f = _fmt(fmt)
+    rows, cols = x.shape
+    dev = x.device
+    re = torch.empty(elem_bytes(rows, cols, f), dtype=torch.uint8, device=dev)
+    ce = torch.empty(elem_bytes(rows, cols, f), dtype=torch.uint8, device=dev)
+    rs = torch.empty(scale_bytes(rows, cols // 32, layout), dtype=torch.uint8, device=dev)
+    cs = torch.empty(scale_bytes(cols, rows // 32, layout), dtype=torch.uint8, device=dev)
+    st = L.lib.mx_quantize_dual(x.data_ptr(), rows, cols, f, ROUNDING[rounding], re.data_ptr(), rs.data_ptr(),
+                                ce.data_ptr(), cs.data_ptr(), LAYOUTS[layout], _stream(stream))
+    L.check(st, "mx_quantize_dual")
+    return (Quantized(re, rs, None, None, rows, cols, f), Quantized(ce, cs, None, None, cols, rows, f))
+
+
+def dequantize(q: Quantized, layout: str = "rowmajor", stream=None) -> torch.Tensor:
+    scales = q.scales if (layout == "rowmajor" or q.scales_alt is None) else q.scales_alt
+    out = torch.empty((q.rows, q.cols), dtype=torch.bfloat16, device=q.elems.device)
+    st = L.lib.mx_dequantize(q.elems.data_ptr(), scales.data_ptr(), _ptr(q.global_scale), q.rows, q.cols, q.fmt,
+                             LAYOUTS[layout], out.data_ptr(), _stream(stream))
+    L.check(st, "mx_dequantize")
+    return out
+
+
+def cast(x: torch.Tensor, fmt="e4m3", stream=None) -> torch.Tensor:
+    """Direct cast with no block scale (codes, FP4 packed two per byte)."""
+    if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("expected a contiguous bf16 CUDA tensor")
+    f = _fmt(fmt)
+    out = torch.empty(elem_bytes(1, x.numel(), f), dtype=torch.uint8, device=x.device)
+    L.check(L.lib.mx_cast(x.data_ptr(), x.numel(), f, out.data_ptr(), _stream(stream)), "mx_cast")
+    return out
+
+
+def gemm(a: Quantized, b: Quantized, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """C = A * B^T for A (M x K) and B (N x K) quantised row-wise with tcgen05 scales."""
+    M, K = a.rows, a.cols
+    N = b.rows
+    if b.cols != K:
+        raise ValueError("K mismatch")
+    sa = a.scales_alt if a.scales_alt is not None else a.scales
+    sb = b.scales_alt if b.scales_alt is not None else b.scales
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.elems.device)
+    A = L.MxOperand(a.elems.data_ptr(), sa.data_ptr(), a.fmt)
+    B = L.MxOperand(b.elems.data_ptr(), sb.data_ptr(), b.fmt)
+    L.check(L.lib.mx_gemm(A, B, out.data_ptr(), M, N, K, _stream(stream)), "mx_gemm")
+    return out
+
+
+def watchdog_status(clear: bool = True) -> int:
+    import ctypes
+    code = ctypes.c_int(0)
+    st = L.lib.mx_watchdog_status(ctypes.byref(code), 1 if clear else 0)
+    if st not in (L.MX_OK, L.MX_ERR_TIMEOUT):
+        L.check(st, "mx_watchdog_status")
+    return code.value

@@ -1,0 +1,293 @@
+// api.cu -- the C ABI of include/mx.h: argument validation, per-device state and dispatch
+// to the kernels.  Validation happens entirely on the host before any CUDA call, so a
+// rejected call never touches the device.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <mutex>
+
+#include "../../include/mx.h"
+#include "internal.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+__device__ int g_watchdog_flag = 0;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+    int *watchdog = nullptr;     // device address of g_watchdog_flag
+    float *partials = nullptr;   // NVFP4 per-CTA maxima (scratch, allocated once)
+    int partials_cap = 0;
+};
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+mx_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = (int)e;
+    return MX_ERR_CUDA;
+}
+
+mx_status device_state(DeviceState **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return MX_ERR_ARG;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState &d = g_dev[dev];
+    if (!d.ready) {
+        e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = cudaGetSymbolAddress(reinterpret_cast<void **>(&d.watchdog), g_watchdog_flag);
+        if (e != cudaSuccess) return cuda_fail(e);
+        d.ready = true;
+    }
+    *out = &d;
+    return MX_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool fmt_ok(int f) { return f >= MX_FMT_E4M3 && f <= MX_FMT_NVFP4; }
+int block_of(int f) { return f == MX_FMT_NVFP4 ? 16 : 32; }
+bool single_layout(int l) { return l == MX_LAYOUT_ROWMAJOR || l == MX_LAYOUT_TCGEN05; }
+
+}  // namespace
+
+namespace mxk {
+void *tensor_map_encoder() {
+    static void *fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = p;
+    });
+    return fn;
+}
+}  // namespace mxk
+
+extern "C" {
+
+int64_t mx_scale_bytes(int64_t rows, int64_t scale_cols, mx_scale_layout layout) {
+    if (rows < 0 || scale_cols < 0) return -1;
+    if (layout == MX_LAYOUT_ROWMAJOR) return rows * scale_cols;
+    if (layout == MX_LAYOUT_TCGEN05) return ((rows + 127) / 128) * ((scale_cols + 3) / 4) * 512;
+    return -1;
+}
+
+const char *mx_status_string(mx_status s) {
+    switch (s) {
+    case MX_OK: return "MX_OK";
+    case MX_ERR_ARG: return "MX_ERR_ARG: null pointer, unknown enum or unsupported combination";
+    case MX_ERR_SHAPE: return "MX_ERR_SHAPE: negative size or size not a multiple of the block/tile";
+    case MX_ERR_ALIGN: return "MX_ERR_ALIGN: pointer not aligned as required";
+    case MX_ERR_LAYOUT: return "MX_ERR_LAYOUT: invalid scale layout mask or missing second scale buffer";
+    case MX_ERR_CUDA: return "MX_ERR_CUDA: CUDA call failed (see mx_last_cuda_error)";
+    case MX_ERR_TIMEOUT: return "MX_ERR_TIMEOUT: a bounded device wait gave up";
+    default: return "unknown mx_status";
+    }
+}
+
+int mx_last_cuda_error(void) { return g_last_cuda_error; }
+
+mx_status mx_watchdog_status(int *code, int clear) {
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e);
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, g_watchdog_flag, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (clear && v) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_watchdog_flag, &zero, sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (code) *code = v;
+    return v ? MX_ERR_TIMEOUT : MX_OK;
+}
+
+mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, mx_axis axis,
+                      mx_scale_rounding rounding, void *out_elems, uint8_t *out_scales,
+                      mx_scale_layout layout, uint8_t *out_scales_alt, float *global_scale,
+                      mx_stream_t stream) {
+    if (!fmt_ok(fmt) || (axis != MX_AXIS_ROW && axis != MX_AXIS_COL) ||
+        (rounding != MX_SCALE_FLOOR_OCP && rounding != MX_SCALE_CEIL_RECIPE))
+        return MX_ERR_ARG;
+    if (fmt == MX_FMT_NVFP4 && axis != MX_AXIS_ROW) return MX_ERR_ARG;
+    if ((fmt == MX_FMT_NVFP4) != (global_scale != nullptr)) return MX_ERR_ARG;
+    if (layout != MX_LAYOUT_ROWMAJOR && layout != MX_LAYOUT_TCGEN05 &&
+        layout != (MX_LAYOUT_ROWMAJOR | MX_LAYOUT_TCGEN05))
+        return MX_ERR_LAYOUT;
+    const bool both = layout == (MX_LAYOUT_ROWMAJOR | MX_LAYOUT_TCGEN05);
+    if (both != (out_scales_alt != nullptr)) return MX_ERR_LAYOUT;
+    if (rows < 0 || cols < 0) return MX_ERR_SHAPE;
+    const int B = block_of(fmt);
+    if ((axis == MX_AXIS_ROW ? cols : rows) % B) return MX_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MX_OK;
+    if (!src || !out_elems || !out_scales) return MX_ERR_ARG;
+    if (!aligned(src, 16) || !aligned(out_elems, 16)) return MX_ERR_ALIGN;
+    if (global_scale && !aligned(global_scale, 4)) return MX_ERR_ALIGN;
+
+    uint8_t *rm = nullptr, *tc = nullptr;
+    if (both) { rm = out_scales; tc = out_scales_alt; }
+    else if (layout == MX_LAYOUT_ROWMAJOR) rm = out_scales;
+    else tc = out_scales;
+
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    const bool ceil = rounding == MX_SCALE_CEIL_RECIPE;
+
+    if (fmt == MX_FMT_NVFP4) {
+        const int np = mxk::nvfp4_partials_count(rows * cols, d->num_sms);
+        {
+            std::lock_guard<std::mutex> lock(g_mu);
+            if (d->partials_cap < np) {
+                if (d->partials) cudaFree(d->partials);
+                d->partials = nullptr;
+                d->partials_cap = 0;
+                e = cudaMalloc(reinterpret_cast<void **>(&d->partials), sizeof(float) * (size_t)np);
+                if (e != cudaSuccess) return cuda_fail(e);
+                d->partials_cap = np;
+            }
+        }
+        e = mxk::launch_nvfp4_amax(src, rows * cols, d->partials, np, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = mxk::launch_nvfp4_quant(src, rows, cols, d->partials, np, global_scale, out_elems, rm, tc,
+                                    d->num_sms, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (tc) {
+            e = mxk::launch_tcgen05_pad(tc, rows, cols / 16, s);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        return MX_OK;
+    }
+
+    if (axis == MX_AXIS_ROW) {
+        e = mxk::launch_quant_rows_mx(src, rows, cols, fmt, ceil, out_elems, rm, tc, d->num_sms, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (tc) {
+            e = mxk::launch_tcgen05_pad(tc, rows, cols / 32, s);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        return MX_OK;
+    }
+
+    // Column-wise: the TMA-staged kernel with only the transposed output enabled.  It
+    // takes one scale layout per call; with both requested, run it once per layout.
+    if (cols % 8 != 0) return MX_ERR_SHAPE;    // the TMA row pitch (cols * 2 bytes) must be a multiple of 16
+    uint8_t *first = rm ? rm : tc;
+    e = mxk::launch_quant_dual(src, rows, cols, fmt, ceil, nullptr, nullptr, out_elems, first, first == tc,
+                               d->watchdog, d->num_sms, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (rm && tc) {
+        e = mxk::launch_quant_dual(src, rows, cols, fmt, ceil, nullptr, nullptr, out_elems, tc, true,
+                                   d->watchdog, d->num_sms, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    if (tc) {
+        e = mxk::launch_tcgen05_pad(tc, cols, rows / 32, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return MX_OK;
+}
+
+mx_status mx_quantize_dual(const void *src, int64_t rows, int64_t cols, mx_fmt fmt,
+                           mx_scale_rounding rounding, void *row_elems, uint8_t *row_scales,
+                           void *col_elems, uint8_t *col_scales, mx_scale_layout layout,
+                           mx_stream_t stream) {
+    if (fmt != MX_FMT_E4M3 && fmt != MX_FMT_E5M2 && fmt != MX_FMT_E2M1) return MX_ERR_ARG;
+    if (rounding != MX_SCALE_FLOOR_OCP && rounding != MX_SCALE_CEIL_RECIPE) return MX_ERR_ARG;
+    if (!single_layout(layout)) return MX_ERR_LAYOUT;
+    if (rows < 0 || cols < 0) return MX_ERR_SHAPE;
+    if (rows % 32 || cols % 32) return MX_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MX_OK;
+    if (!src || !row_elems || !row_scales || !col_elems || !col_scales) return MX_ERR_ARG;
+    if (!aligned(src, 16) || !aligned(row_elems, 16) || !aligned(col_elems, 16)) return MX_ERR_ALIGN;
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool tc = layout == MX_LAYOUT_TCGEN05;
+    cudaError_t e = mxk::launch_quant_dual(src, rows, cols, fmt, rounding == MX_SCALE_CEIL_RECIPE, row_elems,
+                                           row_scales, col_elems, col_scales, tc, d->watchdog, d->num_sms, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (tc) {
+        e = mxk::launch_tcgen05_pad(row_scales, rows, cols / 32, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+        e = mxk::launch_tcgen05_pad(col_scales, cols, rows / 32, s);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return MX_OK;
+}
+
+mx_status mx_dequantize(const void *elems, const uint8_t *scales, const float *global_scale,
+                        int64_t rows, int64_t cols, mx_fmt fmt, mx_scale_layout layout,
+                        void *out_bf16, mx_stream_t stream) {
+    if (!fmt_ok(fmt)) return MX_ERR_ARG;
+    if ((fmt == MX_FMT_NVFP4) != (global_scale != nullptr)) return MX_ERR_ARG;
+    if (!single_layout(layout)) return MX_ERR_LAYOUT;
+    if (rows < 0 || cols < 0) return MX_ERR_SHAPE;
+    if (cols % block_of(fmt)) return MX_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MX_OK;
+    if (!elems || !scales || !out_bf16) return MX_ERR_ARG;
+    if (!aligned(elems, 16) || !aligned(out_bf16, 16)) return MX_ERR_ALIGN;
+    if (global_scale && !aligned(global_scale, 4)) return MX_ERR_ALIGN;
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool tc = layout == MX_LAYOUT_TCGEN05;
+    cudaError_t e = fmt == MX_FMT_NVFP4
+                        ? mxk::launch_dequant_nvfp4(elems, scales, global_scale, rows, cols, tc, out_bf16, d->num_sms, s)
+                        : mxk::launch_dequant_mx(elems, scales, rows, cols, fmt, tc, out_bf16, d->num_sms, s);
+    return e == cudaSuccess ? MX_OK : cuda_fail(e);
+}
+
+mx_status mx_cast(const void *src, int64_t n, mx_fmt fmt, void *out, mx_stream_t stream) {
+    if (fmt != MX_FMT_E4M3 && fmt != MX_FMT_E5M2 && fmt != MX_FMT_E2M1) return MX_ERR_ARG;
+    if (n < 0 || (fmt == MX_FMT_E2M1 && n % 2)) return MX_ERR_SHAPE;
+    if (n == 0) return MX_OK;
+    if (!src || !out) return MX_ERR_ARG;
+    if (!aligned(src, 16) || !aligned(out, 16)) return MX_ERR_ALIGN;
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    cudaError_t e = mxk::launch_cast(src, n, fmt, out, d->num_sms, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MX_OK : cuda_fail(e);
+}
+
+mx_status mx_gemm(mx_operand A, mx_operand B, void *C, int64_t M, int64_t N, int64_t K,
+                  mx_stream_t stream) {
+    if (A.fmt != MX_FMT_E4M3 || (B.fmt != MX_FMT_E4M3 && B.fmt != MX_FMT_E2M1)) return MX_ERR_ARG;
+    if (M < 0 || N < 0 || K < 0) return MX_ERR_SHAPE;
+    if (M % 128 || N % 128 || K % 128) return MX_ERR_SHAPE;
+    if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return MX_ERR_SHAPE;
+    if (M == 0 || N == 0) return MX_OK;
+    if (!A.elems || !A.scales || !B.elems || !B.scales || !C) return MX_ERR_ARG;
+    if (!aligned(A.elems, 32) || !aligned(B.elems, 32) || !aligned(A.scales, 16) || !aligned(B.scales, 16) ||
+        !aligned(C, 16))
+        return MX_ERR_ALIGN;
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (K == 0) {
+        e = cudaMemsetAsync(C, 0, (size_t)(M * N * 2), s);   // empty sum
+        return e == cudaSuccess ? MX_OK : cuda_fail(e);
+    }
+    e = mxk::launch_gemm(A.elems, A.scales, B.elems, B.scales, B.fmt, C, M, N, K, d->watchdog, d->num_sms, s);
+    return e == cudaSuccess ? MX_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,113 @@
+"""The C-ABI library loads, exports every function include/mx.h declares, and rejects
+invalid arguments on the host before any CUDA call (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+
+@pytest.fixture(scope="module")
+def L():
+    from microscaling_precision_number_b200 import build
+    build.build()
+    from microscaling_precision_number_b200 import _lib
+    return _lib
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "mx.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mx_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("mx_quantize", "mx_quantize_dual", "mx_dequantize", "mx_gemm", "mx_cast",
+                     "mx_status_string", "mx_last_cuda_error"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    raw = ctypes.CDLL(L.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), f"libmx.so does not export {name}"
+    assert set(L.EXPORTS) == set(declared_functions())
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert L.lib.mx_status_string(s).startswith(b"MX_")
+    assert b"unknown" in L.lib.mx_status_string(99)
+
+
+def test_scale_bytes(L):
+    assert L.lib.mx_scale_bytes(4096, 128, L.MX_LAYOUT_ROWMAJOR) == 4096 * 128
+    assert L.lib.mx_scale_bytes(4096, 128, L.MX_LAYOUT_TCGEN05) == 32 * 32 * 512
+    assert L.lib.mx_scale_bytes(130, 5, L.MX_LAYOUT_TCGEN05) == 2 * 2 * 512
+    assert L.lib.mx_scale_bytes(-1, 5, L.MX_LAYOUT_TCGEN05) == -1
+    assert L.lib.mx_scale_bytes(1, 1, 3) == -1
+
+
+FAKE = 0x10000   # a 16-byte-aligned non-null address; never dereferenced (rejected first)
+
+
+@pytest.mark.parametrize("args,status", [
+    # bad enum values
+    (dict(fmt=7), "MX_ERR_ARG"), (dict(axis=2), "MX_ERR_ARG"), (dict(rounding=5), "MX_ERR_ARG"),
+    # NVFP4 column-wise unsupported; NVFP4 needs global_scale, MX must not get one
+    (dict(fmt=3, axis=1, g=FAKE), "MX_ERR_ARG"), (dict(fmt=3), "MX_ERR_ARG"), (dict(g=FAKE), "MX_ERR_ARG"),
+    # layouts
+    (dict(layout=0), "MX_ERR_LAYOUT"), (dict(layout=4), "MX_ERR_LAYOUT"), (dict(layout=3), "MX_ERR_LAYOUT"),
+    (dict(layout=1, alt=FAKE), "MX_ERR_LAYOUT"),
+    # shapes
+    (dict(rows=-1), "MX_ERR_SHAPE"), (dict(cols=48), "MX_ERR_SHAPE"), (dict(axis=1, rows=40), "MX_ERR_SHAPE"),
+    (dict(fmt=3, cols=24, g=FAKE), "MX_ERR_SHAPE"),
+    # null / misaligned pointers
+    (dict(src=0), "MX_ERR_ARG"), (dict(out=0), "MX_ERR_ARG"), (dict(sc=0), "MX_ERR_ARG"),
+    (dict(src=FAKE + 8), "MX_ERR_ALIGN"), (dict(out=FAKE + 4), "MX_ERR_ALIGN"),
+    # empty input is valid and launches nothing
+    (dict(rows=0), "MX_OK"), (dict(cols=0), "MX_OK"),
+])
+def test_quantize_validation(L, args, status):
+    a = dict(src=FAKE, rows=64, cols=64, fmt=0, axis=0, rounding=1, out=FAKE, sc=FAKE, layout=1, alt=0, g=0)
+    a.update(args)
+    st = L.lib.mx_quantize(a["src"] or None, a["rows"], a["cols"], a["fmt"], a["axis"], a["rounding"],
+                           a["out"] or None, a["sc"] or None, a["layout"], a["alt"] or None, a["g"] or None, None)
+    assert st == getattr(L, status), L.lib.mx_status_string(st)
+
+
+def test_dual_dequant_cast_gemm_validation(L):
+    lib = L.lib
+    assert lib.mx_quantize_dual(FAKE, 64, 64, 3, 1, FAKE, FAKE, FAKE, FAKE, 1, None) == L.MX_ERR_ARG
+    assert lib.mx_quantize_dual(FAKE, 64, 64, 0, 1, FAKE, FAKE, FAKE, FAKE, 3, None) == L.MX_ERR_LAYOUT
+    assert lib.mx_quantize_dual(FAKE, 48, 64, 0, 1, FAKE, FAKE, FAKE, FAKE, 1, None) == L.MX_ERR_SHAPE
+    assert lib.mx_quantize_dual(FAKE, 64, 64, 0, 1, FAKE, FAKE, None, FAKE, 1, None) == L.MX_ERR_ARG
+    assert lib.mx_quantize_dual(FAKE, 0, 64, 0, 1, None, None, None, None, 1, None) == L.MX_OK
+    assert lib.mx_dequantize(FAKE, FAKE, None, 4, 48, 0, 1, FAKE, None) == L.MX_ERR_SHAPE
+    assert lib.mx_dequantize(FAKE, FAKE, None, 4, 64, 3, 1, FAKE, None) == L.MX_ERR_ARG
+    assert lib.mx_dequantize(FAKE, FAKE, None, 4, 64, 0, 3, FAKE, None) == L.MX_ERR_LAYOUT
+    assert lib.mx_dequantize(FAKE + 2, FAKE, None, 4, 64, 0, 1, FAKE, None) == L.MX_ERR_ALIGN
+    assert lib.mx_cast(FAKE, 7, 2, FAKE, None) == L.MX_ERR_SHAPE
+    assert lib.mx_cast(FAKE, 8, 3, FAKE, None) == L.MX_ERR_ARG
+    assert lib.mx_cast(None, 8, 0, FAKE, None) == L.MX_ERR_ARG
+    assert lib.mx_cast(FAKE, 0, 0, FAKE, None) == L.MX_OK
+    op = lambda fmt, p=FAKE: L.MxOperand(p, FAKE, fmt)
+    assert lib.mx_gemm(op(0), op(1), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG      # E5M2 B unsupported
+    assert lib.mx_gemm(op(2), op(0), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG      # FP4 A unsupported
+    assert lib.mx_gemm(op(0), op(2), FAKE, 100, 128, 128, None) == L.MX_ERR_SHAPE
+    assert lib.mx_gemm(op(0), op(0), FAKE, 128, 128, 96, None) == L.MX_ERR_SHAPE
+    assert lib.mx_gemm(op(0, FAKE + 16), op(0), FAKE, 128, 128, 128, None) == L.MX_ERR_ALIGN
+    assert lib.mx_gemm(op(0), op(0), None, 128, 128, 128, None) == L.MX_ERR_ARG
+    assert lib.mx_gemm(op(0), op(0), FAKE, 0, 128, 128, None) == L.MX_OK
+
+
+def test_product_package_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "microscaling_precision_number_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in text and "from oracle" not in text and "mx_oracle" not in text, f

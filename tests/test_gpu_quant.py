@@ -1,0 +1,259 @@
+"""GPU parity of the quantisers, dequantisers and the direct cast against the CPU oracle,
+through the C ABI.  Element codes and scales must match bit for bit; dequantised values
+bit for bit (NaN matched as NaN)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import microscaling_precision_number_b200 as mx
+    from microscaling_precision_number_b200 import _lib as L
+
+FMT_NAMES = {0: "e4m3", 1: "e5m2", 2: "e2m1"}
+
+
+def to_dev(bits: np.ndarray) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t.cuda()
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy()
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def nan_aware_equal(a_bits: np.ndarray, b_bits: np.ndarray) -> bool:
+    a_nan = ((a_bits & 0x7F80) == 0x7F80) & ((a_bits & 0x7F) != 0)
+    b_nan = ((b_bits & 0x7F80) == 0x7F80) & ((b_bits & 0x7F) != 0)
+    return bool(np.array_equal(a_nan, b_nan) and np.array_equal(a_bits[~a_nan], b_bits[~b_nan]))
+
+
+def with_specials(x: np.ndarray, seed: int) -> np.ndarray:
+    """Sprinkle edge values (zeros, subnormals, huge, Inf, NaN) and an all-zero block."""
+    x = x.copy()
+    rng = np.random.default_rng(seed)
+    sp = synth.special_values_block()
+    idx = rng.choice(x.size, size=min(x.size // 7, 64), replace=False)
+    x.reshape(-1)[idx] = sp[rng.integers(0, sp.size, size=idx.size)]
+    if x.shape[1] >= 32:
+        x[0, :32] = 0
+        x[0, 5] = 0x8000      # -0 in an otherwise zero block
+    return x
+
+
+SHAPES = [(1, 32), (3, 64), (37, 96), (130, 160), (257, 1024)]
+
+
+@pytest.fixture(autouse=True)
+def _no_watchdog():
+    yield
+    assert mx.watchdog_status(clear=True) == 0
+
+
+# ------------------------------------------------------------------ direct cast
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+def test_cast_exhaustive_bf16(oracle, fmt):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = host(mx.cast(to_dev(bits), FMT_NAMES[fmt]))
+    ref = oracle.cast(bits, fmt)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, f"{bad.size} mismatching bytes, first at {bad[:8]}"
+
+
+@pytest.mark.parametrize("n", [2, 10, 30, 1000, 4097 * 8 + 6])
+def test_cast_tail(oracle, n):
+    rng = np.random.default_rng(n)
+    bits = rng.integers(0, 65536, size=n, dtype=np.uint32).astype(np.uint16)
+    for fmt in (0, 2):
+        assert np.array_equal(host(mx.cast(to_dev(bits), FMT_NAMES[fmt])), oracle.cast(bits, fmt))
+
+
+# ------------------------------------------------------------------ row-wise MX
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (0, "floor"), (1, "ceil"), (1, "floor"), (2, "floor"), (2, "ceil")])
+def test_quantize_rowwise_matches_oracle(oracle, shape, fmt, rounding):
+    x = with_specials(synth.mx8_rowwise(*shape, seed=shape[0]), seed=shape[1])
+    q = mx.quantize(to_dev(x), FMT_NAMES[fmt], "row", rounding, layout="both")
+    e_ref, s_ref = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.CEIL if rounding == "ceil" else oracle.FLOOR)
+    assert np.array_equal(host(q.elems), e_ref.reshape(-1))
+    assert np.array_equal(host(q.scales), s_ref.reshape(-1))
+    assert np.array_equal(host(q.scales_alt), oracle.to_tcgen05_layout(s_ref))
+
+
+@pytest.mark.parametrize("layout", ["rowmajor", "tcgen05"])
+def test_quantize_single_layout(oracle, layout):
+    x = synth.weight_fp4(130, 96, seed=3)
+    q = mx.quantize(to_dev(x), "e2m1", "row", "floor", layout=layout)
+    _, s_ref = oracle.quantize_mx(x, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    want = s_ref.reshape(-1) if layout == "rowmajor" else oracle.to_tcgen05_layout(s_ref)
+    assert np.array_equal(host(q.scales), want)
+
+
+def test_tcgen05_padding_is_zeroed(oracle):
+    x = synth.normal(5, 64, seed=2)
+    dev = to_dev(x)
+    rows, cols = x.shape
+    sc = torch.full((mx.scale_bytes(rows, cols // 32, "tcgen05"),), 0xAB, dtype=torch.uint8, device="cuda")
+    el = torch.empty(rows * cols, dtype=torch.uint8, device="cuda")
+    st = L.lib.mx_quantize(dev.data_ptr(), rows, cols, 0, 0, 1, el.data_ptr(), sc.data_ptr(), 2, None, None,
+                           torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    _, s_ref = oracle.quantize_mx(x, 0, 0, 1)
+    assert np.array_equal(host(sc), oracle.to_tcgen05_layout(s_ref))
+
+
+# ------------------------------------------------------------------ column-wise and dual
+@pytest.mark.parametrize("shape", [(32, 32), (64, 96), (96, 200), (160, 384)])
+@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (1, "ceil"), (2, "floor")])
+def test_quantize_colwise_matches_oracle(oracle, shape, fmt, rounding):
+    x = with_specials(synth.activations(*shape, seed=shape[1]), seed=shape[0])
+    rnd = oracle.CEIL if rounding == "ceil" else oracle.FLOOR
+    q = mx.quantize(to_dev(x), FMT_NAMES[fmt], "col", rounding, layout="both")
+    e_ref, s_ref = oracle.quantize_mx(x, fmt, oracle.COL, rnd)
+    assert np.array_equal(host(q.elems), e_ref.reshape(-1))
+    assert np.array_equal(host(q.scales), s_ref.reshape(-1))
+    assert np.array_equal(host(q.scales_alt), oracle.to_tcgen05_layout(s_ref))
+
+
+@pytest.mark.parametrize("shape", [(32, 32), (64, 160), (160, 384), (256, 1024)])
+@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (1, "ceil"), (1, "floor"), (2, "floor")])
+@pytest.mark.parametrize("layout", ["rowmajor", "tcgen05"])
+def test_quantize_dual_matches_oracle(oracle, shape, fmt, rounding, layout):
+    x = with_specials(synth.gradients(*shape, seed=shape[0] + fmt), seed=shape[1])
+    rnd = oracle.CEIL if rounding == "ceil" else oracle.FLOOR
+    qr, qc = mx.quantize_dual(to_dev(x), FMT_NAMES[fmt], rounding, layout)
+    er, sr = oracle.quantize_mx(x, fmt, oracle.ROW, rnd)
+    ec, sc = oracle.quantize_mx(x, fmt, oracle.COL, rnd)
+    tr = (lambda s: s.reshape(-1)) if layout == "rowmajor" else oracle.to_tcgen05_layout
+    assert np.array_equal(host(qr.elems), er.reshape(-1))
+    assert np.array_equal(host(qr.scales), tr(sr))
+    assert np.array_equal(host(qc.elems), ec.reshape(-1))
+    assert np.array_equal(host(qc.scales), tr(sc))
+
+
+# ------------------------------------------------------------------ NVFP4
+@pytest.mark.parametrize("shape", [(1, 16), (5, 48), (130, 256), (64, 4096)])
+@pytest.mark.parametrize("specials", [False, True])
+def test_nvfp4_matches_oracle(oracle, shape, specials):
+    x = synth.weight_fp4(*shape, seed=shape[0])
+    if specials:
+        x = with_specials(x, seed=7)
+    q = mx.quantize(to_dev(x), "nvfp4", "row", "ceil", layout="both")
+    e_ref, s_ref, g_ref = oracle.quantize_nvfp4(x)
+    assert host(q.global_scale)[0] == np.float32(g_ref)
+    assert np.array_equal(host(q.elems), e_ref.reshape(-1))
+    assert np.array_equal(host(q.scales), s_ref.reshape(-1))
+    assert np.array_equal(host(q.scales_alt), oracle.to_tcgen05_layout(s_ref))
+    d = bf16_bits(mx.dequantize(q, "tcgen05"))
+    assert nan_aware_equal(d.reshape(-1), oracle.dequantize_nvfp4(e_ref, s_ref, g_ref, *shape).reshape(-1))
+
+
+def test_nvfp4_degenerate_tensors(oracle):
+    for x in (np.zeros((4, 32), dtype=np.uint16),                          # all zero: g = 1
+              np.full((2, 16), 0x0001, dtype=np.uint16),                   # smallest subnormals
+              np.full((2, 32), 0x7FC0, dtype=np.uint16)):                  # all NaN
+        q = mx.quantize(to_dev(x), "nvfp4", "row", "ceil", layout="rowmajor")
+        e_ref, s_ref, g_ref = oracle.quantize_nvfp4(x)
+        assert host(q.global_scale)[0] == np.float32(g_ref)
+        assert np.array_equal(host(q.elems), e_ref.reshape(-1))
+        assert np.array_equal(host(q.scales), s_ref.reshape(-1))
+
+
+# ------------------------------------------------------------------ dequantisation
+@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("layout", ["rowmajor", "tcgen05"])
+def test_dequantize_matches_oracle(oracle, fmt, layout):
+    x = with_specials(synth.mx8_rowwise(67, 256, seed=fmt), seed=3)
+    q = mx.quantize(to_dev(x), FMT_NAMES[fmt], "row", "ceil", layout="both")
+    e_ref, s_ref = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.CEIL)
+    d = bf16_bits(mx.dequantize(q, layout))
+    assert nan_aware_equal(d.reshape(-1), oracle.dequantize_mx(e_ref, s_ref, 67, 256, fmt).reshape(-1))
+
+
+def test_dequantize_all_scale_codes(oracle):
+    """Every E8M0 code (incl. 2^-127 and NaN) against every element code."""
+    for fmt in (0, 1, 2):
+        ncode = 16 if fmt == 2 else 256
+        codes = np.tile(np.arange(ncode, dtype=np.uint8), 256 * 32 // ncode)[: 256 * 32].reshape(256, 32)
+        scales = np.arange(256, dtype=np.uint8).reshape(256, 1)
+        if fmt == 2:
+            elems = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+        else:
+            elems = codes
+        q = mx.Quantized(torch.from_numpy(np.ascontiguousarray(elems).reshape(-1)).cuda(),
+                         torch.from_numpy(scales.reshape(-1).copy()).cuda(), None, None, 256, 32, fmt)
+        d = bf16_bits(mx.dequantize(q, "rowmajor"))
+        assert nan_aware_equal(d.reshape(-1), oracle.dequantize_mx(elems, scales, 256, 32, fmt).reshape(-1))
+
+
+# ------------------------------------------------------------------ full-size workloads
+def test_config1_mx8_rowwise_full(oracle):
+    x = synth.mx8_rowwise()
+    q = mx.quantize(to_dev(x), "e4m3", "row", "ceil", layout="rowmajor")
+    e_ref, s_ref = oracle.quantize_mx(x, oracle.E4M3, oracle.ROW, oracle.CEIL)
+    assert np.array_equal(host(q.elems), e_ref.reshape(-1))
+    assert np.array_equal(host(q.scales), s_ref.reshape(-1))
+    d = bf16_bits(mx.dequantize(q, "rowmajor"))
+    assert np.array_equal(d.reshape(-1), oracle.dequantize_mx(e_ref, s_ref, 1024, 1024, oracle.E4M3).reshape(-1))
+
+
+def test_config2_weight_full(oracle):
+    x = synth.weight_fp4()
+    dev = to_dev(x)
+    q4 = mx.quantize(dev, "e2m1", "row", "floor", layout="both")
+    e_ref, s_ref = oracle.quantize_mx(x, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    assert np.array_equal(host(q4.elems), e_ref.reshape(-1))
+    assert np.array_equal(host(q4.scales), s_ref.reshape(-1))
+    assert np.array_equal(host(q4.scales_alt), oracle.to_tcgen05_layout(s_ref))
+    qn = mx.quantize(dev, "nvfp4", "row", "ceil", layout="both")
+    e_ref, s_ref, g_ref = oracle.quantize_nvfp4(x)
+    assert host(qn.global_scale)[0] == np.float32(g_ref)
+    assert np.array_equal(host(qn.elems), e_ref.reshape(-1))
+    assert np.array_equal(host(qn.scales), s_ref.reshape(-1))
+    assert np.array_equal(host(qn.scales_alt), oracle.to_tcgen05_layout(s_ref))
+
+
+@pytest.mark.parametrize("which", ["activations", "gradients"])
+def test_config3_dual_full_sampled(oracle, which):
+    """Full-size dual quantisation in the benchmark's launch configuration; sampled
+    32 x 128 tiles checked against the oracle (blocks are independent)."""
+    if which == "activations":
+        x, fmt = synth.activations(), oracle.E4M3
+    else:
+        x, fmt = synth.gradients(), oracle.E5M2
+    R, C = x.shape
+    qr, qc = mx.quantize_dual(to_dev(x), FMT_NAMES[fmt], "ceil", "tcgen05")
+    re_, rs = host(qr.elems).reshape(R, C), host(qr.scales)
+    ce, cs = host(qc.elems).reshape(C, R), host(qc.scales)
+    rng = np.random.default_rng(0)
+    for _ in range(24):
+        r0 = int(rng.integers(0, R // 32)) * 32
+        c0 = int(rng.integers(0, C // 128)) * 128
+        tile = np.ascontiguousarray(x[r0:r0 + 32, c0:c0 + 128])
+        er, sr = oracle.quantize_mx(tile, fmt, oracle.ROW, oracle.CEIL)
+        ec, sc = oracle.quantize_mx(tile, fmt, oracle.COL, oracle.CEIL)
+        assert np.array_equal(re_[r0:r0 + 32, c0:c0 + 128], er)
+        assert np.array_equal(ce[c0:c0 + 128, r0:r0 + 32], ec)
+        for i in range(32):
+            for b in range(4):
+                off = oracle.lib().mxo_tcgen05_scale_offset(r0 + i, c0 // 32 + b, R, C // 32)
+                assert rs[off] == sr[i, b]
+        for j in range(128):
+            off = oracle.lib().mxo_tcgen05_scale_offset(c0 + j, r0 // 32, C, R // 32)
+            assert cs[off] == sc[j, 0]
+    del qr, qc
+    torch.cuda.empty_cache()
+
+
+def test_empty_inputs_launch_nothing():
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    q = mx.quantize(x, "e4m3", "row", "ceil")
+    assert q.elems.numel() == 0
+    assert mx.cast(torch.empty(0, dtype=torch.bfloat16, device="cuda"), "e2m1").numel() == 0
