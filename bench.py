@@ -112,11 +112,16 @@ class ClockSampler:
 
 
 class L2Flush:
+    """Write a 256 MiB buffer (evicts everything), then read a second 256 MiB buffer so
+    L2 is left holding clean lines: the next kernel pays no write-back of the flush."""
+
     def __init__(self, dev):
-        self.buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        self.wbuf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        self.rbuf = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
 
     def __call__(self):
-        self.buf.fill_(1)
+        self.wbuf.fill_(1)
+        self.sink = self.rbuf.sum()
 
 
 def to_dev(bits, dev):
@@ -276,7 +281,7 @@ def run_ours(args, rank, world, dev):
                 "config": {"workload": "weight_4096x4096_mxfp4_floor_and_nvfp4_both_scale_layouts",
                            "shape": [R2, C2], "formats": ["MXFP4 E2M1/E8M0 floor block 32",
                                                           "NVFP4 E2M1/UE4M3+fp32 block 16"],
-                           "step_bytes": STEP_BYTES, "l2": "flushed between steps (256 MiB write)",
+                           "step_bytes": STEP_BYTES, "l2": "flushed between steps (256 MiB write, then 256 MiB read of another buffer)",
                            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": step.launches_per_step * args.steps, "clocks": clk.summary()}

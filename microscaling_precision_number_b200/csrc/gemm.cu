@@ -178,7 +178,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     }
                 }
                 if (*fail_sh) break;
-                mbar_arrive_expect_tx(&full_bar[s], kABytes + kBBytes + kSfaBytes + kSfbBytes);
+                // An E2M1 tile lands in shared memory padded to one byte per element
+                // (16U4_ALIGN16B), but the copy completes only the packed global bytes.
+                mbar_arrive_expect_tx(&full_bar[s], kABytes + (b_fmt_code == 5u ? kBBytes / 2 : kBBytes) +
+                                                        kSfaBytes + kSfbBytes);
                 tma_load_2d(sA + s * kABytes, &tmA, kb * kBK, m_blk * kBM, &full_bar[s]);
                 tma_load_2d(sB + s * kBBytes, &tmB, kb * kBK, n_blk * BN, &full_bar[s]);
                 bulk_load(sSFA + s * kSfaBytes, a_sc + ((int64_t)m_blk * kb128 + kb) * 512, kSfaBytes, &full_bar[s]);

@@ -1,6 +1,11 @@
 """GPU parity of the tcgen05 block-scaled matmul against the oracle's fp64 reference over
-its own dequantised operands: |C_gpu - C_ref| <= 1e-3 * sum_k |a_mk b_nk| for every
-checked entry (the fp32-accumulation tolerance the MX matmul is specified to)."""
+its own dequantised operands.
+
+Tolerance: the fp32 accumulation may differ from the fp64 sum by 1e-3 * sum_k |a_mk b_nk|
+(the bound the MX matmul is specified to), and the bf16 output then rounds that fp32
+value once more, by at most half a bf16 ulp.  So every checked entry must satisfy
+    |C_gpu - C_ref| <= 1e-3 * sum_k |a b| + half_ulp_bf16(|C_ref| + 1e-3 * sum_k |a b|).
+"""
 import numpy as np
 import pytest
 import torch
@@ -21,6 +26,17 @@ def to_dev(bits):
 
 def bf16_to_f64(t):
     return t.float().cpu().numpy().astype(np.float64)
+
+
+def half_ulp_bf16(x):
+    """Half the spacing of bf16 numbers at magnitude x (8 significant bits)."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -133)))
+    return 2.0 ** (np.maximum(e, -126) - 8)
+
+
+def gemm_tolerance(ref, mag):
+    acc = TOL * mag
+    return acc + half_ulp_bf16(np.abs(ref) + acc)
 
 
 @pytest.fixture(autouse=True)
@@ -50,10 +66,14 @@ def run_case(oracle, a_bits, b_bits, b_fmt, pairs=None):
     ref, mag = oracle.gemm_ref(ae, as_, oracle.E4M3, be, bs, b_fmt, len(rows_a), len(rows_b), K, local)
     got = c[pairs[:, 0], pairs[:, 1]]
     err = np.abs(got - ref)
-    bound = TOL * mag
+    bound = gemm_tolerance(ref, mag)
     bad = np.nonzero(~(err <= bound))[0]
     assert bad.size == 0, (f"{bad.size}/{len(pairs)} entries out of tolerance; first "
                            f"{[(tuple(pairs[i]), got[i], ref[i], mag[i]) for i in bad[:4]]}")
+    # fp32 accumulation error is far below a bf16 ulp here: nearly every entry is the
+    # correctly rounded bf16 of the fp64 reference
+    rounded = torch.from_numpy(ref).to(torch.float32).to(torch.bfloat16).double().numpy()
+    assert np.mean(got == rounded) >= 0.95, f"only {np.mean(got == rounded):.3f} of entries round-exact"
     return err, mag
 
 
