@@ -62,7 +62,21 @@ def _load():
     return lib
 
 
-lib = _load()
+class _LazyLib:
+    """Loads libmx.so on first use (so that importing the package never needs the
+    library, e.g. to build it); raises ImportError then if it is missing."""
+    _handle = None
+
+    def load(self):
+        if _LazyLib._handle is None:
+            _LazyLib._handle = _load()
+        return _LazyLib._handle
+
+    def __getattr__(self, name):
+        return getattr(self.load(), name)
+
+
+lib = _LazyLib()
 
 
 def check(status: int, where: str) -> None:
