@@ -57,6 +57,8 @@ bool single_layout(int l) { return l == MX_LAYOUT_ROWMAJOR || l == MX_LAYOUT_TCG
 }  // namespace
 
 namespace mxk {
+void record_cuda_error(cudaError_t e) { g_last_cuda_error = (int)e; }
+
 void *tensor_map_encoder() {
     static void *fn = nullptr;
     static std::once_flag once;

@@ -45,4 +45,7 @@ cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, const void *b_
 // Driver entry point for cuTensorMapEncodeTiled (resolved once, no libcuda link).
 void *tensor_map_encoder();
 
+// Record the CUDA error behind an MX_ERR_CUDA status for mx_last_cuda_error().
+void record_cuda_error(cudaError_t e);
+
 }  // namespace mxk

@@ -1,0 +1,77 @@
+"""The NVFP4 entry point that allocates nothing (mx_quantize_nvfp4_noalloc).
+
+It exists for callers that cannot let the library call cudaMalloc: serving loops that
+reserve all device memory up front and must not take an allocation's implicit device
+synchronisation or out-of-memory risk on the request path, and host frameworks that own
+all device memory through their own allocator.  Its scratch lives in a static device
+array instead of the buffer mx_quantize allocates on first use.
+
+The test calls both entry points through the C ABI on the same inputs, twice in a row
+with different tensors (the second call must not see anything the first left in the
+shared static array), and requires identical codes, scales and tensor scale.  This file
+is named so that pytest collects it last; it also passes when run on its own.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _outputs(rows, cols):
+    from microscaling_precision_number_b200 import _lib as L
+    nbytes_tc = L.lib.mx_scale_bytes(rows, cols // 16, L.MX_LAYOUT_TCGEN05)
+    return dict(elems=torch.empty(rows * cols // 2, dtype=torch.uint8, device="cuda"),
+                scales=torch.empty(rows * cols // 16, dtype=torch.uint8, device="cuda"),
+                scales_tc=torch.full((nbytes_tc,), 0xAB, dtype=torch.uint8, device="cuda"),
+                g=torch.empty(1, dtype=torch.float32, device="cuda"))
+
+
+def _run(fn_name, x, out):
+    from microscaling_precision_number_b200 import _lib as L
+    rows, cols = x.shape
+    stream = torch.cuda.current_stream().cuda_stream
+    both = L.MX_LAYOUT_ROWMAJOR | L.MX_LAYOUT_TCGEN05
+    if fn_name == "noalloc":
+        st = L.lib.mx_quantize_nvfp4_noalloc(x.data_ptr(), rows, cols, out["elems"].data_ptr(),
+                                             out["scales"].data_ptr(), both, out["scales_tc"].data_ptr(),
+                                             out["g"].data_ptr(), stream)
+    else:
+        st = L.lib.mx_quantize(x.data_ptr(), rows, cols, L.MX_FMT_NVFP4, L.MX_AXIS_ROW, L.MX_SCALE_CEIL_RECIPE,
+                               out["elems"].data_ptr(), out["scales"].data_ptr(), both,
+                               out["scales_tc"].data_ptr(), out["g"].data_ptr(), stream)
+    assert st == L.MX_OK, L.lib.mx_status_string(st)
+
+
+def test_noalloc_nvfp4_matches_allocating_entry_point_twice():
+    # first a large-amax weight (many CTAs in the maximum pass), then a smaller tensor
+    # with a much smaller maximum: stale partial maxima from the first call would
+    # change the second call's tensor scale.
+    inputs = [synth.weight_fp4(1024, 4096, seed=21) , synth.normal(96, 160, sigma=1e-3, seed=22)]
+    for bits in inputs:
+        x = _dev_bf16(bits)
+        ref, got = _outputs(*x.shape), _outputs(*x.shape)
+        _run("allocating", x, ref)
+        _run("noalloc", x, got)
+        torch.cuda.synchronize()
+        for k in ("elems", "scales", "scales_tc", "g"):
+            assert torch.equal(got[k], ref[k]), k
+    # sanity: the second tensor's scale is far below the first's
+    assert float(got["g"]) < 1e-4
+
+
+def test_noalloc_nvfp4_validation():
+    from microscaling_precision_number_b200 import _lib as L
+    fake = 0x10000
+    lib = L.lib
+    assert lib.mx_quantize_nvfp4_noalloc(fake, 4, 24, fake, fake, 1, None, fake, None) == L.MX_ERR_SHAPE
+    assert lib.mx_quantize_nvfp4_noalloc(fake, 4, 32, fake, fake, 1, None, None, None) == L.MX_ERR_ARG
+    assert lib.mx_quantize_nvfp4_noalloc(fake, 4, 32, fake, fake, 3, None, fake, None) == L.MX_ERR_LAYOUT
+    assert lib.mx_quantize_nvfp4_noalloc(fake + 8, 4, 32, fake, fake, 1, None, fake, None) == L.MX_ERR_ALIGN
+    assert lib.mx_quantize_nvfp4_noalloc(None, 0, 32, None, None, 1, None, None, None) == L.MX_OK
