@@ -7,8 +7,9 @@ One step = one pass of the weight-quantisation workload over a 4096 x 4096 bf16 
 (N(0, 0.02) with 0.1% N(0, 1) outliers): MXFP4 (E2M1, block 32, E8M0, floor scale) and
 NVFP4 (E2M1, block 16, UE4M3 + fp32 tensor scale), each emitting both the row-major and
 the tcgen05 scale layouts.  value = algorithmic bytes of the step / step time (GB/s).
-The input (32 MiB) is smaller than L2, so L2 is flushed (a 256 MiB write) between timed
-steps, outside the per-step CUDA-event pairs.  Every other row of the hot path (row-wise
+The input (32 MiB) is smaller than L2, so consecutive steps rotate over 8 copies of the
+weight (256 MiB): each step reads its input from HBM.  K steps are timed back to back in
+one CUDA-event pair.  Every other row of the hot path (row-wise
 MXFP8 quantise + dequantise, dual-orientation quantisation, dequantisation, the two
 block-scaled matmuls) is measured in "breakdown", each against its own roofline.
 
@@ -43,6 +44,7 @@ R2 = C2 = 4096
 BYTES_MXFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 32)            # 42,991,616
 BYTES_NVFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 16) + 4         # 44,040,196
 STEP_BYTES = BYTES_MXFP4 + BYTES_NVFP4
+NROT = 8                 # rotating copies of the weight (8 x 32 MiB > 2 x L2)
 
 
 def peaks():
@@ -111,19 +113,6 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-class L2Flush:
-    """Write a 256 MiB buffer (evicts everything), then read a second 256 MiB buffer so
-    L2 is left holding clean lines: the next kernel pays no write-back of the flush."""
-
-    def __init__(self, dev):
-        self.wbuf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-        self.rbuf = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=dev)
-
-    def __call__(self):
-        self.wbuf.fill_(1)
-        self.sink = self.rbuf.sum()
-
-
 def to_dev(bits, dev):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
 
@@ -176,37 +165,40 @@ def run_ours(args, rank, world, dev):
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
     x_bits = synth.weight_fp4(seed=rank)
-    x = to_dev(x_bits, dev)
-    step = WeightQuantStep(mx, x)
-    flush = L2Flush(dev)
+    x0 = to_dev(x_bits, dev)
+    # NROT copies of the weight (8 x 32 MiB, over twice L2): step k works on copy k % NROT,
+    # so every timed step reads its input from HBM without an L2 flush in between.
+    steps = [WeightQuantStep(mx, x0.clone()) for _ in range(NROT)]
 
-    for _ in range(args.warmup):
-        step.mxfp4(sptr)
-        step.nvfp4(sptr)
+    def run_steps(n, which="both"):
+        for k in range(n):
+            s = steps[k % NROT]
+            if which in ("both", "mxfp4"):
+                s.mxfp4(sptr)
+            if which in ("both", "nvfp4"):
+                s.nvfp4(sptr)
+
+    run_steps(max(args.warmup, NROT))
     torch.cuda.synchronize()
 
-    # timed region: K steps, per-call events, L2 flushed between steps (outside the events)
-    ev = [[event_pair(), event_pair()] for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clk:
-        for k in range(args.steps):
-            flush()
-            (a0, a1), (b0, b1) = ev[k]
-            a0.record(stream)
-            step.mxfp4(sptr)
-            a1.record(stream)
-            b0.record(stream)
-            step.nvfp4(sptr)
-            b1.record(stream)
+        # soak: keep the GPU busy with the same steps for ~0.4 s so that the clock samples
+        # below see it under load, then the timed region proper
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < 0.4:
+            run_steps(200)
+            torch.cuda.synchronize()
+        e0, e1 = event_pair()
+        if world > 1:
+            torch.distributed.barrier()
         torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    t_mx = [e[0][0].elapsed_time(e[0][1]) for e in ev]
-    t_nv = [e[1][0].elapsed_time(e[1][1]) for e in ev]
-    step_ms = [a + b for a, b in zip(t_mx, t_nv)]
-    total_ms = sum(step_ms)
+        e0.record(stream)
+        run_steps(args.steps)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+    total_ms = e0.elapsed_time(e1)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -214,25 +206,38 @@ def run_ours(args, rank, world, dev):
     ms_per_step = total_ms / args.steps
     value = STEP_BYTES * world * args.steps / (total_ms * 1e-3) / 1e9
 
-    # dominant call and its roofline
-    mean_mx, mean_nv = statistics.mean(t_mx), statistics.mean(t_nv)
+    # per-call durations for the roofline: many launches of one call per event pair
+    ncall = max(args.steps, 50)
+    per = {}
+    for which in ("mxfp4", "nvfp4"):
+        run_steps(NROT, which)
+        a, b = event_pair()
+        a.record(stream)
+        run_steps(ncall, which)
+        b.record(stream)
+        torch.cuda.synchronize()
+        per[which] = a.elapsed_time(b) / ncall
+    mean_mx, mean_nv = per["mxfp4"], per["nvfp4"]
     if mean_nv >= mean_mx:
-        dom = {"kernel": "mx_quantize(NVFP4): nvfp4_amax_kernel + nvfp4_quant_kernel", "ms": mean_nv,
+        dom = {"kernel": "mx_quantize(NVFP4): nvfp4_amax_bulk_kernel + nvfp4_quant_bulk_kernel", "ms": mean_nv,
                "bytes": BYTES_NVFP4}
     else:
-        dom = {"kernel": "mx_quantize(MXFP4): quant_rows_mx_kernel<E2M1,floor,both layouts>", "ms": mean_mx,
+        dom = {"kernel": "mx_quantize(MXFP4): mx_rows_kernel<E2M1,floor,both layouts>", "ms": mean_mx,
                "bytes": BYTES_MXFP4}
     achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
-                "peak_source": pk["source"] + " copy bandwidth (MEASURED_PEAKS hbm_gbs)",
+                "peak_source": pk["source"] + " copy bandwidth (MEASURED_PEAKS hbm_gbs), burst",
                 "kernel": dom["kernel"], "algorithmic_bytes_per_launch": dom["bytes"],
                 "ms_per_launch": round(dom["ms"], 5),
                 "calls": {"mxfp4_ms": round(mean_mx, 5), "mxfp4_GBps": round(BYTES_MXFP4 / mean_mx / 1e6, 1),
-                          "nvfp4_ms": round(mean_nv, 5), "nvfp4_GBps": round(BYTES_NVFP4 / mean_nv / 1e6, 1)},
+                          "nvfp4_ms": round(mean_nv, 5), "nvfp4_GBps": round(BYTES_NVFP4 / mean_nv / 1e6, 1),
+                          "launches_timed": ncall},
                 "frac_of_nominal_8TBps": round(achieved / HBM_NOMINAL_GBS, 4)}
 
     # end to end through the public API with host buffers (pinned), copies inside the timing
+    step = steps[0]
+    x = step.x
     x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
     outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in step.outputs()]
     h2d = x_host.numel() * 2
@@ -267,7 +272,7 @@ def run_ours(args, rank, world, dev):
 
     breakdown = None
     if not args.no_breakdown and rank == 0:
-        breakdown = run_breakdown(mx, dev, pk, flush)
+        breakdown = run_breakdown(mx, dev, pk)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -281,57 +286,59 @@ def run_ours(args, rank, world, dev):
                 "config": {"workload": "weight_4096x4096_mxfp4_floor_and_nvfp4_both_scale_layouts",
                            "shape": [R2, C2], "formats": ["MXFP4 E2M1/E8M0 floor block 32",
                                                           "NVFP4 E2M1/UE4M3+fp32 block 16"],
-                           "step_bytes": STEP_BYTES, "l2": "flushed between steps (256 MiB write, then 256 MiB read of another buffer)",
+                           "step_bytes": STEP_BYTES,
+                           "l2": f"inputs larger than L2: steps rotate over {NROT} copies of the weight "
+                                 f"({NROT * R2 * C2 * 2 >> 20} MiB)",
                            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": step.launches_per_step * args.steps, "clocks": clk.summary()}
+                "gpu_launches": steps[0].launches_per_step * args.steps, "clocks": clk.summary()}
         if breakdown is not None:
             line["breakdown"] = breakdown
         print(json.dumps(line), flush=True)
 
 
 # ----------------------------------------------------------------------------- breakdown
-def timed(fn, iters, flush, stream):
-    ts = []
-    for _ in range(iters):
-        if flush is not None:
-            flush()
-        a, b = event_pair()
-        a.record(stream)
-        fn()
-        b.record(stream)
-        torch.cuda.synchronize()
-        ts.append(a.elapsed_time(b))
-    return statistics.median(ts)
+def timed(fns, iters, stream):
+    """Mean device time of one call, over `iters` calls cycling through `fns` (one closure
+    per rotating buffer set), in a single event pair."""
+    for f in fns:
+        f()
+    torch.cuda.synchronize()
+    a, b = event_pair()
+    a.record(stream)
+    for i in range(iters):
+        fns[i % len(fns)]()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
 
 
-def run_breakdown(mx, dev, pk, flush):
+def run_breakdown(mx, dev, pk):
     stream = torch.cuda.current_stream()
     out = {}
     hbm = pk["hbm_gbs"]
     mx_peak = 2.0 * pk["bf16_tflops"]          # FP8 / mxf8f6f4 rate = 2 x the bf16 rate
 
-    # C1: MXFP8 E4M3 row-wise quantise + dequantise, 1024 x 1024 (launch-latency bound)
+    # C1: MXFP8 E4M3 row-wise quantise + dequantise, 1024 x 1024, 64 rotating copies (> L2)
     x1 = to_dev(synth.mx8_rowwise(), dev)
-    q1 = mx.quantize(x1, "e4m3", "row", "ceil", layout="rowmajor")
-    for _ in range(5):
-        mx.quantize(x1, "e4m3", "row", "ceil", layout="rowmajor")
-    tq = timed(lambda: mx.quantize(x1, "e4m3", "row", "ceil", layout="rowmajor"), 30, flush, stream)
-    td = timed(lambda: mx.dequantize(q1, "rowmajor"), 30, flush, stream)
+    xs = [x1.clone() for _ in range(64)]
+    qs = [mx.quantize(x, "e4m3", "row", "ceil", layout="rowmajor") for x in xs]
+    tq = timed([lambda x=x: mx.quantize(x, "e4m3", "row", "ceil", layout="rowmajor") for x in xs], 256, stream)
+    td = timed([lambda q=q: mx.dequantize(q, "rowmajor") for q in qs], 256, stream)
     b1 = 1024 * 1024 * 2 + 1024 * 1024 + 1024 * 32
     out["c1_mxfp8_rowwise_1024"] = {"quantize_us": round(tq * 1e3, 2), "dequantize_us": round(td * 1e3, 2),
                                     "quantize_GBps": round(b1 / tq / 1e6, 1),
                                     "dequantize_GBps": round(b1 / td / 1e6, 1),
                                     "frac_hbm": round(b1 / tq / 1e6 / hbm, 4),
-                                    "note": "3.2 MB per call: launch-latency bound"}
-    del x1, q1
+                                    "note": "3.2 MB per call, back-to-back calls: launch-latency bound"}
+    del x1, xs, qs
 
-    # a7: dequantise the config-2 weight (MXFP4 and NVFP4), tcgen05 scales
+    # a7: dequantise the config-2 weight (MXFP4 and NVFP4), tcgen05 scales, 8 rotating copies
     xw = to_dev(synth.weight_fp4(), dev)
-    q4 = mx.quantize(xw, "e2m1", "row", "floor", layout="tcgen05")
-    qn = mx.quantize(xw, "nvfp4", "row", "ceil", layout="tcgen05")
-    t4 = timed(lambda: mx.dequantize(q4, "tcgen05"), 20, flush, stream)
-    tn = timed(lambda: mx.dequantize(qn, "tcgen05"), 20, flush, stream)
+    q4 = [mx.quantize(xw, "e2m1", "row", "floor", layout="tcgen05") for _ in range(NROT)]
+    qn = [mx.quantize(xw, "nvfp4", "row", "ceil", layout="tcgen05") for _ in range(NROT)]
+    t4 = timed([lambda q=q: mx.dequantize(q, "tcgen05") for q in q4], 64, stream)
+    tn = timed([lambda q=q: mx.dequantize(q, "tcgen05") for q in qn], 64, stream)
     bd4 = R2 * C2 // 2 + R2 * C2 // 32 + R2 * C2 * 2
     bdn = R2 * C2 // 2 + R2 * C2 // 16 + 4 + R2 * C2 * 2
     out["a7_dequantize_4096"] = {"mxfp4_GBps": round(bd4 / t4 / 1e6, 1), "mxfp4_frac_hbm": round(bd4 / t4 / 1e6 / hbm, 4),
@@ -345,13 +352,12 @@ def run_breakdown(mx, dev, pk, flush):
         R, C = xb.shape
         x3 = to_dev(xb, dev)
         del xb
-        res = mx.quantize_dual(x3, fmt, "ceil", "tcgen05")
-        t = timed(lambda: mx.quantize_dual(x3, fmt, "ceil", "tcgen05"), 10, None, stream)
+        t = timed([lambda: mx.quantize_dual(x3, fmt, "ceil", "tcgen05")], 10, stream)
         nbytes = R * C * 2 + 2 * (R * C + R * C // 32)
         out[f"c3_dual_{name}"] = {"ms": round(t, 4), "GBps": round(nbytes / t / 1e6, 1),
                                   "frac_hbm": round(nbytes / t / 1e6 / hbm, 4), "algorithmic_bytes": nbytes,
                                   "l2": "input larger than L2"}
-        del x3, res
+        del x3
         torch.cuda.empty_cache()
 
     # C4 / C5: block-scaled matmuls (operands quantised outside the timing)
@@ -361,9 +367,7 @@ def run_breakdown(mx, dev, pk, flush):
         b = mx.quantize(to_dev(synth.normal(N, K, sigma=bsig, seed=41), dev), bfmt, "row",
                         "floor" if bfmt == "e2m1" else "ceil", layout="tcgen05")
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-        for _ in range(3):
-            mx.gemm(a, b, c)
-        t = timed(lambda: mx.gemm(a, b, c), 10, None, stream)
+        t = timed([lambda: mx.gemm(a, b, c)], 10, stream)
         tf = 2.0 * M * N * K / (t * 1e-3) / 1e12
         out[name] = {"ms": round(t, 4), "TFLOPS": round(tf, 1), "frac_mx_peak_measured": round(tf / mx_peak, 4),
                      "mx_peak_measured_TFLOPS": mx_peak, "frac_mx_nominal_4500": round(tf / MX_NOMINAL_TFLOPS, 4),

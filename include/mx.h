@@ -119,15 +119,15 @@ mx_status mx_quantize(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt f
  * mx_quantize_nvfp4_noalloc -- NVFP4 quantisation that never allocates device memory.
  * The pages have no counterpart to this call; it exists for callers of this library.
  *
- * mx_quantize(fmt = MX_FMT_NVFP4) needs a small scratch buffer for per-CTA partial
- * maxima, which the library allocates with cudaMalloc on the first NVFP4 call on each
- * device.  Callers that cannot allow a cudaMalloc -- a serving loop that reserves all
- * device memory at start-up and must not take the implicit device synchronisation or
- * the out-of-memory risk of an allocation on its request path, or a host framework that
- * owns all device memory through its own allocator -- call this variant instead.  It runs
- * the same kernels and produces bit-identical outputs, with the scratch in a fixed
- * static device array of MX_NOALLOC_MAX_PARTIALS fp32 values (4 KiB) that every GPU
- * loading the library holds until the process exits.
+ * mx_quantize(fmt = MX_FMT_NVFP4) needs a small scratch buffer (grid-barrier words and
+ * per-CTA partial maxima), which the library allocates with cudaMalloc on the first
+ * NVFP4 call on each device.  Callers that cannot allow a cudaMalloc -- a serving loop
+ * that reserves all device memory at start-up and must not take the implicit device
+ * synchronisation or the out-of-memory risk of an allocation on its request path, or a
+ * host framework that owns all device memory through its own allocator -- call this
+ * variant instead.  It runs the same kernels and produces bit-identical outputs, with the
+ * scratch in a fixed static device array of 64 + MX_NOALLOC_MAX_PARTIALS fp32 values
+ * (4.25 KiB) that every GPU loading the library holds until the process exits.
  *
  * Arguments are those of mx_quantize with fmt = MX_FMT_NVFP4 and axis = ROW (cols a
  * multiple of 16, global_scale required, same layouts, alignment and ownership).
@@ -137,13 +137,16 @@ mx_status mx_quantize(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt f
  *     cudaGetSymbolAddress; neither allocates).  Make that first call before any stream
  *     capture on that device.
  *   - Limit: the call needs one scratch slot per CTA of its maximum pass, that is
- *     min(ceil(rows * cols / 8192), 4 x the SM count) slots.  A call that would need more
+ *     min(ceil(rows * cols / 8192), 3 x the SM count) slots.  A call that would need more
  *     than MX_NOALLOC_MAX_PARTIALS returns MX_ERR_SHAPE without launching (on a 148-SM
- *     B200 the count never exceeds 592).
+ *     B200 the count never exceeds 444).
  *   - Every call shares the one array, which keeps the previous call's contents.  Each
- *     call writes every slot it later reads, so nothing needs clearing, but calls whose
- *     GPU work overlaps (for example on two streams without ordering between them) race
- *     on the array and may produce wrong results.  Order such calls on one stream.
+ *     call writes every partial-maximum slot it later reads; the barrier words must be
+ *     zero when a call starts: they are zero at load time and every completed call leaves
+ *     them zero (after a watchdog timeout, mx_watchdog_status(clear = 1) zeroes them).
+ *     Calls whose GPU work overlaps (for example on two streams without ordering between
+ *     them) race on the array and may produce wrong results.  Order such calls on one
+ *     stream.
  */
 #define MX_NOALLOC_MAX_PARTIALS 1024
 mx_status mx_quantize_nvfp4_noalloc(const void *src_bf16, int64_t rows, int64_t cols, void *out_elems,

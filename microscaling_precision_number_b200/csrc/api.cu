@@ -59,6 +59,14 @@ bool single_layout(int l) { return l == MX_LAYOUT_ROWMAJOR || l == MX_LAYOUT_TCG
 namespace mxk {
 void record_cuda_error(cudaError_t e) { g_last_cuda_error = (int)e; }
 
+cudaError_t device_info(int *num_sms, int **watchdog) {
+    DeviceState *d = nullptr;
+    if (device_state(&d) != MX_OK) return (cudaError_t)g_last_cuda_error;
+    *num_sms = d->num_sms;
+    *watchdog = d->watchdog;
+    return cudaSuccess;
+}
+
 void *tensor_map_encoder() {
     static void *fn = nullptr;
     static std::once_flag once;
@@ -110,6 +118,13 @@ mx_status mx_watchdog_status(int *code, int clear) {
         const int zero = 0;
         e = cudaMemcpyToSymbol(g_watchdog_flag, &zero, sizeof(int));
         if (e != cudaSuccess) return cuda_fail(e);
+        // a call that gave up may have left grid-barrier words mid-way: reset them
+        if (d->partials) {
+            e = cudaMemset(d->partials, 0, 64 * sizeof(float));
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        e = mxk::noalloc_reset_barrier();
+        if (e != cudaSuccess) return cuda_fail(e);
     }
     if (code) *code = v;
     return v ? MX_ERR_TIMEOUT : MX_OK;
@@ -133,6 +148,7 @@ mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, m
     const int B = block_of(fmt);
     if ((axis == MX_AXIS_ROW ? cols : rows) % B) return MX_ERR_SHAPE;
     if (rows == 0 || cols == 0) return MX_OK;
+    if (!mxk::stream_supported(rows, cols)) return MX_ERR_SHAPE;
     if (!src || !out_elems || !out_scales) return MX_ERR_ARG;
     if (!aligned(src, 16) || !aligned(out_elems, 16)) return MX_ERR_ALIGN;
     if (global_scale && !aligned(global_scale, 4)) return MX_ERR_ALIGN;
@@ -150,22 +166,21 @@ mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, m
     const bool ceil = rounding == MX_SCALE_CEIL_RECIPE;
 
     if (fmt == MX_FMT_NVFP4) {
-        const int np = mxk::nvfp4_partials_count(rows * cols, d->num_sms);
         {
+            // one fixed-size scratch per device, allocated on first use; its barrier words
+            // start at zero and every completed call leaves them at zero
             std::lock_guard<std::mutex> lock(g_mu);
-            if (d->partials_cap < np) {
-                if (d->partials) cudaFree(d->partials);
-                d->partials = nullptr;
-                d->partials_cap = 0;
-                e = cudaMalloc(reinterpret_cast<void **>(&d->partials), sizeof(float) * (size_t)np);
+            if (!d->partials) {
+                const int nf = mxk::stream_nvfp4_scratch_floats(d->num_sms);
+                e = cudaMalloc(reinterpret_cast<void **>(&d->partials), sizeof(float) * (size_t)nf);
                 if (e != cudaSuccess) return cuda_fail(e);
-                d->partials_cap = np;
+                e = cudaMemset(d->partials, 0, sizeof(float) * (size_t)nf);
+                if (e != cudaSuccess) return cuda_fail(e);
+                d->partials_cap = nf;
             }
         }
-        e = mxk::launch_nvfp4_amax(src, rows * cols, d->partials, np, s);
-        if (e != cudaSuccess) return cuda_fail(e);
-        e = mxk::launch_nvfp4_quant(src, rows, cols, d->partials, np, global_scale, out_elems, rm, tc,
-                                    d->num_sms, s);
+        e = mxk::launch_stream_nvfp4(src, rows, cols, d->partials, 3 * d->num_sms, global_scale, out_elems, rm, tc,
+                                     d->watchdog, d->num_sms, s);
         if (e != cudaSuccess) return cuda_fail(e);
         if (tc) {
             e = mxk::launch_tcgen05_pad(tc, rows, cols / 16, s);
@@ -175,7 +190,7 @@ mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, m
     }
 
     if (axis == MX_AXIS_ROW) {
-        e = mxk::launch_quant_rows_mx(src, rows, cols, fmt, ceil, out_elems, rm, tc, d->num_sms, s);
+        e = mxk::launch_stream_rows_mx(src, rows, cols, fmt, ceil, out_elems, rm, tc, d->watchdog, d->num_sms, s);
         if (e != cudaSuccess) return cuda_fail(e);
         if (tc) {
             e = mxk::launch_tcgen05_pad(tc, rows, cols / 32, s);
@@ -241,6 +256,7 @@ mx_status mx_dequantize(const void *elems, const uint8_t *scales, const float *g
     if (rows < 0 || cols < 0) return MX_ERR_SHAPE;
     if (cols % block_of(fmt)) return MX_ERR_SHAPE;
     if (rows == 0 || cols == 0) return MX_OK;
+    if (!mxk::stream_supported(rows, cols)) return MX_ERR_SHAPE;
     if (!elems || !scales || !out_bf16) return MX_ERR_ARG;
     if (!aligned(elems, 16) || !aligned(out_bf16, 16)) return MX_ERR_ALIGN;
     if (global_scale && !aligned(global_scale, 4)) return MX_ERR_ALIGN;
@@ -250,8 +266,10 @@ mx_status mx_dequantize(const void *elems, const uint8_t *scales, const float *g
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool tc = layout == MX_LAYOUT_TCGEN05;
     cudaError_t e = fmt == MX_FMT_NVFP4
-                        ? mxk::launch_dequant_nvfp4(elems, scales, global_scale, rows, cols, tc, out_bf16, d->num_sms, s)
-                        : mxk::launch_dequant_mx(elems, scales, rows, cols, fmt, tc, out_bf16, d->num_sms, s);
+                        ? mxk::launch_stream_dequant_nvfp4(elems, scales, global_scale, rows, cols, tc, out_bf16,
+                                                           d->watchdog, d->num_sms, s)
+                        : mxk::launch_stream_dequant_mx(elems, scales, rows, cols, fmt, tc, out_bf16, d->watchdog,
+                                                        d->num_sms, s);
     return e == cudaSuccess ? MX_OK : cuda_fail(e);
 }
 

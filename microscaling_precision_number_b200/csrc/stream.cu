@@ -1,0 +1,835 @@
+// stream.cu -- bulk-copy pipelined streaming kernels: row-wise MX quantiser, NVFP4
+// tensor maximum and quantiser, MX / NVFP4 dequantisers.
+//
+// Sources (page title, section):
+//   "MXFP4 と NVFP4 は何が違うのか調べてみた"
+//     §2 "MXFP4 はブロック32と E8M0": 32 contiguous elements share one E8M0 scale; a NaN
+//        scale makes the whole block NaN; the element cast rounds to nearest even.
+//     §3 "NVFP4 はブロック16と E4M3、そして二段目": 16-element blocks with an unsigned
+//        E4M3 scale and an FP32 per-tensor scale = tensor amax / (6 * 448).
+//     §4 "精度の差はどこから出るか": floor and no-clip shared-exponent rules.
+//     §7 "ハードウェアの対応状況": MX scales apply as an exponent add (exact); NVFP4 applies
+//        an FP8 multiply then an FP32 multiply.
+//
+// Every kernel here is HBM-bound.  Structure shared by all of them:
+//   - persistent CTAs, a few per SM, walk fixed-size tiles of consecutive blocks;
+//   - one thread streams each tile into a 4-stage shared-memory ring with a single 1-D
+//     bulk copy (cp.async.bulk, completion on an mbarrier), so each SM keeps >100 KB of
+//     loads in flight with almost no issue cost;
+//   - one thread owns one quantisation block: the block maximum and the scale are
+//     computed once per block, never replicated across lanes;
+//   - shared-memory reads of a thread's block are rotated per thread so that every
+//     8-thread wavefront touches 8 distinct 16-byte bank groups (conflict-free);
+//   - 32-bit indices; the tcgen05 scale offset divides by the scales-per-row count with
+//     a precomputed multiply-shift (no integer division instruction).
+// Waits are bounded (watchdog); a CTA that gives up drains its own copies and returns.
+#include <cstdlib>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "codec.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace mxk {
+
+namespace {
+constexpr int kThreads = 256;
+constexpr int kStages = 4;
+constexpr int kTileBytes = 16384;
+constexpr int kCtasPerSm = 3;
+constexpr int kNvfp4PartialsOffset = 64;   // scratch floats: [0, 64) barrier words, then partial maxima
+}  // namespace
+
+// ---- host-computed divider: q = n / d for n < 2^31 --------------------------------------
+struct FastDiv {
+    uint32_t d, mul, shift;
+};
+
+static FastDiv make_fastdiv(uint32_t d) {
+    FastDiv f{d, 0u, 0u};
+    if (d <= 1) return f;
+    uint32_t l = 0;
+    while ((1ull << l) < d) l++;                       // ceil(log2 d)
+    const uint32_t p = 31 + l;
+    f.mul = (uint32_t)(((1ull << p) + d - 1) / d);
+    f.shift = p - 32;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
+    return f.d <= 1 ? n : (__umulhi(n, f.mul) >> f.shift);
+}
+
+// tcgen05 tiling offset of scale (r, c) with S scale columns (col_atoms = ceil(S/4)).
+__device__ __forceinline__ uint32_t tc_offset(uint32_t r, uint32_t c, uint32_t col_atoms) {
+    return (((r >> 7) * col_atoms + (c >> 2)) << 9) | ((r & 31u) << 4) | (((r >> 5) & 3u) << 2) | (c & 3u);
+}
+
+// ---- tile ring ------------------------------------------------------------------------------
+struct Ring {
+    uint8_t *buf;
+    uint64_t *full;
+    int *watchdog;
+    const uint8_t *src;         // global source of the streamed bytes
+    uint32_t tile_bytes;        // bytes per full tile
+    uint64_t total_bytes;       // bytes in the whole stream
+
+    __device__ __forceinline__ uint32_t bytes_of(uint32_t t) const {
+        const uint64_t off = (uint64_t)t * tile_bytes;
+        if (off >= total_bytes) return 0;
+        const uint64_t rem = total_bytes - off;
+        return rem < tile_bytes ? (uint32_t)rem : tile_bytes;
+    }
+    __device__ __forceinline__ void issue(uint32_t t, int s) const {
+        const uint32_t b = bytes_of(t);
+        if (b == 0) {                       // nothing to copy: complete the phase directly
+            mbar_arrive(&full[s]);
+            return;
+        }
+        mbar_arrive_expect_tx(&full[s], b);
+        bulk_load(buf + s * kTileBytes, src + (uint64_t)t * tile_bytes, b, &full[s]);
+    }
+};
+
+// Programmatic dependent launch: block until the previous kernel on the stream has
+// completed and its writes are visible (a no-op without a programmatic predecessor),
+// then let the next kernel's CTAs be scheduled as soon as ours retire.
+__device__ __forceinline__ void pdl_wait_and_release() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Runs body(tile, stage_ptr) over this CTA's tiles with the bulk-copy ring.
+template <typename Body>
+__device__ __forceinline__ void stream_tiles(Ring &ring, uint32_t n_tiles, Body body) {
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        for (int s = 0; s < kStages; s++) mbar_init(&ring.full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    uint32_t issued = 0;                                   // tiles issued by thread 0
+    if (tid == 0)
+        for (int s = 0; s < kStages; s++) {
+            const uint32_t t = blockIdx.x + (uint32_t)s * gridDim.x;
+            if (t < n_tiles) { ring.issue(t, s); issued++; }
+        }
+    uint32_t it = 0;
+    for (uint32_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
+        const int s = (int)(it % kStages);
+        const uint32_t phase = (it / kStages) & 1u;
+        const bool ok = mbar_wait_bounded(&ring.full[s], phase, ring.watchdog, WD_STREAM_FULL);
+        if (ok) body(t, ring.buf + s * kTileBytes);
+        __syncthreads();                                   // stage s is free again
+        if (tid == 0) {
+            const uint32_t tn = t + (uint32_t)kStages * gridDim.x;
+            if (tn < n_tiles && *reinterpret_cast<volatile int *>(ring.watchdog) == 0) {
+                ring.issue(tn, s);
+                issued++;
+            }
+        }
+    }
+    if (tid == 0 && *reinterpret_cast<volatile int *>(ring.watchdog) != 0) {
+        // error path: wait (bounded, short) for every copy this CTA issued
+        for (uint32_t j = it; j < issued; j++)
+            (void)mbar_wait_bounded(&ring.full[j % kStages], (j / kStages) & 1u, nullptr, 0, kDrainLimitNs);
+    }
+}
+
+// Packed fp32 pairs (sm_100a mul.rn.f32x2: two IEEE round-to-nearest products per instruction).
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+    return r;
+}
+__device__ __forceinline__ uint64_t splat2(float a) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// Eight bf16 (one uint4) times a scalar, as eight fp32 (element i in x[i]).
+__device__ __forceinline__ void scale8(const uint4 &v, uint64_t s2, float (&x)[8]) {
+    unpack2(mul2(bf16x2_to_f32x2(v.x), s2), x[0], x[1]);
+    unpack2(mul2(bf16x2_to_f32x2(v.y), s2), x[2], x[3]);
+    unpack2(mul2(bf16x2_to_f32x2(v.z), s2), x[4], x[5]);
+    unpack2(mul2(bf16x2_to_f32x2(v.w), s2), x[6], x[7]);
+}
+
+__device__ __forceinline__ uint32_t amax_words(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __vmaxu2(__vmaxu2(a & 0x7FFF7FFFu, b & 0x7FFF7FFFu), __vmaxu2(c & 0x7FFF7FFFu, d & 0x7FFF7FFFu));
+}
+
+// ---------------------------------------------------------------------------------------
+// Row-wise MX quantiser: thread = one 32-element block (64 input bytes).
+// ---------------------------------------------------------------------------------------
+template <int FMT, bool CEIL, bool RM, bool TC>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+mx_rows_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
+               uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc,
+               int *watchdog) {
+    pdl_wait_and_release();
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages];
+    Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
+              full, watchdog, src, kTileBytes, (uint64_t)n_blocks * 64};
+    constexpr uint32_t kBlocksPerTile = kTileBytes / 64;   // 256 = one per thread
+    const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
+    const uint32_t tid = threadIdx.x;
+    const uint32_t rot = tid >> 1;                          // bank-group rotation
+
+    stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
+        const uint32_t blk = t * kBlocksPerTile + tid;
+        if (blk >= n_blocks) return;
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const uint32_t c = (j + rot) & 3u;
+            v[j] = *reinterpret_cast<const uint4 *>(tile + tid * 64 + c * 16);
+        }
+        uint32_t m = __vmaxu2(amax_words(v[0].x, v[0].y, v[0].z, v[0].w), amax_words(v[1].x, v[1].y, v[1].z, v[1].w));
+        m = __vmaxu2(m, __vmaxu2(amax_words(v[2].x, v[2].y, v[2].z, v[2].w), amax_words(v[3].x, v[3].y, v[3].z, v[3].w)));
+        const uint32_t code = e8m0_from_amax_bits<FMT, CEIL>(hmax(m));
+        const uint64_t mul2x = splat2(e8m0_inverse_multiplier(code));
+        const bool nan_blk = code == 0xFFu;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const uint32_t c = (j + rot) & 3u;                 // which 8-element chunk of the block
+            float x[8];
+            scale8(v[j], mul2x, x);
+            if constexpr (FMT == FMT_E2M1) {
+                const uint32_t q = nan_blk ? 0u : cvt_e2m1x8(x);
+                reinterpret_cast<uint32_t *>(elems)[(size_t)blk * 4 + c] = q;
+            } else {
+                uint2 q = cvt_fp8x8<FMT>(x);
+                if (nan_blk) q = make_uint2(0u, 0u);
+                reinterpret_cast<uint2 *>(elems)[(size_t)blk * 4 + c] = q;
+            }
+        }
+        if constexpr (RM) sc_rm[blk] = (uint8_t)code;
+        if constexpr (TC) {
+            const uint32_t r = fdiv(blk, divS);
+            sc_tc[tc_offset(r, blk - r * divS.d, col_atoms)] = (uint8_t)code;
+        }
+    });
+}
+
+__device__ __forceinline__ uint32_t finite_mask(uint32_t m) {
+    // halfwords >= 0x7F80 (Inf/NaN magnitude) become 0
+    return m & __vcmpltu2(m, 0x7F807F80u);
+}
+
+// ---------------------------------------------------------------------------------------
+// NVFP4 quantisation of one 16 KiB tile (512 blocks of 16; thread = blocks tid, tid+256),
+// read from the shared-memory ring or, for a tile no longer resident, from global memory
+// (normally still in L2).  g is the per-tensor decode scale.
+//   per block: t = amax_b / (6 g), sb = UE4M3(t) (RNE, saturating), d = dec(sb) g,
+//   q = E2M1(x * (1/d)); a block holding a NaN/Inf gets sb = 0x7F and codes 0.
+// ---------------------------------------------------------------------------------------
+// Per-tensor constants of the NVFP4 block math, derived once per CTA from g.
+struct Nvfp4Consts {
+    float six_g;      // 6 g (fp32 RN)
+    float y;          // RN(1 / six_g)
+    bool fast;        // six_g >= 2^-80: t = amax_b / six_g may use the multiply-and-correct form
+};
+
+__device__ __forceinline__ Nvfp4Consts nvfp4_consts(float g, float *rtab) {
+    Nvfp4Consts c;
+    c.six_g = __fmul_rn(6.0f, g);
+    c.y = __frcp_rn(c.six_g);
+    c.fast = c.six_g >= 0x1p-80f;
+    // rtab[sb] = RN(1 / (dec(sb) g)), or 0 when that product is 0 (codes are then 0)
+    if (threadIdx.x < 128) {
+        const float d = __fmul_rn(ue4m3_to_f32(threadIdx.x), g);
+        rtab[threadIdx.x] = d != 0.0f ? __frcp_rn(d) : 0.0f;
+    }
+    __syncthreads();
+    return c;
+}
+
+// In the tile function below, t = RN(a / six_g) is formed as q0 = RN(a y),
+// r = a - q0 six_g (exact by FMA), t = RN(q0 + r y) with y = RN(1 / six_g) when FAST.  That
+// equals the correctly rounded quotient whenever a is at least 2^-100 (checked
+// exhaustively over every bf16 numerator for a wide set of divisors); with six_g >= 2^-80
+// every block whose quotient can reach the smallest UE4M3 subnormal has such a numerator,
+// and smaller quotients encode to 0 either way.  Otherwise the IEEE division is used.
+
+template <bool RM, bool TC, bool FAST>
+__device__ __forceinline__ void nvfp4_quant_tile(const uint8_t *tile, uint32_t t, uint32_t n_blocks,
+                                                 const Nvfp4Consts &cst, const float *rtab, const FastDiv &divS,
+                                                 uint32_t col_atoms, uint8_t *__restrict__ elems,
+                                                 uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc) {
+    // The thread's two blocks (tid, tid + 256) are processed side by side: the common path
+    // has no data-dependent branch, so the two dependency chains interleave.
+    constexpr uint32_t kBlocksPerTile = kTileBytes / 32;    // 512
+    const uint32_t tid = threadIdx.x;
+    const uint32_t rot = (tid >> 2) & 1u;
+    uint32_t blk[2];
+    bool ok[2];
+    uint4 v[2][2];
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+        const uint32_t lb = tid + h * kThreads;
+        blk[h] = t * kBlocksPerTile + lb;
+        ok[h] = blk[h] < n_blocks;
+#pragma unroll
+        for (int j = 0; j < 2; j++)
+            v[h][j] = ok[h] ? *reinterpret_cast<const uint4 *>(tile + lb * 32 + ((j + rot) & 1u) * 16)
+                            : make_uint4(0u, 0u, 0u, 0u);
+    }
+    uint32_t sb[2], q[2][2];
+    float r[2];
+    bool special[2];
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+        const uint32_t m = hmax(__vmaxu2(amax_words(v[h][0].x, v[h][0].y, v[h][0].z, v[h][0].w),
+                                         amax_words(v[h][1].x, v[h][1].y, v[h][1].z, v[h][1].w)));
+        special[h] = m >= 0x7F80u;                           // Inf/NaN in the block
+        const float a = __uint_as_float(m << 16);
+        float tq;
+        if constexpr (FAST) {
+            const float q0 = __fmul_rn(a, cst.y);
+            tq = __fmaf_rn(__fmaf_rn(-q0, cst.six_g, a), cst.y, q0);
+        } else {
+            tq = __fdiv_rn(a, cst.six_g);
+        }
+        sb[h] = cvt_fp8x2<FMT_E4M3>(tq, 0.0f) & 0xFFu;     // tq >= 0: sign bit stays 0
+        r[h] = rtab[sb[h] & 0x7Fu];                          // RN(1 / (dec(sb) g)), 0 if that is 1/0
+    }
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+        const uint64_t r2 = splat2(r[h]);
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+            float x[8];
+            scale8(v[h][j], r2, x);
+            if (__builtin_expect(isinf(r[h]), 0)) {
+                const float in[8] = {bf16_lo(v[h][j].x), bf16_hi(v[h][j].x), bf16_lo(v[h][j].y), bf16_hi(v[h][j].y),
+                                     bf16_lo(v[h][j].z), bf16_hi(v[h][j].z), bf16_lo(v[h][j].w), bf16_hi(v[h][j].w)};
+#pragma unroll
+                for (int i = 0; i < 8; i++)
+                    if (x[i] != x[i]) x[i] = in[i];                // 0 * Inf: keep the signed zero
+            }
+            q[h][j] = cvt_e2m1x8(x);
+        }
+        if (special[h] || r[h] == 0.0f) q[h][0] = q[h][1] = 0u;    // NaN block, or d = 0: codes 0
+        if (special[h]) sb[h] = 0x7Fu;                               // UE4M3 NaN: the block is NaN
+    }
+#pragma unroll
+    for (int h = 0; h < 2; h++) {
+        if (!ok[h]) continue;
+#pragma unroll
+        for (int j = 0; j < 2; j++)
+            reinterpret_cast<uint32_t *>(elems)[(size_t)blk[h] * 2 + ((j + rot) & 1u)] = q[h][j];
+        if constexpr (RM) sc_rm[blk[h]] = (uint8_t)sb[h];
+        if constexpr (TC) {
+            const uint32_t rr = fdiv(blk[h], divS);
+            sc_tc[tc_offset(rr, blk[h] - rr * divS.d, col_atoms)] = (uint8_t)sb[h];
+        }
+    }
+}
+
+// Tensor maximum of every CTA's partial maxima (all CTAs compute the same value in the
+// same order) and the NVFP4 decode scale g = amax / 2688 (1 when the tensor is all zero).
+__device__ __forceinline__ float nvfp4_global_scale(const float *partials, int n_partials, float *warp_max) {
+    const uint32_t tid = threadIdx.x;
+    float a = 0.0f;
+    for (int i = tid; i < n_partials; i += kThreads) a = fmaxf(a, partials[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+    if ((tid & 31) == 0) warp_max[tid >> 5] = a;
+    __syncthreads();
+    a = 0.0f;
+    for (int w = 0; w < kThreads / 32; w++) a = fmaxf(a, warp_max[w]);
+    return a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f);
+}
+
+// Finite |x| maximum of one streamed tile, folded into acc (Inf/NaN excluded).
+__device__ __forceinline__ uint32_t finite_amax_tile(const uint8_t *tile, uint32_t nbytes, uint32_t acc) {
+    const uint32_t tid = threadIdx.x;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const uint32_t off = (tid + j * kThreads) * 16;    // consecutive threads, consecutive 16 B
+        if (off < nbytes) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(tile + off);
+            uint32_t m = amax_words(v.x, v.y, v.z, v.w);
+            if (__builtin_expect((m & 0x7F800000u) == 0x7F800000u || (m & 0x7F80u) == 0x7F80u, 0)) {
+                m = __vmaxu2(__vmaxu2(finite_mask(v.x & 0x7FFF7FFFu), finite_mask(v.y & 0x7FFF7FFFu)),
+                             __vmaxu2(finite_mask(v.z & 0x7FFF7FFFu), finite_mask(v.w & 0x7FFF7FFFu)));
+            }
+            acc = __vmaxu2(acc, m);
+        }
+    }
+    return acc;
+}
+
+// Block-wide maximum of a per-thread packed |x| maximum; thread 0 stores it as fp32.
+__device__ __forceinline__ void store_partial(uint32_t acc, float *dst, uint32_t *warp_u) {
+    const uint32_t tid = threadIdx.x;
+    uint32_t m = hmax(acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) warp_u[tid >> 5] = m;
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t r = 0;
+        for (int w = 0; w < kThreads / 32; w++) r = max(r, warp_u[w]);
+        *dst = __uint_as_float(r << 16);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Grid-wide barrier for a cooperatively launched grid (all CTAs co-resident).
+// bar[0] counts arrivals and is zero between uses (the last arrival resets it);
+// bar[32] (another 128-byte line, so polling does not contend with the arrivals) is a
+// generation number that the last arrival advances.  Arrival is an acq_rel atomic (it
+// publishes this CTA's earlier writes and lets the last arrival see everyone's); waiters
+// poll the generation with acquire loads and a short back-off.  The wait is bounded: on a
+// timeout (or once another CTA has given up) it returns false in every thread.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ bool grid_barrier(unsigned int *bar, uint32_t nctas, int *watchdog) {
+    __syncthreads();
+    int ok = 1;
+    if (threadIdx.x == 0) {
+        unsigned int *cnt = bar, *gen = bar + 32;
+        unsigned int g0, old, cur;
+        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(g0) : "l"(gen) : "memory");
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
+        if (old == nctas - 1) {
+            asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(cnt) : "memory");
+            asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(gen) : "memory");
+        } else {
+            const uint64_t t0 = globaltimer_ns();
+            for (uint32_t i = 1;; i++) {
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(gen) : "memory");
+                if (cur != g0) break;
+                __nanosleep(20);
+                if ((i & 31u) == 0u) {
+                    if (*reinterpret_cast<volatile int *>(watchdog) != 0) { ok = 0; break; }
+                    if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicExch(watchdog, WD_GRID_BARRIER); ok = 0; break; }
+                }
+            }
+        }
+    }
+    return __syncthreads_and(ok) != 0;
+}
+
+// ---------------------------------------------------------------------------------------
+// NVFP4 in one cooperative kernel.
+//   phase 1: stream this CTA's tiles through the ring, fold the finite |x| maximum;
+//   barrier: every CTA has published its partial maximum;
+//   phase 2: every CTA derives g, then quantises its tiles newest first: the last
+//   min(n, stages) tiles are still in its ring, older ones are re-read from global memory
+//   (normally L2).  Inputs up to ~stages x 16 KiB x CTAs are read from HBM once.
+// ---------------------------------------------------------------------------------------
+template <bool RM, bool TC>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+nvfp4_fused_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
+                   float *__restrict__ partials, unsigned int *__restrict__ bar, float *__restrict__ g_out,
+                   uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc,
+                   int *watchdog) {
+    pdl_wait_and_release();
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ float warp_max[kThreads / 32];
+    Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
+              full, watchdog, src, kTileBytes, (uint64_t)n_blocks * 32};
+    constexpr uint32_t kBlocksPerTile = kTileBytes / 32;
+    const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
+
+    uint32_t acc = 0;
+    stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
+        acc = finite_amax_tile(tile, ring.bytes_of(t), acc);
+    });
+    store_partial(acc, partials + blockIdx.x, reinterpret_cast<uint32_t *>(warp_max));
+    if (!grid_barrier(bar, gridDim.x, watchdog)) return;
+
+    const float g = nvfp4_global_scale(partials, (int)gridDim.x, warp_max);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    __shared__ float rtab[128];
+    const Nvfp4Consts cst = nvfp4_consts(g, rtab);
+
+    const uint32_t G = gridDim.x, bid = blockIdx.x;
+    const uint32_t n_my = n_tiles > bid ? (n_tiles - 1 - bid) / G + 1 : 0;
+    for (int32_t j = (int32_t)n_my - 1; j >= 0; j--) {
+        const uint32_t t = bid + (uint32_t)j * G;
+        const bool resident = (uint32_t)j + kStages >= n_my;
+        const uint8_t *base = resident ? ring.buf + (j % kStages) * kTileBytes : src + (size_t)t * kTileBytes;
+        if (cst.fast) nvfp4_quant_tile<RM, TC, true>(base, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
+        else nvfp4_quant_tile<RM, TC, false>(base, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// NVFP4 as two kernels (used when a cooperative launch is not possible).
+// Pass 1: per-CTA maximum of the finite |x| (Inf/NaN excluded).
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+nvfp4_amax_bulk_kernel(const uint8_t *__restrict__ src, uint64_t n_bytes, float *__restrict__ partials,
+                       int *watchdog) {
+    pdl_wait_and_release();
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ uint32_t warp_u[kThreads / 32];
+    Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
+              full, watchdog, src, kTileBytes, n_bytes};
+    const uint32_t n_tiles = (uint32_t)((n_bytes + kTileBytes - 1) / kTileBytes);
+    uint32_t acc = 0;
+    stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
+        acc = finite_amax_tile(tile, ring.bytes_of(t), acc);
+    });
+    store_partial(acc, partials + blockIdx.x, warp_u);
+}
+
+// Pass 2: reads the partial maxima written by pass 1.
+template <bool RM, bool TC>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+nvfp4_quant_bulk_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
+                        const float *__restrict__ partials, int n_partials, float *__restrict__ g_out,
+                        uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc,
+                        int *watchdog) {
+    pdl_wait_and_release();
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ float warp_max[kThreads / 32];
+    Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
+              full, watchdog, src, kTileBytes, (uint64_t)n_blocks * 32};
+    const float g = nvfp4_global_scale(partials, n_partials, warp_max);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    __shared__ float rtab[128];
+    const Nvfp4Consts cst = nvfp4_consts(g, rtab);
+    const uint32_t n_tiles = (n_blocks + kTileBytes / 32 - 1) / (kTileBytes / 32);
+    stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
+        if (cst.fast) nvfp4_quant_tile<RM, TC, true>(tile, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
+        else nvfp4_quant_tile<RM, TC, false>(tile, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
+    });
+}
+
+// ---------------------------------------------------------------------------------------
+// Dequantisers: thread = one block; codes streamed through the ring, scales read
+// directly, bf16 written as 16-byte vectors.
+// ---------------------------------------------------------------------------------------
+template <int FMT, bool TC>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restrict__ scales,
+                       uint32_t n_blocks, FastDiv divS, uint32_t col_atoms, uint4 *__restrict__ out,
+                       int *watchdog) {
+    pdl_wait_and_release();
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages];
+    constexpr uint32_t kCodeBytes = FMT == FMT_E2M1 ? 16 : 32;           // per block
+    constexpr uint32_t kBlocksPerTile = kThreads;                          // one per thread
+    Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
+              full, watchdog, elems, kBlocksPerTile * kCodeBytes, (uint64_t)n_blocks * kCodeBytes};
+    const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
+    const uint32_t tid = threadIdx.x;
+    stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
+        const uint32_t blk = t * kBlocksPerTile + tid;
+        if (blk >= n_blocks) return;
+        uint32_t s;
+        if constexpr (TC) {
+            const uint32_t r = fdiv(blk, divS);
+            s = scales[tc_offset(r, blk - r * divS.d, col_atoms)];
+        } else {
+            s = scales[blk];
+        }
+        const float mul = s == 0xFFu ? __uint_as_float(0x7FC00000u) : e8m0_multiplier(s);
+        uint4 *dst = out + (size_t)blk * 4;
+        if constexpr (FMT == FMT_E2M1) {
+            const uint4 c = *reinterpret_cast<const uint4 *>(tile + tid * 16);
+            const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                float y[8];
+                e2m1x8_to_f32(w[j], y);
+                uint4 o;
+                o.x = f32x2_to_bf16x2(__fmul_rn(y[0], mul), __fmul_rn(y[1], mul));
+                o.y = f32x2_to_bf16x2(__fmul_rn(y[2], mul), __fmul_rn(y[3], mul));
+                o.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
+                o.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
+                dst[j] = o;
+            }
+        } else {
+            const uint32_t rot = (tid >> 2) & 1u;
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const uint32_t hc = (h + rot) & 1u;
+                const uint4 c = *reinterpret_cast<const uint4 *>(tile + tid * 32 + hc * 16);
+                const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                for (int j = 0; j < 2; j++) {
+                    float y[8];
+                    fp8x2_to_f32<FMT>(w[2 * j] & 0xFFFFu, y[0], y[1]);
+                    fp8x2_to_f32<FMT>(w[2 * j] >> 16, y[2], y[3]);
+                    fp8x2_to_f32<FMT>(w[2 * j + 1] & 0xFFFFu, y[4], y[5]);
+                    fp8x2_to_f32<FMT>(w[2 * j + 1] >> 16, y[6], y[7]);
+                    uint4 o;
+                    o.x = f32x2_to_bf16x2(__fmul_rn(y[0], mul), __fmul_rn(y[1], mul));
+                    o.y = f32x2_to_bf16x2(__fmul_rn(y[2], mul), __fmul_rn(y[3], mul));
+                    o.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
+                    o.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
+                    dst[hc * 2 + j] = o;
+                }
+            }
+        }
+    });
+}
+
+template <bool TC>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+dequant_nvfp4_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restrict__ scales,
+                          const float *__restrict__ g_ptr, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
+                          uint4 *__restrict__ out, int *watchdog) {
+    pdl_wait_and_release();
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[kStages];
+    constexpr uint32_t kBlocksPerTile = 2 * kThreads;                      // 8 code bytes each
+    // Bulk copies move whole 16-byte units (block pairs); with an odd block count the
+    // last block's 8 code bytes are read straight from global memory by its thread.
+    Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
+              full, watchdog, elems, kBlocksPerTile * 8, (uint64_t)(n_blocks & ~1u) * 8};
+    const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
+    const uint32_t tid = threadIdx.x;
+    const float g = *g_ptr;
+    stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
+        const uint32_t blk0 = t * kBlocksPerTile + tid * 2;   // two consecutive blocks
+        if (blk0 >= n_blocks) return;
+        uint4 c;
+        if (blk0 + 1 < n_blocks) {
+            c = *reinterpret_cast<const uint4 *>(tile + tid * 16);
+        } else {
+            const uint2 h = *reinterpret_cast<const uint2 *>(elems + (size_t)blk0 * 8);
+            c = make_uint4(h.x, h.y, 0u, 0u);
+        }
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            const uint32_t blk = blk0 + b;
+            if (blk >= n_blocks) break;
+            uint32_t s;
+            if constexpr (TC) {
+                const uint32_t r = fdiv(blk, divS);
+                s = scales[tc_offset(r, blk - r * divS.d, col_atoms)] & 0x7Fu;
+            } else {
+                s = scales[blk] & 0x7Fu;
+            }
+            const float sbv = s == 0x7Fu ? __uint_as_float(0x7FC00000u) : ue4m3_to_f32(s);
+#pragma unroll
+            for (int j = 0; j < 2; j++) {
+                float y[8];
+                e2m1x8_to_f32(w[2 * b + j], y);
+                uint4 o;
+                o.x = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[0], sbv), g), __fmul_rn(__fmul_rn(y[1], sbv), g));
+                o.y = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[2], sbv), g), __fmul_rn(__fmul_rn(y[3], sbv), g));
+                o.z = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[4], sbv), g), __fmul_rn(__fmul_rn(y[5], sbv), g));
+                o.w = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[6], sbv), g), __fmul_rn(__fmul_rn(y[7], sbv), g));
+                out[(size_t)blk * 2 + j] = o;
+            }
+        }
+    });
+}
+
+// ---------------------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------------------
+static int stream_grid(uint32_t n_tiles, int num_sms) {
+    int64_t g = (int64_t)num_sms * kCtasPerSm;
+    if (g > n_tiles) g = n_tiles;
+    return g < 1 ? 1 : (int)g;
+}
+constexpr size_t kStreamSmem = (size_t)kStages * kTileBytes + 128;
+
+// Launch with programmatic dependent launch enabled: the kernel may be scheduled while the
+// previous kernel on the stream drains; its first instruction (griddepcontrol.wait) holds it
+// until that kernel has completed.  `coop` additionally requests a cooperative launch (all
+// CTAs co-resident, needed by the grid barrier).  The shared-memory attribute is set once
+// per device and kernel.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_ex(void (*kernel)(KArgs...), int grid, cudaStream_t st, bool coop, bool pdl,
+                             Args... args) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void *>> configured;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        const auto key = std::make_pair(dev, reinterpret_cast<const void *>(kernel));
+        if (!configured.count(key)) {
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
+            if (e != cudaSuccess) return e;
+            configured.insert(key);
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kStreamSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (pdl) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        n++;
+    }
+    if (coop) {
+        attr[n].id = cudaLaunchAttributeCooperative;
+        attr[n].val.cooperative = 1;
+        n++;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// Set the dynamic shared-memory attribute of a stream kernel (needed before occupancy queries).
+template <typename... KArgs>
+static cudaError_t launch_ex_config(void (*kernel)(KArgs...)) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_stream(void (*kernel)(KArgs...), int grid, cudaStream_t st, Args... args) {
+    return launch_ex(kernel, grid, st, false, true, args...);
+}
+
+bool stream_supported(int64_t rows, int64_t cols) {
+    return rows * cols / 16 < ((int64_t)1 << 31);   // block indices fit 31 bits
+}
+
+template <int FMT, bool CEIL, bool RM, bool TC>
+static cudaError_t launch_rows_t(const void *src, uint32_t n_blocks, FastDiv f, uint32_t col_atoms, void *elems,
+                                 uint8_t *rm, uint8_t *tc, int *wd, int num_sms, cudaStream_t st) {
+    const uint32_t n_tiles = (n_blocks + 255) / 256;
+    return launch_stream(mx_rows_kernel<FMT, CEIL, RM, TC>, stream_grid(n_tiles, num_sms), st,
+                         static_cast<const uint8_t *>(src), n_blocks, f, col_atoms, static_cast<uint8_t *>(elems), rm,
+                         tc, wd);
+}
+
+template <int FMT, bool CEIL>
+static cudaError_t launch_rows_layout(const void *src, uint32_t nb, FastDiv f, uint32_t ca, void *elems, uint8_t *rm,
+                                      uint8_t *tc, int *wd, int num_sms, cudaStream_t st) {
+    if (rm && tc) return launch_rows_t<FMT, CEIL, true, true>(src, nb, f, ca, elems, rm, tc, wd, num_sms, st);
+    if (rm) return launch_rows_t<FMT, CEIL, true, false>(src, nb, f, ca, elems, rm, tc, wd, num_sms, st);
+    return launch_rows_t<FMT, CEIL, false, true>(src, nb, f, ca, elems, rm, tc, wd, num_sms, st);
+}
+
+cudaError_t launch_stream_rows_mx(const void *src, int64_t rows, int64_t cols, int fmt, bool ceil, void *elems,
+                                  uint8_t *rm, uint8_t *tc, int *wd, int num_sms, cudaStream_t st) {
+    const uint32_t n_blocks = (uint32_t)(rows * cols / 32);
+    const uint32_t S = (uint32_t)(cols / 32);
+    const FastDiv f = make_fastdiv(S);
+    const uint32_t ca = (S + 3) / 4;
+    switch (fmt * 2 + (ceil ? 1 : 0)) {
+    case FMT_E4M3 * 2 + 0: return launch_rows_layout<FMT_E4M3, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E4M3 * 2 + 1: return launch_rows_layout<FMT_E4M3, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E5M2 * 2 + 0: return launch_rows_layout<FMT_E5M2, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E5M2 * 2 + 1: return launch_rows_layout<FMT_E5M2, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E2M1 * 2 + 0: return launch_rows_layout<FMT_E2M1, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E2M1 * 2 + 1: return launch_rows_layout<FMT_E2M1, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+int stream_nvfp4_scratch_floats(int num_sms) { return kNvfp4PartialsOffset + kCtasPerSm * num_sms; }
+
+template <bool RM, bool TC>
+static cudaError_t launch_nvfp4_t(const uint8_t *src, uint32_t nb, FastDiv f, uint32_t ca, float *scratch,
+                                  int max_partials, float *g, uint8_t *elems, uint8_t *rm, uint8_t *tc, int *wd,
+                                  int num_sms, cudaStream_t st) {
+    const uint32_t n_tiles = (nb + 511) / 512;
+    float *partials = scratch + kNvfp4PartialsOffset;
+    unsigned int *bar = reinterpret_cast<unsigned int *>(scratch);
+    int grid = stream_grid(n_tiles, num_sms);
+    if (grid > max_partials) grid = max_partials;
+    static const bool two_pass_only = [] {
+        const char *v = getenv("MX_NVFP4_TWO_PASS");
+        return v != nullptr && v[0] == '1';
+    }();
+    if (!two_pass_only) {
+        // one cooperative kernel: every CTA must be resident at once
+        int per_sm = 0;
+        cudaError_t e = launch_ex_config(nvfp4_fused_kernel<RM, TC>);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_fused_kernel<RM, TC>, kThreads, kStreamSmem);
+        if (e != cudaSuccess) return e;
+        const int coop_grid = grid < per_sm * num_sms ? grid : per_sm * num_sms;
+        if (coop_grid >= 1) {
+            e = launch_ex(nvfp4_fused_kernel<RM, TC>, coop_grid, st, true, true, src, nb, f, ca, partials, bar, g,
+                          elems, rm, tc, wd);
+            if (e == cudaSuccess) return e;
+            (void)cudaGetLastError();   // not launchable as requested: clear and fall back
+            e = launch_ex(nvfp4_fused_kernel<RM, TC>, coop_grid, st, true, false, src, nb, f, ca, partials, bar,
+                          g, elems, rm, tc, wd);
+            if (e == cudaSuccess) return e;
+            (void)cudaGetLastError();
+        }
+    }
+    // two kernels: per-CTA maxima, then quantisation
+    cudaError_t e = launch_stream(nvfp4_amax_bulk_kernel, grid, st, src, (uint64_t)nb * 32, partials, wd);
+    if (e != cudaSuccess) return e;
+    return launch_stream(nvfp4_quant_bulk_kernel<RM, TC>, stream_grid(n_tiles, num_sms), st, src, nb, f, ca,
+                         (const float *)partials, grid, g, elems, rm, tc, wd);
+}
+
+cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, float *scratch, int max_partials,
+                                float *g, void *elems, uint8_t *rm, uint8_t *tc, int *wd, int num_sms,
+                                cudaStream_t st) {
+    const uint32_t nb = (uint32_t)(rows * cols / 16), S = (uint32_t)(cols / 16);
+    const FastDiv f = make_fastdiv(S);
+    const uint32_t ca = (S + 3) / 4;
+    const uint8_t *s8 = static_cast<const uint8_t *>(src);
+    uint8_t *e8 = static_cast<uint8_t *>(elems);
+    if (rm && tc) return launch_nvfp4_t<true, true>(s8, nb, f, ca, scratch, max_partials, g, e8, rm, tc, wd, num_sms, st);
+    if (rm) return launch_nvfp4_t<true, false>(s8, nb, f, ca, scratch, max_partials, g, e8, rm, tc, wd, num_sms, st);
+    return launch_nvfp4_t<false, true>(s8, nb, f, ca, scratch, max_partials, g, e8, rm, tc, wd, num_sms, st);
+}
+
+template <int FMT, bool TC>
+static cudaError_t launch_dq_t(const void *elems, const uint8_t *scales, uint32_t nb, FastDiv f, uint32_t ca,
+                               void *out, int *wd, int num_sms, cudaStream_t st) {
+    const uint32_t n_tiles = (nb + kThreads - 1) / kThreads;
+    return launch_stream(dequant_mx_bulk_kernel<FMT, TC>, stream_grid(n_tiles, num_sms), st,
+                         static_cast<const uint8_t *>(elems), scales, nb, f, ca, static_cast<uint4 *>(out), wd);
+}
+
+cudaError_t launch_stream_dequant_mx(const void *elems, const uint8_t *scales, int64_t rows, int64_t cols, int fmt,
+                                     bool tc, void *out, int *wd, int num_sms, cudaStream_t st) {
+    const uint32_t nb = (uint32_t)(rows * cols / 32), S = (uint32_t)(cols / 32);
+    const FastDiv f = make_fastdiv(S);
+    const uint32_t ca = (S + 3) / 4;
+    switch (fmt) {
+    case FMT_E4M3: return tc ? launch_dq_t<FMT_E4M3, true>(elems, scales, nb, f, ca, out, wd, num_sms, st)
+                             : launch_dq_t<FMT_E4M3, false>(elems, scales, nb, f, ca, out, wd, num_sms, st);
+    case FMT_E5M2: return tc ? launch_dq_t<FMT_E5M2, true>(elems, scales, nb, f, ca, out, wd, num_sms, st)
+                             : launch_dq_t<FMT_E5M2, false>(elems, scales, nb, f, ca, out, wd, num_sms, st);
+    case FMT_E2M1: return tc ? launch_dq_t<FMT_E2M1, true>(elems, scales, nb, f, ca, out, wd, num_sms, st)
+                             : launch_dq_t<FMT_E2M1, false>(elems, scales, nb, f, ca, out, wd, num_sms, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_stream_dequant_nvfp4(const void *elems, const uint8_t *scales, const float *g, int64_t rows,
+                                        int64_t cols, bool tc, void *out, int *wd, int num_sms, cudaStream_t st) {
+    const uint32_t nb = (uint32_t)(rows * cols / 16), S = (uint32_t)(cols / 16);
+    const FastDiv f = make_fastdiv(S);
+    const uint32_t ca = (S + 3) / 4;
+    const uint32_t n_tiles = (nb + 2 * kThreads - 1) / (2 * kThreads);
+    const int grid = stream_grid(n_tiles, num_sms);
+    const uint8_t *e8 = static_cast<const uint8_t *>(elems);
+    uint4 *o = static_cast<uint4 *>(out);
+    return tc ? launch_stream(dequant_nvfp4_bulk_kernel<true>, grid, st, e8, scales, g, nb, f, ca, o, wd)
+              : launch_stream(dequant_nvfp4_bulk_kernel<false>, grid, st, e8, scales, g, nb, f, ca, o, wd);
+}
+
+}  // namespace mxk

@@ -257,3 +257,43 @@ def test_empty_inputs_launch_nothing():
     q = mx.quantize(x, "e4m3", "row", "ceil")
     assert q.elems.numel() == 0
     assert mx.cast(torch.empty(0, dtype=torch.bfloat16, device="cuda"), "e2m1").numel() == 0
+
+
+def test_nvfp4_two_kernel_fallback_matches_oracle(tmp_path):
+    """The two-kernel NVFP4 path (used when a cooperative launch is impossible), forced in
+    a child process, gives the oracle's codes, scales and tensor scale."""
+    import os
+    import subprocess
+    import sys
+    script = r'''
+import sys, numpy as np, torch
+sys.path.insert(0, %r)
+import synth, oracle
+import microscaling_precision_number_b200 as mx
+for shape in [(5, 48), (130, 256), (512, 4096)]:
+    x = synth.weight_fp4(*shape, seed=shape[0])
+    t = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
+    q = mx.quantize(t, "nvfp4", "row", "ceil", layout="both")
+    e, s, g = oracle.quantize_nvfp4(x)
+    assert q.global_scale.cpu().numpy()[0] == np.float32(g)
+    assert np.array_equal(q.elems.cpu().numpy(), e.reshape(-1))
+    assert np.array_equal(q.scales.cpu().numpy(), s.reshape(-1))
+    assert np.array_equal(q.scales_alt.cpu().numpy(), oracle.to_tcgen05_layout(s))
+assert mx.watchdog_status() == 0
+print("two-pass ok")
+''' % os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, MX_NVFP4_TWO_PASS="1")
+    r = subprocess.run([sys.executable, "-c", script], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0 and "two-pass ok" in r.stdout, r.stdout + r.stderr
+
+
+@pytest.mark.parametrize("sigma_log2", [-60, -72, -78, -84, -95, -110])
+def test_nvfp4_tiny_tensor_scales(oracle, sigma_log2):
+    """Tensors whose per-tensor scale puts 6g on either side of 2^-80 (where the block
+    scale's quotient switches between the multiply-and-correct form and the IEEE divide)."""
+    x = synth.normal(64, 512, sigma=2.0 ** sigma_log2, seed=-sigma_log2)
+    q = mx.quantize(to_dev(x), "nvfp4", "row", "ceil", layout="rowmajor")
+    e_ref, s_ref, g_ref = oracle.quantize_nvfp4(x)
+    assert host(q.global_scale)[0] == np.float32(g_ref)
+    assert np.array_equal(host(q.elems), e_ref.reshape(-1))
+    assert np.array_equal(host(q.scales), s_ref.reshape(-1))
