@@ -9,7 +9,7 @@ import ctypes
 import os
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmx.so")
+LIB_PATH = os.environ.get("MX_LIB_PATH") or os.path.join(_PKG, "libmx.so")
 
 # enum values of include/mx.h
 MX_OK, MX_ERR_ARG, MX_ERR_SHAPE, MX_ERR_ALIGN, MX_ERR_LAYOUT, MX_ERR_CUDA, MX_ERR_TIMEOUT = range(7)

@@ -14,18 +14,23 @@
 // K-major; scales per 32 along K in the tcgen05 tiling (512-byte atoms of 128 rows x 4
 // scale columns).
 //
-// Kernel structure (one CTA per 128 x 256 output tile, 6 warps):
-//   warp 4  TMA producer: per 128-wide K step, 2-D TMA loads of the A tile (128 x 128 B)
+// Kernel structure: persistent CTAs (one per SM, 10 warps), 128 x 256 output tiles
+// (128 x 128 when N is not a multiple of 256):
+//   warp 8  TMA producer: per 128-wide K step, 2-D TMA loads of the A tile (128 x 128 B)
 //           and the B tile (256 x 128 B, E2M1 expanded by the TMA to one byte per
 //           element) with 128-byte swizzle, plus bulk copies of the matching scale atoms
-//           (1 for A, 2 for B) into a 4-stage shared-memory ring (mbarrier "full").
-//   warp 5  TMEM allocator and MMA issuer: copies the stage's scale atoms into tensor
+//           (1 for A, 2 for B) into a 4-stage shared-memory ring (mbarrier "full"); the
+//           ring runs on across tile boundaries.
+//   warp 9  TMEM allocator and MMA issuer: copies the stage's scale atoms into tensor
 //           memory (tcgen05.cp 32x128b.warpx4), then issues four
 //           tcgen05.mma.kind::mxf8f6f4.block_scale (K = 32 each; the scale byte of each
 //           is selected by the scale-factor id in the instruction descriptor), and
-//           releases the stage with tcgen05.commit on its "empty" barrier.
-//   warps 0-3  epilogue: tcgen05.ld of the 128 x 256 fp32 accumulator, one TMEM lane
-//           (= one output row) per thread, bf16 conversion, 16-byte global stores.
+//           releases the stage with tcgen05.commit on its "empty" barrier; a finished
+//           tile is signalled on "acc_full".
+//   warps 0-7  epilogue: two warps per 32-lane TMEM quadrant (one per column half) load
+//           the fp32 accumulator (tcgen05.ld), convert to bf16 in registers, release the
+//           accumulator on "acc_empty" -- the next tile's MMAs start now -- and then
+//           store their row segments with 16-byte global stores.
 // All waits are bounded by the watchdog; tensor memory is always released.
 #include <cuda.h>
 #include "codec.cuh"
@@ -37,7 +42,9 @@ namespace mxk {
 namespace {
 constexpr int kBM = 128, kBK = 128;                      // tile rows; kBK in elements (= smem bytes)
 constexpr int kStages = 4;
-constexpr int kGemmThreads = 192;
+constexpr int kEpilogueWarps = 8;                  // two per TMEM lane quadrant
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kGemmThreads = 320;
 constexpr int kABytes = kBM * kBK;                       // 16 KiB
 constexpr int kSfaBytes = 512;
 constexpr uint32_t kTmemCols = 512;                      // accumulator (<= 256) + scale slots
@@ -126,12 +133,31 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---- tile order ------------------------------------------------------------------------------
+// Banded raster: N-tiles are grouped into bands of `band` tiles whose B panels fit in L2;
+// within a band the tiles run M-major, so concurrently resident CTAs share A panels and the
+// band's B panels are read from HBM about once.
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int band, int &m_blk, int &n_blk) {
+    const int per_band = tiles_m * band;
+    const int b = t / per_band;
+    const int rem = t - b * per_band;
+    const int n0 = b * band;
+    const int bw = tiles_n - n0 < band ? tiles_n - n0 : band;   // the last band may be narrower
+    m_blk = rem / bw;
+    n_blk = n0 + (rem - m_blk * bw);
+}
+
 // ---- kernel ------------------------------------------------------------------------------
+// Persistent: CTA c processes output tiles c, c + grid, c + 2 grid, ... (row-major over the
+// M/128 x N/BN tile grid).  The TMA producer and the MMA issuer run through the K steps of
+// consecutive tiles without a break (the shared-memory ring spans tiles).  The epilogue
+// drains a finished accumulator into registers, releases it (acc_empty) so that the MMAs
+// of the next tile start at once, and then writes its bf16 rows while they run.
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const uint8_t *__restrict__ a_sc, const uint8_t *__restrict__ b_sc,
-               uint16_t *__restrict__ C, int M, int N, int K, uint32_t b_fmt_code, int *watchdog) {
+               uint16_t *__restrict__ C, int M, int N, int K, uint32_t b_fmt_code, int band, int *watchdog) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;                                   // kStages x 16 KiB (1024-aligned)
@@ -140,125 +166,150 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint8_t *sSFA = sB + kStages * kBBytes;               // kStages x 512 B
     uint8_t *sSFB = sSFA + kStages * kSfaBytes;           // kStages x 512 B per 128 rows of B
 
-    __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], acc_bar;
+    __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], acc_full, acc_empty, drain_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int fail_flag;
     volatile int *fail_sh = &fail_flag;
-    int last_kb[kStages];                                 // producer: last K step armed per stage
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_blk = blockIdx.x, m_blk = blockIdx.y;
     const int num_kb = K / kBK;
+    const int tiles_n = N / BN, tiles_m = M / kBM;
+    const int n_tiles = tiles_m * tiles_n;
 
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
         for (int s = 0; s < kStages; s++) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-        mbar_init(&acc_bar, 1);
+        mbar_init(&acc_full, 1);
+        mbar_init(&acc_empty, kEpilogueWarps);
+        mbar_init(&drain_bar, 1);
         *fail_sh = 0;
         fence_barrier_init();
     }
-    if (warp == 5) tmem_alloc(&tmem_base_sh, kTmemCols);
+    if (warp == kMmaWarp) tmem_alloc(&tmem_base_sh, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_sh;
 
-    if (warp == 4) {
+    int last_it[kStages];                                 // producer: last ring use armed per stage
+    for (int s = 0; s < kStages; s++) last_it[s] = -1;
+    if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer
-        for (int s = 0; s < kStages; s++) last_kb[s] = -1;
         if (lane == 0) {
             const int64_t kb128 = K / 128;
-            for (int kb = 0; kb < num_kb; kb++) {
-                const int s = kb % kStages;
-                if (kb >= kStages) {
-                    if (!mbar_wait_bounded(&empty_bar[s], (uint32_t)((kb / kStages) - 1) & 1u, watchdog, WD_GEMM_EMPTY)) {
+            const uint32_t tx = kABytes + (b_fmt_code == 5u ? kBBytes / 2 : kBBytes) + kSfaBytes + kSfbBytes;
+            int it = 0;
+            for (int t = blockIdx.x; t < n_tiles && !*fail_sh; t += gridDim.x) {
+                int m_blk, n_blk;
+                tile_coords(t, tiles_m, tiles_n, band, m_blk, n_blk);
+                for (int kb = 0; kb < num_kb; kb++, it++) {
+                    const int s = it % kStages;
+                    if (it >= kStages &&
+                        !mbar_wait_bounded(&empty_bar[s], (uint32_t)((it / kStages) - 1) & 1u, watchdog, WD_GEMM_EMPTY)) {
                         *fail_sh = 1;
                         break;
                     }
-                }
-                if (*fail_sh) break;
-                // An E2M1 tile lands in shared memory padded to one byte per element
-                // (16U4_ALIGN16B), but the copy completes only the packed global bytes.
-                mbar_arrive_expect_tx(&full_bar[s], kABytes + (b_fmt_code == 5u ? kBBytes / 2 : kBBytes) +
-                                                        kSfaBytes + kSfbBytes);
-                tma_load_2d(sA + s * kABytes, &tmA, kb * kBK, m_blk * kBM, &full_bar[s]);
-                tma_load_2d(sB + s * kBBytes, &tmB, kb * kBK, n_blk * BN, &full_bar[s]);
-                bulk_load(sSFA + s * kSfaBytes, a_sc + ((int64_t)m_blk * kb128 + kb) * 512, kSfaBytes, &full_bar[s]);
+                    // An E2M1 tile lands in shared memory padded to one byte per element
+                    // (16U4_ALIGN16B), but the copy completes only the packed global bytes.
+                    mbar_arrive_expect_tx(&full_bar[s], tx);
+                    tma_load_2d(sA + s * kABytes, &tmA, kb * kBK, m_blk * kBM, &full_bar[s]);
+                    tma_load_2d(sB + s * kBBytes, &tmB, kb * kBK, n_blk * BN, &full_bar[s]);
+                    bulk_load(sSFA + s * kSfaBytes, a_sc + ((int64_t)m_blk * kb128 + kb) * 512, kSfaBytes, &full_bar[s]);
 #pragma unroll
-                for (int h = 0; h < BN / 128; h++)
-                    bulk_load(sSFB + s * kSfbBytes + h * 512,
-                              b_sc + ((int64_t)((BN / 128) * n_blk + h) * kb128 + kb) * 512, 512, &full_bar[s]);
-                last_kb[s] = kb;
+                    for (int h = 0; h < BN / 128; h++)
+                        bulk_load(sSFB + s * kSfbBytes + h * 512,
+                                  b_sc + ((int64_t)((BN / 128) * n_blk + h) * kb128 + kb) * 512, 512, &full_bar[s]);
+                    last_it[s] = it;
+                }
             }
         }
         __syncwarp();
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            for (int kb = 0; kb < num_kb; kb++) {
-                const int s = kb % kStages;
-                if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(kb / kStages) & 1u, watchdog, WD_GEMM_FULL)) {
+            int it = 0, i = 0;
+            for (int t = blockIdx.x; t < n_tiles && !*fail_sh; t += gridDim.x, i++) {
+                if (i > 0 && !mbar_wait_bounded(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
                     *fail_sh = 1;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sfb_t = tmem + kSfCol0 + s * kSfColsPerStage;
-                const uint32_t sfa_t = sfb_t + 8;
-                tc_cp_sf(sfa_t, smem_u32(sSFA + s * kSfaBytes));
+                for (int kb = 0; kb < num_kb; kb++, it++) {
+                    const int s = it % kStages;
+                    if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(it / kStages) & 1u, watchdog, WD_GEMM_FULL)) {
+                        *fail_sh = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfb_t = tmem + kSfCol0 + s * kSfColsPerStage;
+                    const uint32_t sfa_t = sfb_t + 8;
+                    tc_cp_sf(sfa_t, smem_u32(sSFA + s * kSfaBytes));
 #pragma unroll
-                for (int h = 0; h < BN / 128; h++) tc_cp_sf(sfb_t + 4 * h, smem_u32(sSFB + s * kSfbBytes + h * 512));
-                const uint32_t a_base = smem_u32(sA + s * kABytes);
-                const uint32_t b_base = smem_u32(sB + s * kBBytes);
+                    for (int h = 0; h < BN / 128; h++) tc_cp_sf(sfb_t + 4 * h, smem_u32(sSFB + s * kSfbBytes + h * 512));
+                    const uint32_t a_base = smem_u32(sA + s * kABytes);
+                    const uint32_t b_base = smem_u32(sB + s * kBBytes);
 #pragma unroll
-                for (int k = 0; k < kBK / 32; k++) {
-                    const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
-                    const uint64_t bd = smem_desc(b_base + k * 32, 16, 1024, 2);
-                    tc_mma_mx(tmem, ad, bd, mma_idesc<BN>(b_fmt_code, (uint32_t)k), sfa_t, sfb_t,
-                              (kb > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < kBK / 32; k++) {
+                        const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
+                        const uint64_t bd = smem_desc(b_base + k * 32, 16, 1024, 2);
+                        tc_mma_mx(tmem, ad, bd, mma_idesc<BN>(b_fmt_code, (uint32_t)k), sfa_t, sfb_t,
+                                  (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&empty_bar[s]);
                 }
-                tc_commit(&empty_bar[s]);
+                if (*fail_sh) break;
+                tc_commit(&acc_full);                     // the tile's accumulator is complete
             }
-            tc_commit(&acc_bar);   // completes when every MMA issued above has finished
+            tc_commit(&drain_bar);                        // completes once every MMA above has finished
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ epilogue (warps 0-3)
-        const bool ok = mbar_wait_bounded(&acc_bar, 0u, watchdog, WD_GEMM_ACC);
-        tc_fence_after();
-        if (ok && !*fail_sh) {
-            const int row = m_blk * kBM + warp * 32 + lane;
-            uint16_t *crow = C + (int64_t)row * N + (int64_t)n_blk * BN;
-            const uint32_t t_row = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll 1
-            for (int j = 0; j < BN / 32; j++) {
-                uint32_t r[32];
-                tmem_ld32(t_row + j * 32, r);
-                uint4 *dst = reinterpret_cast<uint4 *>(crow + j * 32);
+        // ------------------------------------------------ epilogue (warps 0-7)
+        // warp w reads TMEM lanes 32 (w % 4) .. + 31 (rows) and columns of half w / 4
+        constexpr int kHalf = BN / 2;
+        const int quad = warp & 3, half = warp >> 2;
+        const uint32_t t_base = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(half * kHalf);
+        int i = 0;
+        for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, i++) {
+            const bool ok = mbar_wait_bounded(&acc_full, (uint32_t)i & 1u, watchdog, WD_GEMM_ACC);
+            if (!ok || *fail_sh) { *fail_sh = 1; break; }
+            tc_fence_after();
+            uint32_t o[kHalf / 2];                        // the thread's row segment as bf16 pairs
 #pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    uint4 o;
-                    o.x = f32x2_to_bf16x2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]));
-                    o.y = f32x2_to_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]));
-                    o.z = f32x2_to_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]));
-                    o.w = f32x2_to_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]));
-                    dst[q] = o;
-                }
+            for (int j = 0; j < kHalf / 32; j++) {
+                uint32_t r[32];
+                tmem_ld32(t_base + j * 32, r);
+#pragma unroll
+                for (int q = 0; q < 16; q++)
+                    o[j * 16 + q] = f32x2_to_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty);       // accumulator may be overwritten now
+            int m_blk, n_blk;
+            tile_coords(t, tiles_m, tiles_n, band, m_blk, n_blk);
+            const int row = m_blk * kBM + quad * 32 + lane;
+            uint4 *dst = reinterpret_cast<uint4 *>(C + (int64_t)row * N + (int64_t)n_blk * BN + half * kHalf);
+            // evict-first stores: the output must not push operand panels out of L2
+#pragma unroll
+            for (int q = 0; q < kHalf / 8; q++) __stcs(dst + q, make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]));
         }
     }
 
+    // teardown: on the error path wait (bounded) for every copy this CTA armed and for
+    // every MMA it issued, so that no copy or MMA touches shared or tensor memory after
+    // they are released
+    __syncthreads();
+    if (*fail_sh && warp == kProducerWarp && lane == 0) {
+        for (int s = 0; s < kStages; s++)
+            if (last_it[s] >= 0)
+                (void)mbar_wait_bounded(&full_bar[s], (uint32_t)(last_it[s] / kStages) & 1u, nullptr, 0, kDrainLimitNs);
+    }
+    if (*fail_sh && warp == kMmaWarp && lane == 0) (void)mbar_wait_bounded(&drain_bar, 0u, nullptr, 0, kDrainLimitNs);
     tc_fence_before();
     __syncthreads();
-    if (*fail_sh && warp == 4 && lane == 0) {
-        // Error path: wait (bounded) for the loads this CTA armed, and for the MMAs it
-        // issued (the final commit above), before shared and tensor memory go away.
-        for (int s = 0; s < kStages; s++)
-            if (last_kb[s] >= 0) (void)mbar_wait_bounded(&full_bar[s], (uint32_t)(last_kb[s] / kStages) & 1u, nullptr, 0, kDrainLimitNs);
-        (void)mbar_wait_bounded(&acc_bar, 0u, nullptr, 0, kDrainLimitNs);
-    }
-    __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -285,7 +336,6 @@ static bool encode_operand(EncodeTiledFn enc, CUtensorMap *tm, const void *ptr, 
 cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, const void *b_elems, const uint8_t *b_sc,
                         int b_fmt, void *c, int64_t M, int64_t N, int64_t K, int *watchdog, int num_sms,
                         cudaStream_t st) {
-    (void)num_sms;
     auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
     if (!enc) return cudaErrorNotSupported;
     CUtensorMap tmA, tmB;
@@ -294,18 +344,24 @@ cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, const void *b_
     const bool wide = N % 256 == 0;
     const int bn = wide ? 256 : 128;
     if (!encode_operand(enc, &tmB, b_elems, N, K, fp4, (uint32_t)bn)) return cudaErrorInvalidValue;
-    const dim3 grid((unsigned)(N / bn), (unsigned)(M / kBM));
+    const int64_t n_tiles = (M / kBM) * (N / bn);
+    // band of N-tiles whose B panels (bn rows x K codes) take at most ~48 MB of L2
+    const int64_t panel = (int64_t)bn * (fp4 ? K / 2 : K);
+    int64_t band = (48ll << 20) / (panel > 0 ? panel : 1);
+    if (band < 1) band = 1;
+    if (band > N / bn) band = N / bn;
+    const dim3 grid((unsigned)(n_tiles < num_sms ? n_tiles : num_sms));
     cudaError_t e;
     if (wide) {
         e = cudaFuncSetAttribute(mx_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<256>::kSmemBytes);
         if (e != cudaSuccess) return e;
         mx_gemm_kernel<256><<<grid, kGemmThreads, Tile<256>::kSmemBytes, st>>>(
-            tmA, tmB, a_sc, b_sc, static_cast<uint16_t *>(c), (int)M, (int)N, (int)K, fp4 ? 5u : 0u, watchdog);
+            tmA, tmB, a_sc, b_sc, static_cast<uint16_t *>(c), (int)M, (int)N, (int)K, fp4 ? 5u : 0u, (int)band, watchdog);
     } else {
         e = cudaFuncSetAttribute(mx_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<128>::kSmemBytes);
         if (e != cudaSuccess) return e;
         mx_gemm_kernel<128><<<grid, kGemmThreads, Tile<128>::kSmemBytes, st>>>(
-            tmA, tmB, a_sc, b_sc, static_cast<uint16_t *>(c), (int)M, (int)N, (int)K, fp4 ? 5u : 0u, watchdog);
+            tmA, tmB, a_sc, b_sc, static_cast<uint16_t *>(c), (int)M, (int)N, (int)K, fp4 ? 5u : 0u, (int)band, watchdog);
     }
     return cudaGetLastError();
 }
