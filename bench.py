@@ -153,7 +153,7 @@ class WeightQuantStep:
         self.sn = torch.empty(R * C // 16, dtype=torch.uint8, device=dev)
         self.snt = torch.empty(mx.scale_bytes(R, C // 16, "tcgen05"), dtype=torch.uint8, device=dev)
         self.g = torch.empty(1, dtype=torch.float32, device=dev)
-        self.launches_per_step = 3      # MXFP4 quantiser; NVFP4 amax + quantiser (no padding at 4096)
+        self.launches_per_step = 2      # MXFP4 quantiser; fused NVFP4 kernel (no padding at 4096)
 
     def mxfp4(self, stream):
         L = self.L
@@ -329,8 +329,10 @@ def run_breakdown(mx, dev, pk):
     x1 = to_dev(synth.mx8_rowwise(), dev)
     xs = [x1.clone() for _ in range(64)]
     qs = [mx.quantize(x, "e4m3", "row", "ceil", layout="rowmajor") for x in xs]
-    tq = timed([lambda x=x: mx.quantize(x, "e4m3", "row", "ceil", layout="rowmajor") for x in xs], 256, stream)
-    td = timed([lambda q=q: mx.dequantize(q, "rowmajor") for q in qs], 256, stream)
+    ys = [torch.empty_like(x) for x in xs]
+    tq = timed([lambda x=x, q=q: mx.quantize(x, "e4m3", "row", "ceil", layout="rowmajor", out=q)
+                for x, q in zip(xs, qs)], 256, stream)
+    td = timed([lambda q=q, y=y: mx.dequantize(q, "rowmajor", out=y) for q, y in zip(qs, ys)], 256, stream)
     b1 = 1024 * 1024 * 2 + 1024 * 1024 + 1024 * 32
     out["c1_mxfp8_rowwise_1024"] = {"quantize_us": round(tq * 1e3, 2), "dequantize_us": round(td * 1e3, 2),
                                     "quantize_GBps": round(b1 / tq / 1e6, 1),
@@ -343,13 +345,14 @@ def run_breakdown(mx, dev, pk):
     xw = to_dev(synth.weight_fp4(), dev)
     q4 = [mx.quantize(xw, "e2m1", "row", "floor", layout="tcgen05") for _ in range(NROT)]
     qn = [mx.quantize(xw, "nvfp4", "row", "ceil", layout="tcgen05") for _ in range(NROT)]
-    t4 = timed([lambda q=q: mx.dequantize(q, "tcgen05") for q in q4], 64, stream)
-    tn = timed([lambda q=q: mx.dequantize(q, "tcgen05") for q in qn], 64, stream)
+    ys = [torch.empty_like(xw) for _ in range(NROT)]
+    t4 = timed([lambda q=q, y=y: mx.dequantize(q, "tcgen05", out=y) for q, y in zip(q4, ys)], 64, stream)
+    tn = timed([lambda q=q, y=y: mx.dequantize(q, "tcgen05", out=y) for q, y in zip(qn, ys)], 64, stream)
     bd4 = R2 * C2 // 2 + R2 * C2 // 32 + R2 * C2 * 2
     bdn = R2 * C2 // 2 + R2 * C2 // 16 + 4 + R2 * C2 * 2
     out["a7_dequantize_4096"] = {"mxfp4_GBps": round(bd4 / t4 / 1e6, 1), "mxfp4_frac_hbm": round(bd4 / t4 / 1e6 / hbm, 4),
                                  "nvfp4_GBps": round(bdn / tn / 1e6, 1), "nvfp4_frac_hbm": round(bdn / tn / 1e6 / hbm, 4)}
-    del xw, q4, qn
+    del xw, q4, qn, ys
 
     # C3: dual-orientation MXFP8, activations (E4M3) and gradients (E5M2), tcgen05 scales
     for name, gen, fmt in (("act_16384x4096_e4m3", synth.activations, "e4m3"),
@@ -358,12 +361,13 @@ def run_breakdown(mx, dev, pk):
         R, C = xb.shape
         x3 = to_dev(xb, dev)
         del xb
-        t = timed([lambda: mx.quantize_dual(x3, fmt, "ceil", "tcgen05")], 10, stream)
+        o3 = mx.quantize_dual(x3, fmt, "ceil", "tcgen05")
+        t = timed([lambda: mx.quantize_dual(x3, fmt, "ceil", "tcgen05", out=o3)], 20, stream)
         nbytes = R * C * 2 + 2 * (R * C + R * C // 32)
         out[f"c3_dual_{name}"] = {"ms": round(t, 4), "GBps": round(nbytes / t / 1e6, 1),
                                   "frac_hbm": round(nbytes / t / 1e6 / hbm, 4), "algorithmic_bytes": nbytes,
                                   "l2": "input larger than L2"}
-        del x3
+        del x3, o3
         torch.cuda.empty_cache()
 
     # C4 / C5: block-scaled matmuls (operands quantised outside the timing)
@@ -432,6 +436,51 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- one case
+def run_case(name, iters, dev):
+    """Run one workload's hot call `iters` times and nothing else (for profiler captures:
+    the launch list then holds only this case's kernels).  Prints the mean device time per
+    call, which under a profiler is not a benchmark number."""
+    import microscaling_precision_number_b200 as mx
+    stream = torch.cuda.current_stream()
+    if name == "weight4096":
+        st = WeightQuantStep(mx, to_dev(synth.weight_fp4(), dev))
+        fns = [lambda: (st.mxfp4(stream.cuda_stream), st.nvfp4(stream.cuda_stream))]
+    elif name == "mx8_1024":
+        x = to_dev(synth.mx8_rowwise(), dev)
+        q = mx.quantize(x, "e4m3", "row", "ceil", layout="rowmajor")
+        y = torch.empty_like(x)
+        fns = [lambda: (mx.quantize(x, "e4m3", "row", "ceil", layout="rowmajor", out=q),
+                        mx.dequantize(q, "rowmajor", out=y))]
+    elif name in ("dual_act", "dual_grad"):
+        gen, fmt = (synth.activations, "e4m3") if name == "dual_act" else (synth.gradients, "e5m2")
+        x = to_dev(gen(), dev)
+        o = mx.quantize_dual(x, fmt, "ceil", "tcgen05")
+        fns = [lambda: mx.quantize_dual(x, fmt, "ceil", "tcgen05", out=o)]
+    elif name == "dequant4096":
+        xw = to_dev(synth.weight_fp4(), dev)
+        q4 = mx.quantize(xw, "e2m1", "row", "floor", layout="tcgen05")
+        qn = mx.quantize(xw, "nvfp4", "row", "ceil", layout="tcgen05")
+        y = torch.empty_like(xw)
+        fns = [lambda: (mx.dequantize(q4, "tcgen05", out=y), mx.dequantize(qn, "tcgen05", out=y))]
+    elif name in ("gemm8192", "gemm_w4a8"):
+        (M, N, K), bfmt, bsig = (((8192, 8192, 8192), "e4m3", 1.0) if name == "gemm8192"
+                                 else ((8192, 14336, 4096), "e2m1", 0.02))
+        a = mx.quantize(to_dev(synth.normal(M, K, seed=40), dev), "e4m3", "row", "ceil", layout="tcgen05")
+        b = mx.quantize(to_dev(synth.normal(N, K, sigma=bsig, seed=41), dev), bfmt, "row",
+                        "floor" if bfmt == "e2m1" else "ceil", layout="tcgen05")
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        fns = [lambda: mx.gemm(a, b, c)]
+    else:
+        raise SystemExit(f"unknown case {name}")
+    t = timed(fns, iters, stream)
+    assert mx.watchdog_status() == 0
+    print(f"{name}: {iters} calls, {t * 1e3:.1f} us per call", flush=True)
+
+
+CASES = ["weight4096", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "gemm8192", "gemm_w4a8"]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -441,7 +490,14 @@ def main():
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--case", choices=CASES, help="run one workload's hot call only (profiling)")
+    ap.add_argument("--iters", type=int, default=3, help="calls for --case (one warm-up call before)")
     args = ap.parse_args()
+    if args.case:
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        run_case(args.case, args.iters, dev)
+        return
     if args.warmup < 3:
         args.warmup = 3
     rank = int(os.environ.get("RANK", "0"))

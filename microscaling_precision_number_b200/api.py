@@ -64,21 +64,32 @@ class Quantized(NamedTuple):
     fmt: int
 
 
+def _buf(out: Optional[torch.Tensor], n: int, dtype, dev, what: str) -> torch.Tensor:
+    """A caller-provided output (checked for size, type and device) or a new one."""
+    if out is None:
+        return torch.empty(n, dtype=dtype, device=dev)
+    if out.dtype != dtype or out.device != dev or not out.is_contiguous() or out.numel() < n:
+        raise ValueError(f"output buffer '{what}' must be a contiguous {dtype} tensor of >= {n} elements on {dev}")
+    return out
+
+
 def quantize(x: torch.Tensor, fmt="e4m3", axis: str = "row", rounding: str = "ceil",
-             layout: str = "rowmajor", stream=None) -> Quantized:
+             layout: str = "rowmajor", stream=None, out: Optional[Quantized] = None) -> Quantized:
+    """Block-scaled quantisation of a bf16 matrix.  `out` (a Quantized from an earlier
+    call with the same arguments) reuses its buffers instead of allocating new ones."""
     _check_src(x)
     f = _fmt(fmt)
     rows, cols = x.shape
     orows, ocols = (rows, cols) if axis == "row" else (cols, rows)
     B = block_of(f)
     dev = x.device
-    elems = torch.empty(elem_bytes(orows, ocols, f), dtype=torch.uint8, device=dev)
     lay = LAYOUTS[layout]
     first = "rowmajor" if layout in ("rowmajor", "both") else "tcgen05"
-    scales = torch.empty(scale_bytes(orows, ocols // B, first), dtype=torch.uint8, device=dev)
-    alt = torch.empty(scale_bytes(orows, ocols // B, "tcgen05"), dtype=torch.uint8, device=dev) \
+    elems = _buf(out and out.elems, elem_bytes(orows, ocols, f), torch.uint8, dev, "elems")
+    scales = _buf(out and out.scales, scale_bytes(orows, ocols // B, first), torch.uint8, dev, "scales")
+    alt = _buf(out and out.scales_alt, scale_bytes(orows, ocols // B, "tcgen05"), torch.uint8, dev, "scales_alt") \
         if layout == "both" else None
-    g = torch.empty(1, dtype=torch.float32, device=dev) if f == L.MX_FMT_NVFP4 else None
+    g = _buf(out and out.global_scale, 1, torch.float32, dev, "global_scale") if f == L.MX_FMT_NVFP4 else None
     st = L.lib.mx_quantize(x.data_ptr(), rows, cols, f, L.MX_AXIS_ROW if axis == "row" else L.MX_AXIS_COL,
                            ROUNDING[rounding], elems.data_ptr(), scales.data_ptr(), lay, _ptr(alt), _ptr(g),
                            _stream(stream))
@@ -86,25 +97,30 @@ def quantize(x: torch.Tensor, fmt="e4m3", axis: str = "row", rounding: str = "ce
     return Quantized(elems, scales, alt, g, orows, ocols, f)
 
 
-def quantize_dual(x: torch.Tensor, fmt="e4m3", rounding: str = "ceil", layout: str = "tcgen05", stream=None):
-    """Row-wise and column-wise (transposed) quantisation from one read of x."""
+def quantize_dual(x: torch.Tensor, fmt="e4m3", rounding: str = "ceil", layout: str = "tcgen05", stream=None,
+                  out: Optional[tuple] = None):
+    """Row-wise and column-wise (transposed) quantisation from one read of x.  `out` (the
+    pair returned by an earlier call with the same arguments) reuses its buffers."""
     _check_src(x)
     f = _fmt(fmt)
     rows, cols = x.shape
     dev = x.device
-    re = torch.empty(elem_bytes(rows, cols, f), dtype=torch.uint8, device=dev)
-    ce = torch.empty(elem_bytes(rows, cols, f), dtype=torch.uint8, device=dev)
-    rs = torch.empty(scale_bytes(rows, cols // 32, layout), dtype=torch.uint8, device=dev)
-    cs = torch.empty(scale_bytes(cols, rows // 32, layout), dtype=torch.uint8, device=dev)
+    o_r, o_c = out if out is not None else (None, None)
+    re = _buf(o_r and o_r.elems, elem_bytes(rows, cols, f), torch.uint8, dev, "row elems")
+    ce = _buf(o_c and o_c.elems, elem_bytes(rows, cols, f), torch.uint8, dev, "col elems")
+    rs = _buf(o_r and o_r.scales, scale_bytes(rows, cols // 32, layout), torch.uint8, dev, "row scales")
+    cs = _buf(o_c and o_c.scales, scale_bytes(cols, rows // 32, layout), torch.uint8, dev, "col scales")
     st = L.lib.mx_quantize_dual(x.data_ptr(), rows, cols, f, ROUNDING[rounding], re.data_ptr(), rs.data_ptr(),
                                 ce.data_ptr(), cs.data_ptr(), LAYOUTS[layout], _stream(stream))
     L.check(st, "mx_quantize_dual")
     return (Quantized(re, rs, None, None, rows, cols, f), Quantized(ce, cs, None, None, cols, rows, f))
 
 
-def dequantize(q: Quantized, layout: str = "rowmajor", stream=None) -> torch.Tensor:
+def dequantize(q: Quantized, layout: str = "rowmajor", stream=None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Codes and scales back to a (rows, cols) bf16 matrix (into `out` when given)."""
     scales = q.scales if (layout == "rowmajor" or q.scales_alt is None) else q.scales_alt
-    out = torch.empty((q.rows, q.cols), dtype=torch.bfloat16, device=q.elems.device)
+    out = _buf(out, q.rows * q.cols, torch.bfloat16, q.elems.device, "out").reshape(-1)[:q.rows * q.cols] \
+        .view(q.rows, q.cols) if out is not None else torch.empty((q.rows, q.cols), dtype=torch.bfloat16, device=q.elems.device)
     st = L.lib.mx_dequantize(q.elems.data_ptr(), scales.data_ptr(), _ptr(q.global_scale), q.rows, q.cols, q.fmt,
                              LAYOUTS[layout], out.data_ptr(), _stream(stream))
     L.check(st, "mx_dequantize")

@@ -31,7 +31,7 @@ __host__ __device__ constexpr int max_sig128(int fmt) { return fmt == FMT_E2M1 ?
 // magnitude >= 0x7F80 (Inf or NaN) yields the NaN scale 0xFF.  A zero block yields
 // s = -127 (code 0).  The exponent is clamped to [-127, 127].
 template <int FMT, bool CEIL>
-__device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t a) {
+__device__ __noinline__ uint32_t e8m0_from_amax_bits_rare(uint32_t a) {
     if (a >= 0x7F80u) return 0xFFu;
     if (a == 0u) return 0u;
     int ef = (int)(a >> 7), mant = (int)(a & 0x7Fu);
@@ -48,6 +48,19 @@ __device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t a) {
     if (CEIL && nm > max_sig128(FMT)) s += 1;   // floor rule would clip: one binade up
     s = s < -127 ? -127 : (s > 127 ? 127 : s);
     return (uint32_t)(s + 127);
+}
+
+// Common case, a normal block maximum (0x80 <= a < 0x7F80): the code is the biased
+// exponent field minus emax_elem (plus one under the no-clip rule when the maximum's
+// significand exceeds the element format's largest), floored at 0.  It never exceeds
+// 253, so e8m0_inverse_multiplier's first branch applies.  Zero, subnormal and Inf/NaN
+// maxima take the general path above (the two agree on every normal a).
+template <int FMT, bool CEIL>
+__device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t a) {
+    if (__builtin_expect(a - 0x80u >= 0x7F00u, 0)) return e8m0_from_amax_bits_rare<FMT, CEIL>(a);
+    int code = (int)(a >> 7) - emax_elem(FMT);
+    if (CEIL) code += (int)((a & 0x7Fu) > (uint32_t)(max_sig128(FMT) - 128));
+    return (uint32_t)(code < 0 ? 0 : code);
 }
 
 // fp32 value 2^-(code-127), the multiplier that brings a block into the element range.

@@ -1,5 +1,5 @@
 // dual.cu -- TMA-staged MX quantiser that reads each bf16 element once and writes the
-// row-wise copy, the column-wise (transposed) copy, or both.
+// column-wise (transposed) copy, alone or together with the row-wise copy.
 //
 // Sources (page title, section):
 //   "MXFP4 と NVFP4 は何が違うのか調べてみた"
@@ -8,170 +8,280 @@
 //     §6 "DeepSeek-V4 の入れ子構造": training uses the weight both as is and transposed;
 //        quantising both orientations from one read avoids re-quantising a transposed copy.
 //
-// Design: persistent CTAs (a multiple of the SM count) walk 32-row x 128-column bf16
-// tiles.  One thread streams tiles into a 4-deep shared-memory ring with 2-D TMA loads
-// (each stage completes an mbarrier); all 256 threads then
-//   - row pass: four lanes per 32-element row block (16-byte shared loads, xor-shuffle
-//     maximum), contiguous 8-byte code stores;
-//   - column pass: two threads per column (16 rows each, maxima exchanged through shared
-//     memory), each writing 16 contiguous codes of the transposed output.
-// Every barrier wait is bounded (watchdog); on a timeout the CTA drains its own TMA loads
-// (bounded) and returns.
+// Design:
+//   - persistent CTAs, two per SM, walk 32-row x 256-column bf16 tiles.  A producer warp
+//     loads each tile as four 32 x 64 boxes (2-D TMA, 128-byte swizzle) into a 6-stage
+//     ring guarded by full / empty mbarriers;
+//   - warp specialisation over the same stage: warps 0-3 run the column pass (one warp
+//     per box, one lane per column pair, 32-bit shared loads), warps 4-7 the row pass (one
+//     lane per 32-element row block, four 16-byte shared loads).  The swizzle makes both
+//     access patterns bank-conflict free.  With only the column output requested, warps
+//     4-7 run the column pass too, on alternate tiles;
+//   - block maxima with the packed bf16 |max| instruction (the column pass reduces two
+//     columns per instruction), scales by the same exponent arithmetic as every other
+//     quantiser, products as packed fp32 pairs, codes by cvt.rn.satfinite;
+//   - each lane writes whole 32-byte sectors (one 256-bit store per FP8 block when the
+//     output is 32-byte aligned).
+// Every barrier wait is bounded (watchdog); the producer drains its own loads before the
+// CTA exits, whatever happened.
 #include <cuda.h>
 #include "codec.cuh"
 #include "internal.h"
 #include "ptx.cuh"
+#include "tiling.cuh"
 
 namespace mxk {
 
 namespace {
-constexpr int kDualThreads = 256;
-constexpr int kTileR = 32, kTileC = 128;
-constexpr int kTileBytes = kTileR * kTileC * 2;   // 8 KiB of bf16
-constexpr int kStages = 4;
+constexpr int kBoxC = 64;                            // bf16 columns per box = one 128-byte swizzle row
+constexpr int kBoxes = 4;
+constexpr int kTileR = 32, kTileC = kBoxC * kBoxes;  // 32 x 256 tile
+constexpr int kBoxBytes = kTileR * kBoxC * 2;        // 4 KiB
+constexpr int kTileBytes = kBoxBytes * kBoxes;       // 16 KiB
+constexpr int kStages = 6;
+constexpr int kProducerWarp = 8;
+constexpr int kDualThreads = 32 * (kProducerWarp + 1);
+constexpr int kCtasPerSm = 2;
+constexpr size_t kDualSmem = (size_t)kStages * kTileBytes + 1024;   // + alignment to 1024
 }  // namespace
 
-template <int FMT, bool CEIL, bool ROW, bool COL, bool TC>
-__global__ void __launch_bounds__(kDualThreads)
-quant_dual_kernel(const __grid_constant__ CUtensorMap tmap, int64_t rows, int64_t cols,
-                  uint8_t *__restrict__ row_elems, uint8_t *__restrict__ row_sc,
-                  uint8_t *__restrict__ col_elems, uint8_t *__restrict__ col_sc, int *watchdog) {
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-    __shared__ __align__(8) uint64_t full_bar[kStages];
-    __shared__ uint32_t s_amax[kDualThreads];
+// 32 bytes at p (w, or zeros when `zero`): one 256-bit store when p is 32-byte aligned,
+// else two 16-byte stores.  The rare zero case is a separate store, not a per-word select.
+__device__ __forceinline__ void store32(uint8_t *p, const uint32_t (&w)[8], bool v8, bool zero) {
+    if (__builtin_expect(zero, 0)) {
+        reinterpret_cast<uint4 *>(p)[0] = make_uint4(0u, 0u, 0u, 0u);
+        reinterpret_cast<uint4 *>(p)[1] = make_uint4(0u, 0u, 0u, 0u);
+    } else if (v8) {
+        asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                     ::"l"(p), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+                     : "memory");
+    } else {
+        reinterpret_cast<uint4 *>(p)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        reinterpret_cast<uint4 *>(p)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+}
 
-    const int tid = threadIdx.x;
-    const int lane = tid & 31;
-    const int64_t tiles_c = (cols + kTileC - 1) / kTileC;
-    const int64_t n_tiles = tiles_c * (rows / kTileR);
-    const int64_t row_S = cols / 32, col_S = rows / 32;
+// Tile order: bands of kBand column tiles, row-tile major inside a band, so that the tiles
+// in flight at any moment span many rows of few columns.  The transposed output of a
+// column then grows by long contiguous runs (and the row-wise output by kBand x 256-byte
+// runs) instead of 32-byte pieces scattered over every column of the matrix.
+constexpr uint32_t kBand = 4;
+struct TileOrder {
+    FastDiv band_tiles;     // tiles per full band (tiles_r * kBand)
+    uint32_t n_full;        // tiles in the full bands
+    FastDiv last_w;         // width of the last, narrower band (tiles_c % kBand), if any
+    uint32_t last_c0;       // its first column tile
+};
 
-    if (tid == 0) {
+__device__ __forceinline__ void tile_coords(uint32_t t, const TileOrder &o, uint32_t &tr, uint32_t &tcl) {
+    if (t < o.n_full) {
+        const uint32_t b = fdiv(t, o.band_tiles), in = t - b * o.band_tiles.d;
+        tr = in / kBand;
+        tcl = b * kBand + in % kBand;
+    } else {
+        const uint32_t in = t - o.n_full;
+        tr = fdiv(in, o.last_w);
+        tcl = o.last_c0 + (in - tr * o.last_w.d);
+    }
+}
+
+// Byte offset of a swizzled 16-byte chunk: row r (128 bytes) of a 1024-byte-aligned box,
+// logical chunk c; the 128-byte swizzle stores it at chunk c ^ (r % 8).
+__device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c) { return r * 128u + ((c ^ (r & 7u)) << 4); }
+
+// Column pass: columns col, col + 1 (box-relative pair q) over the tile's 32 rows.
+template <int FMT, bool CEIL, bool TC>
+__device__ __forceinline__ void column_pair(const uint8_t *box, uint32_t q, uint32_t col, uint32_t rows,
+                                            uint32_t r0, uint32_t tr, uint8_t *__restrict__ col_elems,
+                                            uint8_t *__restrict__ col_sc, uint32_t sc_dim, bool v8) {
+    uint32_t w[32];                                      // row r: bf16 of col (low) and col + 1 (high)
+#pragma unroll
+    for (int r = 0; r < 32; r++)
+        w[r] = *reinterpret_cast<const uint32_t *>(box + swz(r, q >> 2) + ((q & 3u) << 2));
+    uint32_t m[16];
+#pragma unroll
+    for (int i = 0; i < 16; i++) m[i] = absmax_bf16x2(w[2 * i], w[2 * i + 1]);
+#pragma unroll
+    for (int n = 8; n >= 1; n >>= 1)
+#pragma unroll
+        for (int i = 0; i < n; i++) m[i] = absmax_bf16x2(m[i], m[i + n]);
+    const uint32_t code_lo = e8m0_from_amax_bits<FMT, CEIL>(m[0] & 0x7FFFu);
+    const uint32_t code_hi = e8m0_from_amax_bits<FMT, CEIL>((m[0] >> 16) & 0x7FFFu);
+    const uint64_t s_lo = splat2(e8m0_inverse_multiplier(code_lo));
+    const uint64_t s_hi = splat2(e8m0_inverse_multiplier(code_hi));
+    const uint64_t e0 = (uint64_t)col * rows + r0;       // first element of column col in the output
+
+    if constexpr (FMT == FMT_E2M1) {
+        uint32_t o_lo[4], o_hi[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {                    // rows 8k .. 8k + 7
+            float x[8], y[8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const uint32_t a = w[8 * k + 2 * i], b = w[8 * k + 2 * i + 1];
+                unpack2(mul2(pack2(__uint_as_float(a << 16), __uint_as_float(b << 16)), s_lo), x[2 * i], x[2 * i + 1]);
+                unpack2(mul2(pack2(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(b & 0xFFFF0000u)), s_hi),
+                        y[2 * i], y[2 * i + 1]);
+            }
+            o_lo[k] = cvt_e2m1x8(x);
+            o_hi[k] = cvt_e2m1x8(y);
+        }
+        // a NaN scale makes the whole block NaN: its codes are stored as 0
+        uint4 *p = reinterpret_cast<uint4 *>(col_elems + (e0 >> 1));
+        p[0] = code_lo == 0xFFu ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(o_lo[0], o_lo[1], o_lo[2], o_lo[3]);
+        p[rows >> 5] = code_hi == 0xFFu ? make_uint4(0u, 0u, 0u, 0u)     // next column: rows / 2 bytes on
+                                        : make_uint4(o_hi[0], o_hi[1], o_hi[2], o_hi[3]);
+    } else {
+        uint32_t o_lo[8], o_hi[8];
+#pragma unroll
+        for (int i = 0; i < 16; i++) {                   // rows 2i, 2i + 1
+            const uint32_t a = w[2 * i], b = w[2 * i + 1];
+            float x0, x1, y0, y1;
+            unpack2(mul2(pack2(__uint_as_float(a << 16), __uint_as_float(b << 16)), s_lo), x0, x1);
+            unpack2(mul2(pack2(__uint_as_float(a & 0xFFFF0000u), __uint_as_float(b & 0xFFFF0000u)), s_hi), y0, y1);
+            const uint32_t cl = cvt_fp8x2<FMT>(x0, x1), ch = cvt_fp8x2<FMT>(y0, y1);
+            if (i & 1) { o_lo[i >> 1] |= cl << 16; o_hi[i >> 1] |= ch << 16; }
+            else       { o_lo[i >> 1] = cl;        o_hi[i >> 1] = ch; }
+        }
+        store32(col_elems + e0, o_lo, v8, code_lo == 0xFFu);         // NaN scale: codes 0
+        store32(col_elems + e0 + rows, o_hi, v8, code_hi == 0xFFu);
+    }
+    if constexpr (TC) {
+        col_sc[tc_offset(col, tr, sc_dim)] = (uint8_t)code_lo;
+        col_sc[tc_offset(col + 1, tr, sc_dim)] = (uint8_t)code_hi;
+    } else {
+        col_sc[(uint64_t)col * sc_dim + tr] = (uint8_t)code_lo;
+        col_sc[(uint64_t)(col + 1) * sc_dim + tr] = (uint8_t)code_hi;
+    }
+}
+
+// Row pass: the 32-element block of tile row r starting at box-relative chunk 4h.
+template <int FMT, bool CEIL, bool TC>
+__device__ __forceinline__ void row_block(const uint8_t *box, uint32_t r, uint32_t h, uint32_t col, uint32_t cols,
+                                          uint32_t R, uint8_t *__restrict__ row_elems,
+                                          uint8_t *__restrict__ row_sc, uint32_t sc_dim, bool v8) {
+    uint4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; k++) v[k] = *reinterpret_cast<const uint4 *>(box + swz(r, 4u * h + k));
+    uint32_t m[8];
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        m[2 * k] = absmax_bf16x2(v[k].x, v[k].y);
+        m[2 * k + 1] = absmax_bf16x2(v[k].z, v[k].w);
+    }
+#pragma unroll
+    for (int n = 4; n >= 1; n >>= 1)
+#pragma unroll
+        for (int i = 0; i < n; i++) m[i] = absmax_bf16x2(m[i], m[i + n]);
+    const uint32_t code = e8m0_from_amax_bits<FMT, CEIL>(max(m[0] & 0x7FFFu, (m[0] >> 16) & 0x7FFFu));
+    const uint64_t s2 = splat2(e8m0_inverse_multiplier(code));
+    const uint64_t e0 = (uint64_t)R * cols + col;
+
+    if constexpr (FMT == FMT_E2M1) {
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            float x[8];
+            scale8(v[k], s2, x);
+            o[k] = cvt_e2m1x8(x);
+        }
+        *reinterpret_cast<uint4 *>(row_elems + (e0 >> 1)) =
+            code == 0xFFu ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(o[0], o[1], o[2], o[3]);   // NaN scale: codes 0
+    } else {
+        uint32_t o[8];
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            float x[8];
+            scale8(v[k], s2, x);
+            const uint2 q = cvt_fp8x8<FMT>(x);
+            o[2 * k] = q.x;
+            o[2 * k + 1] = q.y;
+        }
+        store32(row_elems + e0, o, v8, code == 0xFFu);                  // NaN scale: codes 0
+    }
+    if constexpr (TC) row_sc[tc_offset(R, col >> 5, sc_dim)] = (uint8_t)code;
+    else row_sc[(uint64_t)R * sc_dim + (col >> 5)] = (uint8_t)code;
+}
+
+// ROW: also write the row-wise output.  sc_dim_*: scales per row (row-major layout) or
+// 4-column atom count (tcgen05 layout) of the row-wise / column-wise scale array.
+template <int FMT, bool CEIL, bool ROW, bool TC>
+__global__ void __launch_bounds__(kDualThreads, kCtasPerSm)
+quant_dual_kernel(const __grid_constant__ CUtensorMap tmap, uint32_t rows, uint32_t cols, uint32_t n_tiles,
+                  TileOrder order, uint8_t *__restrict__ row_elems, uint8_t *__restrict__ row_sc,
+                  uint32_t row_sc_dim, uint8_t *__restrict__ col_elems, uint8_t *__restrict__ col_sc,
+                  uint32_t col_sc_dim, int v8, int *watchdog) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+
+    const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t G = gridDim.x;
+    if (threadIdx.x == 0) {
         prefetch_tensormap(&tmap);
-        for (int s = 0; s < kStages; s++) mbar_init(&full_bar[s], 1);
+        for (int s = 0; s < kStages; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], ROW ? 8 : 4);          // consumer warps per tile
+        }
         fence_barrier_init();
     }
     __syncthreads();
 
-    auto issue = [&](int64_t t, int s) {
-        const int64_t tr = t / tiles_c, tcl = t - tr * tiles_c;
-        mbar_arrive_expect_tx(&full_bar[s], kTileBytes);
-        tma_load_2d(smem + s * kTileBytes, &tmap, (int32_t)(tcl * kTileC), (int32_t)(tr * kTileR), &full_bar[s]);
-    };
-    if (tid == 0)
-        for (int s = 0; s < kStages; s++) {
-            const int64_t t = blockIdx.x + (int64_t)s * gridDim.x;
-            if (t < n_tiles) issue(t, s);
-        }
-
-    int it = 0;
-    bool failed = false;
-    for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
-        const int s = it % kStages;
-        const uint32_t phase = (uint32_t)(it / kStages) & 1u;
-        const bool ok = mbar_wait_bounded(&full_bar[s], phase, watchdog, WD_DUAL_FULL);
-        if (__syncthreads_or(!ok)) { failed = true; break; }
-
-        const uint8_t *tile = smem + s * kTileBytes;
-        const int64_t tr = t / tiles_c, tcl = t - tr * tiles_c;
-        const int64_t r0 = tr * kTileR, c0 = tcl * kTileC;
-
-        if constexpr (ROW) {
+    uint32_t issued = 0;
+    if (warp == kProducerWarp) {
+        if (lane == 0) {
+            for (uint32_t t = blockIdx.x; t < n_tiles; t += G, ++issued) {
+                const uint32_t s = issued % kStages;
+                if (issued >= kStages &&
+                    !mbar_wait_bounded(&empty[s], (issued / kStages - 1) & 1u, watchdog, WD_DUAL_EMPTY))
+                    break;
+                uint32_t tr, tcl;
+                tile_coords(t, order, tr, tcl);
+                mbar_arrive_expect_tx(&full[s], kTileBytes);
 #pragma unroll
-            for (int k = 0; k < 2; k++) {
-                const int j = tid + k * kDualThreads;       // 16-byte chunk within the tile
-                const int rr = j >> 4, c8 = j & 15;
-                const uint4 v = *reinterpret_cast<const uint4 *>(tile + rr * (kTileC * 2) + c8 * 16);
-                uint32_t m = hmax(abs_max_bf16x8(v));
-                m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
-                m = max(m, __shfl_xor_sync(0xffffffffu, m, 2));
-                const int64_t col = c0 + c8 * 8;
+                for (int j = 0; j < kBoxes; j++)
+                    tma_load_2d(smem + s * kTileBytes + j * kBoxBytes, &tmap, (int32_t)(tcl * kTileC + j * kBoxC),
+                                (int32_t)(tr * kTileR), &full[s]);
+            }
+        }
+    } else {
+        const uint32_t grp = warp >> 2, j = warp & 3;    // warp group, box
+        const bool row_pass = ROW && grp == 1;
+        uint32_t it = 0;
+        for (uint32_t t = blockIdx.x; t < n_tiles; t += G, ++it) {
+            if (!ROW && (it & 1u) != grp) continue;       // column-only: groups alternate tiles
+            const uint32_t s = it % kStages;
+            const bool ok = mbar_wait_bounded(&full[s], (it / kStages) & 1u, watchdog, WD_DUAL_FULL);
+            if (!__all_sync(0xFFFFFFFFu, ok)) break;
+            uint32_t tr, tcl;
+            tile_coords(t, order, tr, tcl);
+            const uint32_t r0 = tr * kTileR, c0 = tcl * kTileC + j * kBoxC;
+            const uint8_t *box = smem + s * kTileBytes + j * kBoxBytes;
+            if (row_pass) {
+                const uint32_t h = lane & 1u, col = c0 + 32u * h;
                 if (col < cols) {
-                    const uint32_t code = e8m0_from_amax_bits<FMT, CEIL>(m);
-                    const float mul = e8m0_inverse_multiplier(code);
-                    float x[8];
-                    x[0] = __fmul_rn(bf16_lo(v.x), mul); x[1] = __fmul_rn(bf16_hi(v.x), mul);
-                    x[2] = __fmul_rn(bf16_lo(v.y), mul); x[3] = __fmul_rn(bf16_hi(v.y), mul);
-                    x[4] = __fmul_rn(bf16_lo(v.z), mul); x[5] = __fmul_rn(bf16_hi(v.z), mul);
-                    x[6] = __fmul_rn(bf16_lo(v.w), mul); x[7] = __fmul_rn(bf16_hi(v.w), mul);
-                    const int64_t e = (r0 + rr) * cols + col;          // element index, multiple of 8
-                    if constexpr (FMT == FMT_E2M1) {
-                        uint32_t q = cvt_e2m1x8(x);
-                        if (code == 0xFFu) q = 0u;
-                        reinterpret_cast<uint32_t *>(row_elems)[e >> 3] = q;
-                    } else {
-                        uint2 q = cvt_fp8x8<FMT>(x);
-                        if (code == 0xFFu) q = make_uint2(0u, 0u);
-                        reinterpret_cast<uint2 *>(row_elems)[e >> 3] = q;
-                    }
-                    if ((lane & 3) == 0) {
-                        const int64_t R = r0 + rr, b = col >> 5;
-                        if constexpr (TC) row_sc[tcgen05_scale_offset(R, b, row_S)] = (uint8_t)code;
-                        else row_sc[R * row_S + b] = (uint8_t)code;
-                    }
+                    row_block<FMT, CEIL, TC>(box, lane >> 1, h, col, cols, r0 + (lane >> 1), row_elems, row_sc,
+                                             row_sc_dim, v8 != 0);
+                    row_block<FMT, CEIL, TC>(box, 16 + (lane >> 1), h, col, cols, r0 + 16 + (lane >> 1), row_elems,
+                                             row_sc, row_sc_dim, v8 != 0);
                 }
+            } else {
+                const uint32_t col = c0 + 2u * lane;
+                if (col < cols)
+                    column_pair<FMT, CEIL, TC>(box, lane, col, rows, r0, tr, col_elems, col_sc, col_sc_dim, v8 != 0);
             }
-        }
-
-        if constexpr (COL) {
-            const int c = tid & (kTileC - 1), h = tid >> 7;     // column, 16-row half
-            uint32_t w[8];                                       // 16 bf16, two per word
-            uint32_t m = 0;
-#pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const uint32_t lo = *reinterpret_cast<const uint16_t *>(tile + (16 * h + 2 * i) * (kTileC * 2) + c * 2);
-                const uint32_t hi = *reinterpret_cast<const uint16_t *>(tile + (16 * h + 2 * i + 1) * (kTileC * 2) + c * 2);
-                w[i] = lo | (hi << 16);
-                m = max(m, max(lo & 0x7FFFu, hi & 0x7FFFu));
-            }
-            s_amax[tid] = m;
-            __syncthreads();
-            m = max(s_amax[c], s_amax[c + kTileC]);
-            const int64_t col = c0 + c;
-            if (col < cols) {
-                const uint32_t code = e8m0_from_amax_bits<FMT, CEIL>(m);
-                const float mul = e8m0_inverse_multiplier(code);
-                float x0[8], x1[8];
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    x0[2 * i] = __fmul_rn(bf16_lo(w[i]), mul);
-                    x0[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), mul);
-                    x1[2 * i] = __fmul_rn(bf16_lo(w[i + 4]), mul);
-                    x1[2 * i + 1] = __fmul_rn(bf16_hi(w[i + 4]), mul);
-                }
-                const int64_t e = col * rows + r0 + 16 * h;        // element index, multiple of 16
-                if constexpr (FMT == FMT_E2M1) {
-                    uint2 q = make_uint2(cvt_e2m1x8(x0), cvt_e2m1x8(x1));
-                    if (code == 0xFFu) q = make_uint2(0u, 0u);
-                    reinterpret_cast<uint2 *>(col_elems)[e >> 4] = q;
-                } else {
-                    const uint2 qa = cvt_fp8x8<FMT>(x0), qb = cvt_fp8x8<FMT>(x1);
-                    uint4 q = make_uint4(qa.x, qa.y, qb.x, qb.y);
-                    if (code == 0xFFu) q = make_uint4(0u, 0u, 0u, 0u);
-                    reinterpret_cast<uint4 *>(col_elems)[e >> 4] = q;
-                }
-                if (h == 0) {
-                    if constexpr (TC) col_sc[tcgen05_scale_offset(col, tr, col_S)] = (uint8_t)code;
-                    else col_sc[col * col_S + tr] = (uint8_t)code;
-                }
-            }
-        }
-
-        __syncthreads();   // stage s and s_amax are free again
-        if (tid == 0) {
-            const int64_t tn = t + (int64_t)kStages * gridDim.x;
-            if (tn < n_tiles) issue(tn, s);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
         }
     }
-
-    if (failed && tid == 0) {
-        // Drain: wait (bounded) for the loads this CTA still has in flight.
-        for (int k = 0; k < kStages; k++) {
-            const int j = it + k;
-            const int64_t t = blockIdx.x + (int64_t)j * gridDim.x;
-            if (t >= n_tiles) break;
-            (void)mbar_wait_bounded(&full_bar[j % kStages], (uint32_t)(j / kStages) & 1u, nullptr, 0, kDrainLimitNs);
+    __syncthreads();
+    if (warp == kProducerWarp && lane == 0) {
+        // Wait (bounded, short) for the last load issued into each stage.  On the normal
+        // path every one of them has been consumed and this returns at once; after a
+        // timeout it keeps the CTA alive until its own copies have landed.
+        for (uint32_t s = 0; s < kStages && s < issued; s++) {
+            const uint32_t last = s + ((issued - 1 - s) / kStages) * kStages;
+            (void)mbar_wait_bounded(&full[s], (last / kStages) & 1u, nullptr, 0, kDrainLimitNs);
         }
     }
 }
@@ -181,47 +291,71 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                   CUtensorMapFloatOOBfill);
 
+template <int FMT, bool CEIL, bool ROW, bool TC>
+static cudaError_t launch_dual_k(const CUtensorMap &tm, int grid, uint32_t rows, uint32_t cols, uint32_t n_tiles,
+                                 TileOrder order, uint8_t *re, uint8_t *rs, uint32_t rdim, uint8_t *ce, uint8_t *cs,
+                                 uint32_t cdim, int v8, int *wd, cudaStream_t st) {
+    auto k = quant_dual_kernel<FMT, CEIL, ROW, TC>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDualSmem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kDualThreads, kDualSmem, st>>>(tm, rows, cols, n_tiles, order, re, rs, rdim, ce, cs, cdim, v8, wd);
+    return cudaGetLastError();
+}
+
 template <int FMT, bool CEIL>
-static void launch_dual_t(const CUtensorMap &tm, int grid, size_t smem, int64_t rows, int64_t cols,
-                          uint8_t *re, uint8_t *rs, uint8_t *ce, uint8_t *cs, bool tc, int *wd,
-                          cudaStream_t st) {
-#define MXK_DUAL(R, C, T) quant_dual_kernel<FMT, CEIL, R, C, T><<<grid, kDualThreads, smem, st>>>(tm, rows, cols, re, rs, ce, cs, wd)
-    const bool row = re != nullptr, col = ce != nullptr;
-    if (row && col) { if (tc) MXK_DUAL(true, true, true); else MXK_DUAL(true, true, false); }
-    else if (row)   { if (tc) MXK_DUAL(true, false, true); else MXK_DUAL(true, false, false); }
-    else            { if (tc) MXK_DUAL(false, true, true); else MXK_DUAL(false, true, false); }
-#undef MXK_DUAL
+static cudaError_t launch_dual_t(bool row, bool tc, const CUtensorMap &tm, int grid, uint32_t rows, uint32_t cols,
+                                 uint32_t n_tiles, TileOrder d, uint8_t *re, uint8_t *rs, uint32_t rdim, uint8_t *ce,
+                                 uint8_t *cs, uint32_t cdim, int v8, int *wd, cudaStream_t st) {
+    if (row)
+        return tc ? launch_dual_k<FMT, CEIL, true, true>(tm, grid, rows, cols, n_tiles, d, re, rs, rdim, ce, cs, cdim, v8, wd, st)
+                  : launch_dual_k<FMT, CEIL, true, false>(tm, grid, rows, cols, n_tiles, d, re, rs, rdim, ce, cs, cdim, v8, wd, st);
+    return tc ? launch_dual_k<FMT, CEIL, false, true>(tm, grid, rows, cols, n_tiles, d, re, rs, rdim, ce, cs, cdim, v8, wd, st)
+              : launch_dual_k<FMT, CEIL, false, false>(tm, grid, rows, cols, n_tiles, d, re, rs, rdim, ce, cs, cdim, v8, wd, st);
 }
 
 cudaError_t launch_quant_dual(const void *src, int64_t rows, int64_t cols, int fmt, bool ceil,
                               void *row_elems, uint8_t *row_sc, void *col_elems, uint8_t *col_sc,
                               bool tc, int *watchdog, int num_sms, cudaStream_t st) {
+    // Preconditions (checked by the caller): rows % 32 == 0, cols % 8 == 0 (cols % 32 == 0
+    // with the row-wise output), 16-byte aligned source and outputs, column output present.
+    if (!col_elems || !col_sc) return cudaErrorInvalidValue;
+    const bool row = row_elems != nullptr;
+    if (row && !row_sc) return cudaErrorInvalidValue;
     auto encode = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
     if (!encode) return cudaErrorNotSupported;
     CUtensorMap tm;
     const cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
     const cuuint64_t gstride[1] = {(cuuint64_t)cols * 2};
-    const cuuint32_t box[2] = {kTileC, kTileR};
+    const cuuint32_t box[2] = {kBoxC, kTileR};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = encode(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(src), gdim, gstride, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    const int64_t n_tiles = ((cols + kTileC - 1) / kTileC) * (rows / kTileR);
-    int64_t grid = (int64_t)num_sms * 4;
-    if (grid > n_tiles) grid = n_tiles;
-    const size_t smem = (size_t)kStages * kTileBytes + 128;
+    const uint32_t tiles_c = (uint32_t)((cols + kTileC - 1) / kTileC);
+    const uint32_t n_tiles = tiles_c * (uint32_t)(rows / kTileR);
+    const int grid = (int)(n_tiles < (uint32_t)(kCtasPerSm * num_sms) ? n_tiles : (uint32_t)(kCtasPerSm * num_sms));
+    const uint32_t tiles_r = (uint32_t)(rows / kTileR);
+    TileOrder d;
+    d.band_tiles = make_fastdiv(tiles_r * kBand);
+    d.n_full = tiles_c / kBand * kBand * tiles_r;
+    d.last_w = make_fastdiv(tiles_c % kBand ? tiles_c % kBand : 1);
+    d.last_c0 = tiles_c / kBand * kBand;
+    // scale-array geometry: per-row scale count (row-major) or 4-column atom count (tcgen05)
+    const uint32_t row_S = (uint32_t)(cols / 32), col_S = (uint32_t)(rows / 32);
+    const uint32_t rdim = tc ? (row_S + 3) / 4 : row_S, cdim = tc ? (col_S + 3) / 4 : col_S;
     uint8_t *re = static_cast<uint8_t *>(row_elems), *ce = static_cast<uint8_t *>(col_elems);
+    const int v8 = ((reinterpret_cast<uintptr_t>(re) | reinterpret_cast<uintptr_t>(ce)) & 31u) == 0;
+    const uint32_t R = (uint32_t)rows, C = (uint32_t)cols;
     switch (fmt * 2 + (ceil ? 1 : 0)) {
-    case FMT_E4M3 * 2 + 0: launch_dual_t<FMT_E4M3, false>(tm, (int)grid, smem, rows, cols, re, row_sc, ce, col_sc, tc, watchdog, st); break;
-    case FMT_E4M3 * 2 + 1: launch_dual_t<FMT_E4M3, true>(tm, (int)grid, smem, rows, cols, re, row_sc, ce, col_sc, tc, watchdog, st); break;
-    case FMT_E5M2 * 2 + 0: launch_dual_t<FMT_E5M2, false>(tm, (int)grid, smem, rows, cols, re, row_sc, ce, col_sc, tc, watchdog, st); break;
-    case FMT_E5M2 * 2 + 1: launch_dual_t<FMT_E5M2, true>(tm, (int)grid, smem, rows, cols, re, row_sc, ce, col_sc, tc, watchdog, st); break;
-    case FMT_E2M1 * 2 + 0: launch_dual_t<FMT_E2M1, false>(tm, (int)grid, smem, rows, cols, re, row_sc, ce, col_sc, tc, watchdog, st); break;
-    case FMT_E2M1 * 2 + 1: launch_dual_t<FMT_E2M1, true>(tm, (int)grid, smem, rows, cols, re, row_sc, ce, col_sc, tc, watchdog, st); break;
+    case FMT_E4M3 * 2 + 0: return launch_dual_t<FMT_E4M3, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E4M3 * 2 + 1: return launch_dual_t<FMT_E4M3, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E5M2 * 2 + 0: return launch_dual_t<FMT_E5M2, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E5M2 * 2 + 1: return launch_dual_t<FMT_E5M2, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E2M1 * 2 + 0: return launch_dual_t<FMT_E2M1, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E2M1 * 2 + 1: return launch_dual_t<FMT_E2M1, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace mxk

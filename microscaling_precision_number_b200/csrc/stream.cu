@@ -31,6 +31,7 @@
 #include "codec.cuh"
 #include "internal.h"
 #include "ptx.cuh"
+#include "tiling.cuh"
 
 namespace mxk {
 
@@ -41,31 +42,6 @@ constexpr int kTileBytes = 16384;
 constexpr int kCtasPerSm = 3;
 constexpr int kNvfp4PartialsOffset = 64;   // scratch floats: [0, 64) barrier words, then partial maxima
 }  // namespace
-
-// ---- host-computed divider: q = n / d for n < 2^31 --------------------------------------
-struct FastDiv {
-    uint32_t d, mul, shift;
-};
-
-static FastDiv make_fastdiv(uint32_t d) {
-    FastDiv f{d, 0u, 0u};
-    if (d <= 1) return f;
-    uint32_t l = 0;
-    while ((1ull << l) < d) l++;                       // ceil(log2 d)
-    const uint32_t p = 31 + l;
-    f.mul = (uint32_t)(((1ull << p) + d - 1) / d);
-    f.shift = p - 32;
-    return f;
-}
-
-__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv &f) {
-    return f.d <= 1 ? n : (__umulhi(n, f.mul) >> f.shift);
-}
-
-// tcgen05 tiling offset of scale (r, c) with S scale columns (col_atoms = ceil(S/4)).
-__device__ __forceinline__ uint32_t tc_offset(uint32_t r, uint32_t c, uint32_t col_atoms) {
-    return (((r >> 7) * col_atoms + (c >> 2)) << 9) | ((r & 31u) << 4) | (((r >> 5) & 3u) << 2) | (c & 3u);
-}
 
 // ---- tile ring ------------------------------------------------------------------------------
 struct Ring {
@@ -138,31 +114,21 @@ __device__ __forceinline__ void stream_tiles(Ring &ring, uint32_t n_tiles, Body 
     }
 }
 
-// Packed fp32 pairs (sm_100a mul.rn.f32x2: two IEEE round-to-nearest products per instruction).
-__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
-    return r;
+// |x| maximum (15-bit bf16 magnitude; NaN anywhere gives >= 0x7F80) of a 32-element block
+// held as four uint4 / a 16-element block held as two, by the packed bf16 maximum.
+__device__ __forceinline__ uint32_t absmax_block32(const uint4 (&v)[4]) {
+    uint32_t a = absmax_bf16x2(absmax_bf16x2(v[0].x, v[0].y), absmax_bf16x2(v[0].z, v[0].w));
+    uint32_t b = absmax_bf16x2(absmax_bf16x2(v[1].x, v[1].y), absmax_bf16x2(v[1].z, v[1].w));
+    uint32_t c = absmax_bf16x2(absmax_bf16x2(v[2].x, v[2].y), absmax_bf16x2(v[2].z, v[2].w));
+    uint32_t d = absmax_bf16x2(absmax_bf16x2(v[3].x, v[3].y), absmax_bf16x2(v[3].z, v[3].w));
+    const uint32_t m = absmax_bf16x2(absmax_bf16x2(a, b), absmax_bf16x2(c, d));
+    return max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
 }
-__device__ __forceinline__ uint64_t splat2(float a) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(a));
-    return r;
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ void unpack2(uint64_t v, float &lo, float &hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-// Eight bf16 (one uint4) times a scalar, as eight fp32 (element i in x[i]).
-__device__ __forceinline__ void scale8(const uint4 &v, uint64_t s2, float (&x)[8]) {
-    unpack2(mul2(bf16x2_to_f32x2(v.x), s2), x[0], x[1]);
-    unpack2(mul2(bf16x2_to_f32x2(v.y), s2), x[2], x[3]);
-    unpack2(mul2(bf16x2_to_f32x2(v.z), s2), x[4], x[5]);
-    unpack2(mul2(bf16x2_to_f32x2(v.w), s2), x[6], x[7]);
+__device__ __forceinline__ uint32_t absmax_block16(const uint4 &v0, const uint4 &v1) {
+    const uint32_t a = absmax_bf16x2(absmax_bf16x2(v0.x, v0.y), absmax_bf16x2(v0.z, v0.w));
+    const uint32_t b = absmax_bf16x2(absmax_bf16x2(v1.x, v1.y), absmax_bf16x2(v1.z, v1.w));
+    const uint32_t m = absmax_bf16x2(a, b);
+    return max(m & 0x7FFFu, (m >> 16) & 0x7FFFu);
 }
 
 __device__ __forceinline__ uint32_t amax_words(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -196,9 +162,8 @@ mx_rows_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS,
             const uint32_t c = (j + rot) & 3u;
             v[j] = *reinterpret_cast<const uint4 *>(tile + tid * 64 + c * 16);
         }
-        uint32_t m = __vmaxu2(amax_words(v[0].x, v[0].y, v[0].z, v[0].w), amax_words(v[1].x, v[1].y, v[1].z, v[1].w));
-        m = __vmaxu2(m, __vmaxu2(amax_words(v[2].x, v[2].y, v[2].z, v[2].w), amax_words(v[3].x, v[3].y, v[3].z, v[3].w)));
-        const uint32_t code = e8m0_from_amax_bits<FMT, CEIL>(hmax(m));
+        const uint32_t m = absmax_block32(v);
+        const uint32_t code = e8m0_from_amax_bits<FMT, CEIL>(m);
         const uint64_t mul2x = splat2(e8m0_inverse_multiplier(code));
         const bool nan_blk = code == 0xFFu;
 #pragma unroll
@@ -291,8 +256,7 @@ __device__ __forceinline__ void nvfp4_quant_tile(const uint8_t *tile, uint32_t t
     bool special[2];
 #pragma unroll
     for (int h = 0; h < 2; h++) {
-        const uint32_t m = hmax(__vmaxu2(amax_words(v[h][0].x, v[h][0].y, v[h][0].z, v[h][0].w),
-                                         amax_words(v[h][1].x, v[h][1].y, v[h][1].z, v[h][1].w)));
+        const uint32_t m = absmax_block16(v[h][0], v[h][1]);
         special[h] = m >= 0x7F80u;                           // Inf/NaN in the block
         const float a = __uint_as_float(m << 16);
         float tq;

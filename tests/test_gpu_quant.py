@@ -297,3 +297,24 @@ def test_nvfp4_tiny_tensor_scales(oracle, sigma_log2):
     assert host(q.global_scale)[0] == np.float32(g_ref)
     assert np.array_equal(host(q.elems), e_ref.reshape(-1))
     assert np.array_equal(host(q.scales), s_ref.reshape(-1))
+
+
+def test_output_buffers_are_reused(oracle):
+    """`out=` writes into the caller's buffers (same pointers, same results)."""
+    x = to_dev(synth.activations(64, 256, seed=5))
+    q = mx.quantize(x, "e4m3", "row", "ceil", layout="both")
+    q.elems.zero_(); q.scales.zero_(); q.scales_alt.zero_()
+    q2 = mx.quantize(x, "e4m3", "row", "ceil", layout="both", out=q)
+    assert q2.elems.data_ptr() == q.elems.data_ptr() and q2.scales_alt.data_ptr() == q.scales_alt.data_ptr()
+    ref = mx.quantize(x, "e4m3", "row", "ceil", layout="both")
+    assert torch.equal(q2.elems, ref.elems) and torch.equal(q2.scales, ref.scales)
+    assert torch.equal(q2.scales_alt, ref.scales_alt)
+    d = mx.quantize_dual(x, "e5m2", "floor", "rowmajor")
+    d2 = mx.quantize_dual(x, "e5m2", "floor", "rowmajor", out=d)
+    assert d2[1].elems.data_ptr() == d[1].elems.data_ptr()
+    y = torch.empty_like(x)
+    assert mx.dequantize(q, "tcgen05", out=y).data_ptr() == y.data_ptr()
+    assert torch.equal(y, mx.dequantize(q, "rowmajor"))
+    with pytest.raises(ValueError):
+        mx.quantize(x, "e4m3", "row", "ceil", layout="both", out=mx.Quantized(q.elems[:10], q.scales, q.scales_alt,
+                                                                             None, 64, 256, q.fmt))
