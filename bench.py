@@ -43,6 +43,8 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 R2 = C2 = 4096
 BYTES_MXFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 32)            # 42,991,616
 BYTES_NVFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 16) + 4         # 44,040,196
+NCU_TRAFFIC_NVFP4 = None          # dram read + write bytes of one NVFP4 call (both kernels, ncu)
+NCU_TRAFFIC_MXFP4 = 33565952      # same for mx_rows_kernel<E2M1, floor, both layouts>
 STEP_BYTES = BYTES_MXFP4 + BYTES_NVFP4
 NROT = 8                 # rotating copies of the weight (8 x 32 MiB > 2 x L2)
 
@@ -153,7 +155,7 @@ class WeightQuantStep:
         self.sn = torch.empty(R * C // 16, dtype=torch.uint8, device=dev)
         self.snt = torch.empty(mx.scale_bytes(R, C // 16, "tcgen05"), dtype=torch.uint8, device=dev)
         self.g = torch.empty(1, dtype=torch.float32, device=dev)
-        self.launches_per_step = 2      # MXFP4 quantiser; fused NVFP4 kernel (no padding at 4096)
+        self.launches_per_step = 3      # MXFP4 quantiser; NVFP4 maximum + quantiser (no padding at 4096)
 
     def mxfp4(self, stream):
         L = self.L
@@ -228,15 +230,20 @@ def run_ours(args, rank, world, dev):
         torch.cuda.synchronize()
         per[which] = a.elapsed_time(b) / ncall
     mean_mx, mean_nv = per["mxfp4"], per["nvfp4"]
+    # DRAM bytes per call (read + write) from one ncu capture of the same kernels on this
+    # workload (profiles/nvfp4_and_rows_weight4096.md); ncu replays each launch with a
+    # flushed L2, so a kernel's outputs are still in L2 at its end and count as 0 written
+    # bytes
     if mean_nv >= mean_mx:
-        dom = {"kernel": "mx_quantize(NVFP4): nvfp4_fused_kernel<both layouts> (cooperative)", "ms": mean_nv,
-               "bytes": BYTES_NVFP4}
+        dom = {"kernel": "mx_quantize(NVFP4) call: nvfp4_amax_bulk_kernel + nvfp4_quant_bulk_kernel<both layouts>",
+               "ms": mean_nv,
+               "bytes": BYTES_NVFP4, "traffic": NCU_TRAFFIC_NVFP4}
     else:
         dom = {"kernel": "mx_quantize(MXFP4): mx_rows_kernel<E2M1,floor,both layouts>", "ms": mean_mx,
-               "bytes": BYTES_MXFP4}
+               "bytes": BYTES_MXFP4, "traffic": NCU_TRAFFIC_MXFP4}
     achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": None,
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": dom["traffic"],
                 "peak_source": pk["source"] + " copy bandwidth (MEASURED_PEAKS hbm_gbs), burst",
                 "kernel": dom["kernel"], "algorithmic_bytes_per_launch": dom["bytes"],
                 "ms_per_launch": round(dom["ms"], 5),
@@ -384,6 +391,22 @@ def run_breakdown(mx, dev, pk):
                      "peak_note": "bf16 burst (MEASURED_PEAKS) x 2, the FP8/f8f6f4 to bf16 nominal ratio"}
         del a, b, c
         torch.cuda.empty_cache()
+
+    # next row: FP4 x FP4 block-scaled matmuls (kind::mxf4 and kind::mxf4nvf4), 8192^3,
+    # against the dense FP4 rate (2 x the FP8 rate; 9 PFLOP/s nominal)
+    fp4_peak = 2.0 * mx_peak
+    for name, fmt in (("next_gemm_mxfp4_x_mxfp4_8192", "e2m1"), ("next_gemm_nvfp4_x_nvfp4_8192", "nvfp4")):
+        M = N = K = 8192
+        a = mx.quantize(to_dev(synth.normal(M, K, seed=60), dev), fmt, "row", "floor", layout="tcgen05")
+        b = mx.quantize(to_dev(synth.normal(N, K, sigma=0.02, seed=61), dev), fmt, "row", "floor", layout="tcgen05")
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        t = timed([lambda: mx.gemm(a, b, c)], 10, stream)
+        tf = 2.0 * M * N * K / (t * 1e-3) / 1e12
+        out[name] = {"ms": round(t, 4), "TFLOPS": round(tf, 1), "frac_fp4_peak_measured": round(tf / fp4_peak, 4),
+                     "fp4_peak_measured_TFLOPS": fp4_peak, "frac_fp4_nominal_9000": round(tf / (2 * MX_NOMINAL_TFLOPS), 4),
+                     "peak_note": "bf16 burst (MEASURED_PEAKS) x 4, the FP4 to bf16 nominal ratio"}
+        del a, b, c
+        torch.cuda.empty_cache()
     return out
 
 
@@ -463,6 +486,13 @@ def run_case(name, iters, dev):
         qn = mx.quantize(xw, "nvfp4", "row", "ceil", layout="tcgen05")
         y = torch.empty_like(xw)
         fns = [lambda: (mx.dequantize(q4, "tcgen05", out=y), mx.dequantize(qn, "tcgen05", out=y))]
+    elif name in ("gemm_mxfp4_8192", "gemm_nvfp4_8192"):
+        fmt = "e2m1" if name == "gemm_mxfp4_8192" else "nvfp4"
+        a = mx.quantize(to_dev(synth.normal(8192, 8192, seed=60), dev), fmt, "row", "floor", layout="tcgen05")
+        b = mx.quantize(to_dev(synth.normal(8192, 8192, sigma=0.02, seed=61), dev), fmt, "row", "floor",
+                        layout="tcgen05")
+        c = torch.empty((8192, 8192), dtype=torch.bfloat16, device=dev)
+        fns = [lambda: mx.gemm(a, b, c)]
     elif name in ("gemm8192", "gemm_w4a8"):
         (M, N, K), bfmt, bsig = (((8192, 8192, 8192), "e4m3", 1.0) if name == "gemm8192"
                                  else ((8192, 14336, 4096), "e2m1", 0.02))
@@ -478,7 +508,8 @@ def run_case(name, iters, dev):
     print(f"{name}: {iters} calls, {t * 1e3:.1f} us per call", flush=True)
 
 
-CASES = ["weight4096", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "gemm8192", "gemm_w4a8"]
+CASES = ["weight4096", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "gemm8192", "gemm_w4a8",
+         "gemm_mxfp4_8192", "gemm_nvfp4_8192"]
 
 
 def main():

@@ -119,15 +119,15 @@ mx_status mx_quantize(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt f
  * mx_quantize_nvfp4_noalloc -- NVFP4 quantisation that never allocates device memory.
  * The pages have no counterpart to this call; it exists for callers of this library.
  *
- * mx_quantize(fmt = MX_FMT_NVFP4) needs a small scratch buffer (grid-barrier words and
- * per-CTA partial maxima), which the library allocates with cudaMalloc on the first
+ * mx_quantize(fmt = MX_FMT_NVFP4) needs a small scratch buffer (one partial maximum
+ * per CTA of its tensor-maximum pass), which the library allocates with cudaMalloc on the first
  * NVFP4 call on each device.  Callers that cannot allow a cudaMalloc -- a serving loop
  * that reserves all device memory at start-up and must not take the implicit device
  * synchronisation or the out-of-memory risk of an allocation on its request path, or a
  * host framework that owns all device memory through its own allocator -- call this
  * variant instead.  It runs the same kernels and produces bit-identical outputs, with the
- * scratch in a fixed static device array of 64 + MX_NOALLOC_MAX_PARTIALS fp32 values
- * (4.25 KiB) that every GPU loading the library holds until the process exits.
+ * scratch in a fixed static device array of MX_NOALLOC_MAX_PARTIALS fp32 values (4 KiB)
+ * that every GPU loading the library holds until the process exits.
  *
  * Arguments are those of mx_quantize with fmt = MX_FMT_NVFP4 and axis = ROW (cols a
  * multiple of 16, global_scale required, same layouts, alignment and ownership).
@@ -141,9 +141,7 @@ mx_status mx_quantize(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt f
  *     than MX_NOALLOC_MAX_PARTIALS returns MX_ERR_SHAPE without launching (on a 148-SM
  *     B200 the count never exceeds 444).
  *   - Every call shares the one array, which keeps the previous call's contents.  Each
- *     call writes every partial-maximum slot it later reads; the barrier words must be
- *     zero when a call starts: they are zero at load time and every completed call leaves
- *     them zero (after a watchdog timeout, mx_watchdog_status(clear = 1) zeroes them).
+ *     call writes every partial-maximum slot it later reads, so nothing carries over.
  *     Calls whose GPU work overlaps (for example on two streams without ordering between
  *     them) race on the array and may produce wrong results.  Order such calls on one
  *     stream.
@@ -190,24 +188,34 @@ mx_status mx_cast(const void *src_bf16, int64_t n, mx_fmt fmt, void *out_elems, 
 
 /*
  * One operand of the block-scaled matmul: a rows x K matrix of codes, K-major (each row
- * holds K consecutive codes), with E8M0 scales per 32 along K in the TCGEN05 layout
- * (rows x K/32 scales), exactly as mx_quantize(axis = ROW, layout = TCGEN05) writes it.
+ * holds K consecutive codes; FP4 packed two per byte), with its block scales in the TCGEN05
+ * layout exactly as mx_quantize(axis = ROW, layout = TCGEN05) writes them: E8M0 per 32
+ * along K (rows x K/32) for E4M3 / E2M1, UE4M3 per 16 along K (rows x K/16) for NVFP4.
+ *   global_scale  NVFP4 only: device pointer to the operand's fp32 per-tensor scale g (as
+ *                 written by mx_quantize); NULL for MX operands.
  */
 typedef struct {
     const void *elems;
     const uint8_t *scales;
     mx_fmt fmt;
+    const float *global_scale;
 } mx_operand;
 
 /*
- * mx_gemm -- C = A * B^T with block scaling ([Q] §7; mixed MXFP4 x MXFP8 per [Q] §2
- * and §6): C[m, n] = sum_k dec(A[m,k]) 2^(sA[m,k/32]-127) dec(B[n,k]) 2^(sB[n,k/32]-127),
- * accumulated in fp32 on the tensor cores, written as bf16 (RNE).
- *   A           M x K operand, fmt E4M3 (activations).
- *   B           N x K operand, fmt E4M3 or E2M1 (weights).
+ * mx_gemm -- C = A * B^T with block scaling ([Q] §7; mixed MXFP4 x MXFP8 per [Q] §2 and
+ * §6; FP4 x FP4 per [Q] §7's FP4 tensor-core rate and §3's NVFP4 two-level scale):
+ *   MX:    C[m, n] = sum_k dec(A[m,k]) 2^(sA[m,k/32]-127) dec(B[n,k]) 2^(sB[n,k/32]-127)
+ *   NVFP4: C[m, n] = gA gB sum_k dec(A[m,k]) dec(sA[m,k/16]) dec(B[n,k]) dec(sB[n,k/16])
+ * accumulated in fp32 on the tensor cores (the NVFP4 product gA gB is applied to the fp32
+ * sum), written as bf16 (RNE).
+ *   Format pairs (A, B): (E4M3, E4M3), (E4M3, E2M1) -- activations x weights -- and
+ *   (E2M1, E2M1), (NVFP4, NVFP4); any other pair, or a global_scale that is missing for
+ *   NVFP4 or present for MX, is MX_ERR_ARG.
  *   C_bf16      device, M x N row-major bf16, 16-byte aligned.
- *   Shapes: M and N multiples of 128, K a multiple of 128 (else MX_ERR_SHAPE).
- *   Alignment: elems 32-byte aligned, scales 16-byte aligned (else MX_ERR_ALIGN).
+ *   Shapes: M and N multiples of 128; K a multiple of 128 (8-bit A) or 256 (FP4 x FP4)
+ *   (else MX_ERR_SHAPE).
+ *   Alignment: elems 32-byte aligned, scales 16-byte aligned, global scales 4-byte aligned
+ *   (else MX_ERR_ALIGN).
  */
 mx_status mx_gemm(mx_operand A, mx_operand B, void *C_bf16, int64_t M, int64_t N, int64_t K,
                   mx_stream_t stream);

@@ -26,7 +26,8 @@ MX_NOALLOC_MAX_PARTIALS = 1024
 
 
 class MxOperand(ctypes.Structure):
-    _fields_ = [("elems", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("fmt", ctypes.c_int)]
+    _fields_ = [("elems", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("fmt", ctypes.c_int),
+                ("global_scale", ctypes.c_void_p)]
 
 
 class MxError(RuntimeError):

@@ -138,7 +138,9 @@ def cast(x: torch.Tensor, fmt="e4m3", stream=None) -> torch.Tensor:
 
 
 def gemm(a: Quantized, b: Quantized, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """C = A * B^T for A (M x K) and B (N x K) quantised row-wise with tcgen05 scales."""
+    """C = A * B^T for A (M x K) and B (N x K) quantised row-wise with tcgen05 scales:
+    E4M3 x E4M3, E4M3 x E2M1, E2M1 x E2M1 or NVFP4 x NVFP4 (whose per-tensor scales are
+    applied to the fp32 sum)."""
     M, K = a.rows, a.cols
     N = b.rows
     if b.cols != K:
@@ -147,8 +149,8 @@ def gemm(a: Quantized, b: Quantized, out: Optional[torch.Tensor] = None, stream=
     sb = b.scales_alt if b.scales_alt is not None else b.scales
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a.elems.device)
-    A = L.MxOperand(a.elems.data_ptr(), sa.data_ptr(), a.fmt)
-    B = L.MxOperand(b.elems.data_ptr(), sb.data_ptr(), b.fmt)
+    A = L.MxOperand(a.elems.data_ptr(), sa.data_ptr(), a.fmt, _ptr(a.global_scale))
+    B = L.MxOperand(b.elems.data_ptr(), sb.data_ptr(), b.fmt, _ptr(b.global_scale))
     L.check(L.lib.mx_gemm(A, B, out.data_ptr(), M, N, K, _stream(stream)), "mx_gemm")
     return out
 

@@ -118,13 +118,6 @@ mx_status mx_watchdog_status(int *code, int clear) {
         const int zero = 0;
         e = cudaMemcpyToSymbol(g_watchdog_flag, &zero, sizeof(int));
         if (e != cudaSuccess) return cuda_fail(e);
-        // a call that gave up may have left grid-barrier words mid-way: reset them
-        if (d->partials) {
-            e = cudaMemset(d->partials, 0, 64 * sizeof(float));
-            if (e != cudaSuccess) return cuda_fail(e);
-        }
-        e = mxk::noalloc_reset_barrier();
-        if (e != cudaSuccess) return cuda_fail(e);
     }
     if (code) *code = v;
     return v ? MX_ERR_TIMEOUT : MX_OK;
@@ -167,14 +160,12 @@ mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, m
 
     if (fmt == MX_FMT_NVFP4) {
         {
-            // one fixed-size scratch per device, allocated on first use; its barrier words
-            // start at zero and every completed call leaves them at zero
+            // one fixed-size scratch per device for the per-CTA partial maxima, allocated on
+            // first use (every call writes each slot it later reads)
             std::lock_guard<std::mutex> lock(g_mu);
             if (!d->partials) {
                 const int nf = mxk::stream_nvfp4_scratch_floats(d->num_sms);
                 e = cudaMalloc(reinterpret_cast<void **>(&d->partials), sizeof(float) * (size_t)nf);
-                if (e != cudaSuccess) return cuda_fail(e);
-                e = cudaMemset(d->partials, 0, sizeof(float) * (size_t)nf);
                 if (e != cudaSuccess) return cuda_fail(e);
                 d->partials_cap = nf;
             }
@@ -288,14 +279,18 @@ mx_status mx_cast(const void *src, int64_t n, mx_fmt fmt, void *out, mx_stream_t
 
 mx_status mx_gemm(mx_operand A, mx_operand B, void *C, int64_t M, int64_t N, int64_t K,
                   mx_stream_t stream) {
-    if (A.fmt != MX_FMT_E4M3 || (B.fmt != MX_FMT_E4M3 && B.fmt != MX_FMT_E2M1)) return MX_ERR_ARG;
+    const bool f8 = A.fmt == MX_FMT_E4M3 && (B.fmt == MX_FMT_E4M3 || B.fmt == MX_FMT_E2M1);
+    const bool mxf4 = A.fmt == MX_FMT_E2M1 && B.fmt == MX_FMT_E2M1;
+    const bool nvf4 = A.fmt == MX_FMT_NVFP4 && B.fmt == MX_FMT_NVFP4;
+    if (!f8 && !mxf4 && !nvf4) return MX_ERR_ARG;
+    if (nvf4 != (A.global_scale != nullptr) || nvf4 != (B.global_scale != nullptr)) return MX_ERR_ARG;
     if (M < 0 || N < 0 || K < 0) return MX_ERR_SHAPE;
-    if (M % 128 || N % 128 || K % 128) return MX_ERR_SHAPE;
+    if (M % 128 || N % 128 || K % (f8 ? 128 : 256)) return MX_ERR_SHAPE;
     if (M > (int64_t)1 << 30 || N > (int64_t)1 << 30 || K > (int64_t)1 << 30) return MX_ERR_SHAPE;
     if (M == 0 || N == 0) return MX_OK;
     if (!A.elems || !A.scales || !B.elems || !B.scales || !C) return MX_ERR_ARG;
     if (!aligned(A.elems, 32) || !aligned(B.elems, 32) || !aligned(A.scales, 16) || !aligned(B.scales, 16) ||
-        !aligned(C, 16))
+        !aligned(C, 16) || !aligned(A.global_scale, 4) || !aligned(B.global_scale, 4))
         return MX_ERR_ALIGN;
     DeviceState *d = nullptr;
     mx_status st = device_state(&d);
@@ -306,7 +301,8 @@ mx_status mx_gemm(mx_operand A, mx_operand B, void *C, int64_t M, int64_t N, int
         e = cudaMemsetAsync(C, 0, (size_t)(M * N * 2), s);   // empty sum
         return e == cudaSuccess ? MX_OK : cuda_fail(e);
     }
-    e = mxk::launch_gemm(A.elems, A.scales, B.elems, B.scales, B.fmt, C, M, N, K, d->watchdog, d->num_sms, s);
+    e = mxk::launch_gemm(A.elems, A.scales, A.fmt, A.global_scale, B.elems, B.scales, B.fmt, B.global_scale, C, M,
+                         N, K, d->watchdog, d->num_sms, s);
     return e == cudaSuccess ? MX_OK : cuda_fail(e);
 }
 

@@ -9,9 +9,11 @@
 //        quantising both orientations from one read avoids re-quantising a transposed copy.
 //
 // Design:
-//   - persistent CTAs, two per SM, walk 32-row x 256-column bf16 tiles.  A producer warp
-//     loads each tile as four 32 x 64 boxes (2-D TMA, 128-byte swizzle) into a 6-stage
-//     ring guarded by full / empty mbarriers;
+//   - persistent CTAs, one per SM, walk 32-row x 256-column bf16 tiles.  A producer warp
+//     loads each tile as four 32 x 64 boxes (2-D TMA, 128-byte swizzle) into a 12-stage
+//     ring (192 KiB in flight per SM) guarded by full / empty mbarriers.  One CTA with a
+//     deep ring measured faster than two or three CTAs with shallower rings holding the
+//     same bytes;
 //   - warp specialisation over the same stage: warps 0-3 run the column pass (one warp
 //     per box, one lane per column pair, 32-bit shared loads), warps 4-7 the row pass (one
 //     lane per 32-element row block, four 16-byte shared loads).  The swizzle makes both
@@ -38,10 +40,10 @@ constexpr int kBoxes = 4;
 constexpr int kTileR = 32, kTileC = kBoxC * kBoxes;  // 32 x 256 tile
 constexpr int kBoxBytes = kTileR * kBoxC * 2;        // 4 KiB
 constexpr int kTileBytes = kBoxBytes * kBoxes;       // 16 KiB
-constexpr int kStages = 6;
+constexpr int kStages = 12;
 constexpr int kProducerWarp = 8;
 constexpr int kDualThreads = 32 * (kProducerWarp + 1);
-constexpr int kCtasPerSm = 2;
+constexpr int kCtasPerSm = 1;
 constexpr size_t kDualSmem = (size_t)kStages * kTileBytes + 1024;   // + alignment to 1024
 }  // namespace
 

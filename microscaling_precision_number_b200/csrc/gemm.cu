@@ -39,22 +39,35 @@
 
 namespace mxk {
 
+// MMA kinds: E4M3 x {E4M3, E2M1 expanded to bytes} with E8M0 scales per 32 (one scale
+// per row per K = 32 instruction); E2M1 x E2M1 packed with E8M0 scales per 32 (two per
+// K = 64 instruction); E2M1 x E2M1 packed with UE4M3 scales per 16 (four per K = 64).
+enum : int { KIND_F8F6F4 = 0, KIND_MXF4 = 1, KIND_NVF4 = 2 };
+
 namespace {
-constexpr int kBM = 128, kBK = 128;                      // tile rows; kBK in elements (= smem bytes)
+constexpr int kBM = 128, kBK = 128;                      // tile rows; bytes of K per row per stage
 constexpr int kStages = 4;
 constexpr int kEpilogueWarps = 8;                  // two per TMEM lane quadrant
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kGemmThreads = 320;
 constexpr int kABytes = kBM * kBK;                       // 16 KiB
-constexpr int kSfaBytes = 512;
 constexpr uint32_t kTmemCols = 512;                      // accumulator (<= 256) + scale slots
 constexpr uint32_t kSfCol0 = 256;                        // first scale-slot column
-constexpr uint32_t kSfColsPerStage = 16;                 // B: 8 at +0, A: 4 at +8
-template <int BN> struct Tile {
+template <int BN, int KIND> struct Tile {
+    // K elements per stage (128 bytes of codes per row) and scale atoms (512 B: 128 rows x
+    // 4 scales) per 128 rows per stage
+    static constexpr int kStageK = KIND == KIND_F8F6F4 ? 128 : 256;
+    static constexpr int kAtoms = KIND == KIND_F8F6F4 ? 1 : (KIND == KIND_MXF4 ? 2 : 4);
     static constexpr int kBBytes = BN * kBK;             // 32 KiB for BN = 256
-    static constexpr int kSfbBytes = 512 * (BN / 128);
+    static constexpr int kSfaBytes = 512 * kAtoms;
+    static constexpr int kSfbBytes = 512 * kAtoms * (BN / 128);
+    // tensor-memory scale columns per stage: B atoms first (4 columns per 128 rows), then A
+    static constexpr uint32_t kSfbCols = 4 * kAtoms * (BN / 128);
+    static constexpr uint32_t kSfColsPerStage = kSfbCols + 4 * kAtoms;
     static constexpr int kSmemBytes = kStages * (kABytes + kBBytes + kSfaBytes + kSfbBytes) + 1024;
 };
+static_assert(kSfCol0 + kStages * Tile<256, KIND_NVF4>::kSfColsPerStage <= kTmemCols, "scale slots exceed TMEM");
+static_assert(Tile<256, KIND_NVF4>::kSmemBytes + 256 <= 227 * 1024, "shared memory");
 }  // namespace
 
 // ---- tcgen05 wrappers -------------------------------------------------------------------
@@ -87,30 +100,51 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
-// Instruction descriptor for kind::mxf8f6f4 with block scaling: B scale-factor id in
-// bits 4-5, A format 7-9, B format 10-12 (E4M3 = 0, E2M1 = 5), K-major A and B, N >> 3
-// in 17-22, scale type E8M0 (bit 23 = 1), M >> 4 in 24-28, A scale-factor id in 29-30.
-template <int BN>
+// Instruction descriptor for the block-scaled kinds: B scale-factor id (first scale byte
+// of the 32-bit tensor-memory word) in bits 4-5, A format 7-9, B format 10-12 (mxf8f6f4:
+// E4M3 = 0, E2M1 = 5; mxf4 / mxf4nvf4: E2M1 = 1), K-major A and B, N >> 3 in 17-22, scale
+// type in bit 23 (1 = UE8M0, 0 = UE4M3), M >> 4 in 24-28, A scale-factor id in 29-30,
+// bit 31 = 0 (dense K of 32 for 8-bit kinds, 64 for 4-bit kinds).
+template <int BN, int KIND>
 __device__ __forceinline__ uint32_t mma_idesc(uint32_t b_fmt_code, uint32_t sf_id) {
+    const uint32_t a_fmt = KIND == KIND_F8F6F4 ? 0u : 1u;
+    const uint32_t b_fmt = KIND == KIND_F8F6F4 ? b_fmt_code : 1u;
     uint32_t d = 0;
     d |= (sf_id & 3u) << 4;
-    d |= 0u << 7;                         // A: E4M3
-    d |= (b_fmt_code & 7u) << 10;
+    d |= a_fmt << 7;
+    d |= (b_fmt & 7u) << 10;
     d |= (uint32_t)(BN >> 3) << 17;
-    d |= 1u << 23;                        // UE8M0 scales
+    d |= (KIND == KIND_NVF4 ? 0u : 1u) << 23;
     d |= (uint32_t)(kBM >> 4) << 24;
     d |= (sf_id & 3u) << 29;
     return d;
 }
 
+template <int KIND>
 __device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-        : "memory");
+    if constexpr (KIND == KIND_F8F6F4) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    } else if constexpr (KIND == KIND_MXF4) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+            : "memory");
+    }
 }
 
 // Copy a 512-byte scale atom (32 rows x 16 bytes, contiguous) into 4 TMEM columns,
@@ -153,18 +187,22 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 // consecutive tiles without a break (the shared-memory ring spans tiles).  The epilogue
 // drains a finished accumulator into registers, releases it (acc_empty) so that the MMAs
 // of the next tile start at once, and then writes its bf16 rows while they run.
-template <int BN>
+// alpha = (*ga) * (*gb) multiplies the accumulator before the bf16 conversion (the NVFP4
+// per-tensor scales; ga = gb = nullptr means 1).
+template <int BN, int KIND>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const uint8_t *__restrict__ a_sc, const uint8_t *__restrict__ b_sc,
-               uint16_t *__restrict__ C, int M, int N, int K, uint32_t b_fmt_code, int band, int *watchdog) {
+               const uint8_t *__restrict__ a_sc, const uint8_t *__restrict__ b_sc, const float *__restrict__ ga,
+               const float *__restrict__ gb, uint16_t *__restrict__ C, int M, int N, int K, uint32_t b_fmt_code,
+               int band, int *watchdog) {
+    using T = Tile<BN, KIND>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;                                   // kStages x 16 KiB (1024-aligned)
-    constexpr int kBBytes = Tile<BN>::kBBytes, kSfbBytes = Tile<BN>::kSfbBytes;
+    constexpr int kBBytes = T::kBBytes, kSfaBytes = T::kSfaBytes, kSfbBytes = T::kSfbBytes;
     uint8_t *sB = sA + kStages * kABytes;                 // kStages x BN x 128 B
     uint8_t *sSFA = sB + kStages * kBBytes;               // kStages x 512 B
-    uint8_t *sSFB = sSFA + kStages * kSfaBytes;           // kStages x 512 B per 128 rows of B
+    uint8_t *sSFB = sSFA + kStages * kSfaBytes;           // kStages x kAtoms x 512 B per 128 rows of B
 
     __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], acc_full, acc_empty, drain_bar;
     __shared__ uint32_t tmem_base_sh;
@@ -172,7 +210,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     volatile int *fail_sh = &fail_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_kb = K / kBK;
+    const int num_kb = K / T::kStageK;
     const int tiles_n = N / BN, tiles_m = M / kBM;
     const int n_tiles = tiles_m * tiles_n;
 
@@ -197,8 +235,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            const int64_t kb128 = K / 128;
-            const uint32_t tx = kABytes + (b_fmt_code == 5u ? kBBytes / 2 : kBBytes) + kSfaBytes + kSfbBytes;
+            // scale atoms per 128-row block of an operand (the tcgen05 layout's column-atom count)
+            const int64_t col_atoms = (int64_t)num_kb * T::kAtoms;
+            const bool b_expanded = KIND == KIND_F8F6F4 && b_fmt_code == 5u;
+            const uint32_t tx = kABytes + (b_expanded ? kBBytes / 2 : kBBytes) + kSfaBytes + kSfbBytes;
             int it = 0;
             for (int t = blockIdx.x; t < n_tiles && !*fail_sh; t += gridDim.x) {
                 int m_blk, n_blk;
@@ -210,16 +250,20 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         *fail_sh = 1;
                         break;
                     }
-                    // An E2M1 tile lands in shared memory padded to one byte per element
-                    // (16U4_ALIGN16B), but the copy completes only the packed global bytes.
+                    // An E2M1 tile of the mxf8f6f4 kind lands in shared memory padded to one
+                    // byte per element (16U4_ALIGN16B), but the copy completes only the
+                    // packed global bytes.  Either way a stage holds 128 bytes of K per row.
                     mbar_arrive_expect_tx(&full_bar[s], tx);
                     tma_load_2d(sA + s * kABytes, &tmA, kb * kBK, m_blk * kBM, &full_bar[s]);
                     tma_load_2d(sB + s * kBBytes, &tmB, kb * kBK, n_blk * BN, &full_bar[s]);
-                    bulk_load(sSFA + s * kSfaBytes, a_sc + ((int64_t)m_blk * kb128 + kb) * 512, kSfaBytes, &full_bar[s]);
+                    // the stage's scale atoms are contiguous in the tcgen05 layout
+                    bulk_load(sSFA + s * kSfaBytes, a_sc + ((int64_t)m_blk * col_atoms + (int64_t)kb * T::kAtoms) * 512,
+                              kSfaBytes, &full_bar[s]);
 #pragma unroll
                     for (int h = 0; h < BN / 128; h++)
-                        bulk_load(sSFB + s * kSfbBytes + h * 512,
-                                  b_sc + ((int64_t)((BN / 128) * n_blk + h) * kb128 + kb) * 512, 512, &full_bar[s]);
+                        bulk_load(sSFB + s * kSfbBytes + h * T::kSfaBytes,
+                                  b_sc + ((int64_t)((BN / 128) * n_blk + h) * col_atoms + (int64_t)kb * T::kAtoms) * 512,
+                                  T::kSfaBytes, &full_bar[s]);
                     last_it[s] = it;
                 }
             }
@@ -242,19 +286,32 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t sfb_t = tmem + kSfCol0 + s * kSfColsPerStage;
-                    const uint32_t sfa_t = sfb_t + 8;
-                    tc_cp_sf(sfa_t, smem_u32(sSFA + s * kSfaBytes));
+                    // tensor-memory scale slots of this stage: B atom (a, h) at column
+                    // sfb_t + 4 (a (BN/128) + h), A atom a at sfa_t + 4 a
+                    const uint32_t sfb_t = tmem + kSfCol0 + s * T::kSfColsPerStage;
+                    const uint32_t sfa_t = sfb_t + T::kSfbCols;
 #pragma unroll
-                    for (int h = 0; h < BN / 128; h++) tc_cp_sf(sfb_t + 4 * h, smem_u32(sSFB + s * kSfbBytes + h * 512));
+                    for (int a = 0; a < T::kAtoms; a++) {
+                        tc_cp_sf(sfa_t + 4 * a, smem_u32(sSFA + s * kSfaBytes + a * 512));
+#pragma unroll
+                        for (int h = 0; h < BN / 128; h++)
+                            tc_cp_sf(sfb_t + 4 * (a * (BN / 128) + h),
+                                     smem_u32(sSFB + s * kSfbBytes + h * T::kSfaBytes + a * 512));
+                    }
                     const uint32_t a_base = smem_u32(sA + s * kABytes);
                     const uint32_t b_base = smem_u32(sB + s * kBBytes);
+                    // four instructions per stage, each over 32 bytes of K per row (K = 32 for
+                    // 8-bit codes, 64 for packed 4-bit codes).  Instruction k reads scale atom
+                    // a and, inside its 32-bit words, the scale byte(s) starting at sf_id:
+                    // 1X: a = 0, sf_id = k; 2X: a = k / 2, sf_id = 2 (k % 2); 4X: a = k, sf_id = 0.
 #pragma unroll
-                    for (int k = 0; k < kBK / 32; k++) {
+                    for (int k = 0; k < 4; k++) {
+                        const int a = KIND == KIND_F8F6F4 ? 0 : (KIND == KIND_MXF4 ? k >> 1 : k);
+                        const uint32_t sf_id = KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u);
                         const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
                         const uint64_t bd = smem_desc(b_base + k * 32, 16, 1024, 2);
-                        tc_mma_mx(tmem, ad, bd, mma_idesc<BN>(b_fmt_code, (uint32_t)k), sfa_t, sfb_t,
-                                  (kb > 0 || k > 0) ? 1u : 0u);
+                        tc_mma_mx<KIND>(tmem, ad, bd, mma_idesc<BN, KIND>(b_fmt_code, sf_id), sfa_t + 4 * a,
+                                        sfb_t + 4 * a * (BN / 128), (kb > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty_bar[s]);
                 }
@@ -269,6 +326,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         // warp w reads TMEM lanes 32 (w % 4) .. + 31 (rows) and columns of half w / 4
         constexpr int kHalf = BN / 2;
         const int quad = warp & 3, half = warp >> 2;
+        const float alpha = (ga && gb) ? __fmul_rn(__ldg(ga), __ldg(gb)) : 1.0f;
         const uint32_t t_base = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(half * kHalf);
         int i = 0;
         for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, i++) {
@@ -282,7 +340,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 tmem_ld32(t_base + j * 32, r);
 #pragma unroll
                 for (int q = 0; q < 16; q++)
-                    o[j * 16 + q] = f32x2_to_bf16x2(__uint_as_float(r[2 * q]), __uint_as_float(r[2 * q + 1]));
+                    o[j * 16 + q] = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(r[2 * q]), alpha),
+                                                    __fmul_rn(__uint_as_float(r[2 * q + 1]), alpha));
             }
             tc_fence_before();
             __syncwarp();
@@ -320,50 +379,70 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                   CUtensorMapFloatOOBfill);
 
+// 2-D tensor map over a rows x K operand: 8-bit codes (one byte per element), E2M1 codes
+// expanded to bytes by the copy (16U4_ALIGN16B, mxf8f6f4 kind) or packed E2M1 codes read as
+// bytes (4-bit kinds).  Either way the box is 128 bytes of shared memory per row.
 static bool encode_operand(EncodeTiledFn enc, CUtensorMap *tm, const void *ptr, int64_t rows, int64_t K,
-                           bool fp4, uint32_t box_rows) {
-    const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+                           bool fp4, bool expand, uint32_t box_rows) {
+    const cuuint64_t gdim[2] = {(cuuint64_t)(fp4 && !expand ? K / 2 : K), (cuuint64_t)rows};
     const cuuint64_t gstride[1] = {(cuuint64_t)(fp4 ? K / 2 : K)};
     const cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(tm, fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+    const CUresult r = enc(tm, expand ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                            const_cast<void *>(ptr), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, const void *b_elems, const uint8_t *b_sc,
-                        int b_fmt, void *c, int64_t M, int64_t N, int64_t K, int *watchdog, int num_sms,
-                        cudaStream_t st) {
+template <int BN, int KIND>
+static cudaError_t launch_gemm_k(const CUtensorMap &tmA, const CUtensorMap &tmB, const uint8_t *a_sc,
+                                 const uint8_t *b_sc, const float *ga, const float *gb, void *c, int64_t M,
+                                 int64_t N, int64_t K, uint32_t b_code, int64_t band, int *watchdog, int grid,
+                                 cudaStream_t st) {
+    auto k = mx_gemm_kernel<BN, KIND>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<BN, KIND>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kGemmThreads, Tile<BN, KIND>::kSmemBytes, st>>>(tmA, tmB, a_sc, b_sc, ga, gb, static_cast<uint16_t *>(c),
+                                                             (int)M, (int)N, (int)K, b_code, (int)band, watchdog);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, int a_fmt, const float *ga, const void *b_elems,
+                        const uint8_t *b_sc, int b_fmt, const float *gb, void *c, int64_t M, int64_t N, int64_t K,
+                        int *watchdog, int num_sms, cudaStream_t st) {
     auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
     if (!enc) return cudaErrorNotSupported;
+    int kind;
+    if (a_fmt == FMT_E4M3 && (b_fmt == FMT_E4M3 || b_fmt == FMT_E2M1)) kind = KIND_F8F6F4;
+    else if (a_fmt == FMT_E2M1 && b_fmt == FMT_E2M1) kind = KIND_MXF4;
+    else if (a_fmt == FMT_NVFP4 && b_fmt == FMT_NVFP4) kind = KIND_NVF4;
+    else return cudaErrorInvalidValue;
+    const int stage_k = kind == KIND_F8F6F4 ? 128 : 256;
+    if (K % stage_k) return cudaErrorInvalidValue;
+    const bool a_fp4 = kind != KIND_F8F6F4, b_fp4 = b_fmt != FMT_E4M3;
+    const bool b_expand = kind == KIND_F8F6F4 && b_fp4;
     CUtensorMap tmA, tmB;
-    const bool fp4 = b_fmt == FMT_E2M1;
-    if (!encode_operand(enc, &tmA, a_elems, M, K, false, kBM)) return cudaErrorInvalidValue;
+    if (!encode_operand(enc, &tmA, a_elems, M, K, a_fp4, false, kBM)) return cudaErrorInvalidValue;
     const bool wide = N % 256 == 0;
     const int bn = wide ? 256 : 128;
-    if (!encode_operand(enc, &tmB, b_elems, N, K, fp4, (uint32_t)bn)) return cudaErrorInvalidValue;
+    if (!encode_operand(enc, &tmB, b_elems, N, K, b_fp4, b_expand, (uint32_t)bn)) return cudaErrorInvalidValue;
     const int64_t n_tiles = (M / kBM) * (N / bn);
     // band of N-tiles whose B panels (bn rows x K codes) take at most ~48 MB of L2
-    const int64_t panel = (int64_t)bn * (fp4 ? K / 2 : K);
+    const int64_t panel = (int64_t)bn * (b_fp4 ? K / 2 : K);
     int64_t band = (48ll << 20) / (panel > 0 ? panel : 1);
     if (band < 1) band = 1;
     if (band > N / bn) band = N / bn;
-    const dim3 grid((unsigned)(n_tiles < num_sms ? n_tiles : num_sms));
-    cudaError_t e;
-    if (wide) {
-        e = cudaFuncSetAttribute(mx_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<256>::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        mx_gemm_kernel<256><<<grid, kGemmThreads, Tile<256>::kSmemBytes, st>>>(
-            tmA, tmB, a_sc, b_sc, static_cast<uint16_t *>(c), (int)M, (int)N, (int)K, fp4 ? 5u : 0u, (int)band, watchdog);
-    } else {
-        e = cudaFuncSetAttribute(mx_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<128>::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        mx_gemm_kernel<128><<<grid, kGemmThreads, Tile<128>::kSmemBytes, st>>>(
-            tmA, tmB, a_sc, b_sc, static_cast<uint16_t *>(c), (int)M, (int)N, (int)K, fp4 ? 5u : 0u, (int)band, watchdog);
-    }
-    return cudaGetLastError();
+    const int grid = (int)(n_tiles < num_sms ? n_tiles : num_sms);
+    const uint32_t b_code = b_expand ? 5u : 0u;
+    if (kind == KIND_F8F6F4)
+        return wide ? launch_gemm_k<256, KIND_F8F6F4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, b_code, band, watchdog, grid, st)
+                    : launch_gemm_k<128, KIND_F8F6F4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, b_code, band, watchdog, grid, st);
+    if (kind == KIND_MXF4)
+        return wide ? launch_gemm_k<256, KIND_MXF4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, 0u, band, watchdog, grid, st)
+                    : launch_gemm_k<128, KIND_MXF4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, 0u, band, watchdog, grid, st);
+    return wide ? launch_gemm_k<256, KIND_NVF4>(tmA, tmB, a_sc, b_sc, ga, gb, c, M, N, K, 0u, band, watchdog, grid, st)
+                : launch_gemm_k<128, KIND_NVF4>(tmA, tmB, a_sc, b_sc, ga, gb, c, M, N, K, 0u, band, watchdog, grid, st);
 }
 
 }  // namespace mxk

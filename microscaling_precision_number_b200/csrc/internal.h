@@ -15,13 +15,13 @@ cudaError_t launch_stream_rows_mx(const void *src, int64_t rows, int64_t cols, i
                                   uint8_t *sc_rowmajor, uint8_t *sc_tcgen05, int *watchdog, int num_sms,
                                   cudaStream_t st);
 
-// NVFP4 scratch: 64 floats of grid-barrier words (zero before first use; the kernel
-// leaves them ready for the next call), then one partial maximum per CTA.  Returns the
-// float count the launches below need on a device with num_sms SMs.
+// NVFP4 scratch: one partial maximum per CTA of the maximum pass (no initial value needed:
+// every call writes each slot it later reads).  Returns the float count the launch below
+// needs on a device with num_sms SMs.
 int stream_nvfp4_scratch_floats(int num_sms);
-// NVFP4 quantisation (tensor amax -> g written to *global_scale -> block scales and codes),
-// one cooperative kernel when possible, two kernels otherwise.  At most max_partials CTAs.
-cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, float *scratch, int max_partials,
+// NVFP4 quantisation (tensor amax -> g written to *global_scale -> block scales and codes)
+// as two kernels; the maximum pass uses at most max_partials CTAs.
+cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,
                                 float *global_scale, void *elems, uint8_t *sc_rowmajor, uint8_t *sc_tcgen05,
                                 int *watchdog, int num_sms, cudaStream_t st);
 
@@ -44,9 +44,11 @@ cudaError_t launch_quant_dual(const void *src, int64_t rows, int64_t cols, int f
                               bool tcgen05, int *watchdog, int num_sms, cudaStream_t st);
 
 // ---- gemm.cu -------------------------------------------------------------------------------------
-// tcgen05 block-scaled matmul C = A * B^T (A: M x K E4M3, B: N x K E4M3 or E2M1).
-cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, const void *b_elems,
-                        const uint8_t *b_sc, int b_fmt, void *c, int64_t M, int64_t N, int64_t K,
+// tcgen05 block-scaled matmul C = alpha A * B^T.  Format pairs: E4M3 x {E4M3, E2M1}
+// (K % 128 == 0), E2M1 x E2M1 and NVFP4 x NVFP4 (K % 256 == 0); alpha = (*ga) (*gb) for
+// NVFP4, else 1.
+cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, int a_fmt, const float *ga, const void *b_elems,
+                        const uint8_t *b_sc, int b_fmt, const float *gb, void *c, int64_t M, int64_t N, int64_t K,
                         int *watchdog, int num_sms, cudaStream_t st);
 
 // ---- api.cu --------------------------------------------------------------------------------------
@@ -56,10 +58,5 @@ void *tensor_map_encoder();
 void record_cuda_error(cudaError_t e);
 // Current device's SM count and watchdog-flag address (set up once per device; no allocation).
 cudaError_t device_info(int *num_sms, int **watchdog);
-
-// ---- noalloc.cu ----------------------------------------------------------------------------------
-// Zero the grid-barrier words of the static NVFP4 scratch on the current device (if it has
-// been set up there); used when the watchdog flag is cleared.
-cudaError_t noalloc_reset_barrier();
 
 }  // namespace mxk

@@ -1,7 +1,7 @@
 // noalloc.cu -- NVFP4 quantisation for callers that must not allocate device memory.
 //
-// mx_quantize(fmt = MX_FMT_NVFP4) keeps its scratch (grid-barrier words and per-CTA
-// partial maxima) in a buffer that the library allocates with cudaMalloc on the first
+// mx_quantize(fmt = MX_FMT_NVFP4) keeps its scratch (one partial maximum per CTA of the
+// tensor-maximum pass) in a buffer that the library allocates with cudaMalloc on the first
 // NVFP4 call on each device.  Some callers cannot allow that: a serving loop that
 // reserves all device memory up front and must not take the implicit device
 // synchronisation (or the out-of-memory risk) of a cudaMalloc on its request path, or a
@@ -20,10 +20,8 @@
 #include "../../include/mx.h"
 #include "internal.h"
 
-// 64 floats of grid-barrier words (zero-initialised; every completed call leaves them at
-// zero) followed by one partial maximum per CTA of the maximum pass.
-static constexpr int kBarrierFloats = 64;
-static __device__ __align__(256) float g_noalloc_scratch[kBarrierFloats + MX_NOALLOC_MAX_PARTIALS];
+// One partial maximum per CTA of the maximum pass (each call writes every slot it reads).
+static __device__ __align__(256) float g_noalloc_scratch[MX_NOALLOC_MAX_PARTIALS];
 
 namespace {
 
@@ -62,17 +60,6 @@ mx_status noalloc_setup(NoAllocDevice **out) {
 }
 
 }  // namespace
-
-namespace mxk {
-cudaError_t noalloc_reset_barrier() {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return e;
-    std::lock_guard<std::mutex> lock(g_na_mu);
-    if (!g_na[dev].ready) return cudaSuccess;
-    return cudaMemset(g_na[dev].scratch, 0, kBarrierFloats * sizeof(float));
-}
-}  // namespace mxk
 
 extern "C" mx_status mx_quantize_nvfp4_noalloc(const void *src_bf16, int64_t rows, int64_t cols,
                                                void *out_elems, uint8_t *out_scales,

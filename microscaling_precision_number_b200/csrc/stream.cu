@@ -40,7 +40,6 @@ constexpr int kThreads = 256;
 constexpr int kStages = 4;
 constexpr int kTileBytes = 16384;
 constexpr int kCtasPerSm = 3;
-constexpr int kNvfp4PartialsOffset = 64;   // scratch floats: [0, 64) barrier words, then partial maxima
 }  // namespace
 
 // ---- tile ring ------------------------------------------------------------------------------
@@ -77,9 +76,15 @@ __device__ __forceinline__ void pdl_wait_and_release() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Runs body(tile, stage_ptr) over this CTA's tiles with the bulk-copy ring.
-template <typename Body>
-__device__ __forceinline__ void stream_tiles(Ring &ring, uint32_t n_tiles, Body body) {
+// Runs body(tile, stage_ptr) over this CTA's tiles with the bulk-copy ring.  `after_issue`
+// runs in every thread once the first kStages copies are in flight and before the first
+// tile is consumed (a kernel that must wait for its predecessor's results, but not for its
+// input, waits there so that its first loads overlap the predecessor's tail).
+struct NoPrologue {
+    __device__ __forceinline__ void operator()() const {}
+};
+template <typename Body, typename Prologue = NoPrologue>
+__device__ __forceinline__ void stream_tiles(Ring &ring, uint32_t n_tiles, Body body, Prologue after_issue = {}) {
     const int tid = threadIdx.x;
     if (tid == 0) {
         for (int s = 0; s < kStages; s++) mbar_init(&ring.full[s], 1);
@@ -92,6 +97,7 @@ __device__ __forceinline__ void stream_tiles(Ring &ring, uint32_t n_tiles, Body 
             const uint32_t t = blockIdx.x + (uint32_t)s * gridDim.x;
             if (t < n_tiles) { ring.issue(t, s); issued++; }
         }
+    after_issue();
     uint32_t it = 0;
     for (uint32_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
         const int s = (int)(it % kStages);
@@ -195,8 +201,7 @@ __device__ __forceinline__ uint32_t finite_mask(uint32_t m) {
 
 // ---------------------------------------------------------------------------------------
 // NVFP4 quantisation of one 16 KiB tile (512 blocks of 16; thread = blocks tid, tid+256),
-// read from the shared-memory ring or, for a tile no longer resident, from global memory
-// (normally still in L2).  g is the per-tensor decode scale.
+// read from the shared-memory ring.  g is the per-tensor decode scale.
 //   per block: t = amax_b / (6 g), sb = UE4M3(t) (RNE, saturating), d = dec(sb) g,
 //   q = E2M1(x * (1/d)); a block holding a NaN/Inf gets sb = 0x7F and codes 0.
 // ---------------------------------------------------------------------------------------
@@ -352,90 +357,11 @@ __device__ __forceinline__ void store_partial(uint32_t acc, float *dst, uint32_t
 }
 
 // ---------------------------------------------------------------------------------------
-// Grid-wide barrier for a cooperatively launched grid (all CTAs co-resident).
-// bar[0] counts arrivals and is zero between uses (the last arrival resets it);
-// bar[32] (another 128-byte line, so polling does not contend with the arrivals) is a
-// generation number that the last arrival advances.  Arrival is an acq_rel atomic (it
-// publishes this CTA's earlier writes and lets the last arrival see everyone's); waiters
-// poll the generation with acquire loads and a short back-off.  The wait is bounded: on a
-// timeout (or once another CTA has given up) it returns false in every thread.
-// ---------------------------------------------------------------------------------------
-__device__ __forceinline__ bool grid_barrier(unsigned int *bar, uint32_t nctas, int *watchdog) {
-    __syncthreads();
-    int ok = 1;
-    if (threadIdx.x == 0) {
-        unsigned int *cnt = bar, *gen = bar + 32;
-        unsigned int g0, old, cur;
-        asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(g0) : "l"(gen) : "memory");
-        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(cnt) : "memory");
-        if (old == nctas - 1) {
-            asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(cnt) : "memory");
-            asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(gen) : "memory");
-        } else {
-            const uint64_t t0 = globaltimer_ns();
-            for (uint32_t i = 1;; i++) {
-                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(gen) : "memory");
-                if (cur != g0) break;
-                __nanosleep(20);
-                if ((i & 31u) == 0u) {
-                    if (*reinterpret_cast<volatile int *>(watchdog) != 0) { ok = 0; break; }
-                    if (globaltimer_ns() - t0 > kWaitLimitNs) { atomicExch(watchdog, WD_GRID_BARRIER); ok = 0; break; }
-                }
-            }
-        }
-    }
-    return __syncthreads_and(ok) != 0;
-}
-
-// ---------------------------------------------------------------------------------------
-// NVFP4 in one cooperative kernel.
-//   phase 1: stream this CTA's tiles through the ring, fold the finite |x| maximum;
-//   barrier: every CTA has published its partial maximum;
-//   phase 2: every CTA derives g, then quantises its tiles newest first: the last
-//   min(n, stages) tiles are still in its ring, older ones are re-read from global memory
-//   (normally L2).  Inputs up to ~stages x 16 KiB x CTAs are read from HBM once.
-// ---------------------------------------------------------------------------------------
-template <bool RM, bool TC>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-nvfp4_fused_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
-                   float *__restrict__ partials, unsigned int *__restrict__ bar, float *__restrict__ g_out,
-                   uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc,
-                   int *watchdog) {
-    pdl_wait_and_release();
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages];
-    __shared__ float warp_max[kThreads / 32];
-    Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
-              full, watchdog, src, kTileBytes, (uint64_t)n_blocks * 32};
-    constexpr uint32_t kBlocksPerTile = kTileBytes / 32;
-    const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
-
-    uint32_t acc = 0;
-    stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
-        acc = finite_amax_tile(tile, ring.bytes_of(t), acc);
-    });
-    store_partial(acc, partials + blockIdx.x, reinterpret_cast<uint32_t *>(warp_max));
-    if (!grid_barrier(bar, gridDim.x, watchdog)) return;
-
-    const float g = nvfp4_global_scale(partials, (int)gridDim.x, warp_max);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
-    __shared__ float rtab[128];
-    const Nvfp4Consts cst = nvfp4_consts(g, rtab);
-
-    const uint32_t G = gridDim.x, bid = blockIdx.x;
-    const uint32_t n_my = n_tiles > bid ? (n_tiles - 1 - bid) / G + 1 : 0;
-    for (int32_t j = (int32_t)n_my - 1; j >= 0; j--) {
-        const uint32_t t = bid + (uint32_t)j * G;
-        const bool resident = (uint32_t)j + kStages >= n_my;
-        const uint8_t *base = resident ? ring.buf + (j % kStages) * kTileBytes : src + (size_t)t * kTileBytes;
-        if (cst.fast) nvfp4_quant_tile<RM, TC, true>(base, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
-        else nvfp4_quant_tile<RM, TC, false>(base, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
-    }
-}
-
-// ---------------------------------------------------------------------------------------
-// NVFP4 as two kernels (used when a cooperative launch is not possible).
-// Pass 1: per-CTA maximum of the finite |x| (Inf/NaN excluded).
+// NVFP4 as two kernels.  Pass 1: per-CTA maximum of the finite |x| (Inf/NaN excluded).
+// Pass 2 (below) starts streaming the input before it waits for pass 1, and normally
+// finds it in L2.  A single cooperative kernel that kept each CTA's last tiles in shared
+// memory across a grid barrier measured slower at every size (the cooperative launch and
+// the barrier cost more than the L2 re-read saves).
 // ---------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 nvfp4_amax_bulk_kernel(const uint8_t *__restrict__ src, uint64_t n_bytes, float *__restrict__ partials,
@@ -461,21 +387,26 @@ nvfp4_quant_bulk_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fast
                         const float *__restrict__ partials, int n_partials, float *__restrict__ g_out,
                         uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc,
                         int *watchdog) {
-    pdl_wait_and_release();
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages];
     __shared__ float warp_max[kThreads / 32];
     Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
               full, watchdog, src, kTileBytes, (uint64_t)n_blocks * 32};
-    const float g = nvfp4_global_scale(partials, n_partials, warp_max);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
     __shared__ float rtab[128];
-    const Nvfp4Consts cst = nvfp4_consts(g, rtab);
+    Nvfp4Consts cst;
     const uint32_t n_tiles = (n_blocks + kTileBytes / 32 - 1) / (kTileBytes / 32);
+    // The input is not written by the maximum pass, so the ring starts loading it at once;
+    // the partial maxima are read only after the wait on that pass.
+    auto after_issue = [&]() {
+        pdl_wait_and_release();
+        const float g = nvfp4_global_scale(partials, n_partials, warp_max);
+        if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+        cst = nvfp4_consts(g, rtab);
+    };
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
         if (cst.fast) nvfp4_quant_tile<RM, TC, true>(tile, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
         else nvfp4_quant_tile<RM, TC, false>(tile, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
-    });
+    }, after_issue);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -614,12 +545,10 @@ constexpr size_t kStreamSmem = (size_t)kStages * kTileBytes + 128;
 
 // Launch with programmatic dependent launch enabled: the kernel may be scheduled while the
 // previous kernel on the stream drains; its first instruction (griddepcontrol.wait) holds it
-// until that kernel has completed.  `coop` additionally requests a cooperative launch (all
-// CTAs co-resident, needed by the grid barrier).  The shared-memory attribute is set once
-// per device and kernel.
+// until that kernel has completed.  The shared-memory attribute is set once per device and
+// kernel.
 template <typename... KArgs, typename... Args>
-static cudaError_t launch_ex(void (*kernel)(KArgs...), int grid, cudaStream_t st, bool coop, bool pdl,
-                             Args... args) {
+static cudaError_t launch_stream(void (*kernel)(KArgs...), int grid, cudaStream_t st, Args... args) {
     static std::mutex mu;
     static std::set<std::pair<int, const void *>> configured;
     int dev = 0;
@@ -639,32 +568,12 @@ static cudaError_t launch_ex(void (*kernel)(KArgs...), int grid, cudaStream_t st
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kStreamSmem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    unsigned n = 0;
-    if (pdl) {
-        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[n].val.programmaticStreamSerializationAllowed = 1;
-        n++;
-    }
-    if (coop) {
-        attr[n].id = cudaLaunchAttributeCooperative;
-        attr[n].val.cooperative = 1;
-        n++;
-    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = n;
+    cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
-}
-
-// Set the dynamic shared-memory attribute of a stream kernel (needed before occupancy queries).
-template <typename... KArgs>
-static cudaError_t launch_ex_config(void (*kernel)(KArgs...)) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
-}
-
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_stream(void (*kernel)(KArgs...), int grid, cudaStream_t st, Args... args) {
-    return launch_ex(kernel, grid, st, false, true, args...);
 }
 
 bool stream_supported(int64_t rows, int64_t cols) {
@@ -705,48 +614,23 @@ cudaError_t launch_stream_rows_mx(const void *src, int64_t rows, int64_t cols, i
     }
 }
 
-int stream_nvfp4_scratch_floats(int num_sms) { return kNvfp4PartialsOffset + kCtasPerSm * num_sms; }
+int stream_nvfp4_scratch_floats(int num_sms) { return kCtasPerSm * num_sms; }
 
 template <bool RM, bool TC>
-static cudaError_t launch_nvfp4_t(const uint8_t *src, uint32_t nb, FastDiv f, uint32_t ca, float *scratch,
+static cudaError_t launch_nvfp4_t(const uint8_t *src, uint32_t nb, FastDiv f, uint32_t ca, float *partials,
                                   int max_partials, float *g, uint8_t *elems, uint8_t *rm, uint8_t *tc, int *wd,
                                   int num_sms, cudaStream_t st) {
     const uint32_t n_tiles = (nb + 511) / 512;
-    float *partials = scratch + kNvfp4PartialsOffset;
-    unsigned int *bar = reinterpret_cast<unsigned int *>(scratch);
     int grid = stream_grid(n_tiles, num_sms);
     if (grid > max_partials) grid = max_partials;
-    static const bool two_pass_only = [] {
-        const char *v = getenv("MX_NVFP4_TWO_PASS");
-        return v != nullptr && v[0] == '1';
-    }();
-    if (!two_pass_only) {
-        // one cooperative kernel: every CTA must be resident at once
-        int per_sm = 0;
-        cudaError_t e = launch_ex_config(nvfp4_fused_kernel<RM, TC>);
-        if (e != cudaSuccess) return e;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, nvfp4_fused_kernel<RM, TC>, kThreads, kStreamSmem);
-        if (e != cudaSuccess) return e;
-        const int coop_grid = grid < per_sm * num_sms ? grid : per_sm * num_sms;
-        if (coop_grid >= 1) {
-            e = launch_ex(nvfp4_fused_kernel<RM, TC>, coop_grid, st, true, true, src, nb, f, ca, partials, bar, g,
-                          elems, rm, tc, wd);
-            if (e == cudaSuccess) return e;
-            (void)cudaGetLastError();   // not launchable as requested: clear and fall back
-            e = launch_ex(nvfp4_fused_kernel<RM, TC>, coop_grid, st, true, false, src, nb, f, ca, partials, bar,
-                          g, elems, rm, tc, wd);
-            if (e == cudaSuccess) return e;
-            (void)cudaGetLastError();
-        }
-    }
-    // two kernels: per-CTA maxima, then quantisation
+    // pass 1: per-CTA maxima; pass 2 (programmatic dependent launch): quantisation
     cudaError_t e = launch_stream(nvfp4_amax_bulk_kernel, grid, st, src, (uint64_t)nb * 32, partials, wd);
     if (e != cudaSuccess) return e;
     return launch_stream(nvfp4_quant_bulk_kernel<RM, TC>, stream_grid(n_tiles, num_sms), st, src, nb, f, ca,
                          (const float *)partials, grid, g, elems, rm, tc, wd);
 }
 
-cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, float *scratch, int max_partials,
+cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,
                                 float *g, void *elems, uint8_t *rm, uint8_t *tc, int *wd, int num_sms,
                                 cudaStream_t st) {
     const uint32_t nb = (uint32_t)(rows * cols / 16), S = (uint32_t)(cols / 16);
@@ -754,9 +638,9 @@ cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, flo
     const uint32_t ca = (S + 3) / 4;
     const uint8_t *s8 = static_cast<const uint8_t *>(src);
     uint8_t *e8 = static_cast<uint8_t *>(elems);
-    if (rm && tc) return launch_nvfp4_t<true, true>(s8, nb, f, ca, scratch, max_partials, g, e8, rm, tc, wd, num_sms, st);
-    if (rm) return launch_nvfp4_t<true, false>(s8, nb, f, ca, scratch, max_partials, g, e8, rm, tc, wd, num_sms, st);
-    return launch_nvfp4_t<false, true>(s8, nb, f, ca, scratch, max_partials, g, e8, rm, tc, wd, num_sms, st);
+    if (rm && tc) return launch_nvfp4_t<true, true>(s8, nb, f, ca, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
+    if (rm) return launch_nvfp4_t<true, false>(s8, nb, f, ca, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
+    return launch_nvfp4_t<false, true>(s8, nb, f, ca, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
 }
 
 template <int FMT, bool TC>

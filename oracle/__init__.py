@@ -75,7 +75,7 @@ def lib():
         _lib.mxo_tcgen05_scale_bytes.restype = I64
         _lib.mxo_tcgen05_scale_offset.argtypes = [I64, I64, I64, I64]
         _lib.mxo_tcgen05_scale_offset.restype = I64
-        _lib.mxo_gemm_ref.argtypes = [P, P, I, P, P, I, I64, I64, I64, P, I64, P, P]
+        _lib.mxo_gemm_ref.argtypes = [P, P, I, ctypes.c_double, P, P, I, ctypes.c_double, I64, I64, I64, P, I64, P, P]
         _lib.mxo_gemm_ref.restype = I
     return _lib
 
@@ -193,8 +193,9 @@ def tcgen05_offsets(rows: int, scale_cols: int) -> np.ndarray:
 
 
 # ---------------------------------------------------------------- matmul reference
-def gemm_ref(a_elems, a_scales, a_fmt, b_elems, b_scales, b_fmt, M, N, K, pairs):
-    """fp64 C[m, n] and sum_k |a b| for the requested (m, n) pairs (an array n x 2)."""
+def gemm_ref(a_elems, a_scales, a_fmt, b_elems, b_scales, b_fmt, M, N, K, pairs, a_g=1.0, b_g=1.0):
+    """fp64 C[m, n] and sum_k |a b| for the requested (m, n) pairs (an array n x 2).
+    a_g / b_g: the per-tensor scale of an NVFP4 operand (ignored for MX operands)."""
     pr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
     c = np.zeros(pr.shape[0], dtype=np.float64)
     mag = np.zeros(pr.shape[0], dtype=np.float64)
@@ -202,6 +203,7 @@ def gemm_ref(a_elems, a_scales, a_fmt, b_elems, b_scales, b_fmt, M, N, K, pairs)
     as_ = np.ascontiguousarray(a_scales, dtype=np.uint8)
     be = np.ascontiguousarray(b_elems, dtype=np.uint8)
     bs = np.ascontiguousarray(b_scales, dtype=np.uint8)
-    _check(lib().mxo_gemm_ref(_ptr(ae), _ptr(as_), a_fmt, _ptr(be), _ptr(bs), b_fmt, M, N, K,
+    _check(lib().mxo_gemm_ref(_ptr(ae), _ptr(as_), a_fmt, ctypes.c_double(a_g), _ptr(be), _ptr(bs), b_fmt,
+                              ctypes.c_double(b_g), M, N, K,
                               _ptr(pr), pr.shape[0], _ptr(c), _ptr(mag)), "gemm_ref")
     return c, mag

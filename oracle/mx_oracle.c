@@ -461,22 +461,29 @@ int64_t mxo_tcgen05_scale_offset(int64_t r, int64_t c, int64_t rows, int64_t sca
 /* ------------------------------------------------------------------------- */
 /* Block-scaled matmul reference: C[m,n] = sum_k a(m,k) b(n,k) in fp64 over   */
 /* the dequantised operands, a(m,k) = dec(A_q) * 2^(sA-127) and likewise b   */
-/* (Q§7 scale application; scales per 32 along K).  A is M x K and B is N x K,*/
-/* both K-major, scales row-major M x K/32 and N x K/32.  Computes the npairs */
-/* requested (m, n) entries and, for each, sum_k |a b| (the error budget).    */
+/* (Q§7 scale application; scales per 32 along K).  An NVFP4 operand decodes */
+/* as dec(q) * dec_UE4M3(s) * g with scales per 16 along K and its per-tensor */
+/* g (Q§3 two-level scaling).  A is M x K and B is N x K, both K-major,      */
+/* scales row-major (K/32 or K/16 per row).  Computes the npairs requested   */
+/* (m, n) entries and, for each, sum_k |a b| (the error budget).             */
 /* ------------------------------------------------------------------------- */
-static double mx_operand_value(const uint8_t *elems, const uint8_t *scales, int fmt,
+static double mx_operand_value(const uint8_t *elems, const uint8_t *scales, int fmt, double g,
                                int64_t row, int64_t k, int64_t K) {
-    int fp4 = (fmt == F_E2M1);
+    int fp4 = (fmt == F_E2M1 || fmt == F_NVFP4);
     int64_t row_bytes = fp4 ? K / 2 : K;
     unsigned q = get_code(elems + row * row_bytes, k, fp4);
+    if (fmt == F_NVFP4) {
+        unsigned sb = scales[row * (K / 16) + k / 16];
+        if (sb == 0x7Fu) return NAN;
+        return mxo_decode(K_E2M1, q) * mxo_decode(K_UE4M3, sb) * g;
+    }
     unsigned s = scales[row * (K / 32) + k / 32];
     if (s == 0xFFu) return NAN;
     return ldexp(mxo_decode(elem_kind(fmt), q), (int)s - 127);
 }
 
-int mxo_gemm_ref(const uint8_t *a_elems, const uint8_t *a_scales, int a_fmt,
-                 const uint8_t *b_elems, const uint8_t *b_scales, int b_fmt,
+int mxo_gemm_ref(const uint8_t *a_elems, const uint8_t *a_scales, int a_fmt, double a_g,
+                 const uint8_t *b_elems, const uint8_t *b_scales, int b_fmt, double b_g,
                  int64_t M, int64_t N, int64_t K, const int64_t *pairs, int64_t npairs,
                  double *c, double *abs_sum) {
     if (K % 32) return -1;
@@ -485,8 +492,8 @@ int mxo_gemm_ref(const uint8_t *a_elems, const uint8_t *a_scales, int a_fmt,
         if (m < 0 || m >= M || n < 0 || n >= N) return -1;
         double acc = 0.0, mag = 0.0;
         for (int64_t k = 0; k < K; k++) {
-            double a = mx_operand_value(a_elems, a_scales, a_fmt, m, k, K);
-            double b = mx_operand_value(b_elems, b_scales, b_fmt, n, k, K);
+            double a = mx_operand_value(a_elems, a_scales, a_fmt, a_g, m, k, K);
+            double b = mx_operand_value(b_elems, b_scales, b_fmt, b_g, n, k, K);
             acc += a * b;
             mag += fabs(a * b);
         }

@@ -94,9 +94,16 @@ def test_dual_dequant_cast_gemm_validation(L):
     assert lib.mx_cast(FAKE, 8, 3, FAKE, None) == L.MX_ERR_ARG
     assert lib.mx_cast(None, 8, 0, FAKE, None) == L.MX_ERR_ARG
     assert lib.mx_cast(FAKE, 0, 0, FAKE, None) == L.MX_OK
-    op = lambda fmt, p=FAKE: L.MxOperand(p, FAKE, fmt)
+    op = lambda fmt, p=FAKE, g=None: L.MxOperand(p, FAKE, fmt, g)
     assert lib.mx_gemm(op(0), op(1), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG      # E5M2 B unsupported
-    assert lib.mx_gemm(op(2), op(0), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG      # FP4 A unsupported
+    assert lib.mx_gemm(op(2), op(0), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG      # E2M1 x E4M3 unsupported
+    assert lib.mx_gemm(op(3, g=FAKE), op(2), FAKE, 128, 128, 256, None) == L.MX_ERR_ARG   # NVFP4 x MXFP4
+    assert lib.mx_gemm(op(3), op(3, g=FAKE), FAKE, 128, 128, 256, None) == L.MX_ERR_ARG   # missing g
+    assert lib.mx_gemm(op(2, g=FAKE), op(2), FAKE, 128, 128, 256, None) == L.MX_ERR_ARG   # g on MX
+    assert lib.mx_gemm(op(2), op(2), FAKE, 128, 128, 128, None) == L.MX_ERR_SHAPE    # FP4 x FP4: K % 256
+    assert lib.mx_gemm(op(3, g=FAKE), op(3, g=FAKE), FAKE, 128, 128, 384, None) == L.MX_ERR_SHAPE
+    assert lib.mx_gemm(op(3, g=FAKE + 2), op(3, g=FAKE), FAKE, 128, 128, 256, None) == L.MX_ERR_ALIGN
+    assert lib.mx_gemm(op(2), op(2), FAKE, 0, 128, 256, None) == L.MX_OK
     assert lib.mx_gemm(op(0), op(2), FAKE, 100, 128, 128, None) == L.MX_ERR_SHAPE
     assert lib.mx_gemm(op(0), op(0), FAKE, 128, 128, 96, None) == L.MX_ERR_SHAPE
     assert lib.mx_gemm(op(0, FAKE + 16), op(0), FAKE, 128, 128, 128, None) == L.MX_ERR_ALIGN

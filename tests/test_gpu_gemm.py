@@ -45,25 +45,44 @@ def _no_watchdog():
     assert mx.watchdog_status(clear=True) == 0
 
 
-def run_case(oracle, a_bits, b_bits, b_fmt, pairs=None):
+GPU_FMT = {0: "e4m3", 2: "e2m1", 3: "nvfp4"}
+
+
+def _gpu_quant(bits, fmt):
+    rounding = "floor" if fmt == 2 else "ceil"      # MXFP4 weights: OCP floor; MXFP8: the recipe's
+    return mx.quantize(to_dev(bits), GPU_FMT[fmt], "row", rounding, layout="tcgen05")
+
+
+def _oracle_quant(oracle, bits, rows, fmt):
+    """Oracle codes and scales of the given rows.  NVFP4's per-tensor scale depends on the
+    whole tensor, so the row holding the tensor's largest finite |x| is quantised with the
+    subset (block scales and codes are per row, so the other rows are unchanged)."""
+    if fmt != oracle.NVFP4:
+        e, s = oracle.quantize_mx(bits[rows], fmt, oracle.ROW, oracle.FLOOR if fmt == oracle.E2M1 else oracle.CEIL)
+        return e, s, 1.0
+    mag = (bits & 0x7FFF).astype(np.int64)
+    mag[mag >= 0x7F80] = -1
+    top = int(np.argmax(mag) // bits.shape[1])
+    e, s, g = oracle.quantize_nvfp4(np.ascontiguousarray(np.concatenate([bits[rows], bits[top:top + 1]])))
+    return e[:len(rows)], s[:len(rows)], g
+
+
+def run_case(oracle, a_bits, b_bits, b_fmt, pairs=None, a_fmt=None):
+    a_fmt = oracle.E4M3 if a_fmt is None else a_fmt
     M, K = a_bits.shape
     N = b_bits.shape[0]
-    a_q = mx.quantize(to_dev(a_bits), "e4m3", "row", "ceil", layout="tcgen05")
-    b_q = mx.quantize(to_dev(b_bits), "e2m1" if b_fmt == oracle.E2M1 else "e4m3", "row",
-                      "floor" if b_fmt == oracle.E2M1 else "ceil", layout="tcgen05")
-    c = bf16_to_f64(mx.gemm(a_q, b_q))
+    c = bf16_to_f64(mx.gemm(_gpu_quant(a_bits, a_fmt), _gpu_quant(b_bits, b_fmt)))
     if pairs is None:
         pairs = np.array([(m, n) for m in range(M) for n in range(N)], dtype=np.int64)
     # the oracle quantises the bf16 inputs itself; only the rows it needs
     rows_a = np.unique(pairs[:, 0])
     rows_b = np.unique(pairs[:, 1])
-    ae, as_ = oracle.quantize_mx(a_bits[rows_a], oracle.E4M3, oracle.ROW, oracle.CEIL)
-    be, bs = oracle.quantize_mx(b_bits[rows_b], b_fmt, oracle.ROW,
-                                oracle.FLOOR if b_fmt == oracle.E2M1 else oracle.CEIL)
+    ae, as_, ga = _oracle_quant(oracle, a_bits, rows_a, a_fmt)
+    be, bs, gb = _oracle_quant(oracle, b_bits, rows_b, b_fmt)
     ia = {int(r): i for i, r in enumerate(rows_a)}
     ib = {int(r): i for i, r in enumerate(rows_b)}
     local = np.array([(ia[int(m)], ib[int(n)]) for m, n in pairs], dtype=np.int64)
-    ref, mag = oracle.gemm_ref(ae, as_, oracle.E4M3, be, bs, b_fmt, len(rows_a), len(rows_b), K, local)
+    ref, mag = oracle.gemm_ref(ae, as_, a_fmt, be, bs, b_fmt, len(rows_a), len(rows_b), K, local, a_g=ga, b_g=gb)
     got = c[pairs[:, 0], pairs[:, 1]]
     err = np.abs(got - ref)
     bound = gemm_tolerance(ref, mag)
@@ -132,3 +151,47 @@ def test_config5_gemm_mixed_sampled(oracle):
     b = synth.normal(N, K, sigma=0.02, seed=51)
     run_case(oracle, a, b, oracle.E2M1, sample_pairs(M, N, 192, 5))
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ FP4 x FP4 (kind::mxf4, kind::mxf4nvf4)
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (128, 128, 256), (256, 512, 512), (384, 384, 768)])
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_gemm_fp4_x_fp4_small(oracle, M, N, K, fmt):
+    f = oracle.E2M1 if fmt == "mxfp4" else oracle.NVFP4
+    a = synth.normal(M, K, seed=M + 7)
+    b = synth.weight_fp4(N, K, seed=N + 8)
+    run_case(oracle, a, b, f, a_fmt=f)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_gemm_fp4_x_fp4_one_hot(oracle, fmt):
+    """One nonzero per A row (exactly representable): C is a scaled copy of B's column,
+    which checks the placement of every scale byte along K."""
+    f = oracle.E2M1 if fmt == "mxfp4" else oracle.NVFP4
+    M, N, K = 128, 256, 512
+    a = np.zeros((M, K), dtype=np.uint16)
+    vals = [0x3F80, 0x4040, 0xC0C0, 0x3F00]              # 1, 3, -6, 0.5
+    for m in range(M):
+        a[m, (m * 37) % K] = vals[m % 4]
+    b = synth.mx8_rowwise(N, K, seed=3)
+    run_case(oracle, a, b, f, a_fmt=f)
+
+
+@pytest.mark.parametrize("fmt", ["mxfp4", "nvfp4"])
+def test_gemm_fp4_x_fp4_8192_sampled(oracle, fmt):
+    f = oracle.E2M1 if fmt == "mxfp4" else oracle.NVFP4
+    M = N = K = 8192
+    a = synth.normal(M, K, seed=60)
+    b = synth.normal(N, K, sigma=0.02, seed=61)
+    run_case(oracle, a, b, f, sample_pairs(M, N, 128, 6), a_fmt=f)
+    torch.cuda.empty_cache()
+
+
+def test_gemm_rejects_unsupported_pairs():
+    x = to_dev(synth.normal(128, 256, seed=1))
+    e4 = mx.quantize(x, "e4m3", "row", "ceil", layout="tcgen05")
+    n4 = mx.quantize(x, "nvfp4", "row", "ceil", layout="tcgen05")
+    f4 = mx.quantize(x, "e2m1", "row", "floor", layout="tcgen05")
+    for a, b in ((f4, e4), (n4, f4), (e4, n4)):
+        with pytest.raises(mx.MxError):
+            mx.gemm(a, b)

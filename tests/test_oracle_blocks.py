@@ -268,6 +268,47 @@ def test_gemm_ref_exact_brute_force(oracle):
         assert mag[p] >= abs(c[p])
 
 
+def test_gemm_ref_fp4_operands_exact(oracle):
+    """MXFP4 x MXFP4 and NVFP4 x NVFP4 (with both per-tensor scales) against exact rational
+    arithmetic over independently decoded operands: E2M1 from its value table, UE4M3 block
+    scales by the E4M3 decoder of ml_dtypes, E8M0 as a power of two."""
+    M, N, K = 2, 3, 64
+    a = synth.weight_fp4(M, K, seed=21)
+    b = synth.normal(N, K, seed=22)
+    pairs = [(m, n) for m in range(M) for n in range(N)]
+    # MXFP4 x MXFP4
+    ae, as_ = oracle.quantize_mx(a, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    be, bs = oracle.quantize_mx(b, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    c, mag = oracle.gemm_ref(ae, as_, oracle.E2M1, be, bs, oracle.E2M1, M, N, K, pairs)
+    av = e2m1_values(np.stack([unpack_fp4(r, K) for r in ae]))
+    bv = e2m1_values(np.stack([unpack_fp4(r, K) for r in be]))
+    for p, (m, n) in enumerate(pairs):
+        exact = sum(Fraction(float(av[m, k])) * Fraction(2) ** (int(as_[m, k // 32]) - 127)
+                    * Fraction(float(bv[n, k])) * Fraction(2) ** (int(bs[n, k // 32]) - 127) for k in range(K))
+        assert Fraction(c[p]) == exact
+        assert mag[p] >= abs(c[p])
+    # NVFP4 x NVFP4: dec(q) * dec(sb) * g on each side
+    ae, as_, ga = oracle.quantize_nvfp4(a)
+    be, bs, gb = oracle.quantize_nvfp4(b)
+    c, mag = oracle.gemm_ref(ae, as_, oracle.NVFP4, be, bs, oracle.NVFP4, M, N, K, pairs, a_g=ga, b_g=gb)
+    av = e2m1_values(np.stack([unpack_fp4(r, K) for r in ae]))
+    bv = e2m1_values(np.stack([unpack_fp4(r, K) for r in be]))
+    sa = as_.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    sb = bs.view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    assert np.all(as_ < 0x7F) and np.all(bs < 0x7F)
+    for p, (m, n) in enumerate(pairs):
+        exact = sum(Fraction(float(av[m, k])) * Fraction(float(sa[m, k // 16])) * Fraction(float(ga))
+                    * Fraction(float(bv[n, k])) * Fraction(float(sb[n, k // 16])) * Fraction(float(gb))
+                    for k in range(K))
+        # each fp64 product of two 31-bit significands rounds once, then K additions:
+        # |error| <= (K + 1) u sum|ab| with u = 2^-53
+        assert abs(Fraction(c[p]) - exact) <= (K + 1) * Fraction(2) ** -53 * Fraction(mag[p])
+        assert mag[p] >= abs(c[p])
+    # g enters linearly
+    c2, _ = oracle.gemm_ref(ae, as_, oracle.NVFP4, be, bs, oracle.NVFP4, M, N, K, pairs, a_g=2 * ga, b_g=gb)
+    assert np.allclose(c2, 2 * c, rtol=1e-15, atol=0)
+
+
 def test_gemm_ref_one_hot(oracle):
     K = 96
     a = np.zeros((1, K), dtype=np.uint16)
