@@ -43,8 +43,8 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 R2 = C2 = 4096
 BYTES_MXFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 32)            # 42,991,616
 BYTES_NVFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 16) + 4         # 44,040,196
-NCU_TRAFFIC_NVFP4 = None          # dram read + write bytes of one NVFP4 call (both kernels, ncu)
-NCU_TRAFFIC_MXFP4 = 33565952      # same for mx_rows_kernel<E2M1, floor, both layouts>
+NCU_TRAFFIC_NVFP4 = 67149056      # dram read + write bytes of one NVFP4 call (both kernels, ncu, L2 flushed per kernel)
+NCU_TRAFFIC_MXFP4 = 33568768      # same for mx_rows_kernel<E2M1, floor, both layouts>
 STEP_BYTES = BYTES_MXFP4 + BYTES_NVFP4
 NROT = 8                 # rotating copies of the weight (8 x 32 MiB > 2 x L2)
 
