@@ -20,8 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 ROOT = os.path.dirname(PKG)
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmx.so")
-SOURCES = ["api.cu", "stream.cu", "quant.cu", "dual.cu", "gemm.cu", "noalloc.cu"]
-HEADERS = ["codec.cuh", "ptx.cuh", "tiling.cuh", "internal.h"]
+SOURCES = ["api.cu", "stream.cu", "quant.cu", "dual.cu", "gemm.cu", "gemm2.cu", "noalloc.cu"]
+HEADERS = ["codec.cuh", "ptx.cuh", "tiling.cuh", "umma.cuh", "internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
          "-I" + os.path.join(ROOT, "include")]

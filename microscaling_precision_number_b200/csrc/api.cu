@@ -301,8 +301,13 @@ mx_status mx_gemm(mx_operand A, mx_operand B, void *C, int64_t M, int64_t N, int
         e = cudaMemsetAsync(C, 0, (size_t)(M * N * 2), s);   // empty sum
         return e == cudaSuccess ? MX_OK : cuda_fail(e);
     }
-    e = mxk::launch_gemm(A.elems, A.scales, A.fmt, A.global_scale, B.elems, B.scales, B.fmt, B.global_scale, C, M,
-                         N, K, d->watchdog, d->num_sms, s);
+    // 256 x 256 tiles on CTA pairs when the shape allows, else 128 x {256, 128} tiles
+    if (mxk::gemm_pair_supported(M, N))
+        e = mxk::launch_gemm_pair(A.elems, A.scales, A.fmt, A.global_scale, B.elems, B.scales, B.fmt, B.global_scale,
+                                  C, M, N, K, d->watchdog, d->num_sms, s);
+    else
+        e = mxk::launch_gemm(A.elems, A.scales, A.fmt, A.global_scale, B.elems, B.scales, B.fmt, B.global_scale, C,
+                             M, N, K, d->watchdog, d->num_sms, s);
     return e == cudaSuccess ? MX_OK : cuda_fail(e);
 }
 

@@ -1,0 +1,358 @@
+// gemm2.cu -- the MX block-scaled matmul on CTA pairs (tcgen05 cta_group::2).
+//
+// Sources (page title, section): as gemm.cu --
+//   "MXFP4 と NVFP4 は何が違うのか調べてみた"
+//     §2 "MXFP4 はブロック32と E8M0", §3 "NVFP4 はブロック16と E4M3、そして二段目",
+//     §7 "ハードウェアの対応状況": block-scaled MMA on the 5th-generation tensor cores.
+//
+// Same product, formats and scale handling as gemm.cu, computed per 256 x 256 output tile
+// by a cluster of two CTAs on two SMs:
+//   - each CTA loads its own 128 rows of A and its own 128 rows (of 256) of B, plus its A
+//     rows' scale atoms and the scale atoms of all 256 B rows, with 2-D TMA loads that all
+//     complete on the even CTA's barrier (the `.cta_group::2` form with the peer bit of the
+//     barrier address cleared);
+//   - the even CTA's MMA thread copies the stage's scale atoms (each CTA's own shared
+//     memory into its own tensor memory) and issues tcgen05.mma.cta_group::2 with M = 256:
+//     the tensor core of each SM computes its CTA's 128 rows x 256 columns, reading A from
+//     its own shared memory and B from both CTAs' shared memory;
+//   - commits arrive on the barrier at the same offset in both CTAs (stage release,
+//     accumulator ready); both CTAs' epilogues release the accumulator on the even CTA's
+//     barrier (remote mbarrier arrive).
+// Per SM a K step moves A 16 KiB + half of B 16 KiB instead of 16 + 32 KiB: a third less
+// L2 -> SM traffic for the same MMA work, and 5-6 ring stages fit in shared memory.
+// Every wait is bounded (watchdog); the pair leaves through a bounded handshake after the
+// even CTA has drained its barriers and MMAs, so no copy or MMA touches a CTA that exited.
+#include <cuda.h>
+#include "codec.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+#include "umma.cuh"
+
+namespace mxk {
+
+namespace {
+constexpr int kHalfRows = 128;                       // rows of A and of B per CTA
+constexpr int kPairM = 256, kPairN = 256;            // output tile of the pair
+constexpr int kRowBytes = 128;                       // bytes of K per row per stage
+constexpr int kABytes = kHalfRows * kRowBytes;       // 16 KiB
+constexpr int kBBytes = kHalfRows * kRowBytes;       // 16 KiB (this CTA's half of B)
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kEpilogueWarps = 8;
+constexpr int kPairThreads = 320;
+constexpr uint32_t kTmemCols = 512, kSfCol0 = 256;
+constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;       // shared::cluster address of the even CTA's copy
+
+template <int KIND> struct Pair {
+    static constexpr int kStageK = KIND == KIND_F8F6F4 ? 128 : 256;
+    static constexpr int kAtoms = KIND == KIND_F8F6F4 ? 1 : (KIND == KIND_MXF4 ? 2 : 4);
+    static constexpr int kStages = KIND == KIND_NVF4 ? 5 : 6;
+    static constexpr int kSfaBytes = 512 * kAtoms;   // this CTA's 128 A rows
+    static constexpr int kSfbBytes = 1024 * kAtoms;  // all 256 B rows
+    static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+    static constexpr uint32_t kSfbCols = 8 * kAtoms;              // B atom (a, h) at 4 (2a + h)
+    static constexpr uint32_t kSfColsPerStage = kSfbCols + 4 * kAtoms;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+};
+static_assert(kSfCol0 + Pair<KIND_F8F6F4>::kStages * Pair<KIND_F8F6F4>::kSfColsPerStage <= kTmemCols, "tmem");
+static_assert(kSfCol0 + Pair<KIND_MXF4>::kStages * Pair<KIND_MXF4>::kSfColsPerStage <= kTmemCols, "tmem");
+static_assert(kSfCol0 + Pair<KIND_NVF4>::kStages * Pair<KIND_NVF4>::kSfColsPerStage <= kTmemCols, "tmem");
+static_assert(Pair<KIND_MXF4>::kSmemBytes + 1024 <= 227 * 1024, "shared memory");
+}  // namespace
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 2-D TMA load into this CTA's shared memory whose completion is counted on the even CTA's
+// barrier (same offset).
+__device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const void *tmap, int32_t x, int32_t y,
+                                                 uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y),
+          "r"(smem_u32(bar) & kPeerBitMask)
+        : "memory");
+}
+// Arrive (release, cluster scope) on the barrier at the same offset in CTA `rank`.
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t *bar, uint32_t rank) {
+    uint32_t remote;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(bar)), "r"(rank));
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+
+template <int KIND>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                    const float *__restrict__ ga, const float *__restrict__ gb, uint16_t *__restrict__ C, int M,
+                    int N, int K, uint32_t b_fmt_code, int band, int *watchdog) {
+    using P = Pair<KIND>;
+    constexpr int S = P::kStages;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;                                  // S x 16 KiB (1024-aligned)
+    uint8_t *sB = sA + S * kABytes;                      // S x 16 KiB
+    uint8_t *sSFA = sB + S * kBBytes;                    // S x kAtoms x 512 B
+    uint8_t *sSFB = sSFA + S * P::kSfaBytes;             // S x 2 x kAtoms x 512 B
+
+    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], acc_full, acc_empty, drain_bar, exit_bar;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int fail_flag;
+    volatile int *fail_sh = &fail_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int num_kb = K / P::kStageK;
+    const int tiles_n = N / kPairN, tiles_m = M / kPairM;
+    const int n_tiles = tiles_m * tiles_n;
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmSA);
+        prefetch_tensormap(&tmSB);
+        for (int s = 0; s < S; s++) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+        mbar_init(&acc_full, 1);
+        mbar_init(&acc_empty, 2 * kEpilogueWarps);
+        mbar_init(&drain_bar, 1);
+        mbar_init(&exit_bar, 1);
+        *fail_sh = 0;
+        fence_barrier_init();
+    }
+    if (warp == kMmaWarp) tmem_alloc<2>(&tmem_base_sh, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();                                  // both CTAs' barriers exist before any remote use
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_sh;
+
+    int last_it[S];                                      // producer: last ring use armed per stage
+    for (int s = 0; s < S; s++) last_it[s] = -1;
+    if (warp == kProducerWarp) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            const int col_atoms = num_kb * P::kAtoms;        // scale atoms per 128-row block
+            const bool b_expanded = KIND == KIND_F8F6F4 && b_fmt_code == 5u;
+            const uint32_t tx_pair = 2u * (kABytes + (b_expanded ? kBBytes / 2 : kBBytes) + P::kSfaBytes + P::kSfbBytes);
+            int it = 0;
+            for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs) {
+                int m_blk, n_blk;
+                tile_coords(t, tiles_m, tiles_n, band, m_blk, n_blk);
+                const int a_row = m_blk * kPairM + (int)rank * kHalfRows;
+                const int b_row = n_blk * kPairN + (int)rank * kHalfRows;
+                for (int kb = 0; kb < num_kb; kb++, it++) {
+                    const int s = it % S;
+                    if (it >= S &&
+                        !mbar_wait_bounded(&empty_bar[s], (uint32_t)((it / S) - 1) & 1u, watchdog, WD_GEMM_EMPTY)) {
+                        *fail_sh = 1;
+                        break;
+                    }
+                    if (leader) mbar_arrive_expect_tx(&full_bar[s], tx_pair);
+                    tma_load_2d_pair(sA + s * kABytes, &tmA, kb * kRowBytes, a_row, &full_bar[s]);
+                    tma_load_2d_pair(sB + s * kBBytes, &tmB, kb * kRowBytes, b_row, &full_bar[s]);
+                    // scale atoms as rows of 256 bytes (two per atom); a stage's atoms of one
+                    // 128-row block are contiguous
+                    tma_load_2d_pair(sSFA + s * P::kSfaBytes, &tmSA, 0,
+                                     2 * ((2 * m_blk + (int)rank) * col_atoms + kb * P::kAtoms), &full_bar[s]);
+#pragma unroll
+                    for (int h = 0; h < 2; h++)
+                        tma_load_2d_pair(sSFB + s * P::kSfbBytes + h * P::kSfaBytes, &tmSB, 0,
+                                         2 * ((2 * n_blk + h) * col_atoms + kb * P::kAtoms), &full_bar[s]);
+                    last_it[s] = it;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------ MMA issuer (even CTA only)
+        if (leader && lane == 0) {
+            int it = 0, i = 0;
+            for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs, i++) {
+                if (i > 0 && !mbar_wait_bounded(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
+                    *fail_sh = 1;
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < num_kb; kb++, it++) {
+                    const int s = it % S;
+                    if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
+                        *fail_sh = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfb_t = tmem + kSfCol0 + s * P::kSfColsPerStage;
+                    const uint32_t sfa_t = sfb_t + P::kSfbCols;
+#pragma unroll
+                    for (int a = 0; a < P::kAtoms; a++) {
+                        tc_cp_sf<2>(sfa_t + 4 * a, smem_u32(sSFA + s * P::kSfaBytes + a * 512));
+#pragma unroll
+                        for (int h = 0; h < 2; h++)
+                            tc_cp_sf<2>(sfb_t + 4 * (2 * a + h), smem_u32(sSFB + s * P::kSfbBytes + h * P::kSfaBytes + a * 512));
+                    }
+                    const uint32_t a_base = smem_u32(sA + s * kABytes);
+                    const uint32_t b_base = smem_u32(sB + s * kBBytes);
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        const int a = KIND == KIND_F8F6F4 ? 0 : (KIND == KIND_MXF4 ? k >> 1 : k);
+                        const uint32_t sf_id = KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u);
+                        const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
+                        const uint64_t bd = smem_desc(b_base + k * 32, 16, 1024, 2);
+                        tc_mma_mx<KIND, 2>(tmem, ad, bd, mma_idesc<kPairM, kPairN, KIND>(b_fmt_code, sf_id),
+                                           sfa_t + 4 * a, sfb_t + 8 * a, (kb > 0 || k > 0) ? 1u : 0u);
+                    }
+                    tc_commit_pair(&empty_bar[s]);           // stage s free in both CTAs
+                }
+                if (*fail_sh) break;
+                tc_commit_pair(&acc_full);                   // both halves of the tile are complete
+            }
+            tc_commit_pair(&drain_bar);                      // completes once every MMA above has finished
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue (warps 0-7, both CTAs)
+        constexpr int kHalf = kPairN / 2;
+        const int quad = warp & 3, half = warp >> 2;
+        const uint32_t t_base = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(half * kHalf);
+        const float alpha = (ga && gb) ? __fmul_rn(__ldg(ga), __ldg(gb)) : 1.0f;
+        int i = 0;
+        for (int t = pair; t < n_tiles; t += n_pairs, i++) {
+            const bool ok = mbar_wait_bounded(&acc_full, (uint32_t)i & 1u, watchdog, WD_GEMM_ACC);
+            if (!ok || *fail_sh) { *fail_sh = 1; break; }
+            tc_fence_after();
+            uint32_t o[kHalf / 2];
+#pragma unroll
+            for (int j = 0; j < kHalf / 32; j++) {
+                uint32_t r[32];
+                tmem_ld32(t_base + j * 32, r);
+#pragma unroll
+                for (int q = 0; q < 16; q++)
+                    o[j * 16 + q] = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(r[2 * q]), alpha),
+                                                    __fmul_rn(__uint_as_float(r[2 * q + 1]), alpha));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(&acc_empty, 0);   // on the even CTA's barrier
+            int m_blk, n_blk;
+            tile_coords(t, tiles_m, tiles_n, band, m_blk, n_blk);
+            const int row = m_blk * kPairM + (int)rank * kHalfRows + quad * 32 + lane;
+            uint4 *dst = reinterpret_cast<uint4 *>(C + (int64_t)row * N + (int64_t)n_blk * kPairN + half * kHalf);
+#pragma unroll
+            for (int q = 0; q < kHalf / 8; q++) __stcs(dst + q, make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]));
+        }
+    }
+
+    // teardown: the even CTA waits (bounded) for the copies it counted and for every MMA;
+    // the odd CTA waits for the MMAs too (they write its tensor memory); then a bounded
+    // handshake, so that neither CTA releases tensor memory or exits while the pair's
+    // copies or MMAs may still use the other's memory
+    __syncthreads();
+    if (warp == kMmaWarp && lane == 0) {
+        if (leader && *fail_sh)
+            for (int s = 0; s < S; s++)
+                if (last_it[s] >= 0)
+                    (void)mbar_wait_bounded(&full_bar[s], (uint32_t)(last_it[s] / S) & 1u, nullptr, 0, kDrainLimitNs);
+        (void)mbar_wait_bounded(&drain_bar, 0u, nullptr, 0, kDrainLimitNs);
+        // the odd CTA's copies complete on the even CTA's barriers, so it stays until the
+        // even CTA has drained them: each CTA arrives on the other's exit barrier
+        mbar_arrive_remote(&exit_bar, rank ^ 1u);
+        (void)mbar_wait_bounded(&exit_bar, 0u, nullptr, 0, 2 * kWaitLimitNs);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc<2>(tmem, kTmemCols);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+// Operand codes: rows x K, 128 bytes of K x 128 rows per box, 128-byte swizzle (as gemm.cu).
+static bool encode_codes(EncodeTiledFn enc, CUtensorMap *tm, const void *ptr, int64_t rows, int64_t K, bool fp4,
+                         bool expand) {
+    const cuuint64_t gdim[2] = {(cuuint64_t)(fp4 && !expand ? K / 2 : K), (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)(fp4 ? K / 2 : K)};
+    const cuuint32_t box[2] = {(cuuint32_t)kRowBytes, (cuuint32_t)kHalfRows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(tm, expand ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+               const_cast<void *>(ptr), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// tcgen05-tiled scales (rows/128 x col_atoms atoms of 512 B) viewed as 256-byte rows, two
+// per atom; a box is the kAtoms consecutive atoms of one 128-row block in one stage.
+static bool encode_scales(EncodeTiledFn enc, CUtensorMap *tm, const uint8_t *ptr, int64_t rows, int64_t col_atoms,
+                          int atoms_per_box) {
+    const cuuint64_t gdim[2] = {256, (cuuint64_t)((rows / 128) * col_atoms * 2)};
+    const cuuint64_t gstride[1] = {256};
+    const cuuint32_t box[2] = {256, (cuuint32_t)(2 * atoms_per_box)};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(ptr), gdim, gstride, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int KIND>
+static cudaError_t launch_pair_k(EncodeTiledFn enc, const void *a, const uint8_t *a_sc, const float *ga,
+                                 const void *b, const uint8_t *b_sc, const float *gb, bool b_fp4, bool b_expand,
+                                 void *c, int64_t M, int64_t N, int64_t K, int *watchdog, int num_sms,
+                                 cudaStream_t st) {
+    using P = Pair<KIND>;
+    CUtensorMap tmA, tmB, tmSA, tmSB;
+    const int64_t col_atoms = (K / P::kStageK) * P::kAtoms;
+    if (!encode_codes(enc, &tmA, a, M, K, KIND != KIND_F8F6F4, false) ||
+        !encode_codes(enc, &tmB, b, N, K, b_fp4, b_expand) ||
+        !encode_scales(enc, &tmSA, a_sc, M, col_atoms, P::kAtoms) ||
+        !encode_scales(enc, &tmSB, b_sc, N, col_atoms, P::kAtoms))
+        return cudaErrorInvalidValue;
+    const int64_t n_tiles = (M / kPairM) * (N / kPairN);
+    const int64_t panel = (int64_t)kPairN * (b_fp4 ? K / 2 : K);
+    int64_t band = (48ll << 20) / (panel > 0 ? panel : 1);
+    if (band < 1) band = 1;
+    if (band > N / kPairN) band = N / kPairN;
+    int64_t pairs = num_sms / 2;
+    if (pairs > n_tiles) pairs = n_tiles;
+    if (pairs < 1) pairs = 1;
+    auto k = mx_gemm_pair_kernel<KIND>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    k<<<(unsigned)(2 * pairs), kPairThreads, P::kSmemBytes, st>>>(tmA, tmB, tmSA, tmSB, ga, gb,
+                                                                   static_cast<uint16_t *>(c), (int)M, (int)N,
+                                                                   (int)K, b_expand ? 5u : 0u, (int)band, watchdog);
+    return cudaGetLastError();
+}
+
+bool gemm_pair_supported(int64_t M, int64_t N) { return M % kPairM == 0 && N % kPairN == 0; }
+
+cudaError_t launch_gemm_pair(const void *a_elems, const uint8_t *a_sc, int a_fmt, const float *ga,
+                             const void *b_elems, const uint8_t *b_sc, int b_fmt, const float *gb, void *c,
+                             int64_t M, int64_t N, int64_t K, int *watchdog, int num_sms, cudaStream_t st) {
+    auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
+    if (!enc) return cudaErrorNotSupported;
+    if (!gemm_pair_supported(M, N)) return cudaErrorInvalidValue;
+    if (a_fmt == FMT_E4M3 && (b_fmt == FMT_E4M3 || b_fmt == FMT_E2M1)) {
+        if (K % 128) return cudaErrorInvalidValue;
+        const bool fp4 = b_fmt == FMT_E2M1;
+        return launch_pair_k<KIND_F8F6F4>(enc, a_elems, a_sc, nullptr, b_elems, b_sc, nullptr, fp4, fp4, c, M, N, K,
+                                          watchdog, num_sms, st);
+    }
+    if (K % 256) return cudaErrorInvalidValue;
+    if (a_fmt == FMT_E2M1 && b_fmt == FMT_E2M1)
+        return launch_pair_k<KIND_MXF4>(enc, a_elems, a_sc, nullptr, b_elems, b_sc, nullptr, true, false, c, M, N, K,
+                                        watchdog, num_sms, st);
+    if (a_fmt == FMT_NVFP4 && b_fmt == FMT_NVFP4)
+        return launch_pair_k<KIND_NVF4>(enc, a_elems, a_sc, ga, b_elems, b_sc, gb, true, false, c, M, N, K, watchdog,
+                                        num_sms, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace mxk

@@ -51,6 +51,12 @@ cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, int a_fmt, con
                         const uint8_t *b_sc, int b_fmt, const float *gb, void *c, int64_t M, int64_t N, int64_t K,
                         int *watchdog, int num_sms, cudaStream_t st);
 
+// ---- gemm2.cu: the same matmul on CTA pairs (256 x 256 tiles, tcgen05 cta_group::2) ---------------
+bool gemm_pair_supported(int64_t M, int64_t N);
+cudaError_t launch_gemm_pair(const void *a_elems, const uint8_t *a_sc, int a_fmt, const float *ga,
+                             const void *b_elems, const uint8_t *b_sc, int b_fmt, const float *gb, void *c,
+                             int64_t M, int64_t N, int64_t K, int *watchdog, int num_sms, cudaStream_t st);
+
 // ---- api.cu --------------------------------------------------------------------------------------
 // Driver entry point for cuTensorMapEncodeTiled (resolved once, no libcuda link).
 void *tensor_map_encoder();

@@ -1,0 +1,154 @@
+// umma.cuh -- tcgen05 (5th-generation tensor core) wrappers shared by the block-scaled
+// matmul kernels: tensor-memory allocation, descriptors, the three block-scaled MMA kinds,
+// scale-factor copies into tensor memory, accumulator loads, and the banded tile order.
+#pragma once
+#include <cstdint>
+#include "ptx.cuh"
+
+namespace mxk {
+
+// MMA kinds: E4M3 x {E4M3, E2M1 expanded to bytes} with E8M0 scales per 32 (one scale
+// per row per K = 32 instruction); E2M1 x E2M1 packed with E8M0 scales per 32 (two per
+// K = 64 instruction); E2M1 x E2M1 packed with UE4M3 scales per 16 (four per K = 64).
+enum : int { KIND_F8F6F4 = 0, KIND_MXF4 = 1, KIND_NVF4 = 2 };
+
+// ---- tcgen05 wrappers -------------------------------------------------------------------
+// Tensor-memory allocation by one full warp.  With CG = 2 the instruction is collective
+// over the CTA pair: the warp with the same index in both CTAs executes it, and both pass
+// the same shared-memory offset for the returned address.
+template <int CG = 1>
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t ncols) {
+    if constexpr (CG == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    } else {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+}
+template <int CG = 1>
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    if constexpr (CG == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+    else
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Arrive once on `bar` when every tcgen05 operation this thread issued before has
+// completed.  The pair form arrives on the barrier at the same offset in each CTA of the
+// pair (mask 0b11).
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint64_t *bar) {
+    const uint16_t mask = 3;
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 ::"r"(smem_u32(bar)), "h"(mask) : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 format): start >> 4 in bits 0-13, leading
+// byte offset >> 4 in 16-29, stride byte offset >> 4 in 32-45, descriptor version 1 in
+// bits 46-47, swizzle mode in 61-63 (2 = 128-byte swizzle, 0 = none).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t swz) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)(swz & 7u) << 61;
+    return d;
+}
+
+// Instruction descriptor for the block-scaled kinds: B scale-factor id (first scale byte
+// of the 32-bit tensor-memory word) in bits 4-5, A format 7-9, B format 10-12 (mxf8f6f4:
+// E4M3 = 0, E2M1 = 5; mxf4 / mxf4nvf4: E2M1 = 1), K-major A and B, N >> 3 in 17-22, scale
+// type in bit 23 (1 = UE8M0, 0 = UE4M3), M >> 4 in 24-28, A scale-factor id in 29-30,
+// bit 31 = 0 (dense K of 32 for 8-bit kinds, 64 for 4-bit kinds).
+template <int BM, int BN, int KIND>
+__device__ __forceinline__ uint32_t mma_idesc(uint32_t b_fmt_code, uint32_t sf_id) {
+    const uint32_t a_fmt = KIND == KIND_F8F6F4 ? 0u : 1u;
+    const uint32_t b_fmt = KIND == KIND_F8F6F4 ? b_fmt_code : 1u;
+    uint32_t d = 0;
+    d |= (sf_id & 3u) << 4;
+    d |= a_fmt << 7;
+    d |= (b_fmt & 7u) << 10;
+    d |= (uint32_t)(BN >> 3) << 17;
+    d |= (KIND == KIND_NVF4 ? 0u : 1u) << 23;
+    d |= (uint32_t)(BM >> 4) << 24;
+    d |= (sf_id & 3u) << 29;
+    return d;
+}
+
+template <int KIND, int CG = 1>
+__device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    if constexpr (KIND == KIND_F8F6F4) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::%7.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "n"(CG)
+            : "memory");
+    } else if constexpr (KIND == KIND_MXF4) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::%7.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "n"(CG)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::%7.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+            ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem), "n"(CG)
+            : "memory");
+    }
+}
+
+// Copy a 512-byte scale atom (32 rows x 16 bytes, contiguous) into 4 TMEM columns,
+// replicated into all four 32-lane sub-partitions.
+// With CG = 2 (issued by the pair's MMA thread) each CTA's atom at the same shared-memory
+// offset goes to the same columns of that CTA's own tensor memory.
+template <int CG = 1>
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint32_t saddr) {
+    const uint64_t d = smem_desc(saddr, 16, 128, 0);
+    if constexpr (CG == 1)
+        asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+    else
+        asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---- tile order ------------------------------------------------------------------------------
+// Banded raster: N-tiles are grouped into bands of `band` tiles whose B panels fit in L2;
+// within a band the tiles run M-major, so concurrently resident CTAs share A panels and the
+// band's B panels are read from HBM about once.
+__device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int band, int &m_blk, int &n_blk) {
+    const int per_band = tiles_m * band;
+    const int b = t / per_band;
+    const int rem = t - b * per_band;
+    const int n0 = b * band;
+    const int bw = tiles_n - n0 < band ? tiles_n - n0 : band;   // the last band may be narrower
+    m_blk = rem / bw;
+    n_blk = n0 + (rem - m_blk * bw);
+}
+
+}  // namespace mxk

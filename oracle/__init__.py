@@ -27,8 +27,8 @@ _SRC = os.path.join(_HERE, "mx_oracle.c")
 _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 
 # Format and code-kind identifiers (the same numbering as mx_oracle.c).
-E4M3, E5M2, E2M1, NVFP4 = 0, 1, 2, 3
-K_E4M3, K_E5M2, K_E2M1, K_UE4M3, K_E8M0, K_BF16 = 0, 1, 2, 3, 4, 5
+E4M3, E5M2, E2M1, NVFP4, E2M3, E3M2, INT8 = 0, 1, 2, 3, 4, 5, 6
+K_E4M3, K_E5M2, K_E2M1, K_UE4M3, K_E8M0, K_BF16, K_E2M3, K_E3M2, K_INT8 = 0, 1, 2, 3, 4, 5, 6, 7, 8
 FLOOR, CEIL = 0, 1
 ROW, COL = 0, 1
 
@@ -92,7 +92,7 @@ def _check(rc: int, what: str):
 
 # ---------------------------------------------------------------- scalar codecs
 def decode(kind: int, code: int) -> float:
-    """Exact value of one code (E4M3, E5M2, E2M1, UE4M3, E8M0 or bf16 bits)."""
+    """Exact value of one code (E4M3, E5M2, E2M1, UE4M3, E8M0, bf16 bits, E2M3, E3M2 or INT8)."""
     return lib().mxo_decode(kind, code)
 
 

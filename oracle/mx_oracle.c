@@ -49,9 +49,10 @@
 #include <math.h>
 
 /* Format identifiers (shared numbering with the public ABI enum, an interface only). */
-enum { F_E4M3 = 0, F_E5M2 = 1, F_E2M1 = 2, F_NVFP4 = 3 };
+enum { F_E4M3 = 0, F_E5M2 = 1, F_E2M1 = 2, F_NVFP4 = 3, F_E2M3 = 4, F_E3M2 = 5, F_INT8 = 6 };
 /* Extra code kinds for mxo_decode / mxo_encode. */
-enum { K_E4M3 = 0, K_E5M2 = 1, K_E2M1 = 2, K_UE4M3 = 3, K_E8M0 = 4, K_BF16 = 5 };
+enum { K_E4M3 = 0, K_E5M2 = 1, K_E2M1 = 2, K_UE4M3 = 3, K_E8M0 = 4, K_BF16 = 5, K_E2M3 = 6, K_E3M2 = 7,
+       K_INT8 = 8 };
 enum { R_FLOOR = 0, R_CEIL = 1 };
 
 /* ------------------------------------------------------------------------- */
@@ -62,6 +63,12 @@ enum { R_FLOOR = 0, R_CEIL = 1 };
 /*   E5M2: 1 sign, 5 exponent, 2 mantissa bits, bias 15, IEEE-like Inf/NaN,   */
 /*         max 1.75 * 2^15 = 57344                                            */
 /*   E8M0: 8 exponent bits, bias 127, 0xFF = NaN, no Inf (Q§2)                */
+/*   MXFP6 / MXINT8 element formats (Q§2 lists them as MX family members with */
+/*   6.25 and 8.25 effective bits; their parameters are the OCP MX ones):     */
+/*   E2M3: 1 sign, 2 exponent, 3 mantissa bits, bias 1, no Inf/NaN, max 7.5   */
+/*   E3M2: 1 sign, 3 exponent, 2 mantissa bits, bias 3, no Inf/NaN, max 28    */
+/*   INT8: two's complement q with an implicit factor 2^-6 (value q/64),      */
+/*         symmetric range -127 .. 127 (max 127/64)                           */
 /* ------------------------------------------------------------------------- */
 typedef struct {
     int ebits, mbits, bias;
@@ -78,6 +85,8 @@ static fmt_t fmt_of(int kind) {
     case K_UE4M3: f.ebits = 4; f.mbits = 3; f.bias = 7;  f.has_sign = 0; f.nan_all_ones = 1; break;
     case K_E5M2:  f.ebits = 5; f.mbits = 2; f.bias = 15; f.has_sign = 1; f.ieee_special = 1; break;
     case K_E2M1:  f.ebits = 2; f.mbits = 1; f.bias = 1;  f.has_sign = 1; break;
+    case K_E2M3:  f.ebits = 2; f.mbits = 3; f.bias = 1;  f.has_sign = 1; break;
+    case K_E3M2:  f.ebits = 3; f.mbits = 2; f.bias = 3;  f.has_sign = 1; break;
     case K_BF16:  f.ebits = 8; f.mbits = 7; f.bias = 127; f.has_sign = 1; f.ieee_special = 1; break;
     default: break;
     }
@@ -105,7 +114,7 @@ static unsigned max_code(fmt_t f) {
     unsigned emask = (1u << f.ebits) - 1u, mmask = (1u << f.mbits) - 1u;
     if (f.nan_all_ones) return (emask << f.mbits) | (mmask - 1u);       /* S.1111.110 */
     if (f.ieee_special) return ((emask - 1u) << f.mbits) | mmask;        /* S.11110.11 */
-    return (emask << f.mbits) | mmask;                                  /* E2M1 0.11.1 */
+    return (emask << f.mbits) | mmask;                   /* no specials: all ones (E2M1 0.11.1) */
 }
 
 /* Split a finite positive double into integer significand M and exponent x:  a = M * 2^x. */
@@ -184,6 +193,7 @@ static double decode_e8m0(unsigned c) { return c == 0xFFu ? NAN : ldexp(1.0, (in
 
 double mxo_decode(int kind, unsigned code) {
     if (kind == K_E8M0) return decode_e8m0(code & 0xFFu);
+    if (kind == K_INT8) return ldexp((double)(int8_t)(uint8_t)code, -6);
     return decode_sem(fmt_of(kind), code);
 }
 
@@ -195,10 +205,20 @@ unsigned mxo_encode(double v, int kind) {
         if (isinf(v)) return v > 0 ? 0x7F80u : 0xFF80u;
         return encode_sem(f, v, 1);
     }
+    if (kind == K_INT8) {
+        /* round half to even onto the integers q/64, saturating symmetrically at +-127 */
+        if (isnan(v)) return 0u;
+        double q = v * 64.0;                             /* exact: a power-of-two multiply */
+        long iq = fabs(q) >= 127.5 ? (q > 0 ? 127 : -127) : (long)rint(q);
+        if (iq > 127) iq = 127;
+        if (iq < -127) iq = -127;
+        return (unsigned)(uint8_t)(int8_t)iq;
+    }
     if (isnan(v)) {
         unsigned nbits = (unsigned)(f.has_sign + f.ebits + f.mbits);
         unsigned s = signbit(v) ? (1u << (nbits - 1)) : 0u;
-        if (kind == K_E2M1) return s | max_code(f);      /* no NaN in E2M1: +-6 */
+        if (kind == K_E2M1 || kind == K_E2M3 || kind == K_E3M2)
+            return s | max_code(f);                      /* no NaN in E2M1 / FP6: +-max */
         if (kind == K_UE4M3) return 0x7Fu;
         return s | 0x7Fu;                                /* E4M3 / E5M2 NaN */
     }
@@ -216,10 +236,20 @@ static uint16_t f32_to_bf16(float y) { return (uint16_t)mxo_encode((double)y, K_
 /* ------------------------------------------------------------------------- */
 
 /* Exponent of the element format's largest binade and its largest finite value. */
-static int emax_of(int fmt) { return fmt == F_E4M3 ? 8 : fmt == F_E5M2 ? 15 : 2; }
+static int emax_of(int fmt) {
+    switch (fmt) {
+    case F_E4M3: return 8;     /* 448   = 1.75   x 2^8  */
+    case F_E5M2: return 15;    /* 57344 = 1.75   x 2^15 */
+    case F_E2M3: return 2;     /* 7.5   = 1.875  x 2^2  */
+    case F_E3M2: return 4;     /* 28    = 1.75   x 2^4  */
+    case F_INT8: return 0;     /* 127/64 = 1.984375 x 2^0 */
+    default:     return 2;     /* E2M1: 6 = 1.5 x 2^2 */
+    }
+}
+static int elem_kind(int fmt);
 static double maxval_of(int fmt) {
-    int kind = fmt == F_E4M3 ? K_E4M3 : fmt == F_E5M2 ? K_E5M2 : K_E2M1;
-    fmt_t f = fmt_of(kind);
+    if (fmt == F_INT8) return 127.0 / 64.0;
+    fmt_t f = fmt_of(elem_kind(fmt));
     return decode_sem(f, max_code(f));
 }
 
@@ -256,7 +286,18 @@ int mxo_scale_exponent(double amax, int fmt, int rounding) {
 /* MX block quantisation (Q§2, Q§4): block of 32, E8M0 scale, RNE+saturate.   */
 /* ------------------------------------------------------------------------- */
 
-static int elem_kind(int fmt) { return fmt == F_E4M3 ? K_E4M3 : fmt == F_E5M2 ? K_E5M2 : K_E2M1; }
+static int elem_kind(int fmt) {
+    switch (fmt) {
+    case F_E4M3: return K_E4M3;
+    case F_E5M2: return K_E5M2;
+    case F_E2M3: return K_E2M3;
+    case F_E3M2: return K_E3M2;
+    case F_INT8: return K_INT8;
+    default:     return K_E2M1;
+    }
+}
+/* Element formats of the MX family (block 32, E8M0 scale): E4M3, E5M2, E2M1, E2M3, E3M2, INT8. */
+static int mx_fmt_ok(int fmt) { return (fmt >= F_E4M3 && fmt <= F_E2M1) || (fmt >= F_E2M3 && fmt <= F_INT8); }
 
 /* Quantise one block of n bf16 values; writes n codes (one per entry) and returns the
  * E8M0 scale byte. */
@@ -280,7 +321,8 @@ static unsigned quantize_block_mx(const uint16_t *x, int n, int fmt, int roundin
     return (unsigned)(s + 127);
 }
 
-/* Store code i of a row into an output row (FP8: one byte; FP4: nibble, even low). */
+/* Store code i of a row into an output row (FP8, FP6 in the low 6 bits, INT8: one byte;
+ * FP4: nibble, even low). */
 static void put_code(uint8_t *row, int64_t i, unsigned code, int fp4) {
     if (!fp4) { row[i] = (uint8_t)code; return; }
     uint8_t *p = row + i / 2;
@@ -305,7 +347,7 @@ int mxo_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int 
     const int B = 32;
     int fp4 = (fmt == F_E2M1);
     int64_t out_rows = axis == 0 ? rows : cols, out_cols = axis == 0 ? cols : rows;
-    if (fmt < 0 || fmt > 2 || out_cols % B) return -1;
+    if (!mx_fmt_ok(fmt) || out_cols % B) return -1;
     uint16_t blk[32];
     unsigned codes[32];
     int64_t row_bytes = fp4 ? out_cols / 2 : out_cols;
@@ -326,7 +368,7 @@ int mxo_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int 
 /* Direct element cast with no block scale (the "direct cast" of [P4]). */
 int mxo_cast(const uint16_t *x, int64_t n, int fmt, uint8_t *out) {
     int fp4 = (fmt == F_E2M1);
-    if (fmt < 0 || fmt > 2 || (fp4 && n % 2)) return -1;
+    if (!mx_fmt_ok(fmt) || fmt == F_INT8 || (fp4 && n % 2)) return -1;   /* INT8 needs a scale */
     memset(out, 0, (size_t)(fp4 ? n / 2 : n));
     for (int64_t i = 0; i < n; i++) put_code(out, i, mxo_encode(bf16_value(x[i]), elem_kind(fmt)), fp4);
     return 0;
@@ -409,7 +451,7 @@ int mxo_dequantize_mx(const uint8_t *elems, const uint8_t *scales, int64_t rows,
                       int fmt, uint16_t *out) {
     const int B = 32;
     int fp4 = (fmt == F_E2M1);
-    if (fmt < 0 || fmt > 2 || cols % B) return -1;
+    if (!mx_fmt_ok(fmt) || cols % B) return -1;
     int64_t row_bytes = fp4 ? cols / 2 : cols;
     for (int64_t r = 0; r < rows; r++) {
         for (int64_t j = 0; j < cols; j++) {

@@ -62,17 +62,25 @@ def test_effective_bits(oracle):
         assert (e.nbytes + s.nbytes) * 8 / n == g["bits_mxfp8"][0]
     e, s, _ = oracle.quantize_nvfp4(x)
     assert (e.nbytes + s.nbytes) * 8 / n == g["bits_nvfp4"][0]
+    # MXFP6: 6-bit codes (stored one per byte here) plus the shared scale
+    for fmt in (oracle.E2M3, oracle.E3M2):
+        e, s = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.FLOOR)
+        assert int(e.max()) < 64
+        assert (6 * e.size + 8 * s.nbytes) / n == g["bits_mxfp6"][0]
+    e, s = oracle.quantize_mx(x, oracle.INT8, oracle.ROW, oracle.FLOOR)
+    assert (e.nbytes + s.nbytes) * 8 / n == g["bits_mxint8"][0]
 
 
 # ------------------------------------------------------------------ block assembly
-@pytest.mark.parametrize("fmt_name,rounding", [("E4M3", 1), ("E4M3", 0), ("E5M2", 1), ("E2M1", 0), ("E2M1", 1)])
+@pytest.mark.parametrize("fmt_name,rounding", [("E4M3", 1), ("E4M3", 0), ("E5M2", 1), ("E2M1", 0), ("E2M1", 1),
+                                               ("E2M3", 0), ("E2M3", 1), ("E3M2", 0), ("E3M2", 1)])
 def test_block_codes_are_the_cast_of_scaled_values(oracle, fmt_name, rounding):
     """Each block's codes equal the (brute-force-pinned) direct cast of x * 2^-s, with s
     read back from the E8M0 byte, and the scaled maximum lands per its school."""
     fmt = getattr(oracle, fmt_name)
     x = synth.mx8_rowwise(16, 128, seed=5)
     e, s = oracle.quantize_mx(x, fmt, oracle.ROW, rounding)
-    maxv = {"E4M3": 448.0, "E5M2": 57344.0, "E2M1": 6.0}[fmt_name]
+    maxv = {"E4M3": 448.0, "E5M2": 57344.0, "E2M1": 6.0, "E2M3": 7.5, "E3M2": 28.0}[fmt_name]
     xf = bf16_bits_to_f64(x)
     fp4 = fmt_name == "E2M1"
     for r in range(x.shape[0]):
@@ -90,7 +98,31 @@ def test_block_codes_are_the_cast_of_scaled_values(oracle, fmt_name, rounding):
             if rounding == 1:
                 assert maxv / 2 < top <= maxv
             else:
-                assert 2.0 ** {"E4M3": 8, "E5M2": 15, "E2M1": 2}[fmt_name] <= top
+                assert 2.0 ** {"E4M3": 8, "E5M2": 15, "E2M1": 2, "E2M3": 2, "E3M2": 4}[fmt_name] <= top
+
+
+@pytest.mark.parametrize("rounding", [0, 1])
+def test_int8_block_codes(oracle, rounding):
+    """MXINT8 blocks: codes are the saturating RNE of x * 2^-s * 64 (the pinned element
+    encoder) and the scaled maximum lands per its school ([1, 2) floor; (127/128, 127/64]
+    no-clip)."""
+    x = synth.mx8_rowwise(8, 128, seed=6)
+    e, s = oracle.quantize_mx(x, oracle.INT8, oracle.ROW, rounding)
+    xf = bf16_bits_to_f64(x)
+    for r in range(x.shape[0]):
+        for b in range(4):
+            sc = int(s[r, b]) - 127
+            scaled = np.ldexp(xf[r, 32 * b:32 * b + 32], -sc)
+            ref = [oracle.encode(float(v), oracle.K_INT8) for v in scaled]
+            assert list(e[r, 32 * b:32 * b + 32]) == ref
+            top = np.abs(scaled).max()
+            if rounding == 1:
+                assert 127 / 128 < top <= 127 / 64
+            else:
+                assert 1.0 <= top < 2.0
+    d = bf16_bits_to_f64(oracle.dequantize_mx(e, s, 8, 128, oracle.INT8))
+    q = e.view(np.int8).astype(np.float64) / 64.0
+    assert np.array_equal(d, q * np.ldexp(1.0, np.repeat(s.astype(np.int64) - 127, 32, axis=1)))
 
 
 def test_fp4_nibble_order(oracle):

@@ -2,8 +2,9 @@
 library routines fix (no GPU).
 
 Independent references used here: torch's float8_e4m3fn / float8_e5m2 / float8_e8m0fnu
-dtypes and ml_dtypes' float4_e2m1fn (library decoders and RNE converters), math.ldexp,
-and a brute-force nearest-code search written over the decoded code tables.
+dtypes and ml_dtypes' float4_e2m1fn / float6_e2m3fn / float6_e3m2fn (library decoders and
+RNE converters), math.ldexp, and a brute-force nearest-code search written over the
+decoded code tables.
 """
 import math
 
@@ -32,6 +33,10 @@ def library_decode_table(kind, o):
         return torch.arange(256, dtype=torch.uint8).view(torch.float8_e8m0fnu).double().numpy()
     if kind == o.K_E2M1:
         return np.arange(16, dtype=np.uint8).view(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    if kind == o.K_E2M3:
+        return np.arange(64, dtype=np.uint8).view(ml_dtypes.float6_e2m3fn).astype(np.float64)
+    if kind == o.K_E3M2:
+        return np.arange(64, dtype=np.uint8).view(ml_dtypes.float6_e3m2fn).astype(np.float64)
     raise ValueError(kind)
 
 
@@ -55,7 +60,7 @@ def test_e2m1_value_set_matches_page(oracle):
     assert max(vals) == g["max"][0]
 
 
-@pytest.mark.parametrize("name", ["K_E4M3", "K_E5M2", "K_E2M1", "K_E8M0"])
+@pytest.mark.parametrize("name", ["K_E4M3", "K_E5M2", "K_E2M1", "K_E8M0", "K_E2M3", "K_E3M2"])
 def test_decode_tables_match_library(oracle, name):
     kind = getattr(oracle, name)
     ref = library_decode_table(kind, oracle)
@@ -115,17 +120,19 @@ def brute_force_cast(x, table, mag_codes, sign_bit, nan_code_pos, nan_sign=True)
     return code
 
 
-@pytest.mark.parametrize("fmt_name", ["E4M3", "E5M2", "E2M1"])
+@pytest.mark.parametrize("fmt_name", ["E4M3", "E5M2", "E2M1", "E2M3", "E3M2"])
 def test_exhaustive_bf16_cast_against_brute_force(oracle, fmt_name):
     fmt = getattr(oracle, fmt_name)
-    kind = {"E4M3": oracle.K_E4M3, "E5M2": oracle.K_E5M2, "E2M1": oracle.K_E2M1}[fmt_name]
+    kind = getattr(oracle, "K_" + fmt_name)
     table = library_decode_table(kind, oracle)
     if fmt_name == "E4M3":
         mag_codes, sign_bit, nan_pos = np.arange(0x7F), 0x80, 0x7F
     elif fmt_name == "E5M2":
         mag_codes, sign_bit, nan_pos = np.arange(0x7C), 0x80, 0x7F
-    else:
+    elif fmt_name == "E2M1":
         mag_codes, sign_bit, nan_pos = np.arange(8), 0x8, 0x7   # no NaN: reading is +-6
+    else:
+        mag_codes, sign_bit, nan_pos = np.arange(32), 0x20, 0x1F  # FP6: no NaN, reading +-max
     x = bf16_bits_to_f64(ALL_BF16)
     ref = brute_force_cast(x, table, mag_codes, sign_bit, nan_pos)
     got = oracle.cast(ALL_BF16, fmt)
@@ -144,6 +151,41 @@ def test_cast_matches_torch_in_range(oracle, fmt_name, dtype, maxv):
     ref = torch.from_numpy(x32[ok]).to(dtype).view(torch.uint8).numpy()
     got = oracle.cast(ALL_BF16[ok], getattr(oracle, fmt_name))
     assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("fmt_name,dtype,maxv", [("E2M3", ml_dtypes.float6_e2m3fn, 7.5),
+                                                 ("E3M2", ml_dtypes.float6_e3m2fn, 28.0)])
+def test_fp6_cast_matches_ml_dtypes_in_range(oracle, fmt_name, dtype, maxv):
+    """ml_dtypes' FP6 conversion (round to nearest even) agrees with ours up to the max."""
+    x32 = bf16_bits_to_f64(ALL_BF16).astype(np.float32)
+    ok = np.isfinite(x32) & (np.abs(x32) <= maxv)
+    ref = x32[ok].astype(dtype).view(np.uint8) & 0x3F
+    got = oracle.cast(ALL_BF16[ok], getattr(oracle, fmt_name))
+    assert np.array_equal(got, ref)
+
+
+def test_int8_element_definition(oracle):
+    """MXINT8 element: two's complement q read as q / 64, encoded by round half to even
+    onto that grid and saturated symmetrically at +-127 (brute force over the 255 values)."""
+    codes = np.arange(256)
+    vals = np.array([oracle.decode(oracle.K_INT8, int(c)) for c in codes])
+    assert np.array_equal(vals, codes.astype(np.uint8).view(np.int8).astype(np.float64) / 64.0)
+    grid = np.arange(-127, 128, dtype=np.float64) / 64.0
+    x = bf16_bits_to_f64(ALL_BF16)
+    fin = np.isfinite(x)
+    xs = x[fin]
+    # beyond +-4 the nearest grid point is the end point; clipping keeps the distances exact
+    d = np.abs(np.clip(xs, -4.0, 4.0)[:, None] - grid[None, :])
+    best = d.min(axis=1)
+    cand = d == best[:, None]
+    q = np.arange(-127, 128)
+    # ties: the even integer; beyond the range the end point is nearest anyway
+    pick = np.where(cand.sum(axis=1) > 1, np.argmax(cand & (q[None, :] % 2 == 0), axis=1), np.argmax(cand, axis=1))
+    ref = (q[pick].astype(np.int64) & 0xFF)
+    got = np.array([oracle.encode(float(v), oracle.K_INT8) for v in xs])
+    assert np.array_equal(got, ref)
+    assert oracle.encode(math.inf, oracle.K_INT8) == 127 and oracle.encode(-math.inf, oracle.K_INT8) == 0x81
+    assert oracle.encode(-1e-9, oracle.K_INT8) == 0     # no negative zero in two's complement
 
 
 def test_e2m1_cast_matches_ml_dtypes_in_range(oracle):
@@ -180,7 +222,8 @@ def positive_finite_bf16():
     return b, bf16_bits_to_f64(b)
 
 
-@pytest.mark.parametrize("fmt_name,emax,maxv", [("E4M3", 8, 448.0), ("E5M2", 15, 57344.0), ("E2M1", 2, 6.0)])
+@pytest.mark.parametrize("fmt_name,emax,maxv", [("E4M3", 8, 448.0), ("E5M2", 15, 57344.0), ("E2M1", 2, 6.0),
+                                                ("E2M3", 2, 7.5), ("E3M2", 4, 28.0), ("INT8", 0, 127 / 64)])
 def test_floor_school_landing_interval(oracle, fmt_name, emax, maxv):
     """Floor school: scaled block maximum in [2^emax, 2^(emax+1)) -- [4, 8) for E2M1."""
     g = read_golden("format_constants.txt")
@@ -198,7 +241,8 @@ def test_floor_school_landing_interval(oracle, fmt_name, emax, maxv):
         assert s == math.frexp(a)[1] - 1 - emax
 
 
-@pytest.mark.parametrize("fmt_name,maxv", [("E4M3", 448.0), ("E5M2", 57344.0), ("E2M1", 6.0)])
+@pytest.mark.parametrize("fmt_name,maxv", [("E4M3", 448.0), ("E5M2", 57344.0), ("E2M1", 6.0), ("E2M3", 7.5),
+                                           ("E3M2", 28.0), ("INT8", 127 / 64)])
 def test_ceil_school_landing_interval(oracle, fmt_name, maxv):
     """No-clip school: scaled maximum in (max/2, max] -- (3, 6] for E2M1 -- and the
     scale is the smallest one that does not clip."""
@@ -210,6 +254,9 @@ def test_ceil_school_landing_interval(oracle, fmt_name, maxv):
     for a in amax:
         s = oracle.scale_exponent(a, fmt, oracle.CEIL)
         scaled = math.ldexp(a, -s)
+        if s == 127:                    # clamped to the E8M0 range (INT8 at the largest bf16)
+            assert math.ldexp(a, -128) <= maxv
+            continue
         assert scaled <= maxv, (a, s)
         if s > -127:
             assert maxv / 2 < scaled, (a, s)
