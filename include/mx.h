@@ -65,8 +65,14 @@ typedef enum {
     MX_FMT_E4M3 = 0,     /* MXFP8, E4M3 elements, block 32, E8M0 scale */
     MX_FMT_E5M2 = 1,     /* MXFP8, E5M2 elements, block 32, E8M0 scale */
     MX_FMT_E2M1 = 2,     /* MXFP4, E2M1 elements, block 32, E8M0 scale */
-    MX_FMT_NVFP4 = 3     /* NVFP4, E2M1 elements, block 16, UE4M3 scale, fp32 tensor scale */
+    MX_FMT_NVFP4 = 3,    /* NVFP4, E2M1 elements, block 16, UE4M3 scale, fp32 tensor scale */
+    MX_FMT_E2M3 = 4,     /* MXFP6, E2M3 elements (max 7.5), block 32, E8M0 scale */
+    MX_FMT_E3M2 = 5,     /* MXFP6, E3M2 elements (max 28), block 32, E8M0 scale */
+    MX_FMT_INT8 = 6      /* MXINT8, int8 q read as q / 64 (-127 .. 127), block 32, E8M0 scale */
 } mx_fmt;
+/* Storage: FP8 and INT8 codes take one byte; FP6 codes take one byte each (the 6-bit code
+ * in the low bits, the top two bits zero); FP4 codes pack two per byte, the even element
+ * in the low nibble. */
 
 typedef enum {
     MX_AXIS_ROW = 0,     /* blocks run along a row (contiguous elements) */
@@ -93,15 +99,18 @@ typedef enum {
 int64_t mx_scale_bytes(int64_t rows, int64_t scale_cols, mx_scale_layout layout);
 
 /*
- * mx_quantize -- quantise a bf16 matrix to MXFP8 / MXFP4 / NVFP4 ([Q] §2, §3, §4).
+ * mx_quantize -- quantise a bf16 matrix to MXFP8 / MXFP6 / MXFP4 / MXINT8 / NVFP4
+ * ([Q] §2 and its MX family table, §3, §4).
  *   src_bf16    device, rows x cols bf16 row-major, 16-byte aligned.
- *   fmt         MX_FMT_E4M3 / E5M2 / E2M1 (block 32, E8M0) or MX_FMT_NVFP4 (block 16).
+ *   fmt         MX_FMT_E4M3 / E5M2 / E2M3 / E3M2 / E2M1 / INT8 (block 32, E8M0) or
+ *               MX_FMT_NVFP4 (block 16).
  *   axis        ROW: blocks along rows; output rows x cols, scales rows x cols/B.
  *               COL: blocks down columns; output is the transposed matrix cols x rows
  *               (K-major for a weight-gradient matmul), scales cols x rows/B.
  *               NVFP4 supports ROW only.
  *   rounding    shared-exponent rule (ignored for NVFP4).
- *   out_elems   device, 16-byte aligned; out_rows x out_cols bytes (FP8) or x out_cols/2 (FP4).
+ *   out_elems   device, 16-byte aligned; out_rows x out_cols bytes (FP8, FP6, INT8) or
+ *               x out_cols/2 (FP4).
  *   out_scales  device; first scale layout (the lower set bit of `layout`).
  *   layout      ROWMAJOR, TCGEN05 or both; with both, out_scales gets ROWMAJOR and
  *               out_scales_alt gets TCGEN05 (else out_scales_alt must be NULL).
@@ -158,7 +167,8 @@ mx_status mx_quantize_nvfp4_noalloc(const void *src_bf16, int64_t rows, int64_t 
  *   row_elems / row_scales   as mx_quantize(axis = ROW).
  *   col_elems / col_scales   as mx_quantize(axis = COL): cols x rows, scales cols x rows/32.
  *   layout      exactly one of ROWMAJOR / TCGEN05, used for both scale outputs.
- *   fmt         E4M3, E5M2 or E2M1.  rows and cols are multiples of 32.
+ *   fmt         any MX format (E4M3, E5M2, E2M3, E3M2, E2M1, INT8).  rows and cols are
+ *               multiples of 32.
  */
 mx_status mx_quantize_dual(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt fmt,
                            mx_scale_rounding rounding, void *row_elems, uint8_t *row_scales,
@@ -181,7 +191,8 @@ mx_status mx_dequantize(const void *elems, const uint8_t *scales, const float *g
 /*
  * mx_cast -- the direct cast of [P4] "MXFP4": each bf16 value cast to the element format
  * with no block scale (RNE, saturating).  NaN becomes 0x7F|sign (E4M3, E5M2) or the
- * signed maximum 0x7|sign (E2M1, which has no NaN).
+ * signed maximum 0x7|sign (E2M1) / 0x1F|sign (E2M3, E3M2), formats without NaN.  INT8
+ * needs a scale and is not a cast target (MX_ERR_ARG).
  *   n           element count (even for E2M1); src and out 16-byte aligned.
  */
 mx_status mx_cast(const void *src_bf16, int64_t n, mx_fmt fmt, void *out_elems, mx_stream_t stream);
@@ -190,7 +201,7 @@ mx_status mx_cast(const void *src_bf16, int64_t n, mx_fmt fmt, void *out_elems, 
  * One operand of the block-scaled matmul: a rows x K matrix of codes, K-major (each row
  * holds K consecutive codes; FP4 packed two per byte), with its block scales in the TCGEN05
  * layout exactly as mx_quantize(axis = ROW, layout = TCGEN05) writes them: E8M0 per 32
- * along K (rows x K/32) for E4M3 / E2M1, UE4M3 per 16 along K (rows x K/16) for NVFP4.
+ * along K (rows x K/32) for the MX formats, UE4M3 per 16 along K (rows x K/16) for NVFP4.
  *   global_scale  NVFP4 only: device pointer to the operand's fp32 per-tensor scale g (as
  *                 written by mx_quantize); NULL for MX operands.
  */
@@ -208,9 +219,11 @@ typedef struct {
  *   NVFP4: C[m, n] = gA gB sum_k dec(A[m,k]) dec(sA[m,k/16]) dec(B[n,k]) dec(sB[n,k/16])
  * accumulated in fp32 on the tensor cores (the NVFP4 product gA gB is applied to the fp32
  * sum), written as bf16 (RNE).
- *   Format pairs (A, B): (E4M3, E4M3), (E4M3, E2M1) -- activations x weights -- and
- *   (E2M1, E2M1), (NVFP4, NVFP4); any other pair, or a global_scale that is missing for
- *   NVFP4 or present for MX, is MX_ERR_ARG.
+ *   Format pairs (A, B): A in {E4M3, E5M2, E2M3, E3M2} with B in {E4M3, E5M2, E2M3, E3M2,
+ *   E2M1} (FP8 / FP6 run at the FP8 rate, [Q] §7) -- e.g. activations x MXFP4 weights --
+ *   and (E2M1, E2M1), (NVFP4, NVFP4) at the FP4 rate; any other pair (INT8 has no
+ *   block-scaled tensor-core form), or a global_scale that is missing for NVFP4 or
+ *   present for MX, is MX_ERR_ARG.
  *   C_bf16      device, M x N row-major bf16, 16-byte aligned.
  *   Shapes: M and N multiples of 128; K a multiple of 128 (8-bit A) or 256 (FP4 x FP4)
  *   (else MX_ERR_SHAPE).

@@ -13,7 +13,7 @@ LIB_PATH = os.environ.get("MX_LIB_PATH") or os.path.join(_PKG, "libmx.so")
 
 # enum values of include/mx.h
 MX_OK, MX_ERR_ARG, MX_ERR_SHAPE, MX_ERR_ALIGN, MX_ERR_LAYOUT, MX_ERR_CUDA, MX_ERR_TIMEOUT = range(7)
-MX_FMT_E4M3, MX_FMT_E5M2, MX_FMT_E2M1, MX_FMT_NVFP4 = 0, 1, 2, 3
+MX_FMT_E4M3, MX_FMT_E5M2, MX_FMT_E2M1, MX_FMT_NVFP4, MX_FMT_E2M3, MX_FMT_E3M2, MX_FMT_INT8 = 0, 1, 2, 3, 4, 5, 6
 MX_AXIS_ROW, MX_AXIS_COL = 0, 1
 MX_SCALE_FLOOR_OCP, MX_SCALE_CEIL_RECIPE = 0, 1
 MX_LAYOUT_ROWMAJOR, MX_LAYOUT_TCGEN05 = 1, 2

@@ -10,7 +10,8 @@ import torch
 
 from . import _lib as L
 
-FMTS = {"e4m3": L.MX_FMT_E4M3, "e5m2": L.MX_FMT_E5M2, "e2m1": L.MX_FMT_E2M1, "nvfp4": L.MX_FMT_NVFP4}
+FMTS = {"e4m3": L.MX_FMT_E4M3, "e5m2": L.MX_FMT_E5M2, "e2m1": L.MX_FMT_E2M1, "nvfp4": L.MX_FMT_NVFP4,
+        "e2m3": L.MX_FMT_E2M3, "e3m2": L.MX_FMT_E3M2, "int8": L.MX_FMT_INT8}
 ROUNDING = {"floor": L.MX_SCALE_FLOOR_OCP, "ceil": L.MX_SCALE_CEIL_RECIPE}
 LAYOUTS = {"rowmajor": L.MX_LAYOUT_ROWMAJOR, "tcgen05": L.MX_LAYOUT_TCGEN05,
            "both": L.MX_LAYOUT_ROWMAJOR | L.MX_LAYOUT_TCGEN05}

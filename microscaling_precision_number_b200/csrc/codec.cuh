@@ -18,14 +18,19 @@
 
 namespace mxk {
 
-enum : int { FMT_E4M3 = 0, FMT_E5M2 = 1, FMT_E2M1 = 2, FMT_NVFP4 = 3 };
+enum : int { FMT_E4M3 = 0, FMT_E5M2 = 1, FMT_E2M1 = 2, FMT_NVFP4 = 3, FMT_E2M3 = 4, FMT_E3M2 = 5, FMT_INT8 = 6 };
 
 // Exponent of the largest binade of the element format (448 = 1.75 * 2^8,
-// 57344 = 1.75 * 2^15, 6 = 1.5 * 2^2) and 128 x the significand of its maximum.
+// 57344 = 1.75 * 2^15, 6 = 1.5 * 2^2, 7.5 = 1.875 * 2^2, 28 = 1.75 * 2^4,
+// INT8 127/64 = 1.984375 * 2^0) and 128 x the significand of its maximum.
 __host__ __device__ constexpr int emax_elem(int fmt) {
-    return fmt == FMT_E4M3 ? 8 : (fmt == FMT_E5M2 ? 15 : 2);
+    return fmt == FMT_E4M3 ? 8 : fmt == FMT_E5M2 ? 15 : fmt == FMT_E3M2 ? 4 : fmt == FMT_INT8 ? 0 : 2;
 }
-__host__ __device__ constexpr int max_sig128(int fmt) { return fmt == FMT_E2M1 ? 192 : 224; }
+__host__ __device__ constexpr int max_sig128(int fmt) {
+    return fmt == FMT_E2M1 ? 192 : fmt == FMT_E2M3 ? 240 : fmt == FMT_INT8 ? 254 : 224;
+}
+// Element formats stored one code per byte (FP8, FP6 in the low 6 bits, INT8).
+__host__ __device__ constexpr bool byte_codes(int fmt) { return fmt != FMT_E2M1 && fmt != FMT_NVFP4; }
 
 // E8M0 code from the block maximum given as |x| bf16 bits (0 .. 0x7FFF).  Any
 // magnitude >= 0x7F80 (Inf or NaN) yields the NaN scale 0xFF.  A zero block yields
@@ -52,14 +57,15 @@ __device__ __noinline__ uint32_t e8m0_from_amax_bits_rare(uint32_t a) {
 
 // Common case, a normal block maximum (0x80 <= a < 0x7F80): the code is the biased
 // exponent field minus emax_elem (plus one under the no-clip rule when the maximum's
-// significand exceeds the element format's largest), floored at 0.  It never exceeds
-// 253, so e8m0_inverse_multiplier's first branch applies.  Zero, subnormal and Inf/NaN
-// maxima take the general path above (the two agree on every normal a).
+// significand exceeds the element format's largest), clamped to [0, 254] (the upper
+// clamp only binds for INT8, whose emax_elem is 0).  Zero, subnormal and Inf/NaN maxima
+// take the general path above (the two agree on every normal a).
 template <int FMT, bool CEIL>
 __device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t a) {
     if (__builtin_expect(a - 0x80u >= 0x7F00u, 0)) return e8m0_from_amax_bits_rare<FMT, CEIL>(a);
     int code = (int)(a >> 7) - emax_elem(FMT);
     if (CEIL) code += (int)((a & 0x7Fu) > (uint32_t)(max_sig128(FMT) - 128));
+    if constexpr (emax_elem(FMT) == 0) code = code > 254 ? 254 : code;
     return (uint32_t)(code < 0 ? 0 : code);
 }
 
@@ -96,14 +102,28 @@ __device__ __forceinline__ uint32_t finite_abs_max_bf16x8(const uint4 &v) {
 }
 
 // ---- hardware conversions (round to nearest even, satfinite) ---------------------------
-// Two fp32 -> two FP8 codes in one 16-bit word, `lo` in the low byte.
+// Two fp32 -> two byte codes in one 16-bit word, `lo` in the low byte: FP8, FP6 (6-bit
+// code in the low bits of its byte) by the hardware conversion; INT8 as the MXINT8
+// element (the value times 64, rounded half to even, saturated to -127 .. 127).
 template <int FMT>
 __device__ __forceinline__ uint32_t cvt_fp8x2(float lo, float hi) {
     uint16_t r;
     if constexpr (FMT == FMT_E4M3)
         asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    else
+    else if constexpr (FMT == FMT_E5M2)
         asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    else if constexpr (FMT == FMT_E2M3)
+        asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    else if constexpr (FMT == FMT_E3M2)
+        asm("cvt.rn.satfinite.e3m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    else {
+        int32_t a, b;
+        asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(a) : "f"(__fmul_rn(lo, 64.0f)));
+        asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(b) : "f"(__fmul_rn(hi, 64.0f)));
+        a = max(a, -127);
+        b = max(b, -127);
+        return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8);
+    }
     return (uint32_t)r;
 }
 
@@ -130,15 +150,25 @@ __device__ __forceinline__ uint2 cvt_fp8x8(const float (&x)[8]) {
     return r;
 }
 
-// Two FP8 codes (16-bit word, element 2i low) -> two fp32, exact (via f16x2).
+// Two byte codes (16-bit word, element 2i low) -> two fp32, exact (FP8 / FP6 via f16x2;
+// INT8 as q / 64).
 template <int FMT>
 __device__ __forceinline__ void fp8x2_to_f32(uint32_t codes16, float &lo, float &hi) {
+    if constexpr (FMT == FMT_INT8) {
+        lo = __fmul_rn((float)(int8_t)(codes16 & 0xFFu), 0.015625f);
+        hi = __fmul_rn((float)(int8_t)((codes16 >> 8) & 0xFFu), 0.015625f);
+        return;
+    }
     uint32_t h2;
     uint16_t c = (uint16_t)codes16;
     if constexpr (FMT == FMT_E4M3)
         asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
-    else
+    else if constexpr (FMT == FMT_E5M2)
         asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h2) : "h"(c));
+    else if constexpr (FMT == FMT_E2M3)
+        asm("cvt.rn.f16x2.e2m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    else
+        asm("cvt.rn.f16x2.e3m2x2 %0, %1;" : "=r"(h2) : "h"(c));
     asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
         : "=f"(lo), "=f"(hi) : "r"(h2));
 }

@@ -356,6 +356,12 @@ cudaError_t launch_quant_dual(const void *src, int64_t rows, int64_t cols, int f
     case FMT_E5M2 * 2 + 1: return launch_dual_t<FMT_E5M2, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
     case FMT_E2M1 * 2 + 0: return launch_dual_t<FMT_E2M1, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
     case FMT_E2M1 * 2 + 1: return launch_dual_t<FMT_E2M1, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E2M3 * 2 + 0: return launch_dual_t<FMT_E2M3, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E2M3 * 2 + 1: return launch_dual_t<FMT_E2M3, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E3M2 * 2 + 0: return launch_dual_t<FMT_E3M2, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E3M2 * 2 + 1: return launch_dual_t<FMT_E3M2, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_INT8 * 2 + 0: return launch_dual_t<FMT_INT8, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_INT8 * 2 + 1: return launch_dual_t<FMT_INT8, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -78,8 +78,8 @@ template <int BN, int KIND>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const uint8_t *__restrict__ a_sc, const uint8_t *__restrict__ b_sc, const float *__restrict__ ga,
-               const float *__restrict__ gb, uint16_t *__restrict__ C, int M, int N, int K, uint32_t b_fmt_code,
-               int band, int *watchdog) {
+               const float *__restrict__ gb, uint16_t *__restrict__ C, int M, int N, int K, uint32_t a_fmt_code,
+               uint32_t b_fmt_code, int band, int *watchdog) {
     using T = Tile<BN, KIND>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -195,7 +195,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         const uint32_t sf_id = KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u);
                         const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
                         const uint64_t bd = smem_desc(b_base + k * 32, 16, 1024, 2);
-                        tc_mma_mx<KIND>(tmem, ad, bd, mma_idesc<kBM, BN, KIND>(b_fmt_code, sf_id), sfa_t + 4 * a,
+                        tc_mma_mx<KIND>(tmem, ad, bd, mma_idesc<kBM, BN, KIND>(a_fmt_code, b_fmt_code, sf_id), sfa_t + 4 * a,
                                         sfb_t + 4 * a * (BN / 128), (kb > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty_bar[s]);
@@ -283,13 +283,13 @@ static bool encode_operand(EncodeTiledFn enc, CUtensorMap *tm, const void *ptr, 
 template <int BN, int KIND>
 static cudaError_t launch_gemm_k(const CUtensorMap &tmA, const CUtensorMap &tmB, const uint8_t *a_sc,
                                  const uint8_t *b_sc, const float *ga, const float *gb, void *c, int64_t M,
-                                 int64_t N, int64_t K, uint32_t b_code, int64_t band, int *watchdog, int grid,
-                                 cudaStream_t st) {
+                                 int64_t N, int64_t K, uint32_t a_code, uint32_t b_code, int64_t band, int *watchdog,
+                                 int grid, cudaStream_t st) {
     auto k = mx_gemm_kernel<BN, KIND>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<BN, KIND>::kSmemBytes);
     if (e != cudaSuccess) return e;
     k<<<grid, kGemmThreads, Tile<BN, KIND>::kSmemBytes, st>>>(tmA, tmB, a_sc, b_sc, ga, gb, static_cast<uint16_t *>(c),
-                                                             (int)M, (int)N, (int)K, b_code, (int)band, watchdog);
+                                                             (int)M, (int)N, (int)K, a_code, b_code, (int)band, watchdog);
     return cudaGetLastError();
 }
 
@@ -299,13 +299,13 @@ cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, int a_fmt, con
     auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
     if (!enc) return cudaErrorNotSupported;
     int kind;
-    if (a_fmt == FMT_E4M3 && (b_fmt == FMT_E4M3 || b_fmt == FMT_E2M1)) kind = KIND_F8F6F4;
+    if (f8f6f4_code(a_fmt) >= 0 && a_fmt != FMT_E2M1 && f8f6f4_code(b_fmt) >= 0) kind = KIND_F8F6F4;
     else if (a_fmt == FMT_E2M1 && b_fmt == FMT_E2M1) kind = KIND_MXF4;
     else if (a_fmt == FMT_NVFP4 && b_fmt == FMT_NVFP4) kind = KIND_NVF4;
     else return cudaErrorInvalidValue;
     const int stage_k = kind == KIND_F8F6F4 ? 128 : 256;
     if (K % stage_k) return cudaErrorInvalidValue;
-    const bool a_fp4 = kind != KIND_F8F6F4, b_fp4 = b_fmt != FMT_E4M3;
+    const bool a_fp4 = kind != KIND_F8F6F4, b_fp4 = b_fmt == FMT_E2M1 || b_fmt == FMT_NVFP4;
     const bool b_expand = kind == KIND_F8F6F4 && b_fp4;
     CUtensorMap tmA, tmB;
     if (!encode_operand(enc, &tmA, a_elems, M, K, a_fp4, false, kBM)) return cudaErrorInvalidValue;
@@ -319,15 +319,16 @@ cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, int a_fmt, con
     if (band < 1) band = 1;
     if (band > N / bn) band = N / bn;
     const int grid = (int)(n_tiles < num_sms ? n_tiles : num_sms);
-    const uint32_t b_code = b_expand ? 5u : 0u;
+    const uint32_t a_code = kind == KIND_F8F6F4 ? (uint32_t)f8f6f4_code(a_fmt) : 1u;
+    const uint32_t b_code = kind == KIND_F8F6F4 ? (uint32_t)f8f6f4_code(b_fmt) : 1u;
     if (kind == KIND_F8F6F4)
-        return wide ? launch_gemm_k<256, KIND_F8F6F4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, b_code, band, watchdog, grid, st)
-                    : launch_gemm_k<128, KIND_F8F6F4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, b_code, band, watchdog, grid, st);
+        return wide ? launch_gemm_k<256, KIND_F8F6F4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, a_code, b_code, band, watchdog, grid, st)
+                    : launch_gemm_k<128, KIND_F8F6F4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, a_code, b_code, band, watchdog, grid, st);
     if (kind == KIND_MXF4)
-        return wide ? launch_gemm_k<256, KIND_MXF4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, 0u, band, watchdog, grid, st)
-                    : launch_gemm_k<128, KIND_MXF4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, 0u, band, watchdog, grid, st);
-    return wide ? launch_gemm_k<256, KIND_NVF4>(tmA, tmB, a_sc, b_sc, ga, gb, c, M, N, K, 0u, band, watchdog, grid, st)
-                : launch_gemm_k<128, KIND_NVF4>(tmA, tmB, a_sc, b_sc, ga, gb, c, M, N, K, 0u, band, watchdog, grid, st);
+        return wide ? launch_gemm_k<256, KIND_MXF4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, a_code, b_code, band, watchdog, grid, st)
+                    : launch_gemm_k<128, KIND_MXF4>(tmA, tmB, a_sc, b_sc, nullptr, nullptr, c, M, N, K, a_code, b_code, band, watchdog, grid, st);
+    return wide ? launch_gemm_k<256, KIND_NVF4>(tmA, tmB, a_sc, b_sc, ga, gb, c, M, N, K, a_code, b_code, band, watchdog, grid, st)
+                : launch_gemm_k<128, KIND_NVF4>(tmA, tmB, a_sc, b_sc, ga, gb, c, M, N, K, a_code, b_code, band, watchdog, grid, st);
 }
 
 }  // namespace mxk

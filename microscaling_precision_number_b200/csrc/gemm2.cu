@@ -88,7 +88,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                     const float *__restrict__ ga, const float *__restrict__ gb, uint16_t *__restrict__ C, int M,
-                    int N, int K, uint32_t b_fmt_code, int band, int *watchdog) {
+                    int N, int K, uint32_t a_fmt_code, uint32_t b_fmt_code, int band, int *watchdog) {
     using P = Pair<KIND>;
     constexpr int S = P::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -202,7 +202,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         const uint32_t sf_id = KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u);
                         const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
                         const uint64_t bd = smem_desc(b_base + k * 32, 16, 1024, 2);
-                        tc_mma_mx<KIND, 2>(tmem, ad, bd, mma_idesc<kPairM, kPairN, KIND>(b_fmt_code, sf_id),
+                        tc_mma_mx<KIND, 2>(tmem, ad, bd, mma_idesc<kPairM, kPairN, KIND>(a_fmt_code, b_fmt_code, sf_id),
                                            sfa_t + 4 * a, sfb_t + 8 * a, (kb > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit_pair(&empty_bar[s]);           // stage s free in both CTAs
@@ -304,8 +304,8 @@ static bool encode_scales(EncodeTiledFn enc, CUtensorMap *tm, const uint8_t *ptr
 template <int KIND>
 static cudaError_t launch_pair_k(EncodeTiledFn enc, const void *a, const uint8_t *a_sc, const float *ga,
                                  const void *b, const uint8_t *b_sc, const float *gb, bool b_fp4, bool b_expand,
-                                 void *c, int64_t M, int64_t N, int64_t K, int *watchdog, int num_sms,
-                                 cudaStream_t st) {
+                                 uint32_t a_code, uint32_t b_code, void *c, int64_t M, int64_t N, int64_t K,
+                                 int *watchdog, int num_sms, cudaStream_t st) {
     using P = Pair<KIND>;
     CUtensorMap tmA, tmB, tmSA, tmSB;
     const int64_t col_atoms = (K / P::kStageK) * P::kAtoms;
@@ -327,7 +327,7 @@ static cudaError_t launch_pair_k(EncodeTiledFn enc, const void *a, const uint8_t
     if (e != cudaSuccess) return e;
     k<<<(unsigned)(2 * pairs), kPairThreads, P::kSmemBytes, st>>>(tmA, tmB, tmSA, tmSB, ga, gb,
                                                                    static_cast<uint16_t *>(c), (int)M, (int)N,
-                                                                   (int)K, b_expand ? 5u : 0u, (int)band, watchdog);
+                                                                   (int)K, a_code, b_code, (int)band, watchdog);
     return cudaGetLastError();
 }
 
@@ -339,19 +339,20 @@ cudaError_t launch_gemm_pair(const void *a_elems, const uint8_t *a_sc, int a_fmt
     auto enc = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
     if (!enc) return cudaErrorNotSupported;
     if (!gemm_pair_supported(M, N)) return cudaErrorInvalidValue;
-    if (a_fmt == FMT_E4M3 && (b_fmt == FMT_E4M3 || b_fmt == FMT_E2M1)) {
+    if (f8f6f4_code(a_fmt) >= 0 && a_fmt != FMT_E2M1 && f8f6f4_code(b_fmt) >= 0) {
         if (K % 128) return cudaErrorInvalidValue;
         const bool fp4 = b_fmt == FMT_E2M1;
-        return launch_pair_k<KIND_F8F6F4>(enc, a_elems, a_sc, nullptr, b_elems, b_sc, nullptr, fp4, fp4, c, M, N, K,
+        return launch_pair_k<KIND_F8F6F4>(enc, a_elems, a_sc, nullptr, b_elems, b_sc, nullptr, fp4, fp4,
+                                          (uint32_t)f8f6f4_code(a_fmt), (uint32_t)f8f6f4_code(b_fmt), c, M, N, K,
                                           watchdog, num_sms, st);
     }
     if (K % 256) return cudaErrorInvalidValue;
     if (a_fmt == FMT_E2M1 && b_fmt == FMT_E2M1)
-        return launch_pair_k<KIND_MXF4>(enc, a_elems, a_sc, nullptr, b_elems, b_sc, nullptr, true, false, c, M, N, K,
-                                        watchdog, num_sms, st);
+        return launch_pair_k<KIND_MXF4>(enc, a_elems, a_sc, nullptr, b_elems, b_sc, nullptr, true, false, 1u, 1u, c, M,
+                                        N, K, watchdog, num_sms, st);
     if (a_fmt == FMT_NVFP4 && b_fmt == FMT_NVFP4)
-        return launch_pair_k<KIND_NVF4>(enc, a_elems, a_sc, ga, b_elems, b_sc, gb, true, false, c, M, N, K, watchdog,
-                                        num_sms, st);
+        return launch_pair_k<KIND_NVF4>(enc, a_elems, a_sc, ga, b_elems, b_sc, gb, true, false, 1u, 1u, c, M, N, K,
+                                        watchdog, num_sms, st);
     return cudaErrorInvalidValue;
 }
 

@@ -54,7 +54,8 @@ cudaError_t launch_tcgen05_pad(uint8_t *sc, int64_t rows, int64_t S, cudaStream_
 
 // ---------------------------------------------------------------------------------------
 // Direct cast (no block scale): RNE + saturation by the hardware conversion; NaN is
-// mapped explicitly (0x7F|s for FP8, 0x7|s for E2M1, which has no NaN).
+// mapped explicitly (0x7F|s for FP8; the signed maximum for E2M1 and FP6, which have no
+// NaN: 0x7|s, 0x1F|s).
 // ---------------------------------------------------------------------------------------
 template <int FMT>
 __device__ __forceinline__ void cast8(const uint4 &v, uint8_t *out, int64_t c) {
@@ -72,7 +73,9 @@ __device__ __forceinline__ void cast8(const uint4 &v, uint8_t *out, int64_t c) {
 #pragma unroll
         for (int i = 0; i < 8; i++)
             if (x[i] != x[i]) {
-                const uint32_t nanc = 0x7Fu | (__float_as_uint(x[i]) >> 31 << 7);
+                const uint32_t nanc = (FMT == FMT_E2M3 || FMT == FMT_E3M2)
+                                          ? 0x1Fu | (__float_as_uint(x[i]) >> 31 << 5)
+                                          : 0x7Fu | (__float_as_uint(x[i]) >> 31 << 7);
                 w[i >> 2] = (w[i >> 2] & ~(0xFFu << (8 * (i & 3)))) | (nanc << (8 * (i & 3)));
             }
         reinterpret_cast<uint2 *>(out)[c] = make_uint2(w[0], w[1]);
@@ -112,6 +115,8 @@ cudaError_t launch_cast(const void *src, int64_t n, int fmt, void *out, int num_
     case FMT_E4M3: cast_kernel<FMT_E4M3><<<grid, kThreads, 0, st>>>(s, n_chunks, ts, tail, o); break;
     case FMT_E5M2: cast_kernel<FMT_E5M2><<<grid, kThreads, 0, st>>>(s, n_chunks, ts, tail, o); break;
     case FMT_E2M1: cast_kernel<FMT_E2M1><<<grid, kThreads, 0, st>>>(s, n_chunks, ts, tail, o); break;
+    case FMT_E2M3: cast_kernel<FMT_E2M3><<<grid, kThreads, 0, st>>>(s, n_chunks, ts, tail, o); break;
+    case FMT_E3M2: cast_kernel<FMT_E3M2><<<grid, kThreads, 0, st>>>(s, n_chunks, ts, tail, o); break;
     default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

@@ -610,6 +610,12 @@ cudaError_t launch_stream_rows_mx(const void *src, int64_t rows, int64_t cols, i
     case FMT_E5M2 * 2 + 1: return launch_rows_layout<FMT_E5M2, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
     case FMT_E2M1 * 2 + 0: return launch_rows_layout<FMT_E2M1, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
     case FMT_E2M1 * 2 + 1: return launch_rows_layout<FMT_E2M1, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E2M3 * 2 + 0: return launch_rows_layout<FMT_E2M3, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E2M3 * 2 + 1: return launch_rows_layout<FMT_E2M3, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E3M2 * 2 + 0: return launch_rows_layout<FMT_E3M2, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E3M2 * 2 + 1: return launch_rows_layout<FMT_E3M2, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_INT8 * 2 + 0: return launch_rows_layout<FMT_INT8, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_INT8 * 2 + 1: return launch_rows_layout<FMT_INT8, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -663,6 +669,12 @@ cudaError_t launch_stream_dequant_mx(const void *elems, const uint8_t *scales, i
                              : launch_dq_t<FMT_E5M2, false>(elems, scales, nb, f, ca, out, wd, num_sms, st);
     case FMT_E2M1: return tc ? launch_dq_t<FMT_E2M1, true>(elems, scales, nb, f, ca, out, wd, num_sms, st)
                              : launch_dq_t<FMT_E2M1, false>(elems, scales, nb, f, ca, out, wd, num_sms, st);
+    case FMT_E2M3: return tc ? launch_dq_t<FMT_E2M3, true>(elems, scales, nb, f, ca, out, wd, num_sms, st)
+                        : launch_dq_t<FMT_E2M3, false>(elems, scales, nb, f, ca, out, wd, num_sms, st);
+    case FMT_E3M2: return tc ? launch_dq_t<FMT_E3M2, true>(elems, scales, nb, f, ca, out, wd, num_sms, st)
+                        : launch_dq_t<FMT_E3M2, false>(elems, scales, nb, f, ca, out, wd, num_sms, st);
+    case FMT_INT8: return tc ? launch_dq_t<FMT_INT8, true>(elems, scales, nb, f, ca, out, wd, num_sms, st)
+                        : launch_dq_t<FMT_INT8, false>(elems, scales, nb, f, ca, out, wd, num_sms, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -12,6 +12,12 @@ namespace mxk {
 // K = 64 instruction); E2M1 x E2M1 packed with UE4M3 scales per 16 (four per K = 64).
 enum : int { KIND_F8F6F4 = 0, KIND_MXF4 = 1, KIND_NVF4 = 2 };
 
+// mxf8f6f4 operand format code of an element format (E4M3 0, E5M2 1, E2M3 3, E3M2 4,
+// E2M1 5), or -1 when the format is not an operand of that kind.
+__host__ __device__ constexpr int f8f6f4_code(int fmt) {
+    return fmt == 0 ? 0 : fmt == 1 ? 1 : fmt == 4 ? 3 : fmt == 5 ? 4 : fmt == 2 ? 5 : -1;
+}
+
 // ---- tcgen05 wrappers -------------------------------------------------------------------
 // Tensor-memory allocation by one full warp.  With CG = 2 the instruction is collective
 // over the CTA pair: the warp with the same index in both CTAs executes it, and both pass
@@ -66,12 +72,12 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 
 // Instruction descriptor for the block-scaled kinds: B scale-factor id (first scale byte
 // of the 32-bit tensor-memory word) in bits 4-5, A format 7-9, B format 10-12 (mxf8f6f4:
-// E4M3 = 0, E2M1 = 5; mxf4 / mxf4nvf4: E2M1 = 1), K-major A and B, N >> 3 in 17-22, scale
+// E4M3 = 0, E5M2 = 1, E2M3 = 3, E3M2 = 4, E2M1 = 5; mxf4 / mxf4nvf4: E2M1 = 1), K-major A and B, N >> 3 in 17-22, scale
 // type in bit 23 (1 = UE8M0, 0 = UE4M3), M >> 4 in 24-28, A scale-factor id in 29-30,
 // bit 31 = 0 (dense K of 32 for 8-bit kinds, 64 for 4-bit kinds).
 template <int BM, int BN, int KIND>
-__device__ __forceinline__ uint32_t mma_idesc(uint32_t b_fmt_code, uint32_t sf_id) {
-    const uint32_t a_fmt = KIND == KIND_F8F6F4 ? 0u : 1u;
+__device__ __forceinline__ uint32_t mma_idesc(uint32_t a_fmt_code, uint32_t b_fmt_code, uint32_t sf_id) {
+    const uint32_t a_fmt = KIND == KIND_F8F6F4 ? a_fmt_code : 1u;
     const uint32_t b_fmt = KIND == KIND_F8F6F4 ? b_fmt_code : 1u;
     uint32_t d = 0;
     d |= (sf_id & 3u) << 4;

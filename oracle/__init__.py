@@ -77,6 +77,8 @@ def lib():
         _lib.mxo_tcgen05_scale_offset.restype = I64
         _lib.mxo_gemm_ref.argtypes = [P, P, I, ctypes.c_double, P, P, I, ctypes.c_double, I64, I64, I64, P, I64, P, P]
         _lib.mxo_gemm_ref.restype = I
+        _lib.mxo_mxfp4_to_fp8_blocks.argtypes = [P, P, I64, I64, P, P, P]
+        _lib.mxo_mxfp4_to_fp8_blocks.restype = I
     return _lib
 
 
@@ -207,3 +209,16 @@ def gemm_ref(a_elems, a_scales, a_fmt, b_elems, b_scales, b_fmt, M, N, K, pairs,
                               ctypes.c_double(b_g), M, N, K,
                               _ptr(pr), pr.shape[0], _ptr(c), _ptr(mag)), "gemm_ref")
     return c, mag
+
+
+def mxfp4_to_fp8_blocks(elems: np.ndarray, scales: np.ndarray, rows: int, cols: int):
+    """MXFP4 (packed E2M1, row-major E8M0 per 32) -> E4M3 codes rows x cols, one fp32 scale
+    and one exactness flag per 128 x 128 block (the nested blocks of the pages)."""
+    e = np.ascontiguousarray(elems, dtype=np.uint8)
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    out = np.zeros((rows, cols), dtype=np.uint8)
+    bs = np.zeros((rows // 128, cols // 128), dtype=np.float32)
+    ok = np.zeros((rows // 128, cols // 128), dtype=np.uint8)
+    _check(lib().mxo_mxfp4_to_fp8_blocks(_ptr(e), _ptr(s), rows, cols, _ptr(out), _ptr(bs), _ptr(ok)),
+           "mxfp4_to_fp8_blocks")
+    return out, bs, ok

@@ -544,3 +544,68 @@ int mxo_gemm_ref(const uint8_t *a_elems, const uint8_t *a_scales, int a_fmt, dou
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Nested blocks (Q§6 "DeepSeek-V4 の入れ子構造"): an MXFP4 weight (1 x 32      */
+/* sub-blocks, E8M0 scales) re-expressed as FP8 E4M3 with one scale per      */
+/* 128 x 128 block, which holds 4 x 128 = 512 of the 1 x 32 sub-blocks.  The  */
+/* conversion is lossless while the sub-block scales inside a block do not    */
+/* spread too far; the pages give the condition (a bound on the ratio of the  */
+/* largest to the smallest sub-block scale) but not the bound.  Written out:  */
+/*   s_max  = the largest sub-block exponent (code - 127) among sub-blocks     */
+/*            that are not NaN and hold a nonzero code;                        */
+/*   S      = 2^(s_max - 6): the largest FP4 value 6 * 2^s_max maps to 384,    */
+/*            inside E4M3 (max 448);                                           */
+/*   each element: FP8 code = RNE-saturating E4M3 encoding of                  */
+/*            dec_E2M1(q) * 2^(s_b - s_max + 6) (exact in double);             */
+/*   exact  <=> every nonzero element is representable: with E2M1 values      */
+/*            {1, 1.5} x 2^k (k >= -1) and E4M3's smallest step 2^-9 this is   */
+/*            s_max - s_b <= 14 for every sub-block holding a nonzero code     */
+/*            (the ratio bound 2^14); all-zero and NaN sub-blocks are exempt.  */
+/* A NaN sub-block (scale 0xFF) gives E4M3 NaN codes 0x7F.  A block with no    */
+/* nonzero finite element gets S = 1.                                          */
+/* The oracle decides exactness by comparing values (decode both and check    */
+/* equality), not by the bound, so a test can check the bound against it.     */
+/* elems: rows x cols/2 packed E2M1; scales: rows x cols/32 row-major E8M0;   */
+/* out: rows x cols E4M3 codes; block_scale / exact: (rows/128) x (cols/128). */
+/* ------------------------------------------------------------------------- */
+int mxo_mxfp4_to_fp8_blocks(const uint8_t *elems, const uint8_t *scales, int64_t rows, int64_t cols,
+                            uint8_t *out, float *block_scale, uint8_t *exact) {
+    if (rows % 128 || cols % 128) return -1;
+    const int64_t S = cols / 32, BC = cols / 128;
+    for (int64_t br = 0; br < rows / 128; br++) {
+        for (int64_t bc = 0; bc < BC; bc++) {
+            int smax = INT32_MIN;
+            for (int64_t r = br * 128; r < br * 128 + 128; r++) {
+                for (int64_t b = bc * 4; b < bc * 4 + 4; b++) {
+                    unsigned sc = scales[r * S + b];
+                    if (sc == 0xFFu) continue;
+                    int nonzero = 0;
+                    for (int64_t j = b * 32; j < b * 32 + 32; j++)
+                        if (mxo_decode(K_E2M1, get_code(elems + r * (cols / 2), j, 1)) != 0.0) nonzero = 1;
+                    if (nonzero && (int)sc - 127 > smax) smax = (int)sc - 127;
+                }
+            }
+            if (smax == INT32_MIN) smax = 6;                /* no nonzero finite element: S = 1 */
+            block_scale[br * BC + bc] = (float)ldexp(1.0, smax - 6);
+            int ok = 1;
+            for (int64_t r = br * 128; r < br * 128 + 128; r++) {
+                for (int64_t j = bc * 128; j < bc * 128 + 128; j++) {
+                    unsigned sc = scales[r * S + j / 32];
+                    unsigned q = get_code(elems + r * (cols / 2), j, 1);
+                    unsigned code;
+                    if (sc == 0xFFu) {
+                        code = 0x7Fu;
+                    } else {
+                        double v = ldexp(mxo_decode(K_E2M1, q), (int)sc - 127 - (smax - 6));
+                        code = mxo_encode(v, K_E4M3);
+                        if (mxo_decode(K_E4M3, code) != v) ok = 0;   /* -0 == +0 counts as equal */
+                    }
+                    out[r * cols + j] = (uint8_t)code;
+                }
+            }
+            exact[br * BC + bc] = (uint8_t)ok;
+        }
+    }
+    return 0;
+}

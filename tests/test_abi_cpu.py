@@ -92,10 +92,15 @@ def test_dual_dequant_cast_gemm_validation(L):
     assert lib.mx_dequantize(FAKE + 2, FAKE, None, 4, 64, 0, 1, FAKE, None) == L.MX_ERR_ALIGN
     assert lib.mx_cast(FAKE, 7, 2, FAKE, None) == L.MX_ERR_SHAPE
     assert lib.mx_cast(FAKE, 8, 3, FAKE, None) == L.MX_ERR_ARG
+    assert lib.mx_cast(FAKE, 8, 6, FAKE, None) == L.MX_ERR_ARG        # INT8 needs a scale
+    assert lib.mx_quantize(FAKE, 4, 64, 7, 0, 1, FAKE, FAKE, 1, None, None, None) == L.MX_ERR_ARG
+    assert lib.mx_quantize(FAKE, 4, 64, 6, 0, 1, FAKE, FAKE, 1, None, FAKE, None) == L.MX_ERR_ARG   # g is NVFP4 only
     assert lib.mx_cast(None, 8, 0, FAKE, None) == L.MX_ERR_ARG
     assert lib.mx_cast(FAKE, 0, 0, FAKE, None) == L.MX_OK
     op = lambda fmt, p=FAKE, g=None: L.MxOperand(p, FAKE, fmt, g)
-    assert lib.mx_gemm(op(0), op(1), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG      # E5M2 B unsupported
+    assert lib.mx_gemm(op(0), op(6), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG      # INT8: no tensor-core form
+    assert lib.mx_gemm(op(6), op(0), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG
+    assert lib.mx_gemm(op(4), op(7), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG      # unknown format
     assert lib.mx_gemm(op(2), op(0), FAKE, 128, 128, 128, None) == L.MX_ERR_ARG      # E2M1 x E4M3 unsupported
     assert lib.mx_gemm(op(3, g=FAKE), op(2), FAKE, 128, 128, 256, None) == L.MX_ERR_ARG   # NVFP4 x MXFP4
     assert lib.mx_gemm(op(3), op(3, g=FAKE), FAKE, 128, 128, 256, None) == L.MX_ERR_ARG   # missing g

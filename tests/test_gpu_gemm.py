@@ -45,7 +45,7 @@ def _no_watchdog():
     assert mx.watchdog_status(clear=True) == 0
 
 
-GPU_FMT = {0: "e4m3", 2: "e2m1", 3: "nvfp4"}
+GPU_FMT = {0: "e4m3", 1: "e5m2", 2: "e2m1", 3: "nvfp4", 4: "e2m3", 5: "e3m2"}
 
 
 def _gpu_quant(bits, fmt):
@@ -195,3 +195,14 @@ def test_gemm_rejects_unsupported_pairs():
     for a, b in ((f4, e4), (n4, f4), (e4, n4)):
         with pytest.raises(mx.MxError):
             mx.gemm(a, b)
+
+
+# ------------------------------------------------------------------ FP6 and E5M2 operands (kind::mxf8f6f4)
+@pytest.mark.parametrize("a_fmt,b_fmt", [(4, 4), (5, 2), (1, 0), (0, 5), (4, 1)])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (128, 384, 256)])
+def test_gemm_fp6_fp8_operand_pairs(oracle, a_fmt, b_fmt, M, N, K):
+    """MXFP6 (E2M3, E3M2) and E5M2 operands run on the same tensor-core kind as MXFP8 (the
+    first shape uses CTA pairs, the second single CTAs)."""
+    a = synth.normal(M, K, seed=M + a_fmt)
+    b = synth.weight_fp4(N, K, seed=N + b_fmt) if b_fmt == 2 else synth.normal(N, K, seed=N + b_fmt)
+    run_case(oracle, a, b, b_fmt, a_fmt=a_fmt)

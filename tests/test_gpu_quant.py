@@ -13,7 +13,7 @@ if torch.cuda.is_available():
     import microscaling_precision_number_b200 as mx
     from microscaling_precision_number_b200 import _lib as L
 
-FMT_NAMES = {0: "e4m3", 1: "e5m2", 2: "e2m1"}
+FMT_NAMES = {0: "e4m3", 1: "e5m2", 2: "e2m1", 4: "e2m3", 5: "e3m2", 6: "int8"}
 
 
 def to_dev(bits: np.ndarray) -> torch.Tensor:
@@ -58,7 +58,7 @@ def _no_watchdog():
 
 
 # ------------------------------------------------------------------ direct cast
-@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 4, 5])
 def test_cast_exhaustive_bf16(oracle, fmt):
     bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     got = host(mx.cast(to_dev(bits), FMT_NAMES[fmt]))
@@ -71,13 +71,15 @@ def test_cast_exhaustive_bf16(oracle, fmt):
 def test_cast_tail(oracle, n):
     rng = np.random.default_rng(n)
     bits = rng.integers(0, 65536, size=n, dtype=np.uint32).astype(np.uint16)
-    for fmt in (0, 2):
+    for fmt in (0, 2, 4):
         assert np.array_equal(host(mx.cast(to_dev(bits), FMT_NAMES[fmt])), oracle.cast(bits, fmt))
 
 
 # ------------------------------------------------------------------ row-wise MX
 @pytest.mark.parametrize("shape", SHAPES)
-@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (0, "floor"), (1, "ceil"), (1, "floor"), (2, "floor"), (2, "ceil")])
+@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (0, "floor"), (1, "ceil"), (1, "floor"), (2, "floor"), (2, "ceil"),
+                                          (4, "floor"), (4, "ceil"), (5, "floor"), (5, "ceil"), (6, "floor"),
+                                          (6, "ceil")])
 def test_quantize_rowwise_matches_oracle(oracle, shape, fmt, rounding):
     x = with_specials(synth.mx8_rowwise(*shape, seed=shape[0]), seed=shape[1])
     q = mx.quantize(to_dev(x), FMT_NAMES[fmt], "row", rounding, layout="both")
@@ -111,7 +113,8 @@ def test_tcgen05_padding_is_zeroed(oracle):
 
 # ------------------------------------------------------------------ column-wise and dual
 @pytest.mark.parametrize("shape", [(32, 32), (64, 96), (96, 200), (160, 384)])
-@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (1, "ceil"), (2, "floor")])
+@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (1, "ceil"), (2, "floor"), (4, "ceil"), (5, "floor"),
+                                          (6, "ceil")])
 def test_quantize_colwise_matches_oracle(oracle, shape, fmt, rounding):
     x = with_specials(synth.activations(*shape, seed=shape[1]), seed=shape[0])
     rnd = oracle.CEIL if rounding == "ceil" else oracle.FLOOR
@@ -123,7 +126,8 @@ def test_quantize_colwise_matches_oracle(oracle, shape, fmt, rounding):
 
 
 @pytest.mark.parametrize("shape", [(32, 32), (64, 160), (160, 384), (256, 1024)])
-@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (1, "ceil"), (1, "floor"), (2, "floor")])
+@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (1, "ceil"), (1, "floor"), (2, "floor"), (4, "floor"),
+                                          (5, "ceil"), (6, "floor"), (6, "ceil")])
 @pytest.mark.parametrize("layout", ["rowmajor", "tcgen05"])
 def test_quantize_dual_matches_oracle(oracle, shape, fmt, rounding, layout):
     x = with_specials(synth.gradients(*shape, seed=shape[0] + fmt), seed=shape[1])
@@ -167,7 +171,7 @@ def test_nvfp4_degenerate_tensors(oracle):
 
 
 # ------------------------------------------------------------------ dequantisation
-@pytest.mark.parametrize("fmt", [0, 1, 2])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 4, 5, 6])
 @pytest.mark.parametrize("layout", ["rowmajor", "tcgen05"])
 def test_dequantize_matches_oracle(oracle, fmt, layout):
     x = with_specials(synth.mx8_rowwise(67, 256, seed=fmt), seed=3)
@@ -179,8 +183,8 @@ def test_dequantize_matches_oracle(oracle, fmt, layout):
 
 def test_dequantize_all_scale_codes(oracle):
     """Every E8M0 code (incl. 2^-127 and NaN) against every element code."""
-    for fmt in (0, 1, 2):
-        ncode = 16 if fmt == 2 else 256
+    for fmt in (0, 1, 2, 4, 5, 6):
+        ncode = {2: 16, 4: 64, 5: 64}.get(fmt, 256)         # FP6: the 64 six-bit codes
         codes = np.tile(np.arange(ncode, dtype=np.uint8), 256 * 32 // ncode)[: 256 * 32].reshape(256, 32)
         scales = np.arange(256, dtype=np.uint8).reshape(256, 1)
         if fmt == 2:
