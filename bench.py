@@ -407,6 +407,42 @@ def run_breakdown(mx, dev, pk):
                      "peak_note": "bf16 burst (MEASURED_PEAKS) x 4, the FP4 to bf16 nominal ratio"}
         del a, b, c
         torch.cuda.empty_cache()
+
+    # next row: MXFP6 / MXINT8 row-wise quantisation of the config-3 activations
+    # (16384 x 4096 bf16, one byte per code), against the HBM roofline
+    x3 = to_dev(synth.activations(), dev)
+    R, C = x3.shape
+    for name, fmt in (("next_quant_mxfp6_e2m3_16384x4096", "e2m3"), ("next_quant_mxint8_16384x4096", "int8")):
+        q = mx.quantize(x3, fmt, "row", "ceil", layout="tcgen05")
+        t = timed([lambda q=q: mx.quantize(x3, fmt, "row", "ceil", layout="tcgen05", out=q)], 20, stream)
+        nb = R * C * 2 + R * C + R * C // 32
+        out[name] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1), "frac_hbm": round(nb / t / 1e6 / hbm, 4),
+                     "algorithmic_bytes": nb}
+        del q
+    del x3
+
+    # next row: nested blocks -- the config-5 MXFP4 weight (14336 x 4096) re-expressed as
+    # FP8 E4M3 with 128 x 128 block scales
+    from microscaling_precision_number_b200 import _lib as L
+    xw = to_dev(synth.normal(14336, 4096, sigma=0.02, seed=51), dev)
+    qw = mx.quantize(xw, "e2m1", "row", "floor", layout="rowmajor")
+    R, C = xw.shape
+    del xw
+    o8 = torch.empty(R * C, dtype=torch.uint8, device=dev)
+    bsc = torch.empty((R // 128) * (C // 128), dtype=torch.float32, device=dev)
+    bok = torch.empty((R // 128) * (C // 128), dtype=torch.uint8, device=dev)
+
+    def nested():
+        L.check(L.lib.mx_mxfp4_to_fp8_blocks(qw.elems.data_ptr(), qw.scales.data_ptr(), R, C, o8.data_ptr(),
+                                             bsc.data_ptr(), bok.data_ptr(), stream.cuda_stream),
+                "mx_mxfp4_to_fp8_blocks")
+    t = timed([nested], 20, stream)
+    nb = R * C // 2 + R * C // 32 + R * C + 5 * (R // 128) * (C // 128)
+    out["next_nested_mxfp4_to_fp8_14336x4096"] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1),
+                                                   "frac_hbm": round(nb / t / 1e6 / hbm, 4), "algorithmic_bytes": nb,
+                                                   "blocks_exact": int(bok.sum().item()), "blocks": int(bok.numel())}
+    del qw, o8, bsc, bok
+    torch.cuda.empty_cache()
     return out
 
 

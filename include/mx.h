@@ -233,6 +233,28 @@ typedef struct {
 mx_status mx_gemm(mx_operand A, mx_operand B, void *C_bf16, int64_t M, int64_t N, int64_t K,
                   mx_stream_t stream);
 
+/*
+ * mx_mxfp4_to_fp8_blocks -- the nested blocks of [Q] §6 ("DeepSeek-V4 の入れ子構造"): an
+ * MXFP4 weight (1 x 32 tiles, E8M0 scales) re-expressed as FP8 E4M3 with one scale per
+ * 128 x 128 block, the block scaling FP8 training keeps; a block holds 4 x 128 = 512 tiles.
+ * Per block: s_max = the largest tile exponent (scale code - 127) among tiles that are not
+ * NaN and hold a nonzero code; block scale S = 2^(s_max - 6) (the largest FP4 value
+ * 6 * 2^s_max becomes 384; 1.0 for a block without such a tile); every element becomes
+ * the RNE-saturating E4M3 code of dec(q) * 2^(s_tile - 127) / S; a NaN tile gives 0x7F
+ * codes.  block_exact = 1 when every element of the block decodes back to its FP4 value
+ * (the lossless condition of the pages; it always holds when no nonzero tile is more than
+ * 14 binades below s_max), else 0.
+ *   elems         device, rows x cols/2 packed E2M1 (even element in the low nibble),
+ *                 16-byte aligned, as mx_quantize(E2M1, ROW) writes it.
+ *   scales        device, rows x cols/32 E8M0, ROWMAJOR layout.
+ *   rows, cols    multiples of 128 (else MX_ERR_SHAPE).
+ *   out_fp8       device, rows x cols E4M3 codes, 16-byte aligned.
+ *   block_scales  device, (rows/128) x (cols/128) fp32 (powers of two), 4-byte aligned.
+ *   block_exact   device, (rows/128) x (cols/128) bytes.
+ */
+mx_status mx_mxfp4_to_fp8_blocks(const void *elems, const uint8_t *scales, int64_t rows, int64_t cols,
+                                 void *out_fp8, float *block_scales, uint8_t *block_exact, mx_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *mx_status_string(mx_status status);
 

@@ -316,4 +316,19 @@ mx_status mx_gemm(mx_operand A, mx_operand B, void *C, int64_t M, int64_t N, int
     return e == cudaSuccess ? MX_OK : cuda_fail(e);
 }
 
+mx_status mx_mxfp4_to_fp8_blocks(const void *elems, const uint8_t *scales, int64_t rows, int64_t cols,
+                                 void *out_fp8, float *block_scales, uint8_t *block_exact, mx_stream_t stream) {
+    if (rows < 0 || cols < 0 || rows % 128 || cols % 128) return MX_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MX_OK;
+    if ((rows / 128) * (cols / 128) > 0x7FFFFFFF) return MX_ERR_SHAPE;
+    if (!elems || !scales || !out_fp8 || !block_scales || !block_exact) return MX_ERR_ARG;
+    if (!aligned(elems, 16) || !aligned(out_fp8, 16) || !aligned(block_scales, 4)) return MX_ERR_ALIGN;
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    const cudaError_t e = mxk::launch_mxfp4_to_fp8_blocks(elems, scales, rows, cols, out_fp8, block_scales,
+                                                          block_exact, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MX_OK : cuda_fail(e);
+}
+
 }  // extern "C"

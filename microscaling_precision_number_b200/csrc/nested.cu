@@ -1,0 +1,117 @@
+// nested.cu -- MXFP4 (1 x 32 E2M1 tiles, E8M0 scales) re-expressed as FP8 E4M3 with one
+// power-of-two scale per 128 x 128 block.
+//
+// Source (page title, section):
+//   "MXFP4 と NVFP4 は何が違うのか調べてみた"
+//     §6 "DeepSeek-V4 の入れ子構造": FP8 training keeps 128 x 128 block scaling; each such
+//        block holds 4 x 128 = 512 MXFP4 1 x 32 tiles, and the FP4 -> FP8 dequantisation is
+//        lossless while the ratio of the largest to the smallest tile scale in a block stays
+//        under a bound (E4M3's two extra exponent bits absorb the fine-grained scales).
+//
+// Per 128 x 128 block: s_max = largest tile exponent among tiles that are finite and hold
+// a nonzero code; block scale S = 2^(s_max - 6) (the largest FP4 value 6 * 2^s_max lands
+// on 384, inside E4M3); each element becomes the RNE-saturating E4M3 code of
+// dec(q) * 2^(s_tile - s_max + 6); the block is flagged exact when every element decodes
+// back to its FP4 value (a tile scale at most 14 binades below s_max always is).  NaN tiles
+// give E4M3 NaN codes.  One CTA per block, one thread per 64-element half row (two tiles).
+#include "codec.cuh"
+#include "internal.h"
+
+namespace mxk {
+
+namespace {
+constexpr int kNestThreads = 256;
+constexpr int kNoScale = -100000;
+}  // namespace
+
+__global__ void __launch_bounds__(kNestThreads)
+mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restrict__ scales, int64_t cols,
+                           uint32_t blocks_c, uint8_t *__restrict__ out, float *__restrict__ block_scale,
+                           uint8_t *__restrict__ block_exact) {
+    __shared__ int warp_max[kNestThreads / 32];
+    const uint32_t blk = blockIdx.x;
+    const uint32_t br = blk / blocks_c, bc = blk - br * blocks_c;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t R = (int64_t)br * 128 + (tid >> 1);           // this thread's row
+    const int64_t c0 = (int64_t)bc * 128 + 64 * (tid & 1);      // its first column (two tiles)
+    const int64_t S = cols / 32;
+
+    // 64 packed E2M1 codes (32 bytes) and the two tile scales
+    const uint4 *src = reinterpret_cast<const uint4 *>(elems + ((R * cols + c0) >> 1));
+    const uint4 p0 = src[0], p1 = src[1];
+    const uint32_t sc[2] = {scales[R * S + (c0 >> 5)], scales[R * S + (c0 >> 5) + 1]};
+    const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+
+    // largest exponent among finite tiles holding a nonzero code (E2M1 magnitude bits 0-2)
+    int m = kNoScale;
+#pragma unroll
+    for (int t = 0; t < 2; t++) {
+        const bool nonzero = ((w[4 * t] | w[4 * t + 1] | w[4 * t + 2] | w[4 * t + 3]) & 0x77777777u) != 0u;
+        if (sc[t] != 0xFFu && nonzero) m = max(m, (int)sc[t] - 127);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) warp_max[warp] = m;
+    __syncthreads();
+    int smax = warp_max[0];
+#pragma unroll
+    for (int i = 1; i < kNestThreads / 32; i++) smax = max(smax, warp_max[i]);
+    if (smax == kNoScale) smax = 6;                               // no nonzero finite element: S = 1
+
+    bool exact = true;
+    uint32_t o[16];                                               // 64 E4M3 codes
+#pragma unroll
+    for (int t = 0; t < 2; t++) {
+        const int d = (int)sc[t] - 127 - smax + 6;                // tile exponent relative to S
+        // 2^d as fp32 (0 below 2^-149, where every product encodes to 0 anyway; capped at
+        // 2^126, reached only by tiles whose codes are all zero)
+        const int dc = d > 126 ? 126 : d;
+        const float f = dc >= -126 ? __uint_as_float((uint32_t)(dc + 127) << 23)
+                                   : (dc >= -149 ? __uint_as_float(1u << (dc + 149)) : 0.0f);
+#pragma unroll
+        for (int k = 0; k < 4; k++) {                             // 8 codes per word
+            float y[8];
+            e2m1x8_to_f32(w[4 * t + k], y);
+#pragma unroll
+            for (int i = 0; i < 8; i++) y[i] = __fmul_rn(y[i], f);
+            const uint2 q = cvt_fp8x8<FMT_E4M3>(y);
+            // exact iff every code decodes back to its FP4 value
+            float b[8];
+            fp8x2_to_f32<FMT_E4M3>(q.x & 0xFFFFu, b[0], b[1]);
+            fp8x2_to_f32<FMT_E4M3>(q.x >> 16, b[2], b[3]);
+            fp8x2_to_f32<FMT_E4M3>(q.y & 0xFFFFu, b[4], b[5]);
+            fp8x2_to_f32<FMT_E4M3>(q.y >> 16, b[6], b[7]);
+            // From 2^-126 down the products are exact fp32 values and the round trip decides;
+            // below, every nonzero FP4 value lies under E4M3's smallest step: exact only if
+            // the codes are all zero.
+            const bool zero_word = (w[4 * t + k] & 0x77777777u) == 0u;
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                exact = exact && (sc[t] == 0xFFu || (d >= -126 ? b[i] == y[i] : zero_word));
+            o[8 * t + 2 * k] = sc[t] == 0xFFu ? 0x7F7F7F7Fu : q.x;    // NaN tile: E4M3 NaN
+            o[8 * t + 2 * k + 1] = sc[t] == 0xFFu ? 0x7F7F7F7Fu : q.y;
+        }
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(out + R * cols + c0);
+#pragma unroll
+    for (int i = 0; i < 4; i++) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    const int all_exact = __syncthreads_and(exact ? 1 : 0);
+    if (tid == 0) {
+        const int e = smax - 6;                                   // S = 2^e, e in [-133, 121]
+        block_scale[blk] = e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
+        block_exact[blk] = (uint8_t)all_exact;
+    }
+}
+
+cudaError_t launch_mxfp4_to_fp8_blocks(const void *elems, const uint8_t *scales, int64_t rows, int64_t cols,
+                                       void *out, float *block_scale, uint8_t *block_exact, cudaStream_t st) {
+    const int64_t n_blocks = (rows / 128) * (cols / 128);
+    if (n_blocks <= 0) return cudaSuccess;
+    if (n_blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    mxfp4_to_fp8_blocks_kernel<<<(unsigned)n_blocks, kNestThreads, 0, st>>>(
+        static_cast<const uint8_t *>(elems), scales, cols, (uint32_t)(cols / 128), static_cast<uint8_t *>(out),
+        block_scale, block_exact);
+    return cudaGetLastError();
+}
+
+}  // namespace mxk

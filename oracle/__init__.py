@@ -77,6 +77,8 @@ def lib():
         _lib.mxo_tcgen05_scale_offset.restype = I64
         _lib.mxo_gemm_ref.argtypes = [P, P, I, ctypes.c_double, P, P, I, ctypes.c_double, I64, I64, I64, P, I64, P, P]
         _lib.mxo_gemm_ref.restype = I
+        _lib.mxo_quantize_nvfp4_2d.argtypes = [P, I64, I64, P, P, P]
+        _lib.mxo_quantize_nvfp4_2d.restype = I
         _lib.mxo_mxfp4_to_fp8_blocks.argtypes = [P, P, I64, I64, P, P, P]
         _lib.mxo_mxfp4_to_fp8_blocks.restype = I
     return _lib
@@ -146,6 +148,19 @@ def quantize_nvfp4(x_bf16_bits: np.ndarray):
     g = np.zeros(1, dtype=np.float32)
     _check(lib().mxo_quantize_nvfp4(_ptr(x), rows, cols, _ptr(elems), _ptr(scales), _ptr(g)),
            "quantize_nvfp4")
+    return elems, scales, float(g[0])
+
+
+def quantize_nvfp4_2d(x_bf16_bits: np.ndarray):
+    """NVFP4 with 16 x 16 weight blocks.  Returns (elems rows x cols/2, scales rows x cols/16
+    with each 2-D block's code on its 16 rows, g)."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    rows, cols = x.shape
+    elems = np.zeros((rows, cols // 2), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 16), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    _check(lib().mxo_quantize_nvfp4_2d(_ptr(x), rows, cols, _ptr(elems), _ptr(scales), _ptr(g)),
+           "quantize_nvfp4_2d")
     return elems, scales, float(g[0])
 
 

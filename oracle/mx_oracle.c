@@ -392,52 +392,88 @@ int mxo_cast(const uint16_t *x, int64_t n, int fmt, uint8_t *out) {
  * g is written to *g_out.  rows x cols row-major; blocks along rows (cols % 16 == 0);
  * elems rows x cols/2 bytes (even index low nibble), scales rows x cols/16.
  */
-int mxo_quantize_nvfp4(const uint16_t *x, int64_t rows, int64_t cols, uint8_t *elems,
-                       uint8_t *scales, float *g_out) {
+/* One NVFP4 block of nr rows x 16 columns at (r0, c0) (steps 3-4 above); writes its codes
+ * into elems (packed, row pitch cols/2) and returns the UE4M3 scale code. */
+static unsigned nvfp4_block(const uint16_t *x, int64_t cols, int64_t r0, int64_t c0, int nr, float g,
+                            uint8_t *elems) {
     const int B = 16;
-    if (cols % B) return -1;
+    float amax_b = 0.0f;
+    int nonfinite = 0;
+    for (int rr = 0; rr < nr; rr++)
+        for (int i = 0; i < B; i++) {
+            double v = bf16_value(x[(r0 + rr) * cols + c0 + i]);
+            if (isnan(v) || isinf(v)) nonfinite = 1;
+            else if ((float)fabs(v) > amax_b) amax_b = (float)fabs(v);
+        }
+    if (nonfinite) {
+        for (int rr = 0; rr < nr; rr++)
+            for (int i = 0; i < B; i++) put_code(elems + (r0 + rr) * (cols / 2), c0 + i, 0, 1);
+        return 0x7Fu;
+    }
+    volatile float six_g = 6.0f * g;
+    volatile float t = amax_b / six_g;
+    unsigned sb = mxo_encode((double)t, K_UE4M3);
+    volatile float d = (float)decode_sem(fmt_of(K_UE4M3), sb) * g;
+    for (int rr = 0; rr < nr; rr++)
+        for (int i = 0; i < B; i++) {
+            unsigned q = 0;
+            if (d != 0.0f) {
+                volatile float rcp = 1.0f / d;
+                volatile float xi = (float)bf16_value(x[(r0 + rr) * cols + c0 + i]);
+                volatile float y = xi * rcp;
+                if (isnan(y)) y = xi;     /* 0 * Inf when 1/d overflows: keep the signed zero */
+                q = mxo_encode((double)y, K_E2M1);
+            }
+            put_code(elems + (r0 + rr) * (cols / 2), c0 + i, q, 1);
+        }
+    return sb;
+}
+
+/* Steps 1-2: the per-tensor decode scale g. */
+static float nvfp4_global_scale(const uint16_t *x, int64_t n) {
     float amax_t = 0.0f;
-    for (int64_t i = 0; i < rows * cols; i++) {
+    for (int64_t i = 0; i < n; i++) {
         double v = bf16_value(x[i]);
         if (!isnan(v) && !isinf(v) && (float)fabs(v) > amax_t) amax_t = (float)fabs(v);
     }
     volatile float g = amax_t == 0.0f ? 1.0f : amax_t / 2688.0f;
+    return g;
+}
+
+int mxo_quantize_nvfp4(const uint16_t *x, int64_t rows, int64_t cols, uint8_t *elems,
+                       uint8_t *scales, float *g_out) {
+    const int B = 16;
+    if (cols % B) return -1;
+    const float g = nvfp4_global_scale(x, rows * cols);
     *g_out = g;
     memset(elems, 0, (size_t)(rows * cols / 2));
-    for (int64_t r = 0; r < rows; r++) {
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t b = 0; b < cols / B; b++)
+            scales[r * (cols / B) + b] = (uint8_t)nvfp4_block(x, cols, r, b * B, 1, g, elems);
+    return 0;
+}
+
+/*
+ * Two-dimensional NVFP4 block scaling for weights (Q§4: the 4-bit pre-training recipe
+ * uses two-dimensional block scaling for the weights).  The block is 16 x 16: one UE4M3
+ * scale per 16 rows x 16 columns, the same steps 1-4 over its 256 entries.  The scales
+ * are written in the 1 x 16 layout (rows x cols/16), each 2-D block's code repeated on its
+ * 16 rows, so every 1 x 16 consumer (dequantisation, the matmul) reads them unchanged;
+ * the transposed matrix quantised the same way gives the transposed codes and scales.
+ * rows and cols are multiples of 16.
+ */
+int mxo_quantize_nvfp4_2d(const uint16_t *x, int64_t rows, int64_t cols, uint8_t *elems,
+                          uint8_t *scales, float *g_out) {
+    const int B = 16;
+    if (cols % B || rows % B) return -1;
+    const float g = nvfp4_global_scale(x, rows * cols);
+    *g_out = g;
+    memset(elems, 0, (size_t)(rows * cols / 2));
+    for (int64_t rb = 0; rb < rows / B; rb++)
         for (int64_t b = 0; b < cols / B; b++) {
-            const uint16_t *blk = x + r * cols + b * B;
-            float amax_b = 0.0f;
-            int nonfinite = 0;
-            for (int i = 0; i < B; i++) {
-                double v = bf16_value(blk[i]);
-                if (isnan(v) || isinf(v)) nonfinite = 1;
-                else if ((float)fabs(v) > amax_b) amax_b = (float)fabs(v);
-            }
-            unsigned sb;
-            if (nonfinite) {
-                sb = 0x7Fu;
-                for (int i = 0; i < B; i++) put_code(elems + r * (cols / 2), b * B + i, 0, 1);
-            } else {
-                volatile float six_g = 6.0f * g;
-                volatile float t = amax_b / six_g;
-                sb = mxo_encode((double)t, K_UE4M3);
-                volatile float d = (float)decode_sem(fmt_of(K_UE4M3), sb) * g;
-                for (int i = 0; i < B; i++) {
-                    unsigned q = 0;
-                    if (d != 0.0f) {
-                        volatile float rcp = 1.0f / d;
-                        volatile float xi = (float)bf16_value(blk[i]);
-                        volatile float y = xi * rcp;
-                        if (isnan(y)) y = xi;     /* 0 * Inf when 1/d overflows: keep the signed zero */
-                        q = mxo_encode((double)y, K_E2M1);
-                    }
-                    put_code(elems + r * (cols / 2), b * B + i, q, 1);
-                }
-            }
-            scales[r * (cols / B) + b] = (uint8_t)sb;
+            const unsigned sb = nvfp4_block(x, cols, rb * B, b * B, B, g, elems);
+            for (int rr = 0; rr < B; rr++) scales[(rb * B + rr) * (cols / B) + b] = (uint8_t)sb;
         }
-    }
     return 0;
 }
 

@@ -1,0 +1,84 @@
+"""GPU parity of the nested-block conversion (MXFP4 1 x 32 tiles -> FP8 E4M3 with 128 x 128
+block scales) against the oracle, through the C ABI: codes, block scales and exactness
+flags bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import microscaling_precision_number_b200 as mx
+    from microscaling_precision_number_b200 import _lib as L
+
+
+@pytest.fixture(autouse=True)
+def _no_watchdog():
+    yield
+    assert mx.watchdog_status(clear=True) == 0
+
+
+def run(elems, scales, rows, cols):
+    e = torch.from_numpy(np.ascontiguousarray(elems).reshape(-1)).cuda()
+    s = torch.from_numpy(np.ascontiguousarray(scales).reshape(-1)).cuda()
+    out = torch.empty(rows * cols, dtype=torch.uint8, device="cuda")
+    bs = torch.empty((rows // 128) * (cols // 128), dtype=torch.float32, device="cuda")
+    ok = torch.empty((rows // 128) * (cols // 128), dtype=torch.uint8, device="cuda")
+    st = L.lib.mx_mxfp4_to_fp8_blocks(e.data_ptr(), s.data_ptr(), rows, cols, out.data_ptr(), bs.data_ptr(),
+                                      ok.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert st == L.MX_OK
+    return out.cpu().numpy().reshape(rows, cols), bs.cpu().numpy().reshape(rows // 128, cols // 128), \
+        ok.cpu().numpy().reshape(rows // 128, cols // 128)
+
+
+def check(oracle, elems, scales, rows, cols):
+    got = run(elems, scales, rows, cols)
+    ref = oracle.mxfp4_to_fp8_blocks(elems, scales, rows, cols)
+    for g, r, what in zip(got, ref, ("codes", "block scales", "exact flags")):
+        assert np.array_equal(g, r), what
+    return ref
+
+
+@pytest.mark.parametrize("shape", [(128, 128), (256, 512), (384, 1024)])
+def test_quantised_weights(oracle, shape):
+    x = synth.weight_fp4(*shape, seed=shape[1])
+    e, s = oracle.quantize_mx(x, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    _, _, ok = check(oracle, e, s, *shape)
+    assert np.all(ok == 1)
+
+
+def test_arbitrary_codes_and_scales(oracle):
+    """Random code bytes with random scales (every E8M0 code incl. NaN, wide gaps inside a
+    block, all-zero tiles with large scales): every path of the kernel."""
+    rng = np.random.default_rng(3)
+    rows, cols = 512, 512
+    e = rng.integers(0, 256, size=(rows, cols // 2), dtype=np.uint8)
+    s = rng.integers(0, 256, size=(rows, cols // 32), dtype=np.uint8)
+    e[0:16] = 0                                   # zero tiles in the first block
+    s[200:328, 4:8] = rng.integers(120, 135, size=(128, 4), dtype=np.uint8)   # narrow spread
+    _, _, ok = check(oracle, e, s, rows, cols)
+    assert 0 in ok and 1 in ok
+
+
+@pytest.mark.parametrize("gap,low", [(14, 0.5), (15, 0.5), (15, 1.0), (16, 1.0), (15, 1.5), (40, 1.0), (140, 1.0)])
+def test_scale_gap_edges(oracle, gap, low):
+    x = np.zeros((128, 256), dtype=np.float32)
+    x[0, 0] = 6.0
+    x[5, 32] = low * 2.0 ** -gap if gap < 130 else 0.0
+    x[9, 200] = 3.0 * 2.0 ** -(gap % 64)
+    bits = (torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    e, s = oracle.quantize_mx(bits, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    if gap >= 130:                                 # a tile far below via its scale byte only
+        s[5, 1] = 3
+        e[5, 16] = 0x02
+    check(oracle, e, s, 128, 256)
+
+
+def test_config5_weight(oracle):
+    """The mixed-GEMM weight shape (14336 x 4096, N(0, 0.02)) end to end."""
+    x = synth.normal(14336, 4096, sigma=0.02, seed=51)
+    e, s = oracle.quantize_mx(x, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    _, _, ok = check(oracle, e, s, 14336, 4096)
+    assert np.all(ok == 1)

@@ -366,3 +366,47 @@ def test_tcgen05_tiling_is_a_padded_bijection(oracle):
     assert sorted(off.ravel()) == list(range(512))
     assert np.all(np.diff(off, axis=1) == 1)
     assert np.all(off[32:64] - off[0:32] == 4)
+
+
+# ------------------------------------------------------------------ NVFP4 16 x 16 weight blocks
+def test_nvfp4_2d_blocks_commute_with_transposition(oracle):
+    """Two-dimensional blocks make the weight and its transpose quantise identically ([Q] §4:
+    2-D block scaling for weights): codes and block scales of W^T are those of W, transposed."""
+    x = synth.weight_fp4(64, 96, seed=31)
+    e, s, g = oracle.quantize_nvfp4_2d(x)
+    et, st, gt = oracle.quantize_nvfp4_2d(np.ascontiguousarray(x.T))
+    assert g == gt
+    codes = np.stack([unpack_fp4(r, 96) for r in e])
+    codes_t = np.stack([unpack_fp4(r, 64) for r in et])
+    assert np.array_equal(codes_t, codes.T)
+    blk = s[::16]                                   # one row per 16-row group
+    blk_t = st[::16]
+    assert np.array_equal(blk_t, blk.T)
+    for r in range(64):                             # every row of a group carries its block's scale
+        assert np.array_equal(s[r], s[(r // 16) * 16])
+
+
+def test_nvfp4_2d_reduces_to_1d_on_single_row_blocks(oracle):
+    """A matrix whose 16-row groups each hold one nonzero row: every 2-D block's maximum is
+    that row's 1 x 16 maximum, so the row's codes and scales equal the (pinned) 1-D NVFP4
+    quantisation of the same matrix."""
+    x = synth.weight_fp4(48, 64, seed=32)
+    keep = np.zeros_like(x)
+    for grp in range(3):
+        keep[grp * 16 + 5 * grp] = x[grp * 16 + 5 * grp]
+    e2, s2, g2 = oracle.quantize_nvfp4_2d(keep)
+    e1, s1, g1 = oracle.quantize_nvfp4(keep)
+    assert g1 == g2
+    for grp in range(3):
+        r = grp * 16 + 5 * grp
+        assert np.array_equal(e2[r], e1[r]) and np.array_equal(s2[r], s1[r])
+
+
+def test_nvfp4_2d_nonfinite_block(oracle):
+    x = synth.normal(32, 32, seed=33)
+    x[20, 3] = 0x7FC0                              # NaN in block (1, 0)
+    e, s, g = oracle.quantize_nvfp4_2d(x)
+    assert np.all(s[16:32, 0] == 0x7F) and np.all(s[:16, 0] != 0x7F) and np.all(s[:, 1] != 0x7F)
+    codes = np.stack([unpack_fp4(r, 32) for r in e])
+    assert np.all(codes[16:32, :16] == 0)
+    assert math.isfinite(g)
