@@ -161,6 +161,19 @@ mx_status mx_quantize_nvfp4_noalloc(const void *src_bf16, int64_t rows, int64_t 
                                     float *global_scale, mx_stream_t stream);
 
 /*
+ * mx_quantize_nvfp4_2d -- NVFP4 with two-dimensional 16 x 16 blocks, for weights ([Q] §4:
+ * the 4-bit pre-training recipe scales weights in two-dimensional blocks, so that a weight
+ * and its transpose quantise identically).  Same steps as mx_quantize(fmt = NVFP4) with the
+ * block maximum taken over 16 rows x 16 columns; each block's UE4M3 scale is written to all
+ * 16 of its rows in the usual 1 x 16 layouts (rows x cols/16), so mx_dequantize and mx_gemm
+ * consume the result unchanged.  Arguments as mx_quantize with fmt = NVFP4, axis = ROW;
+ * rows and cols are multiples of 16 (else MX_ERR_SHAPE).
+ */
+mx_status mx_quantize_nvfp4_2d(const void *src_bf16, int64_t rows, int64_t cols, void *out_elems,
+                               uint8_t *out_scales, mx_scale_layout layout, uint8_t *out_scales_alt,
+                               float *global_scale, mx_stream_t stream);
+
+/*
  * mx_quantize_dual -- one pass over a bf16 matrix producing both orientations ([Q] §6:
  * training needs the row-wise copy for the forward matmul and the column-wise copy for
  * the weight-gradient matmul).  The input is read once.

@@ -98,6 +98,23 @@ def quantize(x: torch.Tensor, fmt="e4m3", axis: str = "row", rounding: str = "ce
     return Quantized(elems, scales, alt, g, orows, ocols, f)
 
 
+def quantize_nvfp4_2d(x: torch.Tensor, layout: str = "tcgen05", stream=None) -> Quantized:
+    """NVFP4 with 16 x 16 weight blocks (scales repeated on the 16 rows of each block)."""
+    _check_src(x)
+    rows, cols = x.shape
+    dev = x.device
+    first = "rowmajor" if layout in ("rowmajor", "both") else "tcgen05"
+    elems = torch.empty(rows * cols // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(scale_bytes(rows, cols // 16, first), dtype=torch.uint8, device=dev)
+    alt = torch.empty(scale_bytes(rows, cols // 16, "tcgen05"), dtype=torch.uint8, device=dev) \
+        if layout == "both" else None
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    L.check(L.lib.mx_quantize_nvfp4_2d(x.data_ptr(), rows, cols, elems.data_ptr(), scales.data_ptr(),
+                                       LAYOUTS[layout], _ptr(alt), g.data_ptr(), _stream(stream)),
+            "mx_quantize_nvfp4_2d")
+    return Quantized(elems, scales, alt, g, rows, cols, L.MX_FMT_NVFP4)
+
+
 def quantize_dual(x: torch.Tensor, fmt="e4m3", rounding: str = "ceil", layout: str = "tcgen05", stream=None,
                   out: Optional[tuple] = None):
     """Row-wise and column-wise (transposed) quantisation from one read of x.  `out` (the

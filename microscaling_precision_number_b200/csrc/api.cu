@@ -126,6 +126,19 @@ mx_status mx_watchdog_status(int *code, int clear) {
     return v ? MX_ERR_TIMEOUT : MX_OK;
 }
 
+// One fixed-size scratch per device for the NVFP4 per-CTA partial maxima, allocated on
+// first use (every call writes each slot it later reads).
+static mx_status nvfp4_scratch(DeviceState *d) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!d->partials) {
+        const int nf = mxk::stream_nvfp4_scratch_floats(d->num_sms);
+        const cudaError_t e = cudaMalloc(reinterpret_cast<void **>(&d->partials), sizeof(float) * (size_t)nf);
+        if (e != cudaSuccess) return cuda_fail(e);
+        d->partials_cap = nf;
+    }
+    return MX_OK;
+}
+
 mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, mx_axis axis,
                       mx_scale_rounding rounding, void *out_elems, uint8_t *out_scales,
                       mx_scale_layout layout, uint8_t *out_scales_alt, float *global_scale,
@@ -162,17 +175,8 @@ mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, m
     const bool ceil = rounding == MX_SCALE_CEIL_RECIPE;
 
     if (fmt == MX_FMT_NVFP4) {
-        {
-            // one fixed-size scratch per device for the per-CTA partial maxima, allocated on
-            // first use (every call writes each slot it later reads)
-            std::lock_guard<std::mutex> lock(g_mu);
-            if (!d->partials) {
-                const int nf = mxk::stream_nvfp4_scratch_floats(d->num_sms);
-                e = cudaMalloc(reinterpret_cast<void **>(&d->partials), sizeof(float) * (size_t)nf);
-                if (e != cudaSuccess) return cuda_fail(e);
-                d->partials_cap = nf;
-            }
-        }
+        st = nvfp4_scratch(d);
+        if (st != MX_OK) return st;
         e = mxk::launch_stream_nvfp4(src, rows, cols, d->partials, 3 * d->num_sms, global_scale, out_elems, rm, tc,
                                      d->watchdog, d->num_sms, s);
         if (e != cudaSuccess) return cuda_fail(e);
@@ -328,6 +332,35 @@ mx_status mx_mxfp4_to_fp8_blocks(const void *elems, const uint8_t *scales, int64
     if (st != MX_OK) return st;
     const cudaError_t e = mxk::launch_mxfp4_to_fp8_blocks(elems, scales, rows, cols, out_fp8, block_scales,
                                                           block_exact, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MX_OK : cuda_fail(e);
+}
+
+mx_status mx_quantize_nvfp4_2d(const void *src, int64_t rows, int64_t cols, void *out_elems, uint8_t *out_scales,
+                               mx_scale_layout layout, uint8_t *out_scales_alt, float *global_scale,
+                               mx_stream_t stream) {
+    if (layout != MX_LAYOUT_ROWMAJOR && layout != MX_LAYOUT_TCGEN05 &&
+        layout != (MX_LAYOUT_ROWMAJOR | MX_LAYOUT_TCGEN05))
+        return MX_ERR_LAYOUT;
+    const bool both = layout == (MX_LAYOUT_ROWMAJOR | MX_LAYOUT_TCGEN05);
+    if (both != (out_scales_alt != nullptr)) return MX_ERR_LAYOUT;
+    if (rows < 0 || cols < 0 || rows % 16 || cols % 16) return MX_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MX_OK;
+    if (!mxk::stream_supported(rows, cols)) return MX_ERR_SHAPE;
+    if (!src || !out_elems || !out_scales || !global_scale) return MX_ERR_ARG;
+    if (!aligned(src, 16) || !aligned(out_elems, 16) || !aligned(global_scale, 4)) return MX_ERR_ALIGN;
+    uint8_t *rm = nullptr, *tc = nullptr;
+    if (both) { rm = out_scales; tc = out_scales_alt; }
+    else if (layout == MX_LAYOUT_ROWMAJOR) rm = out_scales;
+    else tc = out_scales;
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    st = nvfp4_scratch(d);
+    if (st != MX_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mxk::launch_stream_nvfp4_2d(src, rows, cols, d->partials, d->partials_cap, global_scale,
+                                                out_elems, rm, tc, d->num_sms, d->watchdog, s);
+    if (e == cudaSuccess && tc) e = mxk::launch_tcgen05_pad(tc, rows, cols / 16, s);
     return e == cudaSuccess ? MX_OK : cuda_fail(e);
 }
 

@@ -25,6 +25,11 @@ cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, flo
                                 float *global_scale, void *elems, uint8_t *sc_rowmajor, uint8_t *sc_tcgen05,
                                 int *watchdog, int num_sms, cudaStream_t st);
 
+// NVFP4 with 16 x 16 blocks (rows, cols multiples of 16); scales in the 1 x 16 layouts.
+cudaError_t launch_stream_nvfp4_2d(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,
+                                   float *g, void *elems, uint8_t *rm, uint8_t *tc, int num_sms, int *wd,
+                                   cudaStream_t st);
+
 cudaError_t launch_stream_dequant_mx(const void *elems, const uint8_t *scales, int64_t rows, int64_t cols, int fmt,
                                      bool tcgen05, void *out, int *watchdog, int num_sms, cudaStream_t st);
 cudaError_t launch_stream_dequant_nvfp4(const void *elems, const uint8_t *scales, const float *g, int64_t rows,

@@ -410,6 +410,76 @@ nvfp4_quant_bulk_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fast
 }
 
 // ---------------------------------------------------------------------------------------
+// NVFP4 with 16 x 16 weight blocks (two-dimensional block scaling for weights, the 4-bit
+// pre-training recipe): second pass after nvfp4_amax_bulk_kernel.  One thread per 16 x 16
+// block; lanes of a warp take neighbouring blocks, so each row of 16 blocks is one
+// coalesced 1 KiB read.  The block maximum covers 256 entries; every other step is the
+// 1 x 16 path's (same fp32 operations in the same order), and the scale is written to the
+// 16 rows of the block in the 1 x 16 layouts.
+// ---------------------------------------------------------------------------------------
+template <bool RM, bool TC>
+__global__ void __launch_bounds__(kThreads)
+nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t n_blocks, FastDiv div_bc,
+                      uint32_t col_atoms, const float *__restrict__ partials, int n_partials,
+                      float *__restrict__ g_out, uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm,
+                      uint8_t *__restrict__ sc_tc) {
+    pdl_wait_and_release();
+    __shared__ float warp_max[kThreads / 32];
+    __shared__ float rtab[128];
+    const float g = nvfp4_global_scale(partials, n_partials, warp_max);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    const Nvfp4Consts cst = nvfp4_consts(g, rtab);
+    const uint32_t S = cols / 16;                                  // scale columns per row
+    for (uint32_t b = blockIdx.x * kThreads + threadIdx.x; b < n_blocks; b += gridDim.x * kThreads) {
+        const uint32_t rb = fdiv(b, div_bc), cb = b - rb * div_bc.d;
+        const uint8_t *base = src + ((size_t)rb * 16 * cols + (size_t)cb * 16) * 2;
+        uint32_t m = 0;
+#pragma unroll 4
+        for (int rr = 0; rr < 16; rr++) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(base + (size_t)rr * cols * 2);
+            m = max(m, absmax_block16(p[0], p[1]));
+        }
+        const bool special = m >= 0x7F80u;                         // Inf/NaN in the block
+        const float a = __uint_as_float(m << 16);
+        float tq;
+        if (cst.fast) {
+            const float q0 = __fmul_rn(a, cst.y);
+            tq = __fmaf_rn(__fmaf_rn(-q0, cst.six_g, a), cst.y, q0);
+        } else {
+            tq = __fdiv_rn(a, cst.six_g);
+        }
+        uint32_t sb = cvt_fp8x2<FMT_E4M3>(tq, 0.0f) & 0xFFu;
+        const float r = rtab[sb & 0x7Fu];
+        const bool zero_codes = special || r == 0.0f;
+        if (special) sb = 0x7Fu;
+        const uint64_t r2 = splat2(r);
+#pragma unroll 4
+        for (int rr = 0; rr < 16; rr++) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(base + (size_t)rr * cols * 2);
+            uint32_t q[2];
+#pragma unroll
+            for (int j = 0; j < 2; j++) {
+                const uint4 v = p[j];
+                float x[8];
+                scale8(v, r2, x);
+                if (__builtin_expect(isinf(r), 0)) {
+                    const float in[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                                         bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+#pragma unroll
+                    for (int i = 0; i < 8; i++)
+                        if (x[i] != x[i]) x[i] = in[i];            // 0 * Inf: keep the signed zero
+                }
+                q[j] = zero_codes ? 0u : cvt_e2m1x8(x);
+            }
+            const uint32_t row = rb * 16 + rr;
+            reinterpret_cast<uint2 *>(elems)[((size_t)row * cols + (size_t)cb * 16) >> 4] = make_uint2(q[0], q[1]);
+            if constexpr (RM) sc_rm[(size_t)row * S + cb] = (uint8_t)sb;
+            if constexpr (TC) sc_tc[tc_offset(row, cb, col_atoms)] = (uint8_t)sb;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
 // Dequantisers: thread = one block; codes streamed through the ring, scales read
 // directly, bf16 written as 16-byte vectors.
 // ---------------------------------------------------------------------------------------
@@ -634,6 +704,33 @@ static cudaError_t launch_nvfp4_t(const uint8_t *src, uint32_t nb, FastDiv f, ui
     if (e != cudaSuccess) return e;
     return launch_stream(nvfp4_quant_bulk_kernel<RM, TC>, stream_grid(n_tiles, num_sms), st, src, nb, f, ca,
                          (const float *)partials, grid, g, elems, rm, tc, wd);
+}
+
+template <bool RM, bool TC>
+static cudaError_t launch_nvfp4_2d_t(const uint8_t *src, int64_t rows, int64_t cols, float *partials,
+                                     int max_partials, float *g, uint8_t *elems, uint8_t *rm, uint8_t *tc, int *wd,
+                                     int num_sms, cudaStream_t st) {
+    const uint64_t nbytes = (uint64_t)rows * cols * 2;
+    const uint32_t n_tiles = (uint32_t)((nbytes + kTileBytes - 1) / kTileBytes);
+    int grid = stream_grid(n_tiles, num_sms);
+    if (grid > max_partials) grid = max_partials;
+    cudaError_t e = launch_stream(nvfp4_amax_bulk_kernel, grid, st, src, nbytes, partials, wd);
+    if (e != cudaSuccess) return e;
+    const uint32_t bc = (uint32_t)(cols / 16), n_blocks = (uint32_t)(rows / 16) * bc;
+    int grid2 = (int)((n_blocks + kThreads - 1) / kThreads);
+    if (grid2 > kCtasPerSm * num_sms) grid2 = kCtasPerSm * num_sms;
+    return launch_stream(nvfp4_2d_quant_kernel<RM, TC>, grid2, st, src, (uint32_t)cols, n_blocks, make_fastdiv(bc),
+                         (bc + 3) / 4, (const float *)partials, grid, g, elems, rm, tc);
+}
+
+cudaError_t launch_stream_nvfp4_2d(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,
+                                   float *g, void *elems, uint8_t *rm, uint8_t *tc, int num_sms, int *wd,
+                                   cudaStream_t st) {
+    const uint8_t *s8 = static_cast<const uint8_t *>(src);
+    uint8_t *e8 = static_cast<uint8_t *>(elems);
+    if (rm && tc) return launch_nvfp4_2d_t<true, true>(s8, rows, cols, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
+    if (rm) return launch_nvfp4_2d_t<true, false>(s8, rows, cols, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
+    return launch_nvfp4_2d_t<false, true>(s8, rows, cols, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
 }
 
 cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,

@@ -77,6 +77,8 @@ def lib():
         _lib.mxo_tcgen05_scale_offset.restype = I64
         _lib.mxo_gemm_ref.argtypes = [P, P, I, ctypes.c_double, P, P, I, ctypes.c_double, I64, I64, I64, P, I64, P, P]
         _lib.mxo_gemm_ref.restype = I
+        _lib.mxo_rht16.argtypes = [P, I64, I64, ctypes.c_uint, P]
+        _lib.mxo_rht16.restype = I
         _lib.mxo_quantize_nvfp4_2d.argtypes = [P, I64, I64, P, P, P]
         _lib.mxo_quantize_nvfp4_2d.restype = I
         _lib.mxo_mxfp4_to_fp8_blocks.argtypes = [P, P, I64, I64, P, P, P]
@@ -237,3 +239,12 @@ def mxfp4_to_fp8_blocks(elems: np.ndarray, scales: np.ndarray, rows: int, cols: 
     _check(lib().mxo_mxfp4_to_fp8_blocks(_ptr(e), _ptr(s), rows, cols, _ptr(out), _ptr(bs), _ptr(ok)),
            "mxfp4_to_fp8_blocks")
     return out, bs, ok
+
+
+def rht16(x_bf16_bits: np.ndarray, sign_mask: int) -> np.ndarray:
+    """16 x 16 random Hadamard transform of every 16 consecutive elements of each row
+    (H16 D x / 4, fp32 butterflies, bf16 result), as bf16 bits."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    out = np.zeros_like(x)
+    _check(lib().mxo_rht16(_ptr(x), x.shape[0], x.shape[1], sign_mask, _ptr(out)), "rht16")
+    return out

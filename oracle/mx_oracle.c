@@ -645,3 +645,42 @@ int mxo_mxfp4_to_fp8_blocks(const uint8_t *elems, const uint8_t *scales, int64_t
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* 16 x 16 random Hadamard transform (Q§4: the 4-bit pre-training recipe      */
+/* applies a 16 x 16 random Hadamard transform to the inputs of the weight    */
+/* gradient).  The pages name the transform but not its form; reading:        */
+/*   for every 16 consecutive elements x of a row: y = H16 D x / 4, with      */
+/*   D = diag(+-1) from a 16-bit sign mask (bit i set: element i negated) and */
+/*   H16 the Sylvester Hadamard matrix (H1 = [1], H2n = [[Hn, Hn], [Hn, -Hn]]),*/
+/*   so that H16 D / 4 is orthogonal; computed as the radix-2 butterfly      */
+/*   (strides 1, 2, 4, 8; (a, b) -> (a + b, a - b)) in fp32 round-to-nearest, */
+/*   the 1/4 applied last (exact), and the result rounded to bf16 (the       */
+/*   tensor's type) before it is quantised.                                  */
+/* ------------------------------------------------------------------------- */
+static void rht16(const uint16_t *x, unsigned sign_mask, uint16_t *y) {
+    volatile float v[16];
+    for (int i = 0; i < 16; i++) {
+        float f = (float)bf16_value(x[i]);
+        v[i] = ((sign_mask >> i) & 1u) ? -f : f;
+    }
+    for (int h = 1; h < 16; h <<= 1)
+        for (int i = 0; i < 16; i += 2 * h)
+            for (int j = i; j < i + h; j++) {
+                volatile float a = v[j], b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+    for (int i = 0; i < 16; i++) {
+        volatile float q = v[i] * 0.25f;
+        y[i] = f32_to_bf16(q);
+    }
+}
+
+/* The transform of a rows x cols bf16 matrix (cols % 16 == 0), row by row. */
+int mxo_rht16(const uint16_t *x, int64_t rows, int64_t cols, unsigned sign_mask, uint16_t *out) {
+    if (cols % 16) return -1;
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c += 16) rht16(x + r * cols + c, sign_mask & 0xFFFFu, out + r * cols + c);
+    return 0;
+}

@@ -307,3 +307,28 @@ def test_output_buffers_are_reused(oracle):
     with pytest.raises(ValueError):
         mx.quantize(x, "e4m3", "row", "ceil", layout="both", out=mx.Quantized(q.elems[:10], q.scales, q.scales_alt,
                                                                              None, 64, 256, q.fmt))
+
+
+# ------------------------------------------------------------------ NVFP4 16 x 16 weight blocks
+@pytest.mark.parametrize("shape", [(16, 16), (48, 96), (160, 256), (1024, 4096)])
+def test_nvfp4_2d_matches_oracle(oracle, shape):
+    x = with_specials(synth.weight_fp4(*shape, seed=shape[0] + 1), seed=shape[1] + 1)
+    q = mx.quantize_nvfp4_2d(to_dev(x), layout="both")
+    e, s, g = oracle.quantize_nvfp4_2d(x)
+    assert host(q.global_scale)[0] == np.float32(g)
+    assert np.array_equal(host(q.elems), e.reshape(-1))
+    assert np.array_equal(host(q.scales), s.reshape(-1))
+    assert np.array_equal(host(q.scales_alt), oracle.to_tcgen05_layout(s))
+
+
+def test_nvfp4_2d_weight_transposes(oracle):
+    """The weight and its transpose quantise to transposed codes and block scales on the GPU."""
+    x = synth.weight_fp4(256, 512, seed=9)
+    q = mx.quantize_nvfp4_2d(to_dev(x), layout="rowmajor")
+    qt = mx.quantize_nvfp4_2d(to_dev(np.ascontiguousarray(x.T)), layout="rowmajor")
+    e = host(q.elems).reshape(256, 256)
+    et = host(qt.elems).reshape(512, 128)
+    codes = np.stack([np.stack([r & 0xF, r >> 4], axis=1).reshape(-1) for r in e])
+    codes_t = np.stack([np.stack([r & 0xF, r >> 4], axis=1).reshape(-1) for r in et])
+    assert np.array_equal(codes_t, codes.T)
+    assert np.array_equal(host(q.scales).reshape(256, 32)[::16], host(qt.scales).reshape(512, 16)[::16].T)

@@ -410,3 +410,43 @@ def test_nvfp4_2d_nonfinite_block(oracle):
     codes = np.stack([unpack_fp4(r, 32) for r in e])
     assert np.all(codes[16:32, :16] == 0)
     assert math.isfinite(g)
+
+
+# ------------------------------------------------------------------ 16 x 16 random Hadamard transform
+def test_rht16_matches_matrix_product(oracle):
+    """On inputs whose butterfly sums are exact in fp32 (small integers and halves), the
+    transform equals scipy's Sylvester Hadamard matrix times the sign-flipped input, / 4,
+    rounded once to bf16 (torch's RNE conversion)."""
+    from scipy.linalg import hadamard
+    rng = np.random.default_rng(41)
+    x = (rng.integers(-64, 65, size=(8, 64)) * 0.5).astype(np.float32)
+    bits = f32_to_bf16_bits(x).reshape(8, 64)
+    H = hadamard(16).astype(np.float64)
+    for mask in (0x0000, 0xFFFF, 0xA5C3, 0x1234):
+        d = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(16)])
+        y = bf16_bits_to_f64(oracle.rht16(bits, mask))
+        xf = bf16_bits_to_f64(bits)
+        ref = np.concatenate([(H @ (d[:, None] * xf[:, c:c + 16].T)).T / 4 for c in range(0, 64, 16)], axis=1)
+        ref = torch.from_numpy(ref).to(torch.bfloat16).double().numpy()
+        assert np.array_equal(y, ref)
+
+
+def test_rht16_is_orthogonal(oracle):
+    """H16 D / 4 is orthogonal: D H16 / 4 undoes it (exactly on exact inputs), and norms are
+    kept up to the bf16 rounding of the outputs."""
+    from scipy.linalg import hadamard
+    rng = np.random.default_rng(42)
+    x = (rng.integers(-8, 9, size=(4, 32)) * 0.25).astype(np.float32)   # outputs exact in bf16
+    bits = f32_to_bf16_bits(x).reshape(4, 32)
+    mask = 0x6C39
+    y = bf16_bits_to_f64(oracle.rht16(bits, mask))
+    d = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(16)])
+    H = hadamard(16).astype(np.float64)
+    back = np.concatenate([(d[:, None] * (H @ y[:, c:c + 16].T)).T / 4 for c in (0, 16)], axis=1)
+    assert np.array_equal(back, bf16_bits_to_f64(bits))
+    z = bf16_bits_to_f64(oracle.rht16(synth.normal(16, 256, seed=43), 0xBEEF))
+    zi = bf16_bits_to_f64(synth.normal(16, 256, seed=43))
+    for r in range(16):
+        for c in range(0, 256, 16):
+            n0, n1 = np.linalg.norm(zi[r, c:c + 16]), np.linalg.norm(z[r, c:c + 16])
+            assert abs(n1 - n0) <= 2.0 ** -7 * n0
