@@ -77,6 +77,10 @@ def lib():
         _lib.mxo_tcgen05_scale_offset.restype = I64
         _lib.mxo_gemm_ref.argtypes = [P, P, I, ctypes.c_double, P, P, I, ctypes.c_double, I64, I64, I64, P, I64, P, P]
         _lib.mxo_gemm_ref.restype = I
+        _lib.mxo_quantize_mx_sr.argtypes = [P, I64, I64, I, I, P, P, P]
+        _lib.mxo_quantize_mx_sr.restype = I
+        _lib.mxo_quantize_nvfp4_sr.argtypes = [P, I64, I64, P, P, P, P]
+        _lib.mxo_quantize_nvfp4_sr.restype = I
         _lib.mxo_rht16.argtypes = [P, I64, I64, ctypes.c_uint, P]
         _lib.mxo_rht16.restype = I
         _lib.mxo_quantize_nvfp4_2d.argtypes = [P, I64, I64, P, P, P]
@@ -248,3 +252,30 @@ def rht16(x_bf16_bits: np.ndarray, sign_mask: int) -> np.ndarray:
     out = np.zeros_like(x)
     _check(lib().mxo_rht16(_ptr(x), x.shape[0], x.shape[1], sign_mask, _ptr(out)), "rht16")
     return out
+
+
+def quantize_mx_sr(x_bf16_bits: np.ndarray, fmt: int, rounding: int, rnd: np.ndarray):
+    """Row-wise MX quantisation with stochastic rounding (one random byte per element)."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    r = np.ascontiguousarray(rnd, dtype=np.uint8)
+    assert r.shape == x.shape
+    rows, cols = x.shape
+    elems = np.zeros((rows, elem_bytes(cols, fmt)), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 32), dtype=np.uint8)
+    _check(lib().mxo_quantize_mx_sr(_ptr(x), rows, cols, fmt, rounding, _ptr(r), _ptr(elems), _ptr(scales)),
+           "quantize_mx_sr")
+    return elems, scales
+
+
+def quantize_nvfp4_sr(x_bf16_bits: np.ndarray, rnd: np.ndarray):
+    """NVFP4 with stochastic rounding of the element cast (one random byte per element)."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    r = np.ascontiguousarray(rnd, dtype=np.uint8)
+    assert r.shape == x.shape
+    rows, cols = x.shape
+    elems = np.zeros((rows, cols // 2), dtype=np.uint8)
+    scales = np.zeros((rows, cols // 16), dtype=np.uint8)
+    g = np.zeros(1, dtype=np.float32)
+    _check(lib().mxo_quantize_nvfp4_sr(_ptr(x), rows, cols, _ptr(r), _ptr(elems), _ptr(scales), _ptr(g)),
+           "quantize_nvfp4_sr")
+    return elems, scales, float(g[0])

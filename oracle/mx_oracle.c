@@ -684,3 +684,110 @@ int mxo_rht16(const uint16_t *x, int64_t rows, int64_t cols, unsigned sign_mask,
         for (int64_t c = 0; c < cols; c += 16) rht16(x + r * cols + c, sign_mask & 0xFFFFu, out + r * cols + c);
     return 0;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Stochastic rounding of the element cast (Q§4: the 4-bit pre-training      */
+/* recipe rounds gradients stochastically; Q§8: P3109 defines stochastic     */
+/* rounding).  The pages fix no procedure; reading, with one random byte r    */
+/* (0..255) per element, passed in by the caller:                            */
+/*   |y| >= the format maximum  -> the maximum (saturation, as the RNE cast); */
+/*   otherwise lo = the largest representable magnitude <= |y| and hi the    */
+/*   next one; |y| == lo -> lo; else hi when 256 (|y| - lo) > r (hi - lo),    */
+/*   lo otherwise -- probability ceil(256 f) / 256 of rounding up for         */
+/*   f = (|y| - lo) / (hi - lo), unbiased to 1/256 of a step;                 */
+/*   the sign is that of y (a zero result keeps it).                         */
+/* lo and hi are found by scanning the decoded code table (no arithmetic     */
+/* shortcut), the comparison is exact in double.                            */
+/* ------------------------------------------------------------------------- */
+static unsigned encode_sr(double y, int kind, unsigned r) {
+    fmt_t f = fmt_of(kind);
+    unsigned nbits = (unsigned)(f.has_sign + f.ebits + f.mbits);
+    unsigned sign = signbit(y) ? (1u << (nbits - 1)) : 0u;
+    unsigned mc = max_code(f);
+    double a = fabs(y);
+    if (a >= decode_sem(f, mc)) return sign | mc;
+    unsigned lo_c = 0, hi_c = mc;
+    double lo = 0.0, hi = decode_sem(f, mc);
+    for (unsigned c = 0; c <= mc; c++) {          /* magnitudes increase with the code */
+        double v = decode_sem(f, c);
+        if (isnan(v) || isinf(v)) continue;
+        if (v <= a && v >= lo) { lo = v; lo_c = c; }
+        if (v > a && v < hi) { hi = v; hi_c = c; }
+    }
+    if (a == lo) return sign | lo_c;
+    return sign | ((256.0 * (a - lo) > (double)r * (hi - lo)) ? hi_c : lo_c);
+}
+
+/* Row-wise MX quantisation with stochastic rounding of the element cast (E4M3, E5M2, E2M1;
+ * the scale is the deterministic shared exponent); rnd: rows x cols random bytes. */
+int mxo_quantize_mx_sr(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int rounding,
+                       const uint8_t *rnd, uint8_t *elems, uint8_t *scales) {
+    const int B = 32;
+    if (!(fmt == F_E4M3 || fmt == F_E5M2 || fmt == F_E2M1) || cols % B) return -1;
+    int fp4 = fmt == F_E2M1;
+    int64_t row_bytes = fp4 ? cols / 2 : cols;
+    memset(elems, 0, (size_t)(rows * row_bytes));
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t b = 0; b < cols / B; b++) {
+            const uint16_t *blk = x + r * cols + b * B;
+            double amax = 0.0;
+            int nonfinite = 0;
+            for (int i = 0; i < B; i++) {
+                double v = bf16_value(blk[i]);
+                if (isnan(v) || isinf(v)) nonfinite = 1;
+                else if (fabs(v) > amax) amax = fabs(v);
+            }
+            if (nonfinite) {
+                scales[r * (cols / B) + b] = 0xFF;
+                continue;                               /* codes stay 0 */
+            }
+            int s = mxo_scale_exponent(amax, fmt, rounding);
+            scales[r * (cols / B) + b] = (uint8_t)(s + 127);
+            for (int i = 0; i < B; i++) {
+                double scaled = ldexp(bf16_value(blk[i]), -s);
+                put_code(elems + r * row_bytes, b * B + i,
+                         encode_sr(scaled, elem_kind(fmt), rnd[r * cols + b * B + i]), fp4);
+            }
+        }
+    return 0;
+}
+
+/* NVFP4 with stochastic rounding of the element cast: steps 1-4 of the NVFP4 path, the
+ * E2M1 code of x_i * (1/d) rounded stochastically (the UE4M3 block scale stays RNE). */
+int mxo_quantize_nvfp4_sr(const uint16_t *x, int64_t rows, int64_t cols, const uint8_t *rnd,
+                          uint8_t *elems, uint8_t *scales, float *g_out) {
+    const int B = 16;
+    if (cols % B) return -1;
+    const float g = nvfp4_global_scale(x, rows * cols);
+    *g_out = g;
+    memset(elems, 0, (size_t)(rows * cols / 2));
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t b = 0; b < cols / B; b++) {
+            const uint16_t *blk = x + r * cols + b * B;
+            float amax_b = 0.0f;
+            int nonfinite = 0;
+            for (int i = 0; i < B; i++) {
+                double v = bf16_value(blk[i]);
+                if (isnan(v) || isinf(v)) nonfinite = 1;
+                else if ((float)fabs(v) > amax_b) amax_b = (float)fabs(v);
+            }
+            if (nonfinite) { scales[r * (cols / B) + b] = 0x7F; continue; }
+            volatile float six_g = 6.0f * g;
+            volatile float t = amax_b / six_g;
+            unsigned sb = mxo_encode((double)t, K_UE4M3);
+            volatile float d = (float)decode_sem(fmt_of(K_UE4M3), sb) * g;
+            scales[r * (cols / B) + b] = (uint8_t)sb;
+            for (int i = 0; i < B; i++) {
+                unsigned q = 0;
+                if (d != 0.0f) {
+                    volatile float rcp = 1.0f / d;
+                    volatile float xi = (float)bf16_value(blk[i]);
+                    volatile float y = xi * rcp;
+                    if (isnan(y)) y = xi;
+                    q = encode_sr((double)y, K_E2M1, rnd[r * cols + b * B + i]);
+                }
+                put_code(elems + r * (cols / 2), b * B + i, q, 1);
+            }
+        }
+    return 0;
+}

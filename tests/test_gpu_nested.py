@@ -57,7 +57,7 @@ def test_arbitrary_codes_and_scales(oracle):
     e = rng.integers(0, 256, size=(rows, cols // 2), dtype=np.uint8)
     s = rng.integers(0, 256, size=(rows, cols // 32), dtype=np.uint8)
     e[0:16] = 0                                   # zero tiles in the first block
-    s[200:328, 4:8] = rng.integers(120, 135, size=(128, 4), dtype=np.uint8)   # narrow spread
+    s[256:384, 4:8] = rng.integers(120, 135, size=(128, 4), dtype=np.uint8)   # narrow spread in block (2, 1)
     _, _, ok = check(oracle, e, s, rows, cols)
     assert 0 in ok and 1 in ok
 
