@@ -161,6 +161,31 @@ mx_status mx_quantize_nvfp4_noalloc(const void *src_bf16, int64_t rows, int64_t 
                                     float *global_scale, mx_stream_t stream);
 
 /*
+ * mx_quantize_train -- the training-side row-wise quantiser ([Q] §4: the 4-bit pre-training
+ * recipe applies a 16 x 16 random Hadamard transform to the inputs of the weight gradient
+ * and rounds gradients stochastically; [Q] §8: stochastic rounding is a P3109 mode).
+ * Same outputs as mx_quantize(axis = ROW) for fmt E4M3, E5M2, E2M1 or NVFP4, with:
+ *   rht16       1: every 16 consecutive elements of a row are first replaced by
+ *               H16 D x / 4 (D = diag of signs: bit i of rht_signs set negates element i;
+ *               H16 the Sylvester Hadamard matrix), computed by radix-2 butterflies
+ *               (strides 1, 2, 4, 8) in fp32 round-to-nearest and rounded to bf16; the
+ *               quantiser (scales, NVFP4 tensor scale included) sees those values.  0: none.
+ *               Applying the same transform to both operands along K leaves A * B^T
+ *               unchanged (H16 D / 4 is orthogonal).
+ *   sr_random   NULL: round to nearest even.  Else device, rows x cols random bytes (one per
+ *               element, 16-byte aligned): a scaled value strictly between its representable
+ *               neighbours lo < |y| < hi becomes hi when 256 (|y| - lo) > r (hi - lo), else
+ *               lo (probability of rounding up ceil(256 f) / 256, f the position between
+ *               them); values at or beyond the maximum saturate.  Scales are unchanged.
+ * Other arguments, shapes, layouts and errors as mx_quantize(axis = ROW).
+ */
+mx_status mx_quantize_train(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt fmt,
+                            mx_scale_rounding rounding, int rht16, unsigned rht_signs,
+                            const uint8_t *sr_random, void *out_elems, uint8_t *out_scales,
+                            mx_scale_layout layout, uint8_t *out_scales_alt, float *global_scale,
+                            mx_stream_t stream);
+
+/*
  * mx_quantize_nvfp4_2d -- NVFP4 with two-dimensional 16 x 16 blocks, for weights ([Q] §4:
  * the 4-bit pre-training recipe scales weights in two-dimensional blocks, so that a weight
  * and its transpose quantise identically).  Same steps as mx_quantize(fmt = NVFP4) with the

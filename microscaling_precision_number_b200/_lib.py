@@ -21,7 +21,7 @@ MX_LAYOUT_ROWMAJOR, MX_LAYOUT_TCGEN05 = 1, 2
 # Every function the header declares (the CPU test checks the library exports them all).
 EXPORTS = ("mx_scale_bytes", "mx_quantize", "mx_quantize_dual", "mx_dequantize", "mx_cast",
            "mx_gemm", "mx_status_string", "mx_last_cuda_error", "mx_watchdog_status",
-           "mx_quantize_nvfp4_noalloc", "mx_mxfp4_to_fp8_blocks", "mx_quantize_nvfp4_2d")
+           "mx_quantize_nvfp4_noalloc", "mx_mxfp4_to_fp8_blocks", "mx_quantize_nvfp4_2d", "mx_quantize_train")
 MX_NOALLOC_MAX_PARTIALS = 1024
 
 
@@ -58,6 +58,8 @@ def _load():
     lib.mx_mxfp4_to_fp8_blocks.argtypes = [P, P, I64, I64, P, P, P, P]
     lib.mx_quantize_nvfp4_2d.argtypes = [P, I64, I64, P, P, I, P, P, P]
     lib.mx_quantize_nvfp4_2d.restype = I
+    lib.mx_quantize_train.argtypes = [P, I64, I64, I, I, I, ctypes.c_uint, P, P, P, I, P, P, P]
+    lib.mx_quantize_train.restype = I
     lib.mx_mxfp4_to_fp8_blocks.restype = I
     lib.mx_gemm.restype = I
     lib.mx_status_string.argtypes = [I]

@@ -98,6 +98,32 @@ def quantize(x: torch.Tensor, fmt="e4m3", axis: str = "row", rounding: str = "ce
     return Quantized(elems, scales, alt, g, orows, ocols, f)
 
 
+def quantize_train(x: torch.Tensor, fmt="e2m1", rounding: str = "floor", rht_signs: Optional[int] = None,
+                   sr_random: Optional[torch.Tensor] = None, layout: str = "tcgen05", stream=None) -> Quantized:
+    """Row-wise quantisation with an optional 16 x 16 random Hadamard transform (rht_signs:
+    the 16-bit sign mask; None for no transform) and optional stochastic rounding
+    (sr_random: a uint8 tensor of x's shape; None for round-to-nearest-even)."""
+    _check_src(x)
+    f = _fmt(fmt)
+    rows, cols = x.shape
+    dev = x.device
+    B = block_of(f)
+    first = "rowmajor" if layout in ("rowmajor", "both") else "tcgen05"
+    elems = torch.empty(elem_bytes(rows, cols, f), dtype=torch.uint8, device=dev)
+    scales = torch.empty(scale_bytes(rows, cols // B, first), dtype=torch.uint8, device=dev)
+    alt = torch.empty(scale_bytes(rows, cols // B, "tcgen05"), dtype=torch.uint8, device=dev) \
+        if layout == "both" else None
+    g = torch.empty(1, dtype=torch.float32, device=dev) if f == L.MX_FMT_NVFP4 else None
+    if sr_random is not None and (sr_random.dtype != torch.uint8 or sr_random.numel() != rows * cols
+                                  or not sr_random.is_contiguous() or sr_random.device != dev):
+        raise ValueError("sr_random must be a contiguous uint8 tensor with one byte per element")
+    L.check(L.lib.mx_quantize_train(x.data_ptr(), rows, cols, f, ROUNDING[rounding], 0 if rht_signs is None else 1,
+                                    0 if rht_signs is None else int(rht_signs) & 0xFFFF, _ptr(sr_random),
+                                    elems.data_ptr(), scales.data_ptr(), LAYOUTS[layout], _ptr(alt), _ptr(g),
+                                    _stream(stream)), "mx_quantize_train")
+    return Quantized(elems, scales, alt, g, rows, cols, f)
+
+
 def quantize_nvfp4_2d(x: torch.Tensor, layout: str = "tcgen05", stream=None) -> Quantized:
     """NVFP4 with 16 x 16 weight blocks (scales repeated on the 16 rows of each block)."""
     _check_src(x)

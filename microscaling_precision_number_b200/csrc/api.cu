@@ -335,6 +335,44 @@ mx_status mx_mxfp4_to_fp8_blocks(const void *elems, const uint8_t *scales, int64
     return e == cudaSuccess ? MX_OK : cuda_fail(e);
 }
 
+mx_status mx_quantize_train(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, mx_scale_rounding rounding,
+                            int rht16, unsigned rht_signs, const uint8_t *sr_random, void *out_elems,
+                            uint8_t *out_scales, mx_scale_layout layout, uint8_t *out_scales_alt, float *global_scale,
+                            mx_stream_t stream) {
+    if (fmt != MX_FMT_E4M3 && fmt != MX_FMT_E5M2 && fmt != MX_FMT_E2M1 && fmt != MX_FMT_NVFP4) return MX_ERR_ARG;
+    if (rounding != MX_SCALE_FLOOR_OCP && rounding != MX_SCALE_CEIL_RECIPE) return MX_ERR_ARG;
+    if (rht16 != 0 && rht16 != 1) return MX_ERR_ARG;
+    if ((fmt == MX_FMT_NVFP4) != (global_scale != nullptr)) return MX_ERR_ARG;
+    if (layout != MX_LAYOUT_ROWMAJOR && layout != MX_LAYOUT_TCGEN05 &&
+        layout != (MX_LAYOUT_ROWMAJOR | MX_LAYOUT_TCGEN05))
+        return MX_ERR_LAYOUT;
+    const bool both = layout == (MX_LAYOUT_ROWMAJOR | MX_LAYOUT_TCGEN05);
+    if (both != (out_scales_alt != nullptr)) return MX_ERR_LAYOUT;
+    if (rows < 0 || cols < 0 || cols % block_of(fmt)) return MX_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MX_OK;
+    if (!mxk::stream_supported(rows, cols)) return MX_ERR_SHAPE;
+    if (!src || !out_elems || !out_scales) return MX_ERR_ARG;
+    if (!aligned(src, 16) || !aligned(out_elems, 16) || !aligned(sr_random, 16) || !aligned(global_scale, 4))
+        return MX_ERR_ALIGN;
+    uint8_t *rm = nullptr, *tc = nullptr;
+    if (both) { rm = out_scales; tc = out_scales_alt; }
+    else if (layout == MX_LAYOUT_ROWMAJOR) rm = out_scales;
+    else tc = out_scales;
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    if (fmt == MX_FMT_NVFP4) {
+        st = nvfp4_scratch(d);
+        if (st != MX_OK) return st;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = mxk::launch_quantize_train(src, rows, cols, fmt, rounding == MX_SCALE_CEIL_RECIPE, rht16 != 0,
+                                               rht_signs & 0xFFFFu, sr_random, d->partials, d->partials_cap,
+                                               global_scale, out_elems, rm, tc, d->num_sms, s);
+    if (e == cudaSuccess && tc) e = mxk::launch_tcgen05_pad(tc, rows, cols / block_of(fmt), s);
+    return e == cudaSuccess ? MX_OK : cuda_fail(e);
+}
+
 mx_status mx_quantize_nvfp4_2d(const void *src, int64_t rows, int64_t cols, void *out_elems, uint8_t *out_scales,
                                mx_scale_layout layout, uint8_t *out_scales_alt, float *global_scale,
                                mx_stream_t stream) {

@@ -62,6 +62,12 @@ cudaError_t launch_gemm_pair(const void *a_elems, const uint8_t *a_sc, int a_fmt
                              const void *b_elems, const uint8_t *b_sc, int b_fmt, const float *gb, void *c,
                              int64_t M, int64_t N, int64_t K, int *watchdog, int num_sms, cudaStream_t st);
 
+// ---- train.cu: row-wise MX / NVFP4 with an optional 16 x 16 random Hadamard transform and
+// optional stochastic rounding (rnd: one random byte per element, or nullptr for RNE) ----------
+cudaError_t launch_quantize_train(const void *src, int64_t rows, int64_t cols, int fmt, bool ceil, bool rht,
+                                  uint32_t signs, const uint8_t *rnd, float *partials, int max_partials, float *g,
+                                  void *elems, uint8_t *rm, uint8_t *tc, int num_sms, cudaStream_t st);
+
 // ---- nested.cu: MXFP4 -> FP8 E4M3 with 128 x 128 block scales ----------------------------------
 cudaError_t launch_mxfp4_to_fp8_blocks(const void *elems, const uint8_t *scales, int64_t rows, int64_t cols,
                                        void *out, float *block_scale, uint8_t *block_exact, cudaStream_t st);

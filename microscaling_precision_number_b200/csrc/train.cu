@@ -1,0 +1,314 @@
+// train.cu -- the training-side variant of the row-wise quantisers: an optional 16 x 16
+// random Hadamard transform of the input and optional stochastic rounding of the element
+// cast, for MXFP8 / MXFP4 (block 32, E8M0) and NVFP4 (block 16, UE4M3 + fp32 tensor scale).
+//
+// Sources (page title, section):
+//   "MXFP4 と NVFP4 は何が違うのか調べてみた"
+//     §4 "精度の差はどこから出るか": the 4-bit pre-training recipe applies a 16 x 16 random
+//        Hadamard transform to the inputs of the weight gradient and rounds gradients
+//        stochastically.
+//     §8 "その後の標準化はどこへ向かっているか": stochastic rounding is among the rounding
+//        modes P3109 defines.
+//
+// Transform: every 16 consecutive elements of a row become H16 D x / 4 (D: sign flips from
+// a 16-bit mask, H16: the Sylvester Hadamard matrix), computed as the radix-2 butterfly
+// (strides 1, 2, 4, 8) in fp32 round-to-nearest, then rounded to bf16; the quantiser then
+// sees those bf16 values.  Stochastic rounding: with the element's random byte r (passed
+// in, one per element), a value strictly between its two representable neighbours lo < |y|
+// < hi rounds to hi when 256 (|y| - lo) > r (hi - lo), else to lo; |y| at or above the
+// maximum saturates; the sign is kept.  Scales are computed exactly as in the RNE path.
+// One thread per quantisation block, blocks of consecutive threads adjacent in memory
+// (coalesced), grid-stride loops; NVFP4 takes a maximum pass and a quantisation pass.
+#include "codec.cuh"
+#include "internal.h"
+#include "ptx.cuh"
+#include "tiling.cuh"
+
+namespace mxk {
+
+namespace {
+constexpr int kTrainThreads = 256;
+}  // namespace
+
+// ---- 16 x 16 random Hadamard transform of 16 bf16 (two uint4, element order) ---------------
+__device__ __forceinline__ void rht16(uint4 &v0, uint4 &v1, uint32_t signs) {
+    float v[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y),
+                   bf16_lo(v0.z), bf16_hi(v0.z), bf16_lo(v0.w), bf16_hi(v0.w),
+                   bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
+                   bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
+#pragma unroll
+    for (int i = 0; i < 16; i++)
+        if ((signs >> i) & 1u) v[i] = -v[i];
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 16; i += 2 * h)
+#pragma unroll
+            for (int j = i; j < i + h; j++) {
+                const float a = v[j], b = v[j + h];
+                v[j] = __fadd_rn(a, b);
+                v[j + h] = __fsub_rn(a, b);
+            }
+#pragma unroll
+    for (int i = 0; i < 16; i++) v[i] = __fmul_rn(v[i], 0.25f);
+    v0 = make_uint4(f32x2_to_bf16x2(v[0], v[1]), f32x2_to_bf16x2(v[2], v[3]), f32x2_to_bf16x2(v[4], v[5]),
+                    f32x2_to_bf16x2(v[6], v[7]));
+    v1 = make_uint4(f32x2_to_bf16x2(v[8], v[9]), f32x2_to_bf16x2(v[10], v[11]), f32x2_to_bf16x2(v[12], v[13]),
+                    f32x2_to_bf16x2(v[14], v[15]));
+}
+
+// ---- stochastic rounding onto the element grid ----------------------------------------------
+// Returns the representable value (lo or hi, signed) that y rounds to with random byte r.
+template <int FMT>
+__device__ __forceinline__ float sr_value(float y, uint32_t r) {
+    constexpr int mbits = FMT == FMT_E4M3 ? 3 : (FMT == FMT_E5M2 ? 2 : 1);
+    constexpr int emin = FMT == FMT_E4M3 ? -6 : (FMT == FMT_E5M2 ? -14 : 0);   // smallest normal exponent
+    constexpr float maxv = FMT == FMT_E4M3 ? 448.0f : (FMT == FMT_E5M2 ? 57344.0f : 6.0f);
+    const float a = fabsf(y);
+    if (!(a < maxv)) return copysignf(maxv, y);
+    const int eb = (int)(__float_as_uint(a) >> 23) - 127;
+    float lo, step;
+    if (eb < emin) {                                              // the format's subnormal grid
+        step = __uint_as_float((uint32_t)(emin - mbits + 127) << 23);
+        lo = __fmul_rn(floorf(__fmul_rn(a, __uint_as_float((uint32_t)(mbits - emin + 127) << 23))), step);
+    } else {                                                      // truncate to mbits mantissa bits
+        lo = __uint_as_float(__float_as_uint(a) & ~((1u << (23 - mbits)) - 1u));
+        step = __uint_as_float((uint32_t)(eb - mbits + 127) << 23);
+    }
+    if (a == lo) return y;
+    const bool up = __fmul_rn(__fsub_rn(a, lo), 256.0f) > __fmul_rn((float)r, step);
+    return copysignf(up ? __fadd_rn(lo, step) : lo, y);
+}
+
+template <int FMT, bool SR>
+__device__ __forceinline__ void round8(float (&x)[8], const uint8_t *rnd) {
+    if constexpr (SR) {
+        const uint2 rb = *reinterpret_cast<const uint2 *>(rnd);
+        const uint32_t w[2] = {rb.x, rb.y};
+#pragma unroll
+        for (int i = 0; i < 8; i++) x[i] = sr_value<FMT>(x[i], (w[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+    }
+}
+
+// ---- row-wise MX with transform / stochastic rounding --------------------------------------
+template <int FMT, bool CEIL, bool RM, bool TC, bool RHT, bool SR>
+__global__ void __launch_bounds__(kTrainThreads)
+mx_train_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
+                uint32_t signs, const uint8_t *__restrict__ rnd, uint8_t *__restrict__ elems,
+                uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (uint32_t blk = blockIdx.x * kTrainThreads + threadIdx.x; blk < n_blocks; blk += gridDim.x * kTrainThreads) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)blk * 64);
+        uint4 v[4] = {p[0], p[1], p[2], p[3]};
+        if constexpr (RHT) {
+            rht16(v[0], v[1], signs);
+            rht16(v[2], v[3], signs);
+        }
+        uint32_t a = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v[0].x, v[0].y), absmax_bf16x2(v[0].z, v[0].w)),
+                                   absmax_bf16x2(absmax_bf16x2(v[1].x, v[1].y), absmax_bf16x2(v[1].z, v[1].w)));
+        a = absmax_bf16x2(a, absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v[2].x, v[2].y), absmax_bf16x2(v[2].z, v[2].w)),
+                                           absmax_bf16x2(absmax_bf16x2(v[3].x, v[3].y), absmax_bf16x2(v[3].z, v[3].w))));
+        const uint32_t code = e8m0_from_amax_bits<FMT, CEIL>(max(a & 0x7FFFu, (a >> 16) & 0x7FFFu));
+        const uint64_t mul2x = splat2(e8m0_inverse_multiplier(code));
+        const bool nan_blk = code == 0xFFu;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            float x[8];
+            scale8(v[j], mul2x, x);
+            round8<FMT, SR>(x, rnd + (size_t)blk * 32 + 8 * j);
+            if constexpr (FMT == FMT_E2M1) {
+                reinterpret_cast<uint32_t *>(elems)[(size_t)blk * 4 + j] = nan_blk ? 0u : cvt_e2m1x8(x);
+            } else {
+                const uint2 q = cvt_fp8x8<FMT>(x);
+                reinterpret_cast<uint2 *>(elems)[(size_t)blk * 4 + j] = nan_blk ? make_uint2(0u, 0u) : q;
+            }
+        }
+        if constexpr (RM) sc_rm[blk] = (uint8_t)code;
+        if constexpr (TC) {
+            const uint32_t r = fdiv(blk, divS);
+            sc_tc[tc_offset(r, blk - r * divS.d, col_atoms)] = (uint8_t)code;
+        }
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- NVFP4 with transform / stochastic rounding ---------------------------------------------
+// Pass 1: per-CTA finite maximum of the (transformed) tensor.
+template <bool RHT>
+__global__ void __launch_bounds__(kTrainThreads)
+nvfp4_train_amax_kernel(const uint8_t *__restrict__ src, uint32_t n_groups, uint32_t signs,
+                        float *__restrict__ partials) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ uint32_t warp_u[kTrainThreads / 32];
+    uint32_t acc = 0;
+    for (uint32_t gi = blockIdx.x * kTrainThreads + threadIdx.x; gi < n_groups; gi += gridDim.x * kTrainThreads) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)gi * 32);
+        uint4 v0 = p[0], v1 = p[1];
+        if constexpr (RHT) rht16(v0, v1, signs);
+        acc = __vmaxu2(acc, finite_abs_max_bf16x8(v0));
+        acc = __vmaxu2(acc, finite_abs_max_bf16x8(v1));
+    }
+    uint32_t m = max(acc & 0xFFFFu, acc >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0) warp_u[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t r = 0;
+        for (int w = 0; w < kTrainThreads / 32; w++) r = max(r, warp_u[w]);
+        partials[blockIdx.x] = __uint_as_float(r << 16);
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Pass 2: g from the partial maxima, then one thread per 16-element block.  The block
+// scale and the quotient follow the RNE path's fp32 steps (t = amax_b / (6 g) by IEEE
+// division, r = 1 / (dec(sb) g)); the element cast is RNE or stochastic.
+template <bool RM, bool TC, bool RHT, bool SR>
+__global__ void __launch_bounds__(kTrainThreads)
+nvfp4_train_quant_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
+                         uint32_t signs, const uint8_t *__restrict__ rnd, const float *__restrict__ partials,
+                         int n_partials, float *__restrict__ g_out, uint8_t *__restrict__ elems,
+                         uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float red[kTrainThreads / 32];
+    float a = 0.0f;
+    for (int i = threadIdx.x; i < n_partials; i += kTrainThreads) a = fmaxf(a, partials[i]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = a;
+    __syncthreads();
+    a = 0.0f;
+    for (int w = 0; w < kTrainThreads / 32; w++) a = fmaxf(a, red[w]);
+    const float g = a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    const float six_g = __fmul_rn(6.0f, g);
+    for (uint32_t blk = blockIdx.x * kTrainThreads + threadIdx.x; blk < n_blocks; blk += gridDim.x * kTrainThreads) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)blk * 32);
+        uint4 v[2] = {p[0], p[1]};
+        if constexpr (RHT) rht16(v[0], v[1], signs);
+        const uint32_t am = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v[0].x, v[0].y), absmax_bf16x2(v[0].z, v[0].w)),
+                                          absmax_bf16x2(absmax_bf16x2(v[1].x, v[1].y), absmax_bf16x2(v[1].z, v[1].w)));
+        const uint32_t m = max(am & 0x7FFFu, (am >> 16) & 0x7FFFu);
+        const bool special = m >= 0x7F80u;
+        const float tq = __fdiv_rn(__uint_as_float(m << 16), six_g);
+        uint32_t sb = cvt_fp8x2<FMT_E4M3>(tq, 0.0f) & 0xFFu;
+        const float d = __fmul_rn(ue4m3_to_f32(sb & 0x7Fu), g);
+        const float r = d != 0.0f ? __frcp_rn(d) : 0.0f;
+        const bool zero_codes = special || d == 0.0f;
+        if (special) sb = 0x7Fu;
+        const uint64_t r2 = splat2(r);
+        uint32_t q[2];
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+            float x[8];
+            scale8(v[j], r2, x);
+            if (__builtin_expect(isinf(r), 0)) {
+                const float in[8] = {bf16_lo(v[j].x), bf16_hi(v[j].x), bf16_lo(v[j].y), bf16_hi(v[j].y),
+                                     bf16_lo(v[j].z), bf16_hi(v[j].z), bf16_lo(v[j].w), bf16_hi(v[j].w)};
+#pragma unroll
+                for (int i = 0; i < 8; i++)
+                    if (x[i] != x[i]) x[i] = in[i];                    // 0 * Inf: keep the signed zero
+            }
+            round8<FMT_E2M1, SR>(x, rnd + (size_t)blk * 16 + 8 * j);
+            q[j] = zero_codes ? 0u : cvt_e2m1x8(x);
+        }
+        reinterpret_cast<uint2 *>(elems)[blk] = make_uint2(q[0], q[1]);
+        if constexpr (RM) sc_rm[blk] = (uint8_t)sb;
+        if constexpr (TC) {
+            const uint32_t rr = fdiv(blk, divS);
+            sc_tc[tc_offset(rr, blk - rr * divS.d, col_atoms)] = (uint8_t)sb;
+        }
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---- launchers ---------------------------------------------------------------------------
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kTrainThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+static int train_grid(uint64_t items, int num_sms) {
+    uint64_t g = (items + kTrainThreads - 1) / kTrainThreads;
+    const uint64_t cap = (uint64_t)num_sms * 8;
+    if (g > cap) g = cap;
+    return g < 1 ? 1 : (int)g;
+}
+
+template <int FMT, bool CEIL, bool RHT, bool SR>
+static cudaError_t launch_mx_train_t(const uint8_t *src, uint32_t nb, FastDiv f, uint32_t ca, uint32_t signs,
+                                     const uint8_t *rnd, uint8_t *e, uint8_t *rm, uint8_t *tc, int num_sms,
+                                     cudaStream_t st) {
+    const int grid = train_grid(nb, num_sms);
+    if (rm && tc) return launch_pdl(mx_train_kernel<FMT, CEIL, true, true, RHT, SR>, grid, st, src, nb, f, ca, signs, rnd, e, rm, tc);
+    if (rm) return launch_pdl(mx_train_kernel<FMT, CEIL, true, false, RHT, SR>, grid, st, src, nb, f, ca, signs, rnd, e, rm, tc);
+    return launch_pdl(mx_train_kernel<FMT, CEIL, false, true, RHT, SR>, grid, st, src, nb, f, ca, signs, rnd, e, rm, tc);
+}
+
+template <int FMT, bool CEIL>
+static cudaError_t launch_mx_train_f(bool rht, bool sr, const uint8_t *src, uint32_t nb, FastDiv f, uint32_t ca,
+                                     uint32_t signs, const uint8_t *rnd, uint8_t *e, uint8_t *rm, uint8_t *tc,
+                                     int num_sms, cudaStream_t st) {
+    if (rht && sr) return launch_mx_train_t<FMT, CEIL, true, true>(src, nb, f, ca, signs, rnd, e, rm, tc, num_sms, st);
+    if (rht) return launch_mx_train_t<FMT, CEIL, true, false>(src, nb, f, ca, signs, rnd, e, rm, tc, num_sms, st);
+    if (sr) return launch_mx_train_t<FMT, CEIL, false, true>(src, nb, f, ca, signs, rnd, e, rm, tc, num_sms, st);
+    return launch_mx_train_t<FMT, CEIL, false, false>(src, nb, f, ca, signs, rnd, e, rm, tc, num_sms, st);
+}
+
+template <bool RHT, bool SR>
+static cudaError_t launch_nvfp4_train_t(const uint8_t *src, uint32_t nb, FastDiv f, uint32_t ca, uint32_t signs,
+                                        const uint8_t *rnd, float *partials, int max_partials, float *g, uint8_t *e,
+                                        uint8_t *rm, uint8_t *tc, int num_sms, cudaStream_t st) {
+    int grid1 = train_grid(nb, num_sms);
+    if (grid1 > max_partials) grid1 = max_partials;
+    cudaError_t err = launch_pdl(nvfp4_train_amax_kernel<RHT>, grid1, st, src, nb, signs, partials);
+    if (err != cudaSuccess) return err;
+    const int grid2 = train_grid(nb, num_sms);
+    const float *cp = partials;
+    if (rm && tc)
+        return launch_pdl(nvfp4_train_quant_kernel<true, true, RHT, SR>, grid2, st, src, nb, f, ca, signs, rnd, cp, grid1, g, e, rm, tc);
+    if (rm)
+        return launch_pdl(nvfp4_train_quant_kernel<true, false, RHT, SR>, grid2, st, src, nb, f, ca, signs, rnd, cp, grid1, g, e, rm, tc);
+    return launch_pdl(nvfp4_train_quant_kernel<false, true, RHT, SR>, grid2, st, src, nb, f, ca, signs, rnd, cp, grid1, g, e, rm, tc);
+}
+
+cudaError_t launch_quantize_train(const void *src, int64_t rows, int64_t cols, int fmt, bool ceil, bool rht,
+                                  uint32_t signs, const uint8_t *rnd, float *partials, int max_partials, float *g,
+                                  void *elems, uint8_t *rm, uint8_t *tc, int num_sms, cudaStream_t st) {
+    const uint8_t *s8 = static_cast<const uint8_t *>(src);
+    uint8_t *e8 = static_cast<uint8_t *>(elems);
+    const bool sr = rnd != nullptr;
+    if (fmt == FMT_NVFP4) {
+        const uint32_t nb = (uint32_t)(rows * cols / 16), S = (uint32_t)(cols / 16);
+        const FastDiv f = make_fastdiv(S);
+        const uint32_t ca = (S + 3) / 4;
+        if (rht && sr) return launch_nvfp4_train_t<true, true>(s8, nb, f, ca, signs, rnd, partials, max_partials, g, e8, rm, tc, num_sms, st);
+        if (rht) return launch_nvfp4_train_t<true, false>(s8, nb, f, ca, signs, rnd, partials, max_partials, g, e8, rm, tc, num_sms, st);
+        if (sr) return launch_nvfp4_train_t<false, true>(s8, nb, f, ca, signs, rnd, partials, max_partials, g, e8, rm, tc, num_sms, st);
+        return launch_nvfp4_train_t<false, false>(s8, nb, f, ca, signs, rnd, partials, max_partials, g, e8, rm, tc, num_sms, st);
+    }
+    const uint32_t nb = (uint32_t)(rows * cols / 32), S = (uint32_t)(cols / 32);
+    const FastDiv f = make_fastdiv(S);
+    const uint32_t ca = (S + 3) / 4;
+    switch (fmt * 2 + (ceil ? 1 : 0)) {
+    case FMT_E4M3 * 2 + 0: return launch_mx_train_f<FMT_E4M3, false>(rht, sr, s8, nb, f, ca, signs, rnd, e8, rm, tc, num_sms, st);
+    case FMT_E4M3 * 2 + 1: return launch_mx_train_f<FMT_E4M3, true>(rht, sr, s8, nb, f, ca, signs, rnd, e8, rm, tc, num_sms, st);
+    case FMT_E5M2 * 2 + 0: return launch_mx_train_f<FMT_E5M2, false>(rht, sr, s8, nb, f, ca, signs, rnd, e8, rm, tc, num_sms, st);
+    case FMT_E5M2 * 2 + 1: return launch_mx_train_f<FMT_E5M2, true>(rht, sr, s8, nb, f, ca, signs, rnd, e8, rm, tc, num_sms, st);
+    case FMT_E2M1 * 2 + 0: return launch_mx_train_f<FMT_E2M1, false>(rht, sr, s8, nb, f, ca, signs, rnd, e8, rm, tc, num_sms, st);
+    case FMT_E2M1 * 2 + 1: return launch_mx_train_f<FMT_E2M1, true>(rht, sr, s8, nb, f, ca, signs, rnd, e8, rm, tc, num_sms, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace mxk

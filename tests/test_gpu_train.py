@@ -1,0 +1,73 @@
+"""GPU parity of the training-side quantiser (16 x 16 random Hadamard transform and
+stochastic rounding, row-wise MX and NVFP4) against the oracle's composition of its
+pinned transform and its pinned rounding, bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import microscaling_precision_number_b200 as mx
+
+FMT = {"e4m3": 0, "e5m2": 1, "e2m1": 2, "nvfp4": 3}
+
+
+@pytest.fixture(autouse=True)
+def _no_watchdog():
+    yield
+    assert mx.watchdog_status(clear=True) == 0
+
+
+def to_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def with_specials(x, seed):
+    x = x.copy()
+    rng = np.random.default_rng(seed)
+    sp = synth.special_values_block()
+    idx = rng.choice(x.size, size=min(x.size // 9, 40), replace=False)
+    x.reshape(-1)[idx] = sp[rng.integers(0, sp.size, size=idx.size)]
+    return x
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2", "e2m1", "nvfp4"])
+@pytest.mark.parametrize("rht,sr", [(True, False), (False, True), (True, True), (False, False)])
+@pytest.mark.parametrize("shape", [(64, 256), (130, 512)])
+def test_train_quantiser_matches_oracle(oracle, fmt, rht, sr, shape):
+    x = with_specials(synth.gradients(*shape, seed=shape[0] + 3), seed=shape[1])
+    rounding = "floor" if fmt == "e2m1" else "ceil"
+    rnd = np.random.default_rng(shape[0]).integers(0, 256, size=shape, dtype=np.uint8) if sr else None
+    signs = 0xA53C if rht else None
+    q = mx.quantize_train(to_dev(x), fmt, rounding, rht_signs=signs,
+                          sr_random=None if rnd is None else torch.from_numpy(rnd).cuda(), layout="both")
+    xt = oracle.rht16(x, signs) if rht else x
+    f = FMT[fmt]
+    rnd_o = oracle.CEIL if rounding == "ceil" else oracle.FLOOR
+    if fmt == "nvfp4":
+        e, s, g = oracle.quantize_nvfp4_sr(xt, rnd) if sr else oracle.quantize_nvfp4(xt)
+        assert q.global_scale.cpu().numpy()[0] == np.float32(g)
+    else:
+        e, s = oracle.quantize_mx_sr(xt, f, rnd_o, rnd) if sr else oracle.quantize_mx(xt, f, oracle.ROW, rnd_o)
+    assert np.array_equal(q.elems.cpu().numpy(), e.reshape(-1))
+    assert np.array_equal(q.scales.cpu().numpy(), s.reshape(-1))
+    assert np.array_equal(q.scales_alt.cpu().numpy(), oracle.to_tcgen05_layout(s))
+
+
+def test_rht_keeps_the_matmul(oracle):
+    """The same transform on both operands along K leaves A * B^T unchanged up to the
+    quantisation (the property that makes it usable on weight-gradient inputs)."""
+    M, N, K = 256, 256, 512
+    a = synth.normal(M, K, seed=1)
+    b = synth.normal(N, K, seed=2)
+    ref = mx.gemm(mx.quantize(to_dev(a), "e4m3", "row", "ceil", layout="tcgen05"),
+                  mx.quantize(to_dev(b), "e4m3", "row", "ceil", layout="tcgen05")).float()
+    got = mx.gemm(mx.quantize_train(to_dev(a), "e4m3", "ceil", rht_signs=0x5A0F),
+                  mx.quantize_train(to_dev(b), "e4m3", "ceil", rht_signs=0x5A0F)).float()
+    exact = to_dev(a).float() @ to_dev(b).float().T
+    rel_ref = ((ref - exact).norm() / exact.norm()).item()
+    rel_got = ((got - exact).norm() / exact.norm()).item()
+    assert rel_got < 3 * rel_ref + 1e-3, (rel_got, rel_ref)
