@@ -378,9 +378,12 @@ def run_breakdown(mx, dev, pk):
         torch.cuda.empty_cache()
 
     # C4 / C5: block-scaled matmuls (operands quantised outside the timing)
-    for name, (M, N, K), bfmt, bsig in (("c4_gemm_e4m3_8192", (8192, 8192, 8192), "e4m3", 1.0),
-                                       ("c5_gemm_e4m3_x_e2m1_8192x14336x4096", (8192, 14336, 4096), "e2m1", 0.02)):
-        a = mx.quantize(to_dev(synth.normal(M, K, seed=40), dev), "e4m3", "row", "ceil", layout="tcgen05")
+    # (plus the next-row MXFP6 x MXFP6 matmul, which runs on the same kind at the same rate)
+    for name, (M, N, K), afmt, bfmt, bsig in (
+            ("c4_gemm_e4m3_8192", (8192, 8192, 8192), "e4m3", "e4m3", 1.0),
+            ("c5_gemm_e4m3_x_e2m1_8192x14336x4096", (8192, 14336, 4096), "e4m3", "e2m1", 0.02),
+            ("next_gemm_mxfp6_e2m3_8192", (8192, 8192, 8192), "e2m3", "e2m3", 1.0)):
+        a = mx.quantize(to_dev(synth.normal(M, K, seed=40), dev), afmt, "row", "ceil", layout="tcgen05")
         b = mx.quantize(to_dev(synth.normal(N, K, sigma=bsig, seed=41), dev), bfmt, "row",
                         "floor" if bfmt == "e2m1" else "ceil", layout="tcgen05")
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
@@ -409,13 +412,13 @@ def run_breakdown(mx, dev, pk):
         torch.cuda.empty_cache()
 
     # next row: MXFP6 / MXINT8 row-wise quantisation of the config-3 activations
-    # (16384 x 4096 bf16, one byte per code), against the HBM roofline
+    # (16384 x 4096 bf16; FP6 codes packed 6 bits each, INT8 one byte), against the HBM roofline
     x3 = to_dev(synth.activations(), dev)
     R, C = x3.shape
     for name, fmt in (("next_quant_mxfp6_e2m3_16384x4096", "e2m3"), ("next_quant_mxint8_16384x4096", "int8")):
         q = mx.quantize(x3, fmt, "row", "ceil", layout="tcgen05")
         t = timed([lambda q=q: mx.quantize(x3, fmt, "row", "ceil", layout="tcgen05", out=q)], 20, stream)
-        nb = R * C * 2 + R * C + R * C // 32
+        nb = R * C * 2 + mx.elem_bytes(R, C, fmt) + R * C // 32
         out[name] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1), "frac_hbm": round(nb / t / 1e6 / hbm, 4),
                      "algorithmic_bytes": nb}
         del q

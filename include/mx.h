@@ -31,8 +31,10 @@
  *     error code is kept per host thread, see mx_last_cuda_error).  Empty inputs
  *     (rows == 0 or cols == 0) are valid and launch nothing.
  *   - bf16 is IEEE binary16-brain (1/8/7), stored as 2-byte little-endian words.
- *   - Element codes: one byte per FP8 code; FP4 codes pack two per byte with the even
- *     element index in the low nibble.
+ *   - Element codes are packed densely along each row: code i occupies bits
+ *     [w*i, w*i + w) of the row read as a little-endian bit string, w the code width.
+ *     FP8 / INT8: one byte per code; FP6: four codes per three bytes (16 per 12 bytes);
+ *     FP4: two per byte, the even element index in the low nibble.
  *   - Overflow saturates to the format maximum (448 E4M3, 57344 E5M2, 6 E2M1); a
  *     block holding a NaN or Inf gets the NaN scale (0xFF E8M0, 0x7F UE4M3) and
  *     element codes 0.
@@ -70,9 +72,8 @@ typedef enum {
     MX_FMT_E3M2 = 5,     /* MXFP6, E3M2 elements (max 28), block 32, E8M0 scale */
     MX_FMT_INT8 = 6      /* MXINT8, int8 q read as q / 64 (-127 .. 127), block 32, E8M0 scale */
 } mx_fmt;
-/* Storage: FP8 and INT8 codes take one byte; FP6 codes take one byte each (the 6-bit code
- * in the low bits, the top two bits zero); FP4 codes pack two per byte, the even element
- * in the low nibble. */
+/* Storage (w bits per code, packed densely along a row): FP8 and INT8 w = 8; FP6 w = 6,
+ * so MXFP6 costs 6 + 8/32 = 6.25 bits per element; FP4 w = 4, even element low. */
 
 typedef enum {
     MX_AXIS_ROW = 0,     /* blocks run along a row (contiguous elements) */
@@ -109,8 +110,8 @@ int64_t mx_scale_bytes(int64_t rows, int64_t scale_cols, mx_scale_layout layout)
  *               (K-major for a weight-gradient matmul), scales cols x rows/B.
  *               NVFP4 supports ROW only.
  *   rounding    shared-exponent rule (ignored for NVFP4).
- *   out_elems   device, 16-byte aligned; out_rows x out_cols bytes (FP8, FP6, INT8) or
- *               x out_cols/2 (FP4).
+ *   out_elems   device, 16-byte aligned; out_rows x (out_cols * w / 8) bytes: w = 8
+ *               (FP8, INT8), 6 (FP6), 4 (FP4).
  *   out_scales  device; first scale layout (the lower set bit of `layout`).
  *   layout      ROWMAJOR, TCGEN05 or both; with both, out_scales gets ROWMAJOR and
  *               out_scales_alt gets TCGEN05 (else out_scales_alt must be NULL).
@@ -231,13 +232,14 @@ mx_status mx_dequantize(const void *elems, const uint8_t *scales, const float *g
  * with no block scale (RNE, saturating).  NaN becomes 0x7F|sign (E4M3, E5M2) or the
  * signed maximum 0x7|sign (E2M1) / 0x1F|sign (E2M3, E3M2), formats without NaN.  INT8
  * needs a scale and is not a cast target (MX_ERR_ARG).
- *   n           element count (even for E2M1); src and out 16-byte aligned.
+ *   n           element count (even for E2M1, a multiple of 4 for FP6: whole bytes of
+ *               packed codes); src and out 16-byte aligned.
  */
 mx_status mx_cast(const void *src_bf16, int64_t n, mx_fmt fmt, void *out_elems, mx_stream_t stream);
 
 /*
  * One operand of the block-scaled matmul: a rows x K matrix of codes, K-major (each row
- * holds K consecutive codes; FP4 packed two per byte), with its block scales in the TCGEN05
+ * holds K consecutive codes, packed as the quantisers write them), with its block scales in the TCGEN05
  * layout exactly as mx_quantize(axis = ROW, layout = TCGEN05) writes them: E8M0 per 32
  * along K (rows x K/32) for the MX formats, UE4M3 per 16 along K (rows x K/16) for NVFP4.
  *   global_scale  NVFP4 only: device pointer to the operand's fp32 per-tensor scale g (as

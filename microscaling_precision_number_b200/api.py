@@ -29,8 +29,15 @@ def is_fp4(fmt) -> bool:
     return _fmt(fmt) in (L.MX_FMT_E2M1, L.MX_FMT_NVFP4)
 
 
+def code_bits(fmt) -> int:
+    """Stored width of one element code: codes are packed densely along a row (FP4 two per
+    byte, FP6 four per three bytes, FP8 / INT8 one per byte)."""
+    f = _fmt(fmt)
+    return 4 if is_fp4(f) else 6 if f in (L.MX_FMT_E2M3, L.MX_FMT_E3M2) else 8
+
+
 def elem_bytes(rows: int, cols: int, fmt) -> int:
-    return rows * cols // 2 if is_fp4(fmt) else rows * cols
+    return rows * cols * code_bits(fmt) // 8
 
 
 def scale_bytes(rows: int, scale_cols: int, layout) -> int:

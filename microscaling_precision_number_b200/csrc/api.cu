@@ -273,7 +273,8 @@ mx_status mx_dequantize(const void *elems, const uint8_t *scales, const float *g
 
 mx_status mx_cast(const void *src, int64_t n, mx_fmt fmt, void *out, mx_stream_t stream) {
     if (!mx_block_fmt(fmt) || fmt == MX_FMT_INT8) return MX_ERR_ARG;
-    if (n < 0 || (fmt == MX_FMT_E2M1 && n % 2)) return MX_ERR_SHAPE;
+    if (n < 0 || (fmt == MX_FMT_E2M1 && n % 2) || ((fmt == MX_FMT_E2M3 || fmt == MX_FMT_E3M2) && n % 4))
+        return MX_ERR_SHAPE;                                  // whole bytes of packed codes
     if (n == 0) return MX_OK;
     if (!src || !out) return MX_ERR_ARG;
     if (!aligned(src, 16) || !aligned(out, 16)) return MX_ERR_ALIGN;

@@ -29,8 +29,47 @@ __host__ __device__ constexpr int emax_elem(int fmt) {
 __host__ __device__ constexpr int max_sig128(int fmt) {
     return fmt == FMT_E2M1 ? 192 : fmt == FMT_E2M3 ? 240 : fmt == FMT_INT8 ? 254 : 224;
 }
-// Element formats stored one code per byte (FP8, FP6 in the low 6 bits, INT8).
-__host__ __device__ constexpr bool byte_codes(int fmt) { return fmt != FMT_E2M1 && fmt != FMT_NVFP4; }
+// Stored width of one element code.  Codes are packed densely along a row: code i at bits
+// [w*i, w*i + w) of the row read as a little-endian bit string -- FP4 two per byte (even
+// index low), FP6 four per three bytes (16 per 12 bytes, the packed form that the TMA
+// 16U6_ALIGN16B type expands for the tensor cores), FP8 / INT8 one per byte.
+__host__ __device__ constexpr int code_bits(int fmt) {
+    return (fmt == FMT_E2M1 || fmt == FMT_NVFP4) ? 4 : (fmt == FMT_E2M3 || fmt == FMT_E3M2) ? 6 : 8;
+}
+__host__ __device__ constexpr bool is_fp6(int fmt) { return fmt == FMT_E2M3 || fmt == FMT_E3M2; }
+
+// Four FP6 codes held one per byte (low 6 bits) -> their 24 packed bits, and back.
+__device__ __forceinline__ uint32_t fp6_pack4(uint32_t w) {
+    return (w & 0x3Fu) | ((w >> 2) & 0xFC0u) | ((w >> 4) & 0x3F000u) | ((w >> 6) & 0xFC0000u);
+}
+__device__ __forceinline__ uint32_t fp6_unpack4(uint32_t p) {
+    return (p & 0x3Fu) | ((p << 2) & 0x3F00u) | ((p << 4) & 0x3F0000u) | ((p << 6) & 0x3F000000u);
+}
+// 4k codes held one per byte (k words) -> 3k packed words (k a multiple of 4: 16 codes ->
+// 12 bytes), and back.
+template <int W>
+__device__ __forceinline__ void fp6_pack(const uint32_t (&w)[W], uint32_t (&o)[W * 3 / 4]) {
+    static_assert(W % 4 == 0, "whole 16-code groups");
+#pragma unroll
+    for (int g = 0; g < W / 4; g++) {
+        const uint32_t p0 = fp6_pack4(w[4 * g]), p1 = fp6_pack4(w[4 * g + 1]);
+        const uint32_t p2 = fp6_pack4(w[4 * g + 2]), p3 = fp6_pack4(w[4 * g + 3]);
+        o[3 * g] = p0 | (p1 << 24);
+        o[3 * g + 1] = (p1 >> 8) | (p2 << 16);
+        o[3 * g + 2] = (p2 >> 16) | (p3 << 8);
+    }
+}
+template <int W>
+__device__ __forceinline__ void fp6_unpack(const uint32_t (&o)[W * 3 / 4], uint32_t (&w)[W]) {
+#pragma unroll
+    for (int g = 0; g < W / 4; g++) {
+        const uint32_t a = o[3 * g], b = o[3 * g + 1], c = o[3 * g + 2];
+        w[4 * g] = fp6_unpack4(a & 0xFFFFFFu);
+        w[4 * g + 1] = fp6_unpack4((a >> 24) | ((b & 0xFFFFu) << 8));
+        w[4 * g + 2] = fp6_unpack4((b >> 16) | ((c & 0xFFu) << 16));
+        w[4 * g + 3] = fp6_unpack4(c >> 8);
+    }
+}
 
 // E8M0 code from the block maximum given as |x| bf16 bits (0 .. 0x7FFF).  Any
 // magnitude >= 0x7F80 (Inf or NaN) yields the NaN scale 0xFF.  A zero block yields

@@ -63,6 +63,22 @@ __device__ __forceinline__ void store32(uint8_t *p, const uint32_t (&w)[8], bool
     }
 }
 
+// The 32 codes (one per byte in w) of the block that starts at element e of an output:
+// FP8 / INT8 as 32 bytes (store32), FP6 packed into 24 bytes (three 8-byte stores; e is a
+// multiple of 32, so the address is 8-byte aligned).
+template <int FMT>
+__device__ __forceinline__ void store_codes(uint8_t *base, uint64_t e, const uint32_t (&w)[8], bool v8, bool zero) {
+    if constexpr (is_fp6(FMT)) {
+        uint32_t o[6];
+        fp6_pack<8>(w, o);
+        uint2 *p = reinterpret_cast<uint2 *>(base + e * 3 / 4);
+#pragma unroll
+        for (int i = 0; i < 3; i++) p[i] = zero ? make_uint2(0u, 0u) : make_uint2(o[2 * i], o[2 * i + 1]);
+    } else {
+        store32(base + e, w, v8, zero);
+    }
+}
+
 // Tile order: bands of kBand column tiles, row-tile major inside a band, so that the tiles
 // in flight at any moment span many rows of few columns.  The transposed output of a
 // column then grows by long contiguous runs (and the row-wise output by kBand x 256-byte
@@ -145,8 +161,8 @@ __device__ __forceinline__ void column_pair(const uint8_t *box, uint32_t q, uint
             if (i & 1) { o_lo[i >> 1] |= cl << 16; o_hi[i >> 1] |= ch << 16; }
             else       { o_lo[i >> 1] = cl;        o_hi[i >> 1] = ch; }
         }
-        store32(col_elems + e0, o_lo, v8, code_lo == 0xFFu);         // NaN scale: codes 0
-        store32(col_elems + e0 + rows, o_hi, v8, code_hi == 0xFFu);
+        store_codes<FMT>(col_elems, e0, o_lo, v8, code_lo == 0xFFu);        // NaN scale: codes 0
+        store_codes<FMT>(col_elems, e0 + rows, o_hi, v8, code_hi == 0xFFu);
     }
     if constexpr (TC) {
         col_sc[tc_offset(col, tr, sc_dim)] = (uint8_t)code_lo;
@@ -199,7 +215,7 @@ __device__ __forceinline__ void row_block(const uint8_t *box, uint32_t r, uint32
             o[2 * k] = q.x;
             o[2 * k + 1] = q.y;
         }
-        store32(row_elems + e0, o, v8, code == 0xFFu);                  // NaN scale: codes 0
+        store_codes<FMT>(row_elems, e0, o, v8, code == 0xFFu);             // NaN scale: codes 0
     }
     if constexpr (TC) row_sc[tc_offset(R, col >> 5, sc_dim)] = (uint8_t)code;
     else row_sc[(uint64_t)R * sc_dim + (col >> 5)] = (uint8_t)code;

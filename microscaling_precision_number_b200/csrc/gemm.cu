@@ -122,8 +122,9 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (lane == 0) {
             // scale atoms per 128-row block of an operand (the tcgen05 layout's column-atom count)
             const int64_t col_atoms = (int64_t)num_kb * T::kAtoms;
-            const bool b_expanded = KIND == KIND_F8F6F4 && b_fmt_code == 5u;
-            const uint32_t tx = kABytes + (b_expanded ? kBBytes / 2 : kBBytes) + kSfaBytes + kSfbBytes;
+            const uint32_t tx = (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kABytes, a_fmt_code) : kABytes) +
+                                (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kBBytes, b_fmt_code) : kBBytes) +
+                                kSfaBytes + kSfbBytes;
             int it = 0;
             for (int t = blockIdx.x; t < n_tiles && !*fail_sh; t += gridDim.x) {
                 int m_blk, n_blk;
@@ -135,9 +136,9 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         *fail_sh = 1;
                         break;
                     }
-                    // An E2M1 tile of the mxf8f6f4 kind lands in shared memory padded to one
-                    // byte per element (16U4_ALIGN16B), but the copy completes only the
-                    // packed global bytes.  Either way a stage holds 128 bytes of K per row.
+                    // E2M1 and FP6 tiles of the mxf8f6f4 kind land in shared memory padded to
+                    // one 16-byte group per 16 codes, but the copy completes only the packed
+                    // global bytes.  Either way a stage holds 128 bytes of K per row.
                     mbar_arrive_expect_tx(&full_bar[s], tx);
                     tma_load_2d(sA + s * kABytes, &tmA, kb * kBK, m_blk * kBM, &full_bar[s]);
                     tma_load_2d(sB + s * kBBytes, &tmB, kb * kBK, n_blk * BN, &full_bar[s]);
@@ -264,16 +265,21 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                   CUtensorMapFloatOOBfill);
 
-// 2-D tensor map over a rows x K operand: 8-bit codes (one byte per element), E2M1 codes
-// expanded to bytes by the copy (16U4_ALIGN16B, mxf8f6f4 kind) or packed E2M1 codes read as
-// bytes (4-bit kinds).  Either way the box is 128 bytes of shared memory per row.
+// 2-D tensor map over a rows x K operand: 8-bit codes (one byte per element); E2M1 or FP6
+// codes expanded by the copy to a 16-byte group per 16 codes (16U4_ALIGN16B /
+// 16U6_ALIGN16B, mxf8f6f4 kind); or packed E2M1 codes read as bytes (4-bit kinds).  Either
+// way the box is 128 bytes of shared memory per row.
 static bool encode_operand(EncodeTiledFn enc, CUtensorMap *tm, const void *ptr, int64_t rows, int64_t K,
-                           bool fp4, bool expand, uint32_t box_rows) {
-    const cuuint64_t gdim[2] = {(cuuint64_t)(fp4 && !expand ? K / 2 : K), (cuuint64_t)rows};
-    const cuuint64_t gstride[1] = {(cuuint64_t)(fp4 ? K / 2 : K)};
+                           int fmt, bool expand, uint32_t box_rows) {
+    const int bits = code_bits(fmt);
+    const cuuint64_t gdim[2] = {(cuuint64_t)(expand || bits == 8 ? K : K * bits / 8), (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)(K * bits / 8)};
     const cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(tm, expand ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+    const CUtensorMapDataType dt = !expand ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : bits == 6 ? CU_TENSOR_MAP_DATA_TYPE_16U6_ALIGN16B
+                                               : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
+    const CUresult r = enc(tm, dt, 2,
                            const_cast<void *>(ptr), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -305,16 +311,17 @@ cudaError_t launch_gemm(const void *a_elems, const uint8_t *a_sc, int a_fmt, con
     else return cudaErrorInvalidValue;
     const int stage_k = kind == KIND_F8F6F4 ? 128 : 256;
     if (K % stage_k) return cudaErrorInvalidValue;
-    const bool a_fp4 = kind != KIND_F8F6F4, b_fp4 = b_fmt == FMT_E2M1 || b_fmt == FMT_NVFP4;
-    const bool b_expand = kind == KIND_F8F6F4 && b_fp4;
+    // sub-byte codes are expanded by the copy for the mxf8f6f4 kind only
+    const bool a_expand = kind == KIND_F8F6F4 && code_bits(a_fmt) < 8;
+    const bool b_expand = kind == KIND_F8F6F4 && code_bits(b_fmt) < 8;
     CUtensorMap tmA, tmB;
-    if (!encode_operand(enc, &tmA, a_elems, M, K, a_fp4, false, kBM)) return cudaErrorInvalidValue;
+    if (!encode_operand(enc, &tmA, a_elems, M, K, a_fmt, a_expand, kBM)) return cudaErrorInvalidValue;
     const bool wide = N % 256 == 0;
     const int bn = wide ? 256 : 128;
-    if (!encode_operand(enc, &tmB, b_elems, N, K, b_fp4, b_expand, (uint32_t)bn)) return cudaErrorInvalidValue;
+    if (!encode_operand(enc, &tmB, b_elems, N, K, b_fmt, b_expand, (uint32_t)bn)) return cudaErrorInvalidValue;
     const int64_t n_tiles = (M / kBM) * (N / bn);
     // band of N-tiles whose B panels (bn rows x K codes) take at most ~48 MB of L2
-    const int64_t panel = (int64_t)bn * (b_fp4 ? K / 2 : K);
+    const int64_t panel = (int64_t)bn * (K * code_bits(b_fmt) / 8);
     int64_t band = (48ll << 20) / (panel > 0 ? panel : 1);
     if (band < 1) band = 1;
     if (band > N / bn) band = N / bn;

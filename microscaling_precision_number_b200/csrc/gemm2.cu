@@ -137,8 +137,10 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             const int col_atoms = num_kb * P::kAtoms;        // scale atoms per 128-row block
-            const bool b_expanded = KIND == KIND_F8F6F4 && b_fmt_code == 5u;
-            const uint32_t tx_pair = 2u * (kABytes + (b_expanded ? kBBytes / 2 : kBBytes) + P::kSfaBytes + P::kSfbBytes);
+            const uint32_t tx_pair =
+                2u * ((KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kABytes, a_fmt_code) : kABytes) +
+                      (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kBBytes, b_fmt_code) : kBBytes) + P::kSfaBytes +
+                      P::kSfbBytes);
             int it = 0;
             for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs) {
                 int m_blk, n_blk;
@@ -275,14 +277,19 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                   CUtensorMapFloatOOBfill);
 
-// Operand codes: rows x K, 128 bytes of K x 128 rows per box, 128-byte swizzle (as gemm.cu).
-static bool encode_codes(EncodeTiledFn enc, CUtensorMap *tm, const void *ptr, int64_t rows, int64_t K, bool fp4,
+// Operand codes: rows x K, 128 bytes of K x 128 rows per box, 128-byte swizzle (as gemm.cu;
+// E2M1 / FP6 codes of the mxf8f6f4 kind expanded by the copy to 16-byte groups).
+static bool encode_codes(EncodeTiledFn enc, CUtensorMap *tm, const void *ptr, int64_t rows, int64_t K, int fmt,
                          bool expand) {
-    const cuuint64_t gdim[2] = {(cuuint64_t)(fp4 && !expand ? K / 2 : K), (cuuint64_t)rows};
-    const cuuint64_t gstride[1] = {(cuuint64_t)(fp4 ? K / 2 : K)};
+    const int bits = code_bits(fmt);
+    const cuuint64_t gdim[2] = {(cuuint64_t)(expand || bits == 8 ? K : K * bits / 8), (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)(K * bits / 8)};
     const cuuint32_t box[2] = {(cuuint32_t)kRowBytes, (cuuint32_t)kHalfRows};
     const cuuint32_t estr[2] = {1, 1};
-    return enc(tm, expand ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+    const CUtensorMapDataType dt = !expand ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : bits == 6 ? CU_TENSOR_MAP_DATA_TYPE_16U6_ALIGN16B
+                                               : CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B;
+    return enc(tm, dt, 2,
                const_cast<void *>(ptr), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -302,20 +309,22 @@ static bool encode_scales(EncodeTiledFn enc, CUtensorMap *tm, const uint8_t *ptr
 }
 
 template <int KIND>
-static cudaError_t launch_pair_k(EncodeTiledFn enc, const void *a, const uint8_t *a_sc, const float *ga,
-                                 const void *b, const uint8_t *b_sc, const float *gb, bool b_fp4, bool b_expand,
-                                 uint32_t a_code, uint32_t b_code, void *c, int64_t M, int64_t N, int64_t K,
-                                 int *watchdog, int num_sms, cudaStream_t st) {
+static cudaError_t launch_pair_k(EncodeTiledFn enc, const void *a, const uint8_t *a_sc, const float *ga, int a_fmt,
+                                 const void *b, const uint8_t *b_sc, const float *gb, int b_fmt, uint32_t a_code,
+                                 uint32_t b_code, void *c, int64_t M, int64_t N, int64_t K, int *watchdog,
+                                 int num_sms, cudaStream_t st) {
     using P = Pair<KIND>;
     CUtensorMap tmA, tmB, tmSA, tmSB;
     const int64_t col_atoms = (K / P::kStageK) * P::kAtoms;
-    if (!encode_codes(enc, &tmA, a, M, K, KIND != KIND_F8F6F4, false) ||
-        !encode_codes(enc, &tmB, b, N, K, b_fp4, b_expand) ||
+    const bool a_expand = KIND == KIND_F8F6F4 && code_bits(a_fmt) < 8;
+    const bool b_expand = KIND == KIND_F8F6F4 && code_bits(b_fmt) < 8;
+    if (!encode_codes(enc, &tmA, a, M, K, a_fmt, a_expand) ||
+        !encode_codes(enc, &tmB, b, N, K, b_fmt, b_expand) ||
         !encode_scales(enc, &tmSA, a_sc, M, col_atoms, P::kAtoms) ||
         !encode_scales(enc, &tmSB, b_sc, N, col_atoms, P::kAtoms))
         return cudaErrorInvalidValue;
     const int64_t n_tiles = (M / kPairM) * (N / kPairN);
-    const int64_t panel = (int64_t)kPairN * (b_fp4 ? K / 2 : K);
+    const int64_t panel = (int64_t)kPairN * (K * code_bits(b_fmt) / 8);
     int64_t band = (48ll << 20) / (panel > 0 ? panel : 1);
     if (band < 1) band = 1;
     if (band > N / kPairN) band = N / kPairN;
@@ -341,17 +350,16 @@ cudaError_t launch_gemm_pair(const void *a_elems, const uint8_t *a_sc, int a_fmt
     if (!gemm_pair_supported(M, N)) return cudaErrorInvalidValue;
     if (f8f6f4_code(a_fmt) >= 0 && a_fmt != FMT_E2M1 && f8f6f4_code(b_fmt) >= 0) {
         if (K % 128) return cudaErrorInvalidValue;
-        const bool fp4 = b_fmt == FMT_E2M1;
-        return launch_pair_k<KIND_F8F6F4>(enc, a_elems, a_sc, nullptr, b_elems, b_sc, nullptr, fp4, fp4,
+        return launch_pair_k<KIND_F8F6F4>(enc, a_elems, a_sc, nullptr, a_fmt, b_elems, b_sc, nullptr, b_fmt,
                                           (uint32_t)f8f6f4_code(a_fmt), (uint32_t)f8f6f4_code(b_fmt), c, M, N, K,
                                           watchdog, num_sms, st);
     }
     if (K % 256) return cudaErrorInvalidValue;
     if (a_fmt == FMT_E2M1 && b_fmt == FMT_E2M1)
-        return launch_pair_k<KIND_MXF4>(enc, a_elems, a_sc, nullptr, b_elems, b_sc, nullptr, true, false, 1u, 1u, c, M,
-                                        N, K, watchdog, num_sms, st);
+        return launch_pair_k<KIND_MXF4>(enc, a_elems, a_sc, nullptr, a_fmt, b_elems, b_sc, nullptr, b_fmt, 1u, 1u, c,
+                                        M, N, K, watchdog, num_sms, st);
     if (a_fmt == FMT_NVFP4 && b_fmt == FMT_NVFP4)
-        return launch_pair_k<KIND_NVF4>(enc, a_elems, a_sc, ga, b_elems, b_sc, gb, true, false, 1u, 1u, c, M, N, K,
+        return launch_pair_k<KIND_NVF4>(enc, a_elems, a_sc, ga, a_fmt, b_elems, b_sc, gb, b_fmt, 1u, 1u, c, M, N, K,
                                         watchdog, num_sms, st);
     return cudaErrorInvalidValue;
 }

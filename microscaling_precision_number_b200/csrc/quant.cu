@@ -8,7 +8,8 @@
 //   implementation-defined overflow of §8 "適合性検証という新しい層").
 //
 // A "chunk" is 16 bytes of bf16 input (8 elements); each thread converts whole chunks
-// with the hardware cvt.rn.satfinite conversions and writes 8 (FP8) or 4 (FP4) bytes.
+// with the hardware cvt.rn.satfinite conversions and writes 8 (FP8), 6 (FP6, packed) or
+// 4 (FP4) bytes.
 #include "codec.cuh"
 #include "internal.h"
 
@@ -78,7 +79,22 @@ __device__ __forceinline__ void cast8(const uint4 &v, uint8_t *out, int64_t c) {
                                           : 0x7Fu | (__float_as_uint(x[i]) >> 31 << 7);
                 w[i >> 2] = (w[i >> 2] & ~(0xFFu << (8 * (i & 3)))) | (nanc << (8 * (i & 3)));
             }
-        reinterpret_cast<uint2 *>(out)[c] = make_uint2(w[0], w[1]);
+        if constexpr (is_fp6(FMT)) {
+            // 8 codes packed into 6 bytes at 6c: a 4-byte and a 2-byte store, in the order
+            // that keeps each aligned (6c is 4-aligned for even c, 2 more for odd c)
+            const uint32_t p0 = fp6_pack4(w[0]), p1 = fp6_pack4(w[1]);
+            const uint32_t lo = p0 | (p1 << 24), hi = p1 >> 8;      // 48 bits
+            uint8_t *d = out + c * 6;
+            if ((c & 1) == 0) {
+                *reinterpret_cast<uint32_t *>(d) = lo;
+                *reinterpret_cast<uint16_t *>(d + 4) = (uint16_t)hi;
+            } else {
+                *reinterpret_cast<uint16_t *>(d) = (uint16_t)lo;
+                *reinterpret_cast<uint32_t *>(d + 2) = (lo >> 16) | (hi << 16);
+            }
+        } else {
+            reinterpret_cast<uint2 *>(out)[c] = make_uint2(w[0], w[1]);
+        }
     }
 }
 
@@ -98,8 +114,8 @@ cast_kernel(const uint4 *__restrict__ src, int64_t n_chunks, const uint16_t *__r
         v.z = t16[4] | ((uint32_t)t16[5] << 16); v.w = t16[6] | ((uint32_t)t16[7] << 16);
         alignas(8) uint8_t tmp[8];
         cast8<FMT>(v, tmp, 0);
-        const int nbytes = FMT == FMT_E2M1 ? tail / 2 : tail;
-        uint8_t *dst = out + (FMT == FMT_E2M1 ? n_chunks * 4 : n_chunks * 8);
+        const int nbytes = tail * code_bits(FMT) / 8;                 // FP6: tail is 4
+        uint8_t *dst = out + n_chunks * code_bits(FMT);
         for (int i = 0; i < nbytes; i++) dst[i] = tmp[i];
     }
 }

@@ -172,18 +172,43 @@ mx_rows_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS,
         const uint32_t code = e8m0_from_amax_bits<FMT, CEIL>(m);
         const uint64_t mul2x = splat2(e8m0_inverse_multiplier(code));
         const bool nan_blk = code == 0xFFu;
+        if constexpr (is_fp6(FMT)) {
+            // the 32 codes are packed into 24 bytes, so the rotated chunks are put back in
+            // order (register selects) before packing
+            uint2 q[4];
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const uint32_t c = (j + rot) & 3u;                 // which 8-element chunk of the block
-            float x[8];
-            scale8(v[j], mul2x, x);
-            if constexpr (FMT == FMT_E2M1) {
-                const uint32_t q = nan_blk ? 0u : cvt_e2m1x8(x);
-                reinterpret_cast<uint32_t *>(elems)[(size_t)blk * 4 + c] = q;
-            } else {
-                uint2 q = cvt_fp8x8<FMT>(x);
-                if (nan_blk) q = make_uint2(0u, 0u);
-                reinterpret_cast<uint2 *>(elems)[(size_t)blk * 4 + c] = q;
+            for (int j = 0; j < 4; j++) {
+                float x[8];
+                scale8(v[j], mul2x, x);
+                q[j] = cvt_fp8x8<FMT>(x);
+            }
+            uint32_t w[8];
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                const uint32_t j = (c - rot) & 3u;              // q[j] holds chunk c
+                const uint2 t = j == 0 ? q[0] : j == 1 ? q[1] : j == 2 ? q[2] : q[3];
+                w[2 * c] = t.x;
+                w[2 * c + 1] = t.y;
+            }
+            uint32_t o[6];
+            fp6_pack<8>(w, o);
+            uint2 *dst = reinterpret_cast<uint2 *>(elems + (size_t)blk * 24);
+#pragma unroll
+            for (int i = 0; i < 3; i++) dst[i] = nan_blk ? make_uint2(0u, 0u) : make_uint2(o[2 * i], o[2 * i + 1]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const uint32_t c = (j + rot) & 3u;             // which 8-element chunk of the block
+                float x[8];
+                scale8(v[j], mul2x, x);
+                if constexpr (FMT == FMT_E2M1) {
+                    const uint32_t q = nan_blk ? 0u : cvt_e2m1x8(x);
+                    reinterpret_cast<uint32_t *>(elems)[(size_t)blk * 4 + c] = q;
+                } else {
+                    uint2 q = cvt_fp8x8<FMT>(x);
+                    if (nan_blk) q = make_uint2(0u, 0u);
+                    reinterpret_cast<uint2 *>(elems)[(size_t)blk * 4 + c] = q;
+                }
             }
         }
         if constexpr (RM) sc_rm[blk] = (uint8_t)code;
@@ -491,10 +516,13 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
     pdl_wait_and_release();
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages];
-    constexpr uint32_t kCodeBytes = FMT == FMT_E2M1 ? 16 : 32;           // per block
+    constexpr uint32_t kCodeBytes = 32 * code_bits(FMT) / 8;              // per block: 16, 24 or 32
     constexpr uint32_t kBlocksPerTile = kThreads;                          // one per thread
+    // Bulk copies move whole 16-byte units; with FP6 (24 bytes a block) and an odd block
+    // count the last block is read straight from global memory by its thread.
+    const uint32_t ring_blocks = is_fp6(FMT) ? (n_blocks & ~1u) : n_blocks;
     Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
-              full, watchdog, elems, kBlocksPerTile * kCodeBytes, (uint64_t)n_blocks * kCodeBytes};
+              full, watchdog, elems, kBlocksPerTile * kCodeBytes, (uint64_t)ring_blocks * kCodeBytes};
     const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
     const uint32_t tid = threadIdx.x;
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
@@ -522,6 +550,28 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
                 o.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
                 o.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
                 dst[j] = o;
+            }
+        } else if constexpr (is_fp6(FMT)) {
+            // 24 bytes = 32 packed codes, as three 8-byte reads (stride 24 B: conflict-free)
+            const uint2 *p = blk < ring_blocks ? reinterpret_cast<const uint2 *>(tile + tid * 24)
+                                               : reinterpret_cast<const uint2 *>(elems + (size_t)blk * 24);
+            const uint2 a = p[0], b = p[1], c = p[2];
+            const uint32_t o[6] = {a.x, a.y, b.x, b.y, c.x, c.y};
+            uint32_t w[8];
+            fp6_unpack<8>(o, w);
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                float y[8];
+                fp8x2_to_f32<FMT>(w[2 * j] & 0xFFFFu, y[0], y[1]);
+                fp8x2_to_f32<FMT>(w[2 * j] >> 16, y[2], y[3]);
+                fp8x2_to_f32<FMT>(w[2 * j + 1] & 0xFFFFu, y[4], y[5]);
+                fp8x2_to_f32<FMT>(w[2 * j + 1] >> 16, y[6], y[7]);
+                uint4 q;
+                q.x = f32x2_to_bf16x2(__fmul_rn(y[0], mul), __fmul_rn(y[1], mul));
+                q.y = f32x2_to_bf16x2(__fmul_rn(y[2], mul), __fmul_rn(y[3], mul));
+                q.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
+                q.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
+                dst[j] = q;
             }
         } else {
             const uint32_t rot = (tid >> 2) & 1u;

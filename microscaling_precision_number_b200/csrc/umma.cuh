@@ -18,6 +18,14 @@ __host__ __device__ constexpr int f8f6f4_code(int fmt) {
     return fmt == 0 ? 0 : fmt == 1 ? 1 : fmt == 4 ? 3 : fmt == 5 ? 4 : fmt == 2 ? 5 : -1;
 }
 
+// Global bytes behind `smem_bytes` of an mxf8f6f4 operand tile.  FP4 (code 5) and FP6
+// (codes 3, 4) are stored packed and the copy expands each 16 codes to a 16-byte group in
+// shared memory (16U4_ALIGN16B: 8 code bytes; 16U6_ALIGN16B: 12); the copy's transaction
+// count is the packed size.
+__host__ __device__ constexpr uint32_t f8f6f4_packed_bytes(uint32_t smem_bytes, uint32_t code) {
+    return code == 5u ? smem_bytes / 2 : (code == 3u || code == 4u) ? smem_bytes / 4 * 3 : smem_bytes;
+}
+
 // ---- tcgen05 wrappers -------------------------------------------------------------------
 // Tensor-memory allocation by one full warp.  With CG = 2 the instruction is collective
 // over the CTA pair: the warp with the same index in both CTAs executes it, and both pass

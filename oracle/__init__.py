@@ -116,8 +116,14 @@ def scale_exponent(amax: float, fmt: int, rounding: int) -> int:
     return lib().mxo_scale_exponent(float(amax), fmt, rounding)
 
 
+def code_bits(fmt: int) -> int:
+    """Stored width of one element code: FP4 4, FP6 6, FP8 / INT8 8."""
+    return 4 if fmt in (E2M1, NVFP4) else 6 if fmt in (E2M3, E3M2) else 8
+
+
 def elem_bytes(n_elems: int, fmt: int) -> int:
-    return n_elems // 2 if fmt in (E2M1, NVFP4) else n_elems
+    """Bytes of n densely packed element codes (n * width / 8)."""
+    return n_elems * code_bits(fmt) // 8
 
 
 # ---------------------------------------------------------------- block operations
@@ -138,7 +144,8 @@ def quantize_mx(x_bf16_bits: np.ndarray, fmt: int, axis: int = ROW, rounding: in
 
 
 def cast(x_bf16_bits: np.ndarray, fmt: int) -> np.ndarray:
-    """Direct element cast with no block scale (codes, FP4 packed two per byte)."""
+    """Direct element cast with no block scale (codes densely packed: FP4 two per byte,
+    FP6 four per three bytes)."""
     x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16).reshape(-1)
     out = np.zeros(elem_bytes(x.size, fmt), dtype=np.uint8)
     _check(lib().mxo_cast(_ptr(x), x.size, fmt, _ptr(out)), "cast")

@@ -40,7 +40,10 @@
  *     (Q§2: a NaN scale makes the whole block NaN, so the codes carry nothing);
  *   - an all-zero block gets s = -127 (E8M0 code 0x00) after the clamp;
  *   - the sign of a zero result is kept (-tiny -> 0x80 for FP8, 0x8 for FP4);
- *   - FP4 codes pack two per byte, even element index in the low nibble;
+ *   - element codes are stored densely, code i of a row at bits [w*i, w*i + w) of the
+ *     row read as a little-endian bit string: FP4 two per byte (even index low), FP6
+ *     four per three bytes, FP8 / INT8 one per byte (the pages give no memory layout;
+ *     dense packing keeps MXFP6 at its 6.25 bits per element);
  *   - column-wise output is the transposed matrix (cols x rows), blocks along rows;
  *   - NVFP4 step order: see mxo_quantize_nvfp4.
  */
@@ -321,17 +324,30 @@ static unsigned quantize_block_mx(const uint16_t *x, int n, int fmt, int roundin
     return (unsigned)(s + 127);
 }
 
-/* Store code i of a row into an output row (FP8, FP6 in the low 6 bits, INT8: one byte;
- * FP4: nibble, even low). */
-static void put_code(uint8_t *row, int64_t i, unsigned code, int fp4) {
-    if (!fp4) { row[i] = (uint8_t)code; return; }
-    uint8_t *p = row + i / 2;
-    if (i % 2 == 0) *p = (uint8_t)((*p & 0xF0u) | (code & 0xFu));
-    else            *p = (uint8_t)((*p & 0x0Fu) | ((code & 0xFu) << 4));
+/* Width in bits of one stored element code: FP8 and INT8 8, FP6 6, FP4 4.             */
+static int code_bits(int fmt) {
+    return (fmt == F_E2M1 || fmt == F_NVFP4) ? 4 : (fmt == F_E2M3 || fmt == F_E3M2) ? 6 : 8;
 }
-static unsigned get_code(const uint8_t *row, int64_t i, int fp4) {
-    if (!fp4) return row[i];
-    return (i % 2 == 0) ? (row[i / 2] & 0xFu) : (row[i / 2] >> 4);
+
+/* Element codes are stored densely along a row: code i occupies bits [w*i, w*i + w) of
+ * the row's bytes read as one little-endian bit string (w = code width).  For FP4 that
+ * is two codes per byte, the even one low; for FP6 four codes per three bytes; for FP8
+ * and INT8 one code per byte.  Written bit by bit, the plainest form of that rule. */
+static void put_code(uint8_t *row, int64_t i, unsigned code, int bits) {
+    for (int b = 0; b < bits; b++) {
+        int64_t at = (int64_t)bits * i + b;
+        uint8_t m = (uint8_t)(1u << (at % 8));
+        if ((code >> b) & 1u) row[at / 8] |= m;
+        else                  row[at / 8] &= (uint8_t)~m;
+    }
+}
+static unsigned get_code(const uint8_t *row, int64_t i, int bits) {
+    unsigned code = 0;
+    for (int b = 0; b < bits; b++) {
+        int64_t at = (int64_t)bits * i + b;
+        code |= (unsigned)((row[at / 8] >> (at % 8)) & 1u) << b;
+    }
+    return code;
 }
 
 /*
@@ -345,12 +361,12 @@ static unsigned get_code(const uint8_t *row, int64_t i, int fp4) {
 int mxo_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int axis, int rounding,
                     uint8_t *elems, uint8_t *scales) {
     const int B = 32;
-    int fp4 = (fmt == F_E2M1);
+    int bits = code_bits(fmt);
     int64_t out_rows = axis == 0 ? rows : cols, out_cols = axis == 0 ? cols : rows;
     if (!mx_fmt_ok(fmt) || out_cols % B) return -1;
     uint16_t blk[32];
     unsigned codes[32];
-    int64_t row_bytes = fp4 ? out_cols / 2 : out_cols;
+    int64_t row_bytes = out_cols * bits / 8;
     memset(elems, 0, (size_t)(out_rows * row_bytes));
     for (int64_t r = 0; r < out_rows; r++) {
         for (int64_t b = 0; b < out_cols / B; b++) {
@@ -359,7 +375,7 @@ int mxo_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int 
                 blk[i] = axis == 0 ? x[r * cols + j] : x[j * cols + r];
             }
             scales[r * (out_cols / B) + b] = (uint8_t)quantize_block_mx(blk, B, fmt, rounding, codes);
-            for (int i = 0; i < B; i++) put_code(elems + r * row_bytes, b * B + i, codes[i], fp4);
+            for (int i = 0; i < B; i++) put_code(elems + r * row_bytes, b * B + i, codes[i], bits);
         }
     }
     return 0;
@@ -367,10 +383,10 @@ int mxo_quantize_mx(const uint16_t *x, int64_t rows, int64_t cols, int fmt, int 
 
 /* Direct element cast with no block scale (the "direct cast" of [P4]). */
 int mxo_cast(const uint16_t *x, int64_t n, int fmt, uint8_t *out) {
-    int fp4 = (fmt == F_E2M1);
-    if (!mx_fmt_ok(fmt) || fmt == F_INT8 || (fp4 && n % 2)) return -1;   /* INT8 needs a scale */
-    memset(out, 0, (size_t)(fp4 ? n / 2 : n));
-    for (int64_t i = 0; i < n; i++) put_code(out, i, mxo_encode(bf16_value(x[i]), elem_kind(fmt)), fp4);
+    int bits = code_bits(fmt);
+    if (!mx_fmt_ok(fmt) || fmt == F_INT8 || (n * bits) % 8) return -1;   /* INT8 needs a scale */
+    memset(out, 0, (size_t)(n * bits / 8));
+    for (int64_t i = 0; i < n; i++) put_code(out, i, mxo_encode(bf16_value(x[i]), elem_kind(fmt)), bits);
     return 0;
 }
 
@@ -407,7 +423,7 @@ static unsigned nvfp4_block(const uint16_t *x, int64_t cols, int64_t r0, int64_t
         }
     if (nonfinite) {
         for (int rr = 0; rr < nr; rr++)
-            for (int i = 0; i < B; i++) put_code(elems + (r0 + rr) * (cols / 2), c0 + i, 0, 1);
+            for (int i = 0; i < B; i++) put_code(elems + (r0 + rr) * (cols / 2), c0 + i, 0, 4);
         return 0x7Fu;
     }
     volatile float six_g = 6.0f * g;
@@ -424,7 +440,7 @@ static unsigned nvfp4_block(const uint16_t *x, int64_t cols, int64_t r0, int64_t
                 if (isnan(y)) y = xi;     /* 0 * Inf when 1/d overflows: keep the signed zero */
                 q = mxo_encode((double)y, K_E2M1);
             }
-            put_code(elems + (r0 + rr) * (cols / 2), c0 + i, q, 1);
+            put_code(elems + (r0 + rr) * (cols / 2), c0 + i, q, 4);
         }
     return sb;
 }
@@ -486,13 +502,13 @@ int mxo_quantize_nvfp4_2d(const uint16_t *x, int64_t rows, int64_t cols, uint8_t
 int mxo_dequantize_mx(const uint8_t *elems, const uint8_t *scales, int64_t rows, int64_t cols,
                       int fmt, uint16_t *out) {
     const int B = 32;
-    int fp4 = (fmt == F_E2M1);
+    int bits = code_bits(fmt);
     if (!mx_fmt_ok(fmt) || cols % B) return -1;
-    int64_t row_bytes = fp4 ? cols / 2 : cols;
+    int64_t row_bytes = cols * bits / 8;
     for (int64_t r = 0; r < rows; r++) {
         for (int64_t j = 0; j < cols; j++) {
             unsigned s = scales[r * (cols / B) + j / B];
-            unsigned q = get_code(elems + r * row_bytes, j, fp4);
+            unsigned q = get_code(elems + r * row_bytes, j, bits);
             double v = s == 0xFFu ? NAN : ldexp(mxo_decode(elem_kind(fmt), q), (int)s - 127);
             out[r * cols + j] = (uint16_t)mxo_encode(v, K_BF16);
         }
@@ -508,7 +524,7 @@ int mxo_dequantize_nvfp4(const uint8_t *elems, const uint8_t *scales, float g, i
     for (int64_t r = 0; r < rows; r++) {
         for (int64_t j = 0; j < cols; j++) {
             unsigned sb = scales[r * (cols / B) + j / B] & 0x7Fu;
-            unsigned q = get_code(elems + r * (cols / 2), j, 1);
+            unsigned q = get_code(elems + r * (cols / 2), j, 4);
             if (sb == 0x7Fu) { out[r * cols + j] = 0x7FC0u; continue; }
             volatile float p = (float)mxo_decode(K_E2M1, q) * (float)mxo_decode(K_UE4M3, sb);
             volatile float y = p * g;
@@ -547,9 +563,9 @@ int64_t mxo_tcgen05_scale_offset(int64_t r, int64_t c, int64_t rows, int64_t sca
 /* ------------------------------------------------------------------------- */
 static double mx_operand_value(const uint8_t *elems, const uint8_t *scales, int fmt, double g,
                                int64_t row, int64_t k, int64_t K) {
-    int fp4 = (fmt == F_E2M1 || fmt == F_NVFP4);
-    int64_t row_bytes = fp4 ? K / 2 : K;
-    unsigned q = get_code(elems + row * row_bytes, k, fp4);
+    int bits = code_bits(fmt);
+    int64_t row_bytes = K * bits / 8;
+    unsigned q = get_code(elems + row * row_bytes, k, bits);
     if (fmt == F_NVFP4) {
         unsigned sb = scales[row * (K / 16) + k / 16];
         if (sb == 0x7Fu) return NAN;
@@ -618,7 +634,7 @@ int mxo_mxfp4_to_fp8_blocks(const uint8_t *elems, const uint8_t *scales, int64_t
                     if (sc == 0xFFu) continue;
                     int nonzero = 0;
                     for (int64_t j = b * 32; j < b * 32 + 32; j++)
-                        if (mxo_decode(K_E2M1, get_code(elems + r * (cols / 2), j, 1)) != 0.0) nonzero = 1;
+                        if (mxo_decode(K_E2M1, get_code(elems + r * (cols / 2), j, 4)) != 0.0) nonzero = 1;
                     if (nonzero && (int)sc - 127 > smax) smax = (int)sc - 127;
                 }
             }
@@ -628,7 +644,7 @@ int mxo_mxfp4_to_fp8_blocks(const uint8_t *elems, const uint8_t *scales, int64_t
             for (int64_t r = br * 128; r < br * 128 + 128; r++) {
                 for (int64_t j = bc * 128; j < bc * 128 + 128; j++) {
                     unsigned sc = scales[r * S + j / 32];
-                    unsigned q = get_code(elems + r * (cols / 2), j, 1);
+                    unsigned q = get_code(elems + r * (cols / 2), j, 4);
                     unsigned code;
                     if (sc == 0xFFu) {
                         code = 0x7Fu;
@@ -724,8 +740,8 @@ int mxo_quantize_mx_sr(const uint16_t *x, int64_t rows, int64_t cols, int fmt, i
                        const uint8_t *rnd, uint8_t *elems, uint8_t *scales) {
     const int B = 32;
     if (!(fmt == F_E4M3 || fmt == F_E5M2 || fmt == F_E2M1) || cols % B) return -1;
-    int fp4 = fmt == F_E2M1;
-    int64_t row_bytes = fp4 ? cols / 2 : cols;
+    int bits = code_bits(fmt);
+    int64_t row_bytes = cols * bits / 8;
     memset(elems, 0, (size_t)(rows * row_bytes));
     for (int64_t r = 0; r < rows; r++)
         for (int64_t b = 0; b < cols / B; b++) {
@@ -746,7 +762,7 @@ int mxo_quantize_mx_sr(const uint16_t *x, int64_t rows, int64_t cols, int fmt, i
             for (int i = 0; i < B; i++) {
                 double scaled = ldexp(bf16_value(blk[i]), -s);
                 put_code(elems + r * row_bytes, b * B + i,
-                         encode_sr(scaled, elem_kind(fmt), rnd[r * cols + b * B + i]), fp4);
+                         encode_sr(scaled, elem_kind(fmt), rnd[r * cols + b * B + i]), bits);
             }
         }
     return 0;
@@ -786,7 +802,7 @@ int mxo_quantize_nvfp4_sr(const uint16_t *x, int64_t rows, int64_t cols, const u
                     if (isnan(y)) y = xi;
                     q = encode_sr((double)y, K_E2M1, rnd[r * cols + b * B + i]);
                 }
-                put_code(elems + r * (cols / 2), b * B + i, q, 1);
+                put_code(elems + r * (cols / 2), b * B + i, q, 4);
             }
         }
     return 0;

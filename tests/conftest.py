@@ -26,6 +26,22 @@ def read_golden(name):
     return out
 
 
+def pack_codes(codes, bits):
+    """Codes (one per entry, last axis along a row) -> the dense little-endian bit packing:
+    code i at bits [bits*i, bits*i + bits) of the row.  numpy's bit routines, independent of
+    the oracle's bit loop and the kernels' word arithmetic."""
+    c = np.asarray(codes, dtype=np.uint8)
+    b = np.unpackbits(c[..., None], axis=-1, bitorder="little")[..., :bits]
+    return np.packbits(b.reshape(*c.shape[:-1], -1), axis=-1, bitorder="little")
+
+
+def unpack_codes(packed, n, bits):
+    """Inverse of pack_codes for rows of n codes."""
+    p = np.asarray(packed, dtype=np.uint8)
+    b = np.unpackbits(p, axis=-1, bitorder="little")[..., :n * bits].reshape(*p.shape[:-1], n, bits)
+    return np.packbits(b, axis=-1, bitorder="little")[..., 0]
+
+
 def f32_to_bf16_bits(values):
     """Exact fp32 values (already bf16-representable) -> bf16 bit patterns."""
     a = np.asarray(values, dtype=np.float32)

@@ -93,6 +93,8 @@ def test_dual_dequant_cast_gemm_validation(L):
     assert lib.mx_cast(FAKE, 7, 2, FAKE, None) == L.MX_ERR_SHAPE
     assert lib.mx_cast(FAKE, 8, 3, FAKE, None) == L.MX_ERR_ARG
     assert lib.mx_cast(FAKE, 8, 6, FAKE, None) == L.MX_ERR_ARG        # INT8 needs a scale
+    assert lib.mx_cast(FAKE, 6, 4, FAKE, None) == L.MX_ERR_SHAPE      # FP6: whole bytes of packed codes
+    assert lib.mx_cast(FAKE, 10, 5, FAKE, None) == L.MX_ERR_SHAPE
     assert lib.mx_quantize(FAKE, 4, 64, 7, 0, 1, FAKE, FAKE, 1, None, None, None) == L.MX_ERR_ARG
     assert lib.mx_quantize(FAKE, 4, 64, 6, 0, 1, FAKE, FAKE, 1, None, FAKE, None) == L.MX_ERR_ARG   # g is NVFP4 only
     assert lib.mx_cast(None, 8, 0, FAKE, None) == L.MX_ERR_ARG

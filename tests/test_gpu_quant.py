@@ -6,6 +6,7 @@ import pytest
 import torch
 
 import synth
+from conftest import pack_codes
 
 pytestmark = pytest.mark.gpu
 
@@ -67,11 +68,15 @@ def test_cast_exhaustive_bf16(oracle, fmt):
     assert bad.size == 0, f"{bad.size} mismatching bytes, first at {bad[:8]}"
 
 
-@pytest.mark.parametrize("n", [2, 10, 30, 1000, 4097 * 8 + 6])
+@pytest.mark.parametrize("n", [2, 4, 10, 28, 1000, 4097 * 8 + 4, 4097 * 8 + 6])
 def test_cast_tail(oracle, n):
     rng = np.random.default_rng(n)
     bits = rng.integers(0, 65536, size=n, dtype=np.uint32).astype(np.uint16)
-    for fmt in (0, 2, 4):
+    for fmt in (0, 2, 4, 5):
+        if fmt in (4, 5) and n % 4:                     # FP6: whole bytes of packed codes only
+            with pytest.raises(mx.MxError):
+                mx.cast(to_dev(bits), FMT_NAMES[fmt])
+            continue
         assert np.array_equal(host(mx.cast(to_dev(bits), FMT_NAMES[fmt])), oracle.cast(bits, fmt))
 
 
@@ -189,6 +194,8 @@ def test_dequantize_all_scale_codes(oracle):
         scales = np.arange(256, dtype=np.uint8).reshape(256, 1)
         if fmt == 2:
             elems = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+        elif fmt in (4, 5):
+            elems = pack_codes(codes, 6)                  # 24 bytes per 32 codes
         else:
             elems = codes
         q = mx.Quantized(torch.from_numpy(np.ascontiguousarray(elems).reshape(-1)).cuda(),

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import synth
-from conftest import f32_to_bf16_bits, read_golden
+from conftest import f32_to_bf16_bits, read_golden, unpack_codes
 from test_oracle_formats import bf16_bits_to_f64, unpack_fp4
 
 
@@ -62,11 +62,10 @@ def test_effective_bits(oracle):
         assert (e.nbytes + s.nbytes) * 8 / n == g["bits_mxfp8"][0]
     e, s, _ = oracle.quantize_nvfp4(x)
     assert (e.nbytes + s.nbytes) * 8 / n == g["bits_nvfp4"][0]
-    # MXFP6: 6-bit codes (stored one per byte here) plus the shared scale
+    # MXFP6: 6-bit codes packed four per three bytes plus the shared scale
     for fmt in (oracle.E2M3, oracle.E3M2):
         e, s = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.FLOOR)
-        assert int(e.max()) < 64
-        assert (6 * e.size + 8 * s.nbytes) / n == g["bits_mxfp6"][0]
+        assert (e.nbytes + s.nbytes) * 8 / n == g["bits_mxfp6"][0]
     e, s = oracle.quantize_mx(x, oracle.INT8, oracle.ROW, oracle.FLOOR)
     assert (e.nbytes + s.nbytes) * 8 / n == g["bits_mxint8"][0]
 
@@ -83,8 +82,9 @@ def test_block_codes_are_the_cast_of_scaled_values(oracle, fmt_name, rounding):
     maxv = {"E4M3": 448.0, "E5M2": 57344.0, "E2M1": 6.0, "E2M3": 7.5, "E3M2": 28.0}[fmt_name]
     xf = bf16_bits_to_f64(x)
     fp4 = fmt_name == "E2M1"
+    fp6 = fmt_name in ("E2M3", "E3M2")
     for r in range(x.shape[0]):
-        codes = unpack_fp4(e[r], 128) if fp4 else e[r]
+        codes = unpack_fp4(e[r], 128) if fp4 else unpack_codes(e[r], 128, 6) if fp6 else e[r]
         for b in range(4):
             sc = int(s[r, b]) - 127
             blk = xf[r, 32 * b:32 * b + 32]
@@ -92,7 +92,7 @@ def test_block_codes_are_the_cast_of_scaled_values(oracle, fmt_name, rounding):
             ref = oracle.cast(f32_to_bf16_bits(scaled.astype(np.float32)), fmt) if np.all(
                 (scaled.astype(np.float32).view(np.uint32) & 0xFFFF) == 0) else None
             assert ref is not None              # power-of-two scaling keeps bf16 exact here
-            ref = unpack_fp4(ref, 32) if fp4 else ref
+            ref = unpack_fp4(ref, 32) if fp4 else unpack_codes(ref, 32, 6) if fp6 else ref
             assert np.array_equal(codes[32 * b:32 * b + 32], ref)
             top = np.abs(scaled).max()
             if rounding == 1:

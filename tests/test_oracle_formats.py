@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from conftest import read_golden
+from conftest import f32_to_bf16_bits, pack_codes, read_golden, unpack_codes
 
 ALL_BF16 = np.arange(65536, dtype=np.uint32).astype(np.uint16)
 
@@ -138,6 +138,8 @@ def test_exhaustive_bf16_cast_against_brute_force(oracle, fmt_name):
     got = oracle.cast(ALL_BF16, fmt)
     if fmt_name == "E2M1":
         got = unpack_fp4(got, ALL_BF16.size)
+    elif fmt_name in ("E2M3", "E3M2"):
+        got = unpack_codes(got, ALL_BF16.size, 6)
     bad = np.nonzero(got.astype(np.int64) != ref)[0]
     assert bad.size == 0, f"{bad.size} mismatches, first bf16 {ALL_BF16[bad[:5]]}"
 
@@ -159,9 +161,32 @@ def test_fp6_cast_matches_ml_dtypes_in_range(oracle, fmt_name, dtype, maxv):
     """ml_dtypes' FP6 conversion (round to nearest even) agrees with ours up to the max."""
     x32 = bf16_bits_to_f64(ALL_BF16).astype(np.float32)
     ok = np.isfinite(x32) & (np.abs(x32) <= maxv)
-    ref = x32[ok].astype(dtype).view(np.uint8) & 0x3F
-    got = oracle.cast(ALL_BF16[ok], getattr(oracle, fmt_name))
+    sel = ALL_BF16[ok][: ok.sum() // 4 * 4]              # FP6 casts take whole bytes: n % 4 == 0
+    ref = x32[ok][: sel.size].astype(dtype).view(np.uint8) & 0x3F
+    got = unpack_codes(oracle.cast(sel, getattr(oracle, fmt_name)), sel.size, 6)
     assert np.array_equal(got, ref)
+
+
+def test_fp6_storage_packing(oracle):
+    """FP6 codes are stored four per three bytes, code i at bits [6i, 6i + 6) of the row.
+    Hand-worked: E2M3 subnormals 0.125, 0.25, 0.375, 0.5 are codes 1, 2, 3, 4 (m / 8 with
+    bias 1), i.e. 1 + 2*2^6 + 3*2^12 + 4*2^18 = 0x103081 -> bytes 81 30 10; the E3M2 max
+    28 (code 0x1F) and -28 (0x3F) alternating give 0x1F | 0x3F << 6 | 0x1F << 12 | 0x3F << 18
+    = 0xFDFFDF -> DF FF FD."""
+    assert list(oracle.cast(f32_to_bf16_bits([0.125, 0.25, 0.375, 0.5]), oracle.E2M3)) == [0x81, 0x30, 0x10]
+    assert list(oracle.cast(f32_to_bf16_bits([28.0, -28.0, 28.0, -28.0]), oracle.E3M2)) == [0xDF, 0xFF, 0xFD]
+    # numpy's bit packing of the per-element codes, over all bf16 inputs
+    for fmt, kind in ((oracle.E2M3, oracle.K_E2M3), (oracle.E3M2, oracle.K_E3M2)):
+        x = ALL_BF16[::7][:4096]
+        codes = np.array([oracle.encode(v, kind) for v in bf16_bits_to_f64(x)], dtype=np.uint8)
+        codes[np.isnan(bf16_bits_to_f64(x))] = 0  # NaN inputs: compared separately below
+        keep = ~np.isnan(bf16_bits_to_f64(x))
+        got = unpack_codes(oracle.cast(x, fmt), x.size, 6)
+        assert np.array_equal(got[keep], codes[keep])
+        assert np.array_equal(pack_codes(got, 6), oracle.cast(x, fmt))
+    # a cast of a count that does not fill whole bytes is refused
+    with pytest.raises(ValueError):
+        oracle.cast(ALL_BF16[:6], oracle.E2M3)
 
 
 def test_int8_element_definition(oracle):
