@@ -431,20 +431,68 @@ def run_breakdown(mx, dev, pk):
     qw = mx.quantize(xw, "e2m1", "row", "floor", layout="rowmajor")
     R, C = xw.shape
     del xw
-    o8 = torch.empty(R * C, dtype=torch.uint8, device=dev)
+    # four rotating (codes, output) sets, 4 x 88 MiB > L2
+    sets = [(qw.elems if i == 0 else qw.elems.clone(), qw.scales if i == 0 else qw.scales.clone(),
+             torch.empty(R * C, dtype=torch.uint8, device=dev)) for i in range(4)]
     bsc = torch.empty((R // 128) * (C // 128), dtype=torch.float32, device=dev)
     bok = torch.empty((R // 128) * (C // 128), dtype=torch.uint8, device=dev)
 
-    def nested():
-        L.check(L.lib.mx_mxfp4_to_fp8_blocks(qw.elems.data_ptr(), qw.scales.data_ptr(), R, C, o8.data_ptr(),
+    def nested(e, sc, o8):
+        L.check(L.lib.mx_mxfp4_to_fp8_blocks(e.data_ptr(), sc.data_ptr(), R, C, o8.data_ptr(),
                                              bsc.data_ptr(), bok.data_ptr(), stream.cuda_stream),
                 "mx_mxfp4_to_fp8_blocks")
-    t = timed([nested], 20, stream)
+    t = timed([lambda st=st: nested(*st) for st in sets], 20, stream)
     nb = R * C // 2 + R * C // 32 + R * C + 5 * (R // 128) * (C // 128)
     out["next_nested_mxfp4_to_fp8_14336x4096"] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1),
                                                    "frac_hbm": round(nb / t / 1e6 / hbm, 4), "algorithmic_bytes": nb,
-                                                   "blocks_exact": int(bok.sum().item()), "blocks": int(bok.numel())}
-    del qw, o8, bsc, bok
+                                                   "blocks_exact": int(bok.sum().item()), "blocks": int(bok.numel()),
+                                                   "l2": "four rotating sets, 352 MiB > L2"}
+    del qw, sets, bsc, bok
+    torch.cuda.empty_cache()
+
+    # next row: training-side quantiser on the config-3 gradient shape (16384 x 14336 bf16):
+    # 16 x 16 random Hadamard transform + stochastic rounding (one random byte per element),
+    # NVFP4 (two passes; the maximum pass's re-read is not counted) and MXFP4; tcgen05 scales
+    R, C = 16384, 14336
+    xg = to_dev(synth.normal(R, C, sigma=1e-3, seed=70), dev)
+    rnd = torch.randint(0, 256, (R * C,), dtype=torch.uint8, device=dev)
+    for name, f, B in (("next_train_nvfp4_rht_sr_16384x14336", L.MX_FMT_NVFP4, 16),
+                       ("next_train_mxfp4_rht_sr_16384x14336", L.MX_FMT_E2M1, 32)):
+        el = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
+        sc = torch.empty(mx.scale_bytes(R, C // B, "tcgen05"), dtype=torch.uint8, device=dev)
+        gs = torch.empty(1, dtype=torch.float32, device=dev) if f == L.MX_FMT_NVFP4 else None
+
+        def train(f=f, el=el, sc=sc, gs=gs):
+            L.check(L.lib.mx_quantize_train(xg.data_ptr(), R, C, f, 0, 1, 0xB5C3, rnd.data_ptr(), el.data_ptr(),
+                                            sc.data_ptr(), L.MX_LAYOUT_TCGEN05, None,
+                                            gs.data_ptr() if gs is not None else None, stream.cuda_stream),
+                    "mx_quantize_train")
+        t = timed([train], 10, stream)
+        nb = R * C * 2 + R * C + R * C // 2 + sc.numel() + (4 if gs is not None else 0)
+        out[name] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1), "frac_hbm": round(nb / t / 1e6 / hbm, 4),
+                     "algorithmic_bytes": nb, "note": "input, random bytes, codes, scales; input larger than L2"}
+        del el, sc, gs
+    del xg, rnd
+    torch.cuda.empty_cache()
+
+    # next row: NVFP4 with 16 x 16 weight blocks on the config-2 weight (4096 x 4096)
+    R = C = 4096
+    xw = to_dev(synth.weight_fp4(), dev)
+    el = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
+    sc = torch.empty(mx.scale_bytes(R, C // 16, "tcgen05"), dtype=torch.uint8, device=dev)
+    gs = torch.empty(1, dtype=torch.float32, device=dev)
+
+    xs = [xw] + [xw.clone() for _ in range(5)]           # six rotating inputs (192 MiB > L2)
+
+    def nvfp4_2d(x):
+        L.check(L.lib.mx_quantize_nvfp4_2d(x.data_ptr(), R, C, el.data_ptr(), sc.data_ptr(), L.MX_LAYOUT_TCGEN05,
+                                           None, gs.data_ptr(), stream.cuda_stream), "mx_quantize_nvfp4_2d")
+    t = timed([lambda x=x: nvfp4_2d(x) for x in xs], 24, stream)
+    nb = R * C * 2 + R * C // 2 + sc.numel() + 4
+    out["next_quant_nvfp4_2d_weight_4096"] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1),
+                                              "frac_hbm": round(nb / t / 1e6 / hbm, 4), "algorithmic_bytes": nb,
+                                              "l2": "six rotating inputs, 192 MiB > L2"}
+    del xw, xs, el, sc, gs
     torch.cuda.empty_cache()
     return out
 
