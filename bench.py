@@ -345,7 +345,29 @@ def run_breakdown(mx, dev, pk):
                                     "quantize_GBps": round(b1 / tq / 1e6, 1),
                                     "dequantize_GBps": round(b1 / td / 1e6, 1),
                                     "frac_hbm": round(b1 / tq / 1e6 / hbm, 4),
-                                    "note": "3.2 MB per call, back-to-back calls: launch-latency bound"}
+                                    "note": "3.2 MB per call, back-to-back calls from Python: host-launch bound"}
+    # the same 64 calls captured once in a CUDA graph and replayed: device time per call
+    try:
+        graphs = []
+        for fn in ("q", "d"):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):                        # captured on torch's side stream
+                for x, q, y in zip(xs, qs, ys):
+                    if fn == "q":
+                        mx.quantize(x, "e4m3", "row", "ceil", layout="rowmajor", out=q)
+                    else:
+                        mx.dequantize(q, "rowmajor", out=y)
+            graphs.append(g)
+        gq, gd = (timed([g.replay], 4, stream) / len(xs) for g in graphs)
+        out["c1_mxfp8_rowwise_1024"].update({"graph_quantize_us": round(gq * 1e3, 2),
+                                             "graph_dequantize_us": round(gd * 1e3, 2),
+                                             "graph_quantize_GBps": round(b1 / gq / 1e6, 1),
+                                             "graph_dequantize_GBps": round(b1 / gd / 1e6, 1),
+                                             "graph_frac_hbm": round(b1 / gq / 1e6 / hbm, 4),
+                                             "graph_note": "64 calls on 64 rotating copies in one CUDA graph"})
+        del graphs
+    except RuntimeError as e:                              # capture refused: report, keep going
+        out["c1_mxfp8_rowwise_1024"]["graph_error"] = str(e)[:200]
     del x1, xs, qs
 
     # a7: dequantise the config-2 weight (MXFP4 and NVFP4), tcgen05 scales, 8 rotating copies
@@ -455,7 +477,7 @@ def run_breakdown(mx, dev, pk):
     # NVFP4 (two passes; the maximum pass's re-read is not counted) and MXFP4; tcgen05 scales
     R, C = 16384, 14336
     xg = to_dev(synth.normal(R, C, sigma=1e-3, seed=70), dev)
-    rnd = torch.randint(0, 256, (R * C,), dtype=torch.uint8, device=dev)
+    rnd = torch.from_numpy(np.random.default_rng(71).integers(0, 256, R * C, dtype=np.uint8)).to(dev)
     for name, f, B in (("next_train_nvfp4_rht_sr_16384x14336", L.MX_FMT_NVFP4, 16),
                        ("next_train_mxfp4_rht_sr_16384x14336", L.MX_FMT_E2M1, 32)):
         el = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
@@ -588,6 +610,31 @@ def run_case(name, iters, dev):
                         "floor" if bfmt == "e2m1" else "ceil", layout="tcgen05")
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         fns = [lambda: mx.gemm(a, b, c)]
+    elif name == "next_rows":
+        # one call of each next-row kernel: training quantiser (NVFP4 and MXFP4, RHT + SR) on an
+        # 8192 x 14336 gradient, nested conversion, MXFP6 matmul, 2-D NVFP4 weight blocks
+        from microscaling_precision_number_b200 import _lib as L
+        xg = to_dev(synth.normal(8192, 14336, sigma=1e-3, seed=70), dev)
+        rnd = torch.from_numpy(np.random.default_rng(71).integers(0, 256, xg.numel(), dtype=np.uint8)).to(dev)
+        xw = to_dev(synth.normal(14336, 4096, sigma=0.02, seed=51), dev)
+        qw = mx.quantize(xw, "e2m1", "row", "floor", layout="rowmajor")
+        o8 = torch.empty(xw.numel(), dtype=torch.uint8, device=dev)
+        bsc = torch.empty(xw.numel() // 16384, dtype=torch.float32, device=dev)
+        bok = torch.empty(xw.numel() // 16384, dtype=torch.uint8, device=dev)
+        a6 = mx.quantize(to_dev(synth.normal(8192, 8192, seed=40), dev), "e2m3", "row", "ceil", layout="tcgen05")
+        b6 = mx.quantize(to_dev(synth.normal(8192, 8192, seed=41), dev), "e2m3", "row", "ceil", layout="tcgen05")
+        c6 = torch.empty((8192, 8192), dtype=torch.bfloat16, device=dev)
+        x2 = to_dev(synth.weight_fp4(), dev)
+        s = stream.cuda_stream
+
+        def all_rows():
+            mx.quantize_train(xg, "nvfp4", "ceil", rht_signs=0xB5C3, sr_random=rnd, layout="tcgen05", stream=stream)
+            mx.quantize_train(xg, "e2m1", "floor", rht_signs=0xB5C3, sr_random=rnd, layout="tcgen05", stream=stream)
+            L.check(L.lib.mx_mxfp4_to_fp8_blocks(qw.elems.data_ptr(), qw.scales.data_ptr(), 14336, 4096,
+                                                 o8.data_ptr(), bsc.data_ptr(), bok.data_ptr(), s), "nested")
+            mx.gemm(a6, b6, c6, stream=stream)
+            mx.quantize_nvfp4_2d(x2, layout="tcgen05", stream=stream)
+        fns = [all_rows]
     else:
         raise SystemExit(f"unknown case {name}")
     t = timed(fns, iters, stream)
@@ -596,7 +643,7 @@ def run_case(name, iters, dev):
 
 
 CASES = ["weight4096", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "gemm8192", "gemm_w4a8",
-         "gemm_mxfp4_8192", "gemm_nvfp4_8192"]
+         "gemm_mxfp4_8192", "gemm_nvfp4_8192", "next_rows"]
 
 
 def main():

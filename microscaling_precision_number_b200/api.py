@@ -190,8 +190,8 @@ def cast(x: torch.Tensor, fmt="e4m3", stream=None) -> torch.Tensor:
 
 def gemm(a: Quantized, b: Quantized, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """C = A * B^T for A (M x K) and B (N x K) quantised row-wise with tcgen05 scales:
-    E4M3 x E4M3, E4M3 x E2M1, E2M1 x E2M1 or NVFP4 x NVFP4 (whose per-tensor scales are
-    applied to the fp32 sum)."""
+    FP8 / FP6 (E4M3, E5M2, E2M3, E3M2) x FP8 / FP6 / E2M1, E2M1 x E2M1, or NVFP4 x NVFP4
+    (whose per-tensor scales are applied to the fp32 sum)."""
     M, K = a.rows, a.cols
     N = b.rows
     if b.cols != K:

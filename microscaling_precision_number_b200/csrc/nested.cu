@@ -14,6 +14,15 @@
 // dec(q) * 2^(s_tile - s_max + 6); the block is flagged exact when every element decodes
 // back to its FP4 value (a tile scale at most 14 binades below s_max always is).  NaN tiles
 // give E4M3 NaN codes.  One CTA per block, one thread per 64-element half row (two tiles).
+//
+// Exactness without a round trip: with d = s_tile - s_max + 6 <= 6 a nonzero product
+// v * 2^d (v = k / 2, k in {1, 2, 3, 4, 6, 8, 12}) stays within 384, so it is an E4M3
+// value iff it is a multiple of E4M3's smallest subnormal 2^-9, i.e. iff d + 8 + tz(k) >= 0
+// (tz: trailing zero bits).  Every code is therefore exact for d >= -8; at d = -9 the
+// magnitudes 0.5 and 1.5 (E2M1 magnitude codes 1, 3) fail, at -10 also 1 and 3 (codes 2,
+// 5), at -11 everything but 4 (code 6), and below -11 every nonzero code.  Those sets are
+// tested on the packed codes with bit operations (b0, b1, b2: the magnitude bits of every
+// nibble).
 #include "codec.cuh"
 #include "internal.h"
 
@@ -23,6 +32,24 @@ namespace {
 constexpr int kNestThreads = 256;
 constexpr int kNoScale = -100000;
 }  // namespace
+
+// Whether the 32 codes of a tile (four words) all survive the move to the E4M3 grid at
+// exponent offset d (rule above).
+__device__ __forceinline__ bool tile_exact(int d, const uint32_t *w) {
+    if (d >= -8) return true;
+    uint32_t bad = 0u;
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+        const uint32_t b0 = w[k] & 0x11111111u, b1 = (w[k] >> 1) & 0x11111111u, b2 = (w[k] >> 2) & 0x11111111u;
+        uint32_t f;
+        if (d == -9) f = b0 & ~b2;                                        // magnitudes 1, 3
+        else if (d == -10) f = (~b2 & (b0 | b1)) | (b2 & b0 & ~b1);      // 1, 2, 3, 5
+        else if (d == -11) f = (b0 | b1 | b2) & ~(~b0 & b1 & b2);         // all nonzero but 6
+        else f = b0 | b1 | b2;                                            // every nonzero code
+        bad |= f;
+    }
+    return bad == 0u;
+}
 
 __global__ void __launch_bounds__(kNestThreads)
 mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restrict__ scales, int64_t cols,
@@ -63,6 +90,7 @@ mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__r
 #pragma unroll
     for (int t = 0; t < 2; t++) {
         const int d = (int)sc[t] - 127 - smax + 6;                // tile exponent relative to S
+        exact = exact && (sc[t] == 0xFFu || tile_exact(d, &w[4 * t]));
         // 2^d as fp32 (0 below 2^-149, where every product encodes to 0 anyway; capped at
         // 2^126, reached only by tiles whose codes are all zero)
         const int dc = d > 126 ? 126 : d;
@@ -75,19 +103,6 @@ mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__r
 #pragma unroll
             for (int i = 0; i < 8; i++) y[i] = __fmul_rn(y[i], f);
             const uint2 q = cvt_fp8x8<FMT_E4M3>(y);
-            // exact iff every code decodes back to its FP4 value
-            float b[8];
-            fp8x2_to_f32<FMT_E4M3>(q.x & 0xFFFFu, b[0], b[1]);
-            fp8x2_to_f32<FMT_E4M3>(q.x >> 16, b[2], b[3]);
-            fp8x2_to_f32<FMT_E4M3>(q.y & 0xFFFFu, b[4], b[5]);
-            fp8x2_to_f32<FMT_E4M3>(q.y >> 16, b[6], b[7]);
-            // From 2^-126 down the products are exact fp32 values and the round trip decides;
-            // below, every nonzero FP4 value lies under E4M3's smallest step: exact only if
-            // the codes are all zero.
-            const bool zero_word = (w[4 * t + k] & 0x77777777u) == 0u;
-#pragma unroll
-            for (int i = 0; i < 8; i++)
-                exact = exact && (sc[t] == 0xFFu || (d >= -126 ? b[i] == y[i] : zero_word));
             o[8 * t + 2 * k] = sc[t] == 0xFFu ? 0x7F7F7F7Fu : q.x;    // NaN tile: E4M3 NaN
             o[8 * t + 2 * k + 1] = sc[t] == 0xFFu ? 0x7F7F7F7Fu : q.y;
         }

@@ -436,34 +436,46 @@ nvfp4_quant_bulk_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fast
 
 // ---------------------------------------------------------------------------------------
 // NVFP4 with 16 x 16 weight blocks (two-dimensional block scaling for weights, the 4-bit
-// pre-training recipe): second pass after nvfp4_amax_bulk_kernel.  One thread per 16 x 16
-// block; lanes of a warp take neighbouring blocks, so each row of 16 blocks is one
-// coalesced 1 KiB read.  The block maximum covers 256 entries; every other step is the
-// 1 x 16 path's (same fp32 operations in the same order), and the scale is written to the
-// 16 rows of the block in the 1 x 16 layouts.
+// pre-training recipe): second pass after nvfp4_amax_bulk_kernel.  A warp takes a strip of
+// 16 horizontally adjacent blocks (16 rows x 256 columns): lane = (row parity, block), so
+// every load and store instruction covers one or two whole 512-byte row segments (codes:
+// 128 bytes, scales: 16 bytes per row).  Each lane holds its block's 8 rows of one parity
+// in registers; the block maximum is its own maximum and its partner lane's (xor 16).
+// Every other step is the 1 x 16 path's (same fp32 operations in the same order), and the
+// block scale is written to each of the block's 16 rows in the 1 x 16 layouts.
 // ---------------------------------------------------------------------------------------
 template <bool RM, bool TC>
-__global__ void __launch_bounds__(kThreads)
-nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t n_blocks, FastDiv div_bc,
+__global__ void __launch_bounds__(kThreads, 2)
+nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t rows, FastDiv div_strips,
                       uint32_t col_atoms, const float *__restrict__ partials, int n_partials,
                       float *__restrict__ g_out, uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm,
                       uint8_t *__restrict__ sc_tc) {
-    pdl_wait_and_release();
     __shared__ float warp_max[kThreads / 32];
     __shared__ float rtab[128];
+    pdl_wait_and_release();
     const float g = nvfp4_global_scale(partials, n_partials, warp_max);
     if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
     const Nvfp4Consts cst = nvfp4_consts(g, rtab);
-    const uint32_t S = cols / 16;                                  // scale columns per row
-    for (uint32_t b = blockIdx.x * kThreads + threadIdx.x; b < n_blocks; b += gridDim.x * kThreads) {
-        const uint32_t rb = fdiv(b, div_bc), cb = b - rb * div_bc.d;
-        const uint8_t *base = src + ((size_t)rb * 16 * cols + (size_t)cb * 16) * 2;
-        uint32_t m = 0;
-#pragma unroll 4
-        for (int rr = 0; rr < 16; rr++) {
-            const uint4 *p = reinterpret_cast<const uint4 *>(base + (size_t)rr * cols * 2);
-            m = max(m, absmax_block16(p[0], p[1]));
+    const uint32_t lane = threadIdx.x & 31, par = lane >> 4, c = lane & 15;
+    const uint32_t S = cols / 16;                                  // blocks (scale columns) per row
+    const uint32_t n_tasks = (rows / 16) * div_strips.d;
+    const uint32_t warps = gridDim.x * (kThreads / 32);
+    // the loop bound is uniform over the warp, so the full-warp shuffle is safe
+    for (uint32_t task = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5); task < n_tasks; task += warps) {
+        const uint32_t rb = fdiv(task, div_strips), cb = (task - rb * div_strips.d) * 16 + c;
+        const bool valid = cb < S;
+        uint4 v[8][2];
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            const uint32_t row = rb * 16 + 2 * k + par;
+            const uint4 *p = reinterpret_cast<const uint4 *>(src + ((size_t)row * cols + (size_t)cb * 16) * 2);
+            v[k][0] = valid ? p[0] : make_uint4(0u, 0u, 0u, 0u);
+            v[k][1] = valid ? p[1] : make_uint4(0u, 0u, 0u, 0u);
         }
+        uint32_t m = 0;
+#pragma unroll
+        for (int k = 0; k < 8; k++) m = max(m, absmax_block16(v[k][0], v[k][1]));
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
         const bool special = m >= 0x7F80u;                         // Inf/NaN in the block
         const float a = __uint_as_float(m << 16);
         float tq;
@@ -478,25 +490,25 @@ nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t n
         const bool zero_codes = special || r == 0.0f;
         if (special) sb = 0x7Fu;
         const uint64_t r2 = splat2(r);
-#pragma unroll 4
-        for (int rr = 0; rr < 16; rr++) {
-            const uint4 *p = reinterpret_cast<const uint4 *>(base + (size_t)rr * cols * 2);
+        if (!valid) continue;
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
             uint32_t q[2];
 #pragma unroll
             for (int j = 0; j < 2; j++) {
-                const uint4 v = p[j];
+                const uint4 u = v[k][j];
                 float x[8];
-                scale8(v, r2, x);
+                scale8(u, r2, x);
                 if (__builtin_expect(isinf(r), 0)) {
-                    const float in[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                                         bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+                    const float in[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
+                                         bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
 #pragma unroll
                     for (int i = 0; i < 8; i++)
                         if (x[i] != x[i]) x[i] = in[i];            // 0 * Inf: keep the signed zero
                 }
                 q[j] = zero_codes ? 0u : cvt_e2m1x8(x);
             }
-            const uint32_t row = rb * 16 + rr;
+            const uint32_t row = rb * 16 + 2 * k + par;
             reinterpret_cast<uint2 *>(elems)[((size_t)row * cols + (size_t)cb * 16) >> 4] = make_uint2(q[0], q[1]);
             if constexpr (RM) sc_rm[(size_t)row * S + cb] = (uint8_t)sb;
             if constexpr (TC) sc_tc[tc_offset(row, cb, col_atoms)] = (uint8_t)sb;
@@ -668,7 +680,21 @@ constexpr size_t kStreamSmem = (size_t)kStages * kTileBytes + 128;
 // until that kernel has completed.  The shared-memory attribute is set once per device and
 // kernel.
 template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl_smem(void (*kernel)(KArgs...), int grid, size_t smem, cudaStream_t st, Args... args);
+
+template <typename... KArgs, typename... Args>
 static cudaError_t launch_stream(void (*kernel)(KArgs...), int grid, cudaStream_t st, Args... args) {
+    return launch_pdl_smem(kernel, grid, kStreamSmem, st, args...);
+}
+
+// As launch_stream, for kernels without the tile ring (no dynamic shared memory).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_direct(void (*kernel)(KArgs...), int grid, cudaStream_t st, Args... args) {
+    return launch_pdl_smem(kernel, grid, 0, st, args...);
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl_smem(void (*kernel)(KArgs...), int grid, size_t smem, cudaStream_t st, Args... args) {
     static std::mutex mu;
     static std::set<std::pair<int, const void *>> configured;
     int dev = 0;
@@ -677,8 +703,8 @@ static cudaError_t launch_stream(void (*kernel)(KArgs...), int grid, cudaStream_
     {
         std::lock_guard<std::mutex> lock(mu);
         const auto key = std::make_pair(dev, reinterpret_cast<const void *>(kernel));
-        if (!configured.count(key)) {
-            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
+        if (smem > 0 && !configured.count(key)) {
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
             if (e != cudaSuccess) return e;
             configured.insert(key);
         }
@@ -686,7 +712,7 @@ static cudaError_t launch_stream(void (*kernel)(KArgs...), int grid, cudaStream_
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kStreamSmem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -766,11 +792,13 @@ static cudaError_t launch_nvfp4_2d_t(const uint8_t *src, int64_t rows, int64_t c
     if (grid > max_partials) grid = max_partials;
     cudaError_t e = launch_stream(nvfp4_amax_bulk_kernel, grid, st, src, nbytes, partials, wd);
     if (e != cudaSuccess) return e;
-    const uint32_t bc = (uint32_t)(cols / 16), n_blocks = (uint32_t)(rows / 16) * bc;
-    int grid2 = (int)((n_blocks + kThreads - 1) / kThreads);
-    if (grid2 > kCtasPerSm * num_sms) grid2 = kCtasPerSm * num_sms;
-    return launch_stream(nvfp4_2d_quant_kernel<RM, TC>, grid2, st, src, (uint32_t)cols, n_blocks, make_fastdiv(bc),
-                         (bc + 3) / 4, (const float *)partials, grid, g, elems, rm, tc);
+    // a warp per strip of 16 blocks (16 x 256 elements); 2 CTAs of 8 warps per SM
+    const uint32_t bc = (uint32_t)(cols / 16), strips = (bc + 15) / 16;
+    const uint32_t n_tasks = (uint32_t)(rows / 16) * strips;
+    int grid2 = (int)((n_tasks + kThreads / 32 - 1) / (kThreads / 32));
+    if (grid2 > 2 * num_sms) grid2 = 2 * num_sms;
+    return launch_direct(nvfp4_2d_quant_kernel<RM, TC>, grid2, st, src, (uint32_t)cols, (uint32_t)rows,
+                         make_fastdiv(strips), (bc + 3) / 4, (const float *)partials, grid, g, elems, rm, tc);
 }
 
 cudaError_t launch_stream_nvfp4_2d(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,

@@ -31,26 +31,60 @@ constexpr int kTrainThreads = 256;
 }  // namespace
 
 // ---- 16 x 16 random Hadamard transform of 16 bf16 (two uint4, element order) ---------------
-__device__ __forceinline__ void rht16(uint4 &v0, uint4 &v1, uint32_t signs) {
-    float v[16] = {bf16_lo(v0.x), bf16_hi(v0.x), bf16_lo(v0.y), bf16_hi(v0.y),
-                   bf16_lo(v0.z), bf16_hi(v0.z), bf16_lo(v0.w), bf16_hi(v0.w),
-                   bf16_lo(v1.x), bf16_hi(v1.x), bf16_lo(v1.y), bf16_hi(v1.y),
-                   bf16_lo(v1.z), bf16_hi(v1.z), bf16_lo(v1.w), bf16_hi(v1.w)};
+// D's sign flips as xor masks on the packed bf16 words (bit 15 / 31 of word i of the
+// first or second uint4 flips element 2i / 2i + 1 of that half), computed once per thread.
+struct RhtSigns {
+    uint32_t w[8];
+};
+__device__ __forceinline__ RhtSigns rht_signs(uint32_t signs) {
+    RhtSigns m;
 #pragma unroll
-    for (int i = 0; i < 16; i++)
-        if ((signs >> i) & 1u) v[i] = -v[i];
+    for (int i = 0; i < 8; i++)
+        m.w[i] = (((signs >> (2 * i)) & 1u) << 15) | (((signs >> (2 * i + 1)) & 1u) << 31);
+    return m;
+}
+
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// The butterfly stages with strides 1, 2 and 4 run on packed pairs P[j] = (v[j], v[j + 8]):
+// both lanes of P[j] +- P[j + h] are stride-h butterflies, so each packed add / sub does two
+// of them with the scalar rounding.  The stride-8 stage pairs the two lanes of one register
+// and runs in scalar; then x 1/4 (exact) and the bf16 rounding.
+__device__ __forceinline__ void rht16(uint4 &v0, uint4 &v1, const RhtSigns &sm) {
+    const uint32_t a[4] = {v0.x ^ sm.w[0], v0.y ^ sm.w[1], v0.z ^ sm.w[2], v0.w ^ sm.w[3]};   // elements 0-7
+    const uint32_t b[4] = {v1.x ^ sm.w[4], v1.y ^ sm.w[5], v1.z ^ sm.w[6], v1.w ^ sm.w[7]};   // elements 8-15
+    uint64_t P[8];
 #pragma unroll
-    for (int h = 1; h < 16; h <<= 1)
+    for (int i = 0; i < 4; i++) {
+        P[2 * i] = pack2(bf16_lo(a[i]), bf16_lo(b[i]));
+        P[2 * i + 1] = pack2(bf16_hi(a[i]), bf16_hi(b[i]));
+    }
 #pragma unroll
-        for (int i = 0; i < 16; i += 2 * h)
+    for (int h = 1; h < 8; h <<= 1)
 #pragma unroll
-            for (int j = i; j < i + h; j++) {
-                const float a = v[j], b = v[j + h];
-                v[j] = __fadd_rn(a, b);
-                v[j + h] = __fsub_rn(a, b);
+        for (int j = 0; j < 8; j++)
+            if ((j & h) == 0) {
+                const uint64_t t = P[j];
+                P[j] = add2(t, P[j + h]);
+                P[j + h] = sub2(t, P[j + h]);
             }
+    float v[16];
 #pragma unroll
-    for (int i = 0; i < 16; i++) v[i] = __fmul_rn(v[i], 0.25f);
+    for (int j = 0; j < 8; j++) {
+        float lo, hi;
+        unpack2(P[j], lo, hi);
+        v[j] = __fmul_rn(__fadd_rn(lo, hi), 0.25f);
+        v[j + 8] = __fmul_rn(__fsub_rn(lo, hi), 0.25f);
+    }
     v0 = make_uint4(f32x2_to_bf16x2(v[0], v[1]), f32x2_to_bf16x2(v[2], v[3]), f32x2_to_bf16x2(v[4], v[5]),
                     f32x2_to_bf16x2(v[6], v[7]));
     v1 = make_uint4(f32x2_to_bf16x2(v[8], v[9]), f32x2_to_bf16x2(v[10], v[11]), f32x2_to_bf16x2(v[12], v[13]),
@@ -59,25 +93,24 @@ __device__ __forceinline__ void rht16(uint4 &v0, uint4 &v1, uint32_t signs) {
 
 // ---- stochastic rounding onto the element grid ----------------------------------------------
 // Returns the representable value (lo or hi, signed) that y rounds to with random byte r.
+// Branch-free: E = max(floor(log2 |y|), emin) is the binade whose grid step 2^(E - mbits)
+// applies (the format's subnormal step below its smallest normal exponent emin; fp32
+// subnormals and zero give emin); u = |y| 2^(mbits - E) is exact and counts grid steps, so
+// lo = trunc(u) steps and the fraction f = u - trunc(u) is exact, and y rounds up iff
+// 256 f > r -- the same test as 256 (|y| - lo) > r (hi - lo).
 template <int FMT>
 __device__ __forceinline__ float sr_value(float y, uint32_t r) {
     constexpr int mbits = FMT == FMT_E4M3 ? 3 : (FMT == FMT_E5M2 ? 2 : 1);
     constexpr int emin = FMT == FMT_E4M3 ? -6 : (FMT == FMT_E5M2 ? -14 : 0);   // smallest normal exponent
     constexpr float maxv = FMT == FMT_E4M3 ? 448.0f : (FMT == FMT_E5M2 ? 57344.0f : 6.0f);
     const float a = fabsf(y);
-    if (!(a < maxv)) return copysignf(maxv, y);
-    const int eb = (int)(__float_as_uint(a) >> 23) - 127;
-    float lo, step;
-    if (eb < emin) {                                              // the format's subnormal grid
-        step = __uint_as_float((uint32_t)(emin - mbits + 127) << 23);
-        lo = __fmul_rn(floorf(__fmul_rn(a, __uint_as_float((uint32_t)(mbits - emin + 127) << 23))), step);
-    } else {                                                      // truncate to mbits mantissa bits
-        lo = __uint_as_float(__float_as_uint(a) & ~((1u << (23 - mbits)) - 1u));
-        step = __uint_as_float((uint32_t)(eb - mbits + 127) << 23);
-    }
-    if (a == lo) return y;
-    const bool up = __fmul_rn(__fsub_rn(a, lo), 256.0f) > __fmul_rn((float)r, step);
-    return copysignf(up ? __fadd_rn(lo, step) : lo, y);
+    const int E = max((int)(__float_as_uint(a) >> 23) - 127, emin);
+    const uint32_t k = (uint32_t)(E - mbits + 127);                // biased exponent of the step
+    const float u = __fmul_rn(a, __uint_as_float((254u - k) << 23)); // |y| / step (exact)
+    const float fl = truncf(u);
+    const bool up = __fmul_rn(__fsub_rn(u, fl), 256.0f) > (float)r;
+    const float v = __fmul_rn(up ? __fadd_rn(fl, 1.0f) : fl, __uint_as_float(k << 23));
+    return copysignf(a < maxv ? v : maxv, y);                      // at or above the maximum: saturate
 }
 
 template <int FMT, bool SR>
@@ -97,12 +130,13 @@ mx_train_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS
                 uint32_t signs, const uint8_t *__restrict__ rnd, uint8_t *__restrict__ elems,
                 uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
+    const RhtSigns sm = rht_signs(signs);
     for (uint32_t blk = blockIdx.x * kTrainThreads + threadIdx.x; blk < n_blocks; blk += gridDim.x * kTrainThreads) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)blk * 64);
         uint4 v[4] = {p[0], p[1], p[2], p[3]};
         if constexpr (RHT) {
-            rht16(v[0], v[1], signs);
-            rht16(v[2], v[3], signs);
+            rht16(v[0], v[1], sm);
+            rht16(v[2], v[3], sm);
         }
         uint32_t a = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v[0].x, v[0].y), absmax_bf16x2(v[0].z, v[0].w)),
                                    absmax_bf16x2(absmax_bf16x2(v[1].x, v[1].y), absmax_bf16x2(v[1].z, v[1].w)));
@@ -141,10 +175,11 @@ nvfp4_train_amax_kernel(const uint8_t *__restrict__ src, uint32_t n_groups, uint
     asm volatile("griddepcontrol.wait;" ::: "memory");
     __shared__ uint32_t warp_u[kTrainThreads / 32];
     uint32_t acc = 0;
+    const RhtSigns sm = rht_signs(signs);
     for (uint32_t gi = blockIdx.x * kTrainThreads + threadIdx.x; gi < n_groups; gi += gridDim.x * kTrainThreads) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)gi * 32);
         uint4 v0 = p[0], v1 = p[1];
-        if constexpr (RHT) rht16(v0, v1, signs);
+        if constexpr (RHT) rht16(v0, v1, sm);
         acc = __vmaxu2(acc, finite_abs_max_bf16x8(v0));
         acc = __vmaxu2(acc, finite_abs_max_bf16x8(v1));
     }
@@ -183,10 +218,11 @@ nvfp4_train_quant_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fas
     const float g = a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f);
     if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
     const float six_g = __fmul_rn(6.0f, g);
+    const RhtSigns sm = rht_signs(signs);
     for (uint32_t blk = blockIdx.x * kTrainThreads + threadIdx.x; blk < n_blocks; blk += gridDim.x * kTrainThreads) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)blk * 32);
         uint4 v[2] = {p[0], p[1]};
-        if constexpr (RHT) rht16(v[0], v[1], signs);
+        if constexpr (RHT) rht16(v[0], v[1], sm);
         const uint32_t am = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v[0].x, v[0].y), absmax_bf16x2(v[0].z, v[0].w)),
                                           absmax_bf16x2(absmax_bf16x2(v[1].x, v[1].y), absmax_bf16x2(v[1].z, v[1].w)));
         const uint32_t m = max(am & 0x7FFFu, (am >> 16) & 0x7FFFu);

@@ -76,6 +76,26 @@ def test_scale_gap_edges(oracle, gap, low):
     check(oracle, e, s, 128, 256)
 
 
+def test_single_tile_offsets_and_magnitudes(oracle):
+    """One 128 x 128 block per (tile offset d, E2M1 magnitude): every other tile of the block
+    sits at d >= -8 (always exact) and one tile holds a single code of the given magnitude
+    at d in -8 .. -13, so the block flag is that code's exactness alone -- the boundary
+    cases of the kernel's closed-form rule against the oracle's round trip."""
+    offsets, mags = list(range(-8, -14, -1)), list(range(1, 8))
+    cases = [(d, m, sign) for d in offsets for m in mags for sign in (0, 8)]
+    rows, cols = 128, 128 * len(cases)
+    e = np.zeros((rows, cols // 2), dtype=np.uint8)
+    s = np.full((rows, cols // 32), 127, dtype=np.uint8)          # tile exponent 0
+    for j, (d, m, sign) in enumerate(cases):
+        e[0, 64 * j] = 0x07                                       # 6.0 * 2^0: s_max = 0
+        s[7, 4 * j + 2] = 127 + d - 6                             # tile exponent d - 6: offset d
+        e[7, 64 * j + 32] = (m | sign) << 4                       # its second code (odd index)
+    _, _, ok = check(oracle, e, s, rows, cols)
+    flags = {c: int(f) for c, f in zip(cases, ok.reshape(-1))}
+    assert flags[(-8, 1, 0)] == 1 and flags[(-9, 1, 0)] == 0 and flags[(-9, 2, 8)] == 1
+    assert flags[(-11, 6, 0)] == 1 and flags[(-11, 7, 0)] == 0 and flags[(-12, 6, 0)] == 0
+
+
 def test_config5_weight(oracle):
     """The mixed-GEMM weight shape (14336 x 4096, N(0, 0.02)) end to end."""
     x = synth.normal(14336, 4096, sigma=0.02, seed=51)

@@ -283,6 +283,31 @@ def test_nvfp4_multi_cta_matches_oracle(oracle, shape):
     assert np.array_equal(host(q.scales_alt), oracle.to_tcgen05_layout(s))
 
 
+@pytest.mark.parametrize("offset", [1, 2, 3])
+def test_nvfp4_unaligned_scale_buffers(oracle, offset):
+    """Scale buffers at byte offsets 1-3 (no 4-byte vector stores possible): same bytes as
+    the oracle, and nothing written outside the buffers."""
+    rows, cols = 96, 512
+    x = synth.weight_fp4(rows, cols, seed=offset)
+    e, s, g = oracle.quantize_nvfp4(x)
+    src = to_dev(x)
+    elems = torch.empty(rows * cols // 2, dtype=torch.uint8, device="cuda")
+    n_rm, n_tc = rows * cols // 16, mx.scale_bytes(rows, cols // 16, "tcgen05")
+    rm = torch.full((n_rm + 8,), 0xA5, dtype=torch.uint8, device="cuda")
+    tc = torch.full((n_tc + 8,), 0xA5, dtype=torch.uint8, device="cuda")
+    gs = torch.empty(1, dtype=torch.float32, device="cuda")
+    st = L.lib.mx_quantize(src.data_ptr(), rows, cols, L.MX_FMT_NVFP4, L.MX_AXIS_ROW, L.MX_SCALE_CEIL_RECIPE,
+                           elems.data_ptr(), rm.data_ptr() + offset, 3, tc.data_ptr() + offset, gs.data_ptr(),
+                           torch.cuda.current_stream().cuda_stream)
+    assert st == L.MX_OK
+    assert np.array_equal(host(elems), e.reshape(-1))
+    rm_h, tc_h = host(rm), host(tc)
+    assert np.array_equal(rm_h[offset:offset + n_rm], s.reshape(-1))
+    assert np.array_equal(tc_h[offset:offset + n_tc], oracle.to_tcgen05_layout(s))
+    assert np.all(rm_h[:offset] == 0xA5) and np.all(rm_h[offset + n_rm:] == 0xA5)
+    assert np.all(tc_h[:offset] == 0xA5) and np.all(tc_h[offset + n_tc:] == 0xA5)
+
+
 @pytest.mark.parametrize("sigma_log2", [-60, -72, -78, -84, -95, -110])
 def test_nvfp4_tiny_tensor_scales(oracle, sigma_log2):
     """Tensors whose per-tensor scale puts 6g on either side of 2^-80 (where the block
