@@ -219,16 +219,10 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             const bool ok = mbar_wait_bounded(&acc_full, (uint32_t)i & 1u, watchdog, WD_GEMM_ACC);
             if (!ok || *fail_sh) { *fail_sh = 1; break; }
             tc_fence_after();
-            uint32_t o[kHalf / 2];                        // the thread's row segment as bf16 pairs
-#pragma unroll
-            for (int j = 0; j < kHalf / 32; j++) {
-                uint32_t r[32];
-                tmem_ld32(t_base + j * 32, r);
-#pragma unroll
-                for (int q = 0; q < 16; q++)
-                    o[j * 16 + q] = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(r[2 * q]), alpha),
-                                                    __fmul_rn(__uint_as_float(r[2 * q + 1]), alpha));
-            }
+            // the whole row segment comes out of tensor memory first (one wait), so the
+            // accumulator is released before the conversion and the stores
+            uint32_t r[kHalf / 32][32];
+            tmem_ld32_batch<kHalf / 32>(t_base, r);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty);       // accumulator may be overwritten now
@@ -238,7 +232,16 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             uint4 *dst = reinterpret_cast<uint4 *>(C + (int64_t)row * N + (int64_t)n_blk * BN + half * kHalf);
             // evict-first stores: the output must not push operand panels out of L2
 #pragma unroll
-            for (int q = 0; q < kHalf / 8; q++) __stcs(dst + q, make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]));
+            for (int j = 0; j < kHalf / 32; j++)
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; e++)
+                        o[e] = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(r[j][8 * q + 2 * e]), alpha),
+                                               __fmul_rn(__uint_as_float(r[j][8 * q + 2 * e + 1]), alpha));
+                    __stcs(dst + 4 * j + q, make_uint4(o[0], o[1], o[2], o[3]));
+                }
         }
     }
 

@@ -138,17 +138,28 @@ __device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint32_t saddr) {
         asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
+// NJ loads of 32 columns (columns taddr + 32 j) issued back to back with one wait for all
+// of them.  The empty asm statements after the wait tie every loaded register to it, so no
+// use of r can be scheduled before the data has landed.
+template <int NJ>
+__device__ __forceinline__ void tmem_ld32_batch(uint32_t taddr, uint32_t (&r)[NJ][32]) {
+#pragma unroll
+    for (int j = 0; j < NJ; j++)
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+            "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+            "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+            : "=r"(r[j][0]), "=r"(r[j][1]), "=r"(r[j][2]), "=r"(r[j][3]), "=r"(r[j][4]), "=r"(r[j][5]),
+              "=r"(r[j][6]), "=r"(r[j][7]), "=r"(r[j][8]), "=r"(r[j][9]), "=r"(r[j][10]), "=r"(r[j][11]),
+              "=r"(r[j][12]), "=r"(r[j][13]), "=r"(r[j][14]), "=r"(r[j][15]), "=r"(r[j][16]), "=r"(r[j][17]),
+              "=r"(r[j][18]), "=r"(r[j][19]), "=r"(r[j][20]), "=r"(r[j][21]), "=r"(r[j][22]), "=r"(r[j][23]),
+              "=r"(r[j][24]), "=r"(r[j][25]), "=r"(r[j][26]), "=r"(r[j][27]), "=r"(r[j][28]), "=r"(r[j][29]),
+              "=r"(r[j][30]), "=r"(r[j][31])
+            : "r"(taddr + 32u * (uint32_t)j));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < NJ; j++)
+        asm volatile("" : "+r"(r[j][0]), "+r"(r[j][1]), "+r"(r[j][2]), "+r"(r[j][3]), "+r"(r[j][4]), "+r"(r[j][5]), "+r"(r[j][6]), "+r"(r[j][7]), "+r"(r[j][8]), "+r"(r[j][9]), "+r"(r[j][10]), "+r"(r[j][11]), "+r"(r[j][12]), "+r"(r[j][13]), "+r"(r[j][14]), "+r"(r[j][15]), "+r"(r[j][16]), "+r"(r[j][17]), "+r"(r[j][18]), "+r"(r[j][19]), "+r"(r[j][20]), "+r"(r[j][21]), "+r"(r[j][22]), "+r"(r[j][23]), "+r"(r[j][24]), "+r"(r[j][25]), "+r"(r[j][26]), "+r"(r[j][27]), "+r"(r[j][28]), "+r"(r[j][29]), "+r"(r[j][30]), "+r"(r[j][31]));
 }
 
 // ---- tile order ------------------------------------------------------------------------------
