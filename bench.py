@@ -111,8 +111,17 @@ class ClockSampler:
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+               "samples": len(sm)}
+        pw = []
+        for ln in getattr(self, "lines", []):
+            try:
+                pw.append(float(ln.split(",")[3]))
+            except (ValueError, IndexError):
+                pass
+        if pw:
+            out["power_w_max"] = max(pw)
+        return out
 
 
 def max_over_ranks(ms, world, dev):
@@ -340,6 +349,18 @@ def best_of(fn, n, stream):
     return best
 
 
+def soak_clocks(fn, seconds=1.5):
+    """SM clock and throttle reasons while fn runs back to back for about `seconds` (the
+    sampler's short idle lead-in and tail are a minority of the samples)."""
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < seconds:
+            for _ in range(16):
+                fn()
+            torch.cuda.synchronize()
+    return clk.summary()
+
+
 def run_breakdown(mx, dev, pk):
     stream = torch.cuda.current_stream()
     out = {}
@@ -427,6 +448,7 @@ def run_breakdown(mx, dev, pk):
         tb = best_of(lambda: mx.gemm(a, b, c), 10, stream)
         tf, tfb = (2.0 * M * N * K / (x * 1e-3) / 1e12 for x in (t, tb))
         out[name] = {"ms": round(t, 4), "TFLOPS": round(tf, 1), "frac_mx_peak_measured": round(tf / mx_peak, 4),
+                     "clocks_back_to_back": soak_clocks(lambda: mx.gemm(a, b, c)),
                      "best_of_10_ms": round(tb, 4), "best_of_10_TFLOPS": round(tfb, 1),
                      "frac_best_of_10_mx_peak_measured": round(tfb / mx_peak, 4),
                      "mx_peak_measured_TFLOPS": mx_peak, "frac_mx_nominal_4500": round(tf / MX_NOMINAL_TFLOPS, 4),
@@ -434,6 +456,36 @@ def run_breakdown(mx, dev, pk):
                                   "ratio; ms / TFLOPS: mean of 10 back-to-back calls"}
         del a, b, c
         torch.cuda.empty_cache()
+
+    # library comparator (not this library's path): cuBLASLt's MXFP8 block-scaled matmul via
+    # torch._scaled_mm on the same config-4 operands -- the E8M0 scales in the tcgen05
+    # tiling are the layout it takes
+    try:
+        M = N = K = 8192
+        a = mx.quantize(to_dev(synth.normal(M, K, seed=40), dev), "e4m3", "row", "ceil", layout="tcgen05")
+        b = mx.quantize(to_dev(synth.normal(N, K, seed=41), dev), "e4m3", "row", "ceil", layout="tcgen05")
+        af = a.elems.view(torch.float8_e4m3fn).view(M, K)
+        bf = b.elems.view(torch.float8_e4m3fn).view(N, K)
+        sa = a.scales.view(torch.float8_e8m0fnu)
+        sb = b.scales.view(torch.float8_e8m0fnu)
+
+        def lib():
+            return torch._scaled_mm(af, bf.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16)
+        ref = lib()
+        ours = mx.gemm(a, b)
+        rel = ((ref.float() - ours.float()).abs().max() / ours.float().abs().max()).item()
+        t = timed([lib], 10, stream)
+        tb = best_of(lib, 10, stream)
+        tf, tfb = (2.0 * M * N * K / (x * 1e-3) / 1e12 for x in (t, tb))
+        out["lib_cublaslt_mxfp8_8192_comparator"] = {
+            "ms": round(t, 4), "TFLOPS": round(tf, 1), "best_of_10_TFLOPS": round(tfb, 1),
+            "frac_mx_peak_measured": round(tf / mx_peak, 4), "max_abs_diff_vs_ours_rel_to_max": rel,
+            "clocks_back_to_back": soak_clocks(lib),
+            "note": "torch._scaled_mm (cuBLASLt) on the same operands: a comparator, not this library's path"}
+        del a, b, af, bf, sa, sb, ref, ours
+    except Exception as e:                                   # comparator unavailable: say why
+        out["lib_cublaslt_mxfp8_8192_comparator"] = {"unavailable": str(e)[:200]}
+    torch.cuda.empty_cache()
 
     # next row: FP4 x FP4 block-scaled matmuls (kind::mxf4 and kind::mxf4nvf4), 8192^3,
     # against the dense FP4 rate (2 x the FP8 rate; 9 PFLOP/s nominal)
@@ -447,6 +499,7 @@ def run_breakdown(mx, dev, pk):
         tb = best_of(lambda: mx.gemm(a, b, c), 10, stream)
         tf, tfb = (2.0 * M * N * K / (x * 1e-3) / 1e12 for x in (t, tb))
         out[name] = {"ms": round(t, 4), "TFLOPS": round(tf, 1), "frac_fp4_peak_measured": round(tf / fp4_peak, 4),
+                     "clocks_back_to_back": soak_clocks(lambda: mx.gemm(a, b, c)),
                      "best_of_10_ms": round(tb, 4), "best_of_10_TFLOPS": round(tfb, 1),
                      "frac_best_of_10_fp4_peak_measured": round(tfb / fp4_peak, 4),
                      "fp4_peak_measured_TFLOPS": fp4_peak, "frac_fp4_nominal_9000": round(tf / (2 * MX_NOMINAL_TFLOPS), 4),
