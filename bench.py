@@ -261,36 +261,71 @@ def run_ours(args, rank, world, dev):
                           "launches_timed": ncall},
                 "frac_of_nominal_8TBps": round(achieved / HBM_NOMINAL_GBS, 4)}
 
-    # end to end through the public API with host buffers (pinned), copies inside the timing
-    step = steps[0]
-    x = step.x
+    # end to end through the public API with host buffers (pinned), copies inside the timing.
+    # Pipelined as a user would run a stream of weights: step k's upload, step k-1's
+    # quantisation and step k-2's download overlap on three streams (two buffer sets,
+    # ordered by events); the serial form (upload, quantise, download on one stream) is
+    # reported beside it.
+    sets = steps[:2]
     x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
-    outs_host = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in step.outputs()]
+    outs_host = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in st.outputs()] for st in sets]
     h2d = x_host.numel() * 2
-    d2h = sum(o.numel() * o.element_size() for o in outs_host)
+    d2h = sum(o.numel() * o.element_size() for o in outs_host[0])
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_up, ev_comp, ev_down = ([torch.cuda.Event() for _ in sets] for _ in range(3))
 
-    def e2e_step():
-        x.copy_(x_host, non_blocking=True)
-        step.mxfp4(sptr)
-        step.nvfp4(sptr)
-        for h, d in zip(outs_host, step.outputs()):
-            h.copy_(d, non_blocking=True)
+    def pipelined(n):
+        for k in range(n):
+            b = k % 2
+            st = sets[b]
+            up.wait_event(ev_comp[b])                  # the buffer's previous step has read it
+            with torch.cuda.stream(up):
+                st.x.copy_(x_host, non_blocking=True)
+            ev_up[b].record(up)
+            stream.wait_event(ev_up[b])
+            stream.wait_event(ev_down[b])              # its previous outputs have been copied out
+            st.mxfp4(sptr)
+            st.nvfp4(sptr)
+            ev_comp[b].record(stream)
+            down.wait_event(ev_comp[b])
+            with torch.cuda.stream(down):
+                for h, d in zip(outs_host[b], st.outputs()):
+                    h.copy_(d, non_blocking=True)
+            ev_down[b].record(down)
 
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e0, e1 = event_pair()
-    if world > 1:
-        torch.distributed.barrier()
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    def serial(n):
+        st = sets[0]
+        for _ in range(n):
+            st.x.copy_(x_host, non_blocking=True)
+            st.mxfp4(sptr)
+            st.nvfp4(sptr)
+            for h, d in zip(outs_host[0], st.outputs()):
+                h.copy_(d, non_blocking=True)
+
+    def timed_e2e(run):
+        run(2)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = event_pair()
+        e0.record(stream)
+        up.wait_event(e0)
+        down.wait_event(e0)
+        run(args.steps)
+        for ev in ev_down:
+            stream.wait_event(ev)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+    e2e_ms = timed_e2e(pipelined)
+    ser_ms = timed_e2e(serial)
     e2e = {"value": round(job_throughput_gbs(STEP_BYTES, args.steps, world, e2e_ms), 2), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "ms_per_step": round(e2e_ms / args.steps, 4)}
+           "ms_per_step": round(e2e_ms / args.steps, 4),
+           "form": "pipelined: upload / quantise / download of consecutive steps overlap on three streams",
+           "serial": {"value": round(job_throughput_gbs(STEP_BYTES, args.steps, world, ser_ms), 2),
+                      "ms_per_step": round(ser_ms / args.steps, 4)}}
 
     breakdown = None
     if not args.no_breakdown and rank == 0:
@@ -685,6 +720,17 @@ def run_case(name, iters, dev):
                         "floor" if bfmt == "e2m1" else "ceil", layout="tcgen05")
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         fns = [lambda: mx.gemm(a, b, c)]
+    elif name == "gemm_cmp":
+        # config-4 operands through this library's matmul and through cuBLASLt's MXFP8
+        # matmul (torch._scaled_mm), one call each per round, for side-by-side counters
+        M = N = K = 8192
+        a = mx.quantize(to_dev(synth.normal(M, K, seed=40), dev), "e4m3", "row", "ceil", layout="tcgen05")
+        b = mx.quantize(to_dev(synth.normal(N, K, seed=41), dev), "e4m3", "row", "ceil", layout="tcgen05")
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        af, bf = a.elems.view(torch.float8_e4m3fn).view(M, K), b.elems.view(torch.float8_e4m3fn).view(N, K)
+        sa, sb = a.scales.view(torch.float8_e8m0fnu), b.scales.view(torch.float8_e8m0fnu)
+        fns = [lambda: (mx.gemm(a, b, c),
+                        torch._scaled_mm(af, bf.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16))]
     elif name == "next_rows":
         # one call of each next-row kernel: training quantiser (NVFP4 and MXFP4, RHT + SR) on an
         # 8192 x 14336 gradient, nested conversion, MXFP6 matmul, 2-D NVFP4 weight blocks
@@ -718,7 +764,7 @@ def run_case(name, iters, dev):
 
 
 CASES = ["weight4096", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "gemm8192", "gemm_w4a8",
-         "gemm_mxfp4_8192", "gemm_nvfp4_8192", "next_rows"]
+         "gemm_mxfp4_8192", "gemm_nvfp4_8192", "gemm_cmp", "next_rows"]
 
 
 def main():

@@ -146,24 +146,25 @@ __device__ __forceinline__ uint32_t finite_abs_max_bf16x8(const uint4 &v) {
 // element (the value times 64, rounded half to even, saturated to -127 .. 127).
 template <int FMT>
 __device__ __forceinline__ uint32_t cvt_fp8x2(float lo, float hi) {
-    uint16_t r;
-    if constexpr (FMT == FMT_E4M3)
-        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    else if constexpr (FMT == FMT_E5M2)
-        asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    else if constexpr (FMT == FMT_E2M3)
-        asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    else if constexpr (FMT == FMT_E3M2)
-        asm("cvt.rn.satfinite.e3m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-    else {
+    if constexpr (FMT == FMT_INT8) {
         int32_t a, b;
         asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(a) : "f"(__fmul_rn(lo, 64.0f)));
         asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(b) : "f"(__fmul_rn(hi, 64.0f)));
         a = max(a, -127);
         b = max(b, -127);
         return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8);
+    } else {
+        uint16_t r;
+        if constexpr (FMT == FMT_E4M3)
+            asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+        else if constexpr (FMT == FMT_E5M2)
+            asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+        else if constexpr (FMT == FMT_E2M3)
+            asm("cvt.rn.satfinite.e2m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+        else
+            asm("cvt.rn.satfinite.e3m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+        return (uint32_t)r;
     }
-    return (uint32_t)r;
 }
 
 // Eight fp32 -> eight E2M1 codes in one 32-bit word (element i in nibble i).
