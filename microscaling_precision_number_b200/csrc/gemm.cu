@@ -158,6 +158,18 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
+            // Everything the issue loop needs is precomputed: one thread issues every
+            // copy and MMA, and at ~4 instructions per 128 tensor cycles its own latency
+            // decides whether the tensor pipe idles.  Descriptors advance by offsets >> 4
+            // (the 14-bit start-address field never overflows inside shared memory).
+            const uint64_t a_d0 = smem_desc(smem_u32(sA), 16, 1024, 2), b_d0 = smem_desc(smem_u32(sB), 16, 1024, 2);
+            const uint64_t sfa_d0 = sf_desc(smem_u32(sSFA)), sfb_d0 = sf_desc(smem_u32(sSFB));
+            uint32_t idesc[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+                idesc[k] = mma_idesc<kBM, BN, KIND>(
+                    a_fmt_code, b_fmt_code,
+                    KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u));
             int it = 0, i = 0;
             for (int t = blockIdx.x; t < n_tiles && !*fail_sh; t += gridDim.x, i++) {
                 if (i > 0 && !mbar_wait_bounded(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
@@ -176,16 +188,17 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     // sfb_t + 4 (a (BN/128) + h), A atom a at sfa_t + 4 a
                     const uint32_t sfb_t = tmem + kSfCol0 + s * T::kSfColsPerStage;
                     const uint32_t sfa_t = sfb_t + T::kSfbCols;
+                    const uint64_t sfa_d = sfa_d0 + (uint64_t)((s * kSfaBytes) >> 4);
+                    const uint64_t sfb_d = sfb_d0 + (uint64_t)((s * kSfbBytes) >> 4);
 #pragma unroll
                     for (int a = 0; a < T::kAtoms; a++) {
-                        tc_cp_sf(sfa_t + 4 * a, smem_u32(sSFA + s * kSfaBytes + a * 512));
+                        tc_cp_sf(sfa_t + 4 * a, sfa_d + (uint64_t)(a * 512 / 16));
 #pragma unroll
                         for (int h = 0; h < BN / 128; h++)
-                            tc_cp_sf(sfb_t + 4 * (a * (BN / 128) + h),
-                                     smem_u32(sSFB + s * kSfbBytes + h * T::kSfaBytes + a * 512));
+                            tc_cp_sf(sfb_t + 4 * (a * (BN / 128) + h), sfb_d + (uint64_t)((h * T::kSfaBytes + a * 512) / 16));
                     }
-                    const uint32_t a_base = smem_u32(sA + s * kABytes);
-                    const uint32_t b_base = smem_u32(sB + s * kBBytes);
+                    const uint64_t a_d = a_d0 + (uint64_t)((s * kABytes) >> 4);
+                    const uint64_t b_d = b_d0 + (uint64_t)((s * kBBytes) >> 4);
                     // four instructions per stage, each over 32 bytes of K per row (K = 32 for
                     // 8-bit codes, 64 for packed 4-bit codes).  Instruction k reads scale atom
                     // a and, inside its 32-bit words, the scale byte(s) starting at sf_id:
@@ -193,10 +206,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
                         const int a = KIND == KIND_F8F6F4 ? 0 : (KIND == KIND_MXF4 ? k >> 1 : k);
-                        const uint32_t sf_id = KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u);
-                        const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
-                        const uint64_t bd = smem_desc(b_base + k * 32, 16, 1024, 2);
-                        tc_mma_mx<KIND>(tmem, ad, bd, mma_idesc<kBM, BN, KIND>(a_fmt_code, b_fmt_code, sf_id), sfa_t + 4 * a,
+                        tc_mma_mx<KIND>(tmem, a_d + (uint64_t)(2 * k), b_d + (uint64_t)(2 * k), idesc[k], sfa_t + 4 * a,
                                         sfb_t + 4 * a * (BN / 128), (kb > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit(&empty_bar[s]);

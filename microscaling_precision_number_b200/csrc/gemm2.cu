@@ -173,6 +173,15 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer (even CTA only)
         if (leader && lane == 0) {
+            // precomputed descriptors on the issuing thread (as in gemm.cu)
+            const uint64_t a_d0 = smem_desc(smem_u32(sA), 16, 1024, 2), b_d0 = smem_desc(smem_u32(sB), 16, 1024, 2);
+            const uint64_t sfa_d0 = sf_desc(smem_u32(sSFA)), sfb_d0 = sf_desc(smem_u32(sSFB));
+            uint32_t idesc[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+                idesc[k] = mma_idesc<kPairM, kPairN, KIND>(
+                    a_fmt_code, b_fmt_code,
+                    KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u));
             int it = 0, i = 0;
             for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs, i++) {
                 if (i > 0 && !mbar_wait_bounded(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
@@ -189,23 +198,22 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     tc_fence_after();
                     const uint32_t sfb_t = tmem + kSfCol0 + s * P::kSfColsPerStage;
                     const uint32_t sfa_t = sfb_t + P::kSfbCols;
+                    const uint64_t sfa_d = sfa_d0 + (uint64_t)((s * P::kSfaBytes) >> 4);
+                    const uint64_t sfb_d = sfb_d0 + (uint64_t)((s * P::kSfbBytes) >> 4);
 #pragma unroll
                     for (int a = 0; a < P::kAtoms; a++) {
-                        tc_cp_sf<2>(sfa_t + 4 * a, smem_u32(sSFA + s * P::kSfaBytes + a * 512));
+                        tc_cp_sf<2>(sfa_t + 4 * a, sfa_d + (uint64_t)(a * 512 / 16));
 #pragma unroll
                         for (int h = 0; h < 2; h++)
-                            tc_cp_sf<2>(sfb_t + 4 * (2 * a + h), smem_u32(sSFB + s * P::kSfbBytes + h * P::kSfaBytes + a * 512));
+                            tc_cp_sf<2>(sfb_t + 4 * (2 * a + h), sfb_d + (uint64_t)((h * P::kSfaBytes + a * 512) / 16));
                     }
-                    const uint32_t a_base = smem_u32(sA + s * kABytes);
-                    const uint32_t b_base = smem_u32(sB + s * kBBytes);
+                    const uint64_t a_d = a_d0 + (uint64_t)((s * kABytes) >> 4);
+                    const uint64_t b_d = b_d0 + (uint64_t)((s * kBBytes) >> 4);
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
                         const int a = KIND == KIND_F8F6F4 ? 0 : (KIND == KIND_MXF4 ? k >> 1 : k);
-                        const uint32_t sf_id = KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u);
-                        const uint64_t ad = smem_desc(a_base + k * 32, 16, 1024, 2);
-                        const uint64_t bd = smem_desc(b_base + k * 32, 16, 1024, 2);
-                        tc_mma_mx<KIND, 2>(tmem, ad, bd, mma_idesc<kPairM, kPairN, KIND>(a_fmt_code, b_fmt_code, sf_id),
-                                           sfa_t + 4 * a, sfb_t + 8 * a, (kb > 0 || k > 0) ? 1u : 0u);
+                        tc_mma_mx<KIND, 2>(tmem, a_d + (uint64_t)(2 * k), b_d + (uint64_t)(2 * k), idesc[k], sfa_t + 4 * a,
+                                           sfb_t + 8 * a, (kb > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit_pair(&empty_bar[s]);           // stage s free in both CTAs
                 }

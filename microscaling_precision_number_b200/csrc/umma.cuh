@@ -129,9 +129,13 @@ __device__ __forceinline__ void tc_mma_mx(uint32_t d_tmem, uint64_t adesc, uint6
 // replicated into all four 32-lane sub-partitions.
 // With CG = 2 (issued by the pair's MMA thread) each CTA's atom at the same shared-memory
 // offset goes to the same columns of that CTA's own tensor memory.
+// Shared-memory descriptor of a scale atom (512 bytes, no swizzle) at saddr.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) { return smem_desc(saddr, 16, 128, 0); }
+
+// The copy with a ready descriptor d (the MMA loops advance one base descriptor by
+// offsets >> 4 instead of rebuilding it on the issuing thread's critical path).
 template <int CG = 1>
-__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint32_t saddr) {
-    const uint64_t d = smem_desc(saddr, 16, 128, 0);
+__device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t d) {
     if constexpr (CG == 1)
         asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
     else
