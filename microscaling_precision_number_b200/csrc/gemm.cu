@@ -44,8 +44,8 @@ namespace {
 constexpr int kBM = 128, kBK = 128;                      // tile rows; bytes of K per row per stage
 constexpr int kStages = 4;
 constexpr int kEpilogueWarps = 8;                  // two per TMEM lane quadrant
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kGemmThreads = 320;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kSfWarp = 10;
+constexpr int kGemmThreads = 352;
 constexpr int kABytes = kBM * kBK;                       // 16 KiB
 constexpr uint32_t kTmemCols = 512;                      // accumulator (<= 256) + scale slots
 constexpr uint32_t kSfCol0 = 256;                        // first scale-slot column
@@ -89,7 +89,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     uint8_t *sSFA = sB + kStages * kBBytes;               // kStages x 512 B
     uint8_t *sSFB = sSFA + kStages * kSfaBytes;           // kStages x kAtoms x 512 B per 128 rows of B
 
-    __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], acc_full, acc_empty, drain_bar;
+    __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], sf_ready[kStages], acc_full, acc_empty,
+        drain_bar, sf_drain;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int fail_flag;
     volatile int *fail_sh = &fail_flag;
@@ -102,10 +103,15 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (threadIdx.x == 0) {
         prefetch_tensormap(&tmA);
         prefetch_tensormap(&tmB);
-        for (int s = 0; s < kStages; s++) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+        for (int s = 0; s < kStages; s++) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+            mbar_init(&sf_ready[s], 1);
+        }
         mbar_init(&acc_full, 1);
         mbar_init(&acc_empty, kEpilogueWarps);
         mbar_init(&drain_bar, 1);
+        mbar_init(&sf_drain, 1);
         *fail_sh = 0;
         fence_barrier_init();
     }
@@ -155,6 +161,42 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             }
         }
         __syncwarp();
+    } else if (warp == kSfWarp) {
+        // ------------------------------------------------ scale-atom copier
+        // Copies each stage's scale atoms into tensor memory as soon as the stage has
+        // landed and signals sf_ready[s] once the copies are complete; the MMA issuer waits
+        // on sf_ready alone.  This takes the copies (3 to 12 per stage) off the single
+        // MMA-issuing thread, whose instruction latency otherwise bounds the tensor pipe.
+        // A stage's scale slot is rewritten only after full[s] of its next use, i.e. after
+        // the MMAs that read it have completed (empty[s]).
+        if (lane == 0) {
+            const uint64_t sfa_d0 = sf_desc(smem_u32(sSFA)), sfb_d0 = sf_desc(smem_u32(sSFB));
+            int it = 0;
+            for (int t = blockIdx.x; t < n_tiles && !*fail_sh; t += gridDim.x) {
+                for (int kb = 0; kb < num_kb; kb++, it++) {
+                    const int s = it % kStages;
+                    if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(it / kStages) & 1u, watchdog, WD_GEMM_FULL)) {
+                        *fail_sh = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfb_t = tmem + kSfCol0 + s * T::kSfColsPerStage;
+                    const uint32_t sfa_t = sfb_t + T::kSfbCols;
+                    const uint64_t sfa_d = sfa_d0 + (uint64_t)((s * kSfaBytes) >> 4);
+                    const uint64_t sfb_d = sfb_d0 + (uint64_t)((s * kSfbBytes) >> 4);
+#pragma unroll
+                    for (int a = 0; a < T::kAtoms; a++) {
+                        tc_cp_sf(sfa_t + 4 * a, sfa_d + (uint64_t)(a * 512 / 16));
+#pragma unroll
+                        for (int h = 0; h < BN / 128; h++)
+                            tc_cp_sf(sfb_t + 4 * (a * (BN / 128) + h), sfb_d + (uint64_t)((h * T::kSfaBytes + a * 512) / 16));
+                    }
+                    tc_commit(&sf_ready[s]);                  // the stage's scales are in tensor memory
+                }
+            }
+            tc_commit(&sf_drain);                         // completes once every copy above has finished
+        }
+        __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -163,7 +205,6 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             // decides whether the tensor pipe idles.  Descriptors advance by offsets >> 4
             // (the 14-bit start-address field never overflows inside shared memory).
             const uint64_t a_d0 = smem_desc(smem_u32(sA), 16, 1024, 2), b_d0 = smem_desc(smem_u32(sB), 16, 1024, 2);
-            const uint64_t sfa_d0 = sf_desc(smem_u32(sSFA)), sfb_d0 = sf_desc(smem_u32(sSFB));
             uint32_t idesc[4];
 #pragma unroll
             for (int k = 0; k < 4; k++)
@@ -179,7 +220,8 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 tc_fence_after();
                 for (int kb = 0; kb < num_kb; kb++, it++) {
                     const int s = it % kStages;
-                    if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(it / kStages) & 1u, watchdog, WD_GEMM_FULL)) {
+                    // the stage's operands have landed and its scales are in tensor memory
+                    if (!mbar_wait_bounded(&sf_ready[s], (uint32_t)(it / kStages) & 1u, watchdog, WD_GEMM_FULL)) {
                         *fail_sh = 1;
                         break;
                     }
@@ -188,15 +230,6 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     // sfb_t + 4 (a (BN/128) + h), A atom a at sfa_t + 4 a
                     const uint32_t sfb_t = tmem + kSfCol0 + s * T::kSfColsPerStage;
                     const uint32_t sfa_t = sfb_t + T::kSfbCols;
-                    const uint64_t sfa_d = sfa_d0 + (uint64_t)((s * kSfaBytes) >> 4);
-                    const uint64_t sfb_d = sfb_d0 + (uint64_t)((s * kSfbBytes) >> 4);
-#pragma unroll
-                    for (int a = 0; a < T::kAtoms; a++) {
-                        tc_cp_sf(sfa_t + 4 * a, sfa_d + (uint64_t)(a * 512 / 16));
-#pragma unroll
-                        for (int h = 0; h < BN / 128; h++)
-                            tc_cp_sf(sfb_t + 4 * (a * (BN / 128) + h), sfb_d + (uint64_t)((h * T::kSfaBytes + a * 512) / 16));
-                    }
                     const uint64_t a_d = a_d0 + (uint64_t)((s * kABytes) >> 4);
                     const uint64_t b_d = b_d0 + (uint64_t)((s * kBBytes) >> 4);
                     // four instructions per stage, each over 32 bytes of K per row (K = 32 for
@@ -265,6 +298,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 (void)mbar_wait_bounded(&full_bar[s], (uint32_t)(last_it[s] / kStages) & 1u, nullptr, 0, kDrainLimitNs);
     }
     if (*fail_sh && warp == kMmaWarp && lane == 0) (void)mbar_wait_bounded(&drain_bar, 0u, nullptr, 0, kDrainLimitNs);
+    if (warp == kSfWarp && lane == 0) (void)mbar_wait_bounded(&sf_drain, 0u, nullptr, 0, kDrainLimitNs);
     tc_fence_before();
     __syncthreads();
     if (warp == kMmaWarp) {

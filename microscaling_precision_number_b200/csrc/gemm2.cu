@@ -36,8 +36,8 @@ constexpr int kPairM = 256, kPairN = 256;            // output tile of the pair
 constexpr int kRowBytes = 128;                       // bytes of K per row per stage
 constexpr int kABytes = kHalfRows * kRowBytes;       // 16 KiB
 constexpr int kBBytes = kHalfRows * kRowBytes;       // 16 KiB (this CTA's half of B)
-constexpr int kProducerWarp = 8, kMmaWarp = 9, kEpilogueWarps = 8;
-constexpr int kPairThreads = 320;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kSfWarp = 10, kEpilogueWarps = 8;
+constexpr int kPairThreads = 352;
 constexpr uint32_t kTmemCols = 512, kSfCol0 = 256;
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;       // shared::cluster address of the even CTA's copy
 
@@ -98,7 +98,8 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint8_t *sSFA = sB + S * kBBytes;                    // S x kAtoms x 512 B
     uint8_t *sSFB = sSFA + S * P::kSfaBytes;             // S x 2 x kAtoms x 512 B
 
-    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], acc_full, acc_empty, drain_bar, exit_bar;
+    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], sf_ready[S], acc_full, acc_empty, drain_bar,
+        sf_drain, exit_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int fail_flag;
     volatile int *fail_sh = &fail_flag;
@@ -116,10 +117,15 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         prefetch_tensormap(&tmB);
         prefetch_tensormap(&tmSA);
         prefetch_tensormap(&tmSB);
-        for (int s = 0; s < S; s++) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+        for (int s = 0; s < S; s++) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+            mbar_init(&sf_ready[s], 1);
+        }
         mbar_init(&acc_full, 1);
         mbar_init(&acc_empty, 2 * kEpilogueWarps);
         mbar_init(&drain_bar, 1);
+        mbar_init(&sf_drain, 1);
         mbar_init(&exit_bar, 1);
         *fail_sh = 0;
         fence_barrier_init();
@@ -170,25 +176,18 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------ MMA issuer (even CTA only)
+    } else if (warp == kSfWarp) {
+        // ------------------------------------------------ scale-atom copier (even CTA only)
+        // Copies each stage's scale atoms into tensor memory (both CTAs') as soon as the
+        // stage has landed, and signals sf_ready[s] once the copies are complete.  The MMA
+        // issuer waits on sf_ready alone (it implies the stage's operands are there), so the
+        // copies leave the single MMA-issuing thread, whose instruction latency otherwise
+        // bounds the tensor pipe.  A stage's scale slot is rewritten only after full[s] of
+        // its next use, i.e. after the MMAs that read it have completed (empty[s]).
         if (leader && lane == 0) {
-            // precomputed descriptors on the issuing thread (as in gemm.cu)
-            const uint64_t a_d0 = smem_desc(smem_u32(sA), 16, 1024, 2), b_d0 = smem_desc(smem_u32(sB), 16, 1024, 2);
             const uint64_t sfa_d0 = sf_desc(smem_u32(sSFA)), sfb_d0 = sf_desc(smem_u32(sSFB));
-            uint32_t idesc[4];
-#pragma unroll
-            for (int k = 0; k < 4; k++)
-                idesc[k] = mma_idesc<kPairM, kPairN, KIND>(
-                    a_fmt_code, b_fmt_code,
-                    KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u));
-            int it = 0, i = 0;
-            for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs, i++) {
-                if (i > 0 && !mbar_wait_bounded(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
-                    *fail_sh = 1;
-                    break;
-                }
-                tc_fence_after();
+            int it = 0;
+            for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs) {
                 for (int kb = 0; kb < num_kb; kb++, it++) {
                     const int s = it % S;
                     if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
@@ -207,6 +206,40 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         for (int h = 0; h < 2; h++)
                             tc_cp_sf<2>(sfb_t + 4 * (2 * a + h), sfb_d + (uint64_t)((h * P::kSfaBytes + a * 512) / 16));
                     }
+                    tc_commit_pair_local(&sf_ready[s]);      // the stage's scales are in tensor memory
+                }
+            }
+            tc_commit_pair_local(&sf_drain);                 // completes once every copy above has finished
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------ MMA issuer (even CTA only)
+        if (leader && lane == 0) {
+            // precomputed descriptors on the issuing thread (as in gemm.cu)
+            const uint64_t a_d0 = smem_desc(smem_u32(sA), 16, 1024, 2), b_d0 = smem_desc(smem_u32(sB), 16, 1024, 2);
+            uint32_t idesc[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+                idesc[k] = mma_idesc<kPairM, kPairN, KIND>(
+                    a_fmt_code, b_fmt_code,
+                    KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u));
+            int it = 0, i = 0;
+            for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs, i++) {
+                if (i > 0 && !mbar_wait_bounded(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
+                    *fail_sh = 1;
+                    break;
+                }
+                tc_fence_after();
+                for (int kb = 0; kb < num_kb; kb++, it++) {
+                    const int s = it % S;
+                    // the stage's operands have landed and its scales are in tensor memory
+                    if (!mbar_wait_bounded(&sf_ready[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
+                        *fail_sh = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sfb_t = tmem + kSfCol0 + s * P::kSfColsPerStage;
+                    const uint32_t sfa_t = sfb_t + P::kSfbCols;
                     const uint64_t a_d = a_d0 + (uint64_t)((s * kABytes) >> 4);
                     const uint64_t b_d = b_d0 + (uint64_t)((s * kBBytes) >> 4);
 #pragma unroll
@@ -270,6 +303,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (last_it[s] >= 0)
                     (void)mbar_wait_bounded(&full_bar[s], (uint32_t)(last_it[s] / S) & 1u, nullptr, 0, kDrainLimitNs);
         (void)mbar_wait_bounded(&drain_bar, 0u, nullptr, 0, kDrainLimitNs);
+        if (leader) (void)mbar_wait_bounded(&sf_drain, 0u, nullptr, 0, kDrainLimitNs);   // scale copies too
         // the odd CTA's copies complete on the even CTA's barriers, so it stays until the
         // even CTA has drained them: each CTA arrives on the other's exit barrier
         mbar_arrive_remote(&exit_bar, rank ^ 1u);
