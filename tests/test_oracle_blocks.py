@@ -135,18 +135,18 @@ def test_fp4_nibble_order(oracle):
 
 def test_colwise_is_rowwise_of_transpose(oracle):
     x = synth.activations(64, 96, seed=2)
-    for fmt in (oracle.E4M3, oracle.E2M1):
+    for fmt in (oracle.E4M3, oracle.E5M2, oracle.E2M1, oracle.E2M3, oracle.E3M2, oracle.INT8):
         ec, sc = oracle.quantize_mx(x, fmt, oracle.COL, oracle.CEIL)
         er, sr = oracle.quantize_mx(np.ascontiguousarray(x.T), fmt, oracle.ROW, oracle.CEIL)
         assert np.array_equal(ec, er) and np.array_equal(sc, sr)
-        assert ec.shape[0] == 96 and sc.shape == (96, 2)
+        assert ec.shape == (96, oracle.elem_bytes(64, fmt)) and sc.shape == (96, 2)
 
 
 def test_nan_or_inf_makes_block_nan(oracle):
     x = synth.normal(2, 64, seed=1)
     x[0, 5] = 0x7FC0      # NaN in block (0, 0)
     x[1, 40] = 0xFF80     # -Inf in block (1, 1)
-    for fmt in (oracle.E4M3, oracle.E5M2, oracle.E2M1):
+    for fmt in (oracle.E4M3, oracle.E5M2, oracle.E2M1, oracle.E2M3, oracle.E3M2, oracle.INT8):
         e, s = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.CEIL)
         assert s[0, 0] == 0xFF and s[1, 1] == 0xFF and s[0, 1] != 0xFF and s[1, 0] != 0xFF
         d = bf16_bits_to_f64(oracle.dequantize_mx(e, s, 2, 64, fmt))
