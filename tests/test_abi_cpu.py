@@ -125,3 +125,54 @@ def test_product_package_does_not_import_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in text and "from oracle" not in text and "mx_oracle" not in text, f
+
+
+# ------------------------------------------------------------------ newer entry points
+@pytest.mark.parametrize("args,status", [
+    (dict(fmt=4), "MX_ERR_ARG"), (dict(fmt=6), "MX_ERR_ARG"),              # FP6 / INT8: not training formats
+    (dict(rounding=2), "MX_ERR_ARG"), (dict(rht=2), "MX_ERR_ARG"),
+    (dict(fmt=3), "MX_ERR_ARG"), (dict(g=FAKE), "MX_ERR_ARG"),             # g exactly for NVFP4
+    (dict(layout=0), "MX_ERR_LAYOUT"), (dict(layout=3), "MX_ERR_LAYOUT"),
+    (dict(rows=-1), "MX_ERR_SHAPE"), (dict(cols=48), "MX_ERR_SHAPE"), (dict(fmt=3, cols=40, g=FAKE), "MX_ERR_SHAPE"),
+    (dict(src=0), "MX_ERR_ARG"), (dict(out=0), "MX_ERR_ARG"), (dict(sc=0), "MX_ERR_ARG"),
+    (dict(src=FAKE + 8), "MX_ERR_ALIGN"), (dict(rnd=FAKE + 8), "MX_ERR_ALIGN"),
+    (dict(fmt=3, g=FAKE + 2), "MX_ERR_ALIGN"),
+    (dict(rows=0), "MX_OK"),
+])
+def test_quantize_train_validation(L, args, status):
+    a = dict(src=FAKE, rows=64, cols=64, fmt=2, rounding=0, rht=1, signs=0xB5C3, rnd=FAKE, out=FAKE, sc=FAKE,
+             layout=2, alt=0, g=0)
+    a.update(args)
+    got = L.lib.mx_quantize_train(a["src"], a["rows"], a["cols"], a["fmt"], a["rounding"], a["rht"], a["signs"],
+                                  a["rnd"] or None, a["out"] or None, a["sc"] or None, a["layout"], a["alt"] or None,
+                                  a["g"] or None, None)
+    assert got == getattr(L, status), (args, got)
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(layout=0), "MX_ERR_LAYOUT"), (dict(layout=1, alt=FAKE), "MX_ERR_LAYOUT"),
+    (dict(rows=24), "MX_ERR_SHAPE"), (dict(cols=40), "MX_ERR_SHAPE"), (dict(rows=-16), "MX_ERR_SHAPE"),
+    (dict(src=0), "MX_ERR_ARG"), (dict(g=0), "MX_ERR_ARG"),
+    (dict(out=FAKE + 4), "MX_ERR_ALIGN"), (dict(g=FAKE + 1), "MX_ERR_ALIGN"),
+    (dict(cols=0), "MX_OK"),
+])
+def test_quantize_nvfp4_2d_validation(L, args, status):
+    a = dict(src=FAKE, rows=32, cols=64, out=FAKE, sc=FAKE, layout=2, alt=0, g=FAKE)
+    a.update(args)
+    got = L.lib.mx_quantize_nvfp4_2d(a["src"], a["rows"], a["cols"], a["out"] or None, a["sc"] or None, a["layout"],
+                                     a["alt"] or None, a["g"] or None, None)
+    assert got == getattr(L, status), (args, got)
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(rows=64), "MX_ERR_SHAPE"), (dict(cols=192), "MX_ERR_SHAPE"), (dict(rows=-128), "MX_ERR_SHAPE"),
+    (dict(elems=0), "MX_ERR_ARG"), (dict(scales=0), "MX_ERR_ARG"), (dict(ok=0), "MX_ERR_ARG"),
+    (dict(elems=FAKE + 8), "MX_ERR_ALIGN"), (dict(out=FAKE + 8), "MX_ERR_ALIGN"), (dict(bs=FAKE + 2), "MX_ERR_ALIGN"),
+    (dict(rows=0), "MX_OK"),
+])
+def test_nested_blocks_validation(L, args, status):
+    a = dict(elems=FAKE, scales=FAKE, rows=128, cols=256, out=FAKE, bs=FAKE, ok=FAKE)
+    a.update(args)
+    got = L.lib.mx_mxfp4_to_fp8_blocks(a["elems"] or None, a["scales"] or None, a["rows"], a["cols"],
+                                       a["out"] or None, a["bs"] or None, a["ok"] or None, None)
+    assert got == getattr(L, status), (args, got)
