@@ -206,3 +206,27 @@ def test_gemm_fp6_fp8_operand_pairs(oracle, a_fmt, b_fmt, M, N, K):
     a = synth.normal(M, K, seed=M + a_fmt)
     b = synth.weight_fp4(N, K, seed=N + b_fmt) if b_fmt == 2 else synth.normal(N, K, seed=N + b_fmt)
     run_case(oracle, a, b, b_fmt, a_fmt=a_fmt)
+
+
+# ------------------------------------------------------------------ an outside check of the scale tiling
+def test_scale_tiling_agrees_with_cublaslt():
+    """The tcgen05 scale tiling is not defined by the pages; cuBLASLt's MXFP8 block-scaled
+    matmul (through torch._scaled_mm) takes its E8M0 scales in the same 128 x 4 atom layout.
+    Fed the very scale bytes this library writes, it must produce the same product (within
+    the matmul tolerance; in practice bit for bit) -- a library-side pin of the tiling, in
+    addition to the oracle parity above.  Skipped when this torch / cuBLAS lacks the call."""
+    M = N = K = 8192
+    a = mx.quantize(to_dev(synth.normal(M, K, seed=40)), "e4m3", "row", "ceil", layout="tcgen05")
+    b = mx.quantize(to_dev(synth.normal(N, K, seed=41)), "e4m3", "row", "ceil", layout="tcgen05")
+    ours = mx.gemm(a, b).float()
+    try:
+        lib = torch._scaled_mm(a.elems.view(torch.float8_e4m3fn).view(M, K),
+                               b.elems.view(torch.float8_e4m3fn).view(N, K).t(),
+                               scale_a=a.scales.view(torch.float8_e8m0fnu),
+                               scale_b=b.scales.view(torch.float8_e8m0fnu), out_dtype=torch.bfloat16).float()
+    except (RuntimeError, TypeError, AttributeError) as e:      # the library call itself is unavailable
+        pytest.skip(f"torch._scaled_mm MXFP8 unavailable: {e}")
+    diff = (ours - lib).abs()
+    scale = ours.abs().max()
+    assert float(diff.max()) <= 2e-3 * float(scale)
+    assert float((diff == 0).float().mean()) >= 0.99
