@@ -57,6 +57,27 @@ def test_train_quantiser_matches_oracle(oracle, fmt, rht, sr, shape):
     assert np.array_equal(q.scales_alt.cpu().numpy(), oracle.to_tcgen05_layout(s))
 
 
+@pytest.mark.parametrize("fmt", ["e2m1", "nvfp4"])
+def test_train_quantiser_multi_cta(oracle, fmt):
+    """A gradient of the benchmark's width (1024 x 14336) with the transform and stochastic
+    rounding: the grid is capped, so every CTA walks several blocks (grid-stride loops) and
+    NVFP4's tensor maximum comes from many partial maxima -- bit for bit as above."""
+    shape = (1024, 14336)
+    x = synth.gradients(*shape, seed=77)
+    rnd = np.random.default_rng(78).integers(0, 256, size=shape, dtype=np.uint8)
+    rounding = "floor" if fmt == "e2m1" else "ceil"
+    q = mx.quantize_train(to_dev(x), fmt, rounding, rht_signs=0xB5C3, sr_random=torch.from_numpy(rnd).cuda(),
+                          layout="tcgen05")
+    xt = oracle.rht16(x, 0xB5C3)
+    if fmt == "nvfp4":
+        e, s, g = oracle.quantize_nvfp4_sr(xt, rnd)
+        assert q.global_scale.cpu().numpy()[0] == np.float32(g)
+    else:
+        e, s = oracle.quantize_mx_sr(xt, FMT[fmt], oracle.FLOOR, rnd)
+    assert np.array_equal(q.elems.cpu().numpy(), e.reshape(-1))
+    assert np.array_equal(q.scales.cpu().numpy(), oracle.to_tcgen05_layout(s))
+
+
 def test_rht_keeps_the_matmul(oracle):
     """The same transform on both operands along K leaves A * B^T unchanged up to the
     quantisation (the property that makes it usable on weight-gradient inputs)."""
