@@ -411,7 +411,7 @@ def run_breakdown(mx, dev, pk):
                 for x, q in zip(xs, qs)], 256, stream)
     td = timed([lambda q=q, y=y: mx.dequantize(q, "rowmajor", out=y) for q, y in zip(qs, ys)], 256, stream)
     b1 = 1024 * 1024 * 2 + 1024 * 1024 + 1024 * 32
-    out["c1_mxfp8_rowwise_1024"] = {"quantize_us": round(tq * 1e3, 2), "dequantize_us": round(td * 1e3, 2),
+    out["mxfp8_rowwise_1024x1024"] = {"quantize_us": round(tq * 1e3, 2), "dequantize_us": round(td * 1e3, 2),
                                     "quantize_GBps": round(b1 / tq / 1e6, 1),
                                     "dequantize_GBps": round(b1 / td / 1e6, 1),
                                     "frac_hbm": round(b1 / tq / 1e6 / hbm, 4),
@@ -429,7 +429,7 @@ def run_breakdown(mx, dev, pk):
                         mx.dequantize(q, "rowmajor", out=y)
             graphs.append(g)
         gq, gd = (timed([g.replay], 4, stream) / len(xs) for g in graphs)
-        out["c1_mxfp8_rowwise_1024"].update({"graph_quantize_us": round(gq * 1e3, 2),
+        out["mxfp8_rowwise_1024x1024"].update({"graph_quantize_us": round(gq * 1e3, 2),
                                              "graph_dequantize_us": round(gd * 1e3, 2),
                                              "graph_quantize_GBps": round(b1 / gq / 1e6, 1),
                                              "graph_dequantize_GBps": round(b1 / gd / 1e6, 1),
@@ -437,10 +437,10 @@ def run_breakdown(mx, dev, pk):
                                              "graph_note": "64 calls on 64 rotating copies in one CUDA graph"})
         del graphs
     except RuntimeError as e:                              # capture refused: report, keep going
-        out["c1_mxfp8_rowwise_1024"]["graph_error"] = str(e)[:200]
+        out["mxfp8_rowwise_1024x1024"]["graph_error"] = str(e)[:200]
     del x1, xs, qs
 
-    # a7: dequantise the config-2 weight (MXFP4 and NVFP4), tcgen05 scales, 8 rotating copies
+    # dequantise the 4096 x 4096 weight (MXFP4 and NVFP4), tcgen05 scales, 8 rotating copies
     xw = to_dev(synth.weight_fp4(), dev)
     q4 = [mx.quantize(xw, "e2m1", "row", "floor", layout="tcgen05") for _ in range(NROT)]
     qn = [mx.quantize(xw, "nvfp4", "row", "ceil", layout="tcgen05") for _ in range(NROT)]
@@ -449,7 +449,7 @@ def run_breakdown(mx, dev, pk):
     tn = timed([lambda q=q, y=y: mx.dequantize(q, "tcgen05", out=y) for q, y in zip(qn, ys)], 64, stream)
     bd4 = R2 * C2 // 2 + R2 * C2 // 32 + R2 * C2 * 2
     bdn = R2 * C2 // 2 + R2 * C2 // 16 + 4 + R2 * C2 * 2
-    out["a7_dequantize_4096"] = {"mxfp4_GBps": round(bd4 / t4 / 1e6, 1), "mxfp4_frac_hbm": round(bd4 / t4 / 1e6 / hbm, 4),
+    out["dequantize_4096x4096"] = {"mxfp4_GBps": round(bd4 / t4 / 1e6, 1), "mxfp4_frac_hbm": round(bd4 / t4 / 1e6 / hbm, 4),
                                  "nvfp4_GBps": round(bdn / tn / 1e6, 1), "nvfp4_frac_hbm": round(bdn / tn / 1e6 / hbm, 4)}
     del xw, q4, qn, ys
 
@@ -463,18 +463,18 @@ def run_breakdown(mx, dev, pk):
         o3 = mx.quantize_dual(x3, fmt, "ceil", "tcgen05")
         t = timed([lambda: mx.quantize_dual(x3, fmt, "ceil", "tcgen05", out=o3)], 20, stream)
         nbytes = R * C * 2 + 2 * (R * C + R * C // 32)
-        out[f"c3_dual_{name}"] = {"ms": round(t, 4), "GBps": round(nbytes / t / 1e6, 1),
+        out[f"dual_{name}"] = {"ms": round(t, 4), "GBps": round(nbytes / t / 1e6, 1),
                                   "frac_hbm": round(nbytes / t / 1e6 / hbm, 4), "algorithmic_bytes": nbytes,
                                   "l2": "input larger than L2"}
         del x3, o3
         torch.cuda.empty_cache()
 
     # C4 / C5: block-scaled matmuls (operands quantised outside the timing)
-    # (plus the next-row MXFP6 x MXFP6 matmul, which runs on the same kind at the same rate)
+    # (plus the MXFP6 x MXFP6 matmul, which runs on the same kind at the same rate)
     for name, (M, N, K), afmt, bfmt, bsig in (
-            ("c4_gemm_e4m3_8192", (8192, 8192, 8192), "e4m3", "e4m3", 1.0),
-            ("c5_gemm_e4m3_x_e2m1_8192x14336x4096", (8192, 14336, 4096), "e4m3", "e2m1", 0.02),
-            ("next_gemm_mxfp6_e2m3_8192", (8192, 8192, 8192), "e2m3", "e2m3", 1.0)):
+            ("gemm_e4m3_8192", (8192, 8192, 8192), "e4m3", "e4m3", 1.0),
+            ("gemm_e4m3_x_e2m1_8192x14336x4096", (8192, 14336, 4096), "e4m3", "e2m1", 0.02),
+            ("gemm_mxfp6_e2m3_8192", (8192, 8192, 8192), "e2m3", "e2m3", 1.0)):
         a = mx.quantize(to_dev(synth.normal(M, K, seed=40), dev), afmt, "row", "ceil", layout="tcgen05")
         b = mx.quantize(to_dev(synth.normal(N, K, sigma=bsig, seed=41), dev), bfmt, "row",
                         "floor" if bfmt == "e2m1" else "ceil", layout="tcgen05")
@@ -493,7 +493,7 @@ def run_breakdown(mx, dev, pk):
         torch.cuda.empty_cache()
 
     # library comparator (not this library's path): cuBLASLt's MXFP8 block-scaled matmul via
-    # torch._scaled_mm on the same config-4 operands -- the E8M0 scales in the tcgen05
+    # torch._scaled_mm on the same 8192^3 E4M3 operands -- the E8M0 scales in the tcgen05
     # tiling are the layout it takes
     try:
         M = N = K = 8192
@@ -512,20 +512,20 @@ def run_breakdown(mx, dev, pk):
         t = timed([lib], 10, stream)
         tb = best_of(lib, 10, stream)
         tf, tfb = (2.0 * M * N * K / (x * 1e-3) / 1e12 for x in (t, tb))
-        out["lib_cublaslt_mxfp8_8192_comparator"] = {
+        out["cublaslt_mxfp8_8192_comparator"] = {
             "ms": round(t, 4), "TFLOPS": round(tf, 1), "best_of_10_TFLOPS": round(tfb, 1),
             "frac_mx_peak_measured": round(tf / mx_peak, 4), "max_abs_diff_vs_ours_rel_to_max": rel,
             "clocks_back_to_back": soak_clocks(lib),
             "note": "torch._scaled_mm (cuBLASLt) on the same operands: a comparator, not this library's path"}
         del a, b, af, bf, sa, sb, ref, ours
     except Exception as e:                                   # comparator unavailable: say why
-        out["lib_cublaslt_mxfp8_8192_comparator"] = {"unavailable": str(e)[:200]}
+        out["cublaslt_mxfp8_8192_comparator"] = {"unavailable": str(e)[:200]}
     torch.cuda.empty_cache()
 
-    # next row: FP4 x FP4 block-scaled matmuls (kind::mxf4 and kind::mxf4nvf4), 8192^3,
+    # FP4 x FP4 block-scaled matmuls (kind::mxf4 and kind::mxf4nvf4), 8192^3,
     # against the dense FP4 rate (2 x the FP8 rate; 9 PFLOP/s nominal)
     fp4_peak = 2.0 * mx_peak
-    for name, fmt in (("next_gemm_mxfp4_x_mxfp4_8192", "e2m1"), ("next_gemm_nvfp4_x_nvfp4_8192", "nvfp4")):
+    for name, fmt in (("gemm_mxfp4_x_mxfp4_8192", "e2m1"), ("gemm_nvfp4_x_nvfp4_8192", "nvfp4")):
         M = N = K = 8192
         a = mx.quantize(to_dev(synth.normal(M, K, seed=60), dev), fmt, "row", "floor", layout="tcgen05")
         b = mx.quantize(to_dev(synth.normal(N, K, sigma=0.02, seed=61), dev), fmt, "row", "floor", layout="tcgen05")
@@ -543,11 +543,11 @@ def run_breakdown(mx, dev, pk):
         del a, b, c
         torch.cuda.empty_cache()
 
-    # next row: MXFP6 / MXINT8 row-wise quantisation of the config-3 activations
+    # MXFP6 / MXINT8 row-wise quantisation of the 16384 x 4096 activations
     # (16384 x 4096 bf16; FP6 codes packed 6 bits each, INT8 one byte), against the HBM roofline
     x3 = to_dev(synth.activations(), dev)
     R, C = x3.shape
-    for name, fmt in (("next_quant_mxfp6_e2m3_16384x4096", "e2m3"), ("next_quant_mxint8_16384x4096", "int8")):
+    for name, fmt in (("quant_mxfp6_e2m3_16384x4096", "e2m3"), ("quant_mxint8_16384x4096", "int8")):
         q = mx.quantize(x3, fmt, "row", "ceil", layout="tcgen05")
         t = timed([lambda q=q: mx.quantize(x3, fmt, "row", "ceil", layout="tcgen05", out=q)], 20, stream)
         nb = R * C * 2 + mx.elem_bytes(R, C, fmt) + R * C // 32
@@ -556,7 +556,7 @@ def run_breakdown(mx, dev, pk):
         del q
     del x3
 
-    # next row: nested blocks -- the config-5 MXFP4 weight (14336 x 4096) re-expressed as
+    # nested blocks -- the 14336 x 4096 MXFP4 weight re-expressed as
     # FP8 E4M3 with 128 x 128 block scales
     from microscaling_precision_number_b200 import _lib as L
     xw = to_dev(synth.normal(14336, 4096, sigma=0.02, seed=51), dev)
@@ -575,21 +575,21 @@ def run_breakdown(mx, dev, pk):
                 "mx_mxfp4_to_fp8_blocks")
     t = timed([lambda st=st: nested(*st) for st in sets], 20, stream)
     nb = R * C // 2 + R * C // 32 + R * C + 5 * (R // 128) * (C // 128)
-    out["next_nested_mxfp4_to_fp8_14336x4096"] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1),
+    out["nested_mxfp4_to_fp8_14336x4096"] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1),
                                                    "frac_hbm": round(nb / t / 1e6 / hbm, 4), "algorithmic_bytes": nb,
                                                    "blocks_exact": int(bok.sum().item()), "blocks": int(bok.numel()),
                                                    "l2": "four rotating sets, 352 MiB > L2"}
     del qw, sets, bsc, bok
     torch.cuda.empty_cache()
 
-    # next row: training-side quantiser on the config-3 gradient shape (16384 x 14336 bf16):
+    # training-side quantiser on the 16384 x 14336 gradient shape (bf16):
     # 16 x 16 random Hadamard transform + stochastic rounding (one random byte per element),
     # NVFP4 (two passes; the maximum pass's re-read is not counted) and MXFP4; tcgen05 scales
     R, C = 16384, 14336
     xg = to_dev(synth.normal(R, C, sigma=1e-3, seed=70), dev)
     rnd = torch.from_numpy(np.random.default_rng(71).integers(0, 256, R * C, dtype=np.uint8)).to(dev)
-    for name, f, B in (("next_train_nvfp4_rht_sr_16384x14336", L.MX_FMT_NVFP4, 16),
-                       ("next_train_mxfp4_rht_sr_16384x14336", L.MX_FMT_E2M1, 32)):
+    for name, f, B in (("train_nvfp4_rht_sr_16384x14336", L.MX_FMT_NVFP4, 16),
+                       ("train_mxfp4_rht_sr_16384x14336", L.MX_FMT_E2M1, 32)):
         el = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
         sc = torch.empty(mx.scale_bytes(R, C // B, "tcgen05"), dtype=torch.uint8, device=dev)
         gs = torch.empty(1, dtype=torch.float32, device=dev) if f == L.MX_FMT_NVFP4 else None
@@ -607,7 +607,7 @@ def run_breakdown(mx, dev, pk):
     del xg, rnd
     torch.cuda.empty_cache()
 
-    # next row: NVFP4 with 16 x 16 weight blocks on the config-2 weight (4096 x 4096)
+    # NVFP4 with 16 x 16 weight blocks on the 4096 x 4096 weight
     R = C = 4096
     xw = to_dev(synth.weight_fp4(), dev)
     el = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
@@ -621,7 +621,7 @@ def run_breakdown(mx, dev, pk):
                                            None, gs.data_ptr(), stream.cuda_stream), "mx_quantize_nvfp4_2d")
     t = timed([lambda x=x: nvfp4_2d(x) for x in xs], 24, stream)
     nb = R * C * 2 + R * C // 2 + sc.numel() + 4
-    out["next_quant_nvfp4_2d_weight_4096"] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1),
+    out["quant_nvfp4_2d_4096x4096"] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1),
                                               "frac_hbm": round(nb / t / 1e6 / hbm, 4), "algorithmic_bytes": nb,
                                               "l2": "six rotating inputs, 192 MiB > L2"}
     del xw, xs, el, sc, gs
@@ -721,7 +721,7 @@ def run_case(name, iters, dev):
         c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
         fns = [lambda: mx.gemm(a, b, c)]
     elif name == "gemm_cmp":
-        # config-4 operands through this library's matmul and through cuBLASLt's MXFP8
+        # the 8192^3 E4M3 operands through this library's matmul and through cuBLASLt's MXFP8
         # matmul (torch._scaled_mm), one call each per round, for side-by-side counters
         M = N = K = 8192
         a = mx.quantize(to_dev(synth.normal(M, K, seed=40), dev), "e4m3", "row", "ceil", layout="tcgen05")
@@ -731,8 +731,8 @@ def run_case(name, iters, dev):
         sa, sb = a.scales.view(torch.float8_e8m0fnu), b.scales.view(torch.float8_e8m0fnu)
         fns = [lambda: (mx.gemm(a, b, c),
                         torch._scaled_mm(af, bf.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16))]
-    elif name == "next_rows":
-        # one call of each next-row kernel: training quantiser (NVFP4 and MXFP4, RHT + SR) on an
+    elif name == "extended":
+        # one call of each extended kernel: training quantiser (NVFP4 and MXFP4, RHT + SR) on an
         # 8192 x 14336 gradient, nested conversion, MXFP6 matmul, 2-D NVFP4 weight blocks
         from microscaling_precision_number_b200 import _lib as L
         xg = to_dev(synth.normal(8192, 14336, sigma=1e-3, seed=70), dev)
@@ -764,7 +764,7 @@ def run_case(name, iters, dev):
 
 
 CASES = ["weight4096", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "gemm8192", "gemm_w4a8",
-         "gemm_mxfp4_8192", "gemm_nvfp4_8192", "gemm_cmp", "next_rows"]
+         "gemm_mxfp4_8192", "gemm_nvfp4_8192", "gemm_cmp", "extended"]
 
 
 def main():

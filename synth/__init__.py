@@ -77,13 +77,3 @@ def special_values_block() -> np.ndarray:
     vals = [0x0000, 0x8000, 0x0001, 0x8001, 0x007F, 0x0080, 0x7F7F, 0xFF7F,
             0x3F80, 0xBF80, 0x4300, 0x43E0, 0x43E8, 0x43F0, 0x4760, 0x4770]
     return np.array(vals, dtype=np.uint16)
-
-
-# Workload table used by the benchmark and the full-size parity tests.
-CONFIGS = {
-    1: dict(name="mx8_rowwise_1024x1024_e4m3_ceil", shape=(1024, 1024)),
-    2: dict(name="weight_4096x4096_mxfp4_floor_and_nvfp4", shape=(4096, 4096)),
-    3: dict(name="dual_act_16384x4096_e4m3_grad_16384x14336_e5m2", shape=(16384, 4096)),
-    4: dict(name="gemm_e4m3xe4m3_8192x8192x8192", shape=(8192, 8192, 8192)),
-    5: dict(name="gemm_e4m3_act_x_e2m1_weight_m8192_n14336_k4096", shape=(8192, 14336, 4096)),
-}

@@ -137,7 +137,7 @@ def sample_pairs(M, N, n, seed):
     return np.concatenate([p, corners]).astype(np.int64)
 
 
-def test_config4_gemm_8192_sampled(oracle):
+def test_gemm_e4m3_8192_sampled(oracle):
     M = N = K = 8192
     a = synth.normal(M, K, seed=40)
     b = synth.normal(N, K, seed=41)
@@ -145,7 +145,7 @@ def test_config4_gemm_8192_sampled(oracle):
     torch.cuda.empty_cache()
 
 
-def test_config5_gemm_mixed_sampled(oracle):
+def test_gemm_e4m3_x_e2m1_8192x14336x4096_sampled(oracle):
     M, N, K = 8192, 14336, 4096
     a = synth.normal(M, K, seed=50)
     b = synth.normal(N, K, sigma=0.02, seed=51)

@@ -96,7 +96,7 @@ def test_single_tile_offsets_and_magnitudes(oracle):
     assert flags[(-11, 6, 0)] == 1 and flags[(-11, 7, 0)] == 0 and flags[(-12, 6, 0)] == 0
 
 
-def test_config5_weight(oracle):
+def test_weight_14336x4096(oracle):
     """The mixed-GEMM weight shape (14336 x 4096, N(0, 0.02)) end to end."""
     x = synth.normal(14336, 4096, sigma=0.02, seed=51)
     e, s = oracle.quantize_mx(x, oracle.E2M1, oracle.ROW, oracle.FLOOR)

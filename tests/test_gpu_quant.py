@@ -205,7 +205,7 @@ def test_dequantize_all_scale_codes(oracle):
 
 
 # ------------------------------------------------------------------ full-size workloads
-def test_config1_mx8_rowwise_full(oracle):
+def test_mx8_rowwise_1024x1024_full(oracle):
     x = synth.mx8_rowwise()
     q = mx.quantize(to_dev(x), "e4m3", "row", "ceil", layout="rowmajor")
     e_ref, s_ref = oracle.quantize_mx(x, oracle.E4M3, oracle.ROW, oracle.CEIL)
@@ -215,7 +215,7 @@ def test_config1_mx8_rowwise_full(oracle):
     assert np.array_equal(d.reshape(-1), oracle.dequantize_mx(e_ref, s_ref, 1024, 1024, oracle.E4M3).reshape(-1))
 
 
-def test_config2_weight_full(oracle):
+def test_weight_4096x4096_full(oracle):
     x = synth.weight_fp4()
     dev = to_dev(x)
     q4 = mx.quantize(dev, "e2m1", "row", "floor", layout="both")
@@ -232,7 +232,7 @@ def test_config2_weight_full(oracle):
 
 
 @pytest.mark.parametrize("which", ["activations", "gradients"])
-def test_config3_dual_full_sampled(oracle, which):
+def test_dual_full_size_sampled(oracle, which):
     """Full-size dual quantisation in the benchmark's launch configuration; sampled
     32 x 128 tiles checked against the oracle (blocks are independent)."""
     if which == "activations":
