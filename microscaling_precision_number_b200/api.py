@@ -63,7 +63,7 @@ def _check_src(x: torch.Tensor):
 
 
 class Quantized(NamedTuple):
-    elems: torch.Tensor          # uint8 codes (FP4: two per byte, even index low nibble)
+    elems: torch.Tensor          # uint8 codes, packed densely (FP4 two per byte, even index low; FP6 four per three bytes)
     scales: torch.Tensor         # uint8 scales in the first layout
     scales_alt: Optional[torch.Tensor]   # tcgen05 scales when layout == "both"
     global_scale: Optional[torch.Tensor]  # NVFP4 fp32 g
