@@ -23,6 +23,11 @@
  *     device (or managed) memory of the current CUDA device.  The library keeps, per
  *     device, only a small scratch array for NVFP4 partial maxima (allocated on the
  *     first NVFP4 call on that device) and a static watchdog flag.
+ *   - NVFP4 calls on one device (mx_quantize with MX_FMT_NVFP4, mx_quantize_train with
+ *     MX_FMT_NVFP4, mx_quantize_nvfp4_2d) share that scratch array: calls whose GPU work
+ *     overlaps -- on two streams with no ordering between them -- race on it and may
+ *     produce a wrong per-tensor scale.  Issue them on one stream, or order the streams
+ *     with events.  The MX formats use no scratch and may overlap freely.
  *   - Execution: every call only validates its arguments on the host and enqueues
  *     kernels on `stream` (0 = the legacy default stream); it returns before the GPU
  *     work finishes.  Nothing is written to any output before the work runs.
