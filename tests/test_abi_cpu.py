@@ -176,3 +176,23 @@ def test_nested_blocks_validation(L, args, status):
     got = L.lib.mx_mxfp4_to_fp8_blocks(a["elems"] or None, a["scales"] or None, a["rows"], a["cols"],
                                        a["out"] or None, a["bs"] or None, a["ok"] or None, None)
     assert got == getattr(L, status), (args, got)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No fallback of any kind: with the shared library absent, the first call raises
+    ImportError, and a CPU tensor is refused rather than quantised on the host."""
+    import subprocess
+    import sys
+    code = (
+        "import torch, microscaling_precision_number_b200 as mx\n"
+        "try:\n"
+        "    mx._lib.lib.load()\n"
+        "except ImportError as e:\n"
+        "    print('import-error', e)\n"
+        "try:\n"
+        "    mx.quantize(torch.zeros(4, 32, dtype=torch.bfloat16), 'e4m3')\n"
+        "except ValueError:\n"
+        "    print('refused-cpu-tensor')\n")
+    env = dict(os.environ, MX_LIB_PATH=str(tmp_path / "absent" / "libmx.so"))
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert "import-error" in out.stdout and "refused-cpu-tensor" in out.stdout, out.stdout + out.stderr
