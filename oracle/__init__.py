@@ -9,10 +9,11 @@ loop per block).  This module only marshals numpy arrays through ctypes and buil
 shared object with gcc when it is missing.
 
 Every function's definition and the passage it follows are documented in ``mx_oracle.c``.
-Parity status: every function here is pinned by the ``-m "not gpu"`` oracle tests
-except the exact NVFP4 step order (pinned only through its invariants and the
-per-tensor-scale definition) and the tcgen05 scale tiling (not defined by the pages;
-pinned on hardware by the block-scaled matmul).
+Parity status: every function here is pinned by the ``-m "not gpu"`` oracle tests, the
+NVFP4 element step (the E2M1 code of the fp32 quotient x / d) exhaustively against
+numpy's IEEE division and an exact nearest-code search.  The tcgen05 scale tiling is
+parity unpinned on the CPU (the pages do not define it; it is pinned on hardware by the
+block-scaled matmul and by cuBLASLt's MXFP8 matmul reading the same scale bytes).
 """
 from __future__ import annotations
 
@@ -77,6 +78,13 @@ def lib():
         _lib.mxo_tcgen05_scale_offset.restype = I64
         _lib.mxo_gemm_ref.argtypes = [P, P, I, ctypes.c_double, P, P, I, ctypes.c_double, I64, I64, I64, P, I64, P, P]
         _lib.mxo_gemm_ref.restype = I
+        _lib.mxo_gemm_ref_block.argtypes = [P, P, I, ctypes.c_double, P, P, I, ctypes.c_double, I64, I64, I64,
+                                            I64, I64, I64, I64, P, P, P, P]
+        _lib.mxo_gemm_ref_block.restype = I
+        _lib.mxo_to_tcgen05_layout.argtypes = [P, I64, I64, P]
+        _lib.mxo_to_tcgen05_layout.restype = I
+        _lib.mxo_from_tcgen05_layout.argtypes = [P, I64, I64, P]
+        _lib.mxo_from_tcgen05_layout.restype = I
         _lib.mxo_quantize_mx_sr.argtypes = [P, I64, I64, I, I, P, P, P]
         _lib.mxo_quantize_mx_sr.restype = I
         _lib.mxo_quantize_nvfp4_sr.argtypes = [P, I64, I64, P, P, P, P]
@@ -205,10 +213,16 @@ def to_tcgen05_layout(scales_rowmajor: np.ndarray) -> np.ndarray:
     s = np.ascontiguousarray(scales_rowmajor, dtype=np.uint8)
     rows, scols = s.shape
     out = np.zeros(tcgen05_scale_bytes(rows, scols), dtype=np.uint8)
-    L = lib()
-    for r in range(rows):
-        for c in range(scols):
-            out[L.mxo_tcgen05_scale_offset(r, c, rows, scols)] = s[r, c]
+    _check(lib().mxo_to_tcgen05_layout(_ptr(s), rows, scols, _ptr(out)), "to_tcgen05_layout")
+    return out
+
+
+def from_tcgen05_layout(tiled: np.ndarray, rows: int, scale_cols: int) -> np.ndarray:
+    """The row-major scale matrix held in a tcgen05-tiled buffer."""
+    t = np.ascontiguousarray(tiled, dtype=np.uint8).reshape(-1)
+    assert t.size >= tcgen05_scale_bytes(rows, scale_cols)
+    out = np.zeros((rows, scale_cols), dtype=np.uint8)
+    _check(lib().mxo_from_tcgen05_layout(_ptr(t), rows, scale_cols, _ptr(out)), "from_tcgen05_layout")
     return out
 
 
@@ -236,6 +250,22 @@ def gemm_ref(a_elems, a_scales, a_fmt, b_elems, b_scales, b_fmt, M, N, K, pairs,
     _check(lib().mxo_gemm_ref(_ptr(ae), _ptr(as_), a_fmt, ctypes.c_double(a_g), _ptr(be), _ptr(bs), b_fmt,
                               ctypes.c_double(b_g), M, N, K,
                               _ptr(pr), pr.shape[0], _ptr(c), _ptr(mag)), "gemm_ref")
+    return c, mag
+
+
+def gemm_ref_block(a_elems, a_scales, a_fmt, b_elems, b_scales, b_fmt, M, N, K, m0, m1, n0, n1, a_g=1.0, b_g=1.0):
+    """fp64 C and sum_k |a b| for every entry of [m0, m1) x [n0, n1), as two arrays."""
+    ae = np.ascontiguousarray(a_elems, dtype=np.uint8)
+    as_ = np.ascontiguousarray(a_scales, dtype=np.uint8)
+    be = np.ascontiguousarray(b_elems, dtype=np.uint8)
+    bs = np.ascontiguousarray(b_scales, dtype=np.uint8)
+    c = np.zeros((m1 - m0, n1 - n0), dtype=np.float64)
+    mag = np.zeros_like(c)
+    ar = np.zeros((m1 - m0, K), dtype=np.float64)
+    br = np.zeros((n1 - n0, K), dtype=np.float64)
+    _check(lib().mxo_gemm_ref_block(_ptr(ae), _ptr(as_), a_fmt, ctypes.c_double(a_g), _ptr(be), _ptr(bs), b_fmt,
+                                    ctypes.c_double(b_g), M, N, K, m0, m1, n0, n1, _ptr(c), _ptr(mag), _ptr(ar),
+                                    _ptr(br)), "gemm_ref_block")
     return c, mag
 
 

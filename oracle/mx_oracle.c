@@ -402,9 +402,11 @@ int mxo_cast(const uint16_t *x, int64_t n, int fmt, uint8_t *out) {
  *   3. per 16-block: amax_b over finite entries; a block holding a NaN or Inf gets the
  *      UE4M3 NaN code 0x7F and all element codes 0;
  *      t = amax_b / (6.0f * g);  sb = UE4M3 RNE-saturated code of t.
- *   4. d = dec(sb) * g.  If d == 0 every code is 0; otherwise r = 1.0f / d and
- *      q_i = E2M1 RNE-saturated code of (x_i * r); when 1/d overflows to Inf and x_i
- *      is a zero, the NaN product is replaced by x_i itself (a signed zero code).
+ *   4. d = dec(sb) * g.  If d == 0 every code is 0; otherwise q_i = E2M1 RNE-saturated
+ *      code of the fp32 quotient x_i / d (one IEEE division, round to nearest; a zero
+ *      x_i gives a zero of its own sign).  Q§3 defines the element as x over the
+ *      two-level scale and Q§7 fixes only the order of the decode multiplies; the
+ *      division by the fp32 decode scale d is the plain reading of that definition.
  * g is written to *g_out.  rows x cols row-major; blocks along rows (cols % 16 == 0);
  * elems rows x cols/2 bytes (even index low nibble), scales rows x cols/16.
  */
@@ -434,10 +436,8 @@ static unsigned nvfp4_block(const uint16_t *x, int64_t cols, int64_t r0, int64_t
         for (int i = 0; i < B; i++) {
             unsigned q = 0;
             if (d != 0.0f) {
-                volatile float rcp = 1.0f / d;
                 volatile float xi = (float)bf16_value(x[(r0 + rr) * cols + c0 + i]);
-                volatile float y = xi * rcp;
-                if (isnan(y)) y = xi;     /* 0 * Inf when 1/d overflows: keep the signed zero */
+                volatile float y = xi / d;
                 q = mxo_encode((double)y, K_E2M1);
             }
             put_code(elems + (r0 + rr) * (cols / 2), c0 + i, q, 4);
@@ -594,6 +594,48 @@ int mxo_gemm_ref(const uint8_t *a_elems, const uint8_t *a_scales, int a_fmt, dou
         c[p] = acc;
         abs_sum[p] = mag;
     }
+    return 0;
+}
+
+/* The same reference for every entry of the rectangle [m0, m1) x [n0, n1) (c and abs_sum
+ * row-major, (m1 - m0) x (n1 - n0)): the rows involved are decoded once into double
+ * buffers, then each entry is the same k = 0 .. K-1 sum as above. */
+int mxo_gemm_ref_block(const uint8_t *a_elems, const uint8_t *a_scales, int a_fmt, double a_g,
+                       const uint8_t *b_elems, const uint8_t *b_scales, int b_fmt, double b_g,
+                       int64_t M, int64_t N, int64_t K, int64_t m0, int64_t m1, int64_t n0, int64_t n1,
+                       double *c, double *abs_sum, double *a_rows, double *b_rows) {
+    if (K % 32 || m0 < 0 || m1 > M || m0 > m1 || n0 < 0 || n1 > N || n0 > n1) return -1;
+    for (int64_t m = m0; m < m1; m++)
+        for (int64_t k = 0; k < K; k++) a_rows[(m - m0) * K + k] = mx_operand_value(a_elems, a_scales, a_fmt, a_g, m, k, K);
+    for (int64_t n = n0; n < n1; n++)
+        for (int64_t k = 0; k < K; k++) b_rows[(n - n0) * K + k] = mx_operand_value(b_elems, b_scales, b_fmt, b_g, n, k, K);
+    for (int64_t m = m0; m < m1; m++)
+        for (int64_t n = n0; n < n1; n++) {
+            const double *a = a_rows + (m - m0) * K, *b = b_rows + (n - n0) * K;
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                acc += a[k] * b[k];
+                mag += fabs(a[k] * b[k]);
+            }
+            c[(m - m0) * (n1 - n0) + (n - n0)] = acc;
+            abs_sum[(m - m0) * (n1 - n0) + (n - n0)] = mag;
+        }
+    return 0;
+}
+
+/* tcgen05 tiling of a whole row-major scale matrix, and back (plain loops over the offset
+ * function above; padding bytes of `tiled` are written 0). */
+int mxo_to_tcgen05_layout(const uint8_t *rowmajor, int64_t rows, int64_t scale_cols, uint8_t *tiled) {
+    memset(tiled, 0, (size_t)mxo_tcgen05_scale_bytes(rows, scale_cols));
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < scale_cols; c++)
+            tiled[mxo_tcgen05_scale_offset(r, c, rows, scale_cols)] = rowmajor[r * scale_cols + c];
+    return 0;
+}
+int mxo_from_tcgen05_layout(const uint8_t *tiled, int64_t rows, int64_t scale_cols, uint8_t *rowmajor) {
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < scale_cols; c++)
+            rowmajor[r * scale_cols + c] = tiled[mxo_tcgen05_scale_offset(r, c, rows, scale_cols)];
     return 0;
 }
 
@@ -769,7 +811,8 @@ int mxo_quantize_mx_sr(const uint16_t *x, int64_t rows, int64_t cols, int fmt, i
 }
 
 /* NVFP4 with stochastic rounding of the element cast: steps 1-4 of the NVFP4 path, the
- * E2M1 code of x_i * (1/d) rounded stochastically (the UE4M3 block scale stays RNE). */
+ * E2M1 code of the fp32 quotient x_i / d rounded stochastically (the UE4M3 block scale
+ * stays RNE). */
 int mxo_quantize_nvfp4_sr(const uint16_t *x, int64_t rows, int64_t cols, const uint8_t *rnd,
                           uint8_t *elems, uint8_t *scales, float *g_out) {
     const int B = 16;
@@ -796,10 +839,8 @@ int mxo_quantize_nvfp4_sr(const uint16_t *x, int64_t rows, int64_t cols, const u
             for (int i = 0; i < B; i++) {
                 unsigned q = 0;
                 if (d != 0.0f) {
-                    volatile float rcp = 1.0f / d;
                     volatile float xi = (float)bf16_value(blk[i]);
-                    volatile float y = xi * rcp;
-                    if (isnan(y)) y = xi;
+                    volatile float y = xi / d;
                     q = encode_sr((double)y, K_E2M1, rnd[r * cols + b * B + i]);
                 }
                 put_code(elems + r * (cols / 2), b * B + i, q, 4);

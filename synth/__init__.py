@@ -77,3 +77,30 @@ def special_values_block() -> np.ndarray:
     vals = [0x0000, 0x8000, 0x0001, 0x8001, 0x007F, 0x0080, 0x7F7F, 0xFF7F,
             0x3F80, 0xBF80, 0x4300, 0x43E0, 0x43E8, 0x43F0, 0x4760, 0x4770]
     return np.array(vals, dtype=np.uint16)
+
+
+def nvfp4_quotient_grid(amax_bits: int, cols: int = 256, seed: int = 0) -> np.ndarray:
+    """Sixteen-element blocks that sweep the NVFP4 scale and element space for a tensor
+    whose largest magnitude is the bf16 pattern ``amax_bits`` (positive, finite).
+
+    Block maxima run over every bf16 magnitude pattern from ``amax_bits - 19*128`` (19
+    binades down, floored at the smallest subnormal) up to ``amax_bits``; the other 15
+    entries of the blocks led by maximum p take, in turn, every magnitude pattern from
+    ``p - 5*128`` up to p (five binades), with random signs; the last block of each
+    maximum is padded with signed zeros.  Rows of ``cols`` entries (a multiple of 16),
+    zero blocks fill the last row.  Pattern arithmetic only: no scale or codec math.
+    """
+    assert 0 < amax_bits < 0x7F80 and cols % 16 == 0
+    rng = np.random.default_rng(seed)
+    blocks = []
+    for p in range(max(1, amax_bits - 19 * 128), amax_bits + 1):
+        xs = np.arange(max(0, p - 5 * 128), p + 1, dtype=np.uint16)
+        pad = (-xs.size) % 15
+        xs = np.concatenate([xs, np.zeros(pad, dtype=np.uint16)]).reshape(-1, 15)
+        lead = np.full((xs.shape[0], 1), p, dtype=np.uint16)
+        blk = np.concatenate([lead, xs], axis=1)
+        blk |= (rng.integers(0, 2, blk.shape, dtype=np.uint16) << 15).astype(np.uint16)
+        blocks.append(blk)
+    b = np.concatenate(blocks, axis=0).reshape(-1)
+    b = np.concatenate([b, np.zeros((-b.size) % cols, dtype=np.uint16)])
+    return b.reshape(-1, cols)

@@ -221,7 +221,8 @@ def bits_to_finite(bits):
 
 def test_nvfp4_block_scale_is_nearest_ue4m3(oracle):
     """sb is the nearest (ties even) UE4M3 code to amax_b / (6 g), found by brute force,
-    and the elements are the nearest E2M1 of x / d (up to the fp32 product)."""
+    and the elements are the E2M1 codes of the fp32 quotient x / d (numpy's IEEE division;
+    the exhaustive form of this pin is in test_oracle_nvfp4_quotient.py)."""
     x = synth.weight_fp4(32, 256, seed=6)
     e, s, g = oracle.quantize_nvfp4(x)
     ue = np.array([oracle.decode(oracle.K_UE4M3, c) for c in range(0x7F)])
@@ -240,7 +241,7 @@ def test_nvfp4_block_scale_is_nearest_ue4m3(oracle):
             if dd == 0:
                 assert np.all(codes[16 * b:16 * b + 16] == 0)
                 continue
-            scaled = blk * (np.float32(1.0) / dd)
+            scaled = blk / dd
             ref = np.array([oracle.encode(float(v), oracle.K_E2M1) for v in scaled])
             assert np.array_equal(codes[16 * b:16 * b + 16], ref)
             # error bound: half the widest E2M1 spacing (1.0) times d, plus clipping above 6
@@ -353,7 +354,41 @@ def test_gemm_ref_one_hot(oracle):
     assert np.array_equal(c, 3.0 * bdec[:, 70])
 
 
+def test_gemm_ref_block_equals_per_entry_reference(oracle):
+    """The rectangle form (rows decoded once) gives exactly the per-entry sums, for MX,
+    mixed and NVFP4 operands."""
+    M, N, K = 24, 40, 256
+    a = synth.normal(M, K, seed=21)
+    b = synth.weight_fp4(N, K, seed=22)
+    pairs = np.array([(m, n) for m in range(3, 19) for n in range(5, 37)], dtype=np.int64)
+    for fa, fb in ((oracle.E4M3, oracle.E4M3), (oracle.E4M3, oracle.E2M1), (oracle.NVFP4, oracle.NVFP4)):
+        if fa == oracle.NVFP4:
+            ae, as_, ga = oracle.quantize_nvfp4(a)
+            be, bs, gb = oracle.quantize_nvfp4(b)
+        else:
+            (ae, as_), ga = oracle.quantize_mx(a, fa, oracle.ROW, oracle.CEIL), 1.0
+            (be, bs), gb = oracle.quantize_mx(b, fb, oracle.ROW, oracle.FLOOR), 1.0
+        c, mag = oracle.gemm_ref(ae, as_, fa, be, bs, fb, M, N, K, pairs, a_g=ga, b_g=gb)
+        cb, magb = oracle.gemm_ref_block(ae, as_, fa, be, bs, fb, M, N, K, 3, 19, 5, 37, a_g=ga, b_g=gb)
+        assert np.array_equal(cb.reshape(-1), c) and np.array_equal(magb.reshape(-1), mag)
+
+
 # ------------------------------------------------------------------ tcgen05 scale tiling
+def test_tcgen05_whole_matrix_tiling_matches_offsets(oracle):
+    """to/from_tcgen05_layout place every scale at its offset, zero the padding and invert
+    each other."""
+    rng = np.random.default_rng(3)
+    for rows, scols in [(128, 4), (130, 5), (300, 33), (1, 1)]:
+        s = rng.integers(1, 256, (rows, scols), dtype=np.uint8)
+        t = oracle.to_tcgen05_layout(s)
+        off = oracle.tcgen05_offsets(rows, scols)
+        assert np.array_equal(t[off], s)
+        pad = np.ones(t.size, dtype=bool)
+        pad[off.reshape(-1)] = False
+        assert np.all(t[pad] == 0)
+        assert np.array_equal(oracle.from_tcgen05_layout(t, rows, scols), s)
+
+
 def test_tcgen05_tiling_is_a_padded_bijection(oracle):
     for rows, scols in [(128, 4), (256, 8), (130, 5), (1, 1), (300, 33)]:
         off = oracle.tcgen05_offsets(rows, scols)
