@@ -317,6 +317,17 @@ int mx_last_cuda_error(void);
  */
 mx_status mx_watchdog_status(int *code, int clear);
 
+/*
+ * Watchdog self-test (a diagnostic, not part of the pages' method): enqueues on `stream`
+ * one kernel whose single wait -- the same bounded barrier wait the pipelined kernels use
+ * -- is on a barrier that nothing ever arrives at.  After `limit_us` microseconds of
+ * device time (1 .. 100000, else MX_ERR_ARG) the wait gives up, records code 9 in the
+ * watchdog flag and the kernel returns normally: no fault, no trap, the context stays
+ * usable.  mx_watchdog_status then reports MX_ERR_TIMEOUT with *code == 9; clear the flag
+ * before further calls (see above).  Allocates nothing.
+ */
+mx_status mx_watchdog_selftest(uint32_t limit_us, mx_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

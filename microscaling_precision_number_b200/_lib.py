@@ -21,7 +21,9 @@ MX_LAYOUT_ROWMAJOR, MX_LAYOUT_TCGEN05 = 1, 2
 # Every function the header declares (the CPU test checks the library exports them all).
 EXPORTS = ("mx_scale_bytes", "mx_quantize", "mx_quantize_dual", "mx_dequantize", "mx_cast",
            "mx_gemm", "mx_status_string", "mx_last_cuda_error", "mx_watchdog_status",
-           "mx_quantize_nvfp4_noalloc", "mx_mxfp4_to_fp8_blocks", "mx_quantize_nvfp4_2d", "mx_quantize_train")
+           "mx_quantize_nvfp4_noalloc", "mx_mxfp4_to_fp8_blocks", "mx_quantize_nvfp4_2d", "mx_quantize_train",
+           "mx_watchdog_selftest")
+WD_SELFTEST = 9
 MX_NOALLOC_MAX_PARTIALS = 1024
 
 
@@ -68,6 +70,8 @@ def _load():
     lib.mx_last_cuda_error.restype = I
     lib.mx_watchdog_status.argtypes = [ctypes.POINTER(ctypes.c_int), I]
     lib.mx_watchdog_status.restype = I
+    lib.mx_watchdog_selftest.argtypes = [ctypes.c_uint32, P]
+    lib.mx_watchdog_selftest.restype = I
     # NVFP4 quantisation without any device allocation (static scratch array)
     lib.mx_quantize_nvfp4_noalloc.argtypes = [P, I64, I64, P, U8P, I, U8P, P, P]
     lib.mx_quantize_nvfp4_noalloc.restype = I

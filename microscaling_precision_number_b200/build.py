@@ -21,7 +21,7 @@ ROOT = os.path.dirname(PKG)
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmx.so")
 SOURCES = ["api.cu", "stream.cu", "quant.cu", "dual.cu", "gemm.cu", "gemm2.cu", "nested.cu", "train.cu", "noalloc.cu"]
-HEADERS = ["codec.cuh", "ptx.cuh", "tiling.cuh", "umma.cuh", "internal.h"]
+HEADERS = ["codec.cuh", "nvfp4.cuh", "ptx.cuh", "tiling.cuh", "umma.cuh", "internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
          "-I" + os.path.join(ROOT, "include")]

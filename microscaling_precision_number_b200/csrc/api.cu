@@ -126,6 +126,16 @@ mx_status mx_watchdog_status(int *code, int clear) {
     return v ? MX_ERR_TIMEOUT : MX_OK;
 }
 
+mx_status mx_watchdog_selftest(uint32_t limit_us, mx_stream_t stream) {
+    if (limit_us < 1 || limit_us > 100000) return MX_ERR_ARG;
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    const cudaError_t e = mxk::launch_watchdog_selftest((uint64_t)limit_us * 1000ull, d->watchdog,
+                                                        reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? MX_OK : cuda_fail(e);
+}
+
 // One fixed-size scratch per device for the NVFP4 per-CTA partial maxima, allocated on
 // first use (every call writes each slot it later reads).
 static mx_status nvfp4_scratch(DeviceState *d) {

@@ -244,10 +244,5 @@ __device__ __forceinline__ float ue4m3_to_f32(uint32_t code) {
     return lo;
 }
 
-// tcgen05 scale tiling: byte offset of scale (r, c) for an output with S scale columns.
-__device__ __forceinline__ int64_t tcgen05_scale_offset(int64_t r, int64_t c, int64_t S) {
-    int64_t col_atoms = (S + 3) >> 2;
-    return (((r >> 7) * col_atoms + (c >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (c & 3);
-}
 
 }  // namespace mxk

@@ -41,6 +41,8 @@ cudaError_t launch_stream_dequant_nvfp4(const void *elems, const uint8_t *scales
 cudaError_t launch_tcgen05_pad(uint8_t *sc, int64_t rows, int64_t S, cudaStream_t st);
 // Direct element cast (no block scale).
 cudaError_t launch_cast(const void *src, int64_t n, int fmt, void *out, int num_sms, cudaStream_t st);
+// One bounded wait on a barrier nothing arrives at (the watchdog's own test).
+cudaError_t launch_watchdog_selftest(uint64_t limit_ns, int *watchdog, cudaStream_t st);
 
 // ---- dual.cu -------------------------------------------------------------------------------------
 // TMA-staged quantiser producing the row-wise and/or the column-wise (transposed) output.

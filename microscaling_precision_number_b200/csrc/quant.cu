@@ -12,6 +12,7 @@
 // 4 (FP4) bytes.
 #include "codec.cuh"
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace mxk {
 
@@ -50,6 +51,25 @@ cudaError_t launch_tcgen05_pad(uint8_t *sc, int64_t rows, int64_t S, cudaStream_
     int64_t grid = (total + 255) / 256;
     if (grid > 4096) grid = 4096;
     tcgen05_pad_kernel<<<(int)grid, 256, 0, st>>>(sc, rows, S, total);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------------
+// Watchdog self-test: one thread waits, with the library's bounded wait and a short limit,
+// on a shared-memory barrier that expects one arrival and never gets it.  The wait gives
+// up after limit_ns, records WD_SELFTEST in the watchdog flag and the kernel returns; no
+// copy or other asynchronous work is in flight, so nothing needs draining.
+// ---------------------------------------------------------------------------------------
+__global__ void watchdog_selftest_kernel(uint64_t limit_ns, int *watchdog) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    (void)mbar_wait_bounded(&bar, 0u, watchdog, WD_SELFTEST, limit_ns);
+}
+
+cudaError_t launch_watchdog_selftest(uint64_t limit_ns, int *watchdog, cudaStream_t st) {
+    watchdog_selftest_kernel<<<1, 32, 0, st>>>(limit_ns, watchdog);
     return cudaGetLastError();
 }
 

@@ -30,6 +30,7 @@
 
 #include "codec.cuh"
 #include "internal.h"
+#include "nvfp4.cuh"
 #include "ptx.cuh"
 #include "tiling.cuh"
 
@@ -228,39 +229,49 @@ __device__ __forceinline__ uint32_t finite_mask(uint32_t m) {
 // NVFP4 quantisation of one 16 KiB tile (512 blocks of 16; thread = blocks tid, tid+256),
 // read from the shared-memory ring.  g is the per-tensor decode scale.
 //   per block: t = amax_b / (6 g), sb = UE4M3(t) (RNE, saturating), d = dec(sb) g,
-//   q = E2M1(x * (1/d)); a block holding a NaN/Inf gets sb = 0x7F and codes 0.
+//   q = E2M1(RN(x / d)); a block holding a NaN/Inf gets sb = 0x7F and codes 0.
 // ---------------------------------------------------------------------------------------
 // Per-tensor constants of the NVFP4 block math, derived once per CTA from g.
 struct Nvfp4Consts {
     float six_g;      // 6 g (fp32 RN)
     float y;          // RN(1 / six_g)
-    bool fast;        // six_g >= 2^-80: t = amax_b / six_g may use the multiply-and-correct form
+    bool fast;        // six_g >= 2^-80: t = amax_b / six_g may use the corrected quotient
 };
 
-__device__ __forceinline__ Nvfp4Consts nvfp4_consts(float g, float *rtab) {
+// Per-code element divisors: qtab[sb] = {d, -RN(1/d)} with d = RN(dec(sb) g).  The second
+// entry is 0 when d < 2^-100 (the quotients then take the IEEE division) and the code 0x7F
+// (only NaN blocks, whose codes are zero) gets {0, 0}.
+__device__ __forceinline__ Nvfp4Consts nvfp4_consts(float g, float2 *qtab) {
     Nvfp4Consts c;
     c.six_g = __fmul_rn(6.0f, g);
     c.y = __frcp_rn(c.six_g);
     c.fast = c.six_g >= 0x1p-80f;
-    // rtab[sb] = RN(1 / (dec(sb) g)), or 0 when that product is 0 (codes are then 0)
     if (threadIdx.x < 128) {
-        const float d = __fmul_rn(ue4m3_to_f32(threadIdx.x), g);
-        rtab[threadIdx.x] = d != 0.0f ? __frcp_rn(d) : 0.0f;
+        const float d = threadIdx.x < 0x7Fu ? __fmul_rn(ue4m3_to_f32(threadIdx.x), g) : 0.0f;
+        qtab[threadIdx.x] = make_float2(d, d >= kQuotFastMin ? -__frcp_rn(d) : 0.0f);
     }
     __syncthreads();
     return c;
 }
 
-// In the tile function below, t = RN(a / six_g) is formed as q0 = RN(a y),
-// r = a - q0 six_g (exact by FMA), t = RN(q0 + r y) with y = RN(1 / six_g) when FAST.  That
-// equals the correctly rounded quotient whenever a is at least 2^-100 (checked
-// exhaustively over every bf16 numerator for a wide set of divisors); with six_g >= 2^-80
-// every block whose quotient can reach the smallest UE4M3 subnormal has such a numerator,
-// and smaller quotients encode to 0 either way.  Otherwise the IEEE division is used.
+// RN(amax_b / six_g): with FAST, Markstein's corrected quotient from the precomputed
+// reciprocal (q0 = RN(a y), r = a - q0 six_g exact by FMA, t = RN(q0 + r y)).  It is the
+// IEEE quotient for every numerator a >= 2^-100; with six_g >= 2^-80 every block whose
+// quotient can reach the smallest UE4M3 subnormal has such a numerator, and smaller
+// quotients encode to 0 either way.  Otherwise the IEEE division.
+template <bool FAST>
+__device__ __forceinline__ float nvfp4_block_quotient(float a, const Nvfp4Consts &cst) {
+    if constexpr (FAST) {
+        const float q0 = __fmul_rn(a, cst.y);
+        return __fmaf_rn(__fmaf_rn(-q0, cst.six_g, a), cst.y, q0);
+    } else {
+        return __fdiv_rn(a, cst.six_g);
+    }
+}
 
 template <bool RM, bool TC, bool FAST>
 __device__ __forceinline__ void nvfp4_quant_tile(const uint8_t *tile, uint32_t t, uint32_t n_blocks,
-                                                 const Nvfp4Consts &cst, const float *rtab, const FastDiv &divS,
+                                                 const Nvfp4Consts &cst, const float2 *qtab, const FastDiv &divS,
                                                  uint32_t col_atoms, uint8_t *__restrict__ elems,
                                                  uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc) {
     // The thread's two blocks (tid, tid + 256) are processed side by side: the common path
@@ -276,47 +287,29 @@ __device__ __forceinline__ void nvfp4_quant_tile(const uint8_t *tile, uint32_t t
         const uint32_t lb = tid + h * kThreads;
         blk[h] = t * kBlocksPerTile + lb;
         ok[h] = blk[h] < n_blocks;
+        // v[h][j] holds 8-element chunk (j + rot) & 1 of the block (rotated shared-memory
+        // reads); codes are computed per chunk and stored back at the chunk's position
 #pragma unroll
         for (int j = 0; j < 2; j++)
             v[h][j] = ok[h] ? *reinterpret_cast<const uint4 *>(tile + lb * 32 + ((j + rot) & 1u) * 16)
                             : make_uint4(0u, 0u, 0u, 0u);
     }
     uint32_t sb[2], q[2][2];
-    float r[2];
+    float2 dq[2];
     bool special[2];
 #pragma unroll
     for (int h = 0; h < 2; h++) {
         const uint32_t m = absmax_block16(v[h][0], v[h][1]);
         special[h] = m >= 0x7F80u;                           // Inf/NaN in the block
-        const float a = __uint_as_float(m << 16);
-        float tq;
-        if constexpr (FAST) {
-            const float q0 = __fmul_rn(a, cst.y);
-            tq = __fmaf_rn(__fmaf_rn(-q0, cst.six_g, a), cst.y, q0);
-        } else {
-            tq = __fdiv_rn(a, cst.six_g);
-        }
+        const float tq = nvfp4_block_quotient<FAST>(__uint_as_float(m << 16), cst);
         sb[h] = cvt_fp8x2<FMT_E4M3>(tq, 0.0f) & 0xFFu;     // tq >= 0: sign bit stays 0
-        r[h] = rtab[sb[h] & 0x7Fu];                          // RN(1 / (dec(sb) g)), 0 if that is 1/0
+        dq[h] = qtab[sb[h] & 0x7Fu];                         // {d, -RN(1/d)}
     }
 #pragma unroll
     for (int h = 0; h < 2; h++) {
-        const uint64_t r2 = splat2(r[h]);
-#pragma unroll
-        for (int j = 0; j < 2; j++) {
-            float x[8];
-            scale8(v[h][j], r2, x);
-            if (__builtin_expect(isinf(r[h]), 0)) {
-                const float in[8] = {bf16_lo(v[h][j].x), bf16_hi(v[h][j].x), bf16_lo(v[h][j].y), bf16_hi(v[h][j].y),
-                                     bf16_lo(v[h][j].z), bf16_hi(v[h][j].z), bf16_lo(v[h][j].w), bf16_hi(v[h][j].w)};
-#pragma unroll
-                for (int i = 0; i < 8; i++)
-                    if (x[i] != x[i]) x[i] = in[i];                // 0 * Inf: keep the signed zero
-            }
-            q[h][j] = cvt_e2m1x8(x);
-        }
-        if (special[h] || r[h] == 0.0f) q[h][0] = q[h][1] = 0u;    // NaN block, or d = 0: codes 0
-        if (special[h]) sb[h] = 0x7Fu;                               // UE4M3 NaN: the block is NaN
+        nvfp4_codes16(v[h][0], v[h][1], dq[h].x, dq[h].y, q[h][0], q[h][1]);
+        if (special[h] || dq[h].x == 0.0f) q[h][0] = q[h][1] = 0u;   // NaN block, or d = 0: codes 0
+        if (special[h]) sb[h] = 0x7Fu;                                 // UE4M3 NaN: the block is NaN
     }
 #pragma unroll
     for (int h = 0; h < 2; h++) {
@@ -417,7 +410,7 @@ nvfp4_quant_bulk_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fast
     __shared__ float warp_max[kThreads / 32];
     Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
               full, watchdog, src, kTileBytes, (uint64_t)n_blocks * 32};
-    __shared__ float rtab[128];
+    __shared__ float2 qtab[128];
     Nvfp4Consts cst;
     const uint32_t n_tiles = (n_blocks + kTileBytes / 32 - 1) / (kTileBytes / 32);
     // The input is not written by the maximum pass, so the ring starts loading it at once;
@@ -426,11 +419,11 @@ nvfp4_quant_bulk_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fast
         pdl_wait_and_release();
         const float g = nvfp4_global_scale(partials, n_partials, warp_max);
         if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
-        cst = nvfp4_consts(g, rtab);
+        cst = nvfp4_consts(g, qtab);
     };
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
-        if (cst.fast) nvfp4_quant_tile<RM, TC, true>(tile, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
-        else nvfp4_quant_tile<RM, TC, false>(tile, t, n_blocks, cst, rtab, divS, col_atoms, elems, sc_rm, sc_tc);
+        if (cst.fast) nvfp4_quant_tile<RM, TC, true>(tile, t, n_blocks, cst, qtab, divS, col_atoms, elems, sc_rm, sc_tc);
+        else nvfp4_quant_tile<RM, TC, false>(tile, t, n_blocks, cst, qtab, divS, col_atoms, elems, sc_rm, sc_tc);
     }, after_issue);
 }
 
@@ -451,11 +444,11 @@ nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t r
                       float *__restrict__ g_out, uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm,
                       uint8_t *__restrict__ sc_tc) {
     __shared__ float warp_max[kThreads / 32];
-    __shared__ float rtab[128];
+    __shared__ float2 qtab[128];
     pdl_wait_and_release();
     const float g = nvfp4_global_scale(partials, n_partials, warp_max);
     if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
-    const Nvfp4Consts cst = nvfp4_consts(g, rtab);
+    const Nvfp4Consts cst = nvfp4_consts(g, qtab);
     const uint32_t lane = threadIdx.x & 31, par = lane >> 4, c = lane & 15;
     const uint32_t S = cols / 16;                                  // blocks (scale columns) per row
     const uint32_t n_tasks = (rows / 16) * div_strips.d;
@@ -478,36 +471,17 @@ nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t r
         m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
         const bool special = m >= 0x7F80u;                         // Inf/NaN in the block
         const float a = __uint_as_float(m << 16);
-        float tq;
-        if (cst.fast) {
-            const float q0 = __fmul_rn(a, cst.y);
-            tq = __fmaf_rn(__fmaf_rn(-q0, cst.six_g, a), cst.y, q0);
-        } else {
-            tq = __fdiv_rn(a, cst.six_g);
-        }
+        const float tq = cst.fast ? nvfp4_block_quotient<true>(a, cst) : nvfp4_block_quotient<false>(a, cst);
         uint32_t sb = cvt_fp8x2<FMT_E4M3>(tq, 0.0f) & 0xFFu;
-        const float r = rtab[sb & 0x7Fu];
-        const bool zero_codes = special || r == 0.0f;
+        const float2 dq = qtab[sb & 0x7Fu];
+        const bool zero_codes = special || dq.x == 0.0f;
         if (special) sb = 0x7Fu;
-        const uint64_t r2 = splat2(r);
         if (!valid) continue;
 #pragma unroll
         for (int k = 0; k < 8; k++) {
             uint32_t q[2];
-#pragma unroll
-            for (int j = 0; j < 2; j++) {
-                const uint4 u = v[k][j];
-                float x[8];
-                scale8(u, r2, x);
-                if (__builtin_expect(isinf(r), 0)) {
-                    const float in[8] = {bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y),
-                                         bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w)};
-#pragma unroll
-                    for (int i = 0; i < 8; i++)
-                        if (x[i] != x[i]) x[i] = in[i];            // 0 * Inf: keep the signed zero
-                }
-                q[j] = zero_codes ? 0u : cvt_e2m1x8(x);
-            }
+            nvfp4_codes16(v[k][0], v[k][1], dq.x, dq.y, q[0], q[1]);
+            if (zero_codes) q[0] = q[1] = 0u;
             const uint32_t row = rb * 16 + 2 * k + par;
             reinterpret_cast<uint2 *>(elems)[((size_t)row * cols + (size_t)cb * 16) >> 4] = make_uint2(q[0], q[1]);
             if constexpr (RM) sc_rm[(size_t)row * S + cb] = (uint8_t)sb;

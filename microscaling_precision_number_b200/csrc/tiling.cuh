@@ -59,12 +59,37 @@ __device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
 __device__ __forceinline__ void unpack2(uint64_t v, float &lo, float &hi) {
     asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
 }
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
 // Eight bf16 (one uint4) times a scalar, as eight fp32 (element i in x[i]).
 __device__ __forceinline__ void scale8(const uint4 &v, uint64_t s2, float (&x)[8]) {
     unpack2(mul2(bf16x2_to_f32x2(v.x), s2), x[0], x[1]);
     unpack2(mul2(bf16x2_to_f32x2(v.y), s2), x[2], x[3]);
     unpack2(mul2(bf16x2_to_f32x2(v.z), s2), x[4], x[5]);
     unpack2(mul2(bf16x2_to_f32x2(v.w), s2), x[6], x[7]);
+}
+
+// Eight bf16 (one uint4) divided by d, returned NEGATED: x[i] = -RN(v_i / d), the
+// correctly rounded fp32 quotient, with nr2 = -RN(1/d) and d2 = d in both lanes.
+// Markstein's FMA-corrected quotient (P. Markstein, "Computation of elementary functions
+// on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34(1), 1990): with y = RN(1/d)
+// and q = RN(v y), the remainder e = v - q d is exact in one FMA and RN(q + e y) is the
+// IEEE quotient, provided no step underflows -- the caller guarantees d >= 2^-100 and
+// needs the exact quotient only where it is >= 1/8, i.e. for |v| >= 2^-103.  Working with
+// -q (q' = RN(-v y), e = RN(q' d + v), result RN(e (-y) + q')) keeps the sign of a zero v,
+// which the positive form would lose in e; callers flip the sign back on the codes.
+__device__ __forceinline__ void neg_quotient8(const uint4 &v, uint64_t nr2, uint64_t d2, float (&x)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint64_t X = bf16x2_to_f32x2(w[i]);
+        const uint64_t Q = mul2(X, nr2);
+        const uint64_t E = fma2(Q, d2, X);
+        unpack2(fma2(E, nr2, Q), x[2 * i], x[2 * i + 1]);
+    }
 }
 
 // ---- packed bf16 block maximum ------------------------------------------------------------

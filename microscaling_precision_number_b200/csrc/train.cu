@@ -21,6 +21,7 @@
 // (coalesced), grid-stride loops; NVFP4 takes a maximum pass and a quantisation pass.
 #include "codec.cuh"
 #include "internal.h"
+#include "nvfp4.cuh"
 #include "ptx.cuh"
 #include "tiling.cuh"
 
@@ -197,8 +198,8 @@ nvfp4_train_amax_kernel(const uint8_t *__restrict__ src, uint32_t n_groups, uint
 }
 
 // Pass 2: g from the partial maxima, then one thread per 16-element block.  The block
-// scale and the quotient follow the RNE path's fp32 steps (t = amax_b / (6 g) by IEEE
-// division, r = 1 / (dec(sb) g)); the element cast is RNE or stochastic.
+// scale and the quotient follow the RNE path's fp32 steps (t = amax_b / (6 g) and
+// RN(x / (dec(sb) g)), both correctly rounded); the element cast is RNE or stochastic.
 template <bool RM, bool TC, bool RHT, bool SR>
 __global__ void __launch_bounds__(kTrainThreads)
 nvfp4_train_quant_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
@@ -229,26 +230,17 @@ nvfp4_train_quant_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fas
         const bool special = m >= 0x7F80u;
         const float tq = __fdiv_rn(__uint_as_float(m << 16), six_g);
         uint32_t sb = cvt_fp8x2<FMT_E4M3>(tq, 0.0f) & 0xFFu;
-        const float d = __fmul_rn(ue4m3_to_f32(sb & 0x7Fu), g);
-        const float r = d != 0.0f ? __frcp_rn(d) : 0.0f;
+        const float d = special ? 0.0f : __fmul_rn(ue4m3_to_f32(sb & 0x7Fu), g);
+        const float nr = d >= kQuotFastMin ? -__frcp_rn(d) : 0.0f;
         const bool zero_codes = special || d == 0.0f;
         if (special) sb = 0x7Fu;
-        const uint64_t r2 = splat2(r);
         uint32_t q[2];
-#pragma unroll
-        for (int j = 0; j < 2; j++) {
-            float x[8];
-            scale8(v[j], r2, x);
-            if (__builtin_expect(isinf(r), 0)) {
-                const float in[8] = {bf16_lo(v[j].x), bf16_hi(v[j].x), bf16_lo(v[j].y), bf16_hi(v[j].y),
-                                     bf16_lo(v[j].z), bf16_hi(v[j].z), bf16_lo(v[j].w), bf16_hi(v[j].w)};
-#pragma unroll
-                for (int i = 0; i < 8; i++)
-                    if (x[i] != x[i]) x[i] = in[i];                    // 0 * Inf: keep the signed zero
-            }
-            round8<FMT_E2M1, SR>(x, rnd + (size_t)blk * 16 + 8 * j);
-            q[j] = zero_codes ? 0u : cvt_e2m1x8(x);
-        }
+        const uint8_t *rb = rnd + (size_t)blk * 16;
+        // the quotients arrive negated; stochastic rounding is odd-symmetric, so it
+        // commutes with the sign flip applied to the codes
+        nvfp4_codes16(v[0], v[1], d, nr, q[0], q[1],
+                      [&](float (&x)[8], int j) { round8<FMT_E2M1, SR>(x, rb + 8 * j); });
+        if (zero_codes) q[0] = q[1] = 0u;
         reinterpret_cast<uint2 *>(elems)[blk] = make_uint2(q[0], q[1]);
         if constexpr (RM) sc_rm[blk] = (uint8_t)sb;
         if constexpr (TC) {

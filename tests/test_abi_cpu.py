@@ -196,3 +196,10 @@ def test_missing_library_fails_loudly(tmp_path):
     env = dict(os.environ, MX_LIB_PATH=str(tmp_path / "absent" / "libmx.so"))
     out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert "import-error" in out.stdout and "refused-cpu-tensor" in out.stdout, out.stdout + out.stderr
+
+
+@pytest.mark.parametrize("limit_us", [0, 100001, 2 ** 32 - 1])
+def test_watchdog_selftest_rejects_limits(L, limit_us):
+    """The watchdog self-test takes a limit of 1 .. 100000 microseconds; anything else is
+    rejected before any CUDA call."""
+    assert L.lib.mx_watchdog_selftest(limit_us, None) == L.MX_ERR_ARG

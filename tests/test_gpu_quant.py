@@ -231,38 +231,6 @@ def test_weight_4096x4096_full(oracle):
     assert np.array_equal(host(qn.scales_alt), oracle.to_tcgen05_layout(s_ref))
 
 
-@pytest.mark.parametrize("which", ["activations", "gradients"])
-def test_dual_full_size_sampled(oracle, which):
-    """Full-size dual quantisation in the benchmark's launch configuration; sampled
-    32 x 128 tiles checked against the oracle (blocks are independent)."""
-    if which == "activations":
-        x, fmt = synth.activations(), oracle.E4M3
-    else:
-        x, fmt = synth.gradients(), oracle.E5M2
-    R, C = x.shape
-    qr, qc = mx.quantize_dual(to_dev(x), FMT_NAMES[fmt], "ceil", "tcgen05")
-    re_, rs = host(qr.elems).reshape(R, C), host(qr.scales)
-    ce, cs = host(qc.elems).reshape(C, R), host(qc.scales)
-    rng = np.random.default_rng(0)
-    for _ in range(24):
-        r0 = int(rng.integers(0, R // 32)) * 32
-        c0 = int(rng.integers(0, C // 128)) * 128
-        tile = np.ascontiguousarray(x[r0:r0 + 32, c0:c0 + 128])
-        er, sr = oracle.quantize_mx(tile, fmt, oracle.ROW, oracle.CEIL)
-        ec, sc = oracle.quantize_mx(tile, fmt, oracle.COL, oracle.CEIL)
-        assert np.array_equal(re_[r0:r0 + 32, c0:c0 + 128], er)
-        assert np.array_equal(ce[c0:c0 + 128, r0:r0 + 32], ec)
-        for i in range(32):
-            for b in range(4):
-                off = oracle.lib().mxo_tcgen05_scale_offset(r0 + i, c0 // 32 + b, R, C // 32)
-                assert rs[off] == sr[i, b]
-        for j in range(128):
-            off = oracle.lib().mxo_tcgen05_scale_offset(c0 + j, r0 // 32, C, R // 32)
-            assert cs[off] == sc[j, 0]
-    del qr, qc
-    torch.cuda.empty_cache()
-
-
 def test_empty_inputs_launch_nothing():
     x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
     q = mx.quantize(x, "e4m3", "row", "ceil")

@@ -20,6 +20,14 @@ import synth
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(autouse=True)
+def _no_watchdog():
+    """No bounded device wait gave up during the test (the flag is read and cleared)."""
+    yield
+    from microscaling_precision_number_b200 import api
+    assert api.watchdog_status(clear=True) == 0
+
+
 def _dev_bf16(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
 
