@@ -3,22 +3,25 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-breakdown]
 
-One step = one pass of the weight-quantisation workload over a 4096 x 4096 bf16 matrix
-(N(0, 0.02) with 0.1% N(0, 1) outliers): MXFP4 (E2M1, block 32, E8M0, floor scale) and
-NVFP4 (E2M1, block 16, UE4M3 + fp32 tensor scale), each emitting both the row-major and
-the tcgen05 scale layouts.  value = algorithmic bytes of the step / step time (GB/s).
-The input (32 MiB) is smaller than L2, so consecutive steps rotate over 8 copies of the
-weight (256 MiB): each step reads its input from HBM.  K steps are timed back to back in
-one CUDA-event pair.  Every other row of the hot path (row-wise
-MXFP8 quantise + dequantise, dual-orientation quantisation, dequantisation, the two
-block-scaled matmuls) is measured in "breakdown", each against its own roofline.
+One step = dual-orientation MXFP8 quantisation (row-wise and column-wise from one read,
+E8M0 scales in the tcgen05 tiling, no-clip scale rule) of the training workload's two
+tensors: the 16384 x 4096 bf16 activations (N(0,1) times a per-channel 2^v, v ~ U[-4, 4])
+in E4M3, and the 16384 x 14336 bf16 gradients (N(0, 1e-3), 5% exact zeros) in E5M2.
+value = algorithmic bytes of the step (read the input once, write both codes and scales
+once: 1,226,833,920 B) / step time (GB/s).  The inputs (604 MB) exceed L2, so consecutive
+steps read HBM without a flush.  K steps are timed back to back in one CUDA-event pair.
+Every other row of the hot path (the 1024^2 MXFP8 quantise + dequantise, the 4096^2 MXFP4
++ NVFP4 weight quantisation, dequantisation, the block-scaled matmuls and the extension
+rows) is measured in "breakdown", each against its own roofline.
 
-Multi-GPU (torchrun): every rank quantises its own weight matrix (independent units, no
+Multi-GPU (torchrun): every rank quantises its own tensors (independent units, no
 data-path collective); value = all ranks' bytes / the slowest rank's time.
 """
 from __future__ import annotations
 
 import argparse
+import concurrent.futures as cf
+import hashlib
 import json
 import os
 import statistics
@@ -39,14 +42,34 @@ HBM_NOMINAL_GBS = 8000.0
 MX_NOMINAL_TFLOPS = 4500.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# algorithmic bytes (read input once + write codes and scales once)
+# the training workload: dual-orientation MXFP8 of activations (E4M3) and gradients (E5M2)
+ACT = (16384, 4096)
+GRAD = (16384, 14336)
+
+
+def dual_bytes(R, C):
+    """Read the bf16 input once; write row-wise and column-wise FP8 codes and E8M0 scales."""
+    return R * C * 2 + 2 * (R * C + R * C // 32)
+
+
+BYTES_ACT = dual_bytes(*ACT)           # 272,629,760
+BYTES_GRAD = dual_bytes(*GRAD)         # 954,204,160
+STEP_BYTES = BYTES_ACT + BYTES_GRAD    # 1,226,833,920
+WORKLOAD = "dual_mxfp8_act_16384x4096_e4m3_and_grad_16384x14336_e5m2_tcgen05_scales"
+
+# DRAM bytes (read + write) of one quant_dual_kernel launch on the gradients, from an ncu
+# capture of the benchmark's own back-to-back sequence (no cache control, no clock
+# control), and the SHA-256 of the kernel source that capture ran: when dual.cu has
+# changed since, the traffic is reported as null.
+NCU_TRAFFIC_GRAD = None
+NCU_TRAFFIC_SRC_SHA = None
+DUAL_SRC = os.path.join(ROOT, "microscaling_precision_number_b200", "csrc", "dual.cu")
+
+# the 4096 x 4096 weight: MXFP4 (floor) + NVFP4, both scale layouts (a breakdown row)
 R2 = C2 = 4096
 BYTES_MXFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 32)            # 42,991,616
 BYTES_NVFP4 = R2 * C2 * 2 + R2 * C2 // 2 + 2 * (R2 * C2 // 16) + 4         # 44,040,196
-NCU_TRAFFIC_NVFP4 = 67149056      # dram read + write bytes of one NVFP4 call (both kernels, ncu, L2 flushed per kernel)
-NCU_TRAFFIC_MXFP4 = 33568768      # same for mx_rows_kernel<E2M1, floor, both layouts>
-STEP_BYTES = BYTES_MXFP4 + BYTES_NVFP4
-NROT = 8                 # rotating copies of the weight (8 x 32 MiB > 2 x L2)
+NROT = 8                 # rotating copies of the 32 MiB weight (8 x 32 MiB > 2 x L2)
 
 
 def peaks():
@@ -59,6 +82,11 @@ def peaks():
                 "source": "measured"}
     except Exception:
         return dict(FALLBACK, source="fallback")
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
 
 
 # ----------------------------------------------------------------------------- utilities
@@ -147,39 +175,41 @@ def event_pair():
 
 
 # ----------------------------------------------------------------------------- our step
-class WeightQuantStep:
-    """MXFP4 (floor) + NVFP4 quantisation of one 4096 x 4096 bf16 weight, both layouts."""
+class DualStep:
+    """Dual-orientation MXFP8 quantisation of the activations (E4M3) and the gradients
+    (E5M2) through the C ABI, tcgen05-tiled scales, no-clip rule."""
 
-    def __init__(self, mx, x_dev):
+    def __init__(self, mx, x_act, x_grad):
         from microscaling_precision_number_b200 import _lib as L
-        self.mx, self.L = mx, L
-        self.x = x_dev
-        dev = x_dev.device
-        R, C = x_dev.shape
-        self.R, self.C = R, C
-        self.e4 = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
-        self.s4 = torch.empty(R * C // 32, dtype=torch.uint8, device=dev)
-        self.s4t = torch.empty(mx.scale_bytes(R, C // 32, "tcgen05"), dtype=torch.uint8, device=dev)
-        self.en = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
-        self.sn = torch.empty(R * C // 16, dtype=torch.uint8, device=dev)
-        self.snt = torch.empty(mx.scale_bytes(R, C // 16, "tcgen05"), dtype=torch.uint8, device=dev)
-        self.g = torch.empty(1, dtype=torch.float32, device=dev)
-        self.launches_per_step = 3      # MXFP4 quantiser; NVFP4 maximum + quantiser (no padding at 4096)
+        self.L = L
+        self.parts = []
+        for x, fmt in ((x_act, L.MX_FMT_E4M3), (x_grad, L.MX_FMT_E5M2)):
+            R, C = x.shape
+            dev = x.device
+            o = dict(x=x, R=R, C=C, fmt=fmt,
+                     re=torch.empty(R * C, dtype=torch.uint8, device=dev),
+                     rs=torch.empty(mx.scale_bytes(R, C // 32, "tcgen05"), dtype=torch.uint8, device=dev),
+                     ce=torch.empty(R * C, dtype=torch.uint8, device=dev),
+                     cs=torch.empty(mx.scale_bytes(C, R // 32, "tcgen05"), dtype=torch.uint8, device=dev))
+            self.parts.append(o)
+        self.launches_per_step = 2
 
-    def mxfp4(self, stream):
-        L = self.L
-        L.check(L.lib.mx_quantize(self.x.data_ptr(), self.R, self.C, L.MX_FMT_E2M1, L.MX_AXIS_ROW,
-                                  L.MX_SCALE_FLOOR_OCP, self.e4.data_ptr(), self.s4.data_ptr(), 3,
-                                  self.s4t.data_ptr(), None, stream), "mx_quantize(mxfp4)")
+    def run_part(self, i, stream):
+        L, o = self.L, self.parts[i]
+        L.check(L.lib.mx_quantize_dual(o["x"].data_ptr(), o["R"], o["C"], o["fmt"], L.MX_SCALE_CEIL_RECIPE,
+                                       o["re"].data_ptr(), o["rs"].data_ptr(), o["ce"].data_ptr(),
+                                       o["cs"].data_ptr(), L.MX_LAYOUT_TCGEN05, None, None, stream),
+                "mx_quantize_dual")
 
-    def nvfp4(self, stream):
-        L = self.L
-        L.check(L.lib.mx_quantize(self.x.data_ptr(), self.R, self.C, L.MX_FMT_NVFP4, L.MX_AXIS_ROW,
-                                  L.MX_SCALE_CEIL_RECIPE, self.en.data_ptr(), self.sn.data_ptr(), 3,
-                                  self.snt.data_ptr(), self.g.data_ptr(), stream), "mx_quantize(nvfp4)")
+    def run(self, stream):
+        self.run_part(0, stream)
+        self.run_part(1, stream)
+
+    def inputs(self):
+        return [o["x"] for o in self.parts]
 
     def outputs(self):
-        return [self.e4, self.s4, self.s4t, self.en, self.sn, self.snt, self.g]
+        return [o[k] for o in self.parts for k in ("re", "rs", "ce", "cs")]
 
 
 def run_ours(args, rank, world, dev):
@@ -189,29 +219,23 @@ def run_ours(args, rank, world, dev):
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
     sptr = stream.cuda_stream
-    x_bits = synth.weight_fp4(seed=rank)
-    x0 = to_dev(x_bits, dev)
-    # NROT copies of the weight (8 x 32 MiB, over twice L2): step k works on copy k % NROT,
-    # so every timed step reads its input from HBM without an L2 flush in between.
-    steps = [WeightQuantStep(mx, x0.clone()) for _ in range(NROT)]
+    a_bits = synth.activations(seed=rank)
+    g_bits = synth.gradients(seed=rank + 1)
+    step = DualStep(mx, to_dev(a_bits, dev), to_dev(g_bits, dev))
 
-    def run_steps(n, which="both"):
-        for k in range(n):
-            s = steps[k % NROT]
-            if which in ("both", "mxfp4"):
-                s.mxfp4(sptr)
-            if which in ("both", "nvfp4"):
-                s.nvfp4(sptr)
+    def run_steps(n):
+        for _ in range(n):
+            step.run(sptr)
 
-    run_steps(max(args.warmup, NROT))
+    run_steps(args.warmup)
     torch.cuda.synchronize()
 
     with ClockSampler(torch.cuda.current_device()) as clk:
-        # soak: keep the GPU busy with the same steps for ~0.4 s so that the clock samples
+        # soak: keep the GPU busy with the same steps for ~0.5 s so that the clock samples
         # below see it under load, then the timed region proper
         t0 = time.perf_counter()
-        while time.perf_counter() - t0 < 0.4:
-            run_steps(200)
+        while time.perf_counter() - t0 < 0.5:
+            run_steps(10)
             torch.cuda.synchronize()
         e0, e1 = event_pair()
         if world > 1:
@@ -227,49 +251,83 @@ def run_ours(args, rank, world, dev):
     ms_per_step = total_ms / args.steps
     value = job_throughput_gbs(STEP_BYTES, args.steps, world, total_ms)
 
-    # per-call durations for the roofline: many launches of one call per event pair
-    ncall = max(args.steps, 50)
+    # the dominant kernel's launch duration: the gradient dual call, back to back on the
+    # launching stream (inputs larger than L2)
+    ncall = max(args.steps, 20)
     per = {}
-    for which in ("mxfp4", "nvfp4"):
-        run_steps(NROT, which)
+    for i, name in ((0, "act"), (1, "grad")):
+        step.run_part(i, sptr)
         a, b = event_pair()
         a.record(stream)
-        run_steps(ncall, which)
+        for _ in range(ncall):
+            step.run_part(i, sptr)
         b.record(stream)
         torch.cuda.synchronize()
-        per[which] = a.elapsed_time(b) / ncall
-    mean_mx, mean_nv = per["mxfp4"], per["nvfp4"]
-    # DRAM bytes per call (read + write) from one ncu capture of the same kernels on this
-    # workload (profiles/nvfp4_and_rows_weight4096.md); ncu replays each launch with a
-    # flushed L2, so a kernel's outputs are still in L2 at its end and count as 0 written
-    # bytes
-    if mean_nv >= mean_mx:
-        dom = {"kernel": "mx_quantize(NVFP4) call: nvfp4_amax_bulk_kernel + nvfp4_quant_bulk_kernel<both layouts>",
-               "ms": mean_nv,
-               "bytes": BYTES_NVFP4, "traffic": NCU_TRAFFIC_NVFP4}
-    else:
-        dom = {"kernel": "mx_quantize(MXFP4): mx_rows_kernel<E2M1,floor,both layouts>", "ms": mean_mx,
-               "bytes": BYTES_MXFP4, "traffic": NCU_TRAFFIC_MXFP4}
-    achieved = dom["bytes"] / (dom["ms"] * 1e-3) / 1e9
+        per[name] = a.elapsed_time(b) / ncall
+    achieved = BYTES_GRAD / (per["grad"] * 1e-3) / 1e9
+    traffic = NCU_TRAFFIC_GRAD if (NCU_TRAFFIC_SRC_SHA is not None and file_sha(DUAL_SRC) == NCU_TRAFFIC_SRC_SHA) \
+        else None
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": dom["traffic"],
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
                 "peak_source": pk["source"] + " copy bandwidth (MEASURED_PEAKS hbm_gbs), burst",
-                "kernel": dom["kernel"], "algorithmic_bytes_per_launch": dom["bytes"],
-                "ms_per_launch": round(dom["ms"], 5),
-                "calls": {"mxfp4_ms": round(mean_mx, 5), "mxfp4_GBps": round(BYTES_MXFP4 / mean_mx / 1e6, 1),
-                          "nvfp4_ms": round(mean_nv, 5), "nvfp4_GBps": round(BYTES_NVFP4 / mean_nv / 1e6, 1),
-                          "launches_timed": ncall},
+                "kernel": "quant_dual_kernel<E5M2, no-clip, tcgen05 scales> (mx_quantize_dual on the gradients)",
+                "algorithmic_bytes_per_launch": BYTES_GRAD, "ms_per_launch": round(per["grad"], 5),
+                "launches_timed": ncall,
+                "calls": {"act_ms": round(per["act"], 5), "act_GBps": round(BYTES_ACT / per["act"] / 1e6, 1),
+                          "act_frac": round(BYTES_ACT / per["act"] / 1e6 / pk["hbm_gbs"], 4),
+                          "grad_ms": round(per["grad"], 5), "grad_GBps": round(BYTES_GRAD / per["grad"] / 1e6, 1)},
                 "frac_of_nominal_8TBps": round(achieved / HBM_NOMINAL_GBS, 4)}
 
-    # end to end through the public API with host buffers (pinned), copies inside the timing.
-    # Pipelined as a user would run a stream of weights: step k's upload, step k-1's
-    # quantisation and step k-2's download overlap on three streams (two buffer sets,
-    # ordered by events); the serial form (upload, quantise, download on one stream) is
-    # reported beside it.
-    sets = steps[:2]
-    x_host = torch.from_numpy(x_bits.view(np.int16)).view(torch.bfloat16).pin_memory()
+    e2e = run_e2e(args, step, world, dev, stream, sptr, a_bits, g_bits)
+
+    breakdown = None
+    if not args.no_breakdown and rank == 0:
+        del step
+        torch.cuda.empty_cache()
+        breakdown = run_breakdown(mx, dev, pk, cpu=(world == 1 and not args.no_cpu_baseline))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(a_bits, g_bits, target_s=args.cpu_seconds)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (numpy default_rng; activations seed = rank, gradients seed = rank + 1)",
+                "config": {"workload": WORKLOAD,
+                           "tensors": {"activations": {"shape": list(ACT), "format": "MXFP8 E4M3",
+                                                       "bytes": BYTES_ACT},
+                                       "gradients": {"shape": list(GRAD), "format": "MXFP8 E5M2",
+                                                     "bytes": BYTES_GRAD}},
+                           "orientations": "row-wise and column-wise (transposed) from one read",
+                           "scale_rule": "no-clip (ceil), E8M0, block 32", "scale_layout": "tcgen05",
+                           "step_bytes": STEP_BYTES,
+                           "l2": "inputs larger than L2 (604 MB per step), no flush needed",
+                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": step_launches(args.steps), "clocks": clk.summary()}
+        if breakdown is not None:
+            line["breakdown"] = breakdown
+        print(json.dumps(line), flush=True)
+
+
+def step_launches(steps):
+    return 2 * steps                   # one quant_dual_kernel launch per tensor
+
+
+def run_e2e(args, step, world, dev, stream, sptr, a_bits, g_bits):
+    """The same step through the C ABI with host buffers: every step uploads both bf16
+    inputs from pinned host memory and downloads all codes and scales.  Pipelined as a
+    stream of training steps would run: the upload of step k, the quantisation of step k-1
+    and the download of step k-2 overlap on three streams, with two device buffer sets
+    ordered by events; the serial form (upload, quantise, download on one stream) is
+    reported beside it."""
+    import microscaling_precision_number_b200 as mx
+    sets = [step, DualStep(mx, torch.empty_like(step.parts[0]["x"]), torch.empty_like(step.parts[1]["x"]))]
+    x_host = [torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).pin_memory() for b in (a_bits, g_bits)]
     outs_host = [[torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in st.outputs()] for st in sets]
-    h2d = x_host.numel() * 2
+    h2d = sum(x.numel() * 2 for x in x_host)
     d2h = sum(o.numel() * o.element_size() for o in outs_host[0])
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
     ev_up, ev_comp, ev_down = ([torch.cuda.Event() for _ in sets] for _ in range(3))
@@ -280,12 +338,12 @@ def run_ours(args, rank, world, dev):
             st = sets[b]
             up.wait_event(ev_comp[b])                  # the buffer's previous step has read it
             with torch.cuda.stream(up):
-                st.x.copy_(x_host, non_blocking=True)
+                for d, h in zip(st.inputs(), x_host):
+                    d.copy_(h, non_blocking=True)
             ev_up[b].record(up)
             stream.wait_event(ev_up[b])
             stream.wait_event(ev_down[b])              # its previous outputs have been copied out
-            st.mxfp4(sptr)
-            st.nvfp4(sptr)
+            st.run(sptr)
             ev_comp[b].record(stream)
             down.wait_event(ev_comp[b])
             with torch.cuda.stream(down):
@@ -296,9 +354,9 @@ def run_ours(args, rank, world, dev):
     def serial(n):
         st = sets[0]
         for _ in range(n):
-            st.x.copy_(x_host, non_blocking=True)
-            st.mxfp4(sptr)
-            st.nvfp4(sptr)
+            for d, h in zip(st.inputs(), x_host):
+                d.copy_(h, non_blocking=True)
+            st.run(sptr)
             for h, d in zip(outs_host[0], st.outputs()):
                 h.copy_(d, non_blocking=True)
 
@@ -320,38 +378,54 @@ def run_ours(args, rank, world, dev):
 
     e2e_ms = timed_e2e(pipelined)
     ser_ms = timed_e2e(serial)
-    e2e = {"value": round(job_throughput_gbs(STEP_BYTES, args.steps, world, e2e_ms), 2), "unit": "GB/s",
+    out = {"value": round(job_throughput_gbs(STEP_BYTES, args.steps, world, e2e_ms), 2), "unit": "GB/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": round(e2e_ms / args.steps, 4),
            "form": "pipelined: upload / quantise / download of consecutive steps overlap on three streams",
            "serial": {"value": round(job_throughput_gbs(STEP_BYTES, args.steps, world, ser_ms), 2),
-                      "ms_per_step": round(ser_ms / args.steps, 4)}}
+                      "ms_per_step": round(ser_ms / args.steps, 4)},
+           "note": "host<->device copies over PCIe bound this number"}
+    del sets[1], outs_host, x_host
+    return out
 
-    breakdown = None
-    if not args.no_breakdown and rank == 0:
-        breakdown = run_breakdown(mx, dev, pk)
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(x_bits, target_s=args.cpu_seconds)
+class WeightQuantStep:
+    """MXFP4 (floor) + NVFP4 quantisation of one 4096 x 4096 bf16 weight, both layouts."""
 
-    if rank == 0:
-        line = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-                "data": "synthetic (numpy default_rng, seed = rank)",
-                "config": {"workload": "weight_4096x4096_mxfp4_floor_and_nvfp4_both_scale_layouts",
-                           "shape": [R2, C2], "formats": ["MXFP4 E2M1/E8M0 floor block 32",
-                                                          "NVFP4 E2M1/UE4M3+fp32 block 16"],
-                           "step_bytes": STEP_BYTES,
-                           "l2": f"inputs larger than L2: steps rotate over {NROT} copies of the weight "
-                                 f"({NROT * R2 * C2 * 2 >> 20} MiB)",
-                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": steps[0].launches_per_step * args.steps, "clocks": clk.summary()}
-        if breakdown is not None:
-            line["breakdown"] = breakdown
-        print(json.dumps(line), flush=True)
+    def __init__(self, mx, x_dev):
+        from microscaling_precision_number_b200 import _lib as L
+        self.mx, self.L = mx, L
+        self.x = x_dev
+        dev = x_dev.device
+        R, C = x_dev.shape
+        self.R, self.C = R, C
+        self.e4 = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
+        self.s4 = torch.empty(R * C // 32, dtype=torch.uint8, device=dev)
+        self.s4t = torch.empty(mx.scale_bytes(R, C // 32, "tcgen05"), dtype=torch.uint8, device=dev)
+        self.en = torch.empty(R * C // 2, dtype=torch.uint8, device=dev)
+        self.sn = torch.empty(R * C // 16, dtype=torch.uint8, device=dev)
+        self.snt = torch.empty(mx.scale_bytes(R, C // 16, "tcgen05"), dtype=torch.uint8, device=dev)
+        self.g = torch.empty(1, dtype=torch.float32, device=dev)
+
+    def mxfp4(self, stream):
+        L = self.L
+        L.check(L.lib.mx_quantize(self.x.data_ptr(), self.R, self.C, L.MX_FMT_E2M1, L.MX_AXIS_ROW,
+                                  L.MX_SCALE_FLOOR_OCP, self.e4.data_ptr(), self.s4.data_ptr(), 3,
+                                  self.s4t.data_ptr(), None, stream), "mx_quantize(mxfp4)")
+
+    def nvfp4(self, stream):
+        L = self.L
+        L.check(L.lib.mx_quantize(self.x.data_ptr(), self.R, self.C, L.MX_FMT_NVFP4, L.MX_AXIS_ROW,
+                                  L.MX_SCALE_CEIL_RECIPE, self.en.data_ptr(), self.sn.data_ptr(), 3,
+                                  self.snt.data_ptr(), self.g.data_ptr(), stream), "mx_quantize(nvfp4)")
+
+    def both(self, stream):
+        """Both encodings in one call (the MX pass supplies the NVFP4 tensor maximum)."""
+        L = self.L
+        L.check(L.lib.mx_quantize_mx_nvfp4(self.x.data_ptr(), self.R, self.C, L.MX_FMT_E2M1, L.MX_SCALE_FLOOR_OCP,
+                                           self.e4.data_ptr(), self.s4.data_ptr(), 3, self.s4t.data_ptr(),
+                                           self.en.data_ptr(), self.sn.data_ptr(), 3, self.snt.data_ptr(),
+                                           self.g.data_ptr(), stream), "mx_quantize_mx_nvfp4")
 
 
 # ----------------------------------------------------------------------------- breakdown
@@ -396,7 +470,7 @@ def soak_clocks(fn, seconds=1.5):
     return clk.summary()
 
 
-def run_breakdown(mx, dev, pk):
+def run_breakdown(mx, dev, pk, cpu=False):
     stream = torch.cuda.current_stream()
     out = {}
     hbm = pk["hbm_gbs"]
@@ -453,21 +527,29 @@ def run_breakdown(mx, dev, pk):
                                  "nvfp4_GBps": round(bdn / tn / 1e6, 1), "nvfp4_frac_hbm": round(bdn / tn / 1e6 / hbm, 4)}
     del xw, q4, qn, ys
 
-    # C3: dual-orientation MXFP8, activations (E4M3) and gradients (E5M2), tcgen05 scales
-    for name, gen, fmt in (("act_16384x4096_e4m3", synth.activations, "e4m3"),
-                           ("grad_16384x14336_e5m2", synth.gradients, "e5m2")):
-        xb = gen()
-        R, C = xb.shape
-        x3 = to_dev(xb, dev)
-        del xb
-        o3 = mx.quantize_dual(x3, fmt, "ceil", "tcgen05")
-        t = timed([lambda: mx.quantize_dual(x3, fmt, "ceil", "tcgen05", out=o3)], 20, stream)
-        nbytes = R * C * 2 + 2 * (R * C + R * C // 32)
-        out[f"dual_{name}"] = {"ms": round(t, 4), "GBps": round(nbytes / t / 1e6, 1),
-                                  "frac_hbm": round(nbytes / t / 1e6 / hbm, 4), "algorithmic_bytes": nbytes,
-                                  "l2": "input larger than L2"}
-        del x3, o3
-        torch.cuda.empty_cache()
+    # the 4096 x 4096 weight: MXFP4 (floor) and NVFP4, both scale layouts, each call on
+    # eight rotating copies (256 MiB > L2); one step = both calls
+    xw0 = to_dev(synth.weight_fp4(), dev)
+    wsteps = [WeightQuantStep(mx, xw0.clone()) for _ in range(NROT)]
+    sptr = stream.cuda_stream
+    t4 = timed([lambda s=s: s.mxfp4(sptr) for s in wsteps], 64, stream)
+    tn = timed([lambda s=s: s.nvfp4(sptr) for s in wsteps], 64, stream)
+    tb = timed([lambda s=s: (s.mxfp4(sptr), s.nvfp4(sptr)) for s in wsteps], 64, stream)
+    tf = timed([lambda s=s: s.both(sptr) for s in wsteps], 64, stream)
+    out["weight_4096x4096_mxfp4_floor_and_nvfp4_both_layouts"] = {
+        "step_us": round(tb * 1e3, 2), "step_GBps": round((BYTES_MXFP4 + BYTES_NVFP4) / tb / 1e6, 1),
+        "step_frac_hbm": round((BYTES_MXFP4 + BYTES_NVFP4) / tb / 1e6 / hbm, 4),
+        "one_call_us": round(tf * 1e3, 2), "one_call_GBps": round((BYTES_MXFP4 + BYTES_NVFP4) / tf / 1e6, 1),
+        "one_call_frac_hbm": round((BYTES_MXFP4 + BYTES_NVFP4) / tf / 1e6 / hbm, 4),
+        "one_call_note": "mx_quantize_mx_nvfp4: both encodings, the MX pass supplies the NVFP4 tensor maximum",
+        "mxfp4_us": round(t4 * 1e3, 2), "mxfp4_GBps": round(BYTES_MXFP4 / t4 / 1e6, 1),
+        "mxfp4_frac_hbm": round(BYTES_MXFP4 / t4 / 1e6 / hbm, 4),
+        "nvfp4_us": round(tn * 1e3, 2), "nvfp4_GBps": round(BYTES_NVFP4 / tn / 1e6, 1),
+        "nvfp4_frac_hbm": round(BYTES_NVFP4 / tn / 1e6 / hbm, 4),
+        "algorithmic_bytes": {"mxfp4": BYTES_MXFP4, "nvfp4": BYTES_NVFP4},
+        "l2": f"{NROT} rotating copies of the weight ({NROT * R2 * C2 * 2 >> 20} MiB)"}
+    del wsteps, xw0
+    torch.cuda.empty_cache()
 
     # C4 / C5: block-scaled matmuls (operands quantised outside the timing)
     # (plus the MXFP6 x MXFP6 matmul, which runs on the same kind at the same rate)
@@ -482,7 +564,12 @@ def run_breakdown(mx, dev, pk):
         t = timed([lambda: mx.gemm(a, b, c)], 10, stream)
         tb = best_of(lambda: mx.gemm(a, b, c), 10, stream)
         tf, tfb = (2.0 * M * N * K / (x * 1e-3) / 1e12 for x in (t, tb))
+        if cpu and name != "gemm_mxfp6_e2m3_8192":
+            cpu_gemm = gemm_cpu_baseline((M, N, K), afmt, bfmt, bsig)
+        else:
+            cpu_gemm = None
         out[name] = {"ms": round(t, 4), "TFLOPS": round(tf, 1), "frac_mx_peak_measured": round(tf / mx_peak, 4),
+                     "cpu_baseline": cpu_gemm,
                      "clocks_back_to_back": soak_clocks(lambda: mx.gemm(a, b, c)),
                      "best_of_10_ms": round(tb, 4), "best_of_10_TFLOPS": round(tfb, 1),
                      "frac_best_of_10_mx_peak_measured": round(tfb / mx_peak, 4),
@@ -630,50 +717,97 @@ def run_breakdown(mx, dev, pk):
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def cpu_baseline(x_bits, target_s=12.0):
-    """The oracle as it stands, single-threaded, on a bounded row sample of the workload."""
+def _workers():
+    return max(1, min(64, os.cpu_count() or 1))
+
+
+def cpu_baseline(a_bits, g_bits, target_s=12.0, band=64):
+    """The oracle as it stands on a bounded sample of the workload: bands of `band`
+    consecutive rows of both tensors, each band quantised row-wise and column-wise by the
+    oracle with tcgen05-tiled scales; bands run on all host cores (one oracle call per
+    thread).  value = the workload's bytes for the rows done / wall time."""
     import oracle
     oracle.lib()
-    rows = 64
+    R = ACT[0]
+    bands = list(range(0, R, band))
+    workers = _workers()
+
+    def one(r0):
+        for x, fmt in ((a_bits, oracle.E4M3), (g_bits, oracle.E5M2)):
+            xs = np.ascontiguousarray(x[r0:r0 + band])
+            _, s = oracle.quantize_mx(xs, fmt, oracle.ROW, oracle.CEIL)
+            oracle.to_tcgen05_layout(s)
+            _, s = oracle.quantize_mx(xs, fmt, oracle.COL, oracle.CEIL)
+            oracle.to_tcgen05_layout(s)
+        return band
+
     t0 = time.perf_counter()
-    done_rows = 0
-    while True:
-        xs = np.ascontiguousarray(x_bits[done_rows % R2: done_rows % R2 + rows])
-        e4, s4 = oracle.quantize_mx(xs, oracle.E2M1, oracle.ROW, oracle.FLOOR)
-        oracle.to_tcgen05_layout(s4)
-        en, sn, g = oracle.quantize_nvfp4(xs)
-        oracle.to_tcgen05_layout(sn)
-        done_rows += rows
-        if time.perf_counter() - t0 > target_s or done_rows >= R2:
-            break
+    done = 0
+    with cf.ThreadPoolExecutor(workers) as ex:
+        i = 0
+        while i < len(bands) and time.perf_counter() - t0 < target_s:
+            chunk = bands[i:i + workers]
+            done += sum(ex.map(one, chunk))
+            i += len(chunk)
     dt = time.perf_counter() - t0
-    bytes_done = STEP_BYTES * done_rows / R2
-    return {"value": round(bytes_done / dt / 1e9, 5), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done_rows} of {R2} rows of the 4096x4096 weight (MXFP4 + NVFP4, both layouts), "
-                      f"{dt:.1f} s single-threaded", "seconds": round(dt, 2)}
+    return {"value": round(STEP_BYTES * done / R / dt / 1e9, 5), "unit": "GB/s", "cores": workers, "kind": "oracle",
+            "sample": f"{done} of {R} rows of both tensors (bands of {band} rows, row- and column-wise, "
+                      f"tcgen05 scales), {dt:.1f} s on {workers} threads", "seconds": round(dt, 2)}
+
+
+def gemm_cpu_baseline(shape, afmt, bfmt, bsig, target_s=6.0):
+    """The oracle's fp64 matmul reference (one plain k-loop per entry) on sampled entries of
+    the benchmark's operands, on all host cores; TFLOP/s = 2 K x entries / wall time."""
+    import oracle
+    M, N, K = shape
+    fm = {"e4m3": oracle.E4M3, "e2m1": oracle.E2M1, "e2m3": oracle.E2M3}
+    rng = np.random.default_rng(5)
+    ra = np.sort(rng.choice(M, 32, replace=False))
+    rb = np.sort(rng.choice(N, 32, replace=False))
+    a = synth.normal(M, K, seed=40)[ra]
+    b = synth.normal(N, K, sigma=bsig, seed=41)[rb]
+    ae, as_ = oracle.quantize_mx(a, fm[afmt], oracle.ROW, oracle.CEIL)
+    be, bs = oracle.quantize_mx(b, fm[bfmt], oracle.ROW, oracle.FLOOR if bfmt == "e2m1" else oracle.CEIL)
+    pairs = np.array([(i, j) for i in range(32) for j in range(32)], dtype=np.int64)
+    workers = _workers()
+    chunks = [pairs[i::workers] for i in range(workers)]
+
+    def one(p):
+        oracle.gemm_ref(ae, as_, fm[afmt], be, bs, fm[bfmt], 32, 32, K, p)
+        return len(p)
+
+    t0 = time.perf_counter()
+    done = 0
+    with cf.ThreadPoolExecutor(workers) as ex:
+        while time.perf_counter() - t0 < target_s:
+            done += sum(ex.map(one, chunks))
+    dt = time.perf_counter() - t0
+    return {"value": round(2.0 * K * done / dt / 1e12, 8), "unit": "TFLOP/s", "cores": workers, "kind": "oracle",
+            "sample": f"{done} entries of C ({len(pairs)} distinct, K = {K}), fp64, {dt:.1f} s on {workers} threads"}
 
 
 def run_reference(args, rank, world):
-    """The oracle as the reference arm: rank 0 only, bounded sample per step."""
+    """The oracle as the reference arm: rank 0 only, a bounded sample per step."""
     if rank != 0:
         return
-    x_bits = synth.weight_fp4(seed=0)
+    a_bits = synth.activations(seed=0)
+    g_bits = synth.gradients(seed=1)
     per_step = max(1.0, args.cpu_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_baseline(x_bits, target_s=per_step)
+        cpu_baseline(a_bits, g_bits, target_s=per_step)
     vals, secs = [], []
     for _ in range(args.steps):
-        r = cpu_baseline(x_bits, target_s=per_step)
+        r = cpu_baseline(a_bits, g_bits, target_s=per_step)
         vals.append(r["value"])
         secs.append(r["seconds"])
-        sample = r["sample"]
+        sample, cores = r["sample"], r["cores"]
     v = statistics.mean(vals)
     line = {"impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic (numpy default_rng, seed 0)",
-            "config": {"workload": "weight_4096x4096_mxfp4_floor_and_nvfp4_both_scale_layouts", "shape": [R2, C2]},
-            "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": round(v, 5)},
+            "data": "synthetic (numpy default_rng; activations seed 0, gradients seed 1)",
+            "config": {"workload": WORKLOAD, "step_bytes": STEP_BYTES},
+            "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample, "value": round(v, 5)},
             "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -688,6 +822,13 @@ def run_case(name, iters, dev):
     if name == "weight4096":
         st = WeightQuantStep(mx, to_dev(synth.weight_fp4(), dev))
         fns = [lambda: (st.mxfp4(stream.cuda_stream), st.nvfp4(stream.cuda_stream))]
+    elif name == "weight4096_one_call":
+        st = WeightQuantStep(mx, to_dev(synth.weight_fp4(), dev))
+        fns = [lambda: st.both(stream.cuda_stream)]
+    elif name == "step":
+        # the headline step itself (both dual calls), for the launch list and DRAM traffic
+        st = DualStep(mx, to_dev(synth.activations(), dev), to_dev(synth.gradients(), dev))
+        fns = [lambda: st.run(stream.cuda_stream)]
     elif name == "mx8_1024":
         x = to_dev(synth.mx8_rowwise(), dev)
         q = mx.quantize(x, "e4m3", "row", "ceil", layout="rowmajor")
@@ -763,7 +904,7 @@ def run_case(name, iters, dev):
     print(f"{name}: {iters} calls, {t * 1e3:.1f} us per call", flush=True)
 
 
-CASES = ["weight4096", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "gemm8192", "gemm_w4a8",
+CASES = ["step", "weight4096", "weight4096_one_call", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "gemm8192", "gemm_w4a8",
          "gemm_mxfp4_8192", "gemm_nvfp4_8192", "gemm_cmp", "extended"]
 
 

@@ -24,8 +24,8 @@
  *     device, only a small scratch array for NVFP4 partial maxima (allocated on the
  *     first NVFP4 call on that device) and a static watchdog flag.
  *   - NVFP4 calls on one device (mx_quantize with MX_FMT_NVFP4, mx_quantize_train with
- *     MX_FMT_NVFP4, mx_quantize_nvfp4_2d) share that scratch array: calls whose GPU work
- *     overlaps -- on two streams with no ordering between them -- race on it and may
+ *     MX_FMT_NVFP4, mx_quantize_nvfp4_2d, mx_quantize_mx_nvfp4) share that scratch array:
+ *     calls whose GPU work overlaps -- on two streams with no ordering between them -- race on it and may
  *     produce a wrong per-tensor scale.  Issue them on one stream, or order the streams
  *     with events.  The MX formats use no scratch and may overlap freely.
  *   - Execution: every call only validates its arguments on the host and enqueues
@@ -205,19 +205,43 @@ mx_status mx_quantize_nvfp4_2d(const void *src_bf16, int64_t rows, int64_t cols,
                                float *global_scale, mx_stream_t stream);
 
 /*
+ * mx_quantize_mx_nvfp4 -- row-wise MX quantisation (any MX format) and NVFP4 quantisation
+ * of the same bf16 tensor in one call, the two encodings of one weight that [Q] §4
+ * ("同じ E2M1 でも、別仕様である") compares.  The input is read from memory once for both
+ * maxima: the MX pass also reduces the tensor's finite |x| maximum, so the NVFP4 pass runs
+ * without a maximum pass of its own (it re-reads the input, from L2 when it fits there).
+ * Results are bit-identical to mx_quantize(fmt, ROW, rounding, mx_*) followed by
+ * mx_quantize(NVFP4, ROW, nv_*).
+ *   fmt, rounding, mx_elems, mx_scales, mx_layout, mx_scales_alt
+ *                 the MX output, as mx_quantize(axis = ROW); cols % 32 == 0.
+ *   nv_elems, nv_scales, nv_layout, nv_scales_alt, global_scale
+ *                 the NVFP4 output, as mx_quantize(fmt = NVFP4).
+ * Uses the NVFP4 partial-maxima scratch (the ordering rule above applies).
+ */
+mx_status mx_quantize_mx_nvfp4(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt fmt,
+                               mx_scale_rounding rounding, void *mx_elems, uint8_t *mx_scales,
+                               mx_scale_layout mx_layout, uint8_t *mx_scales_alt, void *nv_elems,
+                               uint8_t *nv_scales, mx_scale_layout nv_layout, uint8_t *nv_scales_alt,
+                               float *global_scale, mx_stream_t stream);
+
+/*
  * mx_quantize_dual -- one pass over a bf16 matrix producing both orientations ([Q] §6:
  * training needs the row-wise copy for the forward matmul and the column-wise copy for
  * the weight-gradient matmul).  The input is read once.
  *   row_elems / row_scales   as mx_quantize(axis = ROW).
  *   col_elems / col_scales   as mx_quantize(axis = COL): cols x rows, scales cols x rows/32.
- *   layout      exactly one of ROWMAJOR / TCGEN05, used for both scale outputs.
+ *   layout      ROWMAJOR, TCGEN05 or both (bitwise or), used for both orientations.  With
+ *               one layout, row_scales / col_scales are in it and the two *_alt pointers
+ *               must be NULL; with both, row_scales / col_scales are ROWMAJOR and
+ *               row_scales_alt / col_scales_alt (device, non-NULL) TCGEN05 -- all four
+ *               are written by the same single pass.
  *   fmt         any MX format (E4M3, E5M2, E2M3, E3M2, E2M1, INT8).  rows and cols are
  *               multiples of 32.
  */
 mx_status mx_quantize_dual(const void *src_bf16, int64_t rows, int64_t cols, mx_fmt fmt,
                            mx_scale_rounding rounding, void *row_elems, uint8_t *row_scales,
                            void *col_elems, uint8_t *col_scales, mx_scale_layout layout,
-                           mx_stream_t stream);
+                           uint8_t *row_scales_alt, uint8_t *col_scales_alt, mx_stream_t stream);
 
 /*
  * mx_dequantize -- codes and scales back to bf16 ([Q] §7: MX is an exponent add,

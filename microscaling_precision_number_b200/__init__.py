@@ -8,7 +8,9 @@ include/mx.h (libmx.so).  This package is the thin Python binding over that ABI.
 from . import _lib
 from ._lib import MxError
 from .api import (Quantized, block_of, cast, dequantize, elem_bytes, gemm, is_fp4, quantize,
-                  quantize_dual, quantize_nvfp4_2d, quantize_train, scale_bytes, watchdog_status)
+                  quantize_dual, quantize_mx_nvfp4, quantize_nvfp4_2d, quantize_train, scale_bytes,
+                  watchdog_status)
 
 __all__ = ["MxError", "Quantized", "block_of", "cast", "dequantize", "elem_bytes", "gemm", "is_fp4", "quantize",
-           "quantize_dual", "quantize_nvfp4_2d", "quantize_train", "scale_bytes", "watchdog_status", "_lib"]
+           "quantize_dual", "quantize_mx_nvfp4", "quantize_nvfp4_2d", "quantize_train", "scale_bytes",
+           "watchdog_status", "_lib"]

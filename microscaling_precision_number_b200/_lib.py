@@ -22,7 +22,7 @@ MX_LAYOUT_ROWMAJOR, MX_LAYOUT_TCGEN05 = 1, 2
 EXPORTS = ("mx_scale_bytes", "mx_quantize", "mx_quantize_dual", "mx_dequantize", "mx_cast",
            "mx_gemm", "mx_status_string", "mx_last_cuda_error", "mx_watchdog_status",
            "mx_quantize_nvfp4_noalloc", "mx_mxfp4_to_fp8_blocks", "mx_quantize_nvfp4_2d", "mx_quantize_train",
-           "mx_watchdog_selftest")
+           "mx_watchdog_selftest", "mx_quantize_mx_nvfp4")
 WD_SELFTEST = 9
 MX_NOALLOC_MAX_PARTIALS = 1024
 
@@ -50,7 +50,7 @@ def _load():
     lib.mx_scale_bytes.restype = I64
     lib.mx_quantize.argtypes = [P, I64, I64, I, I, I, P, U8P, I, U8P, P, P]
     lib.mx_quantize.restype = I
-    lib.mx_quantize_dual.argtypes = [P, I64, I64, I, I, P, U8P, P, U8P, I, P]
+    lib.mx_quantize_dual.argtypes = [P, I64, I64, I, I, P, U8P, P, U8P, I, U8P, U8P, P]
     lib.mx_quantize_dual.restype = I
     lib.mx_dequantize.argtypes = [P, U8P, P, I64, I64, I, I, P, P]
     lib.mx_dequantize.restype = I
@@ -70,6 +70,8 @@ def _load():
     lib.mx_last_cuda_error.restype = I
     lib.mx_watchdog_status.argtypes = [ctypes.POINTER(ctypes.c_int), I]
     lib.mx_watchdog_status.restype = I
+    lib.mx_quantize_mx_nvfp4.argtypes = [P, I64, I64, I, I, P, U8P, I, U8P, P, U8P, I, U8P, P, P]
+    lib.mx_quantize_mx_nvfp4.restype = I
     lib.mx_watchdog_selftest.argtypes = [ctypes.c_uint32, P]
     lib.mx_watchdog_selftest.restype = I
     # NVFP4 quantisation without any device allocation (static scratch array)

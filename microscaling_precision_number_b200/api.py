@@ -131,6 +131,33 @@ def quantize_train(x: torch.Tensor, fmt="e2m1", rounding: str = "floor", rht_sig
     return Quantized(elems, scales, alt, g, rows, cols, f)
 
 
+def quantize_mx_nvfp4(x: torch.Tensor, fmt="e2m1", rounding: str = "floor", layout: str = "both",
+                      nv_layout: str = "both", stream=None):
+    """Row-wise MX quantisation (any MX format) and NVFP4 quantisation of the same tensor in
+    one call, reading its maximum once (the MX pass also yields the NVFP4 tensor maximum).
+    Returns (mx Quantized, nvfp4 Quantized), bit-identical to two quantize() calls."""
+    _check_src(x)
+    f = _fmt(fmt)
+    rows, cols = x.shape
+    dev = x.device
+
+    def outs(fm, B, lay):
+        first = "rowmajor" if lay in ("rowmajor", "both") else "tcgen05"
+        e = torch.empty(elem_bytes(rows, cols, fm), dtype=torch.uint8, device=dev)
+        sc = torch.empty(scale_bytes(rows, cols // B, first), dtype=torch.uint8, device=dev)
+        alt = torch.empty(scale_bytes(rows, cols // B, "tcgen05"), dtype=torch.uint8, device=dev) \
+            if lay == "both" else None
+        return e, sc, alt
+
+    me, ms, ma = outs(f, 32, layout)
+    ne, ns, na = outs(L.MX_FMT_NVFP4, 16, nv_layout)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    L.check(L.lib.mx_quantize_mx_nvfp4(x.data_ptr(), rows, cols, f, ROUNDING[rounding], me.data_ptr(), ms.data_ptr(),
+                                       LAYOUTS[layout], _ptr(ma), ne.data_ptr(), ns.data_ptr(), LAYOUTS[nv_layout],
+                                       _ptr(na), g.data_ptr(), _stream(stream)), "mx_quantize_mx_nvfp4")
+    return (Quantized(me, ms, ma, None, rows, cols, f), Quantized(ne, ns, na, g, rows, cols, L.MX_FMT_NVFP4))
+
+
 def quantize_nvfp4_2d(x: torch.Tensor, layout: str = "tcgen05", stream=None) -> Quantized:
     """NVFP4 with 16 x 16 weight blocks (scales repeated on the 16 rows of each block)."""
     _check_src(x)
@@ -157,14 +184,19 @@ def quantize_dual(x: torch.Tensor, fmt="e4m3", rounding: str = "ceil", layout: s
     rows, cols = x.shape
     dev = x.device
     o_r, o_c = out if out is not None else (None, None)
+    first = "rowmajor" if layout in ("rowmajor", "both") else "tcgen05"
     re = _buf(o_r and o_r.elems, elem_bytes(rows, cols, f), torch.uint8, dev, "row elems")
     ce = _buf(o_c and o_c.elems, elem_bytes(rows, cols, f), torch.uint8, dev, "col elems")
-    rs = _buf(o_r and o_r.scales, scale_bytes(rows, cols // 32, layout), torch.uint8, dev, "row scales")
-    cs = _buf(o_c and o_c.scales, scale_bytes(cols, rows // 32, layout), torch.uint8, dev, "col scales")
+    rs = _buf(o_r and o_r.scales, scale_bytes(rows, cols // 32, first), torch.uint8, dev, "row scales")
+    cs = _buf(o_c and o_c.scales, scale_bytes(cols, rows // 32, first), torch.uint8, dev, "col scales")
+    ra = ca = None
+    if layout == "both":
+        ra = _buf(o_r and o_r.scales_alt, scale_bytes(rows, cols // 32, "tcgen05"), torch.uint8, dev, "row scales_alt")
+        ca = _buf(o_c and o_c.scales_alt, scale_bytes(cols, rows // 32, "tcgen05"), torch.uint8, dev, "col scales_alt")
     st = L.lib.mx_quantize_dual(x.data_ptr(), rows, cols, f, ROUNDING[rounding], re.data_ptr(), rs.data_ptr(),
-                                ce.data_ptr(), cs.data_ptr(), LAYOUTS[layout], _stream(stream))
+                                ce.data_ptr(), cs.data_ptr(), LAYOUTS[layout], _ptr(ra), _ptr(ca), _stream(stream))
     L.check(st, "mx_quantize_dual")
-    return (Quantized(re, rs, None, None, rows, cols, f), Quantized(ce, cs, None, None, cols, rows, f))
+    return (Quantized(re, rs, ra, None, rows, cols, f), Quantized(ce, cs, ca, None, cols, rows, f))
 
 
 def dequantize(q: Quantized, layout: str = "rowmajor", stream=None, out: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <mutex>
+#include <utility>
 
 #include "../../include/mx.h"
 #include "internal.h"
@@ -187,7 +188,7 @@ mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, m
     if (fmt == MX_FMT_NVFP4) {
         st = nvfp4_scratch(d);
         if (st != MX_OK) return st;
-        e = mxk::launch_stream_nvfp4(src, rows, cols, d->partials, 3 * d->num_sms, global_scale, out_elems, rm, tc,
+        e = mxk::launch_stream_nvfp4(src, rows, cols, d->partials, 3 * d->num_sms, 0, global_scale, out_elems, rm, tc,
                                      d->watchdog, d->num_sms, s);
         if (e != cudaSuccess) return cuda_fail(e);
         if (tc) {
@@ -198,7 +199,8 @@ mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, m
     }
 
     if (axis == MX_AXIS_ROW) {
-        e = mxk::launch_stream_rows_mx(src, rows, cols, fmt, ceil, out_elems, rm, tc, d->watchdog, d->num_sms, s);
+        e = mxk::launch_stream_rows_mx(src, rows, cols, fmt, ceil, out_elems, rm, tc, nullptr, d->watchdog,
+                                       d->num_sms, s);
         if (e != cudaSuccess) return cuda_fail(e);
         if (tc) {
             e = mxk::launch_tcgen05_pad(tc, rows, cols / 32, s);
@@ -207,18 +209,12 @@ mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, m
         return MX_OK;
     }
 
-    // Column-wise: the TMA-staged kernel with only the transposed output enabled.  It
-    // takes one scale layout per call; with both requested, run it once per layout.
+    // Column-wise: the TMA-staged kernel with only the transposed output enabled; the
+    // requested scale layouts (one or both) are written by the same pass.
     if (cols % 8 != 0) return MX_ERR_SHAPE;    // the TMA row pitch (cols * 2 bytes) must be a multiple of 16
-    uint8_t *first = rm ? rm : tc;
-    e = mxk::launch_quant_dual(src, rows, cols, fmt, ceil, nullptr, nullptr, out_elems, first, first == tc,
+    e = mxk::launch_quant_dual(src, rows, cols, fmt, ceil, nullptr, nullptr, nullptr, out_elems, rm, tc,
                                d->watchdog, d->num_sms, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    if (rm && tc) {
-        e = mxk::launch_quant_dual(src, rows, cols, fmt, ceil, nullptr, nullptr, out_elems, tc, true,
-                                   d->watchdog, d->num_sms, s);
-        if (e != cudaSuccess) return cuda_fail(e);
-    }
     if (tc) {
         e = mxk::launch_tcgen05_pad(tc, cols, rows / 32, s);
         if (e != cudaSuccess) return cuda_fail(e);
@@ -226,30 +222,84 @@ mx_status mx_quantize(const void *src, int64_t rows, int64_t cols, mx_fmt fmt, m
     return MX_OK;
 }
 
+mx_status mx_quantize_mx_nvfp4(const void *src, int64_t rows, int64_t cols, mx_fmt fmt,
+                               mx_scale_rounding rounding, void *mx_elems, uint8_t *mx_scales,
+                               mx_scale_layout mx_layout, uint8_t *mx_scales_alt, void *nv_elems,
+                               uint8_t *nv_scales, mx_scale_layout nv_layout, uint8_t *nv_scales_alt,
+                               float *global_scale, mx_stream_t stream) {
+    if (!mx_block_fmt(fmt)) return MX_ERR_ARG;
+    if (rounding != MX_SCALE_FLOOR_OCP && rounding != MX_SCALE_CEIL_RECIPE) return MX_ERR_ARG;
+    const int both = MX_LAYOUT_ROWMAJOR | MX_LAYOUT_TCGEN05;
+    for (const auto &[lay, alt] : {std::pair<int, const uint8_t *>{mx_layout, mx_scales_alt},
+                                   std::pair<int, const uint8_t *>{nv_layout, nv_scales_alt}}) {
+        if (!single_layout(lay) && lay != both) return MX_ERR_LAYOUT;
+        if ((lay == both) != (alt != nullptr)) return MX_ERR_LAYOUT;
+    }
+    if (rows < 0 || cols < 0) return MX_ERR_SHAPE;
+    if (cols % 32) return MX_ERR_SHAPE;
+    if (rows == 0 || cols == 0) return MX_OK;
+    if (!mxk::stream_supported(rows, cols)) return MX_ERR_SHAPE;
+    if (!src || !mx_elems || !mx_scales || !nv_elems || !nv_scales || !global_scale) return MX_ERR_ARG;
+    if (!aligned(src, 16) || !aligned(mx_elems, 16) || !aligned(nv_elems, 16)) return MX_ERR_ALIGN;
+    if (!aligned(global_scale, 4)) return MX_ERR_ALIGN;
+    uint8_t *mrm = mx_layout == MX_LAYOUT_TCGEN05 ? nullptr : mx_scales;
+    uint8_t *mtc = mx_layout == MX_LAYOUT_TCGEN05 ? mx_scales : mx_scales_alt;
+    uint8_t *nrm = nv_layout == MX_LAYOUT_TCGEN05 ? nullptr : nv_scales;
+    uint8_t *ntc = nv_layout == MX_LAYOUT_TCGEN05 ? nv_scales : nv_scales_alt;
+
+    DeviceState *d = nullptr;
+    mx_status st = device_state(&d);
+    if (st != MX_OK) return st;
+    st = nvfp4_scratch(d);
+    if (st != MX_OK) return st;
+    const int n_partials = mxk::stream_rows_grid(rows, cols, d->num_sms);
+    if (n_partials > d->partials_cap) return MX_ERR_SHAPE;      // cannot happen: both are 3 x SMs at most
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // the MX pass also leaves the NVFP4 partial maxima; the NVFP4 pass then skips its own
+    // maximum pass (programmatic dependent launch orders it after the MX pass)
+    cudaError_t e = mxk::launch_stream_rows_mx(src, rows, cols, fmt, rounding == MX_SCALE_CEIL_RECIPE, mx_elems, mrm,
+                                               mtc, d->partials, d->watchdog, d->num_sms, s);
+    if (e == cudaSuccess)
+        e = mxk::launch_stream_nvfp4(src, rows, cols, d->partials, d->partials_cap, n_partials, global_scale, nv_elems,
+                                     nrm, ntc, d->watchdog, d->num_sms, s);
+    if (e == cudaSuccess && mtc) e = mxk::launch_tcgen05_pad(mtc, rows, cols / 32, s);
+    if (e == cudaSuccess && ntc) e = mxk::launch_tcgen05_pad(ntc, rows, cols / 16, s);
+    return e == cudaSuccess ? MX_OK : cuda_fail(e);
+}
+
 mx_status mx_quantize_dual(const void *src, int64_t rows, int64_t cols, mx_fmt fmt,
                            mx_scale_rounding rounding, void *row_elems, uint8_t *row_scales,
                            void *col_elems, uint8_t *col_scales, mx_scale_layout layout,
-                           mx_stream_t stream) {
+                           uint8_t *row_scales_alt, uint8_t *col_scales_alt, mx_stream_t stream) {
     if (!mx_block_fmt(fmt)) return MX_ERR_ARG;
     if (rounding != MX_SCALE_FLOOR_OCP && rounding != MX_SCALE_CEIL_RECIPE) return MX_ERR_ARG;
-    if (!single_layout(layout)) return MX_ERR_LAYOUT;
+    const bool both = layout == (MX_LAYOUT_ROWMAJOR | MX_LAYOUT_TCGEN05);
+    if (!single_layout(layout) && !both) return MX_ERR_LAYOUT;
+    if (both != (row_scales_alt != nullptr) || both != (col_scales_alt != nullptr)) return MX_ERR_LAYOUT;
     if (rows < 0 || cols < 0) return MX_ERR_SHAPE;
     if (rows % 32 || cols % 32) return MX_ERR_SHAPE;
     if (rows == 0 || cols == 0) return MX_OK;
     if (!src || !row_elems || !row_scales || !col_elems || !col_scales) return MX_ERR_ARG;
     if (!aligned(src, 16) || !aligned(row_elems, 16) || !aligned(col_elems, 16)) return MX_ERR_ALIGN;
+    uint8_t *row_rm = nullptr, *row_tc = nullptr, *col_rm = nullptr, *col_tc = nullptr;
+    if (both) {
+        row_rm = row_scales; row_tc = row_scales_alt; col_rm = col_scales; col_tc = col_scales_alt;
+    } else if (layout == MX_LAYOUT_ROWMAJOR) {
+        row_rm = row_scales; col_rm = col_scales;
+    } else {
+        row_tc = row_scales; col_tc = col_scales;
+    }
     DeviceState *d = nullptr;
     mx_status st = device_state(&d);
     if (st != MX_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const bool tc = layout == MX_LAYOUT_TCGEN05;
     cudaError_t e = mxk::launch_quant_dual(src, rows, cols, fmt, rounding == MX_SCALE_CEIL_RECIPE, row_elems,
-                                           row_scales, col_elems, col_scales, tc, d->watchdog, d->num_sms, s);
+                                           row_rm, row_tc, col_elems, col_rm, col_tc, d->watchdog, d->num_sms, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    if (tc) {
-        e = mxk::launch_tcgen05_pad(row_scales, rows, cols / 32, s);
+    if (row_tc) {
+        e = mxk::launch_tcgen05_pad(row_tc, rows, cols / 32, s);
         if (e != cudaSuccess) return cuda_fail(e);
-        e = mxk::launch_tcgen05_pad(col_scales, cols, rows / 32, s);
+        e = mxk::launch_tcgen05_pad(col_tc, cols, rows / 32, s);
         if (e != cudaSuccess) return cuda_fail(e);
     }
     return MX_OK;

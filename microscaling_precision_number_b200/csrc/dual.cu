@@ -107,11 +107,25 @@ __device__ __forceinline__ void tile_coords(uint32_t t, const TileOrder &o, uint
 // logical chunk c; the 128-byte swizzle stores it at chunk c ^ (r % 8).
 __device__ __forceinline__ uint32_t swz(uint32_t r, uint32_t c) { return r * 128u + ((c ^ (r & 7u)) << 4); }
 
+// Where the scales of one orientation go: a row-major array of S scales per row and/or
+// the tcgen05 tiling with `atoms` 4-column atoms per 128 rows (either pointer may be null
+// according to the RM / TC template flags).
+struct ScaleOut {
+    uint8_t *rm;
+    uint8_t *tc;
+    uint32_t S, atoms;
+};
+template <bool RM, bool TC>
+__device__ __forceinline__ void put_scale(const ScaleOut &o, uint32_t r, uint32_t c, uint32_t code) {
+    if constexpr (RM) o.rm[(uint64_t)r * o.S + c] = (uint8_t)code;
+    if constexpr (TC) o.tc[tc_offset(r, c, o.atoms)] = (uint8_t)code;
+}
+
 // Column pass: columns col, col + 1 (box-relative pair q) over the tile's 32 rows.
-template <int FMT, bool CEIL, bool TC>
+template <int FMT, bool CEIL, bool RM, bool TC>
 __device__ __forceinline__ void column_pair(const uint8_t *box, uint32_t q, uint32_t col, uint32_t rows,
                                             uint32_t r0, uint32_t tr, uint8_t *__restrict__ col_elems,
-                                            uint8_t *__restrict__ col_sc, uint32_t sc_dim, bool v8) {
+                                            const ScaleOut &col_sc, bool v8) {
     uint32_t w[32];                                      // row r: bf16 of col (low) and col + 1 (high)
 #pragma unroll
     for (int r = 0; r < 32; r++)
@@ -164,20 +178,15 @@ __device__ __forceinline__ void column_pair(const uint8_t *box, uint32_t q, uint
         store_codes<FMT>(col_elems, e0, o_lo, v8, code_lo == 0xFFu);        // NaN scale: codes 0
         store_codes<FMT>(col_elems, e0 + rows, o_hi, v8, code_hi == 0xFFu);
     }
-    if constexpr (TC) {
-        col_sc[tc_offset(col, tr, sc_dim)] = (uint8_t)code_lo;
-        col_sc[tc_offset(col + 1, tr, sc_dim)] = (uint8_t)code_hi;
-    } else {
-        col_sc[(uint64_t)col * sc_dim + tr] = (uint8_t)code_lo;
-        col_sc[(uint64_t)(col + 1) * sc_dim + tr] = (uint8_t)code_hi;
-    }
+    put_scale<RM, TC>(col_sc, col, tr, code_lo);
+    put_scale<RM, TC>(col_sc, col + 1, tr, code_hi);
 }
 
 // Row pass: the 32-element block of tile row r starting at box-relative chunk 4h.
-template <int FMT, bool CEIL, bool TC>
+template <int FMT, bool CEIL, bool RM, bool TC>
 __device__ __forceinline__ void row_block(const uint8_t *box, uint32_t r, uint32_t h, uint32_t col, uint32_t cols,
-                                          uint32_t R, uint8_t *__restrict__ row_elems,
-                                          uint8_t *__restrict__ row_sc, uint32_t sc_dim, bool v8) {
+                                          uint32_t R, uint8_t *__restrict__ row_elems, const ScaleOut &row_sc,
+                                          bool v8) {
     uint4 v[4];
 #pragma unroll
     for (int k = 0; k < 4; k++) v[k] = *reinterpret_cast<const uint4 *>(box + swz(r, 4u * h + k));
@@ -217,18 +226,16 @@ __device__ __forceinline__ void row_block(const uint8_t *box, uint32_t r, uint32
         }
         store_codes<FMT>(row_elems, e0, o, v8, code == 0xFFu);             // NaN scale: codes 0
     }
-    if constexpr (TC) row_sc[tc_offset(R, col >> 5, sc_dim)] = (uint8_t)code;
-    else row_sc[(uint64_t)R * sc_dim + (col >> 5)] = (uint8_t)code;
+    put_scale<RM, TC>(row_sc, R, col >> 5, code);
 }
 
-// ROW: also write the row-wise output.  sc_dim_*: scales per row (row-major layout) or
-// 4-column atom count (tcgen05 layout) of the row-wise / column-wise scale array.
-template <int FMT, bool CEIL, bool ROW, bool TC>
+// ROW: also write the row-wise output.  RM / TC: write the scales in the row-major layout,
+// the tcgen05 tiling, or both (one pass either way).
+template <int FMT, bool CEIL, bool ROW, bool RM, bool TC>
 __global__ void __launch_bounds__(kDualThreads, kCtasPerSm)
 quant_dual_kernel(const __grid_constant__ CUtensorMap tmap, uint32_t rows, uint32_t cols, uint32_t n_tiles,
-                  TileOrder order, uint8_t *__restrict__ row_elems, uint8_t *__restrict__ row_sc,
-                  uint32_t row_sc_dim, uint8_t *__restrict__ col_elems, uint8_t *__restrict__ col_sc,
-                  uint32_t col_sc_dim, int v8, int *watchdog) {
+                  TileOrder order, uint8_t *__restrict__ row_elems, ScaleOut row_sc,
+                  uint8_t *__restrict__ col_elems, ScaleOut col_sc, int v8, int *watchdog) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
@@ -243,6 +250,11 @@ quant_dual_kernel(const __grid_constant__ CUtensorMap tmap, uint32_t rows, uint3
         }
         fence_barrier_init();
     }
+    // Programmatic dependent launch: the set-up above overlaps the previous kernel's tail;
+    // nothing is read or written in global memory before that kernel has completed.  The
+    // next kernel may then be launched at once (its CTAs start as ours retire).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __syncthreads();
 
     uint32_t issued = 0;
@@ -278,15 +290,15 @@ quant_dual_kernel(const __grid_constant__ CUtensorMap tmap, uint32_t rows, uint3
             if (row_pass) {
                 const uint32_t h = lane & 1u, col = c0 + 32u * h;
                 if (col < cols) {
-                    row_block<FMT, CEIL, TC>(box, lane >> 1, h, col, cols, r0 + (lane >> 1), row_elems, row_sc,
-                                             row_sc_dim, v8 != 0);
-                    row_block<FMT, CEIL, TC>(box, 16 + (lane >> 1), h, col, cols, r0 + 16 + (lane >> 1), row_elems,
-                                             row_sc, row_sc_dim, v8 != 0);
+                    row_block<FMT, CEIL, RM, TC>(box, lane >> 1, h, col, cols, r0 + (lane >> 1), row_elems, row_sc,
+                                                 v8 != 0);
+                    row_block<FMT, CEIL, RM, TC>(box, 16 + (lane >> 1), h, col, cols, r0 + 16 + (lane >> 1),
+                                                 row_elems, row_sc, v8 != 0);
                 }
             } else {
                 const uint32_t col = c0 + 2u * lane;
                 if (col < cols)
-                    column_pair<FMT, CEIL, TC>(box, lane, col, rows, r0, tr, col_elems, col_sc, col_sc_dim, v8 != 0);
+                    column_pair<FMT, CEIL, RM, TC>(box, lane, col, rows, r0, tr, col_elems, col_sc, v8 != 0);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
@@ -309,36 +321,56 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
                                   CUtensorMapFloatOOBfill);
 
-template <int FMT, bool CEIL, bool ROW, bool TC>
+template <int FMT, bool CEIL, bool ROW, bool RM, bool TC>
 static cudaError_t launch_dual_k(const CUtensorMap &tm, int grid, uint32_t rows, uint32_t cols, uint32_t n_tiles,
-                                 TileOrder order, uint8_t *re, uint8_t *rs, uint32_t rdim, uint8_t *ce, uint8_t *cs,
-                                 uint32_t cdim, int v8, int *wd, cudaStream_t st) {
-    auto k = quant_dual_kernel<FMT, CEIL, ROW, TC>;
+                                 TileOrder order, uint8_t *re, const ScaleOut &rs, uint8_t *ce, const ScaleOut &cs,
+                                 int v8, int *wd, cudaStream_t st) {
+    auto k = quant_dual_kernel<FMT, CEIL, ROW, RM, TC>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDualSmem);
     if (e != cudaSuccess) return e;
-    k<<<grid, kDualThreads, kDualSmem, st>>>(tm, rows, cols, n_tiles, order, re, rs, rdim, ce, cs, cdim, v8, wd);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kDualThreads);
+    cfg.dynamicSmemBytes = kDualSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, tm, rows, cols, n_tiles, order, re, rs, ce, cs, v8, wd);
+}
+
+template <int FMT, bool CEIL, bool ROW>
+static cudaError_t launch_dual_l(const CUtensorMap &tm, int grid, uint32_t rows, uint32_t cols, uint32_t n_tiles,
+                                 TileOrder d, uint8_t *re, const ScaleOut &rs, uint8_t *ce, const ScaleOut &cs,
+                                 int v8, int *wd, cudaStream_t st) {
+    if (cs.rm && cs.tc)
+        return launch_dual_k<FMT, CEIL, ROW, true, true>(tm, grid, rows, cols, n_tiles, d, re, rs, ce, cs, v8, wd, st);
+    if (cs.rm)
+        return launch_dual_k<FMT, CEIL, ROW, true, false>(tm, grid, rows, cols, n_tiles, d, re, rs, ce, cs, v8, wd, st);
+    return launch_dual_k<FMT, CEIL, ROW, false, true>(tm, grid, rows, cols, n_tiles, d, re, rs, ce, cs, v8, wd, st);
 }
 
 template <int FMT, bool CEIL>
-static cudaError_t launch_dual_t(bool row, bool tc, const CUtensorMap &tm, int grid, uint32_t rows, uint32_t cols,
-                                 uint32_t n_tiles, TileOrder d, uint8_t *re, uint8_t *rs, uint32_t rdim, uint8_t *ce,
-                                 uint8_t *cs, uint32_t cdim, int v8, int *wd, cudaStream_t st) {
-    if (row)
-        return tc ? launch_dual_k<FMT, CEIL, true, true>(tm, grid, rows, cols, n_tiles, d, re, rs, rdim, ce, cs, cdim, v8, wd, st)
-                  : launch_dual_k<FMT, CEIL, true, false>(tm, grid, rows, cols, n_tiles, d, re, rs, rdim, ce, cs, cdim, v8, wd, st);
-    return tc ? launch_dual_k<FMT, CEIL, false, true>(tm, grid, rows, cols, n_tiles, d, re, rs, rdim, ce, cs, cdim, v8, wd, st)
-              : launch_dual_k<FMT, CEIL, false, false>(tm, grid, rows, cols, n_tiles, d, re, rs, rdim, ce, cs, cdim, v8, wd, st);
+static cudaError_t launch_dual_t(bool row, const CUtensorMap &tm, int grid, uint32_t rows, uint32_t cols,
+                                 uint32_t n_tiles, TileOrder d, uint8_t *re, const ScaleOut &rs, uint8_t *ce,
+                                 const ScaleOut &cs, int v8, int *wd, cudaStream_t st) {
+    return row ? launch_dual_l<FMT, CEIL, true>(tm, grid, rows, cols, n_tiles, d, re, rs, ce, cs, v8, wd, st)
+               : launch_dual_l<FMT, CEIL, false>(tm, grid, rows, cols, n_tiles, d, re, rs, ce, cs, v8, wd, st);
 }
 
 cudaError_t launch_quant_dual(const void *src, int64_t rows, int64_t cols, int fmt, bool ceil,
-                              void *row_elems, uint8_t *row_sc, void *col_elems, uint8_t *col_sc,
-                              bool tc, int *watchdog, int num_sms, cudaStream_t st) {
+                              void *row_elems, uint8_t *row_rm, uint8_t *row_tc, void *col_elems, uint8_t *col_rm,
+                              uint8_t *col_tc, int *watchdog, int num_sms, cudaStream_t st) {
     // Preconditions (checked by the caller): rows % 32 == 0, cols % 8 == 0 (cols % 32 == 0
-    // with the row-wise output), 16-byte aligned source and outputs, column output present.
-    if (!col_elems || !col_sc) return cudaErrorInvalidValue;
+    // with the row-wise output), 16-byte aligned source and outputs, column output present
+    // with at least one scale layout; the row-wise output, when present, gets the same
+    // scale layouts as the column-wise one.
+    if (!col_elems || (!col_rm && !col_tc)) return cudaErrorInvalidValue;
     const bool row = row_elems != nullptr;
-    if (row && !row_sc) return cudaErrorInvalidValue;
+    if (row && ((row_rm != nullptr) != (col_rm != nullptr) || (row_tc != nullptr) != (col_tc != nullptr)))
+        return cudaErrorInvalidValue;
     auto encode = reinterpret_cast<EncodeTiledFn>(tensor_map_encoder());
     if (!encode) return cudaErrorNotSupported;
     CUtensorMap tm;
@@ -359,25 +391,26 @@ cudaError_t launch_quant_dual(const void *src, int64_t rows, int64_t cols, int f
     d.n_full = tiles_c / kBand * kBand * tiles_r;
     d.last_w = make_fastdiv(tiles_c % kBand ? tiles_c % kBand : 1);
     d.last_c0 = tiles_c / kBand * kBand;
-    // scale-array geometry: per-row scale count (row-major) or 4-column atom count (tcgen05)
+    // scale-array geometry: scales per row (row-major) and 4-column atoms (tcgen05)
     const uint32_t row_S = (uint32_t)(cols / 32), col_S = (uint32_t)(rows / 32);
-    const uint32_t rdim = tc ? (row_S + 3) / 4 : row_S, cdim = tc ? (col_S + 3) / 4 : col_S;
+    const ScaleOut rs{row_rm, row_tc, row_S, (row_S + 3) / 4};
+    const ScaleOut cs{col_rm, col_tc, col_S, (col_S + 3) / 4};
     uint8_t *re = static_cast<uint8_t *>(row_elems), *ce = static_cast<uint8_t *>(col_elems);
     const int v8 = ((reinterpret_cast<uintptr_t>(re) | reinterpret_cast<uintptr_t>(ce)) & 31u) == 0;
     const uint32_t R = (uint32_t)rows, C = (uint32_t)cols;
     switch (fmt * 2 + (ceil ? 1 : 0)) {
-    case FMT_E4M3 * 2 + 0: return launch_dual_t<FMT_E4M3, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_E4M3 * 2 + 1: return launch_dual_t<FMT_E4M3, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_E5M2 * 2 + 0: return launch_dual_t<FMT_E5M2, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_E5M2 * 2 + 1: return launch_dual_t<FMT_E5M2, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_E2M1 * 2 + 0: return launch_dual_t<FMT_E2M1, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_E2M1 * 2 + 1: return launch_dual_t<FMT_E2M1, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_E2M3 * 2 + 0: return launch_dual_t<FMT_E2M3, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_E2M3 * 2 + 1: return launch_dual_t<FMT_E2M3, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_E3M2 * 2 + 0: return launch_dual_t<FMT_E3M2, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_E3M2 * 2 + 1: return launch_dual_t<FMT_E3M2, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_INT8 * 2 + 0: return launch_dual_t<FMT_INT8, false>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
-    case FMT_INT8 * 2 + 1: return launch_dual_t<FMT_INT8, true>(row, tc, tm, grid, R, C, n_tiles, d, re, row_sc, rdim, ce, col_sc, cdim, v8, watchdog, st);
+    case FMT_E4M3 * 2 + 0: return launch_dual_t<FMT_E4M3, false>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_E4M3 * 2 + 1: return launch_dual_t<FMT_E4M3, true>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_E5M2 * 2 + 0: return launch_dual_t<FMT_E5M2, false>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_E5M2 * 2 + 1: return launch_dual_t<FMT_E5M2, true>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_E2M1 * 2 + 0: return launch_dual_t<FMT_E2M1, false>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_E2M1 * 2 + 1: return launch_dual_t<FMT_E2M1, true>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_E2M3 * 2 + 0: return launch_dual_t<FMT_E2M3, false>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_E2M3 * 2 + 1: return launch_dual_t<FMT_E2M3, true>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_E3M2 * 2 + 0: return launch_dual_t<FMT_E3M2, false>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_E3M2 * 2 + 1: return launch_dual_t<FMT_E3M2, true>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_INT8 * 2 + 0: return launch_dual_t<FMT_INT8, false>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
+    case FMT_INT8 * 2 + 1: return launch_dual_t<FMT_INT8, true>(row, tm, grid, R, C, n_tiles, d, re, rs, ce, cs, v8, watchdog, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -10,20 +10,25 @@ namespace mxk {
 // True when the block indices of a rows x cols tensor fit the kernels' 31-bit indexing.
 bool stream_supported(int64_t rows, int64_t cols);
 
-// Row-wise MX quantiser (blocks of 32 along rows); row-major and/or tcgen05 scales.
+// Row-wise MX quantiser (blocks of 32 along rows); row-major and/or tcgen05 scales.  With
+// `partials` non-null, each of its stream_rows_grid() CTAs also writes the finite |x|
+// maximum of what it read to partials[cta] (the NVFP4 per-tensor maximum's partials).
+int stream_rows_grid(int64_t rows, int64_t cols, int num_sms);
 cudaError_t launch_stream_rows_mx(const void *src, int64_t rows, int64_t cols, int fmt, bool ceil, void *elems,
-                                  uint8_t *sc_rowmajor, uint8_t *sc_tcgen05, int *watchdog, int num_sms,
-                                  cudaStream_t st);
+                                  uint8_t *sc_rowmajor, uint8_t *sc_tcgen05, float *partials, int *watchdog,
+                                  int num_sms, cudaStream_t st);
 
 // NVFP4 scratch: one partial maximum per CTA of the maximum pass (no initial value needed:
 // every call writes each slot it later reads).  Returns the float count the launch below
 // needs on a device with num_sms SMs.
 int stream_nvfp4_scratch_floats(int num_sms);
 // NVFP4 quantisation (tensor amax -> g written to *global_scale -> block scales and codes)
-// as two kernels; the maximum pass uses at most max_partials CTAs.
+// as two kernels; the maximum pass uses at most max_partials CTAs.  n_given > 0: the
+// n_given partial maxima are already in `partials` (written by an earlier kernel on the
+// stream) and only the quantisation pass runs.
 cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,
-                                float *global_scale, void *elems, uint8_t *sc_rowmajor, uint8_t *sc_tcgen05,
-                                int *watchdog, int num_sms, cudaStream_t st);
+                                int n_given, float *global_scale, void *elems, uint8_t *sc_rowmajor,
+                                uint8_t *sc_tcgen05, int *watchdog, int num_sms, cudaStream_t st);
 
 // NVFP4 with 16 x 16 blocks (rows, cols multiples of 16); scales in the 1 x 16 layouts.
 cudaError_t launch_stream_nvfp4_2d(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,
@@ -45,10 +50,12 @@ cudaError_t launch_cast(const void *src, int64_t n, int fmt, void *out, int num_
 cudaError_t launch_watchdog_selftest(uint64_t limit_ns, int *watchdog, cudaStream_t st);
 
 // ---- dual.cu -------------------------------------------------------------------------------------
-// TMA-staged quantiser producing the row-wise and/or the column-wise (transposed) output.
+// TMA-staged quantiser producing the column-wise (transposed) output and optionally the
+// row-wise one (row_elems non-null), with scales in the row-major layout (*_rm), the
+// tcgen05 tiling (*_tc) or both; the row-wise output takes the same layouts.
 cudaError_t launch_quant_dual(const void *src, int64_t rows, int64_t cols, int fmt, bool ceil,
-                              void *row_elems, uint8_t *row_sc, void *col_elems, uint8_t *col_sc,
-                              bool tcgen05, int *watchdog, int num_sms, cudaStream_t st);
+                              void *row_elems, uint8_t *row_rm, uint8_t *row_tc, void *col_elems, uint8_t *col_rm,
+                              uint8_t *col_tc, int *watchdog, int num_sms, cudaStream_t st);
 
 // ---- gemm.cu -------------------------------------------------------------------------------------
 // tcgen05 block-scaled matmul C = alpha A * B^T.  Format pairs: E4M3 x {E4M3, E2M1}

@@ -90,7 +90,7 @@ extern "C" mx_status mx_quantize_nvfp4_noalloc(const void *src_bf16, int64_t row
     if (needed > MX_NOALLOC_MAX_PARTIALS) return MX_ERR_SHAPE;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = mxk::launch_stream_nvfp4(src_bf16, rows, cols, d->scratch, MX_NOALLOC_MAX_PARTIALS,
+    cudaError_t e = mxk::launch_stream_nvfp4(src_bf16, rows, cols, d->scratch, MX_NOALLOC_MAX_PARTIALS, 0,
                                              global_scale, out_elems, rm, tc, d->watchdog, d->num_sms, s);
     if (e == cudaSuccess && tc) e = mxk::launch_tcgen05_pad(tc, rows, cols / 16, s);
     if (e != cudaSuccess) { mxk::record_cuda_error(e); return MX_ERR_CUDA; }

@@ -142,23 +142,44 @@ __device__ __forceinline__ uint32_t amax_words(uint32_t a, uint32_t b, uint32_t 
     return __vmaxu2(__vmaxu2(a & 0x7FFF7FFFu, b & 0x7FFF7FFFu), __vmaxu2(c & 0x7FFF7FFFu, d & 0x7FFF7FFFu));
 }
 
+// Block-wide maximum of a per-thread |x| maximum (bf16 bits in either half); thread 0
+// stores it as fp32.
+__device__ __forceinline__ void store_partial(uint32_t acc, float *dst, uint32_t *warp_u) {
+    const uint32_t tid = threadIdx.x;
+    uint32_t m = hmax(acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) warp_u[tid >> 5] = m;
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t r = 0;
+        for (int w = 0; w < kThreads / 32; w++) r = max(r, warp_u[w]);
+        *dst = __uint_as_float(r << 16);
+    }
+}
+
 // ---------------------------------------------------------------------------------------
 // Row-wise MX quantiser: thread = one 32-element block (64 input bytes).
 // ---------------------------------------------------------------------------------------
+// partials: when non-null, the CTA also reduces the finite |x| maximum of everything it
+// read (Inf / NaN excluded) into partials[blockIdx.x] -- the NVFP4 per-tensor maximum of
+// the same tensor, so that an NVFP4 quantisation of it needs no maximum pass of its own.
 template <int FMT, bool CEIL, bool RM, bool TC>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 mx_rows_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
                uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc,
-               int *watchdog) {
+               float *__restrict__ partials, int *watchdog) {
     pdl_wait_and_release();
     extern __shared__ __align__(128) uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ uint32_t warp_u[kThreads / 32];
     Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
               full, watchdog, src, kTileBytes, (uint64_t)n_blocks * 64};
     constexpr uint32_t kBlocksPerTile = kTileBytes / 64;   // 256 = one per thread
     const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
     const uint32_t tid = threadIdx.x;
     const uint32_t rot = tid >> 1;                          // bank-group rotation
+    uint32_t finite_acc = 0;                                // finite |x| maximum (bf16 bits)
 
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
         const uint32_t blk = t * kBlocksPerTile + tid;
@@ -170,6 +191,13 @@ mx_rows_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS,
             v[j] = *reinterpret_cast<const uint4 *>(tile + tid * 64 + c * 16);
         }
         const uint32_t m = absmax_block32(v);
+        if (partials) {
+            uint32_t f = m;
+            if (__builtin_expect(m >= 0x7F80u, 0))          // Inf / NaN in the block: mask them out
+                f = hmax(__vmaxu2(__vmaxu2(finite_abs_max_bf16x8(v[0]), finite_abs_max_bf16x8(v[1])),
+                                  __vmaxu2(finite_abs_max_bf16x8(v[2]), finite_abs_max_bf16x8(v[3]))));
+            finite_acc = max(finite_acc, f);
+        }
         const uint32_t code = e8m0_from_amax_bits<FMT, CEIL>(m);
         const uint64_t mul2x = splat2(e8m0_inverse_multiplier(code));
         const bool nan_blk = code == 0xFFu;
@@ -218,6 +246,7 @@ mx_rows_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS,
             sc_tc[tc_offset(r, blk - r * divS.d, col_atoms)] = (uint8_t)code;
         }
     });
+    if (partials) store_partial(finite_acc, partials + blockIdx.x, warp_u);
 }
 
 __device__ __forceinline__ uint32_t finite_mask(uint32_t m) {
@@ -359,20 +388,6 @@ __device__ __forceinline__ uint32_t finite_amax_tile(const uint8_t *tile, uint32
     return acc;
 }
 
-// Block-wide maximum of a per-thread packed |x| maximum; thread 0 stores it as fp32.
-__device__ __forceinline__ void store_partial(uint32_t acc, float *dst, uint32_t *warp_u) {
-    const uint32_t tid = threadIdx.x;
-    uint32_t m = hmax(acc);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((tid & 31) == 0) warp_u[tid >> 5] = m;
-    __syncthreads();
-    if (tid == 0) {
-        uint32_t r = 0;
-        for (int w = 0; w < kThreads / 32; w++) r = max(r, warp_u[w]);
-        *dst = __uint_as_float(r << 16);
-    }
-}
 
 // ---------------------------------------------------------------------------------------
 // NVFP4 as two kernels.  Pass 1: per-CTA maximum of the finite |x| (Inf/NaN excluded).
@@ -702,40 +717,46 @@ bool stream_supported(int64_t rows, int64_t cols) {
 
 template <int FMT, bool CEIL, bool RM, bool TC>
 static cudaError_t launch_rows_t(const void *src, uint32_t n_blocks, FastDiv f, uint32_t col_atoms, void *elems,
-                                 uint8_t *rm, uint8_t *tc, int *wd, int num_sms, cudaStream_t st) {
-    const uint32_t n_tiles = (n_blocks + 255) / 256;
-    return launch_stream(mx_rows_kernel<FMT, CEIL, RM, TC>, stream_grid(n_tiles, num_sms), st,
-                         static_cast<const uint8_t *>(src), n_blocks, f, col_atoms, static_cast<uint8_t *>(elems), rm,
-                         tc, wd);
+                                 uint8_t *rm, uint8_t *tc, float *partials, int grid, int *wd, cudaStream_t st) {
+    return launch_stream(mx_rows_kernel<FMT, CEIL, RM, TC>, grid, st, static_cast<const uint8_t *>(src), n_blocks, f,
+                         col_atoms, static_cast<uint8_t *>(elems), rm, tc, partials, wd);
 }
 
 template <int FMT, bool CEIL>
 static cudaError_t launch_rows_layout(const void *src, uint32_t nb, FastDiv f, uint32_t ca, void *elems, uint8_t *rm,
-                                      uint8_t *tc, int *wd, int num_sms, cudaStream_t st) {
-    if (rm && tc) return launch_rows_t<FMT, CEIL, true, true>(src, nb, f, ca, elems, rm, tc, wd, num_sms, st);
-    if (rm) return launch_rows_t<FMT, CEIL, true, false>(src, nb, f, ca, elems, rm, tc, wd, num_sms, st);
-    return launch_rows_t<FMT, CEIL, false, true>(src, nb, f, ca, elems, rm, tc, wd, num_sms, st);
+                                      uint8_t *tc, float *p, int grid, int *wd, cudaStream_t st) {
+    if (rm && tc) return launch_rows_t<FMT, CEIL, true, true>(src, nb, f, ca, elems, rm, tc, p, grid, wd, st);
+    if (rm) return launch_rows_t<FMT, CEIL, true, false>(src, nb, f, ca, elems, rm, tc, p, grid, wd, st);
+    return launch_rows_t<FMT, CEIL, false, true>(src, nb, f, ca, elems, rm, tc, p, grid, wd, st);
+}
+
+// Grid of the row-wise MX kernel for a rows x cols tensor (its CTA count is also the number
+// of partial maxima it writes when asked to).
+int stream_rows_grid(int64_t rows, int64_t cols, int num_sms) {
+    const uint32_t n_tiles = (uint32_t)((rows * cols / 32 + 255) / 256);
+    return stream_grid(n_tiles, num_sms);
 }
 
 cudaError_t launch_stream_rows_mx(const void *src, int64_t rows, int64_t cols, int fmt, bool ceil, void *elems,
-                                  uint8_t *rm, uint8_t *tc, int *wd, int num_sms, cudaStream_t st) {
+                                  uint8_t *rm, uint8_t *tc, float *partials, int *wd, int num_sms, cudaStream_t st) {
     const uint32_t n_blocks = (uint32_t)(rows * cols / 32);
     const uint32_t S = (uint32_t)(cols / 32);
     const FastDiv f = make_fastdiv(S);
     const uint32_t ca = (S + 3) / 4;
+    const int g = stream_rows_grid(rows, cols, num_sms);
     switch (fmt * 2 + (ceil ? 1 : 0)) {
-    case FMT_E4M3 * 2 + 0: return launch_rows_layout<FMT_E4M3, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_E4M3 * 2 + 1: return launch_rows_layout<FMT_E4M3, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_E5M2 * 2 + 0: return launch_rows_layout<FMT_E5M2, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_E5M2 * 2 + 1: return launch_rows_layout<FMT_E5M2, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_E2M1 * 2 + 0: return launch_rows_layout<FMT_E2M1, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_E2M1 * 2 + 1: return launch_rows_layout<FMT_E2M1, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_E2M3 * 2 + 0: return launch_rows_layout<FMT_E2M3, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_E2M3 * 2 + 1: return launch_rows_layout<FMT_E2M3, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_E3M2 * 2 + 0: return launch_rows_layout<FMT_E3M2, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_E3M2 * 2 + 1: return launch_rows_layout<FMT_E3M2, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_INT8 * 2 + 0: return launch_rows_layout<FMT_INT8, false>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
-    case FMT_INT8 * 2 + 1: return launch_rows_layout<FMT_INT8, true>(src, n_blocks, f, ca, elems, rm, tc, wd, num_sms, st);
+    case FMT_E4M3 * 2 + 0: return launch_rows_layout<FMT_E4M3, false>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_E4M3 * 2 + 1: return launch_rows_layout<FMT_E4M3, true>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_E5M2 * 2 + 0: return launch_rows_layout<FMT_E5M2, false>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_E5M2 * 2 + 1: return launch_rows_layout<FMT_E5M2, true>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_E2M1 * 2 + 0: return launch_rows_layout<FMT_E2M1, false>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_E2M1 * 2 + 1: return launch_rows_layout<FMT_E2M1, true>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_E2M3 * 2 + 0: return launch_rows_layout<FMT_E2M3, false>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_E2M3 * 2 + 1: return launch_rows_layout<FMT_E2M3, true>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_E3M2 * 2 + 0: return launch_rows_layout<FMT_E3M2, false>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_E3M2 * 2 + 1: return launch_rows_layout<FMT_E3M2, true>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_INT8 * 2 + 0: return launch_rows_layout<FMT_INT8, false>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
+    case FMT_INT8 * 2 + 1: return launch_rows_layout<FMT_INT8, true>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -744,14 +765,18 @@ int stream_nvfp4_scratch_floats(int num_sms) { return kCtasPerSm * num_sms; }
 
 template <bool RM, bool TC>
 static cudaError_t launch_nvfp4_t(const uint8_t *src, uint32_t nb, FastDiv f, uint32_t ca, float *partials,
-                                  int max_partials, float *g, uint8_t *elems, uint8_t *rm, uint8_t *tc, int *wd,
-                                  int num_sms, cudaStream_t st) {
+                                  int max_partials, int n_given, float *g, uint8_t *elems, uint8_t *rm, uint8_t *tc,
+                                  int *wd, int num_sms, cudaStream_t st) {
     const uint32_t n_tiles = (nb + 511) / 512;
-    int grid = stream_grid(n_tiles, num_sms);
-    if (grid > max_partials) grid = max_partials;
-    // pass 1: per-CTA maxima; pass 2 (programmatic dependent launch): quantisation
-    cudaError_t e = launch_stream(nvfp4_amax_bulk_kernel, grid, st, src, (uint64_t)nb * 32, partials, wd);
-    if (e != cudaSuccess) return e;
+    int grid = n_given;
+    if (grid == 0) {
+        // pass 1: per-CTA maxima
+        grid = stream_grid(n_tiles, num_sms);
+        if (grid > max_partials) grid = max_partials;
+        cudaError_t e = launch_stream(nvfp4_amax_bulk_kernel, grid, st, src, (uint64_t)nb * 32, partials, wd);
+        if (e != cudaSuccess) return e;
+    }
+    // pass 2 (programmatic dependent launch): quantisation
     return launch_stream(nvfp4_quant_bulk_kernel<RM, TC>, stream_grid(n_tiles, num_sms), st, src, nb, f, ca,
                          (const float *)partials, grid, g, elems, rm, tc, wd);
 }
@@ -786,16 +811,18 @@ cudaError_t launch_stream_nvfp4_2d(const void *src, int64_t rows, int64_t cols, 
 }
 
 cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,
-                                float *g, void *elems, uint8_t *rm, uint8_t *tc, int *wd, int num_sms,
+                                int n_given, float *g, void *elems, uint8_t *rm, uint8_t *tc, int *wd, int num_sms,
                                 cudaStream_t st) {
     const uint32_t nb = (uint32_t)(rows * cols / 16), S = (uint32_t)(cols / 16);
     const FastDiv f = make_fastdiv(S);
     const uint32_t ca = (S + 3) / 4;
     const uint8_t *s8 = static_cast<const uint8_t *>(src);
     uint8_t *e8 = static_cast<uint8_t *>(elems);
-    if (rm && tc) return launch_nvfp4_t<true, true>(s8, nb, f, ca, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
-    if (rm) return launch_nvfp4_t<true, false>(s8, nb, f, ca, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
-    return launch_nvfp4_t<false, true>(s8, nb, f, ca, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
+    if (rm && tc)
+        return launch_nvfp4_t<true, true>(s8, nb, f, ca, partials, max_partials, n_given, g, e8, rm, tc, wd, num_sms, st);
+    if (rm)
+        return launch_nvfp4_t<true, false>(s8, nb, f, ca, partials, max_partials, n_given, g, e8, rm, tc, wd, num_sms, st);
+    return launch_nvfp4_t<false, true>(s8, nb, f, ca, partials, max_partials, n_given, g, e8, rm, tc, wd, num_sms, st);
 }
 
 template <int FMT, bool TC>

@@ -81,11 +81,16 @@ def test_quantize_validation(L, args, status):
 
 def test_dual_dequant_cast_gemm_validation(L):
     lib = L.lib
-    assert lib.mx_quantize_dual(FAKE, 64, 64, 3, 1, FAKE, FAKE, FAKE, FAKE, 1, None) == L.MX_ERR_ARG
-    assert lib.mx_quantize_dual(FAKE, 64, 64, 0, 1, FAKE, FAKE, FAKE, FAKE, 3, None) == L.MX_ERR_LAYOUT
-    assert lib.mx_quantize_dual(FAKE, 48, 64, 0, 1, FAKE, FAKE, FAKE, FAKE, 1, None) == L.MX_ERR_SHAPE
-    assert lib.mx_quantize_dual(FAKE, 64, 64, 0, 1, FAKE, FAKE, None, FAKE, 1, None) == L.MX_ERR_ARG
-    assert lib.mx_quantize_dual(FAKE, 0, 64, 0, 1, None, None, None, None, 1, None) == L.MX_OK
+    assert lib.mx_quantize_dual(FAKE, 64, 64, 3, 1, FAKE, FAKE, FAKE, FAKE, 1, None, None, None) == L.MX_ERR_ARG
+    # both layouts need both alternate buffers; a single layout takes none
+    assert lib.mx_quantize_dual(FAKE, 64, 64, 0, 1, FAKE, FAKE, FAKE, FAKE, 3, None, None, None) == L.MX_ERR_LAYOUT
+    assert lib.mx_quantize_dual(FAKE, 64, 64, 0, 1, FAKE, FAKE, FAKE, FAKE, 3, FAKE, None, None) == L.MX_ERR_LAYOUT
+    assert lib.mx_quantize_dual(FAKE, 64, 64, 0, 1, FAKE, FAKE, FAKE, FAKE, 1, FAKE, FAKE, None) == L.MX_ERR_LAYOUT
+    assert lib.mx_quantize_dual(FAKE, 64, 64, 0, 1, FAKE, FAKE, FAKE, FAKE, 4, None, None, None) == L.MX_ERR_LAYOUT
+    assert lib.mx_quantize_dual(FAKE, 48, 64, 0, 1, FAKE, FAKE, FAKE, FAKE, 1, None, None, None) == L.MX_ERR_SHAPE
+    assert lib.mx_quantize_dual(FAKE, 64, 64, 0, 1, FAKE, FAKE, None, FAKE, 1, None, None, None) == L.MX_ERR_ARG
+    assert lib.mx_quantize_dual(FAKE, 0, 64, 0, 1, None, None, None, None, 1, None, None, None) == L.MX_OK
+    assert lib.mx_quantize_dual(FAKE, 0, 64, 0, 1, None, None, None, None, 3, FAKE, FAKE, None) == L.MX_OK
     assert lib.mx_dequantize(FAKE, FAKE, None, 4, 48, 0, 1, FAKE, None) == L.MX_ERR_SHAPE
     assert lib.mx_dequantize(FAKE, FAKE, None, 4, 64, 3, 1, FAKE, None) == L.MX_ERR_ARG
     assert lib.mx_dequantize(FAKE, FAKE, None, 4, 64, 0, 3, FAKE, None) == L.MX_ERR_LAYOUT
@@ -203,3 +208,25 @@ def test_watchdog_selftest_rejects_limits(L, limit_us):
     """The watchdog self-test takes a limit of 1 .. 100000 microseconds; anything else is
     rejected before any CUDA call."""
     assert L.lib.mx_watchdog_selftest(limit_us, None) == L.MX_ERR_ARG
+
+
+def test_mx_nvfp4_pair_validation(L):
+    """mx_quantize_mx_nvfp4 rejects bad formats, layouts, shapes and pointers on the host."""
+    f = FAKE
+    q = L.lib.mx_quantize_mx_nvfp4
+    # (fmt, rounding, mx_layout, mx_alt, nv_layout, nv_alt, cols, g, src) -> status
+    cases = [
+        ((3, 1, 1, None, 1, None, 64, f, f), L.MX_ERR_ARG),        # NVFP4 is not an MX format
+        ((2, 7, 1, None, 1, None, 64, f, f), L.MX_ERR_ARG),        # bad rounding
+        ((2, 0, 3, None, 1, None, 64, f, f), L.MX_ERR_LAYOUT),     # both layouts need the second buffer
+        ((2, 0, 1, None, 3, None, 64, f, f), L.MX_ERR_LAYOUT),
+        ((2, 0, 1, f, 1, None, 64, f, f), L.MX_ERR_LAYOUT),        # one layout takes none
+        ((2, 0, 0, None, 1, None, 64, f, f), L.MX_ERR_LAYOUT),
+        ((2, 0, 1, None, 1, None, 48, f, f), L.MX_ERR_SHAPE),      # cols % 32
+        ((2, 0, 1, None, 1, None, 64, None, f), L.MX_ERR_ARG),     # NVFP4 needs the tensor-scale slot
+        ((2, 0, 1, None, 1, None, 64, f, f + 8), L.MX_ERR_ALIGN),
+    ]
+    for (fmt, rnd, ml, ma, nl, na, cols, g, src), want in cases:
+        st = q(src, 64, cols, fmt, rnd, f, f, ml, ma, f, f, nl, na, g, None)
+        assert st == want, (fmt, rnd, ml, nl, cols, L.lib.mx_status_string(st))
+    assert q(None, 0, 64, 2, 0, None, None, 1, None, None, None, 1, None, None, None) == L.MX_OK

@@ -42,12 +42,21 @@ def test_dual_full_size_every_byte(oracle, which):
     against the oracle's row-wise and column-wise quantisation of the whole tensor."""
     x, fmt = (synth.activations(), 0) if which == "activations" else (synth.gradients(), 1)
     R, C = x.shape
-    qr, qc = mx.quantize_dual(to_dev(x), FMT_NAMES[fmt], "ceil", "tcgen05")
+    xd = to_dev(x)
+    qr, qc = mx.quantize_dual(xd, FMT_NAMES[fmt], "ceil", "tcgen05")
     re_, rs, ce, cs = quantize_mx_both(oracle, x, fmt, oracle.CEIL)
     assert np.array_equal(host(qr.elems).reshape(R, C), re_)
     assert np.array_equal(host(qc.elems).reshape(C, R), ce)
     assert np.array_equal(host(qr.scales), oracle.to_tcgen05_layout(rs))
     assert np.array_equal(host(qc.scales), oracle.to_tcgen05_layout(cs))
+    del qr, qc
+    # both scale layouts from the same single pass
+    qr, qc = mx.quantize_dual(xd, FMT_NAMES[fmt], "ceil", "both")
+    assert np.array_equal(host(qr.scales).reshape(R, C // 32), rs)
+    assert np.array_equal(host(qc.scales).reshape(C, R // 32), cs)
+    assert np.array_equal(host(qr.scales_alt), oracle.to_tcgen05_layout(rs))
+    assert np.array_equal(host(qc.scales_alt), oracle.to_tcgen05_layout(cs))
+    assert np.array_equal(host(qc.elems).reshape(C, R), ce)
 
 
 @pytest.mark.parametrize("fmt", [4, 5, 6])

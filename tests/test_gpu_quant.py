@@ -133,18 +133,21 @@ def test_quantize_colwise_matches_oracle(oracle, shape, fmt, rounding):
 @pytest.mark.parametrize("shape", [(32, 32), (64, 160), (160, 384), (256, 1024)])
 @pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (1, "ceil"), (1, "floor"), (2, "floor"), (4, "floor"),
                                           (5, "ceil"), (6, "floor"), (6, "ceil")])
-@pytest.mark.parametrize("layout", ["rowmajor", "tcgen05"])
+@pytest.mark.parametrize("layout", ["rowmajor", "tcgen05", "both"])
 def test_quantize_dual_matches_oracle(oracle, shape, fmt, rounding, layout):
     x = with_specials(synth.gradients(*shape, seed=shape[0] + fmt), seed=shape[1])
     rnd = oracle.CEIL if rounding == "ceil" else oracle.FLOOR
     qr, qc = mx.quantize_dual(to_dev(x), FMT_NAMES[fmt], rounding, layout)
     er, sr = oracle.quantize_mx(x, fmt, oracle.ROW, rnd)
     ec, sc = oracle.quantize_mx(x, fmt, oracle.COL, rnd)
-    tr = (lambda s: s.reshape(-1)) if layout == "rowmajor" else oracle.to_tcgen05_layout
+    tr = oracle.to_tcgen05_layout if layout == "tcgen05" else (lambda s: s.reshape(-1))
     assert np.array_equal(host(qr.elems), er.reshape(-1))
     assert np.array_equal(host(qr.scales), tr(sr))
     assert np.array_equal(host(qc.elems), ec.reshape(-1))
     assert np.array_equal(host(qc.scales), tr(sc))
+    if layout == "both":                                  # the tcgen05 copies from the same pass
+        assert np.array_equal(host(qr.scales_alt), oracle.to_tcgen05_layout(sr))
+        assert np.array_equal(host(qc.scales_alt), oracle.to_tcgen05_layout(sc))
 
 
 # ------------------------------------------------------------------ NVFP4
@@ -332,3 +335,25 @@ def test_nvfp4_2d_weight_transposes(oracle):
     codes_t = np.stack([np.stack([r & 0xF, r >> 4], axis=1).reshape(-1) for r in et])
     assert np.array_equal(codes_t, codes.T)
     assert np.array_equal(host(q.scales).reshape(256, 32)[::16], host(qt.scales).reshape(512, 16)[::16].T)
+
+
+# ------------------------------------------------------------------ MX and NVFP4 of one tensor
+@pytest.mark.parametrize("shape", [(1, 32), (37, 96), (130, 256), (512, 4096), (4096, 4096)])
+@pytest.mark.parametrize("fmt,rounding", [(2, "floor"), (0, "ceil"), (6, "ceil")])
+@pytest.mark.parametrize("specials", [False, True])
+def test_mx_nvfp4_pair_matches_oracle(oracle, shape, fmt, rounding, specials):
+    """One call quantising the same weight to an MX format and to NVFP4 (the MX pass supplies
+    the NVFP4 tensor maximum, Inf / NaN excluded) equals the oracle for both."""
+    x = synth.weight_fp4(*shape, seed=shape[0] + fmt)
+    if specials:
+        x = with_specials(x, seed=shape[1])
+    qm, qn = mx.quantize_mx_nvfp4(to_dev(x), FMT_NAMES[fmt], rounding)
+    e, s = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.CEIL if rounding == "ceil" else oracle.FLOOR)
+    assert np.array_equal(host(qm.elems), e.reshape(-1))
+    assert np.array_equal(host(qm.scales), s.reshape(-1))
+    assert np.array_equal(host(qm.scales_alt), oracle.to_tcgen05_layout(s))
+    e, s, g = oracle.quantize_nvfp4(x)
+    assert host(qn.global_scale)[0] == np.float32(g)
+    assert np.array_equal(host(qn.elems), e.reshape(-1))
+    assert np.array_equal(host(qn.scales), s.reshape(-1))
+    assert np.array_equal(host(qn.scales_alt), oracle.to_tcgen05_layout(s))
