@@ -14,19 +14,21 @@
 // K-major; scales per 32 along K in the tcgen05 tiling (512-byte atoms of 128 rows x 4
 // scale columns).
 //
-// Kernel structure: persistent CTAs (one per SM, 10 warps), 128 x 256 output tiles
+// Kernel structure: persistent CTAs (one per SM, 11 warps), 128 x 256 output tiles
 // (128 x 128 when N is not a multiple of 256):
 //   warp 8  TMA producer: per 128-wide K step, 2-D TMA loads of the A tile (128 x 128 B)
 //           and the B tile (256 x 128 B, E2M1 expanded by the TMA to one byte per
 //           element) with 128-byte swizzle, plus bulk copies of the matching scale atoms
 //           (1 for A, 2 for B) into a 4-stage shared-memory ring (mbarrier "full"); the
 //           ring runs on across tile boundaries.
-//   warp 9  TMEM allocator and MMA issuer: copies the stage's scale atoms into tensor
-//           memory (tcgen05.cp 32x128b.warpx4), then issues four
+//   warp 10 scale copier: copies the stage's scale atoms into tensor memory
+//           (tcgen05.cp 32x128b.warpx4) and commits to the stage's "sf_ready" barrier.
+//   warp 9  TMEM allocator and MMA issuer: waits on "sf_ready", issues four
 //           tcgen05.mma.kind::mxf8f6f4.block_scale (K = 32 each; the scale byte of each
 //           is selected by the scale-factor id in the instruction descriptor), and
 //           releases the stage with tcgen05.commit on its "empty" barrier; a finished
 //           tile is signalled on "acc_full".
+//   The three issuing warps run their loops converged and issue from one elected lane.
 //   warps 0-7  epilogue: two warps per 32-lane TMEM quadrant (one per column half) load
 //           the fp32 accumulator (tcgen05.ld), convert to bf16 in registers, release the
 //           accumulator on "acc_empty" -- the next tile's MMAs start now -- and then
@@ -125,23 +127,24 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     for (int s = 0; s < kStages; s++) last_it[s] = -1;
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer
-        if (lane == 0) {
-            // scale atoms per 128-row block of an operand (the tcgen05 layout's column-atom count)
-            const int64_t col_atoms = (int64_t)num_kb * T::kAtoms;
-            const uint32_t tx = (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kABytes, a_fmt_code) : kABytes) +
-                                (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kBBytes, b_fmt_code) : kBBytes) +
-                                kSfaBytes + kSfbBytes;
-            int it = 0;
-            for (int t = blockIdx.x; t < n_tiles && !*fail_sh; t += gridDim.x) {
-                int m_blk, n_blk;
-                tile_coords(t, tiles_m, tiles_n, band, m_blk, n_blk);
-                for (int kb = 0; kb < num_kb; kb++, it++) {
-                    const int s = it % kStages;
-                    if (it >= kStages &&
-                        !mbar_wait_bounded(&empty_bar[s], (uint32_t)((it / kStages) - 1) & 1u, watchdog, WD_GEMM_EMPTY)) {
-                        *fail_sh = 1;
-                        break;
-                    }
+        // the whole warp runs the loop (warp-uniform waits); one elected lane issues
+        // scale atoms per 128-row block of an operand (the tcgen05 layout's column-atom count)
+        const int64_t col_atoms = (int64_t)num_kb * T::kAtoms;
+        const uint32_t tx = (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kABytes, a_fmt_code) : kABytes) +
+                            (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kBBytes, b_fmt_code) : kBBytes) +
+                            kSfaBytes + kSfbBytes;
+        int it = 0;
+        for (int t = blockIdx.x; t < n_tiles && !warp_failed(fail_sh); t += gridDim.x) {
+            int m_blk, n_blk;
+            tile_coords(t, tiles_m, tiles_n, band, m_blk, n_blk);
+            for (int kb = 0; kb < num_kb; kb++, it++) {
+                const int s = it % kStages;
+                if (it >= kStages &&
+                    !warp_wait(&empty_bar[s], (uint32_t)((it / kStages) - 1) & 1u, watchdog, WD_GEMM_EMPTY)) {
+                    *fail_sh = 1;
+                    break;
+                }
+                if (elect_one()) {
                     // E2M1 and FP6 tiles of the mxf8f6f4 kind land in shared memory padded to
                     // one 16-byte group per 16 codes, but the copy completes only the packed
                     // global bytes.  Either way a stage holds 128 bytes of K per row.
@@ -156,34 +159,33 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         bulk_load(sSFB + s * kSfbBytes + h * T::kSfaBytes,
                                   b_sc + ((int64_t)((BN / 128) * n_blk + h) * col_atoms + (int64_t)kb * T::kAtoms) * 512,
                                   T::kSfaBytes, &full_bar[s]);
-                    last_it[s] = it;
                 }
+                __syncwarp();
+                last_it[s] = it;
             }
         }
-        __syncwarp();
     } else if (warp == kSfWarp) {
         // ------------------------------------------------ scale-atom copier
         // Copies each stage's scale atoms into tensor memory as soon as the stage has
         // landed and signals sf_ready[s] once the copies are complete; the MMA issuer waits
-        // on sf_ready alone.  This takes the copies (3 to 12 per stage) off the single
-        // MMA-issuing thread, whose instruction latency otherwise bounds the tensor pipe.
-        // A stage's scale slot is rewritten only after full[s] of its next use, i.e. after
+        // on sf_ready alone, so the copies (3 to 12 per stage) stay off the MMA warp.  A
+        // stage's scale slot is rewritten only after full[s] of its next use, i.e. after
         // the MMAs that read it have completed (empty[s]).
-        if (lane == 0) {
-            const uint64_t sfa_d0 = sf_desc(smem_u32(sSFA)), sfb_d0 = sf_desc(smem_u32(sSFB));
-            int it = 0;
-            for (int t = blockIdx.x; t < n_tiles && !*fail_sh; t += gridDim.x) {
-                for (int kb = 0; kb < num_kb; kb++, it++) {
-                    const int s = it % kStages;
-                    if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(it / kStages) & 1u, watchdog, WD_GEMM_FULL)) {
-                        *fail_sh = 1;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sfb_t = tmem + kSfCol0 + s * T::kSfColsPerStage;
-                    const uint32_t sfa_t = sfb_t + T::kSfbCols;
-                    const uint64_t sfa_d = sfa_d0 + (uint64_t)((s * kSfaBytes) >> 4);
-                    const uint64_t sfb_d = sfb_d0 + (uint64_t)((s * kSfbBytes) >> 4);
+        const uint64_t sfa_d0 = sf_desc(smem_u32(sSFA)), sfb_d0 = sf_desc(smem_u32(sSFB));
+        int it = 0;
+        for (int t = blockIdx.x; t < n_tiles && !warp_failed(fail_sh); t += gridDim.x) {
+            for (int kb = 0; kb < num_kb; kb++, it++) {
+                const int s = it % kStages;
+                if (!warp_wait(&full_bar[s], (uint32_t)(it / kStages) & 1u, watchdog, WD_GEMM_FULL)) {
+                    *fail_sh = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sfb_t = tmem + kSfCol0 + s * T::kSfColsPerStage;
+                const uint32_t sfa_t = sfb_t + T::kSfbCols;
+                const uint64_t sfa_d = sfa_d0 + (uint64_t)((s * kSfaBytes) >> 4);
+                const uint64_t sfb_d = sfb_d0 + (uint64_t)((s * kSfbBytes) >> 4);
+                if (elect_one()) {
 #pragma unroll
                     for (int a = 0; a < T::kAtoms; a++) {
                         tc_cp_sf(sfa_t + 4 * a, sfa_d + (uint64_t)(a * 512 / 16));
@@ -193,49 +195,49 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     }
                     tc_commit(&sf_ready[s]);                  // the stage's scales are in tensor memory
                 }
+                __syncwarp();
             }
-            tc_commit(&sf_drain);                         // completes once every copy above has finished
         }
+        if (elect_one()) tc_commit(&sf_drain);            // completes once every copy above has finished
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            // Everything the issue loop needs is precomputed: one thread issues every
-            // copy and MMA, and at ~4 instructions per 128 tensor cycles its own latency
-            // decides whether the tensor pipe idles.  Descriptors advance by offsets >> 4
-            // (the 14-bit start-address field never overflows inside shared memory).
-            const uint64_t a_d0 = smem_desc(smem_u32(sA), 16, 1024, 2), b_d0 = smem_desc(smem_u32(sB), 16, 1024, 2);
-            uint32_t idesc[4];
+        // Descriptors are precomputed and advance by offsets >> 4 (the 14-bit start-address
+        // field never overflows inside shared memory); the whole warp runs the loop and one
+        // elected lane issues each stage's MMAs and its commit.
+        const uint64_t a_d0 = smem_desc(smem_u32(sA), 16, 1024, 2), b_d0 = smem_desc(smem_u32(sB), 16, 1024, 2);
+        uint32_t idesc[4];
 #pragma unroll
-            for (int k = 0; k < 4; k++)
-                idesc[k] = mma_idesc<kBM, BN, KIND>(
-                    a_fmt_code, b_fmt_code,
-                    KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u));
-            int it = 0, i = 0;
-            for (int t = blockIdx.x; t < n_tiles && !*fail_sh; t += gridDim.x, i++) {
-                if (i > 0 && !mbar_wait_bounded(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
+        for (int k = 0; k < 4; k++)
+            idesc[k] = mma_idesc<kBM, BN, KIND>(
+                a_fmt_code, b_fmt_code,
+                KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u));
+        int it = 0, i = 0;
+        for (int t = blockIdx.x; t < n_tiles && !warp_failed(fail_sh); t += gridDim.x, i++) {
+            if (i > 0 && !warp_wait(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
+                *fail_sh = 1;
+                break;
+            }
+            tc_fence_after();
+            for (int kb = 0; kb < num_kb; kb++, it++) {
+                const int s = it % kStages;
+                // the stage's operands have landed and its scales are in tensor memory
+                if (!warp_wait(&sf_ready[s], (uint32_t)(it / kStages) & 1u, watchdog, WD_GEMM_FULL)) {
                     *fail_sh = 1;
                     break;
                 }
                 tc_fence_after();
-                for (int kb = 0; kb < num_kb; kb++, it++) {
-                    const int s = it % kStages;
-                    // the stage's operands have landed and its scales are in tensor memory
-                    if (!mbar_wait_bounded(&sf_ready[s], (uint32_t)(it / kStages) & 1u, watchdog, WD_GEMM_FULL)) {
-                        *fail_sh = 1;
-                        break;
-                    }
-                    tc_fence_after();
-                    // tensor-memory scale slots of this stage: B atom (a, h) at column
-                    // sfb_t + 4 (a (BN/128) + h), A atom a at sfa_t + 4 a
-                    const uint32_t sfb_t = tmem + kSfCol0 + s * T::kSfColsPerStage;
-                    const uint32_t sfa_t = sfb_t + T::kSfbCols;
-                    const uint64_t a_d = a_d0 + (uint64_t)((s * kABytes) >> 4);
-                    const uint64_t b_d = b_d0 + (uint64_t)((s * kBBytes) >> 4);
-                    // four instructions per stage, each over 32 bytes of K per row (K = 32 for
-                    // 8-bit codes, 64 for packed 4-bit codes).  Instruction k reads scale atom
-                    // a and, inside its 32-bit words, the scale byte(s) starting at sf_id:
-                    // 1X: a = 0, sf_id = k; 2X: a = k / 2, sf_id = 2 (k % 2); 4X: a = k, sf_id = 0.
+                // tensor-memory scale slots of this stage: B atom (a, h) at column
+                // sfb_t + 4 (a (BN/128) + h), A atom a at sfa_t + 4 a
+                const uint32_t sfb_t = tmem + kSfCol0 + s * T::kSfColsPerStage;
+                const uint32_t sfa_t = sfb_t + T::kSfbCols;
+                const uint64_t a_d = a_d0 + (uint64_t)((s * kABytes) >> 4);
+                const uint64_t b_d = b_d0 + (uint64_t)((s * kBBytes) >> 4);
+                // four instructions per stage, each over 32 bytes of K per row (K = 32 for
+                // 8-bit codes, 64 for packed 4-bit codes).  Instruction k reads scale atom
+                // a and, inside its 32-bit words, the scale byte(s) starting at sf_id:
+                // 1X: a = 0, sf_id = k; 2X: a = k / 2, sf_id = 2 (k % 2); 4X: a = k, sf_id = 0.
+                if (elect_one()) {
 #pragma unroll
                     for (int k = 0; k < 4; k++) {
                         const int a = KIND == KIND_F8F6F4 ? 0 : (KIND == KIND_MXF4 ? k >> 1 : k);
@@ -244,11 +246,13 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     }
                     tc_commit(&empty_bar[s]);
                 }
-                if (*fail_sh) break;
-                tc_commit(&acc_full);                     // the tile's accumulator is complete
+                __syncwarp();
             }
-            tc_commit(&drain_bar);                        // completes once every MMA above has finished
+            if (warp_failed(fail_sh)) break;
+            if (elect_one()) tc_commit(&acc_full);        // the tile's accumulator is complete
+            __syncwarp();
         }
+        if (elect_one()) tc_commit(&drain_bar);           // completes once every MMA above has finished
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue (warps 0-7)

@@ -41,21 +41,28 @@ constexpr int kPairThreads = 352;
 constexpr uint32_t kTmemCols = 512, kSfCol0 = 256;
 constexpr uint32_t kPeerBitMask = 0xFEFFFFFFu;       // shared::cluster address of the even CTA's copy
 
-template <int KIND> struct Pair {
-    static constexpr int kStageK = KIND == KIND_F8F6F4 ? 128 : 256;
-    static constexpr int kAtoms = KIND == KIND_F8F6F4 ? 1 : (KIND == KIND_MXF4 ? 2 : 4);
-    static constexpr int kStages = KIND == KIND_NVF4 ? 5 : 6;
+// A pipeline stage holds SUB sub-tiles of 128 bytes of K per row (one 128-byte-swizzled TMA
+// box each): 4 x SUB MMAs per stage, so the per-stage barrier wait and commit of the
+// issuing thread are shared by more tensor work.
+template <int KIND, int SUB> struct Pair {
+    static constexpr int kSubK = KIND == KIND_F8F6F4 ? 128 : 256;          // K per sub-tile
+    static constexpr int kStageK = kSubK * SUB;
+    static constexpr int kSubAtoms = KIND == KIND_F8F6F4 ? 1 : (KIND == KIND_MXF4 ? 2 : 4);
+    static constexpr int kAtoms = kSubAtoms * SUB;   // scale atoms per 128 rows per stage
     static constexpr int kSfaBytes = 512 * kAtoms;   // this CTA's 128 A rows
     static constexpr int kSfbBytes = 1024 * kAtoms;  // all 256 B rows
-    static constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+    static constexpr int kAStage = kABytes * SUB, kBStage = kBBytes * SUB;
+    static constexpr int kStageBytes = kAStage + kBStage + kSfaBytes + kSfbBytes;
+    static constexpr int kStages = (220 * 1024) / kStageBytes > 6 ? 6 : (220 * 1024) / kStageBytes;
     static constexpr uint32_t kSfbCols = 8 * kAtoms;              // B atom (a, h) at 4 (2a + h)
     static constexpr uint32_t kSfColsPerStage = kSfbCols + 4 * kAtoms;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+    static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "tensor-memory scale slots");
+    static_assert(kSmemBytes + 1024 <= 227 * 1024, "shared memory");
+    static_assert(kStages >= 2, "pipeline depth");
 };
-static_assert(kSfCol0 + Pair<KIND_F8F6F4>::kStages * Pair<KIND_F8F6F4>::kSfColsPerStage <= kTmemCols, "tmem");
-static_assert(kSfCol0 + Pair<KIND_MXF4>::kStages * Pair<KIND_MXF4>::kSfColsPerStage <= kTmemCols, "tmem");
-static_assert(kSfCol0 + Pair<KIND_NVF4>::kStages * Pair<KIND_NVF4>::kSfColsPerStage <= kTmemCols, "tmem");
-static_assert(Pair<KIND_MXF4>::kSmemBytes + 1024 <= 227 * 1024, "shared memory");
+// Sub-tiles per stage for each kind (the depth of the ring follows from the stage size).
+template <int KIND> constexpr int kPairSub = 1;
 }  // namespace
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -83,19 +90,19 @@ __device__ __forceinline__ void mbar_arrive_remote(uint64_t *bar, uint32_t rank)
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 
-template <int KIND>
+template <int KIND, int SUB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                     const float *__restrict__ ga, const float *__restrict__ gb, uint16_t *__restrict__ C, int M,
                     int N, int K, uint32_t a_fmt_code, uint32_t b_fmt_code, int band, int *watchdog) {
-    using P = Pair<KIND>;
+    using P = Pair<KIND, SUB>;
     constexpr int S = P::kStages;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem;                                  // S x 16 KiB (1024-aligned)
-    uint8_t *sB = sA + S * kABytes;                      // S x 16 KiB
-    uint8_t *sSFA = sB + S * kBBytes;                    // S x kAtoms x 512 B
+    uint8_t *sA = smem;                                  // S x SUB x 16 KiB (1024-aligned)
+    uint8_t *sB = sA + S * P::kAStage;                   // S x SUB x 16 KiB
+    uint8_t *sSFA = sB + S * P::kBStage;                 // S x kAtoms x 512 B
     uint8_t *sSFB = sSFA + S * P::kSfaBytes;             // S x 2 x kAtoms x 512 B
 
     __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], sf_ready[S], acc_full, acc_empty, drain_bar,
@@ -141,28 +148,32 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     for (int s = 0; s < S; s++) last_it[s] = -1;
     if (warp == kProducerWarp) {
         // ------------------------------------------------ TMA producer (both CTAs)
-        if (lane == 0) {
-            const int col_atoms = num_kb * P::kAtoms;        // scale atoms per 128-row block
-            const uint32_t tx_pair =
-                2u * ((KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kABytes, a_fmt_code) : kABytes) +
-                      (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kBBytes, b_fmt_code) : kBBytes) + P::kSfaBytes +
-                      P::kSfbBytes);
-            int it = 0;
-            for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs) {
-                int m_blk, n_blk;
-                tile_coords(t, tiles_m, tiles_n, band, m_blk, n_blk);
-                const int a_row = m_blk * kPairM + (int)rank * kHalfRows;
-                const int b_row = n_blk * kPairN + (int)rank * kHalfRows;
-                for (int kb = 0; kb < num_kb; kb++, it++) {
-                    const int s = it % S;
-                    if (it >= S &&
-                        !mbar_wait_bounded(&empty_bar[s], (uint32_t)((it / S) - 1) & 1u, watchdog, WD_GEMM_EMPTY)) {
-                        *fail_sh = 1;
-                        break;
-                    }
+        // the whole warp runs the loop; one elected lane issues the copies
+        const int col_atoms = num_kb * P::kAtoms;            // scale atoms per 128-row block
+        const uint32_t tx_pair =
+            2u * (SUB * ((KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kABytes, a_fmt_code) : kABytes) +
+                         (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kBBytes, b_fmt_code) : kBBytes)) +
+                  P::kSfaBytes + P::kSfbBytes);
+        int it = 0;
+        for (int t = pair; t < n_tiles && !warp_failed(fail_sh); t += n_pairs) {
+            int m_blk, n_blk;
+            tile_coords(t, tiles_m, tiles_n, band, m_blk, n_blk);
+            const int a_row = m_blk * kPairM + (int)rank * kHalfRows;
+            const int b_row = n_blk * kPairN + (int)rank * kHalfRows;
+            for (int kb = 0; kb < num_kb; kb++, it++) {
+                const int s = it % S;
+                if (it >= S && !warp_wait(&empty_bar[s], (uint32_t)((it / S) - 1) & 1u, watchdog, WD_GEMM_EMPTY)) {
+                    *fail_sh = 1;
+                    break;
+                }
+                if (elect_one()) {
                     if (leader) mbar_arrive_expect_tx(&full_bar[s], tx_pair);
-                    tma_load_2d_pair(sA + s * kABytes, &tmA, kb * kRowBytes, a_row, &full_bar[s]);
-                    tma_load_2d_pair(sB + s * kBBytes, &tmB, kb * kRowBytes, b_row, &full_bar[s]);
+#pragma unroll
+                    for (int j = 0; j < SUB; j++) {
+                        const int kx = (kb * SUB + j) * kRowBytes;
+                        tma_load_2d_pair(sA + s * P::kAStage + j * kABytes, &tmA, kx, a_row, &full_bar[s]);
+                        tma_load_2d_pair(sB + s * P::kBStage + j * kBBytes, &tmB, kx, b_row, &full_bar[s]);
+                    }
                     // scale atoms as rows of 256 bytes (two per atom); a stage's atoms of one
                     // 128-row block are contiguous
                     tma_load_2d_pair(sSFA + s * P::kSfaBytes, &tmSA, 0,
@@ -171,26 +182,25 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int h = 0; h < 2; h++)
                         tma_load_2d_pair(sSFB + s * P::kSfbBytes + h * P::kSfaBytes, &tmSB, 0,
                                          2 * ((2 * n_blk + h) * col_atoms + kb * P::kAtoms), &full_bar[s]);
-                    last_it[s] = it;
                 }
+                __syncwarp();
+                last_it[s] = it;
             }
         }
-        __syncwarp();
     } else if (warp == kSfWarp) {
         // ------------------------------------------------ scale-atom copier (even CTA only)
         // Copies each stage's scale atoms into tensor memory (both CTAs') as soon as the
         // stage has landed, and signals sf_ready[s] once the copies are complete.  The MMA
         // issuer waits on sf_ready alone (it implies the stage's operands are there), so the
-        // copies leave the single MMA-issuing thread, whose instruction latency otherwise
-        // bounds the tensor pipe.  A stage's scale slot is rewritten only after full[s] of
-        // its next use, i.e. after the MMAs that read it have completed (empty[s]).
-        if (leader && lane == 0) {
+        // copies stay off the MMA-issuing warp.  A stage's scale slot is rewritten only after
+        // full[s] of its next use, i.e. after the MMAs that read it have completed (empty[s]).
+        if (leader) {
             const uint64_t sfa_d0 = sf_desc(smem_u32(sSFA)), sfb_d0 = sf_desc(smem_u32(sSFB));
             int it = 0;
-            for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs) {
+            for (int t = pair; t < n_tiles && !warp_failed(fail_sh); t += n_pairs) {
                 for (int kb = 0; kb < num_kb; kb++, it++) {
                     const int s = it % S;
-                    if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
+                    if (!warp_wait(&full_bar[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
                         *fail_sh = 1;
                         break;
                     }
@@ -199,23 +209,28 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const uint32_t sfa_t = sfb_t + P::kSfbCols;
                     const uint64_t sfa_d = sfa_d0 + (uint64_t)((s * P::kSfaBytes) >> 4);
                     const uint64_t sfb_d = sfb_d0 + (uint64_t)((s * P::kSfbBytes) >> 4);
+                    if (elect_one()) {
 #pragma unroll
-                    for (int a = 0; a < P::kAtoms; a++) {
-                        tc_cp_sf<2>(sfa_t + 4 * a, sfa_d + (uint64_t)(a * 512 / 16));
+                        for (int a = 0; a < P::kAtoms; a++) {
+                            tc_cp_sf<2>(sfa_t + 4 * a, sfa_d + (uint64_t)(a * 512 / 16));
 #pragma unroll
-                        for (int h = 0; h < 2; h++)
-                            tc_cp_sf<2>(sfb_t + 4 * (2 * a + h), sfb_d + (uint64_t)((h * P::kSfaBytes + a * 512) / 16));
+                            for (int h = 0; h < 2; h++)
+                                tc_cp_sf<2>(sfb_t + 4 * (2 * a + h),
+                                            sfb_d + (uint64_t)((h * P::kSfaBytes + a * 512) / 16));
+                        }
+                        tc_commit_pair_local(&sf_ready[s]);  // the stage's scales are in tensor memory
                     }
-                    tc_commit_pair_local(&sf_ready[s]);      // the stage's scales are in tensor memory
+                    __syncwarp();
                 }
             }
-            tc_commit_pair_local(&sf_drain);                 // completes once every copy above has finished
+            if (elect_one()) tc_commit_pair_local(&sf_drain);   // completes once every copy has finished
+            __syncwarp();
         }
-        __syncwarp();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------ MMA issuer (even CTA only)
-        if (leader && lane == 0) {
-            // precomputed descriptors on the issuing thread (as in gemm.cu)
+        if (leader) {
+            // descriptors precomputed and advanced by offsets; the whole warp runs the loop
+            // and one elected lane issues each stage's MMAs and its commit
             const uint64_t a_d0 = smem_desc(smem_u32(sA), 16, 1024, 2), b_d0 = smem_desc(smem_u32(sB), 16, 1024, 2);
             uint32_t idesc[4];
 #pragma unroll
@@ -224,8 +239,8 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     a_fmt_code, b_fmt_code,
                     KIND == KIND_F8F6F4 ? (uint32_t)k : (KIND == KIND_MXF4 ? 2u * (k & 1) : 0u));
             int it = 0, i = 0;
-            for (int t = pair; t < n_tiles && !*fail_sh; t += n_pairs, i++) {
-                if (i > 0 && !mbar_wait_bounded(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
+            for (int t = pair; t < n_tiles && !warp_failed(fail_sh); t += n_pairs, i++) {
+                if (i > 0 && !warp_wait(&acc_empty, (uint32_t)(i - 1) & 1u, watchdog, WD_GEMM_ACC)) {
                     *fail_sh = 1;
                     break;
                 }
@@ -233,29 +248,37 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 for (int kb = 0; kb < num_kb; kb++, it++) {
                     const int s = it % S;
                     // the stage's operands have landed and its scales are in tensor memory
-                    if (!mbar_wait_bounded(&sf_ready[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
+                    if (!warp_wait(&sf_ready[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
                         *fail_sh = 1;
                         break;
                     }
                     tc_fence_after();
                     const uint32_t sfb_t = tmem + kSfCol0 + s * P::kSfColsPerStage;
                     const uint32_t sfa_t = sfb_t + P::kSfbCols;
-                    const uint64_t a_d = a_d0 + (uint64_t)((s * kABytes) >> 4);
-                    const uint64_t b_d = b_d0 + (uint64_t)((s * kBBytes) >> 4);
+                    if (elect_one()) {
 #pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        const int a = KIND == KIND_F8F6F4 ? 0 : (KIND == KIND_MXF4 ? k >> 1 : k);
-                        tc_mma_mx<KIND, 2>(tmem, a_d + (uint64_t)(2 * k), b_d + (uint64_t)(2 * k), idesc[k], sfa_t + 4 * a,
-                                           sfb_t + 8 * a, (kb > 0 || k > 0) ? 1u : 0u);
+                        for (int j = 0; j < SUB; j++) {
+                            const uint64_t a_d = a_d0 + (uint64_t)((s * P::kAStage + j * kABytes) >> 4);
+                            const uint64_t b_d = b_d0 + (uint64_t)((s * P::kBStage + j * kBBytes) >> 4);
+#pragma unroll
+                            for (int k = 0; k < 4; k++) {
+                                const int a = j * P::kSubAtoms +
+                                              (KIND == KIND_F8F6F4 ? 0 : (KIND == KIND_MXF4 ? k >> 1 : k));
+                                tc_mma_mx<KIND, 2>(tmem, a_d + (uint64_t)(2 * k), b_d + (uint64_t)(2 * k), idesc[k],
+                                                   sfa_t + 4 * a, sfb_t + 8 * a, (kb > 0 || j > 0 || k > 0) ? 1u : 0u);
+                            }
+                        }
+                        tc_commit_pair(&empty_bar[s]);       // stage s free in both CTAs
                     }
-                    tc_commit_pair(&empty_bar[s]);           // stage s free in both CTAs
+                    __syncwarp();
                 }
-                if (*fail_sh) break;
-                tc_commit_pair(&acc_full);                   // both halves of the tile are complete
+                if (warp_failed(fail_sh)) break;
+                if (elect_one()) tc_commit_pair(&acc_full);  // both halves of the tile are complete
+                __syncwarp();
             }
-            tc_commit_pair(&drain_bar);                      // completes once every MMA above has finished
+            if (elect_one()) tc_commit_pair(&drain_bar);     // completes once every MMA above has finished
+            __syncwarp();
         }
-        __syncwarp();
     } else {
         // ------------------------------------------------ epilogue (warps 0-7, both CTAs)
         constexpr int kHalf = kPairN / 2;
@@ -297,11 +320,14 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     // handshake, so that neither CTA releases tensor memory or exits while the pair's
     // copies or MMAs may still use the other's memory
     __syncthreads();
+    // error path: the even CTA's producer (whose record of the armed stages this is) waits
+    // for the pair's copies that were counted on its barriers
+    if (warp == kProducerWarp && lane == 0 && leader && *fail_sh)
+        for (int s = 0; s < S; s++)
+            if (last_it[s] >= 0)
+                (void)mbar_wait_bounded(&full_bar[s], (uint32_t)(last_it[s] / S) & 1u, nullptr, 0, kDrainLimitNs);
+    __syncthreads();
     if (warp == kMmaWarp && lane == 0) {
-        if (leader && *fail_sh)
-            for (int s = 0; s < S; s++)
-                if (last_it[s] >= 0)
-                    (void)mbar_wait_bounded(&full_bar[s], (uint32_t)(last_it[s] / S) & 1u, nullptr, 0, kDrainLimitNs);
         (void)mbar_wait_bounded(&drain_bar, 0u, nullptr, 0, kDrainLimitNs);
         if (leader) (void)mbar_wait_bounded(&sf_drain, 0u, nullptr, 0, kDrainLimitNs);   // scale copies too
         // the odd CTA's copies complete on the even CTA's barriers, so it stays until the
@@ -353,12 +379,12 @@ static bool encode_scales(EncodeTiledFn enc, CUtensorMap *tm, const uint8_t *ptr
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KIND>
-static cudaError_t launch_pair_k(EncodeTiledFn enc, const void *a, const uint8_t *a_sc, const float *ga, int a_fmt,
+template <int KIND, int SUB>
+static cudaError_t launch_pair_s(EncodeTiledFn enc, const void *a, const uint8_t *a_sc, const float *ga, int a_fmt,
                                  const void *b, const uint8_t *b_sc, const float *gb, int b_fmt, uint32_t a_code,
                                  uint32_t b_code, void *c, int64_t M, int64_t N, int64_t K, int *watchdog,
                                  int num_sms, cudaStream_t st) {
-    using P = Pair<KIND>;
+    using P = Pair<KIND, SUB>;
     CUtensorMap tmA, tmB, tmSA, tmSB;
     const int64_t col_atoms = (K / P::kStageK) * P::kAtoms;
     const bool a_expand = KIND == KIND_F8F6F4 && code_bits(a_fmt) < 8;
@@ -376,13 +402,27 @@ static cudaError_t launch_pair_k(EncodeTiledFn enc, const void *a, const uint8_t
     int64_t pairs = num_sms / 2;
     if (pairs > n_tiles) pairs = n_tiles;
     if (pairs < 1) pairs = 1;
-    auto k = mx_gemm_pair_kernel<KIND>;
+    auto k = mx_gemm_pair_kernel<KIND, SUB>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P::kSmemBytes);
     if (e != cudaSuccess) return e;
     k<<<(unsigned)(2 * pairs), kPairThreads, P::kSmemBytes, st>>>(tmA, tmB, tmSA, tmSB, ga, gb,
                                                                    static_cast<uint16_t *>(c), (int)M, (int)N,
                                                                    (int)K, a_code, b_code, (int)band, watchdog);
     return cudaGetLastError();
+}
+
+// The kind's sub-tiles per stage when K is a multiple of the stage's K, else one.
+template <int KIND>
+static cudaError_t launch_pair_k(EncodeTiledFn enc, const void *a, const uint8_t *a_sc, const float *ga, int a_fmt,
+                                 const void *b, const uint8_t *b_sc, const float *gb, int b_fmt, uint32_t a_code,
+                                 uint32_t b_code, void *c, int64_t M, int64_t N, int64_t K, int *watchdog,
+                                 int num_sms, cudaStream_t st) {
+    constexpr int SUB = kPairSub<KIND>;
+    if (SUB > 1 && K % Pair<KIND, SUB>::kStageK == 0)
+        return launch_pair_s<KIND, SUB>(enc, a, a_sc, ga, a_fmt, b, b_sc, gb, b_fmt, a_code, b_code, c, M, N, K,
+                                        watchdog, num_sms, st);
+    return launch_pair_s<KIND, 1>(enc, a, a_sc, ga, a_fmt, b, b_sc, gb, b_fmt, a_code, b_code, c, M, N, K, watchdog,
+                                  num_sms, st);
 }
 
 bool gemm_pair_supported(int64_t M, int64_t N) { return M % kPairM == 0 && N % kPairN == 0; }
