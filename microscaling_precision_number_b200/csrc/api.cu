@@ -3,10 +3,12 @@
 // rejected call never touches the device.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cstdlib>
 #include <mutex>
 #include <utility>
 
 #include "../../include/mx.h"
+#include "checked.cuh"
 #include "internal.h"
 
 namespace {
@@ -70,6 +72,27 @@ cudaError_t device_info(int *num_sms, int **watchdog) {
     *watchdog = d->watchdog;
     return cudaSuccess;
 }
+
+#ifdef MX_CHECKED
+cudaError_t set_out_ranges_impl(const OutRange *r, int n, int *flag, cudaStream_t st, CheckState *sym) {
+    CheckState h = {};
+    h.flag = flag;
+    for (int i = 0; i < n; i++) {
+        if (!r[i].base) continue;
+        const uint64_t lo = reinterpret_cast<uint64_t>(r[i].base);
+        h.lo[h.n] = lo;
+        h.hi[h.n] = lo + r[i].bytes;
+        h.n++;
+    }
+    // test hook: shorten the last registered range (stores beyond it are then refused)
+    if (const char *shrink = std::getenv("MX_CHECKED_SHRINK")) {
+        const uint64_t k = std::strtoull(shrink, nullptr, 10);
+        if (h.n > 0 && h.hi[h.n - 1] - h.lo[h.n - 1] > k) h.hi[h.n - 1] -= k;
+    }
+    // pageable source: staged by the runtime before the call returns, so `h` may go
+    return cudaMemcpyAsync(sym, &h, sizeof h, cudaMemcpyHostToDevice, st);
+}
+#endif
 
 void *tensor_map_encoder() {
     static void *fn = nullptr;
@@ -369,10 +392,9 @@ mx_status mx_gemm(mx_operand A, mx_operand B, void *C, int64_t M, int64_t N, int
         e = cudaMemsetAsync(C, 0, (size_t)(M * N * 2), s);   // empty sum
         return e == cudaSuccess ? MX_OK : cuda_fail(e);
     }
-    // 256 x 256 tiles on CTA pairs when the shape allows (measured 1-3% faster for the
-    // 8-bit and MXFP4 kinds), else 128 x {256, 128} tiles; NVFP4 x NVFP4 stays on single
-    // CTAs, whose 4-stage ring measured 6% faster than the pair's 5 stages there
-    if (mxk::gemm_pair_supported(M, N) && !nvf4)
+    // 256 x 256 tiles on CTA pairs when the shape allows (8192^3: 1-3% faster than single
+    // CTAs for the 8-bit and MXFP4 kinds, 13% for NVFP4 x NVFP4), else 128 x {256, 128} tiles
+    if (mxk::gemm_pair_supported(M, N))
         e = mxk::launch_gemm_pair(A.elems, A.scales, A.fmt, A.global_scale, B.elems, B.scales, B.fmt, B.global_scale,
                                   C, M, N, K, d->watchdog, d->num_sms, s);
     else

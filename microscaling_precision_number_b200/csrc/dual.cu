@@ -27,6 +27,7 @@
 // Every barrier wait is bounded (watchdog); the producer drains its own loads before the
 // CTA exits, whatever happened.
 #include <cuda.h>
+#include "checked.cuh"
 #include "codec.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -50,6 +51,7 @@ constexpr size_t kDualSmem = (size_t)kStages * kTileBytes + 1024;   // + alignme
 // 32 bytes at p (w, or zeros when `zero`): one 256-bit store when p is 32-byte aligned,
 // else two 16-byte stores.  The rare zero case is a separate store, not a per-word select.
 __device__ __forceinline__ void store32(uint8_t *p, const uint32_t (&w)[8], bool v8, bool zero) {
+    if (!out_ok(p, 32)) return;
     if (__builtin_expect(zero, 0)) {
         reinterpret_cast<uint4 *>(p)[0] = make_uint4(0u, 0u, 0u, 0u);
         reinterpret_cast<uint4 *>(p)[1] = make_uint4(0u, 0u, 0u, 0u);
@@ -73,7 +75,7 @@ __device__ __forceinline__ void store_codes(uint8_t *base, uint64_t e, const uin
         fp6_pack<8>(w, o);
         uint2 *p = reinterpret_cast<uint2 *>(base + e * 3 / 4);
 #pragma unroll
-        for (int i = 0; i < 3; i++) p[i] = zero ? make_uint2(0u, 0u) : make_uint2(o[2 * i], o[2 * i + 1]);
+        for (int i = 0; i < 3; i++) out_store(p + i, zero ? make_uint2(0u, 0u) : make_uint2(o[2 * i], o[2 * i + 1]));
     } else {
         store32(base + e, w, v8, zero);
     }
@@ -117,8 +119,8 @@ struct ScaleOut {
 };
 template <bool RM, bool TC>
 __device__ __forceinline__ void put_scale(const ScaleOut &o, uint32_t r, uint32_t c, uint32_t code) {
-    if constexpr (RM) o.rm[(uint64_t)r * o.S + c] = (uint8_t)code;
-    if constexpr (TC) o.tc[tc_offset(r, c, o.atoms)] = (uint8_t)code;
+    if constexpr (RM) out_store(o.rm + (uint64_t)r * o.S + c, (uint8_t)code);
+    if constexpr (TC) out_store(o.tc + tc_offset(r, c, o.atoms), (uint8_t)code);
 }
 
 // Column pass: columns col, col + 1 (box-relative pair q) over the tile's 32 rows.
@@ -160,9 +162,9 @@ __device__ __forceinline__ void column_pair(const uint8_t *box, uint32_t q, uint
         }
         // a NaN scale makes the whole block NaN: its codes are stored as 0
         uint4 *p = reinterpret_cast<uint4 *>(col_elems + (e0 >> 1));
-        p[0] = code_lo == 0xFFu ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(o_lo[0], o_lo[1], o_lo[2], o_lo[3]);
-        p[rows >> 5] = code_hi == 0xFFu ? make_uint4(0u, 0u, 0u, 0u)     // next column: rows / 2 bytes on
-                                        : make_uint4(o_hi[0], o_hi[1], o_hi[2], o_hi[3]);
+        out_store(p, code_lo == 0xFFu ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(o_lo[0], o_lo[1], o_lo[2], o_lo[3]));
+        out_store(p + (rows >> 5), code_hi == 0xFFu ? make_uint4(0u, 0u, 0u, 0u)     // next column: rows / 2 bytes on
+                                                    : make_uint4(o_hi[0], o_hi[1], o_hi[2], o_hi[3]));
     } else {
         uint32_t o_lo[8], o_hi[8];
 #pragma unroll
@@ -212,8 +214,8 @@ __device__ __forceinline__ void row_block(const uint8_t *box, uint32_t r, uint32
             scale8(v[k], s2, x);
             o[k] = cvt_e2m1x8(x);
         }
-        *reinterpret_cast<uint4 *>(row_elems + (e0 >> 1)) =
-            code == 0xFFu ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(o[0], o[1], o[2], o[3]);   // NaN scale: codes 0
+        out_store(reinterpret_cast<uint4 *>(row_elems + (e0 >> 1)),
+                  code == 0xFFu ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(o[0], o[1], o[2], o[3]));   // NaN scale: codes 0
     } else {
         uint32_t o[8];
 #pragma unroll
@@ -395,6 +397,13 @@ cudaError_t launch_quant_dual(const void *src, int64_t rows, int64_t cols, int f
     const uint32_t row_S = (uint32_t)(cols / 32), col_S = (uint32_t)(rows / 32);
     const ScaleOut rs{row_rm, row_tc, row_S, (row_S + 3) / 4};
     const ScaleOut cs{col_rm, col_tc, col_S, (col_S + 3) / 4};
+    const uint64_t code_bytes = (uint64_t)(rows * cols * code_bits(fmt) / 8);
+    const uint64_t row_tc_bytes = (uint64_t)((rows + 127) / 128) * ((row_S + 3) / 4) * 512;
+    const uint64_t col_tc_bytes = (uint64_t)((cols + 127) / 128) * ((col_S + 3) / 4) * 512;
+    const OutRange out[6] = {{row_elems, code_bytes}, {row_rm, (uint64_t)rows * row_S}, {row_tc, row_tc_bytes},
+                             {col_elems, code_bytes}, {col_rm, (uint64_t)cols * col_S}, {col_tc, col_tc_bytes}};
+    const cudaError_t re_err = set_out_ranges(out, st);
+    if (re_err != cudaSuccess) return re_err;
     uint8_t *re = static_cast<uint8_t *>(row_elems), *ce = static_cast<uint8_t *>(col_elems);
     const int v8 = ((reinterpret_cast<uintptr_t>(re) | reinterpret_cast<uintptr_t>(ce)) & 31u) == 0;
     const uint32_t R = (uint32_t)rows, C = (uint32_t)cols;

@@ -35,6 +35,7 @@
 //           store their row segments with 16-byte global stores.
 // All waits are bounded by the watchdog; tensor memory is always released.
 #include <cuda.h>
+#include "checked.cuh"
 #include "codec.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -287,7 +288,7 @@ mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                     for (int e = 0; e < 4; e++)
                         o[e] = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(r[j][8 * q + 2 * e]), alpha),
                                                __fmul_rn(__uint_as_float(r[j][8 * q + 2 * e + 1]), alpha));
-                    __stcs(dst + 4 * j + q, make_uint4(o[0], o[1], o[2], o[3]));
+                    if (out_ok(dst + 4 * j + q, 16)) __stcs(dst + 4 * j + q, make_uint4(o[0], o[1], o[2], o[3]));
                 }
         }
     }
@@ -343,7 +344,10 @@ static cudaError_t launch_gemm_k(const CUtensorMap &tmA, const CUtensorMap &tmB,
                                  int64_t N, int64_t K, uint32_t a_code, uint32_t b_code, int64_t band, int *watchdog,
                                  int grid, cudaStream_t st) {
     auto k = mx_gemm_kernel<BN, KIND>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<BN, KIND>::kSmemBytes);
+    const OutRange rng[1] = {{c, (uint64_t)(M * N * 2)}};
+    cudaError_t e = set_out_ranges(rng, st);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<BN, KIND>::kSmemBytes);
     if (e != cudaSuccess) return e;
     k<<<grid, kGemmThreads, Tile<BN, KIND>::kSmemBytes, st>>>(tmA, tmB, a_sc, b_sc, ga, gb, static_cast<uint16_t *>(c),
                                                              (int)M, (int)N, (int)K, a_code, b_code, (int)band, watchdog);

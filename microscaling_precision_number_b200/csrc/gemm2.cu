@@ -23,6 +23,7 @@
 // Every wait is bounded (watchdog); the pair leaves through a bounded handshake after the
 // even CTA has drained its barriers and MMAs, so no copy or MMA touches a CTA that exited.
 #include <cuda.h>
+#include "checked.cuh"
 #include "codec.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -310,7 +311,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     for (int e = 0; e < 4; e++)
                         o[e] = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(r[j][8 * q + 2 * e]), alpha),
                                                __fmul_rn(__uint_as_float(r[j][8 * q + 2 * e + 1]), alpha));
-                    __stcs(dst + 4 * j + q, make_uint4(o[0], o[1], o[2], o[3]));
+                    if (out_ok(dst + 4 * j + q, 16)) __stcs(dst + 4 * j + q, make_uint4(o[0], o[1], o[2], o[3]));
                 }
         }
     }
@@ -403,7 +404,10 @@ static cudaError_t launch_pair_s(EncodeTiledFn enc, const void *a, const uint8_t
     if (pairs > n_tiles) pairs = n_tiles;
     if (pairs < 1) pairs = 1;
     auto k = mx_gemm_pair_kernel<KIND, SUB>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P::kSmemBytes);
+    const OutRange rng[1] = {{c, (uint64_t)(M * N * 2)}};
+    cudaError_t e = set_out_ranges(rng, st);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, P::kSmemBytes);
     if (e != cudaSuccess) return e;
     k<<<(unsigned)(2 * pairs), kPairThreads, P::kSmemBytes, st>>>(tmA, tmB, tmSA, tmSB, ga, gb,
                                                                    static_cast<uint16_t *>(c), (int)M, (int)N,

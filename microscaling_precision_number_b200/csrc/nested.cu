@@ -23,6 +23,7 @@
 // 5), at -11 everything but 4 (code 6), and below -11 every nonzero code.  Those sets are
 // tested on the packed codes with bit operations (b0, b1, b2: the magnitude bits of every
 // nibble).
+#include "checked.cuh"
 #include "codec.cuh"
 #include "internal.h"
 
@@ -109,12 +110,13 @@ mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__r
     }
     uint4 *dst = reinterpret_cast<uint4 *>(out + R * cols + c0);
 #pragma unroll
-    for (int i = 0; i < 4; i++) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    for (int i = 0; i < 4; i++) out_store(dst + i, make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
     const int all_exact = __syncthreads_and(exact ? 1 : 0);
     if (tid == 0) {
         const int e = smax - 6;                                   // S = 2^e, e in [-133, 121]
-        block_scale[blk] = e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149));
-        block_exact[blk] = (uint8_t)all_exact;
+        out_store(block_scale + blk,
+                  e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(1u << (e + 149)));
+        out_store(block_exact + blk, (uint8_t)all_exact);
     }
 }
 
@@ -123,6 +125,10 @@ cudaError_t launch_mxfp4_to_fp8_blocks(const void *elems, const uint8_t *scales,
     const int64_t n_blocks = (rows / 128) * (cols / 128);
     if (n_blocks <= 0) return cudaSuccess;
     if (n_blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+    const OutRange rng[3] = {{out, (uint64_t)(rows * cols)}, {block_scale, (uint64_t)n_blocks * 4},
+                             {block_exact, (uint64_t)n_blocks}};
+    const cudaError_t e = set_out_ranges(rng, st);
+    if (e != cudaSuccess) return e;
     mxfp4_to_fp8_blocks_kernel<<<(unsigned)n_blocks, kNestThreads, 0, st>>>(
         static_cast<const uint8_t *>(elems), scales, cols, (uint32_t)(cols / 128), static_cast<uint8_t *>(out),
         block_scale, block_exact);

@@ -75,6 +75,25 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t phase,
     }
 }
 
+// ---- warp-uniform issue ---------------------------------------------------------------------
+// The issuing warps of the matmuls (and the dual quantiser's producer) run their loops with all 32 lanes converged and let one
+// elected lane issue each group of tcgen05 / TMA instructions.  Measured on B200: a
+// tcgen05.mma stream issued this way sustains one M = 256 x N = 256 x K = 32 pair MMA per
+// 128 cycles (the tensor pipe's rate), whereas the same loop run by lane 0 alone inside a
+// divergent branch issued one per ~560 cycles.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
+    return pred != 0;
+}
+// Bounded wait by a whole warp; true only if every lane saw the phase complete.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t phase, int *watchdog, int code) {
+    const bool ok = mbar_wait_bounded(bar, phase, watchdog, code);
+    return __all_sync(0xffffffffu, ok);
+}
+// A shared failure flag read uniformly by a warp.
+__device__ __forceinline__ bool warp_failed(volatile int *flag) { return __any_sync(0xffffffffu, *flag != 0); }
+
 // Short limit for error-path drains of a CTA's own in-flight copies.
 constexpr uint64_t kDrainLimitNs = 20000000ull;   // 20 ms
 

@@ -10,6 +10,7 @@
 // A "chunk" is 16 bytes of bf16 input (8 elements); each thread converts whole chunks
 // with the hardware cvt.rn.satfinite conversions and writes 8 (FP8), 6 (FP6, packed) or
 // 4 (FP4) bytes.
+#include "checked.cuh"
 #include "codec.cuh"
 #include "internal.h"
 #include "ptx.cuh"
@@ -41,7 +42,7 @@ __global__ void tcgen05_pad_kernel(uint8_t *__restrict__ sc, int64_t rows, int64
         const int64_t rb = atom / col_atoms, cb = atom - rb * col_atoms;
         const int64_t r = rb * 128 + (w >> 4) + ((w >> 2) & 3) * 32;
         const int64_t c = cb * 4 + (w & 3);
-        if (r >= rows || c >= S) sc[off] = 0;
+        if (r >= rows || c >= S) out_store(sc + off, (uint8_t)0);
     }
 }
 
@@ -50,6 +51,9 @@ cudaError_t launch_tcgen05_pad(uint8_t *sc, int64_t rows, int64_t S, cudaStream_
     const int64_t total = ((rows + 127) / 128) * ((S + 3) / 4) * 512;
     int64_t grid = (total + 255) / 256;
     if (grid > 4096) grid = 4096;
+    const OutRange rng[1] = {{sc, (uint64_t)total}};
+    const cudaError_t e = set_out_ranges(rng, st);
+    if (e != cudaSuccess) return e;
     tcgen05_pad_kernel<<<(int)grid, 256, 0, st>>>(sc, rows, S, total);
     return cudaGetLastError();
 }
@@ -78,7 +82,15 @@ cudaError_t launch_watchdog_selftest(uint64_t limit_ns, int *watchdog, cudaStrea
 // mapped explicitly (0x7F|s for FP8; the signed maximum for E2M1 and FP6, which have no
 // NaN: 0x7|s, 0x1F|s).
 // ---------------------------------------------------------------------------------------
-template <int FMT>
+// st(p, v): the store of the codes -- bounds-checked for the output buffer (GLOBAL), plain
+// for the tail's local staging buffer.
+template <bool GLOBAL, typename T>
+__device__ __forceinline__ void st(T *p, T v) {
+    if constexpr (GLOBAL) out_store(p, v);
+    else *p = v;
+}
+
+template <int FMT, bool GLOBAL = true>
 __device__ __forceinline__ void cast8(const uint4 &v, uint8_t *out, int64_t c) {
     const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
                         bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
@@ -87,7 +99,7 @@ __device__ __forceinline__ void cast8(const uint4 &v, uint8_t *out, int64_t c) {
 #pragma unroll
         for (int i = 0; i < 8; i++)
             if (x[i] != x[i]) q = (q & ~(0xFu << (4 * i))) | ((0x7u | (__float_as_uint(x[i]) >> 31 << 3)) << (4 * i));
-        reinterpret_cast<uint32_t *>(out)[c] = q;
+        st<GLOBAL>(reinterpret_cast<uint32_t *>(out) + c, q);
     } else {
         uint2 q = cvt_fp8x8<FMT>(x);
         uint32_t w[2] = {q.x, q.y};
@@ -106,14 +118,14 @@ __device__ __forceinline__ void cast8(const uint4 &v, uint8_t *out, int64_t c) {
             const uint32_t lo = p0 | (p1 << 24), hi = p1 >> 8;      // 48 bits
             uint8_t *d = out + c * 6;
             if ((c & 1) == 0) {
-                *reinterpret_cast<uint32_t *>(d) = lo;
-                *reinterpret_cast<uint16_t *>(d + 4) = (uint16_t)hi;
+                st<GLOBAL>(reinterpret_cast<uint32_t *>(d), lo);
+                st<GLOBAL>(reinterpret_cast<uint16_t *>(d + 4), (uint16_t)hi);
             } else {
-                *reinterpret_cast<uint16_t *>(d) = (uint16_t)lo;
-                *reinterpret_cast<uint32_t *>(d + 2) = (lo >> 16) | (hi << 16);
+                st<GLOBAL>(reinterpret_cast<uint16_t *>(d), (uint16_t)lo);
+                st<GLOBAL>(reinterpret_cast<uint32_t *>(d + 2), (lo >> 16) | (hi << 16));
             }
         } else {
-            reinterpret_cast<uint2 *>(out)[c] = make_uint2(w[0], w[1]);
+            st<GLOBAL>(reinterpret_cast<uint2 *>(out) + c, make_uint2(w[0], w[1]));
         }
     }
 }
@@ -133,10 +145,10 @@ cast_kernel(const uint4 *__restrict__ src, int64_t n_chunks, const uint16_t *__r
         v.x = t16[0] | ((uint32_t)t16[1] << 16); v.y = t16[2] | ((uint32_t)t16[3] << 16);
         v.z = t16[4] | ((uint32_t)t16[5] << 16); v.w = t16[6] | ((uint32_t)t16[7] << 16);
         alignas(8) uint8_t tmp[8];
-        cast8<FMT>(v, tmp, 0);
+        cast8<FMT, false>(v, tmp, 0);
         const int nbytes = tail * code_bits(FMT) / 8;                 // FP6: tail is 4
         uint8_t *dst = out + n_chunks * code_bits(FMT);
-        for (int i = 0; i < nbytes; i++) dst[i] = tmp[i];
+        for (int i = 0; i < nbytes; i++) out_store(dst + i, tmp[i]);
     }
 }
 
@@ -147,6 +159,9 @@ cudaError_t launch_cast(const void *src, int64_t n, int fmt, void *out, int num_
     const uint4 *s = static_cast<const uint4 *>(src);
     const uint16_t *ts = static_cast<const uint16_t *>(src) + n_chunks * 8;
     uint8_t *o = static_cast<uint8_t *>(out);
+    const OutRange rng[1] = {{out, (uint64_t)(n * code_bits(fmt) / 8)}};
+    const cudaError_t e = set_out_ranges(rng, st);
+    if (e != cudaSuccess) return e;
     switch (fmt) {
     case FMT_E4M3: cast_kernel<FMT_E4M3><<<grid, kThreads, 0, st>>>(s, n_chunks, ts, tail, o); break;
     case FMT_E5M2: cast_kernel<FMT_E5M2><<<grid, kThreads, 0, st>>>(s, n_chunks, ts, tail, o); break;

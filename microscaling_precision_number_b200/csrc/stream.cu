@@ -28,6 +28,7 @@
 #include <set>
 #include <utility>
 
+#include "checked.cuh"
 #include "codec.cuh"
 #include "internal.h"
 #include "nvfp4.cuh"
@@ -154,7 +155,7 @@ __device__ __forceinline__ void store_partial(uint32_t acc, float *dst, uint32_t
     if (tid == 0) {
         uint32_t r = 0;
         for (int w = 0; w < kThreads / 32; w++) r = max(r, warp_u[w]);
-        *dst = __uint_as_float(r << 16);
+        out_store(dst, __uint_as_float(r << 16));
     }
 }
 
@@ -223,7 +224,7 @@ mx_rows_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS,
             fp6_pack<8>(w, o);
             uint2 *dst = reinterpret_cast<uint2 *>(elems + (size_t)blk * 24);
 #pragma unroll
-            for (int i = 0; i < 3; i++) dst[i] = nan_blk ? make_uint2(0u, 0u) : make_uint2(o[2 * i], o[2 * i + 1]);
+            for (int i = 0; i < 3; i++) out_store(dst + i, nan_blk ? make_uint2(0u, 0u) : make_uint2(o[2 * i], o[2 * i + 1]));
         } else {
 #pragma unroll
             for (int j = 0; j < 4; j++) {
@@ -232,18 +233,18 @@ mx_rows_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS,
                 scale8(v[j], mul2x, x);
                 if constexpr (FMT == FMT_E2M1) {
                     const uint32_t q = nan_blk ? 0u : cvt_e2m1x8(x);
-                    reinterpret_cast<uint32_t *>(elems)[(size_t)blk * 4 + c] = q;
+                    out_store(reinterpret_cast<uint32_t *>(elems) + (size_t)blk * 4 + c, q);
                 } else {
                     uint2 q = cvt_fp8x8<FMT>(x);
                     if (nan_blk) q = make_uint2(0u, 0u);
-                    reinterpret_cast<uint2 *>(elems)[(size_t)blk * 4 + c] = q;
+                    out_store(reinterpret_cast<uint2 *>(elems) + (size_t)blk * 4 + c, q);
                 }
             }
         }
-        if constexpr (RM) sc_rm[blk] = (uint8_t)code;
+        if constexpr (RM) out_store(sc_rm + blk, (uint8_t)code);
         if constexpr (TC) {
             const uint32_t r = fdiv(blk, divS);
-            sc_tc[tc_offset(r, blk - r * divS.d, col_atoms)] = (uint8_t)code;
+            out_store(sc_tc + tc_offset(r, blk - r * divS.d, col_atoms), (uint8_t)code);
         }
     });
     if (partials) store_partial(finite_acc, partials + blockIdx.x, warp_u);
@@ -343,13 +344,14 @@ __device__ __forceinline__ void nvfp4_quant_tile(const uint8_t *tile, uint32_t t
 #pragma unroll
     for (int h = 0; h < 2; h++) {
         if (!ok[h]) continue;
-#pragma unroll
-        for (int j = 0; j < 2; j++)
-            reinterpret_cast<uint32_t *>(elems)[(size_t)blk[h] * 2 + ((j + rot) & 1u)] = q[h][j];
-        if constexpr (RM) sc_rm[blk[h]] = (uint8_t)sb[h];
+        // the block's 8 code bytes in element order as one 8-byte store (a warp writes 256
+        // contiguous bytes per instruction)
+        out_store(reinterpret_cast<uint2 *>(elems) + blk[h],
+                  rot ? make_uint2(q[h][1], q[h][0]) : make_uint2(q[h][0], q[h][1]));
+        if constexpr (RM) out_store(sc_rm + blk[h], (uint8_t)sb[h]);
         if constexpr (TC) {
             const uint32_t rr = fdiv(blk[h], divS);
-            sc_tc[tc_offset(rr, blk[h] - rr * divS.d, col_atoms)] = (uint8_t)sb[h];
+            out_store(sc_tc + tc_offset(rr, blk[h] - rr * divS.d, col_atoms), (uint8_t)sb[h]);
         }
     }
 }
@@ -433,7 +435,7 @@ nvfp4_quant_bulk_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fast
     auto after_issue = [&]() {
         pdl_wait_and_release();
         const float g = nvfp4_global_scale(partials, n_partials, warp_max);
-        if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+        if (blockIdx.x == 0 && threadIdx.x == 0) out_store(g_out, g);
         cst = nvfp4_consts(g, qtab);
     };
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
@@ -462,7 +464,7 @@ nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t r
     __shared__ float2 qtab[128];
     pdl_wait_and_release();
     const float g = nvfp4_global_scale(partials, n_partials, warp_max);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    if (blockIdx.x == 0 && threadIdx.x == 0) out_store(g_out, g);
     const Nvfp4Consts cst = nvfp4_consts(g, qtab);
     const uint32_t lane = threadIdx.x & 31, par = lane >> 4, c = lane & 15;
     const uint32_t S = cols / 16;                                  // blocks (scale columns) per row
@@ -498,9 +500,9 @@ nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t r
             nvfp4_codes16(v[k][0], v[k][1], dq.x, dq.y, q[0], q[1]);
             if (zero_codes) q[0] = q[1] = 0u;
             const uint32_t row = rb * 16 + 2 * k + par;
-            reinterpret_cast<uint2 *>(elems)[((size_t)row * cols + (size_t)cb * 16) >> 4] = make_uint2(q[0], q[1]);
-            if constexpr (RM) sc_rm[(size_t)row * S + cb] = (uint8_t)sb;
-            if constexpr (TC) sc_tc[tc_offset(row, cb, col_atoms)] = (uint8_t)sb;
+            out_store(reinterpret_cast<uint2 *>(elems) + (((size_t)row * cols + (size_t)cb * 16) >> 4), make_uint2(q[0], q[1]));
+            if constexpr (RM) out_store(sc_rm + (size_t)row * S + cb, (uint8_t)sb);
+            if constexpr (TC) out_store(sc_tc + tc_offset(row, cb, col_atoms), (uint8_t)sb);
         }
     }
 }
@@ -550,7 +552,7 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
                 o.y = f32x2_to_bf16x2(__fmul_rn(y[2], mul), __fmul_rn(y[3], mul));
                 o.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
                 o.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
-                dst[j] = o;
+                out_store(dst + j, o);
             }
         } else if constexpr (is_fp6(FMT)) {
             // 24 bytes = 32 packed codes, as three 8-byte reads (stride 24 B: conflict-free)
@@ -572,7 +574,7 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
                 q.y = f32x2_to_bf16x2(__fmul_rn(y[2], mul), __fmul_rn(y[3], mul));
                 q.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
                 q.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
-                dst[j] = q;
+                out_store(dst + j, q);
             }
         } else {
             const uint32_t rot = (tid >> 2) & 1u;
@@ -593,7 +595,7 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
                     o.y = f32x2_to_bf16x2(__fmul_rn(y[2], mul), __fmul_rn(y[3], mul));
                     o.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
                     o.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
-                    dst[hc * 2 + j] = o;
+                    out_store(dst + hc * 2 + j, o);
                 }
             }
         }
@@ -648,7 +650,7 @@ dequant_nvfp4_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__re
                 o.y = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[2], sbv), g), __fmul_rn(__fmul_rn(y[3], sbv), g));
                 o.z = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[4], sbv), g), __fmul_rn(__fmul_rn(y[5], sbv), g));
                 o.w = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[6], sbv), g), __fmul_rn(__fmul_rn(y[7], sbv), g));
-                out[(size_t)blk * 2 + j] = o;
+                out_store(out + (size_t)blk * 2 + j, o);
             }
         }
     });
@@ -711,6 +713,9 @@ static cudaError_t launch_pdl_smem(void (*kernel)(KArgs...), int grid, size_t sm
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Bytes of a tcgen05-tiled scale array of rows x S scales (512-byte atoms of 128 x 4).
+static uint64_t tc_bytes(int64_t rows, int64_t S) { return (uint64_t)((rows + 127) / 128) * ((S + 3) / 4) * 512; }
+
 bool stream_supported(int64_t rows, int64_t cols) {
     return rows * cols / 16 < ((int64_t)1 << 31);   // block indices fit 31 bits
 }
@@ -744,6 +749,10 @@ cudaError_t launch_stream_rows_mx(const void *src, int64_t rows, int64_t cols, i
     const FastDiv f = make_fastdiv(S);
     const uint32_t ca = (S + 3) / 4;
     const int g = stream_rows_grid(rows, cols, num_sms);
+    const OutRange out[4] = {{elems, (uint64_t)(rows * cols * code_bits(fmt) / 8)}, {rm, (uint64_t)(rows * cols / 32)},
+                             {tc, tc_bytes(rows, S)}, {partials, (uint64_t)g * 4}};
+    cudaError_t e = set_out_ranges(out, st);
+    if (e != cudaSuccess) return e;
     switch (fmt * 2 + (ceil ? 1 : 0)) {
     case FMT_E4M3 * 2 + 0: return launch_rows_layout<FMT_E4M3, false>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
     case FMT_E4M3 * 2 + 1: return launch_rows_layout<FMT_E4M3, true>(src, n_blocks, f, ca, elems, rm, tc, partials, g, wd, st);
@@ -803,6 +812,10 @@ static cudaError_t launch_nvfp4_2d_t(const uint8_t *src, int64_t rows, int64_t c
 cudaError_t launch_stream_nvfp4_2d(const void *src, int64_t rows, int64_t cols, float *partials, int max_partials,
                                    float *g, void *elems, uint8_t *rm, uint8_t *tc, int num_sms, int *wd,
                                    cudaStream_t st) {
+    const OutRange out[5] = {{elems, (uint64_t)(rows * cols / 2)}, {rm, (uint64_t)(rows * cols / 16)},
+                             {tc, tc_bytes(rows, cols / 16)}, {g, 4}, {partials, (uint64_t)max_partials * 4}};
+    cudaError_t e = set_out_ranges(out, st);
+    if (e != cudaSuccess) return e;
     const uint8_t *s8 = static_cast<const uint8_t *>(src);
     uint8_t *e8 = static_cast<uint8_t *>(elems);
     if (rm && tc) return launch_nvfp4_2d_t<true, true>(s8, rows, cols, partials, max_partials, g, e8, rm, tc, wd, num_sms, st);
@@ -816,6 +829,10 @@ cudaError_t launch_stream_nvfp4(const void *src, int64_t rows, int64_t cols, flo
     const uint32_t nb = (uint32_t)(rows * cols / 16), S = (uint32_t)(cols / 16);
     const FastDiv f = make_fastdiv(S);
     const uint32_t ca = (S + 3) / 4;
+    const OutRange out[5] = {{elems, (uint64_t)(rows * cols / 2)}, {rm, (uint64_t)(rows * cols / 16)},
+                             {tc, tc_bytes(rows, S)}, {g, 4}, {partials, (uint64_t)max_partials * 4}};
+    cudaError_t e = set_out_ranges(out, st);
+    if (e != cudaSuccess) return e;
     const uint8_t *s8 = static_cast<const uint8_t *>(src);
     uint8_t *e8 = static_cast<uint8_t *>(elems);
     if (rm && tc)
@@ -838,6 +855,9 @@ cudaError_t launch_stream_dequant_mx(const void *elems, const uint8_t *scales, i
     const uint32_t nb = (uint32_t)(rows * cols / 32), S = (uint32_t)(cols / 32);
     const FastDiv f = make_fastdiv(S);
     const uint32_t ca = (S + 3) / 4;
+    const OutRange orng[1] = {{out, (uint64_t)(rows * cols * 2)}};
+    cudaError_t e = set_out_ranges(orng, st);
+    if (e != cudaSuccess) return e;
     switch (fmt) {
     case FMT_E4M3: return tc ? launch_dq_t<FMT_E4M3, true>(elems, scales, nb, f, ca, out, wd, num_sms, st)
                              : launch_dq_t<FMT_E4M3, false>(elems, scales, nb, f, ca, out, wd, num_sms, st);
@@ -862,6 +882,9 @@ cudaError_t launch_stream_dequant_nvfp4(const void *elems, const uint8_t *scales
     const uint32_t ca = (S + 3) / 4;
     const uint32_t n_tiles = (nb + 2 * kThreads - 1) / (2 * kThreads);
     const int grid = stream_grid(n_tiles, num_sms);
+    const OutRange orng[1] = {{out, (uint64_t)(rows * cols * 2)}};
+    cudaError_t e = set_out_ranges(orng, st);
+    if (e != cudaSuccess) return e;
     const uint8_t *e8 = static_cast<const uint8_t *>(elems);
     uint4 *o = static_cast<uint4 *>(out);
     return tc ? launch_stream(dequant_nvfp4_bulk_kernel<true>, grid, st, e8, scales, g, nb, f, ca, o, wd)

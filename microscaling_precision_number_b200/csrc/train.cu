@@ -19,6 +19,7 @@
 // maximum saturates; the sign is kept.  Scales are computed exactly as in the RNE path.
 // One thread per quantisation block, blocks of consecutive threads adjacent in memory
 // (coalesced), grid-stride loops; NVFP4 takes a maximum pass and a quantisation pass.
+#include "checked.cuh"
 #include "codec.cuh"
 #include "internal.h"
 #include "nvfp4.cuh"
@@ -152,16 +153,16 @@ mx_train_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS
             scale8(v[j], mul2x, x);
             round8<FMT, SR>(x, rnd + (size_t)blk * 32 + 8 * j);
             if constexpr (FMT == FMT_E2M1) {
-                reinterpret_cast<uint32_t *>(elems)[(size_t)blk * 4 + j] = nan_blk ? 0u : cvt_e2m1x8(x);
+                out_store(reinterpret_cast<uint32_t *>(elems) + (size_t)blk * 4 + j, nan_blk ? 0u : cvt_e2m1x8(x));
             } else {
                 const uint2 q = cvt_fp8x8<FMT>(x);
-                reinterpret_cast<uint2 *>(elems)[(size_t)blk * 4 + j] = nan_blk ? make_uint2(0u, 0u) : q;
+                out_store(reinterpret_cast<uint2 *>(elems) + (size_t)blk * 4 + j, nan_blk ? make_uint2(0u, 0u) : q);
             }
         }
-        if constexpr (RM) sc_rm[blk] = (uint8_t)code;
+        if constexpr (RM) out_store(sc_rm + blk, (uint8_t)code);
         if constexpr (TC) {
             const uint32_t r = fdiv(blk, divS);
-            sc_tc[tc_offset(r, blk - r * divS.d, col_atoms)] = (uint8_t)code;
+            out_store(sc_tc + tc_offset(r, blk - r * divS.d, col_atoms), (uint8_t)code);
         }
     }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -192,7 +193,7 @@ nvfp4_train_amax_kernel(const uint8_t *__restrict__ src, uint32_t n_groups, uint
     if (threadIdx.x == 0) {
         uint32_t r = 0;
         for (int w = 0; w < kTrainThreads / 32; w++) r = max(r, warp_u[w]);
-        partials[blockIdx.x] = __uint_as_float(r << 16);
+        out_store(partials + blockIdx.x, __uint_as_float(r << 16));
     }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
@@ -217,7 +218,7 @@ nvfp4_train_quant_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fas
     a = 0.0f;
     for (int w = 0; w < kTrainThreads / 32; w++) a = fmaxf(a, red[w]);
     const float g = a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+    if (blockIdx.x == 0 && threadIdx.x == 0) out_store(g_out, g);
     const float six_g = __fmul_rn(6.0f, g);
     const RhtSigns sm = rht_signs(signs);
     for (uint32_t blk = blockIdx.x * kTrainThreads + threadIdx.x; blk < n_blocks; blk += gridDim.x * kTrainThreads) {
@@ -241,11 +242,11 @@ nvfp4_train_quant_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fas
         nvfp4_codes16(v[0], v[1], d, nr, q[0], q[1],
                       [&](float (&x)[8], int j) { round8<FMT_E2M1, SR>(x, rb + 8 * j); });
         if (zero_codes) q[0] = q[1] = 0u;
-        reinterpret_cast<uint2 *>(elems)[blk] = make_uint2(q[0], q[1]);
-        if constexpr (RM) sc_rm[blk] = (uint8_t)sb;
+        out_store(reinterpret_cast<uint2 *>(elems) + blk, make_uint2(q[0], q[1]));
+        if constexpr (RM) out_store(sc_rm + blk, (uint8_t)sb);
         if constexpr (TC) {
             const uint32_t rr = fdiv(blk, divS);
-            sc_tc[tc_offset(rr, blk - rr * divS.d, col_atoms)] = (uint8_t)sb;
+            out_store(sc_tc + tc_offset(rr, blk - rr * divS.d, col_atoms), (uint8_t)sb);
         }
     }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -316,6 +317,14 @@ cudaError_t launch_quantize_train(const void *src, int64_t rows, int64_t cols, i
     const uint8_t *s8 = static_cast<const uint8_t *>(src);
     uint8_t *e8 = static_cast<uint8_t *>(elems);
     const bool sr = rnd != nullptr;
+    {
+        const int64_t B = fmt == FMT_NVFP4 ? 16 : 32, S = cols / B;
+        const OutRange out[5] = {{elems, (uint64_t)(rows * cols * code_bits(fmt) / 8)}, {rm, (uint64_t)(rows * S)},
+                                 {tc, (uint64_t)((rows + 127) / 128) * ((S + 3) / 4) * 512}, {g, 4},
+                                 {partials, (uint64_t)max_partials * 4}};
+        const cudaError_t e = set_out_ranges(out, st);
+        if (e != cudaSuccess) return e;
+    }
     if (fmt == FMT_NVFP4) {
         const uint32_t nb = (uint32_t)(rows * cols / 16), S = (uint32_t)(cols / 16);
         const FastDiv f = make_fastdiv(S);

@@ -171,25 +171,6 @@ __device__ __forceinline__ void tmem_ld32_batch(uint32_t taddr, uint32_t (&r)[NJ
         asm volatile("" : "+r"(r[j][0]), "+r"(r[j][1]), "+r"(r[j][2]), "+r"(r[j][3]), "+r"(r[j][4]), "+r"(r[j][5]), "+r"(r[j][6]), "+r"(r[j][7]), "+r"(r[j][8]), "+r"(r[j][9]), "+r"(r[j][10]), "+r"(r[j][11]), "+r"(r[j][12]), "+r"(r[j][13]), "+r"(r[j][14]), "+r"(r[j][15]), "+r"(r[j][16]), "+r"(r[j][17]), "+r"(r[j][18]), "+r"(r[j][19]), "+r"(r[j][20]), "+r"(r[j][21]), "+r"(r[j][22]), "+r"(r[j][23]), "+r"(r[j][24]), "+r"(r[j][25]), "+r"(r[j][26]), "+r"(r[j][27]), "+r"(r[j][28]), "+r"(r[j][29]), "+r"(r[j][30]), "+r"(r[j][31]));
 }
 
-// ---- warp-uniform issue ---------------------------------------------------------------------
-// The issuing warps of the matmuls run their loops with all 32 lanes converged and let one
-// elected lane issue each group of tcgen05 / TMA instructions.  Measured on B200: a
-// tcgen05.mma stream issued this way sustains one M = 256 x N = 256 x K = 32 pair MMA per
-// 128 cycles (the tensor pipe's rate), whereas the same loop run by lane 0 alone inside a
-// divergent branch issued one per ~560 cycles.
-__device__ __forceinline__ bool elect_one() {
-    uint32_t pred = 0;
-    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
-    return pred != 0;
-}
-// Bounded wait by a whole warp; true only if every lane saw the phase complete.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t phase, int *watchdog, int code) {
-    const bool ok = mbar_wait_bounded(bar, phase, watchdog, code);
-    return __all_sync(0xffffffffu, ok);
-}
-// A shared failure flag read uniformly by a warp.
-__device__ __forceinline__ bool warp_failed(volatile int *flag) { return __any_sync(0xffffffffu, *flag != 0); }
-
 // ---- tile order ------------------------------------------------------------------------------
 // Banded raster: N-tiles are grouped into bands of `band` tiles whose B panels fit in L2;
 // within a band the tiles run M-major, so concurrently resident CTAs share A panels and the
