@@ -104,7 +104,8 @@ __device__ __forceinline__ void stream_tiles(Ring &ring, uint32_t n_tiles, Body 
     for (uint32_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++it) {
         const int s = (int)(it % kStages);
         const uint32_t phase = (it / kStages) & 1u;
-        const bool ok = mbar_wait_bounded(&ring.full[s], phase, ring.watchdog, WD_STREAM_FULL);
+        // warp-uniform outcome (bodies may use full-warp shuffles)
+        const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&ring.full[s], phase, ring.watchdog, WD_STREAM_FULL));
         if (ok) body(t, ring.buf + s * kTileBytes);
         __syncthreads();                                   // stage s is free again
         if (tid == 0) {
@@ -508,8 +509,10 @@ nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t r
 }
 
 // ---------------------------------------------------------------------------------------
-// Dequantisers: thread = one block; codes streamed through the ring, scales read
-// directly, bf16 written as 16-byte vectors.
+// Dequantisers: codes streamed through the ring; each thread reads the scale of one block
+// (two for NVFP4) directly; the bf16 output is written in 16-byte chunks of 8 elements,
+// the lanes of a warp taking consecutive chunks so that every store instruction covers
+// 512 contiguous bytes (FP6: thread = one block, 64 bytes).
 // ---------------------------------------------------------------------------------------
 template <int FMT, bool TC>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
@@ -527,34 +530,24 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
     Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
               full, watchdog, elems, kBlocksPerTile * kCodeBytes, (uint64_t)ring_blocks * kCodeBytes};
     const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
-    const uint32_t tid = threadIdx.x;
+    const uint32_t tid = threadIdx.x, lane = tid & 31u, wbase = tid & ~31u;
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
         const uint32_t blk = t * kBlocksPerTile + tid;
-        if (blk >= n_blocks) return;
-        uint32_t s;
-        if constexpr (TC) {
-            const uint32_t r = fdiv(blk, divS);
-            s = scales[tc_offset(r, blk - r * divS.d, col_atoms)];
-        } else {
-            s = scales[blk];
-        }
-        const float mul = s == 0xFFu ? __uint_as_float(0x7FC00000u) : e8m0_multiplier(s);
-        uint4 *dst = out + (size_t)blk * 4;
-        if constexpr (FMT == FMT_E2M1) {
-            const uint4 c = *reinterpret_cast<const uint4 *>(tile + tid * 16);
-            const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                float y[8];
-                e2m1x8_to_f32(w[j], y);
-                uint4 o;
-                o.x = f32x2_to_bf16x2(__fmul_rn(y[0], mul), __fmul_rn(y[1], mul));
-                o.y = f32x2_to_bf16x2(__fmul_rn(y[2], mul), __fmul_rn(y[3], mul));
-                o.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
-                o.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
-                out_store(dst + j, o);
+        // this thread's block scale as an fp32 multiplier (0 past the end, NaN for 0xFF)
+        float mul = 0.0f;
+        if (blk < n_blocks) {
+            uint32_t s;
+            if constexpr (TC) {
+                const uint32_t r = fdiv(blk, divS);
+                s = scales[tc_offset(r, blk - r * divS.d, col_atoms)];
+            } else {
+                s = scales[blk];
             }
-        } else if constexpr (is_fp6(FMT)) {
+            mul = s == 0xFFu ? __uint_as_float(0x7FC00000u) : e8m0_multiplier(s);
+        }
+        if constexpr (is_fp6(FMT)) {
+            if (blk >= n_blocks) return;
+            uint4 *dst = out + (size_t)blk * 4;
             // 24 bytes = 32 packed codes, as three 8-byte reads (stride 24 B: conflict-free)
             const uint2 *p = blk < ring_blocks ? reinterpret_cast<const uint2 *>(tile + tid * 24)
                                                : reinterpret_cast<const uint2 *>(elems + (size_t)blk * 24);
@@ -577,26 +570,33 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
                 out_store(dst + j, q);
             }
         } else {
-            const uint32_t rot = (tid >> 2) & 1u;
+            // The warp's 32 blocks are 128 chunks of 8 elements; in round j lane l converts
+            // chunk 32 j + l, so every store instruction of the warp writes 512 contiguous
+            // bytes.  The chunk's block scale comes from its owner lane by a shuffle.
+            constexpr uint32_t kChunkBytes = kCodeBytes / 4;               // 4 (FP4) or 8
+            const uint8_t *wcodes = tile + wbase * kCodeBytes;
+            uint4 *wout = out + ((size_t)t * kBlocksPerTile + wbase) * 4;
 #pragma unroll
-            for (int h = 0; h < 2; h++) {
-                const uint32_t hc = (h + rot) & 1u;
-                const uint4 c = *reinterpret_cast<const uint4 *>(tile + tid * 32 + hc * 16);
-                const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-                for (int j = 0; j < 2; j++) {
-                    float y[8];
-                    fp8x2_to_f32<FMT>(w[2 * j] & 0xFFFFu, y[0], y[1]);
-                    fp8x2_to_f32<FMT>(w[2 * j] >> 16, y[2], y[3]);
-                    fp8x2_to_f32<FMT>(w[2 * j + 1] & 0xFFFFu, y[4], y[5]);
-                    fp8x2_to_f32<FMT>(w[2 * j + 1] >> 16, y[6], y[7]);
-                    uint4 o;
-                    o.x = f32x2_to_bf16x2(__fmul_rn(y[0], mul), __fmul_rn(y[1], mul));
-                    o.y = f32x2_to_bf16x2(__fmul_rn(y[2], mul), __fmul_rn(y[3], mul));
-                    o.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
-                    o.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
-                    out_store(dst + hc * 2 + j, o);
+            for (int j = 0; j < 4; j++) {
+                const uint32_t q = 32u * j + lane, lb = q >> 2;               // chunk, block in the warp
+                const float m = __shfl_sync(0xFFFFFFFFu, mul, (int)lb);
+                if (t * kBlocksPerTile + wbase + lb >= n_blocks) continue;
+                float y[8];
+                if constexpr (FMT == FMT_E2M1) {
+                    e2m1x8_to_f32(*reinterpret_cast<const uint32_t *>(wcodes + q * kChunkBytes), y);
+                } else {
+                    const uint2 c = *reinterpret_cast<const uint2 *>(wcodes + q * kChunkBytes);
+                    fp8x2_to_f32<FMT>(c.x & 0xFFFFu, y[0], y[1]);
+                    fp8x2_to_f32<FMT>(c.x >> 16, y[2], y[3]);
+                    fp8x2_to_f32<FMT>(c.y & 0xFFFFu, y[4], y[5]);
+                    fp8x2_to_f32<FMT>(c.y >> 16, y[6], y[7]);
                 }
+                uint4 o;
+                o.x = f32x2_to_bf16x2(__fmul_rn(y[0], m), __fmul_rn(y[1], m));
+                o.y = f32x2_to_bf16x2(__fmul_rn(y[2], m), __fmul_rn(y[3], m));
+                o.z = f32x2_to_bf16x2(__fmul_rn(y[4], m), __fmul_rn(y[5], m));
+                o.w = f32x2_to_bf16x2(__fmul_rn(y[6], m), __fmul_rn(y[7], m));
+                out_store(wout + q, o);
             }
         }
     });
@@ -616,42 +616,52 @@ dequant_nvfp4_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__re
     Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
               full, watchdog, elems, kBlocksPerTile * 8, (uint64_t)(n_blocks & ~1u) * 8};
     const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
-    const uint32_t tid = threadIdx.x;
+    const uint32_t tid = threadIdx.x, lane = tid & 31u, wbase = 2u * (tid & ~31u);   // warp's first block
     const float g = *g_ptr;
+    const uint32_t ring_blocks = n_blocks & ~1u;
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
-        const uint32_t blk0 = t * kBlocksPerTile + tid * 2;   // two consecutive blocks
-        if (blk0 >= n_blocks) return;
-        uint4 c;
-        if (blk0 + 1 < n_blocks) {
-            c = *reinterpret_cast<const uint4 *>(tile + tid * 16);
-        } else {
-            const uint2 h = *reinterpret_cast<const uint2 *>(elems + (size_t)blk0 * 8);
-            c = make_uint4(h.x, h.y, 0u, 0u);
-        }
-        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        // this thread's two blocks' UE4M3 scales (0 past the end, NaN for 0x7F)
+        const uint32_t blk0 = t * kBlocksPerTile + tid * 2;
+        float sbv[2];
 #pragma unroll
         for (int b = 0; b < 2; b++) {
             const uint32_t blk = blk0 + b;
-            if (blk >= n_blocks) break;
-            uint32_t s;
-            if constexpr (TC) {
-                const uint32_t r = fdiv(blk, divS);
-                s = scales[tc_offset(r, blk - r * divS.d, col_atoms)] & 0x7Fu;
-            } else {
-                s = scales[blk] & 0x7Fu;
+            sbv[b] = 0.0f;
+            if (blk < n_blocks) {
+                uint32_t s;
+                if constexpr (TC) {
+                    const uint32_t r = fdiv(blk, divS);
+                    s = scales[tc_offset(r, blk - r * divS.d, col_atoms)] & 0x7Fu;
+                } else {
+                    s = scales[blk] & 0x7Fu;
+                }
+                sbv[b] = s == 0x7Fu ? __uint_as_float(0x7FC00000u) : ue4m3_to_f32(s);
             }
-            const float sbv = s == 0x7Fu ? __uint_as_float(0x7FC00000u) : ue4m3_to_f32(s);
+        }
+        // The warp's 64 blocks are 128 chunks of 8 elements; in round j lane l converts
+        // chunk 32 j + l (block 16 j + l / 2, owned by lane 8 j + l / 4), so every store
+        // instruction of the warp writes 512 contiguous bytes.
+        const uint32_t wblk = t * kBlocksPerTile + wbase;
+        uint4 *wout = out + (size_t)wblk * 2;
 #pragma unroll
-            for (int j = 0; j < 2; j++) {
-                float y[8];
-                e2m1x8_to_f32(w[2 * b + j], y);
-                uint4 o;
-                o.x = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[0], sbv), g), __fmul_rn(__fmul_rn(y[1], sbv), g));
-                o.y = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[2], sbv), g), __fmul_rn(__fmul_rn(y[3], sbv), g));
-                o.z = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[4], sbv), g), __fmul_rn(__fmul_rn(y[5], sbv), g));
-                o.w = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[6], sbv), g), __fmul_rn(__fmul_rn(y[7], sbv), g));
-                out_store(out + (size_t)blk * 2 + j, o);
-            }
+        for (int j = 0; j < 4; j++) {
+            const uint32_t q = 32u * j + lane, lb = q >> 1;
+            const float s0 = __shfl_sync(0xFFFFFFFFu, sbv[0], (int)(lb >> 1));
+            const float s1 = __shfl_sync(0xFFFFFFFFu, sbv[1], (int)(lb >> 1));
+            const float sb = (lb & 1u) ? s1 : s0;
+            const uint32_t blk = wblk + lb;
+            if (blk >= n_blocks) continue;
+            const uint32_t c = blk < ring_blocks
+                                   ? *reinterpret_cast<const uint32_t *>(tile + (size_t)(wbase + lb) * 8 + (q & 1u) * 4)
+                                   : *reinterpret_cast<const uint32_t *>(elems + (size_t)blk * 8 + (q & 1u) * 4);
+            float y[8];
+            e2m1x8_to_f32(c, y);
+            uint4 o;
+            o.x = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[0], sb), g), __fmul_rn(__fmul_rn(y[1], sb), g));
+            o.y = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[2], sb), g), __fmul_rn(__fmul_rn(y[3], sb), g));
+            o.z = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[4], sb), g), __fmul_rn(__fmul_rn(y[5], sb), g));
+            o.w = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[6], sb), g), __fmul_rn(__fmul_rn(y[7], sb), g));
+            out_store(wout + q, o);
         }
     });
 }
