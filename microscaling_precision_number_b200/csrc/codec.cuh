@@ -213,9 +213,8 @@ __device__ __forceinline__ void fp8x2_to_f32(uint32_t codes16, float &lo, float 
         : "=f"(lo), "=f"(hi) : "r"(h2));
 }
 
-// Eight E2M1 codes (nibble i = element i) -> eight fp32, exact.
-__device__ __forceinline__ void e2m1x8_to_f32(uint32_t codes, float (&y)[8]) {
-    uint32_t h[4];
+// Eight E2M1 codes (nibble i = element i) -> four f16x2 words (element 2i low), exact.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t codes, uint32_t (&h)[4]) {
     asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
         "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
         "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
@@ -223,11 +222,20 @@ __device__ __forceinline__ void e2m1x8_to_f32(uint32_t codes, float (&y)[8]) {
         "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
         "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
         : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(codes));
+}
+
+// f16x2 word -> two fp32 (low half in lo), exact.
+__device__ __forceinline__ void f16x2_to_f32(uint32_t h2, float &lo, float &hi) {
+    asm("{\n\t.reg .f16 l, hh;\n\tmov.b32 {l, hh}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, hh;\n\t}"
+        : "=f"(lo), "=f"(hi) : "r"(h2));
+}
+
+// Eight E2M1 codes (nibble i = element i) -> eight fp32, exact.
+__device__ __forceinline__ void e2m1x8_to_f32(uint32_t codes, float (&y)[8]) {
+    uint32_t h[4];
+    e2m1x8_to_f16x2(codes, h);
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-        asm("{\n\t.reg .f16 l, hh;\n\tmov.b32 {l, hh}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, hh;\n\t}"
-            : "=f"(y[2 * i]), "=f"(y[2 * i + 1]) : "r"(h[i]));
-    }
+    for (int i = 0; i < 4; i++) f16x2_to_f32(h[i], y[2 * i], y[2 * i + 1]);
 }
 
 // Two fp32 -> bf16x2 word (round to nearest even), `lo` in the low half.

@@ -514,6 +514,19 @@ nvfp4_2d_quant_kernel(const uint8_t *__restrict__ src, uint32_t cols, uint32_t r
 // the lanes of a warp taking consecutive chunks so that every store instruction covers
 // 512 contiguous bytes (FP6: thread = one block, 64 bytes).
 // ---------------------------------------------------------------------------------------
+// Eight fp32 times the scale m (m2 = m in both lanes), each product rounded to fp32 and then
+// to bf16: one packed fp32 product per element pair.
+__device__ __forceinline__ uint4 scaled_bf16x8(const float (&y)[8], uint64_t m2) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        float lo, hi;
+        unpack2(mul2(pack2(y[2 * i], y[2 * i + 1]), m2), lo, hi);
+        w[i] = f32x2_to_bf16x2(lo, hi);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 template <int FMT, bool TC>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restrict__ scales,
@@ -562,12 +575,7 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
                 fp8x2_to_f32<FMT>(w[2 * j] >> 16, y[2], y[3]);
                 fp8x2_to_f32<FMT>(w[2 * j + 1] & 0xFFFFu, y[4], y[5]);
                 fp8x2_to_f32<FMT>(w[2 * j + 1] >> 16, y[6], y[7]);
-                uint4 q;
-                q.x = f32x2_to_bf16x2(__fmul_rn(y[0], mul), __fmul_rn(y[1], mul));
-                q.y = f32x2_to_bf16x2(__fmul_rn(y[2], mul), __fmul_rn(y[3], mul));
-                q.z = f32x2_to_bf16x2(__fmul_rn(y[4], mul), __fmul_rn(y[5], mul));
-                q.w = f32x2_to_bf16x2(__fmul_rn(y[6], mul), __fmul_rn(y[7], mul));
-                out_store(dst + j, q);
+                out_store(dst + j, scaled_bf16x8(y, splat2(mul)));
             }
         } else {
             // The warp's 32 blocks are 128 chunks of 8 elements; in round j lane l converts
@@ -591,12 +599,7 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
                     fp8x2_to_f32<FMT>(c.y & 0xFFFFu, y[4], y[5]);
                     fp8x2_to_f32<FMT>(c.y >> 16, y[6], y[7]);
                 }
-                uint4 o;
-                o.x = f32x2_to_bf16x2(__fmul_rn(y[0], m), __fmul_rn(y[1], m));
-                o.y = f32x2_to_bf16x2(__fmul_rn(y[2], m), __fmul_rn(y[3], m));
-                o.z = f32x2_to_bf16x2(__fmul_rn(y[4], m), __fmul_rn(y[5], m));
-                o.w = f32x2_to_bf16x2(__fmul_rn(y[6], m), __fmul_rn(y[7], m));
-                out_store(wout + q, o);
+                out_store(wout + q, scaled_bf16x8(y, splat2(m)));
             }
         }
     });
@@ -617,26 +620,29 @@ dequant_nvfp4_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__re
               full, watchdog, elems, kBlocksPerTile * 8, (uint64_t)(n_blocks & ~1u) * 8};
     const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
     const uint32_t tid = threadIdx.x, lane = tid & 31u, wbase = 2u * (tid & ~31u);   // warp's first block
-    const float g = *g_ptr;
+    const uint64_t g2 = splat2(*g_ptr);
     const uint32_t ring_blocks = n_blocks & ~1u;
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
-        // this thread's two blocks' UE4M3 scales (0 past the end, NaN for 0x7F)
+        // this thread's two blocks' UE4M3 scales as f16x2 words holding dec(sb) twice (0 past
+        // the end; code 0x7F decodes to NaN).  dec(q) dec(sb) is exact in f16: at most 6
+        // significant bits, magnitudes 2^-10 .. 2688, so the packed f16 product equals the
+        // fp32 one and only the product with g rounds.
         const uint32_t blk0 = t * kBlocksPerTile + tid * 2;
-        float sbv[2];
+        uint32_t sbh[2];
 #pragma unroll
         for (int b = 0; b < 2; b++) {
             const uint32_t blk = blk0 + b;
-            sbv[b] = 0.0f;
+            uint32_t s = 0;
             if (blk < n_blocks) {
-                uint32_t s;
                 if constexpr (TC) {
                     const uint32_t r = fdiv(blk, divS);
                     s = scales[tc_offset(r, blk - r * divS.d, col_atoms)] & 0x7Fu;
                 } else {
                     s = scales[blk] & 0x7Fu;
                 }
-                sbv[b] = s == 0x7Fu ? __uint_as_float(0x7FC00000u) : ue4m3_to_f32(s);
             }
+            const uint16_t s2 = (uint16_t)(s | (s << 8));
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(sbh[b]) : "h"(s2));
         }
         // The warp's 64 blocks are 128 chunks of 8 elements; in round j lane l converts
         // chunk 32 j + l (block 16 j + l / 2, owned by lane 8 j + l / 4), so every store
@@ -646,22 +652,24 @@ dequant_nvfp4_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__re
 #pragma unroll
         for (int j = 0; j < 4; j++) {
             const uint32_t q = 32u * j + lane, lb = q >> 1;
-            const float s0 = __shfl_sync(0xFFFFFFFFu, sbv[0], (int)(lb >> 1));
-            const float s1 = __shfl_sync(0xFFFFFFFFu, sbv[1], (int)(lb >> 1));
-            const float sb = (lb & 1u) ? s1 : s0;
+            const uint32_t s0 = __shfl_sync(0xFFFFFFFFu, sbh[0], (int)(lb >> 1));
+            const uint32_t s1 = __shfl_sync(0xFFFFFFFFu, sbh[1], (int)(lb >> 1));
+            const uint32_t sb = (lb & 1u) ? s1 : s0;
             const uint32_t blk = wblk + lb;
             if (blk >= n_blocks) continue;
             const uint32_t c = blk < ring_blocks
                                    ? *reinterpret_cast<const uint32_t *>(tile + (size_t)(wbase + lb) * 8 + (q & 1u) * 4)
                                    : *reinterpret_cast<const uint32_t *>(elems + (size_t)blk * 8 + (q & 1u) * 4);
+            uint32_t h[4];
+            e2m1x8_to_f16x2(c, h);
             float y[8];
-            e2m1x8_to_f32(c, y);
-            uint4 o;
-            o.x = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[0], sb), g), __fmul_rn(__fmul_rn(y[1], sb), g));
-            o.y = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[2], sb), g), __fmul_rn(__fmul_rn(y[3], sb), g));
-            o.z = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[4], sb), g), __fmul_rn(__fmul_rn(y[5], sb), g));
-            o.w = f32x2_to_bf16x2(__fmul_rn(__fmul_rn(y[6], sb), g), __fmul_rn(__fmul_rn(y[7], sb), g));
-            out_store(wout + q, o);
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                uint32_t p;
+                asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p) : "r"(h[i]), "r"(sb));
+                f16x2_to_f32(p, y[2 * i], y[2 * i + 1]);
+            }
+            out_store(wout + q, scaled_bf16x8(y, g2));
         }
     });
 }
