@@ -61,8 +61,8 @@ WORKLOAD = "dual_mxfp8_act_16384x4096_e4m3_and_grad_16384x14336_e5m2_tcgen05_sca
 # capture of the benchmark's own back-to-back sequence (no cache control, no clock
 # control), and the SHA-256 of the kernel source that capture ran: when dual.cu has
 # changed since, the traffic is reported as null.
-NCU_TRAFFIC_GRAD = 957941333      # mean of 3 launches: read ~470.05 MB + write ~487.89 MB
-NCU_TRAFFIC_SRC_SHA = "dfceb4fce6e1983c72ec847cb1f19a6ffc7d5744c5a8326223337e72398de251"
+NCU_TRAFFIC_GRAD = 955429547      # mean of 3 launches: read ~469.86 MB + write ~485.57 MB
+NCU_TRAFFIC_SRC_SHA = "4016d5c75a5aca8215a7468d27bf3cac2d3800e9b1cbad20f510c165b58de969"
 DUAL_SRC = os.path.join(ROOT, "microscaling_precision_number_b200", "csrc", "dual.cu")
 
 # the 4096 x 4096 weight: MXFP4 (floor) + NVFP4, both scale layouts (a breakdown row)
