@@ -9,8 +9,8 @@
 // by a cluster of two CTAs on two SMs:
 //   - each CTA loads its own 128 rows of A and its own 128 rows (of 256) of B, plus its A
 //     rows' scale atoms and the scale atoms of all 256 B rows, with 2-D TMA loads that all
-//     complete on the even CTA's barrier (the `.cta_group::2` form with the peer bit of the
-//     barrier address cleared);
+//     complete on the even CTA's barriers (the `.cta_group::2` form with the peer bit of the
+//     barrier address cleared; scale atoms and operand tiles on separate barriers);
 //   - the even CTA's MMA thread copies the stage's scale atoms (each CTA's own shared
 //     memory into its own tensor memory) and issues tcgen05.mma.cta_group::2 with M = 256:
 //     the tensor core of each SM computes its CTA's 128 rows x 256 columns, reading A from
@@ -106,7 +106,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     uint8_t *sSFA = sB + S * P::kBStage;                 // S x kAtoms x 512 B
     uint8_t *sSFB = sSFA + S * P::kSfaBytes;             // S x 2 x kAtoms x 512 B
 
-    __shared__ __align__(8) uint64_t full_bar[S], empty_bar[S], sf_ready[S], acc_full, acc_empty, drain_bar,
+    __shared__ __align__(8) uint64_t full_bar[S], sf_full[S], empty_bar[S], sf_ready[S], acc_full, acc_empty, drain_bar,
         sf_drain, exit_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int fail_flag;
@@ -127,6 +127,7 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         prefetch_tensormap(&tmSB);
         for (int s = 0; s < S; s++) {
             mbar_init(&full_bar[s], 1);
+            mbar_init(&sf_full[s], 1);
             mbar_init(&empty_bar[s], 1);
             mbar_init(&sf_ready[s], 1);
         }
@@ -151,10 +152,10 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // ------------------------------------------------ TMA producer (both CTAs)
         // the whole warp runs the loop; one elected lane issues the copies
         const int col_atoms = num_kb * P::kAtoms;            // scale atoms per 128-row block
-        const uint32_t tx_pair =
-            2u * (SUB * ((KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kABytes, a_fmt_code) : kABytes) +
-                         (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kBBytes, b_fmt_code) : kBBytes)) +
-                  P::kSfaBytes + P::kSfbBytes);
+        const uint32_t tx_ops =
+            2u * SUB * ((KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kABytes, a_fmt_code) : kABytes) +
+                        (KIND == KIND_F8F6F4 ? f8f6f4_packed_bytes(kBBytes, b_fmt_code) : kBBytes));
+        const uint32_t tx_sf = 2u * (P::kSfaBytes + P::kSfbBytes);
         int it = 0;
         for (int t = pair; t < n_tiles && !warp_failed(fail_sh); t += n_pairs) {
             int m_blk, n_blk;
@@ -168,21 +169,25 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     break;
                 }
                 if (elect_one()) {
-                    if (leader) mbar_arrive_expect_tx(&full_bar[s], tx_pair);
+                    if (leader) {
+                        mbar_arrive_expect_tx(&sf_full[s], tx_sf);
+                        mbar_arrive_expect_tx(&full_bar[s], tx_ops);
+                    }
+                    // scale atoms first, on their own barrier, so that their copy into tensor
+                    // memory overlaps the landing of the operand tiles; atoms as rows of 256
+                    // bytes (two per atom), a stage's atoms of one 128-row block contiguous
+                    tma_load_2d_pair(sSFA + s * P::kSfaBytes, &tmSA, 0,
+                                     2 * ((2 * m_blk + (int)rank) * col_atoms + kb * P::kAtoms), &sf_full[s]);
+#pragma unroll
+                    for (int h = 0; h < 2; h++)
+                        tma_load_2d_pair(sSFB + s * P::kSfbBytes + h * P::kSfaBytes, &tmSB, 0,
+                                         2 * ((2 * n_blk + h) * col_atoms + kb * P::kAtoms), &sf_full[s]);
 #pragma unroll
                     for (int j = 0; j < SUB; j++) {
                         const int kx = (kb * SUB + j) * kRowBytes;
                         tma_load_2d_pair(sA + s * P::kAStage + j * kABytes, &tmA, kx, a_row, &full_bar[s]);
                         tma_load_2d_pair(sB + s * P::kBStage + j * kBBytes, &tmB, kx, b_row, &full_bar[s]);
                     }
-                    // scale atoms as rows of 256 bytes (two per atom); a stage's atoms of one
-                    // 128-row block are contiguous
-                    tma_load_2d_pair(sSFA + s * P::kSfaBytes, &tmSA, 0,
-                                     2 * ((2 * m_blk + (int)rank) * col_atoms + kb * P::kAtoms), &full_bar[s]);
-#pragma unroll
-                    for (int h = 0; h < 2; h++)
-                        tma_load_2d_pair(sSFB + s * P::kSfbBytes + h * P::kSfaBytes, &tmSB, 0,
-                                         2 * ((2 * n_blk + h) * col_atoms + kb * P::kAtoms), &full_bar[s]);
                 }
                 __syncwarp();
                 last_it[s] = it;
@@ -190,18 +195,20 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     } else if (warp == kSfWarp) {
         // ------------------------------------------------ scale-atom copier (even CTA only)
-        // Copies each stage's scale atoms into tensor memory (both CTAs') as soon as the
-        // stage has landed, and signals sf_ready[s] once the copies are complete.  The MMA
-        // issuer waits on sf_ready alone (it implies the stage's operands are there), so the
-        // copies stay off the MMA-issuing warp.  A stage's scale slot is rewritten only after
-        // full[s] of its next use, i.e. after the MMAs that read it have completed (empty[s]).
+        // Copies each stage's scale atoms into tensor memory (both CTAs') as soon as they
+        // have landed (sf_full[s]: the atoms travel apart from the operand tiles and are
+        // issued first, so the copies overlap the tiles' landing), and signals sf_ready[s]
+        // once the copies are complete.  The MMA issuer waits on full[s] (operands) and
+        // sf_ready[s], so the copies stay off the MMA-issuing warp.  A stage's scale slot is
+        // rewritten only after sf_full[s] of its next use, which the producer arms after
+        // empty[s], i.e. after the MMAs that read the slot have completed.
         if (leader) {
             const uint64_t sfa_d0 = sf_desc(smem_u32(sSFA)), sfb_d0 = sf_desc(smem_u32(sSFB));
             int it = 0;
             for (int t = pair; t < n_tiles && !warp_failed(fail_sh); t += n_pairs) {
                 for (int kb = 0; kb < num_kb; kb++, it++) {
                     const int s = it % S;
-                    if (!warp_wait(&full_bar[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
+                    if (!warp_wait(&sf_full[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
                         *fail_sh = 1;
                         break;
                     }
@@ -249,7 +256,8 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 for (int kb = 0; kb < num_kb; kb++, it++) {
                     const int s = it % S;
                     // the stage's operands have landed and its scales are in tensor memory
-                    if (!warp_wait(&sf_ready[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
+                    if (!warp_wait(&full_bar[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL) ||
+                        !warp_wait(&sf_ready[s], (uint32_t)(it / S) & 1u, watchdog, WD_GEMM_FULL)) {
                         *fail_sh = 1;
                         break;
                     }
@@ -325,8 +333,10 @@ mx_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     // for the pair's copies that were counted on its barriers
     if (warp == kProducerWarp && lane == 0 && leader && *fail_sh)
         for (int s = 0; s < S; s++)
-            if (last_it[s] >= 0)
+            if (last_it[s] >= 0) {
+                (void)mbar_wait_bounded(&sf_full[s], (uint32_t)(last_it[s] / S) & 1u, nullptr, 0, kDrainLimitNs);
                 (void)mbar_wait_bounded(&full_bar[s], (uint32_t)(last_it[s] / S) & 1u, nullptr, 0, kDrainLimitNs);
+            }
     __syncthreads();
     if (warp == kMmaWarp && lane == 0) {
         (void)mbar_wait_bounded(&drain_bar, 0u, nullptr, 0, kDrainLimitNs);
