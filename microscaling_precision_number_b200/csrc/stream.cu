@@ -544,20 +544,25 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
               full, watchdog, elems, kBlocksPerTile * kCodeBytes, (uint64_t)ring_blocks * kCodeBytes};
     const uint32_t n_tiles = (n_blocks + kBlocksPerTile - 1) / kBlocksPerTile;
     const uint32_t tid = threadIdx.x, lane = tid & 31u, wbase = tid & ~31u;
+    // this thread's block scale of tile t (0x100 past the end); loaded one tile ahead, so
+    // that its latency overlaps the previous tile instead of stalling the current one
+    auto scale_of = [&](uint32_t t) -> uint32_t {
+        const uint32_t blk = t * kBlocksPerTile + tid;
+        if (t >= n_tiles || blk >= n_blocks) return 0x100u;
+        if constexpr (TC) {
+            const uint32_t r = fdiv(blk, divS);
+            return scales[tc_offset(r, blk - r * divS.d, col_atoms)];
+        } else {
+            return scales[blk];
+        }
+    };
+    uint32_t s_next = scale_of(blockIdx.x);
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
         const uint32_t blk = t * kBlocksPerTile + tid;
-        // this thread's block scale as an fp32 multiplier (0 past the end, NaN for 0xFF)
-        float mul = 0.0f;
-        if (blk < n_blocks) {
-            uint32_t s;
-            if constexpr (TC) {
-                const uint32_t r = fdiv(blk, divS);
-                s = scales[tc_offset(r, blk - r * divS.d, col_atoms)];
-            } else {
-                s = scales[blk];
-            }
-            mul = s == 0xFFu ? __uint_as_float(0x7FC00000u) : e8m0_multiplier(s);
-        }
+        const uint32_t s = s_next;
+        s_next = scale_of(t + gridDim.x);
+        // the block scale as an fp32 multiplier (0 past the end, NaN for 0xFF)
+        const float mul = s == 0x100u ? 0.0f : s == 0xFFu ? __uint_as_float(0x7FC00000u) : e8m0_multiplier(s);
         if constexpr (is_fp6(FMT)) {
             if (blk >= n_blocks) return;
             uint4 *dst = out + (size_t)blk * 4;
@@ -622,25 +627,35 @@ dequant_nvfp4_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__re
     const uint32_t tid = threadIdx.x, lane = tid & 31u, wbase = 2u * (tid & ~31u);   // warp's first block
     const uint64_t g2 = splat2(*g_ptr);
     const uint32_t ring_blocks = n_blocks & ~1u;
+    // this thread's two UE4M3 block scales of tile t (0 past the end), loaded one tile ahead
+    auto scales_of = [&](uint32_t t, uint32_t (&sc)[2]) {
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            const uint32_t blk = t * kBlocksPerTile + tid * 2 + b;
+            sc[b] = 0u;
+            if (t < n_tiles && blk < n_blocks) {
+                if constexpr (TC) {
+                    const uint32_t r = fdiv(blk, divS);
+                    sc[b] = scales[tc_offset(r, blk - r * divS.d, col_atoms)];
+                } else {
+                    sc[b] = scales[blk];
+                }
+            }
+        }
+    };
+    uint32_t sc_next[2];
+    scales_of(blockIdx.x, sc_next);
     stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
         // this thread's two blocks' UE4M3 scales as f16x2 words holding dec(sb) twice (0 past
         // the end; code 0x7F decodes to NaN).  dec(q) dec(sb) is exact in f16: at most 6
         // significant bits, magnitudes 2^-10 .. 2688, so the packed f16 product equals the
         // fp32 one and only the product with g rounds.
-        const uint32_t blk0 = t * kBlocksPerTile + tid * 2;
+        const uint32_t sc[2] = {sc_next[0], sc_next[1]};
+        scales_of(t + gridDim.x, sc_next);
         uint32_t sbh[2];
 #pragma unroll
         for (int b = 0; b < 2; b++) {
-            const uint32_t blk = blk0 + b;
-            uint32_t s = 0;
-            if (blk < n_blocks) {
-                if constexpr (TC) {
-                    const uint32_t r = fdiv(blk, divS);
-                    s = scales[tc_offset(r, blk - r * divS.d, col_atoms)] & 0x7Fu;
-                } else {
-                    s = scales[blk] & 0x7Fu;
-                }
-            }
+            const uint32_t s = sc[b] & 0x7Fu;
             const uint16_t s2 = (uint16_t)(s | (s << 8));
             asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(sbh[b]) : "h"(s2));
         }
