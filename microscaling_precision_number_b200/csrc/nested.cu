@@ -56,7 +56,8 @@ __global__ void __launch_bounds__(kNestThreads)
 mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restrict__ scales, int64_t cols,
                            uint32_t blocks_c, uint8_t *__restrict__ out, float *__restrict__ block_scale,
                            uint8_t *__restrict__ block_exact) {
-    __shared__ int warp_max[kNestThreads / 32];
+    __shared__ __align__(16) int warp_max[kNestThreads / 32];
+    static_assert(kNestThreads / 32 == 8, "the block maximum reads the eight warp maxima as two int4");
     const uint32_t blk = blockIdx.x;
     const uint32_t br = blk / blocks_c, bc = blk - br * blocks_c;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -77,13 +78,11 @@ mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__r
         const bool nonzero = ((w[4 * t] | w[4 * t + 1] | w[4 * t + 2] | w[4 * t + 3]) & 0x77777777u) != 0u;
         if (sc[t] != 0xFFu && nonzero) m = max(m, (int)sc[t] - 127);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    m = __reduce_max_sync(0xFFFFFFFFu, m);                       // one redux instruction per warp
     if (lane == 0) warp_max[warp] = m;
     __syncthreads();
-    int smax = warp_max[0];
-#pragma unroll
-    for (int i = 1; i < kNestThreads / 32; i++) smax = max(smax, warp_max[i]);
+    const int4 wa = *reinterpret_cast<const int4 *>(&warp_max[0]), wb = *reinterpret_cast<const int4 *>(&warp_max[4]);
+    int smax = max(max(max(wa.x, wa.y), max(wa.z, wa.w)), max(max(wb.x, wb.y), max(wb.z, wb.w)));
     if (smax == kNoScale) smax = 6;                               // no nonzero finite element: S = 1
 
     bool exact = true;

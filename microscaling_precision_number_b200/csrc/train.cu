@@ -178,7 +178,26 @@ nvfp4_train_amax_kernel(const uint8_t *__restrict__ src, uint32_t n_groups, uint
     __shared__ uint32_t warp_u[kTrainThreads / 32];
     uint32_t acc = 0;
     const RhtSigns sm = rht_signs(signs);
-    for (uint32_t gi = blockIdx.x * kTrainThreads + threadIdx.x; gi < n_groups; gi += gridDim.x * kTrainThreads) {
+    // kUnroll groups per trip, all loads issued before the first transform
+    constexpr uint32_t kUnroll = 4;
+    const uint32_t stride = gridDim.x * kTrainThreads;
+    uint32_t gi = blockIdx.x * kTrainThreads + threadIdx.x;
+    for (; gi + (kUnroll - 1) * stride < n_groups; gi += kUnroll * stride) {
+        uint4 v[kUnroll][2];
+#pragma unroll
+        for (uint32_t u = 0; u < kUnroll; u++) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)(gi + u * stride) * 32);
+            v[u][0] = p[0];
+            v[u][1] = p[1];
+        }
+#pragma unroll
+        for (uint32_t u = 0; u < kUnroll; u++) {
+            if constexpr (RHT) rht16(v[u][0], v[u][1], sm);
+            acc = __vmaxu2(acc, finite_abs_max_bf16x8(v[u][0]));
+            acc = __vmaxu2(acc, finite_abs_max_bf16x8(v[u][1]));
+        }
+    }
+    for (; gi < n_groups; gi += stride) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)gi * 32);
         uint4 v0 = p[0], v1 = p[1];
         if constexpr (RHT) rht16(v0, v1, sm);
