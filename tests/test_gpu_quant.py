@@ -207,6 +207,28 @@ def test_dequantize_all_scale_codes(oracle):
         assert nan_aware_equal(d.reshape(-1), oracle.dequantize_mx(elems, scales, 256, 32, fmt).reshape(-1))
 
 
+@pytest.mark.parametrize("fmt", [0, 1, 2, 4, 5, 6, "nvfp4"])
+@pytest.mark.parametrize("layout", ["rowmajor", "tcgen05"])
+def test_dequantize_many_tiles_per_cta(oracle, fmt, layout):
+    """Shapes with more ring tiles than resident CTAs (each CTA walks several tiles and
+    loads the next tile's block scales ahead), an odd block count (FP6 and NVFP4 read the
+    last block from global memory) and a ragged last tile."""
+    rows, cols = (12289, 496) if fmt == "nvfp4" else (12289, 480)
+    x = with_specials(synth.mx8_rowwise(rows, cols, seed=11), seed=5)
+    if fmt == "nvfp4":
+        q = mx.quantize(to_dev(x), "nvfp4", "row", "ceil", layout="both")
+        e_ref, s_ref, g_ref = oracle.quantize_nvfp4(x)
+        assert np.array_equal(host(q.elems), e_ref.reshape(-1))
+        ref = oracle.dequantize_nvfp4(e_ref, s_ref, g_ref, rows, cols)
+    else:
+        q = mx.quantize(to_dev(x), FMT_NAMES[fmt], "row", "ceil", layout="both")
+        e_ref, s_ref = oracle.quantize_mx(x, fmt, oracle.ROW, oracle.CEIL)
+        assert np.array_equal(host(q.elems), e_ref.reshape(-1))
+        ref = oracle.dequantize_mx(e_ref, s_ref, rows, cols, fmt)
+    d = bf16_bits(mx.dequantize(q, layout))
+    assert nan_aware_equal(d.reshape(-1), ref.reshape(-1))
+
+
 # ------------------------------------------------------------------ full-size workloads
 def test_mx8_rowwise_1024x1024_full(oracle):
     x = synth.mx8_rowwise()
