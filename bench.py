@@ -527,6 +527,23 @@ def run_breakdown(mx, dev, pk, cpu=False):
                                  "nvfp4_GBps": round(bdn / tn / 1e6, 1), "nvfp4_frac_hbm": round(bdn / tn / 1e6 / hbm, 4)}
     del xw, q4, qn, ys
 
+    # dequantise the 16384 x 4096 activations (MXFP8 E4M3, MXFP4, NVFP4; tcgen05 scales):
+    # codes + scales in, 128 MiB of bf16 out, each call larger than L2
+    xa = to_dev(synth.activations(), dev)
+    ya = torch.empty_like(xa)
+    RA, CA = xa.shape
+    da = {}
+    for fmt, rnd, bpe, blk in (("e4m3", "ceil", 1.0, 32), ("e2m1", "floor", 0.5, 32), ("nvfp4", "ceil", 0.5, 16)):
+        q = mx.quantize(xa, fmt, "row", rnd, layout="tcgen05")
+        t = timed([lambda q=q: mx.dequantize(q, "tcgen05", out=ya)], 20, stream)
+        nb = int(RA * CA * bpe) + RA * CA // blk + (4 if fmt == "nvfp4" else 0) + RA * CA * 2
+        da[fmt + "_us"] = round(t * 1e3, 2)
+        da[fmt + "_GBps"] = round(nb / t / 1e6, 1)
+        da[fmt + "_frac_hbm"] = round(nb / t / 1e6 / hbm, 4)
+        del q
+    out["dequantize_16384x4096"] = da
+    del xa, ya
+
     # the 4096 x 4096 weight: MXFP4 (floor) and NVFP4, both scale layouts, each call on
     # eight rotating copies (256 MiB > L2); one step = both calls
     xw0 = to_dev(synth.weight_fp4(), dev)
@@ -846,6 +863,12 @@ def run_case(name, iters, dev):
         qn = mx.quantize(xw, "nvfp4", "row", "ceil", layout="tcgen05")
         y = torch.empty_like(xw)
         fns = [lambda: (mx.dequantize(q4, "tcgen05", out=y), mx.dequantize(qn, "tcgen05", out=y))]
+    elif name == "dequant_act":
+        xa = to_dev(synth.activations(), dev)
+        qs = [mx.quantize(xa, f, "row", r, layout="tcgen05") for f, r in (("e4m3", "ceil"), ("e2m1", "floor"),
+                                                                           ("nvfp4", "ceil"))]
+        y = torch.empty_like(xa)
+        fns = [lambda: [mx.dequantize(q, "tcgen05", out=y) for q in qs]]
     elif name in ("gemm_mxfp4_8192", "gemm_nvfp4_8192"):
         fmt = "e2m1" if name == "gemm_mxfp4_8192" else "nvfp4"
         a = mx.quantize(to_dev(synth.normal(8192, 8192, seed=60), dev), fmt, "row", "floor", layout="tcgen05")
@@ -904,7 +927,8 @@ def run_case(name, iters, dev):
     print(f"{name}: {iters} calls, {t * 1e3:.1f} us per call", flush=True)
 
 
-CASES = ["step", "weight4096", "weight4096_one_call", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "gemm8192", "gemm_w4a8",
+CASES = ["step", "weight4096", "weight4096_one_call", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "dequant_act",
+         "gemm8192", "gemm_w4a8",
          "gemm_mxfp4_8192", "gemm_nvfp4_8192", "gemm_cmp", "extended"]
 
 
