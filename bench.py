@@ -295,16 +295,7 @@ def run_ours(args, rank, world, dev):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (numpy default_rng; activations seed = rank, gradients seed = rank + 1)",
-                "config": {"workload": WORKLOAD,
-                           "tensors": {"activations": {"shape": list(ACT), "format": "MXFP8 E4M3",
-                                                       "bytes": BYTES_ACT},
-                                       "gradients": {"shape": list(GRAD), "format": "MXFP8 E5M2",
-                                                     "bytes": BYTES_GRAD}},
-                           "orientations": "row-wise and column-wise (transposed) from one read",
-                           "scale_rule": "no-clip (ceil), E8M0, block 32", "scale_layout": "tcgen05",
-                           "step_bytes": STEP_BYTES,
-                           "l2": "inputs larger than L2 (604 MB per step), no flush needed",
-                           "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                "config": step_config(world),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": step_launches(args.steps), "clocks": clk.summary()}
         if breakdown is not None:
@@ -803,6 +794,18 @@ def gemm_cpu_baseline(shape, afmt, bfmt, bsig, target_s=6.0):
             "sample": f"{done} entries of C ({len(pairs)} distinct, K = {K}), fp64, {dt:.1f} s on {workers} threads"}
 
 
+def step_config(world):
+    """The headline workload's description, the same in both arms' lines."""
+    return {"workload": WORKLOAD,
+            "tensors": {"activations": {"shape": list(ACT), "format": "MXFP8 E4M3", "bytes": BYTES_ACT},
+                        "gradients": {"shape": list(GRAD), "format": "MXFP8 E5M2", "bytes": BYTES_GRAD}},
+            "orientations": "row-wise and column-wise (transposed) from one read",
+            "scale_rule": "no-clip (ceil), E8M0, block 32", "scale_layout": "tcgen05",
+            "step_bytes": STEP_BYTES,
+            "l2": "inputs larger than L2 (604 MB per step), no flush needed",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
 def run_reference(args, rank, world):
     """The oracle as the reference arm: rank 0 only, a bounded sample per step."""
     if rank != 0:
@@ -823,7 +826,7 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(secs), 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic (numpy default_rng; activations seed 0, gradients seed 1)",
-            "config": {"workload": WORKLOAD, "step_bytes": STEP_BYTES},
+            "config": step_config(world),
             "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample, "value": round(v, 5)},
             "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
