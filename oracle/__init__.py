@@ -11,9 +11,10 @@ shared object with gcc when it is missing.
 Every function's definition and the passage it follows are documented in ``mx_oracle.c``.
 Parity status: every function here is pinned by the ``-m "not gpu"`` oracle tests, the
 NVFP4 element step (the E2M1 code of the fp32 quotient x / d) exhaustively against
-numpy's IEEE division and an exact nearest-code search.  The tcgen05 scale tiling is
-parity unpinned on the CPU (the pages do not define it; it is pinned on hardware by the
-block-scaled matmul and by cuBLASLt's MXFP8 matmul reading the same scale bytes).
+numpy's IEEE division and an exact nearest-code search.  The tcgen05 scale tiling, which
+the pages do not define, is pinned on the CPU against vLLM's implementation of the
+block-scaling-factor layout cuBLAS documents, and on hardware by the block-scaled matmul
+and by cuBLASLt's MXFP8 matmul reading the same scale bytes.
 """
 from __future__ import annotations
 
