@@ -91,20 +91,30 @@ mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__r
     for (int t = 0; t < 2; t++) {
         const int d = (int)sc[t] - 127 - smax + 6;                // tile exponent relative to S
         exact = exact && (sc[t] == 0xFFu || tile_exact(d, &w[4 * t]));
-        // 2^d as fp32 (0 below 2^-149, where every product encodes to 0 anyway; capped at
-        // 2^126, reached only by tiles whose codes are all zero)
-        const int dc = d > 126 ? 126 : d;
-        const float f = dc >= -126 ? __uint_as_float((uint32_t)(dc + 127) << 23)
-                                   : (dc >= -149 ? __uint_as_float(1u << (dc + 149)) : 0.0f);
+        // 2^d as an f16 pair, exact for -24 <= d <= 6 (f16 subnormals below 2^-14); 0 below
+        // 2^-24, where every product (at most 6 * 2^-25) encodes to E4M3 zero anyway; capped
+        // at 2^6, which larger d reach only for tiles whose codes are all zero.  An E2M1 value
+        // has at most 2 significant bits, so every product that can encode to a nonzero E4M3
+        // code (>= 2^-10) is exact in f16, and the smaller ones encode to a zero of the same
+        // sign through f16 as through fp32: the codes are the fp32 path's, with one packed
+        // f16 product and one packed conversion per element pair.
+        const int dh = d > 6 ? 6 : d;
+        const uint32_t fb = dh >= -14 ? (uint32_t)(dh + 15) << 10 : (dh >= -24 ? 1u << (dh + 24) : 0u);
+        const uint32_t f2 = fb | (fb << 16);
 #pragma unroll
         for (int k = 0; k < 4; k++) {                             // 8 codes per word
-            float y[8];
-            e2m1x8_to_f32(w[4 * t + k], y);
+            uint32_t h[4], c[4];
+            e2m1x8_to_f16x2(w[4 * t + k], h);
 #pragma unroll
-            for (int i = 0; i < 8; i++) y[i] = __fmul_rn(y[i], f);
-            const uint2 q = cvt_fp8x8<FMT_E4M3>(y);
-            o[8 * t + 2 * k] = sc[t] == 0xFFu ? 0x7F7F7F7Fu : q.x;    // NaN tile: E4M3 NaN
-            o[8 * t + 2 * k + 1] = sc[t] == 0xFFu ? 0x7F7F7F7Fu : q.y;
+            for (int i = 0; i < 4; i++) {
+                uint32_t p;
+                uint16_t q2;
+                asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p) : "r"(h[i]), "r"(f2));
+                asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(q2) : "r"(p));
+                c[i] = q2;
+            }
+            o[8 * t + 2 * k] = sc[t] == 0xFFu ? 0x7F7F7F7Fu : (c[0] | (c[1] << 16));    // NaN tile: E4M3 NaN
+            o[8 * t + 2 * k + 1] = sc[t] == 0xFFu ? 0x7F7F7F7Fu : (c[2] | (c[3] << 16));
         }
     }
     uint4 *dst = reinterpret_cast<uint4 *>(out + R * cols + c0);
