@@ -61,8 +61,8 @@ WORKLOAD = "dual_mxfp8_act_16384x4096_e4m3_and_grad_16384x14336_e5m2_tcgen05_sca
 # capture of the benchmark's own back-to-back sequence (no cache control, no clock
 # control), and the SHA-256 of the kernel source that capture ran: when dual.cu has
 # changed since, the traffic is reported as null.
-NCU_TRAFFIC_GRAD = 955429547      # mean of 3 launches: read ~469.86 MB + write ~485.57 MB
-NCU_TRAFFIC_SRC_SHA = "4016d5c75a5aca8215a7468d27bf3cac2d3800e9b1cbad20f510c165b58de969"
+NCU_TRAFFIC_GRAD = 955400107      # mean of 3 launches: read ~469.88 MB + write ~485.52 MB
+NCU_TRAFFIC_SRC_SHA = "d3e0aad265bfe978daae80f6618d0c20056e6cd34940c0736dbd8f49b43c169a"
 DUAL_SRC = os.path.join(ROOT, "microscaling_precision_number_b200", "csrc", "dual.cu")
 
 # the 4096 x 4096 weight: MXFP4 (floor) + NVFP4, both scale layouts (a breakdown row)

@@ -11,7 +11,8 @@
 // Design:
 //   - persistent CTAs, one per SM, walk 32-row x 256-column bf16 tiles.  A producer warp
 //     loads each tile as four 32 x 64 boxes (2-D TMA, 128-byte swizzle) into a 7-stage
-//     ring (112 KiB in flight per SM) guarded by full / empty mbarriers.  Measured on the
+//     ring (112 KiB in flight per SM; 8 stages for the column-only form, see kStagesOf)
+//     guarded by full / empty mbarriers.  Measured on the
 //     16384 x 4096 and 16384 x 14336 inputs, 7 stages beat both shallower (4, 6) and
 //     deeper rings (8, 10, 12, 13), and one CTA per SM beat two or three CTAs with
 //     shallower rings;
@@ -42,11 +43,18 @@ constexpr int kBoxes = 4;
 constexpr int kTileR = 32, kTileC = kBoxC * kBoxes;  // 32 x 256 tile
 constexpr int kBoxBytes = kTileR * kBoxC * 2;        // 4 KiB
 constexpr int kTileBytes = kBoxBytes * kBoxes;       // 16 KiB
-constexpr int kStages = 7;
+// Ring depth: 7 stages when both orientations are written (every consumer warp takes every
+// tile), 8 when only the column-wise output is (the two warp groups take alternate tiles).
+// With alternating groups the depth must be even: each stage then belongs to one group,
+// whose waits on it follow its phases one by one.  With an odd depth a group's next use of
+// a stage is two phases after its last one, and a parity wait cannot tell "two phases on"
+// from "the phase the other group is still waiting for": it would pass early.
+template <bool ROW> constexpr int kStagesOf = ROW ? 7 : 8;
+constexpr int kMaxStages = 8;
 constexpr int kProducerWarp = 8;
 constexpr int kDualThreads = 32 * (kProducerWarp + 1);
 constexpr int kCtasPerSm = 1;
-constexpr size_t kDualSmem = (size_t)kStages * kTileBytes + 1024;   // + alignment to 1024
+template <bool ROW> constexpr size_t kDualSmem = (size_t)kStagesOf<ROW> * kTileBytes + 1024;   // + alignment
 }  // namespace
 
 // 32 bytes at p (w, or zeros when `zero`): one 256-bit store when p is 32-byte aligned,
@@ -241,7 +249,9 @@ quant_dual_kernel(const __grid_constant__ CUtensorMap tmap, uint32_t rows, uint3
                   uint8_t *__restrict__ col_elems, ScaleOut col_sc, int v8, int *watchdog) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ __align__(8) uint64_t full[kStages], empty[kStages];
+    constexpr int kStages = kStagesOf<ROW>;
+    static_assert(ROW || kStages % 2 == 0, "alternating consumer groups need an even ring depth");
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
 
     const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t G = gridDim.x;
@@ -329,12 +339,12 @@ static cudaError_t launch_dual_k(const CUtensorMap &tm, int grid, uint32_t rows,
                                  TileOrder order, uint8_t *re, const ScaleOut &rs, uint8_t *ce, const ScaleOut &cs,
                                  int v8, int *wd, cudaStream_t st) {
     auto k = quant_dual_kernel<FMT, CEIL, ROW, RM, TC>;
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDualSmem);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDualSmem<ROW>);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kDualThreads);
-    cfg.dynamicSmemBytes = kDualSmem;
+    cfg.dynamicSmemBytes = kDualSmem<ROW>;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

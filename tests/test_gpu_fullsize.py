@@ -84,6 +84,23 @@ def test_colwise_16384x4096_every_byte(oracle, fmt, rounding):
     assert np.array_equal(host(q.scales_alt), oracle.to_tcgen05_layout(s))
 
 
+def test_colwise_gradients_back_to_back(oracle):
+    """Column-wise only on the 16384 x 14336 gradients (E5M2, tcgen05 scales), launched 12
+    times back to back into separate outputs: the two consumer warp groups take alternate
+    ring tiles there, so each launch must equal the oracle (launch-to-launch timing must not
+    change a byte)."""
+    x = synth.gradients()
+    xd = to_dev(x)
+    outs = [mx.quantize(xd, "e5m2", "col", "ceil", layout="tcgen05") for _ in range(12)]
+    torch.cuda.synchronize()
+    e, s = quantize_mx_rows(oracle, np.ascontiguousarray(x.T), 1, oracle.CEIL)
+    assert np.array_equal(host(outs[0].elems), e.reshape(-1))
+    assert np.array_equal(host(outs[0].scales), oracle.to_tcgen05_layout(s))
+    for q in outs[1:]:
+        assert torch.equal(q.elems, outs[0].elems)
+        assert torch.equal(q.scales, outs[0].scales)
+
+
 def _check(got, ref, mag, where):
     err = np.abs(got - ref)
     bad = np.nonzero(~(err <= gemm_tolerance(ref, mag)))
