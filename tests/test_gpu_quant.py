@@ -130,6 +130,32 @@ def test_quantize_colwise_matches_oracle(oracle, shape, fmt, rounding):
     assert np.array_equal(host(q.scales_alt), oracle.to_tcgen05_layout(s_ref))
 
 
+@pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (1, "floor"), (2, "floor"), (4, "ceil"), (5, "floor"),
+                                          (6, "ceil")])
+def test_colwise_and_dual_many_tiles_per_cta(oracle, fmt, rounding):
+    """The TMA-staged kernel on shapes with several ring tiles per CTA and a ragged last
+    column tile inside a narrower last band: column-only (two warp groups on alternate
+    tiles, 2048 x 2312: a last tile 8 columns wide) and both orientations (2048 x 2336: a
+    last tile 32 columns wide), both scale layouts."""
+    rnd = oracle.CEIL if rounding == "ceil" else oracle.FLOOR
+    x = with_specials(synth.gradients(2048, 2312, seed=40 + fmt), seed=fmt)
+    q = mx.quantize(to_dev(x), FMT_NAMES[fmt], "col", rounding, layout="both")
+    e_ref, s_ref = oracle.quantize_mx(x, fmt, oracle.COL, rnd)
+    assert np.array_equal(host(q.elems), e_ref.reshape(-1))
+    assert np.array_equal(host(q.scales), s_ref.reshape(-1))
+    assert np.array_equal(host(q.scales_alt), oracle.to_tcgen05_layout(s_ref))
+    x = with_specials(synth.gradients(2048, 2336, seed=50 + fmt), seed=fmt)
+    qr, qc = mx.quantize_dual(to_dev(x), FMT_NAMES[fmt], rounding, "both")
+    er, sr = oracle.quantize_mx(x, fmt, oracle.ROW, rnd)
+    ec, sc = oracle.quantize_mx(x, fmt, oracle.COL, rnd)
+    assert np.array_equal(host(qr.elems), er.reshape(-1))
+    assert np.array_equal(host(qr.scales), sr.reshape(-1))
+    assert np.array_equal(host(qr.scales_alt), oracle.to_tcgen05_layout(sr))
+    assert np.array_equal(host(qc.elems), ec.reshape(-1))
+    assert np.array_equal(host(qc.scales), sc.reshape(-1))
+    assert np.array_equal(host(qc.scales_alt), oracle.to_tcgen05_layout(sc))
+
+
 @pytest.mark.parametrize("shape", [(32, 32), (64, 160), (160, 384), (256, 1024)])
 @pytest.mark.parametrize("fmt,rounding", [(0, "ceil"), (1, "ceil"), (1, "floor"), (2, "floor"), (4, "floor"),
                                           (5, "ceil"), (6, "floor"), (6, "ceil")])
