@@ -649,6 +649,15 @@ def run_breakdown(mx, dev, pk, cpu=False):
         out[name] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1), "frac_hbm": round(nb / t / 1e6 / hbm, 4),
                      "algorithmic_bytes": nb}
         del q
+    # row-wise MXFP8 (E4M3) and column-wise-only MXFP8 of the same activations (the
+    # transposed output alone: mx_quantize with axis = COL), tcgen05 scales
+    for name, axis in (("quant_mxfp8_rowwise_16384x4096", "row"), ("quant_mxfp8_colwise_16384x4096", "col")):
+        q = mx.quantize(x3, "e4m3", axis, "ceil", layout="tcgen05")
+        t = timed([lambda q=q, axis=axis: mx.quantize(x3, "e4m3", axis, "ceil", layout="tcgen05", out=q)], 20, stream)
+        nb = R * C * 2 + R * C + R * C // 32
+        out[name] = {"ms": round(t, 4), "GBps": round(nb / t / 1e6, 1), "frac_hbm": round(nb / t / 1e6 / hbm, 4),
+                     "algorithmic_bytes": nb}
+        del q
     del x3
 
     # nested blocks -- the 14336 x 4096 MXFP4 weight re-expressed as
