@@ -875,6 +875,13 @@ def run_case(name, iters, dev):
         qn = mx.quantize(xw, "nvfp4", "row", "ceil", layout="tcgen05")
         y = torch.empty_like(xw)
         fns = [lambda: (mx.dequantize(q4, "tcgen05", out=y), mx.dequantize(qn, "tcgen05", out=y))]
+    elif name == "quant_act":
+        # row-wise and column-wise-only MXFP8 (E4M3, no-clip, tcgen05 scales) of the activations
+        xa = to_dev(synth.activations(), dev)
+        qr = mx.quantize(xa, "e4m3", "row", "ceil", layout="tcgen05")
+        qc = mx.quantize(xa, "e4m3", "col", "ceil", layout="tcgen05")
+        fns = [lambda: (mx.quantize(xa, "e4m3", "row", "ceil", layout="tcgen05", out=qr),
+                        mx.quantize(xa, "e4m3", "col", "ceil", layout="tcgen05", out=qc))]
     elif name == "dequant_act":
         xa = to_dev(synth.activations(), dev)
         qs = [mx.quantize(xa, f, "row", r, layout="tcgen05") for f, r in (("e4m3", "ceil"), ("e2m1", "floor"),
@@ -940,6 +947,7 @@ def run_case(name, iters, dev):
 
 
 CASES = ["step", "weight4096", "weight4096_one_call", "mx8_1024", "dual_act", "dual_grad", "dequant4096", "dequant_act",
+         "quant_act",
          "gemm8192", "gemm_w4a8",
          "gemm_mxfp4_8192", "gemm_nvfp4_8192", "gemm_cmp", "extended"]
 

@@ -12,7 +12,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
 // Watchdog codes (what timed out).
 enum : int { WD_DUAL_FULL = 1, WD_GEMM_FULL = 2, WD_GEMM_EMPTY = 3, WD_GEMM_ACC = 4, WD_GEMM_DRAIN = 5,
-             WD_STREAM_FULL = 6, WD_DUAL_EMPTY = 8, WD_SELFTEST = 9 };
+             WD_STREAM_FULL = 6, WD_STREAM_EMPTY = 7, WD_DUAL_EMPTY = 8, WD_SELFTEST = 9 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

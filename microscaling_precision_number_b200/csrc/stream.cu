@@ -82,14 +82,25 @@ __device__ __forceinline__ void pdl_wait_and_release() {
 // runs in every thread once the first kStages copies are in flight and before the first
 // tile is consumed (a kernel that must wait for its predecessor's results, but not for its
 // input, waits there so that its first loads overlap the predecessor's tail).
+// A stage is refilled once every warp is done with it.  By default the CTA synchronises
+// after each tile and thread 0 refills at once.  With WARP_RELEASE each warp releases the
+// stage on an "empty" barrier (ring.full holds kStages full barriers, then kStages empty
+// ones) and thread 0 waits for the release, so only warp 0 waits for the slowest warp and
+// the others run on into stages already loaded: measured 5-7% faster for the dequantisers
+// (their warps drift with the store traffic) but 3-7% slower for the quantisers, where the
+// refill then comes later than after a hardware barrier.
 struct NoPrologue {
     __device__ __forceinline__ void operator()() const {}
 };
-template <typename Body, typename Prologue = NoPrologue>
+template <bool WARP_RELEASE = false, typename Body, typename Prologue = NoPrologue>
 __device__ __forceinline__ void stream_tiles(Ring &ring, uint32_t n_tiles, Body body, Prologue after_issue = {}) {
     const int tid = threadIdx.x;
+    uint64_t *empty = ring.full + kStages;
     if (tid == 0) {
-        for (int s = 0; s < kStages; s++) mbar_init(&ring.full[s], 1);
+        for (int s = 0; s < kStages; s++) {
+            mbar_init(&ring.full[s], 1);
+            if constexpr (WARP_RELEASE) mbar_init(&empty[s], kThreads / 32);
+        }
         fence_barrier_init();
     }
     __syncthreads();
@@ -107,10 +118,18 @@ __device__ __forceinline__ void stream_tiles(Ring &ring, uint32_t n_tiles, Body 
         // warp-uniform outcome (bodies may use full-warp shuffles)
         const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&ring.full[s], phase, ring.watchdog, WD_STREAM_FULL));
         if (ok) body(t, ring.buf + s * kTileBytes);
-        __syncthreads();                                   // stage s is free again
-        if (tid == 0) {
-            const uint32_t tn = t + (uint32_t)kStages * gridDim.x;
-            if (tn < n_tiles && *reinterpret_cast<volatile int *>(ring.watchdog) == 0) {
+        const uint32_t tn = t + (uint32_t)kStages * gridDim.x;
+        if constexpr (WARP_RELEASE) {
+            __syncwarp();
+            if ((tid & 31) == 0) mbar_arrive(&empty[s]);   // this warp is done with stage s
+            if (tid == 0 && tn < n_tiles && *reinterpret_cast<volatile int *>(ring.watchdog) == 0 &&
+                mbar_wait_bounded(&empty[s], phase, ring.watchdog, WD_STREAM_EMPTY)) {
+                ring.issue(tn, s);
+                issued++;
+            }
+        } else {
+            __syncthreads();                               // stage s is free again
+            if (tid == 0 && tn < n_tiles && *reinterpret_cast<volatile int *>(ring.watchdog) == 0) {
                 ring.issue(tn, s);
                 issued++;
             }
@@ -121,6 +140,7 @@ __device__ __forceinline__ void stream_tiles(Ring &ring, uint32_t n_tiles, Body 
         for (uint32_t j = it; j < issued; j++)
             (void)mbar_wait_bounded(&ring.full[j % kStages], (j / kStages) & 1u, nullptr, 0, kDrainLimitNs);
     }
+    if constexpr (WARP_RELEASE) __syncthreads();           // warps leave the loop together
 }
 
 // |x| maximum (15-bit bf16 magnitude; NaN anywhere gives >= 0x7F80) of a 32-element block
@@ -173,7 +193,7 @@ mx_rows_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS,
                float *__restrict__ partials, int *watchdog) {
     pdl_wait_and_release();
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ __align__(8) uint64_t full[2 * kStages];   // full, then empty barriers
     __shared__ uint32_t warp_u[kThreads / 32];
     Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
               full, watchdog, src, kTileBytes, (uint64_t)n_blocks * 64};
@@ -404,7 +424,7 @@ nvfp4_amax_bulk_kernel(const uint8_t *__restrict__ src, uint64_t n_bytes, float 
                        int *watchdog) {
     pdl_wait_and_release();
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ __align__(8) uint64_t full[2 * kStages];   // full, then empty barriers
     __shared__ uint32_t warp_u[kThreads / 32];
     Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
               full, watchdog, src, kTileBytes, n_bytes};
@@ -424,7 +444,7 @@ nvfp4_quant_bulk_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fast
                         uint8_t *__restrict__ elems, uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc,
                         int *watchdog) {
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ __align__(8) uint64_t full[2 * kStages];   // full, then empty barriers
     __shared__ float warp_max[kThreads / 32];
     Ring ring{reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127)),
               full, watchdog, src, kTileBytes, (uint64_t)n_blocks * 32};
@@ -534,7 +554,7 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
                        int *watchdog) {
     pdl_wait_and_release();
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ __align__(8) uint64_t full[2 * kStages];   // full, then empty barriers
     constexpr uint32_t kCodeBytes = 32 * code_bits(FMT) / 8;              // per block: 16, 24 or 32
     constexpr uint32_t kBlocksPerTile = kThreads;                          // one per thread
     // Bulk copies move whole 16-byte units; with FP6 (24 bytes a block) and an odd block
@@ -557,7 +577,7 @@ dequant_mx_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restr
         }
     };
     uint32_t s_next = scale_of(blockIdx.x);
-    stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
+    stream_tiles<true>(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
         const uint32_t blk = t * kBlocksPerTile + tid;
         const uint32_t s = s_next;
         s_next = scale_of(t + gridDim.x);
@@ -617,7 +637,7 @@ dequant_nvfp4_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__re
                           uint4 *__restrict__ out, int *watchdog) {
     pdl_wait_and_release();
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[kStages];
+    __shared__ __align__(8) uint64_t full[2 * kStages];   // full, then empty barriers
     constexpr uint32_t kBlocksPerTile = 2 * kThreads;                      // 8 code bytes each
     // Bulk copies move whole 16-byte units (block pairs); with an odd block count the
     // last block's 8 code bytes are read straight from global memory by its thread.
@@ -645,7 +665,7 @@ dequant_nvfp4_bulk_kernel(const uint8_t *__restrict__ elems, const uint8_t *__re
     };
     uint32_t sc_next[2];
     scales_of(blockIdx.x, sc_next);
-    stream_tiles(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
+    stream_tiles<true>(ring, n_tiles, [&](uint32_t t, const uint8_t *tile) {
         // this thread's two blocks' UE4M3 scales as f16x2 words holding dec(sb) twice (0 past
         // the end; code 0x7F decodes to NaN).  dec(q) dec(sb) is exact in f16: at most 6
         // significant bits, magnitudes 2^-10 .. 2688, so the packed f16 product equals the
