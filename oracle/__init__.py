@@ -11,7 +11,10 @@ shared object with gcc when it is missing.
 Every function's definition and the passage it follows are documented in ``mx_oracle.c``.
 Parity status: every function here is pinned by the ``-m "not gpu"`` oracle tests, the
 NVFP4 element step (the E2M1 code of the fp32 quotient x / d) exhaustively against
-numpy's IEEE division and an exact nearest-code search.  The tcgen05 scale tiling, which
+numpy's IEEE division and an exact nearest-code search, and the whole NVFP4 quantiser
+against vLLM's torch reference quantiser (equal codes except one-step differences at
+rounding midpoints, where the two place their fp32 roundings differently).  The tcgen05
+scale tiling, which
 the pages do not define, is pinned on the CPU against vLLM's implementation of the
 block-scaling-factor layout cuBLAS documents, and on hardware by the block-scaled matmul
 and by cuBLASLt's MXFP8 matmul reading the same scale bytes.
