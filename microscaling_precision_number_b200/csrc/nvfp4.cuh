@@ -47,4 +47,42 @@ __device__ __forceinline__ void nvfp4_codes16(const uint4 &v0, const uint4 &v1, 
     q1 = cvt_e2m1x8(x[1]) ^ 0x88888888u;
 }
 
+// Per-tensor constants of the NVFP4 block math, derived once per CTA from g.
+struct Nvfp4Consts {
+    float six_g;      // 6 g (fp32 RN)
+    float y;          // RN(1 / six_g)
+    bool fast;        // six_g >= 2^-80: t = amax_b / six_g may use the corrected quotient
+};
+
+// Per-code element divisors: qtab[sb] = {d, -RN(1/d)} with d = RN(dec(sb) g).  The second
+// entry is 0 when d < 2^-100 (the quotients then take the IEEE division) and the code 0x7F
+// (only NaN blocks, whose codes are zero) gets {0, 0}.
+__device__ __forceinline__ Nvfp4Consts nvfp4_consts(float g, float2 *qtab) {
+    Nvfp4Consts c;
+    c.six_g = __fmul_rn(6.0f, g);
+    c.y = __frcp_rn(c.six_g);
+    c.fast = c.six_g >= 0x1p-80f;
+    if (threadIdx.x < 128) {
+        const float d = threadIdx.x < 0x7Fu ? __fmul_rn(ue4m3_to_f32(threadIdx.x), g) : 0.0f;
+        qtab[threadIdx.x] = make_float2(d, d >= kQuotFastMin ? -__frcp_rn(d) : 0.0f);
+    }
+    __syncthreads();
+    return c;
+}
+
+// RN(amax_b / six_g): with FAST, Markstein's corrected quotient from the precomputed
+// reciprocal (q0 = RN(a y), r = a - q0 six_g exact by FMA, t = RN(q0 + r y)).  It is the
+// IEEE quotient for every numerator a >= 2^-100; with six_g >= 2^-80 every block whose
+// quotient can reach the smallest UE4M3 subnormal has such a numerator, and smaller
+// quotients encode to 0 either way.  Otherwise the IEEE division.
+template <bool FAST>
+__device__ __forceinline__ float nvfp4_block_quotient(float a, const Nvfp4Consts &cst) {
+    if constexpr (FAST) {
+        const float q0 = __fmul_rn(a, cst.y);
+        return __fmaf_rn(__fmaf_rn(-q0, cst.six_g, a), cst.y, q0);
+    } else {
+        return __fdiv_rn(a, cst.six_g);
+    }
+}
+
 }  // namespace mxk

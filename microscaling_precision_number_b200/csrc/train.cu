@@ -57,62 +57,100 @@ __device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
     return d;
 }
 
-// The butterfly stages with strides 1, 2 and 4 run on packed pairs P[j] = (v[j], v[j + 8]):
-// both lanes of P[j] +- P[j + h] are stride-h butterflies, so each packed add / sub does two
-// of them with the scalar rounding.  The stride-8 stage pairs the two lanes of one register
-// and runs in scalar; then x 1/4 (exact) and the bf16 rounding.
-__device__ __forceinline__ void rht16(uint4 &v0, uint4 &v1, const RhtSigns &sm) {
-    const uint32_t a[4] = {v0.x ^ sm.w[0], v0.y ^ sm.w[1], v0.z ^ sm.w[2], v0.w ^ sm.w[3]};   // elements 0-7
-    const uint32_t b[4] = {v1.x ^ sm.w[4], v1.y ^ sm.w[5], v1.z ^ sm.w[6], v1.w ^ sm.w[7]};   // elements 8-15
-    uint64_t P[8];
+// The transform runs on two groups at once (a: one group's elements 0-7 and 8-15, b:
+// another's): lane 0 of every packed fp32 pair holds group a, lane 1 group b, so all four
+// butterfly stages (x_j, x_j+h) <- (x_j + x_j+h, x_j - x_j+h) for h = 1, 2, 4, 8 and the
+// x 1/4 run as packed pairs, each lane with the scalar round-to-nearest of one group.
+__device__ __forceinline__ void rht16x2_stages(const uint4 &a0, const uint4 &a1, const uint4 &b0, const uint4 &b1,
+                                               const RhtSigns &sm, uint64_t (&Q)[16]) {
+    const uint32_t wa[8] = {a0.x ^ sm.w[0], a0.y ^ sm.w[1], a0.z ^ sm.w[2], a0.w ^ sm.w[3],
+                            a1.x ^ sm.w[4], a1.y ^ sm.w[5], a1.z ^ sm.w[6], a1.w ^ sm.w[7]};
+    const uint32_t wb[8] = {b0.x ^ sm.w[0], b0.y ^ sm.w[1], b0.z ^ sm.w[2], b0.w ^ sm.w[3],
+                            b1.x ^ sm.w[4], b1.y ^ sm.w[5], b1.z ^ sm.w[6], b1.w ^ sm.w[7]};
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-        P[2 * i] = pack2(bf16_lo(a[i]), bf16_lo(b[i]));
-        P[2 * i + 1] = pack2(bf16_hi(a[i]), bf16_hi(b[i]));
+    for (int i = 0; i < 8; i++) {
+        Q[2 * i] = pack2(bf16_lo(wa[i]), bf16_lo(wb[i]));
+        Q[2 * i + 1] = pack2(bf16_hi(wa[i]), bf16_hi(wb[i]));
     }
 #pragma unroll
-    for (int h = 1; h < 8; h <<= 1)
+    for (int h = 1; h < 16; h <<= 1)
 #pragma unroll
-        for (int j = 0; j < 8; j++)
+        for (int j = 0; j < 16; j++)
             if ((j & h) == 0) {
-                const uint64_t t = P[j];
-                P[j] = add2(t, P[j + h]);
-                P[j + h] = sub2(t, P[j + h]);
+                const uint64_t t = Q[j];
+                Q[j] = add2(t, Q[j + h]);
+                Q[j + h] = sub2(t, Q[j + h]);
             }
-    float v[16];
+}
+
+__device__ __forceinline__ void rht16x2(uint4 &a0, uint4 &a1, uint4 &b0, uint4 &b1, const RhtSigns &sm) {
+    uint64_t Q[16];
+    rht16x2_stages(a0, a1, b0, b1, sm, Q);
+    const uint64_t quarter = splat2(0.25f);
+    float A[16], B[16];
 #pragma unroll
-    for (int j = 0; j < 8; j++) {
-        float lo, hi;
-        unpack2(P[j], lo, hi);
-        v[j] = __fmul_rn(__fadd_rn(lo, hi), 0.25f);
-        v[j + 8] = __fmul_rn(__fsub_rn(lo, hi), 0.25f);
+    for (int j = 0; j < 16; j++) unpack2(mul2(Q[j], quarter), A[j], B[j]);
+    a0 = make_uint4(f32x2_to_bf16x2(A[0], A[1]), f32x2_to_bf16x2(A[2], A[3]), f32x2_to_bf16x2(A[4], A[5]),
+                    f32x2_to_bf16x2(A[6], A[7]));
+    a1 = make_uint4(f32x2_to_bf16x2(A[8], A[9]), f32x2_to_bf16x2(A[10], A[11]), f32x2_to_bf16x2(A[12], A[13]),
+                    f32x2_to_bf16x2(A[14], A[15]));
+    b0 = make_uint4(f32x2_to_bf16x2(B[0], B[1]), f32x2_to_bf16x2(B[2], B[3]), f32x2_to_bf16x2(B[4], B[5]),
+                    f32x2_to_bf16x2(B[6], B[7]));
+    b1 = make_uint4(f32x2_to_bf16x2(B[8], B[9]), f32x2_to_bf16x2(B[10], B[11]), f32x2_to_bf16x2(B[12], B[13]),
+                    f32x2_to_bf16x2(B[14], B[15]));
+}
+
+// Largest finite |y| over the two groups' butterfly outputs y, before the x 1/4.  The
+// transformed element is RN_bf16(y / 4): y / 4 is exact (y is a multiple of 2^-133, the
+// bf16 spacing at the bottom, and cannot overflow), and for finite y it stays finite in
+// bf16 (|y / 4| < 2^126).  Rounding is monotone, so the largest finite transformed
+// magnitude is RN_bf16(m / 4) with m the value returned here; NaNs drop out of fmaxf, and
+// an infinite y (an infinite input, or an fp32 overflow inside the butterfly) sends the
+// group pair down the rare path that skips it.
+__device__ __forceinline__ float rht16x2_absmax(const uint4 &a0, const uint4 &a1, const uint4 &b0, const uint4 &b1,
+                                                const RhtSigns &sm) {
+    uint64_t Q[16];
+    rht16x2_stages(a0, a1, b0, b1, sm, Q);
+    float y[32];
+#pragma unroll
+    for (int j = 0; j < 16; j++) unpack2(Q[j], y[2 * j], y[2 * j + 1]);
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 32; j++) m = fmaxf(m, fabsf(y[j]));
+    if (__builtin_expect(m == __int_as_float(0x7F800000), 0)) {
+        m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 32; j++)
+            if (fabsf(y[j]) != __int_as_float(0x7F800000)) m = fmaxf(m, fabsf(y[j]));
     }
-    v0 = make_uint4(f32x2_to_bf16x2(v[0], v[1]), f32x2_to_bf16x2(v[2], v[3]), f32x2_to_bf16x2(v[4], v[5]),
-                    f32x2_to_bf16x2(v[6], v[7]));
-    v1 = make_uint4(f32x2_to_bf16x2(v[8], v[9]), f32x2_to_bf16x2(v[10], v[11]), f32x2_to_bf16x2(v[12], v[13]),
-                    f32x2_to_bf16x2(v[14], v[15]));
+    return m;
 }
 
 // ---- stochastic rounding onto the element grid ----------------------------------------------
 // Returns the representable value (lo or hi, signed) that y rounds to with random byte r.
-// Branch-free: E = max(floor(log2 |y|), emin) is the binade whose grid step 2^(E - mbits)
-// applies (the format's subnormal step below its smallest normal exponent emin; fp32
-// subnormals and zero give emin); u = |y| 2^(mbits - E) is exact and counts grid steps, so
-// lo = trunc(u) steps and the fraction f = u - trunc(u) is exact, and y rounds up iff
-// 256 f > r -- the same test as 256 (|y| - lo) > r (hi - lo).
+// At or above the format's smallest normal 2^emin, the grid step of |y|'s binade is bit
+// w = 23 - mbits of its fp32 pattern, so the w low bits L are |y| - lo in units of 2^-w grid
+// steps, and 256 (|y| - lo) > r (hi - lo) reads L > r 2^(w - 8): exactly
+// when L + (2^w - 1 - r 2^(w - 8)) carries into bit w.  Adding that and clearing the w low
+// bits gives lo or hi (a carry out of the mantissa steps into the next binade, as the grid
+// does).  Below 2^emin the grid has the fixed subnormal step 2^(emin - mbits), which is also
+// the step of the binade [2^emin, 2^(emin + 1)]: |y| + 2^emin rounded toward +infinity lands
+// there, and rounding up to the next fp32 keeps the decision (L is then the ceiling of the
+// exact distance, compared strictly against an integer); subtracting 2^emin is exact.
+// |y| at or above the maximum saturates (Inf included); the sign is kept.
 template <int FMT>
 __device__ __forceinline__ float sr_value(float y, uint32_t r) {
     constexpr int mbits = FMT == FMT_E4M3 ? 3 : (FMT == FMT_E5M2 ? 2 : 1);
     constexpr int emin = FMT == FMT_E4M3 ? -6 : (FMT == FMT_E5M2 ? -14 : 0);   // smallest normal exponent
     constexpr float maxv = FMT == FMT_E4M3 ? 448.0f : (FMT == FMT_E5M2 ? 57344.0f : 6.0f);
+    constexpr uint32_t w = 23 - mbits, low = (1u << w) - 1u;
+    constexpr float minnorm = emin >= 0 ? (float)(1 << emin) : 1.0f / (float)(1 << -emin);
     const float a = fabsf(y);
-    const int E = max((int)(__float_as_uint(a) >> 23) - 127, emin);
-    const uint32_t k = (uint32_t)(E - mbits + 127);                // biased exponent of the step
-    const float u = __fmul_rn(a, __uint_as_float((254u - k) << 23)); // |y| / step (exact)
-    const float fl = truncf(u);
-    const bool up = __fmul_rn(__fsub_rn(u, fl), 256.0f) > (float)r;
-    const float v = __fmul_rn(up ? __fadd_rn(fl, 1.0f) : fl, __uint_as_float(k << 23));
-    return copysignf(a < maxv ? v : maxv, y);                      // at or above the maximum: saturate
+    const bool sub = a < minnorm;
+    const float ap = sub ? __fadd_ru(a, minnorm) : a;
+    float v = __uint_as_float((__float_as_uint(ap) + low - (r << (w - 8))) & ~low);
+    if (sub) v = __fsub_rn(v, minnorm);
+    return copysignf(fminf(v, maxv), y);
 }
 
 template <int FMT, bool SR>
@@ -136,10 +174,7 @@ mx_train_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS
     for (uint32_t blk = blockIdx.x * kTrainThreads + threadIdx.x; blk < n_blocks; blk += gridDim.x * kTrainThreads) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)blk * 64);
         uint4 v[4] = {p[0], p[1], p[2], p[3]};
-        if constexpr (RHT) {
-            rht16(v[0], v[1], sm);
-            rht16(v[2], v[3], sm);
-        }
+        if constexpr (RHT) rht16x2(v[0], v[1], v[2], v[3], sm);
         uint32_t a = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v[0].x, v[0].y), absmax_bf16x2(v[0].z, v[0].w)),
                                    absmax_bf16x2(absmax_bf16x2(v[1].x, v[1].y), absmax_bf16x2(v[1].z, v[1].w)));
         a = absmax_bf16x2(a, absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v[2].x, v[2].y), absmax_bf16x2(v[2].z, v[2].w)),
@@ -176,10 +211,11 @@ nvfp4_train_amax_kernel(const uint8_t *__restrict__ src, uint32_t n_groups, uint
                         float *__restrict__ partials) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     __shared__ uint32_t warp_u[kTrainThreads / 32];
-    uint32_t acc = 0;
+    uint32_t acc = 0;       // without the transform: bf16 magnitude bits, two lanes
+    float accf = 0.0f;      // with it: the largest finite butterfly output, before the x 1/4
     const RhtSigns sm = rht_signs(signs);
     // kUnroll groups per trip, all loads issued before the first transform
-    constexpr uint32_t kUnroll = 4;
+    constexpr uint32_t kUnroll = 2;
     const uint32_t stride = gridDim.x * kTrainThreads;
     uint32_t gi = blockIdx.x * kTrainThreads + threadIdx.x;
     for (; gi + (kUnroll - 1) * stride < n_groups; gi += kUnroll * stride) {
@@ -190,21 +226,31 @@ nvfp4_train_amax_kernel(const uint8_t *__restrict__ src, uint32_t n_groups, uint
             v[u][0] = p[0];
             v[u][1] = p[1];
         }
+        if constexpr (RHT) {
 #pragma unroll
-        for (uint32_t u = 0; u < kUnroll; u++) {
-            if constexpr (RHT) rht16(v[u][0], v[u][1], sm);
-            acc = __vmaxu2(acc, finite_abs_max_bf16x8(v[u][0]));
-            acc = __vmaxu2(acc, finite_abs_max_bf16x8(v[u][1]));
+            for (uint32_t u = 0; u < kUnroll; u += 2)
+                accf = fmaxf(accf, rht16x2_absmax(v[u][0], v[u][1], v[u + 1][0], v[u + 1][1], sm));
+        } else {
+#pragma unroll
+            for (uint32_t u = 0; u < kUnroll; u++) {
+                acc = __vmaxu2(acc, finite_abs_max_bf16x8(v[u][0]));
+                acc = __vmaxu2(acc, finite_abs_max_bf16x8(v[u][1]));
+            }
         }
     }
     for (; gi < n_groups; gi += stride) {
         const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)gi * 32);
-        uint4 v0 = p[0], v1 = p[1];
-        if constexpr (RHT) rht16(v0, v1, sm);
-        acc = __vmaxu2(acc, finite_abs_max_bf16x8(v0));
-        acc = __vmaxu2(acc, finite_abs_max_bf16x8(v1));
+        const uint4 v0 = p[0], v1 = p[1];
+        if constexpr (RHT) {
+            accf = fmaxf(accf, rht16x2_absmax(v0, v1, v0, v1, sm));   // one group, in both lanes
+        } else {
+            acc = __vmaxu2(acc, finite_abs_max_bf16x8(v0));
+            acc = __vmaxu2(acc, finite_abs_max_bf16x8(v1));
+        }
     }
-    uint32_t m = max(acc & 0xFFFFu, acc >> 16);
+    uint32_t m;
+    if constexpr (RHT) m = f32x2_to_bf16x2(__fmul_rn(accf, 0.25f), 0.0f) & 0xFFFFu;
+    else m = max(acc & 0xFFFFu, acc >> 16);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if ((threadIdx.x & 31) == 0) warp_u[threadIdx.x >> 5] = m;
@@ -217,9 +263,11 @@ nvfp4_train_amax_kernel(const uint8_t *__restrict__ src, uint32_t n_groups, uint
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Pass 2: g from the partial maxima, then one thread per 16-element block.  The block
-// scale and the quotient follow the RNE path's fp32 steps (t = amax_b / (6 g) and
-// RN(x / (dec(sb) g)), both correctly rounded); the element cast is RNE or stochastic.
+// Pass 2: g from the partial maxima, then two consecutive 16-element blocks per thread (so
+// the transform runs on both at once).  The block scale and the quotient follow the RNE
+// path's fp32 steps (t = amax_b / (6 g) and RN(x / (dec(sb) g)), both correctly rounded,
+// from the per-tensor constants and the per-code divisor table); the element cast is RNE or
+// stochastic.
 template <bool RM, bool TC, bool RHT, bool SR>
 __global__ void __launch_bounds__(kTrainThreads)
 nvfp4_train_quant_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, FastDiv divS, uint32_t col_atoms,
@@ -228,6 +276,7 @@ nvfp4_train_quant_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fas
                          uint8_t *__restrict__ sc_rm, uint8_t *__restrict__ sc_tc) {
     asm volatile("griddepcontrol.wait;" ::: "memory");
     __shared__ float red[kTrainThreads / 32];
+    __shared__ float2 qtab[128];
     float a = 0.0f;
     for (int i = threadIdx.x; i < n_partials; i += kTrainThreads) a = fmaxf(a, partials[i]);
 #pragma unroll
@@ -238,34 +287,55 @@ nvfp4_train_quant_kernel(const uint8_t *__restrict__ src, uint32_t n_blocks, Fas
     for (int w = 0; w < kTrainThreads / 32; w++) a = fmaxf(a, red[w]);
     const float g = a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f);
     if (blockIdx.x == 0 && threadIdx.x == 0) out_store(g_out, g);
-    const float six_g = __fmul_rn(6.0f, g);
+    const Nvfp4Consts cst = nvfp4_consts(g, qtab);
     const RhtSigns sm = rht_signs(signs);
-    for (uint32_t blk = blockIdx.x * kTrainThreads + threadIdx.x; blk < n_blocks; blk += gridDim.x * kTrainThreads) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)blk * 32);
-        uint4 v[2] = {p[0], p[1]};
-        if constexpr (RHT) rht16(v[0], v[1], sm);
-        const uint32_t am = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v[0].x, v[0].y), absmax_bf16x2(v[0].z, v[0].w)),
-                                          absmax_bf16x2(absmax_bf16x2(v[1].x, v[1].y), absmax_bf16x2(v[1].z, v[1].w)));
-        const uint32_t m = max(am & 0x7FFFu, (am >> 16) & 0x7FFFu);
-        const bool special = m >= 0x7F80u;
-        const float tq = __fdiv_rn(__uint_as_float(m << 16), six_g);
-        uint32_t sb = cvt_fp8x2<FMT_E4M3>(tq, 0.0f) & 0xFFu;
-        const float d = special ? 0.0f : __fmul_rn(ue4m3_to_f32(sb & 0x7Fu), g);
-        const float nr = d >= kQuotFastMin ? -__frcp_rn(d) : 0.0f;
-        const bool zero_codes = special || d == 0.0f;
-        if (special) sb = 0x7Fu;
-        uint32_t q[2];
-        const uint8_t *rb = rnd + (size_t)blk * 16;
-        // the quotients arrive negated; stochastic rounding is odd-symmetric, so it
-        // commutes with the sign flip applied to the codes
-        nvfp4_codes16(v[0], v[1], d, nr, q[0], q[1],
-                      [&](float (&x)[8], int j) { round8<FMT_E2M1, SR>(x, rb + 8 * j); });
-        if (zero_codes) q[0] = q[1] = 0u;
-        out_store(reinterpret_cast<uint2 *>(elems) + blk, make_uint2(q[0], q[1]));
-        if constexpr (RM) out_store(sc_rm + blk, (uint8_t)sb);
-        if constexpr (TC) {
-            const uint32_t rr = fdiv(blk, divS);
-            out_store(sc_tc + tc_offset(rr, blk - rr * divS.d, col_atoms), (uint8_t)sb);
+    const uint32_t n_pairs = (n_blocks + 1) / 2;
+    for (uint32_t pi = blockIdx.x * kTrainThreads + threadIdx.x; pi < n_pairs; pi += gridDim.x * kTrainThreads) {
+        const uint32_t blk0 = 2 * pi;
+        const bool two = blk0 + 1 < n_blocks;
+        const uint4 *p = reinterpret_cast<const uint4 *>(src + (size_t)blk0 * 32);
+        uint4 v[4];
+        v[0] = p[0];
+        v[1] = p[1];
+        v[2] = two ? p[2] : v[0];
+        v[3] = two ? p[3] : v[1];
+        if constexpr (RHT) rht16x2(v[0], v[1], v[2], v[3], sm);
+        uint32_t q[4], sbs[2];
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            const uint4 &v0 = v[2 * b], &v1 = v[2 * b + 1];
+            const uint32_t am = absmax_bf16x2(absmax_bf16x2(absmax_bf16x2(v0.x, v0.y), absmax_bf16x2(v0.z, v0.w)),
+                                              absmax_bf16x2(absmax_bf16x2(v1.x, v1.y), absmax_bf16x2(v1.z, v1.w)));
+            const uint32_t m = max(am & 0x7FFFu, (am >> 16) & 0x7FFFu);
+            const bool special = m >= 0x7F80u;
+            const float tq = cst.fast ? nvfp4_block_quotient<true>(__uint_as_float(m << 16), cst)
+                                      : nvfp4_block_quotient<false>(__uint_as_float(m << 16), cst);
+            uint32_t sb = cvt_fp8x2<FMT_E4M3>(tq, 0.0f) & 0x7Fu;
+            const float2 dn = qtab[sb];
+            const float d = special ? 0.0f : dn.x;
+            if (special) sb = 0x7Fu;
+            // the quotients arrive negated; stochastic rounding is odd-symmetric, so it
+            // commutes with the sign flip applied to the codes
+            const uint8_t *rb = rnd + (size_t)(blk0 + b) * 16;
+            nvfp4_codes16(v0, v1, d, dn.y, q[2 * b], q[2 * b + 1],
+                          [&](float (&x)[8], int j) { round8<FMT_E2M1, SR>(x, rb + 8 * j); });
+            if (special || d == 0.0f) q[2 * b] = q[2 * b + 1] = 0u;
+            sbs[b] = sb;
+        }
+        if (two) {
+            out_store(reinterpret_cast<uint4 *>(elems) + pi, make_uint4(q[0], q[1], q[2], q[3]));
+        } else {
+            out_store(reinterpret_cast<uint2 *>(elems) + blk0, make_uint2(q[0], q[1]));
+        }
+#pragma unroll
+        for (int b = 0; b < 2; b++) {
+            if (b == 1 && !two) break;
+            const uint32_t blk = blk0 + b;
+            if constexpr (RM) out_store(sc_rm + blk, (uint8_t)sbs[b]);
+            if constexpr (TC) {
+                const uint32_t rr = fdiv(blk, divS);
+                out_store(sc_tc + tc_offset(rr, blk - rr * divS.d, col_atoms), (uint8_t)sbs[b]);
+            }
         }
     }
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -321,7 +391,7 @@ static cudaError_t launch_nvfp4_train_t(const uint8_t *src, uint32_t nb, FastDiv
     if (grid1 > max_partials) grid1 = max_partials;
     cudaError_t err = launch_pdl(nvfp4_train_amax_kernel<RHT>, grid1, st, src, nb, signs, partials);
     if (err != cudaSuccess) return err;
-    const int grid2 = train_grid(nb, num_sms);
+    const int grid2 = train_grid((nb + 1) / 2, num_sms);
     const float *cp = partials;
     if (rm && tc)
         return launch_pdl(nvfp4_train_quant_kernel<true, true, RHT, SR>, grid2, st, src, nb, f, ca, signs, rnd, cp, grid1, g, e, rm, tc);

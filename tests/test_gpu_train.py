@@ -57,6 +57,65 @@ def test_train_quantiser_matches_oracle(oracle, fmt, rht, sr, shape):
     assert np.array_equal(q.scales_alt.cpu().numpy(), oracle.to_tcgen05_layout(s))
 
 
+@pytest.mark.parametrize("rht,sr", [(True, True), (False, True), (True, False)])
+@pytest.mark.parametrize("shape", [(33, 208), (1, 16), (3, 48)])
+def test_train_nvfp4_odd_block_count(oracle, rht, sr, shape):
+    """NVFP4 with an odd number of 16-element blocks (the quantisation pass takes two blocks
+    per thread; the last thread has one), row-major and tcgen05 scales."""
+    x = with_specials(synth.gradients(*shape, seed=shape[0] + 11), seed=shape[1] + 1)
+    rnd = np.random.default_rng(shape[1]).integers(0, 256, size=shape, dtype=np.uint8) if sr else None
+    signs = 0x5AC3 if rht else None
+    q = mx.quantize_train(to_dev(x), "nvfp4", "ceil", rht_signs=signs,
+                          sr_random=None if rnd is None else torch.from_numpy(rnd).cuda(), layout="both")
+    xt = oracle.rht16(x, signs) if rht else x
+    e, s, g = oracle.quantize_nvfp4_sr(xt, rnd) if sr else oracle.quantize_nvfp4(xt)
+    assert q.global_scale.cpu().numpy()[0] == np.float32(g)
+    assert np.array_equal(q.elems.cpu().numpy(), e.reshape(-1))
+    assert np.array_equal(q.scales.cpu().numpy(), s.reshape(-1))
+    assert np.array_equal(q.scales_alt.cpu().numpy(), oracle.to_tcgen05_layout(s))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "e2m1", "e4m3"])
+@pytest.mark.parametrize("sr", [False, True])
+def test_train_transform_nonfinite(oracle, fmt, sr):
+    """The transform meets Inf, NaN and fp32 overflow: groups holding +Inf, -Inf or NaN, two
+    largest-finite bf16 values whose butterfly sums overflow to Inf, and a pair whose sum
+    cancels while the difference overflows.  The tensor maximum (NVFP4) is taken over the
+    finite transformed values only; bit for bit against the oracle."""
+    x = synth.gradients(64, 256, seed=91)
+    big, nbig = 0x7F7F, 0xFF7F
+    plants = {(0, 3): 0x7F80, (1, 20): 0xFF80, (2, 40): 0x7FC0,          # +Inf, -Inf, NaN
+              (3, 64): big, (3, 65): big,                                   # sums overflow
+              (4, 96): big, (4, 104): nbig,                                 # cancel / overflow
+              (5, 130): big, (6, 200): nbig}                                # lone extremes
+    for (r, c), v in plants.items():
+        x[r, c] = v
+    shape = x.shape
+    rnd = np.random.default_rng(92).integers(0, 256, size=shape, dtype=np.uint8) if sr else None
+    rounding = "floor" if fmt == "e2m1" else "ceil"
+    q = mx.quantize_train(to_dev(x), fmt, rounding, rht_signs=0x9E37,
+                          sr_random=None if rnd is None else torch.from_numpy(rnd).cuda(), layout="both")
+    xt = oracle.rht16(x, 0x9E37)
+    if fmt == "nvfp4":
+        e, s, g = oracle.quantize_nvfp4_sr(xt, rnd) if sr else oracle.quantize_nvfp4(xt)
+        assert q.global_scale.cpu().numpy()[0] == np.float32(g)
+    else:
+        rnd_o = oracle.CEIL if rounding == "ceil" else oracle.FLOOR
+        e, s = oracle.quantize_mx_sr(xt, FMT[fmt], rnd_o, rnd) if sr else oracle.quantize_mx(xt, FMT[fmt], oracle.ROW, rnd_o)
+    assert np.array_equal(q.elems.cpu().numpy(), e.reshape(-1))
+    assert np.array_equal(q.scales.cpu().numpy(), s.reshape(-1))
+    assert np.array_equal(q.scales_alt.cpu().numpy(), oracle.to_tcgen05_layout(s))
+
+
+def test_oracle_transform_overflows_where_planted(oracle):
+    """CPU-side check that the planted pairs above do drive the fp32 butterfly to Inf (so
+    the test reaches the kernels' non-finite path)."""
+    x = synth.gradients(64, 256, seed=91)
+    x[3, 64] = x[3, 65] = 0x7F7F
+    xt = oracle.rht16(x, 0x9E37)
+    assert np.any((xt[3, 64:80] & 0x7FFF) == 0x7F80)
+
+
 @pytest.mark.parametrize("fmt", ["e2m1", "nvfp4"])
 def test_train_quantiser_multi_cta(oracle, fmt):
     """A gradient of the benchmark's width (1024 x 14336) with the transform and stochastic
