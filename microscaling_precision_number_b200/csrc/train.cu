@@ -127,39 +127,55 @@ __device__ __forceinline__ float rht16x2_absmax(const uint4 &a0, const uint4 &a1
 }
 
 // ---- stochastic rounding onto the element grid ----------------------------------------------
-// Returns the representable value (lo or hi, signed) that y rounds to with random byte r.
-// At or above the format's smallest normal 2^emin, the grid step of |y|'s binade is bit
-// w = 23 - mbits of its fp32 pattern, so the w low bits L are |y| - lo in units of 2^-w grid
-// steps, and 256 (|y| - lo) > r (hi - lo) reads L > r 2^(w - 8): exactly
-// when L + (2^w - 1 - r 2^(w - 8)) carries into bit w.  Adding that and clearing the w low
-// bits gives lo or hi (a carry out of the mantissa steps into the next binade, as the grid
-// does).  Below 2^emin the grid has the fixed subnormal step 2^(emin - mbits), which is also
-// the step of the binade [2^emin, 2^(emin + 1)]: |y| + 2^emin rounded toward +infinity lands
-// there, and rounding up to the next fp32 keeps the decision (L is then the ceiling of the
-// exact distance, compared strictly against an integer); subtracting 2^emin is exact.
-// |y| at or above the maximum saturates (Inf included); the sign is kept.
+// Rounds y to lo or hi, its representable neighbours, with random byte r; rsh is r shifted
+// up by kSrShift<FMT> = w - 8.  At or above the format's smallest normal 2^emin, the grid
+// step of |y|'s binade is bit w = 23 - mbits of its fp32 pattern, so the w low bits L are
+// |y| - lo in units of 2^-w grid steps, and 256 (|y| - lo) > r (hi - lo) reads L > r 2^(w - 8):
+// exactly when L + (2^w - 1 - r 2^(w - 8)) carries into bit w.  Adding that and clearing the
+// w low bits gives lo or hi (a carry out of the mantissa steps into the next binade, as the
+// grid does).  Below 2^emin the grid has the fixed subnormal step 2^(emin - mbits), which is
+// also the step of the binade [2^emin, 2^(emin + 1)]: |y| + 2^emin rounded toward +infinity
+// lands there, and rounding up to the next fp32 keeps the decision (L is then the ceiling
+// of the exact distance, compared strictly against an integer); subtracting 2^emin is
+// exact.  The sign is kept.  A result above the format's maximum (|y| at or above it rounds
+// to the maximum or past it, up to the next power of two; Inf stays Inf) is brought to the
+// maximum by the saturating conversion that every caller applies next.
+template <int FMT> constexpr int kSrMbits = FMT == FMT_E4M3 ? 3 : (FMT == FMT_E5M2 ? 2 : 1);
+template <int FMT> constexpr int kSrShift = 23 - kSrMbits<FMT> - 8;
 template <int FMT>
-__device__ __forceinline__ float sr_value(float y, uint32_t r) {
-    constexpr int mbits = FMT == FMT_E4M3 ? 3 : (FMT == FMT_E5M2 ? 2 : 1);
+__device__ __forceinline__ float sr_value(float y, uint32_t rsh) {
     constexpr int emin = FMT == FMT_E4M3 ? -6 : (FMT == FMT_E5M2 ? -14 : 0);   // smallest normal exponent
-    constexpr float maxv = FMT == FMT_E4M3 ? 448.0f : (FMT == FMT_E5M2 ? 57344.0f : 6.0f);
-    constexpr uint32_t w = 23 - mbits, low = (1u << w) - 1u;
+    constexpr uint32_t low = (1u << (23 - kSrMbits<FMT>)) - 1u;
     constexpr float minnorm = emin >= 0 ? (float)(1 << emin) : 1.0f / (float)(1 << -emin);
     const float a = fabsf(y);
     const bool sub = a < minnorm;
     const float ap = sub ? __fadd_ru(a, minnorm) : a;
-    float v = __uint_as_float((__float_as_uint(ap) + low - (r << (w - 8))) & ~low);
+    float v = __uint_as_float((__float_as_uint(ap) + low - rsh) & ~low);
     if (sub) v = __fsub_rn(v, minnorm);
-    return copysignf(fminf(v, maxv), y);
+    return copysignf(v, y);
+}
+
+// Byte k of word, shifted to start at bit SH (2 instructions).
+template <int SH, int K>
+__device__ __forceinline__ uint32_t byte_at(uint32_t word) {
+    constexpr uint32_t mask = 0xFFu << SH;
+    if constexpr (8 * K <= SH) return (word << (SH - 8 * K)) & mask;
+    else return (word >> (8 * K - SH)) & mask;
 }
 
 template <int FMT, bool SR>
 __device__ __forceinline__ void round8(float (&x)[8], const uint8_t *rnd) {
     if constexpr (SR) {
+        constexpr int sh = kSrShift<FMT>;
         const uint2 rb = *reinterpret_cast<const uint2 *>(rnd);
-        const uint32_t w[2] = {rb.x, rb.y};
-#pragma unroll
-        for (int i = 0; i < 8; i++) x[i] = sr_value<FMT>(x[i], (w[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+        x[0] = sr_value<FMT>(x[0], byte_at<sh, 0>(rb.x));
+        x[1] = sr_value<FMT>(x[1], byte_at<sh, 1>(rb.x));
+        x[2] = sr_value<FMT>(x[2], byte_at<sh, 2>(rb.x));
+        x[3] = sr_value<FMT>(x[3], byte_at<sh, 3>(rb.x));
+        x[4] = sr_value<FMT>(x[4], byte_at<sh, 0>(rb.y));
+        x[5] = sr_value<FMT>(x[5], byte_at<sh, 1>(rb.y));
+        x[6] = sr_value<FMT>(x[6], byte_at<sh, 2>(rb.y));
+        x[7] = sr_value<FMT>(x[7], byte_at<sh, 3>(rb.y));
     }
 }
 
