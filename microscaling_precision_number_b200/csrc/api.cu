@@ -276,7 +276,7 @@ mx_status mx_quantize_mx_nvfp4(const void *src, int64_t rows, int64_t cols, mx_f
     st = nvfp4_scratch(d);
     if (st != MX_OK) return st;
     const int n_partials = mxk::stream_rows_grid(rows, cols, d->num_sms);
-    if (n_partials > d->partials_cap) return MX_ERR_SHAPE;      // cannot happen: both are 3 x SMs at most
+    if (n_partials > d->partials_cap) return MX_ERR_SHAPE;      // cannot happen: 3 per SM, the scratch holds 8
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // the MX pass also leaves the NVFP4 partial maxima; the NVFP4 pass then skips its own
     // maximum pass (programmatic dependent launch orders it after the MX pass)

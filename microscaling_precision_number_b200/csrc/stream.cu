@@ -785,7 +785,9 @@ cudaError_t launch_stream_rows_mx(const void *src, int64_t rows, int64_t cols, i
     }
 }
 
-int stream_nvfp4_scratch_floats(int num_sms) { return kCtasPerSm * num_sms; }
+// Partial maxima: one per CTA of the streaming maximum pass (kCtasPerSm per SM) or of the
+// training quantiser's maximum pass (at most 8 per SM).
+int stream_nvfp4_scratch_floats(int num_sms) { return (kCtasPerSm > 8 ? kCtasPerSm : 8) * num_sms; }
 
 template <bool RM, bool TC>
 static cudaError_t launch_nvfp4_t(const uint8_t *src, uint32_t nb, FastDiv f, uint32_t ca, float *partials,
