@@ -147,11 +147,13 @@ __device__ __forceinline__ float sr_value(float y, uint32_t rsh) {
     constexpr int emin = FMT == FMT_E4M3 ? -6 : (FMT == FMT_E5M2 ? -14 : 0);   // smallest normal exponent
     constexpr uint32_t low = (1u << (23 - kSrMbits<FMT>)) - 1u;
     constexpr float minnorm = emin >= 0 ? (float)(1 << emin) : 1.0f / (float)(1 << -emin);
-    // c = 2^emin below it, else 0: adding and subtracting 0 is exact, so one selected
-    // constant serves both steps
-    const float c = fabsf(y) < minnorm ? minnorm : 0.0f;
-    const float ap = __fadd_ru(fabsf(y), c);
-    const float v = __fsub_rn(__uint_as_float((__float_as_uint(ap) + low - rsh) & ~low), c);
+    // s = 1 below 2^emin, else 0, from one saturating FMA on the FMA pipe (the integer and
+    // compare steps of this routine fill the ALU pipe): (2^emin - |y|) 2^100 is at least
+    // 2^(emin + 76) >= 1 whenever it is positive.  Adding and subtracting s 2^emin is exact
+    // or, for the shift into the subnormal binade, the rounding toward +infinity.
+    const float s = __saturatef(__fmaf_rn(-fabsf(y), 0x1p100f, minnorm * 0x1p100f));
+    const float ap = __fmaf_ru(s, minnorm, fabsf(y));
+    const float v = __fmaf_rn(-s, minnorm, __uint_as_float((__float_as_uint(ap) + low - rsh) & ~low));
     return copysignf(v, y);
 }
 
