@@ -52,6 +52,10 @@ __device__ __forceinline__ bool tile_exact(int d, const uint32_t *w) {
     return bad == 0u;
 }
 
+// WIDE (codes and output 32-byte aligned, scales 2-byte aligned): each thread's 32 bytes of
+// codes in one 256-bit load, its two tile scales in one 16-bit load and its 64 output codes
+// in two 256-bit stores, halving the load / store instructions of the narrow form.
+template <bool WIDE>
 __global__ void __launch_bounds__(kNestThreads)
 mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__restrict__ scales, int64_t cols,
                            uint32_t blocks_c, uint8_t *__restrict__ out, float *__restrict__ block_scale,
@@ -66,10 +70,21 @@ mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__r
     const int64_t S = cols / 32;
 
     // 64 packed E2M1 codes (32 bytes) and the two tile scales
-    const uint4 *src = reinterpret_cast<const uint4 *>(elems + ((R * cols + c0) >> 1));
-    const uint4 p0 = src[0], p1 = src[1];
-    const uint32_t sc[2] = {scales[R * S + (c0 >> 5)], scales[R * S + (c0 >> 5) + 1]};
-    const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    uint32_t w[8], sc[2];
+    if constexpr (WIDE) {
+        asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
+                     : "l"(elems + ((R * cols + c0) >> 1)));
+        const uint32_t s2 = *reinterpret_cast<const uint16_t *>(scales + R * S + (c0 >> 5));
+        sc[0] = s2 & 0xFFu;
+        sc[1] = s2 >> 8;
+    } else {
+        const uint4 *src = reinterpret_cast<const uint4 *>(elems + ((R * cols + c0) >> 1));
+        const uint4 p0 = src[0], p1 = src[1];
+        w[0] = p0.x, w[1] = p0.y, w[2] = p0.z, w[3] = p0.w, w[4] = p1.x, w[5] = p1.y, w[6] = p1.z, w[7] = p1.w;
+        sc[0] = scales[R * S + (c0 >> 5)];
+        sc[1] = scales[R * S + (c0 >> 5) + 1];
+    }
 
     // largest exponent among finite tiles holding a nonzero code (E2M1 magnitude bits 0-2)
     int m = kNoScale;
@@ -117,9 +132,21 @@ mxfp4_to_fp8_blocks_kernel(const uint8_t *__restrict__ elems, const uint8_t *__r
             o[8 * t + 2 * k + 1] = sc[t] == 0xFFu ? 0x7F7F7F7Fu : (c[2] | (c[3] << 16));
         }
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(out + R * cols + c0);
+    if constexpr (WIDE) {
 #pragma unroll
-    for (int i = 0; i < 4; i++) out_store(dst + i, make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
+        for (int i = 0; i < 2; i++) {
+            uint8_t *p = out + R * cols + c0 + 32 * i;
+            if (out_ok(p, 32))
+                asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                             ::"l"(p), "r"(o[8 * i]), "r"(o[8 * i + 1]), "r"(o[8 * i + 2]), "r"(o[8 * i + 3]),
+                             "r"(o[8 * i + 4]), "r"(o[8 * i + 5]), "r"(o[8 * i + 6]), "r"(o[8 * i + 7])
+                             : "memory");
+        }
+    } else {
+        uint4 *dst = reinterpret_cast<uint4 *>(out + R * cols + c0);
+#pragma unroll
+        for (int i = 0; i < 4; i++) out_store(dst + i, make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]));
+    }
     const int all_exact = __syncthreads_and(exact ? 1 : 0);
     if (tid == 0) {
         const int e = smax - 6;                                   // S = 2^e, e in [-133, 121]
@@ -138,9 +165,12 @@ cudaError_t launch_mxfp4_to_fp8_blocks(const void *elems, const uint8_t *scales,
                              {block_exact, (uint64_t)n_blocks}};
     const cudaError_t e = set_out_ranges(rng, st);
     if (e != cudaSuccess) return e;
-    mxfp4_to_fp8_blocks_kernel<<<(unsigned)n_blocks, kNestThreads, 0, st>>>(
-        static_cast<const uint8_t *>(elems), scales, cols, (uint32_t)(cols / 128), static_cast<uint8_t *>(out),
-        block_scale, block_exact);
+    const bool wide = ((reinterpret_cast<uintptr_t>(elems) | reinterpret_cast<uintptr_t>(out)) & 31u) == 0 &&
+                      (reinterpret_cast<uintptr_t>(scales) & 1u) == 0;
+    auto k = wide ? mxfp4_to_fp8_blocks_kernel<true> : mxfp4_to_fp8_blocks_kernel<false>;
+    k<<<(unsigned)n_blocks, kNestThreads, 0, st>>>(static_cast<const uint8_t *>(elems), scales, cols,
+                                                    (uint32_t)(cols / 128), static_cast<uint8_t *>(out), block_scale,
+                                                    block_exact);
     return cudaGetLastError();
 }
 

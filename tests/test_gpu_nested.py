@@ -20,10 +20,15 @@ def _no_watchdog():
     assert mx.watchdog_status(clear=True) == 0
 
 
-def run(elems, scales, rows, cols):
-    e = torch.from_numpy(np.ascontiguousarray(elems).reshape(-1)).cuda()
-    s = torch.from_numpy(np.ascontiguousarray(scales).reshape(-1)).cuda()
-    out = torch.empty(rows * cols, dtype=torch.uint8, device="cuda")
+def run(elems, scales, rows, cols, offsets=(0, 0, 0)):
+    """offsets: byte offsets of the codes, the scales and the output inside larger buffers
+    (16 / 1 / 16 break the 32-byte and 2-byte alignment of the wide loads and stores)."""
+    eo, so, oo = offsets
+    e = torch.zeros(eo + elems.size, dtype=torch.uint8, device="cuda")[eo:]
+    e.copy_(torch.from_numpy(np.ascontiguousarray(elems).reshape(-1)))
+    s = torch.zeros(so + scales.size, dtype=torch.uint8, device="cuda")[so:]
+    s.copy_(torch.from_numpy(np.ascontiguousarray(scales).reshape(-1)))
+    out = torch.empty(oo + rows * cols, dtype=torch.uint8, device="cuda")[oo:]
     bs = torch.empty((rows // 128) * (cols // 128), dtype=torch.float32, device="cuda")
     ok = torch.empty((rows // 128) * (cols // 128), dtype=torch.uint8, device="cuda")
     st = L.lib.mx_mxfp4_to_fp8_blocks(e.data_ptr(), s.data_ptr(), rows, cols, out.data_ptr(), bs.data_ptr(),
@@ -33,8 +38,8 @@ def run(elems, scales, rows, cols):
         ok.cpu().numpy().reshape(rows // 128, cols // 128)
 
 
-def check(oracle, elems, scales, rows, cols):
-    got = run(elems, scales, rows, cols)
+def check(oracle, elems, scales, rows, cols, offsets=(0, 0, 0)):
+    got = run(elems, scales, rows, cols, offsets)
     ref = oracle.mxfp4_to_fp8_blocks(elems, scales, rows, cols)
     for g, r, what in zip(got, ref, ("codes", "block scales", "exact flags")):
         assert np.array_equal(g, r), what
@@ -47,6 +52,19 @@ def test_quantised_weights(oracle, shape):
     e, s = oracle.quantize_mx(x, oracle.E2M1, oracle.ROW, oracle.FLOOR)
     _, _, ok = check(oracle, e, s, *shape)
     assert np.all(ok == 1)
+
+
+@pytest.mark.parametrize("offsets", [(16, 0, 0), (0, 1, 0), (0, 0, 16), (16, 1, 16)])
+def test_unaligned_buffers(oracle, offsets):
+    """Buffers that are 16-byte (codes, output) or 1-byte (scales) aligned only: the kernel
+    takes its narrow-access form; same results."""
+    rng = np.random.default_rng(5)
+    rows, cols = 256, 384
+    x = synth.weight_fp4(rows, cols, seed=17)
+    e, s = oracle.quantize_mx(x, oracle.E2M1, oracle.ROW, oracle.FLOOR)
+    s = s.copy()
+    s[128:, :2] = rng.integers(100, 140, size=(128, 2), dtype=np.uint8)
+    check(oracle, e, s, rows, cols, offsets)
 
 
 def test_arbitrary_codes_and_scales(oracle):
