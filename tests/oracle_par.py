@@ -87,3 +87,65 @@ def gemm_ref_tile(oracle, ae, as_, a_fmt, be, bs, b_fmt, M, N, K, m0, m1, n0, n1
     with cf.ThreadPoolExecutor(WORKERS) as ex:
         list(ex.map(work, range(m0, m1, rows_per_task)))
     return c, mag
+
+
+def rht16_rows(oracle, x, signs, slab=512):
+    """The oracle's 16 x 16 transform of every row group of x, slab by slab."""
+    R, C = x.shape
+    out = np.empty_like(x)
+
+    def work(r0):
+        r1 = min(R, r0 + slab)
+        out[r0:r1] = oracle.rht16(np.ascontiguousarray(x[r0:r1]), signs)
+
+    with cf.ThreadPoolExecutor(WORKERS) as ex:
+        list(ex.map(work, range(0, R, slab)))
+    return out
+
+
+def quantize_mx_sr_rows(oracle, x, fmt, rounding, rnd, slab=512):
+    """Row-wise MX quantisation with stochastic rounding (rnd: one byte per element)."""
+    R, C = x.shape
+    bits = oracle.code_bits(fmt)
+    re_ = np.zeros((R, C * bits // 8), dtype=np.uint8)
+    rs = np.zeros((R, C // 32), dtype=np.uint8)
+
+    def work(r0):
+        r1 = min(R, r0 + slab)
+        re_[r0:r1], rs[r0:r1] = oracle.quantize_mx_sr(np.ascontiguousarray(x[r0:r1]), fmt, rounding,
+                                                      np.ascontiguousarray(rnd[r0:r1]))
+
+    with cf.ThreadPoolExecutor(WORKERS) as ex:
+        list(ex.map(work, range(0, R, slab)))
+    return re_, rs
+
+
+def quantize_nvfp4_sr_rows(oracle, x, rnd, slab=512):
+    """NVFP4 with stochastic rounding of the whole tensor, slab by slab.  The per-tensor
+    scale depends on the tensor's largest finite magnitude, so every slab goes to the
+    oracle together with one row that holds that maximum (appended after the slab; its
+    outputs are dropped): the oracle then derives the tensor's own scale for each slab.
+    Returns (elems rows x cols/2, scales rows x cols/16, g)."""
+    R, C = x.shape
+    mag = (x & 0x7FFF).astype(np.uint16)
+    finite = mag < 0x7F80
+    r_max = int(np.argmax(np.where(finite, mag, 0).max(axis=1)))
+    extra = np.ascontiguousarray(x[r_max:r_max + 1])
+    extra_rnd = np.zeros((1, C), dtype=np.uint8)
+    re_ = np.zeros((R, C // 2), dtype=np.uint8)
+    rs = np.zeros((R, C // 16), dtype=np.uint8)
+    gs = {}
+
+    def work(r0):
+        r1 = min(R, r0 + slab)
+        xs = np.concatenate([x[r0:r1], extra])
+        rn = np.concatenate([rnd[r0:r1], extra_rnd])
+        e, s, g = oracle.quantize_nvfp4_sr(np.ascontiguousarray(xs), np.ascontiguousarray(rn))
+        re_[r0:r1], rs[r0:r1] = e[:r1 - r0], s[:r1 - r0]
+        gs[r0] = g
+
+    with cf.ThreadPoolExecutor(WORKERS) as ex:
+        list(ex.map(work, range(0, R, slab)))
+    g_all = set(gs.values())
+    assert len(g_all) == 1
+    return re_, rs, g_all.pop()

@@ -9,7 +9,8 @@ import pytest
 import torch
 
 import synth
-from oracle_par import gemm_ref_pairs, gemm_ref_tile, quantize_mx_both, quantize_mx_rows
+from oracle_par import (gemm_ref_pairs, gemm_ref_tile, quantize_mx_both, quantize_mx_rows, quantize_mx_sr_rows,
+                        quantize_nvfp4_sr_rows, rht16_rows)
 from test_gpu_gemm import gemm_tolerance
 
 pytestmark = pytest.mark.gpu
@@ -57,6 +58,28 @@ def test_dual_full_size_every_byte(oracle, which):
     assert np.array_equal(host(qr.scales_alt), oracle.to_tcgen05_layout(rs))
     assert np.array_equal(host(qc.scales_alt), oracle.to_tcgen05_layout(cs))
     assert np.array_equal(host(qc.elems).reshape(C, R), ce)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "e2m1"])
+def test_train_16384x14336_every_byte(oracle, fmt):
+    """The training quantiser in the benchmark's launch: the 16384 x 14336 gradient shape
+    (N(0, 1e-3) values), the 16 x 16 transform with signs 0xB5C3 and stochastic rounding
+    from one random byte per element, tcgen05 scales -- every code and scale byte against
+    the oracle's transform followed by its quantisation, in row slabs."""
+    R, C = 16384, 14336
+    x = synth.normal(R, C, sigma=1e-3, seed=70)
+    rnd = np.random.default_rng(71).integers(0, 256, size=(R, C), dtype=np.uint8)
+    rounding = "ceil" if fmt == "nvfp4" else "floor"
+    q = mx.quantize_train(to_dev(x), fmt, rounding, rht_signs=0xB5C3, sr_random=torch.from_numpy(rnd).cuda(),
+                          layout="tcgen05")
+    xt = rht16_rows(oracle, x, 0xB5C3)
+    if fmt == "nvfp4":
+        e, s, g = quantize_nvfp4_sr_rows(oracle, xt, rnd)
+        assert host(q.global_scale)[0] == np.float32(g)
+    else:
+        e, s = quantize_mx_sr_rows(oracle, xt, 2, oracle.FLOOR, rnd)
+    assert np.array_equal(host(q.elems).reshape(R, -1), e)
+    assert np.array_equal(host(q.scales), oracle.to_tcgen05_layout(s))
 
 
 @pytest.mark.parametrize("fmt", [4, 5, 6])
