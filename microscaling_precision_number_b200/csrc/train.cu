@@ -127,11 +127,11 @@ __device__ __forceinline__ float rht16x2_absmax(const uint4 &a0, const uint4 &a1
 }
 
 // ---- stochastic rounding onto the element grid ----------------------------------------------
-// Rounds y to lo or hi, its representable neighbours, with random byte r; rsh is r shifted
-// up by kSrShift<FMT> = w - 8.  At or above the format's smallest normal 2^emin, the grid
-// step of |y|'s binade is bit w = 23 - mbits of its fp32 pattern, so the w low bits L are
-// |y| - lo in units of 2^-w grid steps, and 256 (|y| - lo) > r (hi - lo) reads L > r 2^(w - 8):
-// exactly when L + (2^w - 1 - r 2^(w - 8)) carries into bit w.  Adding that and clearing the
+// Rounds y to lo or hi, its representable neighbours, with random byte r; carry is
+// 2^w - 1 - r 2^(w - 8) (see carry_term).  At or above the format's smallest normal 2^emin,
+// the grid step of |y|'s binade is bit w = 23 - mbits of its fp32 pattern, so the w low bits
+// L are |y| - lo in units of 2^-w grid steps, and 256 (|y| - lo) > r (hi - lo) reads
+// L > r 2^(w - 8): exactly when L + carry carries into bit w.  Adding carry and clearing the
 // w low bits gives lo or hi (a carry out of the mantissa steps into the next binade, as the
 // grid does).  Below 2^emin the grid has the fixed subnormal step 2^(emin - mbits), which is
 // also the step of the binade [2^emin, 2^(emin + 1)]: |y| + 2^emin rounded toward +infinity
@@ -143,7 +143,7 @@ __device__ __forceinline__ float rht16x2_absmax(const uint4 &a0, const uint4 &a1
 template <int FMT> constexpr int kSrMbits = FMT == FMT_E4M3 ? 3 : (FMT == FMT_E5M2 ? 2 : 1);
 template <int FMT> constexpr int kSrShift = 23 - kSrMbits<FMT> - 8;
 template <int FMT>
-__device__ __forceinline__ float sr_value(float y, uint32_t rsh) {
+__device__ __forceinline__ float sr_value(float y, uint32_t carry) {
     constexpr int emin = FMT == FMT_E4M3 ? -6 : (FMT == FMT_E5M2 ? -14 : 0);   // smallest normal exponent
     constexpr uint32_t low = (1u << (23 - kSrMbits<FMT>)) - 1u;
     constexpr float minnorm = emin >= 0 ? (float)(1 << emin) : 1.0f / (float)(1 << -emin);
@@ -153,16 +153,22 @@ __device__ __forceinline__ float sr_value(float y, uint32_t rsh) {
     // or, for the shift into the subnormal binade, the rounding toward +infinity.
     const float s = __saturatef(__fmaf_rn(-fabsf(y), 0x1p100f, minnorm * 0x1p100f));
     const float ap = __fmaf_ru(s, minnorm, fabsf(y));
-    const float v = __fmaf_rn(-s, minnorm, __uint_as_float((__float_as_uint(ap) + low - rsh) & ~low));
+    // the integer add written as a multiply-add (measured faster: the ALU pipe, not the
+    // FMA pipe, holds these kernels)
+    uint32_t t;
+    asm("mad.lo.u32 %0, %1, 1, %2;" : "=r"(t) : "r"(carry), "r"(__float_as_uint(ap)));
+    const float v = __fmaf_rn(-s, minnorm, __uint_as_float(t & ~low));
     return copysignf(v, y);
 }
 
-// Byte k of word, shifted to start at bit SH (2 instructions).
+// The carry term 2^w - 1 - r 2^(w - 8) for the random byte r = byte K of word (w - 8 = SH):
+// the byte by one permute, the rest by one integer multiply-add.
 template <int SH, int K>
-__device__ __forceinline__ uint32_t byte_at(uint32_t word) {
-    constexpr uint32_t mask = 0xFFu << SH;
-    if constexpr (8 * K <= SH) return (word << (SH - 8 * K)) & mask;
-    else return (word >> (8 * K - SH)) & mask;
+__device__ __forceinline__ uint32_t carry_term(uint32_t word) {
+    const uint32_t r = __byte_perm(word, 0u, 0x4440u | K);
+    uint32_t x;
+    asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(x) : "r"(r), "r"(0u - (1u << SH)), "r"((1u << (SH + 8)) - 1u));
+    return x;
 }
 
 template <int FMT, bool SR>
@@ -170,14 +176,14 @@ __device__ __forceinline__ void round8(float (&x)[8], const uint8_t *rnd) {
     if constexpr (SR) {
         constexpr int sh = kSrShift<FMT>;
         const uint2 rb = *reinterpret_cast<const uint2 *>(rnd);
-        x[0] = sr_value<FMT>(x[0], byte_at<sh, 0>(rb.x));
-        x[1] = sr_value<FMT>(x[1], byte_at<sh, 1>(rb.x));
-        x[2] = sr_value<FMT>(x[2], byte_at<sh, 2>(rb.x));
-        x[3] = sr_value<FMT>(x[3], byte_at<sh, 3>(rb.x));
-        x[4] = sr_value<FMT>(x[4], byte_at<sh, 0>(rb.y));
-        x[5] = sr_value<FMT>(x[5], byte_at<sh, 1>(rb.y));
-        x[6] = sr_value<FMT>(x[6], byte_at<sh, 2>(rb.y));
-        x[7] = sr_value<FMT>(x[7], byte_at<sh, 3>(rb.y));
+        x[0] = sr_value<FMT>(x[0], carry_term<sh, 0>(rb.x));
+        x[1] = sr_value<FMT>(x[1], carry_term<sh, 1>(rb.x));
+        x[2] = sr_value<FMT>(x[2], carry_term<sh, 2>(rb.x));
+        x[3] = sr_value<FMT>(x[3], carry_term<sh, 3>(rb.x));
+        x[4] = sr_value<FMT>(x[4], carry_term<sh, 0>(rb.y));
+        x[5] = sr_value<FMT>(x[5], carry_term<sh, 1>(rb.y));
+        x[6] = sr_value<FMT>(x[6], carry_term<sh, 2>(rb.y));
+        x[7] = sr_value<FMT>(x[7], carry_term<sh, 3>(rb.y));
     }
 }
 
