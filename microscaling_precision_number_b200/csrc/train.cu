@@ -17,8 +17,9 @@
 // in, one per element), a value strictly between its two representable neighbours lo < |y|
 // < hi rounds to hi when 256 (|y| - lo) > r (hi - lo), else to lo; |y| at or above the
 // maximum saturates; the sign is kept.  Scales are computed exactly as in the RNE path.
-// One thread per quantisation block, blocks of consecutive threads adjacent in memory
-// (coalesced), grid-stride loops; NVFP4 takes a maximum pass and a quantisation pass.
+// One thread per 32-element MX block or per two 16-element NVFP4 blocks (two transform
+// groups either way), consecutive threads on adjacent blocks (coalesced), grid-stride
+// loops; NVFP4 takes a maximum pass and a quantisation pass.
 #include "checked.cuh"
 #include "codec.cuh"
 #include "internal.h"
